@@ -1,0 +1,351 @@
+"""The CSA / HCA attention layer, step by step, in float64 (oracle; test infrastructure only).
+
+Notation follows the pages: m tokens per compressed entry (m' for HCA), top-k
+selected entries, a window of w = 128 uncompressed recent tokens, H query
+heads sharing one KV head of dimension D, rotary on the last d_r = 64 dims.
+
+Readings taken where the pages are silent (each repeated at its function):
+
+R1  Overlap is look-back: entry i pools raw rows [(i-ov)m, (i+1)m), clipped at
+    row 0 ("each compressed entry draws from 2m source entries while the
+    sequence still shrinks by m" -- "DeepSeek-V4: Making a Million Tokens
+    Affordable", "Two ways to shrink attention, interleaved").  HCA uses ov=0.
+R2  "learned per-token compression weights and positional biases" (same
+    section) = one gate logit per raw row and channel plus one bias per window
+    slot and channel, normalised by a softmax over the window's rows, per
+    channel.
+R3  Entry i is rotated at position pos0 + i*m and is visible to a query at
+    position t iff its last row pos0 + (i+1)m - 1 <= t (causally complete).
+R4  Window rows are the most recent w raw rows including the current one,
+    rotated at their own positions, not normalised; entries and window rows
+    are separate key sets and nothing is de-duplicated.
+R5  Index score s_i = sum_h w_h * ReLU(sigma_q,h * sigma_k,i * <q_h, k_i>)
+    over H_I indexer heads (the pages give no formula: "the page does not give
+    V4's exact scorer" -- "DeepSeek-V4, explained.", glossary).
+R6  Top-k: the k largest scores, ties to the smaller entry index; returned in
+    ascending entry order; fewer than k visible entries -> all of them, then -1.
+R7  Logits l_j = <q~, k~_j> / sqrt(D); sink: p_j = e^{l_j} / (e^{s_h} + sum e^{l}).
+R8  RoPE: interleaved pairs (D-64+2u, D-64+2u+1), theta_u = base^(-2u/64),
+    angle pos*theta_u in float64.
+R9  RMSNorm eps = 1e-6 with a learnable per-channel weight gamma.
+"""
+
+import numpy as np
+
+from . import formats as F
+
+
+# --------------------------------------------------------------------------- rotary / norm
+
+def rope_cos_sin(pos, d_rope: int, base: float):
+    """cos, sin of pos * theta_u for u < d_rope/2 (R8), float64 [..., d_rope/2].
+
+    "RoPE is applied to only the last 64 dimensions" -- "DeepSeek-V4: Making a
+    Million Tokens Affordable", "Two ways to shrink attention, interleaved".
+    """
+    pos = np.asarray(pos, dtype=np.float64)
+    u = np.arange(d_rope // 2, dtype=np.float64)
+    theta = np.power(float(base), -2.0 * u / d_rope)
+    ang = pos[..., None] * theta
+    return np.cos(ang), np.sin(ang)
+
+
+def rope(x, pos, d_rope: int, base: float):
+    """Rotate the last d_rope dims of x [..., D] by position pos (broadcast on x's leading dims)."""
+    x = np.array(x, dtype=np.float64, copy=True)
+    D = x.shape[-1]
+    c, s = rope_cos_sin(pos, d_rope, base)
+    a = x[..., D - d_rope::2].copy()
+    b = x[..., D - d_rope + 1::2].copy()
+    x[..., D - d_rope::2] = a * c - b * s
+    x[..., D - d_rope + 1::2] = a * s + b * c
+    return x
+
+
+def rms_norm(x, gamma, eps: float):
+    """x / sqrt(mean(x^2) + eps) * gamma (R9).
+
+    "queries and compressed entries get an extra RMSNorm before core attention"
+    -- "DeepSeek-V4: Making a Million Tokens Affordable", "Two ways to shrink
+    attention, interleaved".
+    """
+    x = np.asarray(x, dtype=np.float64)
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return x * r * np.asarray(gamma, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------- compression (a2)
+
+def entry_rows(i: int, m: int, ov: int):
+    """Raw row indices (relative to pos0) pooled into entry i, and their window slots (R1)."""
+    lo = (i - ov) * m
+    rows = np.arange(max(lo, 0), (i + 1) * m)
+    return rows, rows - lo
+
+
+def pool_entry(raw_rows, gate_rows, bias, slots):
+    """Per-channel softmax-weighted sum of one entry's source rows (R2).
+
+    raw_rows, gate_rows: [r, D]; bias: [(1+ov)m, D]; slots: window slot of each row.
+    "compresses the key-value cache of every group of m consecutive tokens into
+    one entry using learned compression weights and positional biases" --
+    "DeepSeek-V4 Explained: ...", "The attention stack, and why it is two mechanisms".
+    """
+    z = np.asarray(gate_rows, np.float64) + np.asarray(bias, np.float64)[slots]
+    z = z - z.max(axis=0, keepdims=True)
+    a = np.exp(z)
+    a = a / a.sum(axis=0, keepdims=True)
+    return (a * np.asarray(raw_rows, np.float64)).sum(axis=0)
+
+
+def compress(raw, gate, bias, gamma, m, ov, d_rope, base, pos0, entries, raw_first_row=0):
+    """Entries (float64 [len(entries), D]) from uncompressed rows.
+
+    raw, gate: float64 [n_rows, D] holding raw rows raw_first_row.. (relative to
+    pos0).  Each entry: pool (R1, R2) -> RMSNorm (R9) -> rotate at pos0 + i*m (R3).
+    """
+    out = []
+    for i in entries:
+        rows, slots = entry_rows(int(i), m, ov)
+        idx = rows - raw_first_row
+        assert idx.min() >= 0 and idx.max() < raw.shape[0], "source rows not provided"
+        e = pool_entry(raw[idx], gate[idx], bias, slots)
+        e = rms_norm(e, gamma, 1e-6)
+        out.append(rope(e, pos0 + int(i) * m, d_rope, base))
+    return np.stack(out) if out else np.zeros((0, raw.shape[1]))
+
+
+# --------------------------------------------------------------------------- visibility
+
+def n_visible(t, pos0: int, m: int):
+    """Number of causally complete entries for a query at position t (R3)."""
+    return (np.asarray(t, np.int64) - pos0 + 1) // m
+
+
+def window_row_ids(t: int, pos0: int, w: int):
+    """Raw row indices of the sliding window of a query at position t (R4)."""
+    r = t - pos0
+    return np.arange(max(0, r - w + 1), r + 1)
+
+
+# --------------------------------------------------------------------------- indexer (a3) and top-k (a4)
+
+def index_scores(iq, iq_scale, head_w, ik, ik_scale):
+    """s_i = sum_h w_h * ReLU(sigma_q,h * sigma_k,i * <q_h, k_i>) (R5).
+
+    iq [H_I, d_I], iq_scale [H_I], head_w [H_I], ik [N, d_I], ik_scale [N].
+    "a Lightning Indexer scores them in a low-rank way" -- "DeepSeek-V4
+    Explained: ..."; "a separate lightning indexer, a few small heads run in
+    FP8, scores individual past tokens" -- "DeepSeek-V4, explained.", step 3.
+    """
+    dots = np.asarray(ik, np.float64) @ np.asarray(iq, np.float64).T          # [N, H_I]
+    z = dots * np.asarray(ik_scale, np.float64)[:, None] * np.asarray(iq_scale, np.float64)[None, :]
+    return np.maximum(z, 0.0) @ np.asarray(head_w, np.float64)
+
+
+def top_k(scores, k: int):
+    """Indices of the k largest scores, ties to the smaller index, ascending, -1 padded (R6).
+
+    "Keep the k highest-scoring blocks" -- "DeepSeek-V4, explained.", step 4;
+    "a top-k selector keeps only the best ones for core attention" --
+    "DeepSeek-V4: Making a Million Tokens Affordable".
+    """
+    s = np.asarray(scores, np.float64)
+    order = sorted(range(len(s)), key=lambda i: (-s[i], i))   # stable, explicit tie rule
+    keep = np.array(sorted(order[:k]), dtype=np.int64)
+    out = np.full(k, -1, dtype=np.int64)
+    out[:len(keep)] = keep
+    return out
+
+
+def top_k_fast(scores, k: int):
+    """Same result as top_k via a stable sort (for large N)."""
+    s = np.asarray(scores, np.float64)
+    order = np.argsort(-s, kind="stable")
+    keep = np.sort(order[:k])
+    out = np.full(k, -1, dtype=np.int64)
+    out[:len(keep)] = keep
+    return out
+
+
+# --------------------------------------------------------------------------- core attention (a5 / a6)
+
+def prep_query(q, gamma_q, t, d_rope, base, eps=1e-6):
+    """q~ = RoPE_t(RMSNorm(q) * gamma_q) per head (a1)."""
+    return rope(rms_norm(q, gamma_q, eps), t, d_rope, base)
+
+
+def attend(q, t, rows, sinks, gamma_q, d_rope, base, scale=None, eps=1e-6):
+    """Shared-KV multi-query attention with sinks and inverse RoPE on the output.
+
+    q [H, D] (raw), rows [R, D] (keys = values), sinks [H] -> o [H, D].
+    "a compressed entry serves as both key and value ... RoPE at position -i is
+    applied back to the attention output so the result carries relative
+    positions ... learnable attention sinks let a head route its attention
+    mass to nothing at all" -- "DeepSeek-V4: Making a Million Tokens
+    Affordable", "Two ways to shrink attention, interleaved"; "an
+    attention-sink term lets each head's scores sum to less than one" --
+    "DeepSeek-V4 Explained: ...".  Readings R7, R8, R9.
+    """
+    rows = np.asarray(rows, np.float64)
+    D = rows.shape[-1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    qt = prep_query(q, gamma_q, t, d_rope, base, eps)
+    logits = (qt @ rows.T) * scale                                   # [H, R]
+    s = np.asarray(sinks, np.float64)
+    M = np.maximum(s, logits.max(axis=1) if logits.shape[1] else s)
+    e = np.exp(logits - M[:, None])
+    Z = np.exp(s - M) + e.sum(axis=1)
+    p = e / Z[:, None]
+    o = p @ rows
+    return rope(o, -float(t), d_rope, base)
+
+
+def attention_probs(q, t, rows, sinks, gamma_q, d_rope, base, scale=None, eps=1e-6):
+    """The attention weights p [H, R] of `attend` (for the sink pins)."""
+    rows = np.asarray(rows, np.float64)
+    D = rows.shape[-1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    qt = prep_query(q, gamma_q, t, d_rope, base, eps)
+    logits = (qt @ rows.T) * scale
+    s = np.asarray(sinks, np.float64)
+    M = np.maximum(s, logits.max(axis=1))
+    e = np.exp(logits - M[:, None])
+    return e / (np.exp(s - M) + e.sum(axis=1))[:, None]
+
+
+# --------------------------------------------------------------------------- one decode step (a7)
+
+class LayerSpec:
+    """The hyper-parameters one step needs (plain attributes, no behaviour)."""
+
+    def __init__(self, kind, m, ov, top_k, H, D, d_rope=64, rope_base=10000.0, window=128,
+                 H_I=0, d_I=0, kv_format="bf16", idx_format="e4m3", act_format="bf16",
+                 eps=1e-6, pos0=0, scale=None):
+        self.kind, self.m, self.ov, self.top_k = kind, m, ov, top_k
+        self.H, self.D, self.d_rope, self.rope_base, self.window = H, D, d_rope, rope_base, window
+        self.H_I, self.d_I = H_I, d_I
+        self.kv_format, self.idx_format, self.act_format = kv_format, idx_format, act_format
+        self.eps, self.pos0, self.scale = eps, pos0, scale
+
+    @classmethod
+    def of(cls, layer, pos0=0):
+        return cls(layer.kind, layer.m, layer.ov, layer.top_k, layer.H, layer.D, layer.d_rope,
+                   layer.rope_base, layer.window, layer.H_I, layer.d_I, layer.kv_format,
+                   layer.idx_format, layer.act_format, layer.eps, pos0)
+
+
+def append_window_row(L, x_row, t):
+    """Stored window row of the token at position t: RoPE_t(x), not normalised (R4)."""
+    return F.encode_rows(rope(x_row, t, L.d_rope, L.rope_base), L.kv_format, L.d_rope)
+
+
+def decode_step(L, st, b: int):
+    """One decode step of sequence b: append -> compress (if a group completes) -> select -> attend.
+
+    ``st`` holds the state and step inputs in storage form (the keys of
+    csa_synth.decode_inputs); it is not modified.  Returns a dict with the
+    output o [H, D] (float64), the new window row and (when a group completed)
+    the new entry's index and stored row, the scores and the selected indices.
+    """
+    t = int(st["t"][b])
+    r = t - L.pos0
+    m, ov, D = L.m, L.ov, L.D
+    rr = (1 + ov) * m
+    res = {}
+    x_new = F.decode_act(st["x_new"][b], L.act_format)
+    g_new = F.decode_act(st["g_new"][b], L.act_format)
+    # append the new token to the window ring and the uncompressed ring
+    wrow = append_window_row(L, x_new, t)
+    res["window_row"] = wrow
+    window = st["window"][b].copy()
+    window[r % L.window] = wrow
+    raw_ring = F.decode_act(st["raw_ring"][b], L.act_format).copy()
+    gate_ring = F.decode_act(st["gate_ring"][b], L.act_format).copy()
+    raw_ring[r % rr] = x_new
+    gate_ring[r % rr] = g_new
+    # compress the entry completed by this token
+    entries = st["entries"][b]
+    new_entry = None
+    if (r + 1) % m == 0:
+        i = (r + 1) // m - 1
+        rows, slots = entry_rows(i, m, ov)
+        e = pool_entry(raw_ring[rows % rr], gate_ring[rows % rr], st["pos_bias"], slots)
+        e = rope(rms_norm(e, st["gamma_kv"], L.eps), L.pos0 + i * m, L.d_rope, L.rope_base)
+        new_entry = (i, F.encode_rows(e, L.kv_format, L.d_rope))
+        res["entry"] = new_entry
+    n_vis = int(n_visible(t, L.pos0, m))
+
+    def entry_values(ids):
+        raw_bytes = entries[ids].copy()
+        if new_entry is not None:
+            raw_bytes[ids == new_entry[0]] = new_entry[1]
+        return F.decode_rows(raw_bytes, L.kv_format, D, L.d_rope)
+
+    if L.kind == "csa":
+        iq = F.decode_idx(st["idx_q"][b], L.idx_format)
+        ik = F.decode_idx(st["idx_k"][b][:n_vis], L.idx_format)
+        s = index_scores(iq, st["idx_q_scale"][b], st["head_w"][b], ik, st["idx_k_scale"][b][:n_vis])
+        sel = top_k_fast(s, L.top_k)
+        res["scores"], res["topk"] = s, sel
+        ent = entry_values(sel[sel >= 0])
+    else:
+        ent = entry_values(np.arange(n_vis))
+    wids = window_row_ids(t, L.pos0, L.window)
+    win = F.decode_rows(window[wids % L.window], L.kv_format, D, L.d_rope)
+    rows = np.concatenate([ent, win], axis=0)
+    q = F.decode_act(st["q"][b], L.act_format)
+    res["o"] = attend(q, t, rows, st["sinks"], st["gamma_q"], L.d_rope, L.rope_base, L.scale, L.eps)
+    res["n_rows"] = rows.shape[0]
+    return res
+
+
+# --------------------------------------------------------------------------- chunked prefill
+
+def prefill_caches(L, pf, b: int):
+    """Entries and window ring after appending a prefill chunk (compress + append).
+
+    pf holds csa_synth.prefill_inputs' keys.  Returns (entries bytes, window
+    bytes, first new entry, number of new entries).
+    """
+    m, ov = L.m, L.ov
+    prefix, n, Tq = pf["prefix"], pf["n"], pf["Tq"]
+    raw = F.decode_act(pf["raw"][b], L.act_format)
+    gate = F.decode_act(pf["gate"][b], L.act_format)
+    first = pf["raw_first_row"]
+    window = pf["window"][b].copy()
+    cap = window.shape[0]
+    for r in range(prefix, n):
+        window[r % cap] = append_window_row(L, raw[r - first], L.pos0 + r)
+    e0, e1 = prefix // m, n // m
+    entries = pf["entries"][b].copy()
+    if e1 > e0:
+        vals = compress(raw, gate, pf["pos_bias"], pf["gamma_kv"], m, ov, L.d_rope, L.rope_base,
+                        L.pos0, range(e0, e1), raw_first_row=first)
+        entries[e0:e1] = F.encode_rows(vals, L.kv_format, L.d_rope)
+    return entries, window, e0, e1 - e0
+
+
+def prefill_query(L, pf, entries, window, b: int, j: int):
+    """Output of query j of the chunk (position prefix + j) given the updated caches."""
+    t = int(pf["t"][b, j])
+    n_vis = int(n_visible(t, L.pos0, L.m))
+    res = {}
+    if L.kind == "csa":
+        iq = F.decode_idx(pf["idx_q"][b, j], L.idx_format)
+        ik = F.decode_idx(pf["idx_k"][b][:n_vis], L.idx_format)
+        s = index_scores(iq, pf["idx_q_scale"][b, j], pf["head_w"][b, j], ik, pf["idx_k_scale"][b][:n_vis])
+        sel = top_k_fast(s, L.top_k)
+        res["scores"], res["topk"] = s, sel
+        ids = sel[sel >= 0]
+    else:
+        ids = np.arange(n_vis)
+    ent = F.decode_rows(entries[ids], L.kv_format, L.D, L.d_rope)
+    wids = window_row_ids(t, L.pos0, L.window)
+    win = F.decode_rows(window[wids % window.shape[0]], L.kv_format, L.D, L.d_rope)
+    rows = np.concatenate([ent, win], axis=0)
+    q = F.decode_act(pf["q"][b, j], L.act_format)
+    res["o"] = attend(q, t, rows, pf["sinks"], pf["gamma_q"], L.d_rope, L.rope_base, L.scale, L.eps)
+    return res
