@@ -141,7 +141,7 @@ def decode_inputs(wl: Workload, li: int = 0, n=None, entry_cap=None):
     n = wl.n if n is None else n
     B = wl.B
     N = n // layer.m
-    cap = N if entry_cap is None else entry_cap
+    cap = max(N, 1) if entry_cap is None else entry_cap
     rr = raw_ring_rows(layer)
     d = _common(wl, li, layer, (B,))
     d.update({

@@ -1,0 +1,269 @@
+/*
+ * csa.h -- C ABI of the B200 (sm_100a) CSA / HCA compressed-attention operator.
+ *
+ * One attention layer of DeepSeek-V4's hybrid attention, as the explainer
+ * pages describe it:
+ *
+ *   CSA ("compressed sparse attention"): every m consecutive raw KV rows are
+ *   pooled into one compressed entry with learned per-channel gate logits and
+ *   positional biases over an overlapping 2m-row window; a lightning indexer
+ *   scores the causally complete entries against the query; the top-k
+ *   entries plus a sliding window of the w most recent raw rows are attended
+ *   by shared-KV multi-query attention with a per-head sink logit, RMSNorm on
+ *   queries and entries, rotary embedding on the last 64 dims only, and the
+ *   inverse rotation applied to the output.
+ *     - "DeepSeek-V4: Making a Million Tokens Affordable", section "Two ways
+ *       to shrink attention, interleaved" (m=4, top-k=1024, overlap 2m, sink,
+ *       RMSNorm, partial RoPE, inverse RoPE on the output, 128-token window).
+ *     - "DeepSeek-V4 Explained: Compressed Sparse Attention and 1M Context at
+ *       10% KV", section "The attention stack, and why it is two mechanisms"
+ *       (compression weights and positional biases, lightning indexer,
+ *       shared-KV multi-query layout, BF16 rotary dims + FP8 remainder).
+ *   HCA ("heavily compressed attention"): the same path with m'=128, no
+ *   overlap, no indexer and dense attention over every visible entry.
+ *     - same page, same section ("m' = 128 ... dense over what remains").
+ *
+ * The pages give no formula for the indexer or the gate and no storage
+ * layout; the definitions this library implements are stated at each call.
+ *
+ * Conventions (every call):
+ *   - Returns csa_status_t; CSA_OK = 0.  Argument errors are detected on the
+ *     host, before any launch, and leave all buffers untouched;
+ *     csa_last_error() then describes the failure (thread-local string).
+ *   - Every pointer is a DEVICE pointer owned by the caller, 16-byte aligned,
+ *     unless marked "host".  The library allocates nothing on the hot calls.
+ *   - Calls are asynchronous on the given CUDA stream (a cudaStream_t passed
+ *     as void*; NULL = legacy default stream).  Device-side faults surface at
+ *     the caller's next synchronisation.  Kernels contain only bounded waits:
+ *     a wait that gives up sets a bit in the workspace's device error word,
+ *     read back by csa_device_error().
+ *   - Workspace: csa_workspace_size() bytes of device memory, zero-filled by
+ *     the caller before its FIRST use (the library leaves its counters at zero
+ *     after every call).  Concurrent calls must not share a workspace.
+ *   - Positions: q_pos[b * Tq + j] (device int64) is the absolute position t
+ *     of query token j of sequence b; raw row index r = t - pos0.
+ *
+ * Stored-row formats (kv_format), one row = one compressed entry or one
+ * window row, row_bytes = csa_row_bytes():
+ *   CSA_FMT_F32   D float32.
+ *   CSA_FMT_BF16  D bfloat16.
+ *   CSA_FMT_MIXED D+80 bytes: FP8-e4m3 codes of dims [0, D-64) at byte 0,
+ *                 bfloat16 of the 64 rotary dims at byte D-64, float32 scale
+ *                 sigma at byte D+64, zero padding.  value = code * sigma for
+ *                 the FP8 part; sigma is the smallest power of two with
+ *                 max|x| / sigma <= 448 (1 for an all-zero part), codes are
+ *                 round-to-nearest-even with saturation.
+ *
+ * Rotary convention: interleaved pairs (D-64+2u, D-64+2u+1), u < 32, angle
+ * pos * base^(-2u/64) formed and reduced in float64.
+ */
+#ifndef CSA_B200_CSA_H_
+#define CSA_B200_CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CSA_API __attribute__((visibility("default")))
+#else
+#define CSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum csa_status {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = 1,     /* bad pointer, size, alignment or layer field */
+  CSA_ERR_UNSUPPORTED = 2,     /* valid, but no kernel for this shape / format */
+  CSA_ERR_WORKSPACE = 3,       /* workspace missing or smaller than csa_workspace_size() */
+  CSA_ERR_CUDA = 4,            /* a CUDA runtime call failed (message in csa_last_error) */
+  CSA_ERR_DEVICE_TIMEOUT = 5   /* a bounded device wait gave up (csa_device_error) */
+} csa_status_t;
+
+enum {
+  CSA_FMT_F32 = 0,
+  CSA_FMT_BF16 = 1,
+  CSA_FMT_MIXED = 2,           /* kv_format only */
+  CSA_FMT_E4M3 = 3             /* idx_format only */
+};
+
+enum { CSA_KIND_CSA = 0, CSA_KIND_HCA = 1 };
+
+/* One layer's hyper-parameters. */
+typedef struct csa_layer {
+  int32_t kind;          /* CSA_KIND_CSA or CSA_KIND_HCA */
+  int32_t B;             /* sequences */
+  int32_t H;             /* query heads (all share the one KV head) */
+  int32_t D;             /* KV / head dim; the last d_rope dims are rotary */
+  int32_t d_rope;        /* must be 64 */
+  int32_t m;             /* raw rows per compressed entry (4 for CSA, 128 for HCA) */
+  int32_t overlap;       /* 1: entry i pools raw rows [(i-1)m, (i+1)m); 0: [im, (i+1)m) */
+  int32_t top_k;         /* CSA: entries kept per query; ignored for HCA */
+  int32_t window;        /* w: most recent raw rows attended uncompressed (incl. current) */
+  int32_t H_I;           /* CSA: indexer heads */
+  int32_t d_I;           /* CSA: indexer head dim */
+  int32_t kv_format;     /* CSA_FMT_F32 | CSA_FMT_BF16 | CSA_FMT_MIXED */
+  int32_t idx_format;    /* CSA_FMT_F32 | CSA_FMT_E4M3 (index keys and index queries) */
+  int32_t act_format;    /* CSA_FMT_F32 | CSA_FMT_BF16: queries, raw rows, gate logits, output */
+  double rope_base;      /* rotary base (10000) */
+  float eps;             /* RMSNorm epsilon (1e-6) */
+  float softmax_scale;   /* logit scale; 0 selects 1/sqrt(D) */
+  int64_t pos0;          /* absolute position of raw row 0 */
+} csa_layer_t;
+
+/* Per-layer caches (state carried across decode steps; caller-owned). */
+typedef struct csa_cache {
+  void* entries;          /* [B][entry_cap][row_bytes] compressed entries, entry i at slot i */
+  int64_t entry_cap;      /* capacity in entries per sequence */
+  void* idx_keys;         /* CSA: [B][entry_cap][d_I] index keys (e4m3 codes or float32) */
+  const float* idx_key_scale; /* CSA: [B][entry_cap] per-key scale (all 1 for float32 keys) */
+  void* window;           /* [B][window_cap][row_bytes]: raw row r's rotated row at slot r mod window_cap */
+  int64_t window_cap;     /* >= window; >= Tq + window - 1 for a Tq-token chunk */
+  void* raw;              /* [B][raw_cap][D] un-rotated raw rows (act_format); row r at slot (r - raw_base) mod raw_cap */
+  void* gate;             /* [B][raw_cap][D] gate logits, same indexing as raw */
+  int64_t raw_cap;        /* decode: >= (1+overlap)*m; prefill: the chunk plus overlap*m look-back rows */
+  int64_t raw_base;       /* raw row stored at slot 0 (0 for a ring) */
+} csa_cache_t;
+
+/* Learned per-layer parameters. */
+typedef struct csa_params {
+  const float* pos_bias;  /* [(1+overlap)*m][D] positional bias per window slot and channel */
+  const float* gamma_kv;  /* [D] RMSNorm weight of compressed entries, or NULL (= 1) */
+  const float* gamma_q;   /* [D] RMSNorm weight of queries, or NULL (= 1) */
+  const float* sinks;     /* [H] per-head sink logits */
+} csa_params_t;
+
+/* Operation selector for csa_workspace_size(). */
+enum {
+  CSA_OP_INDEX_TOPK = 0,
+  CSA_OP_SPARSE_ATTEND = 1,
+  CSA_OP_HCA_ATTEND = 2,
+  CSA_OP_DECODE_STEP = 3,   /* csa_decode_step / hca_decode_step */
+  CSA_OP_PREFILL = 4        /* csa_prefill */
+};
+
+/* Bytes of one stored row for the layer's kv_format (host). */
+CSA_API size_t csa_row_bytes(const csa_layer_t* L);
+
+/* Workspace bytes an operation needs for Tq queries per sequence and caches
+ * of entry_cap entries (host; 0 if the layer is invalid). */
+CSA_API size_t csa_workspace_size(const csa_layer_t* L, int32_t op, int32_t Tq, int64_t entry_cap);
+
+/* Thread-local text of the last error returned on this thread (host). */
+CSA_API const char* csa_last_error(void);
+
+/* Library version string (host). */
+CSA_API const char* csa_version(void);
+
+/* Reads and clears the workspace's device error word (synchronises the
+ * stream).  *code gets the bits set by kernels whose bounded waits gave up
+ * (0 = none); returns CSA_ERR_DEVICE_TIMEOUT if any bit was set. */
+CSA_API csa_status_t csa_device_error(void* workspace, size_t ws_bytes, void* stream, int32_t* code);
+
+/* Append Tq new tokens per sequence: raw rows x_new[b][j] (and gate rows
+ * g_new) are written into the raw / gate rings at slot (r - raw_base) mod
+ * raw_cap (skipped when x_new is NULL: the rows are then already in the raw
+ * buffer), and each token's window row RoPE_t(x) -- rotated at its own
+ * position, not normalised -- is stored at window slot r mod window_cap.
+ *   x_new, g_new: [B][Tq][D] act_format, or both NULL.
+ * The sliding window is the pages' "small sliding-window branch of
+ * uncompressed recent tokens" ("DeepSeek-V4 Explained: ...", "The attention
+ * stack, and why it is two mechanisms"). */
+CSA_API csa_status_t csa_append(const csa_layer_t* L, const csa_cache_t* cache,
+                        const void* x_new, const void* g_new,
+                        const int64_t* q_pos, int32_t Tq, void* stream);
+
+/* Compress every entry completed by the Tq tokens at q_pos (entry i is
+ * completed by raw row (i+1)m - 1).  Entry i = RoPE_{pos0 + i m}(RMSNorm(e) *
+ * gamma_kv) with e_c = sum_r softmax_r(gate[r][c] + pos_bias[r - (i-ov)m][c])
+ * * raw[r][c] over raw rows r in [(i-ov)m, (i+1)m) clipped at 0, written to
+ * entries[b][i] in kv_format.  The raw buffer must hold those rows.
+ * Pages: "compresses the key-value cache of every group of m consecutive
+ * tokens into one entry using learned compression weights and positional
+ * biases" ("DeepSeek-V4 Explained: ..."); "each compressed entry draws from
+ * 2m source entries while the sequence still shrinks by m" ("DeepSeek-V4:
+ * Making a Million Tokens Affordable", "Two ways to shrink attention"). */
+CSA_API csa_status_t csa_compress(const csa_layer_t* L, const csa_cache_t* cache,
+                          const csa_params_t* P, const int64_t* q_pos, int32_t Tq,
+                          void* stream);
+
+/* Lightning indexer + top-k (CSA).  For query (b, j) at position t, entry i
+ * is visible iff pos0 + (i+1)m - 1 <= t; its score is
+ *   s_i = sum_h head_w[h] * max(0, idx_q_scale[h] * idx_key_scale[i] * <idx_q[h], idx_key[i]>)
+ * and the k highest scores are kept, ties to the smaller index, written in
+ * ascending entry order to topk_idx[b][j][0..k), padded with -1 when fewer
+ * than k entries are visible.
+ *   idx_q:       [B][Tq][H_I][d_I] e4m3 codes or float32
+ *   idx_q_scale: [B][Tq][H_I] float32;  head_w: [B][Tq][H_I] float32
+ *   n_max:       entries scored per query (<= entry_cap; entries beyond the
+ *                query's visible count are excluded)
+ *   topk_idx:    [B][Tq][top_k] int32 (output)
+ *   scores:      [B][Tq][n_max] float32 (output, optional: NULL keeps them in the workspace)
+ * Pages: "a Lightning Indexer scores them in a low-rank way and each query
+ * attends only to the top-k compressed entries" ("DeepSeek-V4 Explained");
+ * "a few small heads run in FP8" ("DeepSeek-V4, explained.", step 3). */
+CSA_API csa_status_t csa_index_topk(const csa_layer_t* L, const csa_cache_t* cache,
+                            const void* idx_q, const float* idx_q_scale, const float* head_w,
+                            const int64_t* q_pos, int32_t Tq, int64_t n_max,
+                            int32_t* topk_idx, float* scores,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/* Sparse shared-KV multi-query attention (CSA).  For query (b, j) at t:
+ *   q~_h = RoPE_t(RMSNorm(q_h) * gamma_q);   keys = values = the selected
+ *   entries topk_idx[b][j][*] (-1 skipped) plus the window rows r in
+ *   [max(0, r_t - w + 1), r_t];  l_j = <q~_h, k_j> * softmax_scale;
+ *   o_h = sum_j e^{l_j} k_j / (e^{sink_h} + sum_j e^{l_j});  out = RoPE_{-t}(o_h).
+ *   q:   [B][Tq][H][D] act_format;  out: [B][Tq][H][D] act_format.
+ * Pages: "a compressed entry serves as both key and value ... RoPE at
+ * position -i is applied back to the attention output"; "learnable attention
+ * sinks" ("DeepSeek-V4: Making a Million Tokens Affordable"). */
+CSA_API csa_status_t csa_sparse_attend(const csa_layer_t* L, const csa_cache_t* cache,
+                               const csa_params_t* P, const void* q, const int64_t* q_pos,
+                               int32_t Tq, const int32_t* topk_idx, void* out,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+/* Dense attention over every visible entry i < n_visible(t) (HCA) plus the
+ * window rows, otherwise as csa_sparse_attend.  n_max bounds the visible
+ * entries (<= entry_cap).
+ * Pages: "keep attention fully dense over what remains. No indexer, no
+ * top-k" ("DeepSeek-V4: Making a Million Tokens Affordable"). */
+CSA_API csa_status_t hca_attend(const csa_layer_t* L, const csa_cache_t* cache,
+                        const csa_params_t* P, const void* q, const int64_t* q_pos,
+                        int32_t Tq, int64_t n_max, void* out,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* One fused CSA decode step for token t = q_pos[b] of every sequence:
+ * csa_append (x_new, g_new) -> csa_compress (when t completes a group) ->
+ * csa_index_topk over entry_cap entries -> csa_sparse_attend.  Tq = 1.
+ * topk_idx: [B][top_k] int32 output, or NULL (kept in the workspace). */
+CSA_API csa_status_t csa_decode_step(const csa_layer_t* L, const csa_cache_t* cache,
+                             const csa_params_t* P, const void* q,
+                             const void* idx_q, const float* idx_q_scale, const float* head_w,
+                             const void* x_new, const void* g_new, const int64_t* q_pos,
+                             void* out, int32_t* topk_idx,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* One fused HCA decode step: csa_append -> csa_compress -> hca_attend. */
+CSA_API csa_status_t hca_decode_step(const csa_layer_t* L, const csa_cache_t* cache,
+                             const csa_params_t* P, const void* q,
+                             const void* x_new, const void* g_new, const int64_t* q_pos,
+                             void* out, void* workspace, size_t ws_bytes, void* stream);
+
+/* Chunked prefill of Tq tokens per sequence (CSA or HCA): csa_append of the
+ * chunk's window rows (raw rows already in cache->raw), csa_compress of the
+ * entries the chunk completes, then per query the indexer + top-k (CSA) and
+ * attention.  n_max = entries visible to the chunk's last query. */
+CSA_API csa_status_t csa_prefill(const csa_layer_t* L, const csa_cache_t* cache,
+                         const csa_params_t* P, const void* q,
+                         const void* idx_q, const float* idx_q_scale, const float* head_w,
+                         const int64_t* q_pos, int32_t Tq, int64_t n_max,
+                         void* out, int32_t* topk_idx,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif  /* CSA_B200_CSA_H_ */

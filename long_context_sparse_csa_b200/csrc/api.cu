@@ -1,0 +1,462 @@
+// C ABI of the CSA/HCA operator: argument checks, workspace layout, launches.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "csa.h"
+#include "kernels.h"
+
+using namespace csa;
+
+namespace {
+
+thread_local std::string g_err;
+
+csa_status_t fail(csa_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+csa_status_t cuda_fail(cudaError_t e, const char* where) {
+  return fail(CSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int num_sms() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static int cached[64] = {0};
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+size_t row_bytes_of(const csa_layer_t* L) {
+  switch (L->kv_format) {
+    case CSA_FMT_F32: return 4 * (size_t)L->D;
+    case CSA_FMT_BF16: return 2 * (size_t)L->D;
+    case CSA_FMT_MIXED: return (size_t)L->D + 80;
+    default: return 0;
+  }
+}
+
+csa_status_t check_layer(const csa_layer_t* L) {
+  if (!L) return fail(CSA_ERR_INVALID_ARG, "layer is NULL");
+  if (L->kind != CSA_KIND_CSA && L->kind != CSA_KIND_HCA) return fail(CSA_ERR_INVALID_ARG, "kind %d", L->kind);
+  if (L->B < 1 || L->H < 1) return fail(CSA_ERR_INVALID_ARG, "B=%d H=%d", L->B, L->H);
+  if (L->D < 128 || L->D > 1024 || L->D % 128) return fail(CSA_ERR_UNSUPPORTED, "D=%d (needs a multiple of 128, <= 1024)", L->D);
+  if (L->d_rope != 64) return fail(CSA_ERR_UNSUPPORTED, "d_rope=%d (only 64)", L->d_rope);
+  if (L->m < 1) return fail(CSA_ERR_INVALID_ARG, "m=%d", L->m);
+  if (L->overlap != 0 && L->overlap != 1) return fail(CSA_ERR_INVALID_ARG, "overlap=%d", L->overlap);
+  if (L->window < 1) return fail(CSA_ERR_INVALID_ARG, "window=%d", L->window);
+  if (L->kv_format != CSA_FMT_F32 && L->kv_format != CSA_FMT_BF16 && L->kv_format != CSA_FMT_MIXED)
+    return fail(CSA_ERR_INVALID_ARG, "kv_format=%d", L->kv_format);
+  if (L->act_format != CSA_FMT_F32 && L->act_format != CSA_FMT_BF16)
+    return fail(CSA_ERR_INVALID_ARG, "act_format=%d", L->act_format);
+  if (!(L->rope_base > 0)) return fail(CSA_ERR_INVALID_ARG, "rope_base must be > 0");
+  if (!(L->eps >= 0)) return fail(CSA_ERR_INVALID_ARG, "eps must be >= 0");
+  if (L->kind == CSA_KIND_CSA) {
+    if (L->top_k < 1) return fail(CSA_ERR_INVALID_ARG, "top_k=%d", L->top_k);
+    if (L->H_I < 1 || L->d_I < 1) return fail(CSA_ERR_INVALID_ARG, "H_I=%d d_I=%d", L->H_I, L->d_I);
+    if (L->idx_format != CSA_FMT_F32 && L->idx_format != CSA_FMT_E4M3)
+      return fail(CSA_ERR_INVALID_ARG, "idx_format=%d", L->idx_format);
+    if (L->d_I % 16) return fail(CSA_ERR_UNSUPPORTED, "d_I=%d (needs a multiple of 16)", L->d_I);
+    if ((size_t)L->H_I * L->d_I * 4 > 96 * 1024) return fail(CSA_ERR_UNSUPPORTED, "H_I*d_I too large");
+  }
+  return CSA_OK;
+}
+
+LayerArgs layer_args(const csa_layer_t* L) {
+  LayerArgs a;
+  a.B = L->B; a.H = L->H; a.D = L->D; a.d_rope = L->d_rope; a.m = L->m; a.ov = L->overlap;
+  a.top_k = L->top_k; a.window = L->window; a.H_I = L->H_I; a.d_I = L->d_I;
+  a.kv_fmt = L->kv_format; a.idx_fmt = L->idx_format; a.act_fmt = L->act_format;
+  a.row_bytes = (int)row_bytes_of(L);
+  a.rope_base = L->rope_base;
+  a.eps = L->eps;
+  a.scale = L->softmax_scale > 0 ? L->softmax_scale : 1.0f / sqrtf((float)L->D);
+  a.pos0 = L->pos0;
+  return a;
+}
+
+CacheArgs cache_args(const csa_cache_t* c) {
+  CacheArgs a;
+  a.entries = static_cast<uint8_t*>(c->entries);
+  a.entry_cap = c->entry_cap;
+  a.idx_keys = static_cast<const uint8_t*>(c->idx_keys);
+  a.idx_key_scale = c->idx_key_scale;
+  a.window = static_cast<uint8_t*>(c->window);
+  a.window_cap = c->window_cap;
+  a.raw = static_cast<uint8_t*>(c->raw);
+  a.gate = static_cast<uint8_t*>(c->gate);
+  a.raw_cap = c->raw_cap;
+  a.raw_base = c->raw_base;
+  return a;
+}
+
+csa_status_t need_ptr(const void* p, const char* name, size_t align = 16) {
+  if (!p) return fail(CSA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(p, align)) return fail(CSA_ERR_INVALID_ARG, "%s is not %zu-byte aligned", name, align);
+  return CSA_OK;
+}
+
+#define CSA_TRY(x)                     \
+  do {                                 \
+    csa_status_t _st = (x);            \
+    if (_st != CSA_OK) return _st;     \
+  } while (0)
+
+csa_status_t check_cache_attend(const csa_layer_t* L, const csa_cache_t* c) {
+  if (!c) return fail(CSA_ERR_INVALID_ARG, "cache is NULL");
+  CSA_TRY(need_ptr(c->entries, "cache.entries"));
+  CSA_TRY(need_ptr(c->window, "cache.window"));
+  if (c->entry_cap < 1) return fail(CSA_ERR_INVALID_ARG, "entry_cap=%lld", (long long)c->entry_cap);
+  if (c->window_cap < L->window) return fail(CSA_ERR_INVALID_ARG, "window_cap < window");
+  return CSA_OK;
+}
+
+csa_status_t check_cache_raw(const csa_layer_t* L, const csa_cache_t* c, bool need_gate) {
+  CSA_TRY(need_ptr(c->raw, "cache.raw"));
+  if (need_gate) CSA_TRY(need_ptr(c->gate, "cache.gate"));
+  if (c->raw_cap < 1) return fail(CSA_ERR_INVALID_ARG, "raw_cap=%lld", (long long)c->raw_cap);
+  (void)L;
+  return CSA_OK;
+}
+
+// ----------------------------------------------------------------------------- workspace layout
+constexpr size_t kAlign = 256;
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Workspace {
+  size_t err = 0;          // int error word
+  size_t scores = 0, scores_bytes = 0;
+  size_t topk = 0, topk_bytes = 0;
+  size_t part = 0, part_bytes = 0;
+  size_t total = 0;
+};
+
+Workspace layout(const csa_layer_t* L, int op, int32_t Tq, int64_t n_max) {
+  Workspace w;
+  const LayerArgs la = layer_args(L);
+  const size_t rows = (size_t)L->B * (size_t)(Tq > 0 ? Tq : 1);
+  size_t off = up(64);
+  const bool csa = L->kind == CSA_KIND_CSA;
+  if (csa && (op == CSA_OP_INDEX_TOPK || op == CSA_OP_DECODE_STEP || op == CSA_OP_PREFILL)) {
+    w.scores = off; w.scores_bytes = rows * (size_t)(n_max > 0 ? n_max : 1) * 4; off = up(off + w.scores_bytes);
+  }
+  if (csa && (op == CSA_OP_DECODE_STEP || op == CSA_OP_PREFILL)) {
+    w.topk = off; w.topk_bytes = rows * (size_t)L->top_k * 4; off = up(off + w.topk_bytes);
+  }
+  if (op == CSA_OP_SPARSE_ATTEND || op == CSA_OP_HCA_ATTEND || op == CSA_OP_DECODE_STEP || op == CSA_OP_PREFILL) {
+    const bool dense = (op == CSA_OP_HCA_ATTEND) || !csa;
+    const int64_t slots = (dense ? (n_max > 0 ? n_max : 1) : (int64_t)L->top_k) + L->window;
+    const int splits = attend_num_splits(la, (int)rows, slots, num_sms());
+    w.part = off; w.part_bytes = attend_partial_bytes(la, (int)rows, splits); off = up(off + w.part_bytes);
+  }
+  w.total = off;
+  return w;
+}
+
+csa_status_t check_ws(const Workspace& w, void* ws, size_t ws_bytes) {
+  if (!ws) return fail(CSA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", w.total);
+  if (!aligned(ws, kAlign)) return fail(CSA_ERR_WORKSPACE, "workspace must be %zu-byte aligned", kAlign);
+  if (ws_bytes < w.total) return fail(CSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, w.total);
+  return CSA_OK;
+}
+
+uint8_t* at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
+
+// ----------------------------------------------------------------------------- step bodies
+csa_status_t run_append_compress(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P,
+                                 const void* x_new, const void* g_new, const int64_t* q_pos, int32_t Tq,
+                                 bool do_append, bool do_compress, cudaStream_t s) {
+  AppendCompressArgs a;
+  a.L = layer_args(L);
+  a.C = cache_args(cache);
+  a.q_pos = q_pos;
+  a.Tq = Tq;
+  a.x_new = static_cast<const uint8_t*>(x_new);
+  a.g_new = static_cast<const uint8_t*>(g_new);
+  a.pos_bias = P ? P->pos_bias : nullptr;
+  a.gamma_kv = P ? P->gamma_kv : nullptr;
+  a.do_append = do_append;
+  a.do_compress = do_compress;
+  cudaError_t e = launch_append_compress(a, L->B, Tq, s);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e, "append/compress launch");
+}
+
+csa_status_t run_index_topk(const csa_layer_t* L, const csa_cache_t* cache, const void* idx_q,
+                            const float* idx_q_scale, const float* head_w, const int64_t* q_pos, int32_t Tq,
+                            int64_t n_max, int32_t* topk, float* scores, int* err, cudaStream_t s) {
+  IndexArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = L->B; a.Tq = Tq; a.H_I = L->H_I; a.d_I = L->d_I; a.m = L->m;
+  a.idx_fmt = L->idx_format;
+  a.n_max = n_max; a.entry_cap = cache->entry_cap; a.pos0 = L->pos0;
+  a.q_pos = q_pos;
+  a.idx_q = static_cast<const uint8_t*>(idx_q);
+  a.idx_k = static_cast<const uint8_t*>(cache->idx_keys);
+  a.k_scale = cache->idx_key_scale;
+  a.q_scale = idx_q_scale;
+  a.head_w = head_w;
+  a.scores = scores;
+  a.err = err;
+  cudaError_t e = launch_index_scores(a, num_sms(), s);
+  if (e != cudaSuccess) return cuda_fail(e, "index-score launch");
+  TopkArgs t;
+  t.scores = scores; t.n_max = n_max; t.rows = L->B * Tq; t.Tq = Tq; t.m = L->m; t.k = L->top_k;
+  t.pos0 = L->pos0; t.q_pos = q_pos; t.out = topk;
+  e = launch_topk(t, s);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e, "top-k launch");
+}
+
+csa_status_t run_attend(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P, const void* q,
+                        const int64_t* q_pos, int32_t Tq, const int32_t* topk, int64_t n_max, void* out,
+                        const Workspace& w, void* ws, cudaStream_t s) {
+  AttendArgs a;
+  a.L = layer_args(L);
+  if (attend_head_group(a.L) == 0 && L->H > 32)
+    return fail(CSA_ERR_UNSUPPORTED, "attention: H=%d needs D=512 with bf16/mixed rows and H%%32==0, or H<=32", L->H);
+  a.C = cache_args(cache);
+  a.q = static_cast<const uint8_t*>(q);
+  a.q_pos = q_pos;
+  a.Tq = Tq;
+  a.rows = L->B * Tq;
+  a.topk = topk;
+  a.n_max = n_max;
+  a.gamma_q = P->gamma_q;
+  a.sinks = P->sinks;
+  const int64_t slots = (topk ? (int64_t)L->top_k : n_max) + L->window;
+  a.splits = attend_num_splits(a.L, a.rows, slots, num_sms());
+  if (attend_partial_bytes(a.L, a.rows, a.splits) > w.part_bytes)
+    return fail(CSA_ERR_WORKSPACE, "workspace too small for the attention partials");
+  a.part = reinterpret_cast<float*>(at(ws, w.part));
+  a.out = static_cast<uint8_t*>(out);
+  cudaError_t e = launch_attend(a, s);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e, "attention launch");
+}
+
+csa_status_t check_params(const csa_layer_t* L, const csa_params_t* P, bool need_bias) {
+  if (!P) return fail(CSA_ERR_INVALID_ARG, "params is NULL");
+  if (need_bias) CSA_TRY(need_ptr(P->pos_bias, "params.pos_bias"));
+  if (!P->sinks && !need_bias) return fail(CSA_ERR_INVALID_ARG, "params.sinks is NULL");
+  (void)L;
+  return CSA_OK;
+}
+
+}  // namespace
+
+// ============================================================================= exported
+extern "C" {
+
+size_t csa_row_bytes(const csa_layer_t* L) { return L ? row_bytes_of(L) : 0; }
+
+size_t csa_workspace_size(const csa_layer_t* L, int32_t op, int32_t Tq, int64_t entry_cap) {
+  if (check_layer(L) != CSA_OK) return 0;
+  return layout(L, op, Tq, entry_cap).total;
+}
+
+const char* csa_last_error(void) { return g_err.c_str(); }
+
+const char* csa_version(void) { return "csa-b200 0.1 (sm_100a)"; }
+
+csa_status_t csa_device_error(void* workspace, size_t ws_bytes, void* stream, int32_t* code) {
+  if (!workspace || ws_bytes < 4) return fail(CSA_ERR_WORKSPACE, "workspace is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess && v) e = cudaMemsetAsync(workspace, 0, 4, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "csa_device_error");
+  if (code) *code = v;
+  return v ? fail(CSA_ERR_DEVICE_TIMEOUT, "device error word 0x%x", v) : CSA_OK;
+}
+
+csa_status_t csa_append(const csa_layer_t* L, const csa_cache_t* cache, const void* x_new, const void* g_new,
+                        const int64_t* q_pos, int32_t Tq, void* stream) {
+  CSA_TRY(check_layer(L));
+  if (!cache) return fail(CSA_ERR_INVALID_ARG, "cache is NULL");
+  CSA_TRY(need_ptr(cache->window, "cache.window"));
+  CSA_TRY(check_cache_raw(L, cache, x_new != nullptr));
+  CSA_TRY(need_ptr(q_pos, "q_pos", 8));
+  if (Tq < 1) return fail(CSA_ERR_INVALID_ARG, "Tq=%d", Tq);
+  if ((x_new == nullptr) != (g_new == nullptr)) return fail(CSA_ERR_INVALID_ARG, "x_new and g_new must both be given or both NULL");
+  if (x_new) { CSA_TRY(need_ptr(x_new, "x_new")); CSA_TRY(need_ptr(g_new, "g_new")); }
+  if (cache->window_cap < L->window) return fail(CSA_ERR_INVALID_ARG, "window_cap < window");
+  return run_append_compress(L, cache, nullptr, x_new, g_new, q_pos, Tq, true, false, static_cast<cudaStream_t>(stream));
+}
+
+csa_status_t csa_compress(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P,
+                          const int64_t* q_pos, int32_t Tq, void* stream) {
+  CSA_TRY(check_layer(L));
+  if (!cache) return fail(CSA_ERR_INVALID_ARG, "cache is NULL");
+  CSA_TRY(need_ptr(cache->entries, "cache.entries"));
+  CSA_TRY(check_cache_raw(L, cache, true));
+  CSA_TRY(check_params(L, P, true));
+  CSA_TRY(need_ptr(q_pos, "q_pos", 8));
+  if (Tq < 1) return fail(CSA_ERR_INVALID_ARG, "Tq=%d", Tq);
+  return run_append_compress(L, cache, P, nullptr, nullptr, q_pos, Tq, false, true, static_cast<cudaStream_t>(stream));
+}
+
+csa_status_t csa_index_topk(const csa_layer_t* L, const csa_cache_t* cache, const void* idx_q,
+                            const float* idx_q_scale, const float* head_w, const int64_t* q_pos, int32_t Tq,
+                            int64_t n_max, int32_t* topk_idx, float* scores, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  CSA_TRY(check_layer(L));
+  if (L->kind != CSA_KIND_CSA) return fail(CSA_ERR_INVALID_ARG, "csa_index_topk needs a CSA layer");
+  if (!cache) return fail(CSA_ERR_INVALID_ARG, "cache is NULL");
+  CSA_TRY(need_ptr(cache->idx_keys, "cache.idx_keys"));
+  CSA_TRY(need_ptr(cache->idx_key_scale, "cache.idx_key_scale", 4));
+  CSA_TRY(need_ptr(idx_q, "idx_q"));
+  CSA_TRY(need_ptr(idx_q_scale, "idx_q_scale", 4));
+  CSA_TRY(need_ptr(head_w, "head_w", 4));
+  CSA_TRY(need_ptr(q_pos, "q_pos", 8));
+  CSA_TRY(need_ptr(topk_idx, "topk_idx", 4));
+  if (Tq < 1) return fail(CSA_ERR_INVALID_ARG, "Tq=%d", Tq);
+  if (n_max < 0 || n_max > cache->entry_cap) return fail(CSA_ERR_INVALID_ARG, "n_max=%lld outside [0, entry_cap]", (long long)n_max);
+  const Workspace w = layout(L, CSA_OP_INDEX_TOPK, Tq, n_max);
+  CSA_TRY(check_ws(w, workspace, ws_bytes));
+  if (scores) CSA_TRY(need_ptr(scores, "scores", 4));
+  float* sc = scores ? scores : reinterpret_cast<float*>(at(workspace, w.scores));
+  return run_index_topk(L, cache, idx_q, idx_q_scale, head_w, q_pos, Tq, n_max, topk_idx, sc,
+                        reinterpret_cast<int*>(at(workspace, w.err)), static_cast<cudaStream_t>(stream));
+}
+
+csa_status_t csa_sparse_attend(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P,
+                               const void* q, const int64_t* q_pos, int32_t Tq, const int32_t* topk_idx,
+                               void* out, void* workspace, size_t ws_bytes, void* stream) {
+  CSA_TRY(check_layer(L));
+  if (L->kind != CSA_KIND_CSA) return fail(CSA_ERR_INVALID_ARG, "csa_sparse_attend needs a CSA layer");
+  CSA_TRY(check_cache_attend(L, cache));
+  CSA_TRY(check_params(L, P, false));
+  CSA_TRY(need_ptr(P->sinks, "params.sinks", 4));
+  CSA_TRY(need_ptr(q, "q"));
+  CSA_TRY(need_ptr(q_pos, "q_pos", 8));
+  CSA_TRY(need_ptr(topk_idx, "topk_idx", 4));
+  CSA_TRY(need_ptr(out, "out"));
+  if (Tq < 1) return fail(CSA_ERR_INVALID_ARG, "Tq=%d", Tq);
+  const Workspace w = layout(L, CSA_OP_SPARSE_ATTEND, Tq, cache->entry_cap);
+  CSA_TRY(check_ws(w, workspace, ws_bytes));
+  return run_attend(L, cache, P, q, q_pos, Tq, topk_idx, cache->entry_cap, out, w, workspace,
+                    static_cast<cudaStream_t>(stream));
+}
+
+csa_status_t hca_attend(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P, const void* q,
+                        const int64_t* q_pos, int32_t Tq, int64_t n_max, void* out, void* workspace,
+                        size_t ws_bytes, void* stream) {
+  CSA_TRY(check_layer(L));
+  CSA_TRY(check_cache_attend(L, cache));
+  CSA_TRY(check_params(L, P, false));
+  CSA_TRY(need_ptr(P->sinks, "params.sinks", 4));
+  CSA_TRY(need_ptr(q, "q"));
+  CSA_TRY(need_ptr(q_pos, "q_pos", 8));
+  CSA_TRY(need_ptr(out, "out"));
+  if (Tq < 1) return fail(CSA_ERR_INVALID_ARG, "Tq=%d", Tq);
+  if (n_max < 0 || n_max > cache->entry_cap) return fail(CSA_ERR_INVALID_ARG, "n_max outside [0, entry_cap]");
+  const Workspace w = layout(L, CSA_OP_HCA_ATTEND, Tq, n_max);
+  CSA_TRY(check_ws(w, workspace, ws_bytes));
+  return run_attend(L, cache, P, q, q_pos, Tq, nullptr, n_max, out, w, workspace, static_cast<cudaStream_t>(stream));
+}
+
+csa_status_t csa_decode_step(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P, const void* q,
+                             const void* idx_q, const float* idx_q_scale, const float* head_w, const void* x_new,
+                             const void* g_new, const int64_t* q_pos, void* out, int32_t* topk_idx,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  CSA_TRY(check_layer(L));
+  if (L->kind != CSA_KIND_CSA) return fail(CSA_ERR_INVALID_ARG, "csa_decode_step needs a CSA layer");
+  CSA_TRY(check_cache_attend(L, cache));
+  CSA_TRY(check_cache_raw(L, cache, true));
+  CSA_TRY(need_ptr(cache->idx_keys, "cache.idx_keys"));
+  CSA_TRY(need_ptr(cache->idx_key_scale, "cache.idx_key_scale", 4));
+  CSA_TRY(check_params(L, P, true));
+  CSA_TRY(need_ptr(P->sinks, "params.sinks", 4));
+  CSA_TRY(need_ptr(q, "q"));
+  CSA_TRY(need_ptr(idx_q, "idx_q"));
+  CSA_TRY(need_ptr(idx_q_scale, "idx_q_scale", 4));
+  CSA_TRY(need_ptr(head_w, "head_w", 4));
+  CSA_TRY(need_ptr(x_new, "x_new"));
+  CSA_TRY(need_ptr(g_new, "g_new"));
+  CSA_TRY(need_ptr(q_pos, "q_pos", 8));
+  CSA_TRY(need_ptr(out, "out"));
+  if (topk_idx) CSA_TRY(need_ptr(topk_idx, "topk_idx", 4));
+  if (cache->raw_cap < (1 + L->overlap) * (int64_t)L->m) return fail(CSA_ERR_INVALID_ARG, "raw_cap < (1+overlap)*m");
+  const Workspace w = layout(L, CSA_OP_DECODE_STEP, 1, cache->entry_cap);
+  CSA_TRY(check_ws(w, workspace, ws_bytes));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CSA_TRY(run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, s));
+  int32_t* tk = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(at(workspace, w.topk));
+  CSA_TRY(run_index_topk(L, cache, idx_q, idx_q_scale, head_w, q_pos, 1, cache->entry_cap, tk,
+                         reinterpret_cast<float*>(at(workspace, w.scores)), reinterpret_cast<int*>(at(workspace, w.err)), s));
+  return run_attend(L, cache, P, q, q_pos, 1, tk, cache->entry_cap, out, w, workspace, s);
+}
+
+csa_status_t hca_decode_step(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P, const void* q,
+                             const void* x_new, const void* g_new, const int64_t* q_pos, void* out,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  CSA_TRY(check_layer(L));
+  CSA_TRY(check_cache_attend(L, cache));
+  CSA_TRY(check_cache_raw(L, cache, true));
+  CSA_TRY(check_params(L, P, true));
+  CSA_TRY(need_ptr(P->sinks, "params.sinks", 4));
+  CSA_TRY(need_ptr(q, "q"));
+  CSA_TRY(need_ptr(x_new, "x_new"));
+  CSA_TRY(need_ptr(g_new, "g_new"));
+  CSA_TRY(need_ptr(q_pos, "q_pos", 8));
+  CSA_TRY(need_ptr(out, "out"));
+  if (cache->raw_cap < (1 + L->overlap) * (int64_t)L->m) return fail(CSA_ERR_INVALID_ARG, "raw_cap < (1+overlap)*m");
+  const Workspace w = layout(L, CSA_OP_HCA_ATTEND, 1, cache->entry_cap);
+  CSA_TRY(check_ws(w, workspace, ws_bytes));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CSA_TRY(run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, s));
+  return run_attend(L, cache, P, q, q_pos, 1, nullptr, cache->entry_cap, out, w, workspace, s);
+}
+
+csa_status_t csa_prefill(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P, const void* q,
+                         const void* idx_q, const float* idx_q_scale, const float* head_w, const int64_t* q_pos,
+                         int32_t Tq, int64_t n_max, void* out, int32_t* topk_idx, void* workspace, size_t ws_bytes,
+                         void* stream) {
+  CSA_TRY(check_layer(L));
+  CSA_TRY(check_cache_attend(L, cache));
+  CSA_TRY(check_cache_raw(L, cache, true));
+  CSA_TRY(check_params(L, P, true));
+  CSA_TRY(need_ptr(P->sinks, "params.sinks", 4));
+  CSA_TRY(need_ptr(q, "q"));
+  CSA_TRY(need_ptr(q_pos, "q_pos", 8));
+  CSA_TRY(need_ptr(out, "out"));
+  if (Tq < 1) return fail(CSA_ERR_INVALID_ARG, "Tq=%d", Tq);
+  if (n_max < 0 || n_max > cache->entry_cap) return fail(CSA_ERR_INVALID_ARG, "n_max outside [0, entry_cap]");
+  if (cache->window_cap < (int64_t)Tq + L->window - 1)
+    return fail(CSA_ERR_INVALID_ARG, "window_cap must hold Tq + window - 1 rows for a chunk");
+  const bool csa = L->kind == CSA_KIND_CSA;
+  if (csa) {
+    CSA_TRY(need_ptr(cache->idx_keys, "cache.idx_keys"));
+    CSA_TRY(need_ptr(cache->idx_key_scale, "cache.idx_key_scale", 4));
+    CSA_TRY(need_ptr(idx_q, "idx_q"));
+    CSA_TRY(need_ptr(idx_q_scale, "idx_q_scale", 4));
+    CSA_TRY(need_ptr(head_w, "head_w", 4));
+    if (topk_idx) CSA_TRY(need_ptr(topk_idx, "topk_idx", 4));
+  }
+  const Workspace w = layout(L, CSA_OP_PREFILL, Tq, n_max);
+  CSA_TRY(check_ws(w, workspace, ws_bytes));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CSA_TRY(run_append_compress(L, cache, P, nullptr, nullptr, q_pos, Tq, true, true, s));
+  int32_t* tk = nullptr;
+  if (csa) {
+    tk = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(at(workspace, w.topk));
+    CSA_TRY(run_index_topk(L, cache, idx_q, idx_q_scale, head_w, q_pos, Tq, n_max, tk,
+                           reinterpret_cast<float*>(at(workspace, w.scores)), reinterpret_cast<int*>(at(workspace, w.err)), s));
+  }
+  return run_attend(L, cache, P, q, q_pos, Tq, tk, n_max, out, w, workspace, s);
+}
+
+}  // extern "C"

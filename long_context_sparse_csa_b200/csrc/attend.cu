@@ -1,0 +1,588 @@
+// Shared-KV multi-query attention over gathered KV rows with a sink logit.
+//
+// "a compressed entry serves as both key and value ... RoPE at position -i is
+// applied back to the attention output so the result carries relative
+// positions ... learnable attention sinks let a head route its attention
+// mass to nothing at all" and "queries and compressed entries get an extra
+// RMSNorm" -- "DeepSeek-V4: Making a Million Tokens Affordable", section
+// "Two ways to shrink attention, interleaved".  "Fetching whole contiguous
+// blocks, shared by the heads that share keys" -- "DeepSeek-V4, explained.",
+// step 8: every gathered row is loaded once per CTA and used by all of the
+// CTA's heads.
+//
+// Key slots of a query at raw row r_t: [0, n_sel) are compressed entries
+// (the top-k list for CSA, -1 skipped; every visible entry for HCA), then
+// [n_sel, n_sel + n_win) are the window rows r_t - n_win + 1 .. r_t.
+//
+// Tensor-core kernel (D = 512, BF16 or mixed BF16/FP8 rows): a CTA owns one
+// query, a group of HG heads (M = HG) and a contiguous range of 64-slot key
+// tiles.  Each tile is gathered row by row (16-byte vector loads; FP8 codes
+// times the row's power-of-two scale convert exactly to BF16) into a swizzled
+// shared-memory tile, S = Q K^T and O += P V run as bf16 mma.sync with fp32
+// accumulation and an online softmax.  When several CTAs split one query's
+// slots, each writes (O, m, l) and a combine kernel merges the splits with
+// the sink and applies the inverse rotation.
+#include "kernels.h"
+
+namespace csa {
+
+namespace {
+
+constexpr int kD = 512;
+constexpr int kTile = 64;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const uint8_t* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  return (uint32_t)f_to_bf16_bits(lo) | ((uint32_t)f_to_bf16_bits(hi) << 16);
+}
+
+// Swizzled byte offset of 16-byte chunk `ch` of row `row` in a tile whose rows are `pitch` bytes.
+__device__ __forceinline__ uint32_t swz(int row, int ch, int pitch) {
+  return (uint32_t)(row * pitch + (((ch ^ (row & 7))) << 4));
+}
+
+struct SlotInfo {
+  int64_t rt, n_sel, n_win, R;
+};
+
+__device__ __forceinline__ SlotInfo slot_info(const AttendArgs& a, int64_t t) {
+  SlotInfo s;
+  s.rt = t - a.L.pos0;
+  const int64_t r1 = s.rt + 1 > 0 ? s.rt + 1 : 0;
+  const int64_t nvis = r1 / a.L.m;
+  s.n_sel = a.topk ? (int64_t)a.L.top_k : (nvis < a.n_max ? nvis : a.n_max);
+  s.n_win = r1 < a.L.window ? r1 : a.L.window;
+  s.R = s.n_sel + s.n_win;
+  return s;
+}
+
+// Stored row of key slot s, or null when the slot holds nothing (-1 or out of range).
+__device__ __forceinline__ const uint8_t* slot_row(const AttendArgs& a, const SlotInfo& si, int row, int b,
+                                                   int64_t s) {
+  const CacheArgs& C = a.C;
+  if (s < si.n_sel) {
+    const int64_t e = a.topk ? (int64_t)a.topk[(size_t)row * a.L.top_k + s] : s;
+    if (e < 0 || e >= C.entry_cap) return nullptr;
+    return C.entries + ((size_t)b * C.entry_cap + (size_t)e) * a.L.row_bytes;
+  }
+  if (s < si.R) {
+    const int64_t wr = si.rt - si.n_win + 1 + (s - si.n_sel);
+    return C.window + ((size_t)b * C.window_cap + (size_t)(wr % C.window_cap)) * a.L.row_bytes;
+  }
+  return nullptr;
+}
+
+template <int HG, int FMT>
+__global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_constant__ AttendArgs a) {
+  constexpr int NW = HG / 4;          // warps
+  constexpr int NT = NW * 32;         // threads
+  constexpr int MT = HG / 16;         // m-tiles (16 heads each)
+  constexpr int DW = kD / NW;         // output dims per warp in P*V
+  constexpr int NTW = DW / 8;         // n-tiles per warp in P*V
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* Qs = smem;                                   // [HG][1024]  bf16 q~
+  uint8_t* Ks = Qs + HG * 1024;                         // [64][1024]  bf16 key/value tile
+  uint8_t* Ps = Ks + kTile * 1024;                      // [HG][128]   bf16 probabilities
+  float* pmax = reinterpret_cast<float*>(Ps + HG * 128);  // [4][HG]
+  float* psum = pmax + 4 * HG;                          // [4][HG]
+  float* m_run = psum + 4 * HG;                         // [HG]
+  float* l_run = m_run + HG;                            // [HG]
+  float* corr = l_run + HG;                             // [HG]
+  float* cs = corr + HG;                                // [32]
+  float* sn = cs + 32;                                  // [32]
+  const uint8_t** rowptr = reinterpret_cast<const uint8_t**>(sn + 32);  // [64]
+
+  const LayerArgs& L = a.L;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tq = lane & 3;
+  const int row = blockIdx.z, hg = blockIdx.y, sp = blockIdx.x;
+  const int b = row / a.Tq;
+  const int64_t t = a.q_pos[row];
+  const SlotInfo si = slot_info(a, t);
+  const int64_t T = (si.R + kTile - 1) / kTile;
+  const int64_t t0 = T * sp / a.splits, t1 = T * (sp + 1) / a.splits;
+  const float cl2 = L.scale * kLog2e;
+
+  if (tid < 32) {
+    float c, s;
+    rope_cos_sin((double)t, tid, 64, L.rope_base, &c, &s);
+    cs[tid] = c;
+    sn[tid] = s;
+  }
+  if (tid < HG) { m_run[tid] = -INFINITY; l_run[tid] = 0.f; }
+  __syncthreads();
+
+  // ---------------------------------------------------------------- q~ = RoPE_t(RMSNorm(q) * gamma_q), bf16
+  const size_t ab = L.act_fmt == CSA_FMT_F32 ? 4 : 2;
+  for (int hh = warp; hh < HG; hh += NW) {
+    const int h = hg * HG + hh;
+    const uint8_t* qrow = a.q + ((size_t)row * L.H + h) * kD * ab;
+    float v[16];
+#pragma unroll
+    for (int k = 0; k < 16; k += 4) load_act4(qrow, L.act_fmt, 16 * lane + k, v + k);
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) ss += v[k] * v[k];
+    ss = warp_sum(ss);
+    const float rs = 1.0f / sqrtf(ss / (float)kD + L.eps);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] *= rs * (a.gamma_q ? a.gamma_q[16 * lane + k] : 1.f);
+    if (lane >= 28) {
+#pragma unroll
+      for (int k = 0; k < 16; k += 2) {
+        const int u = (16 * lane + k - (kD - 64)) >> 1;
+        const float x0 = v[k], x1 = v[k + 1];
+        v[k] = x0 * cs[u] - x1 * sn[u];
+        v[k + 1] = x0 * sn[u] + x1 * cs[u];
+      }
+    }
+    uint4 p0, p1;
+    p0.x = pack_bf16x2(v[0], v[1]); p0.y = pack_bf16x2(v[2], v[3]);
+    p0.z = pack_bf16x2(v[4], v[5]); p0.w = pack_bf16x2(v[6], v[7]);
+    p1.x = pack_bf16x2(v[8], v[9]); p1.y = pack_bf16x2(v[10], v[11]);
+    p1.z = pack_bf16x2(v[12], v[13]); p1.w = pack_bf16x2(v[14], v[15]);
+    *reinterpret_cast<uint4*>(Qs + swz(hh, 2 * lane, 1024)) = p0;
+    *reinterpret_cast<uint4*>(Qs + swz(hh, 2 * lane + 1, 1024)) = p1;
+  }
+
+  float o[MT][NTW][4];
+#pragma unroll
+  for (int i = 0; i < MT; ++i)
+#pragma unroll
+    for (int j = 0; j < NTW; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o[i][j][k] = 0.f;
+  __syncthreads();
+
+  const int mt = warp >> 2, np = warp & 3;   // S-phase tile of this warp: heads mt*16.., slots np*16..
+  for (int64_t tile = t0; tile < t1; ++tile) {
+    const int64_t s0 = tile * kTile;
+    if (tid < kTile) rowptr[tid] = slot_row(a, si, row, b, s0 + tid);
+    __syncthreads();
+
+    // ------------------------------------------------------------ gather the key/value tile (bf16, swizzled)
+    if (FMT == CSA_FMT_BF16) {
+      for (int idx = tid; idx < kTile * 64; idx += NT) {
+        const int rr = idx >> 6, ch = idx & 63;
+        const uint8_t* p = rowptr[rr];
+        const uint4 v = p ? ldg_nc_v4(p + ch * 16) : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(Ks + swz(rr, ch, 1024)) = v;
+      }
+    } else {
+      for (int idx = tid; idx < kTile * 36; idx += NT) {
+        const int rr = idx / 36, ch = idx % 36;
+        const uint8_t* p = rowptr[rr];
+        if (ch < 28) {
+          uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
+          if (p) {
+            const uint4 c = ldg_nc_v4(p + ch * 16);
+            const float sig = __ldg(reinterpret_cast<const float*>(p + kD + 64));
+            const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+            uint32_t outw[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float f0 = e4m3_to_f((uint8_t)(w[q] & 0xFF)) * sig;
+              const float f1 = e4m3_to_f((uint8_t)((w[q] >> 8) & 0xFF)) * sig;
+              const float f2 = e4m3_to_f((uint8_t)((w[q] >> 16) & 0xFF)) * sig;
+              const float f3 = e4m3_to_f((uint8_t)(w[q] >> 24)) * sig;
+              outw[2 * q] = pack_bf16x2(f0, f1);
+              outw[2 * q + 1] = pack_bf16x2(f2, f3);
+            }
+            lo = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+            hi = make_uint4(outw[4], outw[5], outw[6], outw[7]);
+          }
+          *reinterpret_cast<uint4*>(Ks + swz(rr, 2 * ch, 1024)) = lo;
+          *reinterpret_cast<uint4*>(Ks + swz(rr, 2 * ch + 1, 1024)) = hi;
+        } else {
+          const int c2 = ch - 28;
+          const uint4 v = p ? ldg_nc_v4(p + (kD - 64) + c2 * 16) : make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(Ks + swz(rr, 56 + c2, 1024)) = v;
+        }
+      }
+    }
+    __syncthreads();
+
+    // ------------------------------------------------------------ S = Q K^T for (heads mt*16.., slots np*16..)
+    float sacc[2][4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) sacc[i][k] = 0.f;
+    {
+      const int mi = lane >> 3;
+      const int qrow = mt * 16 + (lane & 7) + ((mi & 1) << 3);
+      const int krow = np * 16 + (lane & 7) + ((mi >> 1) << 3);
+#pragma unroll 8
+      for (int ks = 0; ks < kD / 16; ++ks) {
+        uint32_t af[4], b0, b1, b2, b3;
+        ldsm_x4(smem_addr(Qs + swz(qrow, 2 * ks + (mi >> 1), 1024)), af[0], af[1], af[2], af[3]);
+        ldsm_x4(smem_addr(Ks + swz(krow, 2 * ks + (mi & 1), 1024)), b0, b1, b2, b3);
+        mma_bf16(sacc[0], af, b0, b1);
+        mma_bf16(sacc[1], af, b2, b3);
+      }
+    }
+    float pm0 = -INFINITY, pm1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int col = np * 16 + nt * 8 + 2 * tq + (i & 1);
+        const float v = rowptr[col] ? sacc[nt][i] * cl2 : -INFINITY;
+        sacc[nt][i] = v;
+        if (i < 2) pm0 = fmaxf(pm0, v); else pm1 = fmaxf(pm1, v);
+      }
+    pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, 1));
+    pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, 2));
+    pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, 1));
+    pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, 2));
+    if (tq == 0) {
+      pmax[np * HG + mt * 16 + g] = pm0;
+      pmax[np * HG + mt * 16 + g + 8] = pm1;
+    }
+    __syncthreads();
+    if (tid < HG) {
+      const float tm = fmaxf(fmaxf(pmax[tid], pmax[HG + tid]), fmaxf(pmax[2 * HG + tid], pmax[3 * HG + tid]));
+      const float mo = m_run[tid];
+      const float mn = fmaxf(mo, tm);
+      corr[tid] = (mn == -INFINITY) ? 1.f : exp2f(mo - mn);
+      m_run[tid] = mn;
+    }
+    __syncthreads();
+
+    // ------------------------------------------------------------ P = exp2(S - m), bf16 into shared memory
+    {
+      const float mn0 = m_run[mt * 16 + g], mn1 = m_run[mt * 16 + g + 8];
+      float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int col = np * 16 + nt * 8 + 2 * tq;
+        const float p0 = mn0 == -INFINITY ? 0.f : exp2f(sacc[nt][0] - mn0);
+        const float p1 = mn0 == -INFINITY ? 0.f : exp2f(sacc[nt][1] - mn0);
+        const float p2 = mn1 == -INFINITY ? 0.f : exp2f(sacc[nt][2] - mn1);
+        const float p3 = mn1 == -INFINITY ? 0.f : exp2f(sacc[nt][3] - mn1);
+        const uint32_t w01 = pack_bf16x2(p0, p1), w23 = pack_bf16x2(p2, p3);
+        ps0 += bf16_bits_to_f(w01 & 0xFFFFu) + bf16_bits_to_f(w01 >> 16);
+        ps1 += bf16_bits_to_f(w23 & 0xFFFFu) + bf16_bits_to_f(w23 >> 16);
+        const int h0 = mt * 16 + g, h1 = h0 + 8;
+        *reinterpret_cast<uint32_t*>(Ps + swz(h0, col >> 3, 128) + (col & 7) * 2) = w01;
+        *reinterpret_cast<uint32_t*>(Ps + swz(h1, col >> 3, 128) + (col & 7) * 2) = w23;
+      }
+      ps0 += __shfl_xor_sync(0xffffffffu, ps0, 1);
+      ps0 += __shfl_xor_sync(0xffffffffu, ps0, 2);
+      ps1 += __shfl_xor_sync(0xffffffffu, ps1, 1);
+      ps1 += __shfl_xor_sync(0xffffffffu, ps1, 2);
+      if (tq == 0) {
+        psum[np * HG + mt * 16 + g] = ps0;
+        psum[np * HG + mt * 16 + g + 8] = ps1;
+      }
+    }
+    __syncthreads();
+    if (tid < HG)
+      l_run[tid] = l_run[tid] * corr[tid] + (psum[tid] + psum[HG + tid]) + (psum[2 * HG + tid] + psum[3 * HG + tid]);
+
+    // ------------------------------------------------------------ O = O * corr + P V (warp owns dims warp*DW..)
+#pragma unroll
+    for (int m2 = 0; m2 < MT; ++m2) {
+      const float c0 = corr[m2 * 16 + g], c1 = corr[m2 * 16 + g + 8];
+#pragma unroll
+      for (int j = 0; j < NTW; ++j) {
+        o[m2][j][0] *= c0; o[m2][j][1] *= c0;
+        o[m2][j][2] *= c1; o[m2][j][3] *= c1;
+      }
+    }
+    {
+      const int mi = lane >> 3;
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk) {
+        uint32_t pa[MT][4];
+#pragma unroll
+        for (int m2 = 0; m2 < MT; ++m2) {
+          const int prow = m2 * 16 + (lane & 7) + ((mi & 1) << 3);
+          ldsm_x4(smem_addr(Ps + swz(prow, 2 * kk + (mi >> 1), 128)), pa[m2][0], pa[m2][1], pa[m2][2], pa[m2][3]);
+        }
+        const int krow = kk * 16 + (lane & 7) + ((mi & 1) << 3);
+#pragma unroll
+        for (int n2 = 0; n2 < NTW / 2; ++n2) {
+          uint32_t b0, b1, b2, b3;
+          const int ch = (warp * DW + n2 * 16) / 8 + (mi >> 1);
+          ldsm_x4_t(smem_addr(Ks + swz(krow, ch, 1024)), b0, b1, b2, b3);
+#pragma unroll
+          for (int m2 = 0; m2 < MT; ++m2) {
+            mma_bf16(o[m2][2 * n2], pa[m2], b0, b1);
+            mma_bf16(o[m2][2 * n2 + 1], pa[m2], b2, b3);
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---------------------------------------------------------------- epilogue
+  if (a.splits > 1) {
+    float* part = a.part + (((size_t)row * (L.H / HG) + hg) * a.splits + sp) * (size_t)(HG * (kD + 2));
+#pragma unroll
+    for (int m2 = 0; m2 < MT; ++m2)
+#pragma unroll
+      for (int j = 0; j < NTW; ++j) {
+        const int dim = warp * DW + j * 8 + 2 * tq;
+        const int h0 = m2 * 16 + g;
+        *reinterpret_cast<float2*>(part + (size_t)h0 * kD + dim) = make_float2(o[m2][j][0], o[m2][j][1]);
+        *reinterpret_cast<float2*>(part + (size_t)(h0 + 8) * kD + dim) = make_float2(o[m2][j][2], o[m2][j][3]);
+      }
+    if (tid < HG) {
+      part[HG * kD + tid] = m_run[tid];
+      part[HG * kD + HG + tid] = l_run[tid];
+    }
+    return;
+  }
+  // single split: merge the sink, normalise, rotate back by -t, store
+  if (tid < HG) {
+    const float sk = a.sinks[hg * HG + tid] * kLog2e;
+    const float mo = m_run[tid];
+    const float M = fmaxf(mo, sk);
+    const float den = l_run[tid] * exp2f(mo - M) + exp2f(sk - M);
+    corr[tid] = exp2f(mo - M) / den;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int m2 = 0; m2 < MT; ++m2)
+#pragma unroll
+    for (int j = 0; j < NTW; ++j) {
+      const int dim = warp * DW + j * 8 + 2 * tq;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int hl = m2 * 16 + g + half * 8;
+        float x0 = o[m2][j][2 * half] * corr[hl], x1 = o[m2][j][2 * half + 1] * corr[hl];
+        if (dim >= kD - 64) {
+          const int u = (dim - (kD - 64)) >> 1;
+          const float c = cs[u], s = sn[u];
+          const float y0 = x0 * c + x1 * s, y1 = -x0 * s + x1 * c;
+          x0 = y0; x1 = y1;
+        }
+        const size_t off = ((size_t)row * L.H + hg * HG + hl) * kD + dim;
+        if (L.act_fmt == CSA_FMT_F32) {
+          *reinterpret_cast<float2*>(a.out + off * 4) = make_float2(x0, x1);
+        } else {
+          *reinterpret_cast<uint32_t*>(a.out + off * 2) = pack_bf16x2(x0, x1);
+        }
+      }
+    }
+}
+
+// Merge the splits of one (query, head): sink, normalisation, inverse rotation.
+template <int HG>
+__global__ void attend_combine_kernel(const __grid_constant__ AttendArgs a) {
+  const LayerArgs& L = a.L;
+  const int h = blockIdx.x, row = blockIdx.y;
+  const int hg = h / HG, hl = h % HG;
+  const float* base = a.part + ((size_t)row * (L.H / HG) + hg) * a.splits * (size_t)(HG * (kD + 2));
+  const size_t pstride = (size_t)HG * (kD + 2);
+  const float sk = a.sinks[h] * kLog2e;
+  float M = sk;
+  for (int s = 0; s < a.splits; ++s) M = fmaxf(M, base[s * pstride + HG * kD + hl]);
+  float den = exp2f(sk - M);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const int d0 = threadIdx.x * 4;
+  for (int s = 0; s < a.splits; ++s) {
+    const float* p = base + s * pstride;
+    const float ms = p[HG * kD + hl];
+    const float f = exp2f(ms - M);
+    den += p[HG * kD + HG + hl] * f;
+    const float4 v = *reinterpret_cast<const float4*>(p + (size_t)hl * kD + d0);
+    acc[0] += v.x * f; acc[1] += v.y * f; acc[2] += v.z * f; acc[3] += v.w * f;
+  }
+  const float inv = 1.f / den;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] *= inv;
+  if (d0 >= kD - 64) {
+    const int64_t t = a.q_pos[row];
+#pragma unroll
+    for (int k = 0; k < 4; k += 2) {
+      float c, s;
+      rope_cos_sin(-(double)t, (d0 + k - (kD - 64)) >> 1, 64, L.rope_base, &c, &s);
+      const float x0 = acc[k], x1 = acc[k + 1];
+      acc[k] = x0 * c - x1 * s;
+      acc[k + 1] = x0 * s + x1 * c;
+    }
+  }
+  uint8_t* dst = a.out + ((size_t)row * L.H + h) * kD * (L.act_fmt == CSA_FMT_F32 ? 4 : 2);
+  store_act4(dst, L.act_fmt, d0, acc);
+}
+
+// CUDA-core attention for other shapes / float32 rows: one warp per head, one CTA per query.
+__global__ void attend_generic_kernel(const __grid_constant__ AttendArgs a) {
+  const LayerArgs& L = a.L;
+  const int lane = threadIdx.x & 31, h = threadIdx.x >> 5;
+  const int row = blockIdx.x, b = row / a.Tq;
+  const int D = L.D, dpl = D / 32, dn = D - L.d_rope;
+  const int64_t t = a.q_pos[row];
+  const SlotInfo si = slot_info(a, t);
+  float q[32], o[32];
+  const size_t ab = L.act_fmt == CSA_FMT_F32 ? 4 : 2;
+  const uint8_t* qrow = a.q + ((size_t)row * L.H + h) * D * ab;
+  float ss = 0.f;
+  for (int k = 0; k < dpl; ++k) {
+    const int d = lane * dpl + k;
+    q[k] = L.act_fmt == CSA_FMT_F32 ? reinterpret_cast<const float*>(qrow)[d]
+                                    : bf16_bits_to_f(reinterpret_cast<const uint16_t*>(qrow)[d]);
+    ss += q[k] * q[k];
+    o[k] = 0.f;
+  }
+  ss = warp_sum(ss);
+  const float rs = 1.0f / sqrtf(ss / (float)D + L.eps);
+  for (int k = 0; k < dpl; ++k) q[k] *= rs * (a.gamma_q ? a.gamma_q[lane * dpl + k] : 1.f);
+  for (int k = 0; k + 1 < dpl; k += 2) {
+    const int d = lane * dpl + k;
+    if (d >= dn) {
+      float c, s;
+      rope_cos_sin((double)t, (d - dn) >> 1, L.d_rope, L.rope_base, &c, &s);
+      const float x0 = q[k], x1 = q[k + 1];
+      q[k] = x0 * c - x1 * s;
+      q[k + 1] = x0 * s + x1 * c;
+    }
+  }
+  float m = -INFINITY, l = 0.f;
+  for (int64_t s = 0; s < si.R; ++s) {
+    const uint8_t* p = slot_row(a, si, row, b, s);
+    if (!p) continue;
+    float kv[32];
+    float sig = 1.f;
+    if (L.kv_fmt == CSA_FMT_MIXED) sig = *reinterpret_cast<const float*>(p + D + 64);
+    float dot = 0.f;
+    for (int k = 0; k < dpl; ++k) {
+      const int d = lane * dpl + k;
+      float v;
+      if (L.kv_fmt == CSA_FMT_F32) v = reinterpret_cast<const float*>(p)[d];
+      else if (L.kv_fmt == CSA_FMT_BF16) v = bf16_bits_to_f(reinterpret_cast<const uint16_t*>(p)[d]);
+      else v = d < dn ? e4m3_to_f(p[d]) * sig : bf16_bits_to_f(reinterpret_cast<const uint16_t*>(p + dn)[d - dn]);
+      kv[k] = v;
+      dot += q[k] * v;
+    }
+    dot = warp_sum(dot) * L.scale;
+    if (dot > m) {
+      const float c = expf(m - dot);
+      l = l * c + 1.f;
+      for (int k = 0; k < dpl; ++k) o[k] = o[k] * c + kv[k];
+      m = dot;
+    } else {
+      const float pe = expf(dot - m);
+      l += pe;
+      for (int k = 0; k < dpl; ++k) o[k] += pe * kv[k];
+    }
+  }
+  const float sk = a.sinks[h];
+  const float M = fmaxf(m, sk);
+  const float f = expf(m - M) / (l * expf(m - M) + expf(sk - M));
+  for (int k = 0; k < dpl; ++k) o[k] *= f;
+  for (int k = 0; k + 1 < dpl; k += 2) {
+    const int d = lane * dpl + k;
+    if (d >= dn) {
+      float c, s;
+      rope_cos_sin(-(double)t, (d - dn) >> 1, L.d_rope, L.rope_base, &c, &s);
+      const float x0 = o[k], x1 = o[k + 1];
+      o[k] = x0 * c - x1 * s;
+      o[k + 1] = x0 * s + x1 * c;
+    }
+  }
+  uint8_t* dst = a.out + ((size_t)row * L.H + h) * D * ab;
+  for (int k = 0; k < dpl; ++k) {
+    const int d = lane * dpl + k;
+    if (L.act_fmt == CSA_FMT_F32) reinterpret_cast<float*>(dst)[d] = o[k];
+    else reinterpret_cast<uint16_t*>(dst)[d] = f_to_bf16_bits(o[k]);
+  }
+}
+
+template <int HG>
+size_t mma_smem_bytes() {
+  return (size_t)HG * 1024 + (size_t)kTile * 1024 + (size_t)HG * 128 + (11 * HG + 64) * sizeof(float) +
+         kTile * sizeof(void*);
+}
+
+template <int HG, int FMT>
+cudaError_t launch_mma(const AttendArgs& a, cudaStream_t s) {
+  const size_t smem = mma_smem_bytes<HG>();
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(attend_mma_kernel<HG, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  dim3 grid(a.splits, a.L.H / HG, a.rows);
+  attend_mma_kernel<HG, FMT><<<grid, HG * 8, smem, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || a.splits == 1) return e;
+  attend_combine_kernel<HG><<<dim3(a.L.H, a.rows), kD / 4, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int attend_head_group(const LayerArgs& L) {
+  if (L.D != kD || L.d_rope != 64) return 0;
+  if (L.kv_fmt != CSA_FMT_BF16 && L.kv_fmt != CSA_FMT_MIXED) return 0;
+  if (L.H % 64 == 0 && L.H <= 64) return 64;
+  if (L.H % 32 == 0) return 32;
+  return 0;
+}
+
+int attend_num_splits(const LayerArgs& L, int rows, int64_t slots, int num_sms) {
+  const int HG = attend_head_group(L);
+  if (HG == 0) return 1;
+  const int64_t pairs = (int64_t)rows * (L.H / HG);
+  const int64_t tiles = (slots + kTile - 1) / kTile;
+  int64_t want = (2 * (int64_t)num_sms + pairs - 1) / pairs;
+  if (want > tiles) want = tiles;
+  if (want < 1) want = 1;
+  return (int)want;
+}
+
+size_t attend_partial_bytes(const LayerArgs& L, int rows, int splits) {
+  const int HG = attend_head_group(L);
+  if (HG == 0 || splits <= 1) return 0;
+  return (size_t)rows * (L.H / HG) * splits * HG * (kD + 2) * sizeof(float);
+}
+
+cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
+  if (a.rows <= 0) return cudaSuccess;
+  const int HG = attend_head_group(a.L);
+  if (HG == 0) {
+    attend_generic_kernel<<<a.rows, a.L.H * 32, 0, s>>>(a);
+    return cudaGetLastError();
+  }
+  const bool mixed = a.L.kv_fmt == CSA_FMT_MIXED;
+  if (HG == 64) return mixed ? launch_mma<64, CSA_FMT_MIXED>(a, s) : launch_mma<64, CSA_FMT_BF16>(a, s);
+  return mixed ? launch_mma<32, CSA_FMT_MIXED>(a, s) : launch_mma<32, CSA_FMT_BF16>(a, s);
+}
+
+}  // namespace csa

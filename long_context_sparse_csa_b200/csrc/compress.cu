@@ -1,0 +1,154 @@
+// Append new tokens to the caches and compress completed groups into entries.
+//
+// Compression follows "DeepSeek-V4: Making a Million Tokens Affordable",
+// section "Two ways to shrink attention, interleaved" (each entry pools m
+// tokens, drawing from 2m source rows with overlap) and "DeepSeek-V4
+// Explained: ...", section "The attention stack, and why it is two
+// mechanisms" (learned compression weights and positional biases): per
+// channel, a softmax over the window's rows of gate logit + slot bias weights
+// the raw rows; the pooled vector gets an RMSNorm and rotary embedding on its
+// last 64 dims at position pos0 + i*m, and is stored in the cache format.
+//
+// One CTA per (token, sequence), D/4 threads, 4 consecutive channels per
+// thread; raw rows are read once with 8/16-byte vector loads and the
+// per-channel softmax runs online in registers.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace csa {
+
+namespace {
+
+__device__ __forceinline__ void rope4(float v[4], int c0, const LayerArgs& L, double pos) {
+  const int dn = L.D - L.d_rope;
+  if (c0 < dn) return;
+  const int u = (c0 - dn) >> 1;
+  float c, s, a, b;
+  rope_cos_sin(pos, u, L.d_rope, L.rope_base, &c, &s);
+  a = v[0]; b = v[1];
+  v[0] = a * c - b * s; v[1] = a * s + b * c;
+  rope_cos_sin(pos, u + 1, L.d_rope, L.rope_base, &c, &s);
+  a = v[2]; b = v[3];
+  v[2] = a * c - b * s; v[3] = a * s + b * c;
+}
+
+// Block-cooperative store of one row in the cache format (all threads call).
+__device__ __forceinline__ void pack_row(uint8_t* dst, const LayerArgs& L, int c0, const float v[4],
+                                         float* scratch) {
+  if (L.kv_fmt == CSA_FMT_F32) {
+    *reinterpret_cast<float4*>(dst + 4 * (size_t)c0) = make_float4(v[0], v[1], v[2], v[3]);
+    return;
+  }
+  if (L.kv_fmt == CSA_FMT_BF16) {
+    store_act4(dst, CSA_FMT_BF16, c0, v);
+    return;
+  }
+  const int dn = L.D - L.d_rope;
+  float am = 0.f;
+  if (c0 < dn) am = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+  am = block_max(am, scratch);
+  float inv;
+  const float sig = pow2_scale(am, &inv);
+  if (c0 < dn) {
+    uint32_t w = (uint32_t)f_to_e4m3_sat(v[0] * inv) | ((uint32_t)f_to_e4m3_sat(v[1] * inv) << 8) |
+                 ((uint32_t)f_to_e4m3_sat(v[2] * inv) << 16) | ((uint32_t)f_to_e4m3_sat(v[3] * inv) << 24);
+    *reinterpret_cast<uint32_t*>(dst + c0) = w;
+  } else {
+    store_act4(dst + dn, CSA_FMT_BF16, c0 - dn, v);
+  }
+  if (threadIdx.x == 0) {
+    *reinterpret_cast<float*>(dst + L.D + 64) = sig;
+    *reinterpret_cast<uint32_t*>(dst + L.D + 68) = 0u;
+    *reinterpret_cast<uint2*>(dst + L.D + 72) = make_uint2(0u, 0u);
+  }
+}
+
+__global__ void append_compress_kernel(const __grid_constant__ AppendCompressArgs a) {
+  __shared__ float scratch[32];
+  const LayerArgs& L = a.L;
+  const CacheArgs& C = a.C;
+  const int j = blockIdx.x, b = blockIdx.y;
+  const int c0 = threadIdx.x * 4;
+  const int64_t t = a.q_pos[(int64_t)b * a.Tq + j];
+  const int64_t r = t - L.pos0;
+  if (r < 0) return;  // uniform over the block
+  const size_t arow = (size_t)L.D * act_bytes(L.act_fmt);
+  const bool have_new = a.x_new != nullptr;
+  float x[4], g[4] = {0.f, 0.f, 0.f, 0.f};
+  if (have_new) {
+    load_act4(a.x_new + ((size_t)b * a.Tq + j) * arow, L.act_fmt, c0, x);
+    load_act4(a.g_new + ((size_t)b * a.Tq + j) * arow, L.act_fmt, c0, g);
+  } else {
+    const int64_t s = ring_slot(r, C.raw_base, C.raw_cap);
+    load_act4(C.raw + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, x);
+  }
+
+  if (a.do_append) {
+    if (have_new) {
+      const int64_t s = ring_slot(r, C.raw_base, C.raw_cap);
+      store_act4(C.raw + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, x);
+      store_act4(C.gate + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, g);
+    }
+    float w[4] = {x[0], x[1], x[2], x[3]};
+    rope4(w, c0, L, (double)t);
+    uint8_t* dst = C.window + ((size_t)b * C.window_cap + (size_t)(r % C.window_cap)) * L.row_bytes;
+    pack_row(dst, L, c0, w, scratch);
+  }
+
+  if (a.do_compress && ((r + 1) % L.m) == 0) {
+    const int64_t i = (r + 1) / L.m - 1;
+    const int64_t lo = (i - L.ov) * (int64_t)L.m;
+    const int64_t r_begin = lo < 0 ? 0 : lo;
+    float mx[4], sum[4], acc[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) { mx[k] = -INFINITY; sum[k] = 0.f; acc[k] = 0.f; }
+    for (int64_t rr = r_begin; rr <= r; ++rr) {
+      float xv[4], gv[4];
+      if (rr == r && have_new) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) { xv[k] = x[k]; gv[k] = g[k]; }
+      } else {
+        const int64_t s = ring_slot(rr, C.raw_base, C.raw_cap);
+        load_act4(C.raw + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, xv);
+        load_act4(C.gate + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, gv);
+      }
+      const float4 bias = *reinterpret_cast<const float4*>(a.pos_bias + (size_t)(rr - lo) * L.D + c0);
+      const float bz[4] = {bias.x, bias.y, bias.z, bias.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float z = gv[k] + bz[k];
+        if (z > mx[k]) {
+          const float sc = expf(mx[k] - z);
+          sum[k] = sum[k] * sc + 1.f;
+          acc[k] = acc[k] * sc + xv[k];
+          mx[k] = z;
+        } else {
+          const float e = expf(z - mx[k]);
+          sum[k] += e;
+          acc[k] += e * xv[k];
+        }
+      }
+    }
+    float e[4];
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) { e[k] = acc[k] / sum[k]; ss += e[k] * e[k]; }
+    ss = block_sum(ss, scratch);
+    const float rs = 1.0f / sqrtf(ss / (float)L.D + L.eps);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) e[k] *= rs * (a.gamma_kv ? a.gamma_kv[c0 + k] : 1.f);
+    rope4(e, c0, L, (double)(L.pos0 + i * (int64_t)L.m));
+    uint8_t* dst = C.entries + ((size_t)b * C.entry_cap + (size_t)i) * L.row_bytes;
+    pack_row(dst, L, c0, e, scratch);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_append_compress(const AppendCompressArgs& a, int B, int Tq, cudaStream_t s) {
+  dim3 grid(Tq, B);
+  append_compress_kernel<<<grid, a.L.D / 4, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

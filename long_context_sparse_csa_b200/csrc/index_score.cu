@@ -1,0 +1,334 @@
+// Lightning-indexer scores:  s_i = sum_h w_h * ReLU(sigma_q,h * sigma_k,i * <q_h, k_i>).
+//
+// The pages give the indexer only in words: "a Lightning Indexer scores them
+// in a low-rank way" ("DeepSeek-V4 Explained: ...", section "The attention
+// stack, and why it is two mechanisms") and "a separate lightning indexer, a
+// few small heads run in FP8, scores individual past tokens" ("DeepSeek-V4,
+// explained.", step 3 of "For one query ... works like this").  This file
+// holds the multi-head ReLU-weighted dot product the operator defines.
+//
+// Tensor-core path (FP8 e4m3 keys, d_I = 128): the score tile of 128 entries
+// x (QN queries * H_I heads) is one tcgen05 kind::f8f6f4 MMA chain (M = 128
+// entries, N = QN*H_I, K = 128 in four K=32 steps) with A = index keys staged
+// by TMA in the 128-byte swizzle layout and B = index queries, accumulating
+// in TMEM.  A persistent CTA per SM runs a 3-role pipeline: warp 0 issues TMA
+// loads into a 6-stage ring, warp 1 issues the MMAs into two TMEM
+// accumulators, warps 2-5 read the accumulator back with tcgen05.ld, apply
+// the ReLU / head-weight epilogue and store the fp32 scores (coalesced).
+// Decode streams the keys once from HBM; it is a bandwidth-bound kernel whose
+// MMA keeps the 64 FLOP/byte of 32 heads off the CUDA cores.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace csa {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kStages = 6;
+constexpr int kTileE = 128;                 // entries per tile (MMA M)
+constexpr int kDI = 128;                    // index-key bytes per entry
+constexpr int kTileBytes = kTileE * kDI;    // 16 KB
+constexpr int kThreads = 192;               // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+
+struct Item {
+  int b, j0, et;
+  int64_t g;
+  bool valid;
+};
+
+__device__ __forceinline__ int64_t n_visible(const IndexArgs& a, int b, int j) {
+  const int64_t t = a.q_pos[(int64_t)b * a.Tq + j];
+  const int64_t r1 = t - a.pos0 + 1;
+  const int64_t nv = r1 > 0 ? r1 / a.m : 0;
+  return nv < a.n_max ? nv : a.n_max;
+}
+
+__device__ __forceinline__ Item item_at(const IndexArgs& a, int64_t w) {
+  Item it;
+  it.g = w / a.tiles_per_group;
+  it.et = (int)(w % a.tiles_per_group);
+  it.b = (int)(it.g / a.groups_per_seq);
+  it.j0 = (int)(it.g % a.groups_per_seq) * a.QN;
+  const int j1 = min(it.j0 + a.QN, a.Tq);
+  int64_t nv = 0;
+  for (int j = it.j0; j < j1; ++j) nv = max(nv, n_visible(a, it.b, j));
+  it.valid = (int64_t)it.et * kTileE < nv;
+  return it;
+}
+
+struct __align__(8) Barriers {
+  uint64_t full[kStages], empty[kStages];
+  uint64_t bfull[2], bempty[2];
+  uint64_t tfull[2], tempty[2];
+  uint32_t tmem_base;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                      const __grid_constant__ IndexArgs a, int N, uint32_t tmem_cols) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* A = smem;                                  // [kStages][kTileBytes]
+  uint8_t* Bq = A + kStages * kTileBytes;             // [2][N * 128]
+  Barriers* bars = reinterpret_cast<Barriers*>(Bq + 2 * N * kDI);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t w0 = a.total_items * blockIdx.x / gridDim.x;
+  const int64_t w1 = a.total_items * (blockIdx.x + 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&bars->full[s], 1); mbar_init(&bars->empty[s], 1); }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->bfull[s], 1); mbar_init(&bars->bempty[s], 1);
+      mbar_init(&bars->tfull[s], 1); mbar_init(&bars->tempty[s], 128);
+    }
+    fence_barrier_init();
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&qmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t prev_g = -1;
+      int gi = -1;
+      int issued_par[kStages];
+      for (int s = 0; s < kStages; ++s) issued_par[s] = -1;
+      int b_issued_par[2] = {-1, -1};
+      bool ok = true;
+      for (int64_t w = w0; w < w1 && ok; ++w) {
+        const Item it = item_at(a, w);
+        if (!it.valid) continue;
+        if (it.g != prev_g) {
+          prev_g = it.g;
+          ++gi;
+          const int slot = gi & 1;
+          const uint32_t use = (uint32_t)(gi >> 1);
+          if (!mbar_wait(&bars->bempty[slot], (use & 1u) ^ 1u)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars->bfull[slot], (uint32_t)(N * kDI));
+          tma_load_2d(Bq + slot * N * kDI, &qmap, &bars->bfull[slot], 0,
+                      (int)(((int64_t)it.b * a.Tq + it.j0) * a.H_I));
+          b_issued_par[slot] = (int)(use & 1u);
+        }
+        if (!mbar_wait(&bars->empty[stage], phase ^ 1u)) { ok = false; break; }
+        mbar_arrive_expect_tx(&bars->full[stage], (uint32_t)kTileBytes);
+        tma_load_2d(A + stage * kTileBytes, &kmap, &bars->full[stage], 0,
+                    (int)((int64_t)it.b * a.entry_cap + (int64_t)it.et * kTileE));
+        issued_par[stage] = (int)phase;
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) set_device_error(a.err, kErrWaitTimeout);
+      // never leave a bulk copy in flight when the CTA exits
+      for (int s = 0; s < kStages; ++s)
+        if (issued_par[s] >= 0) mbar_wait(&bars->full[s], (uint32_t)issued_par[s]);
+      for (int s = 0; s < 2; ++s)
+        if (b_issued_par[s] >= 0) mbar_wait(&bars->bfull[s], (uint32_t)b_issued_par[s]);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      const uint32_t idesc = instr_desc(128, N, 0u);
+      int stage = 0, acc = 0, gi = -1;
+      uint32_t phase = 0, acc_phase = 0;
+      int64_t prev_g = -1;
+      int last_acc = -1;
+      uint32_t last_acc_par = 0;
+      bool ok = true;
+      for (int64_t w = w0; w < w1; ++w) {
+        const Item it = item_at(a, w);
+        if (!it.valid) continue;
+        if (it.g != prev_g) {
+          prev_g = it.g;
+          ++gi;
+          if (!mbar_wait(&bars->bfull[gi & 1], (uint32_t)((gi >> 1) & 1))) { ok = false; break; }
+        }
+        const int slot = gi & 1;
+        if (!mbar_wait(&bars->full[stage], phase)) { ok = false; break; }
+        if (!mbar_wait(&bars->tempty[acc], acc_phase ^ 1u)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t ad = desc_kmajor_sw128(smem_u32(A + stage * kTileBytes));
+        const uint64_t bd = desc_kmajor_sw128(smem_u32(Bq + slot * N * kDI));
+#pragma unroll
+        for (int kk = 0; kk < kDI / 32; ++kk)
+          umma_f8f6f4(tmem + (uint32_t)(acc * N), ad + 2u * kk, bd + 2u * kk, idesc, kk > 0 ? 1u : 0u);
+        umma_commit(&bars->empty[stage]);
+        umma_commit(&bars->tfull[acc]);
+        last_acc = acc;
+        last_acc_par = acc_phase;
+        // release the query tile after the group's last valid item in this CTA
+        bool last_of_group = (w + 1 >= w1);
+        if (!last_of_group) {
+          const Item nx = item_at(a, w + 1);
+          last_of_group = (nx.g != it.g) || !nx.valid;
+        }
+        if (last_of_group) umma_commit(&bars->bempty[slot]);
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) set_device_error(a.err, kErrWaitTimeout);
+      // the accumulator must be idle before TMEM is released
+      if (last_acc >= 0) mbar_wait(&bars->tfull[last_acc], last_acc_par);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 2..5)
+    const int quarter = warp & 3;              // TMEM lanes [32*quarter, 32*quarter + 32)
+    const int e_loc = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int64_t w = w0; w < w1; ++w) {
+      const Item it = item_at(a, w);
+      if (!it.valid) continue;
+      if (!mbar_wait(&bars->tfull[acc], acc_phase)) { ok = false; break; }
+      tc_fence_after();
+      const int64_t e = (int64_t)it.et * kTileE + e_loc;
+      const bool in_range = e < a.n_max;
+      const float ks = in_range ? __ldg(a.k_scale + (int64_t)it.b * a.entry_cap + e) : 0.f;
+      const int j1 = min(it.j0 + a.QN, a.Tq);
+      for (int j = it.j0; j < j1; ++j) {
+        const int64_t row = (int64_t)it.b * a.Tq + j;
+        const float* qs = a.q_scale + row * a.H_I;
+        const float* hw = a.head_w + row * a.H_I;
+        float s = 0.f;
+        for (int hc = 0; hc < a.H_I; hc += 16) {
+          float v[16];
+          tmem_ld_32x32b_x16(lane_addr + (uint32_t)(acc * N + (j - it.j0) * a.H_I + hc), v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < 16; ++h) s += __ldg(hw + hc + h) * fmaxf(v[h] * (__ldg(qs + hc + h) * ks), 0.f);
+        }
+        if (in_range) a.scores[row * a.n_max + e] = (e < n_visible(a, it.b, j)) ? s : -INFINITY;
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (!ok) set_device_error(a.err, kErrWaitTimeout);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols);
+  }
+}
+
+// CUDA-core path for float32 index tensors or shapes the tensor-core kernel does not take.
+__global__ void index_score_generic_kernel(const __grid_constant__ IndexArgs a) {
+  extern __shared__ float qv[];                      // [H_I][d_I]
+  const int64_t row = blockIdx.y;
+  const int b = (int)(row / a.Tq), j = (int)(row % a.Tq);
+  const int nq = a.H_I * a.d_I;
+  for (int i = threadIdx.x; i < nq; i += blockDim.x) {
+    qv[i] = a.idx_fmt == CSA_FMT_F32 ? reinterpret_cast<const float*>(a.idx_q)[row * nq + i]
+                                     : e4m3_to_f(a.idx_q[row * nq + i]);
+  }
+  __syncthreads();
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= a.n_max) return;
+  if (e >= n_visible(a, b, j)) { a.scores[row * a.n_max + e] = -INFINITY; return; }
+  const int64_t krow = (int64_t)b * a.entry_cap + e;
+  const float ks = a.k_scale[krow];
+  float s = 0.f;
+  for (int h = 0; h < a.H_I; ++h) {
+    float dot = 0.f;
+    if (a.idx_fmt == CSA_FMT_F32) {
+      const float* k = reinterpret_cast<const float*>(a.idx_k) + krow * a.d_I;
+      for (int d = 0; d < a.d_I; ++d) dot += qv[h * a.d_I + d] * k[d];
+    } else {
+      const uint8_t* k = a.idx_k + krow * a.d_I;
+      for (int d = 0; d < a.d_I; ++d) dot += qv[h * a.d_I + d] * e4m3_to_f(k[d]);
+    }
+    s += a.head_w[row * a.H_I + h] * fmaxf(dot * (a.q_scale[row * a.H_I + h] * ks), 0.f);
+  }
+  a.scores[row * a.n_max + e] = s;
+}
+
+// ----------------------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2D byte tensor [rows][128] with a 128-byte-swizzled box of box_rows x 128.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kDI, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kDI};
+  cuuint32_t box[2] = {(cuuint32_t)kDI, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool index_tc_supported(int idx_fmt, int H_I, int d_I) {
+  return idx_fmt == CSA_FMT_E4M3 && d_I == kDI && (H_I == 16 || H_I == 32 || H_I == 64);
+}
+
+cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
+  if (a.n_max <= 0 || a.Tq <= 0 || a.B <= 0) return cudaSuccess;
+  if (!index_tc_supported(a.idx_fmt, a.H_I, a.d_I)) {
+    dim3 grid((unsigned)((a.n_max + 127) / 128), (unsigned)(a.B * a.Tq));
+    const size_t sm = (size_t)a.H_I * a.d_I * sizeof(float);
+    if (sm > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(index_score_generic_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)sm);
+      if (e != cudaSuccess) return e;
+    }
+    index_score_generic_kernel<<<grid, 128, sm, s>>>(a);
+    return cudaGetLastError();
+  }
+  a.QN = a.Tq == 1 ? 1 : min(256 / a.H_I, a.Tq);
+  const int N = a.QN * a.H_I;
+  a.tiles_per_group = (int)((a.n_max + kTileE - 1) / kTileE);
+  a.groups_per_seq = (a.Tq + a.QN - 1) / a.QN;
+  a.total_items = (int64_t)a.B * a.groups_per_seq * a.tiles_per_group;
+  CUtensorMap kmap, qmap;
+  if (!make_map(&kmap, a.idx_k, (uint64_t)a.B * a.entry_cap, kTileE)) return cudaErrorInvalidValue;
+  if (!make_map(&qmap, a.idx_q, (uint64_t)a.B * a.Tq * a.H_I, (uint32_t)N)) return cudaErrorInvalidValue;
+  uint32_t cols = 32;
+  while (cols < (uint32_t)(2 * N)) cols <<= 1;
+  const size_t smem = 1024 + (size_t)kStages * kTileBytes + 2 * (size_t)N * kDI + sizeof(Barriers) + 64;
+  static size_t configured = 0;
+  if (smem > configured) {
+    cudaError_t e = cudaFuncSetAttribute(index_score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  const int64_t grid = a.total_items < num_sms ? a.total_items : num_sms;
+  index_score_tc_kernel<<<(unsigned)grid, kThreads, smem, s>>>(kmap, qmap, a, N, cols);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

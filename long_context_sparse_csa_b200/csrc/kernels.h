@@ -1,0 +1,82 @@
+// Launch-argument structs and launchers of the CSA/HCA kernels (internal).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace csa {
+
+// ----------------------------------------------------------------------------- append + compress
+struct AppendCompressArgs {
+  LayerArgs L;
+  CacheArgs C;
+  const int64_t* q_pos;
+  int Tq;
+  const uint8_t* x_new;   // [B][Tq][D] act, or null (rows already in C.raw)
+  const uint8_t* g_new;
+  const float* pos_bias;  // [(1+ov)m][D]
+  const float* gamma_kv;  // [D] or null
+  int do_append;
+  int do_compress;
+};
+cudaError_t launch_append_compress(const AppendCompressArgs& a, int B, int Tq, cudaStream_t s);
+
+// ----------------------------------------------------------------------------- indexer
+struct IndexArgs {
+  int B, Tq, H_I, d_I, m;
+  int idx_fmt;
+  int64_t n_max, entry_cap, pos0;
+  const int64_t* q_pos;
+  const uint8_t* idx_q;     // [B][Tq][H_I][d_I]
+  const uint8_t* idx_k;     // [B][entry_cap][d_I]
+  const float* k_scale;     // [B][entry_cap]
+  const float* q_scale;     // [B][Tq][H_I]
+  const float* head_w;      // [B][Tq][H_I]
+  float* scores;            // [B][Tq][n_max]
+  int* err;
+  // tensor-core path tiling
+  int QN;                   // queries per MMA N-tile (N = QN * H_I)
+  int tiles_per_group;      // ceil(n_max / 128)
+  int groups_per_seq;       // ceil(Tq / QN)
+  int64_t total_items;      // B * groups_per_seq * tiles_per_group
+};
+// True when the tcgen05 FP8 kernel handles this shape.
+bool index_tc_supported(int idx_fmt, int H_I, int d_I);
+cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s);
+
+// ----------------------------------------------------------------------------- top-k
+struct TopkArgs {
+  const float* scores;      // [rows][n_max]
+  int64_t n_max;
+  int rows, Tq, m, k;
+  int64_t pos0;
+  const int64_t* q_pos;     // [rows]
+  int32_t* out;             // [rows][k]
+};
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
+
+// ----------------------------------------------------------------------------- attention
+struct AttendArgs {
+  LayerArgs L;
+  CacheArgs C;
+  const uint8_t* q;         // [rows][H][D] act
+  const int64_t* q_pos;     // [rows]
+  int Tq, rows;
+  const int32_t* topk;      // CSA: [rows][k]; null for dense (HCA)
+  int64_t n_max;            // dense: entries bound
+  const float* gamma_q;     // [D] or null
+  const float* sinks;       // [H]
+  int splits;               // CTAs per (row, head group) along the key slots
+  float* part;              // [rows][H/HG][splits][HG*(D+2)] partial (O, m, l)
+  uint8_t* out;             // [rows][H][D] act
+};
+// Head-group size of the tensor-core attention kernel for this layer (0: generic kernel).
+int attend_head_group(const LayerArgs& L);
+int attend_num_splits(const LayerArgs& L, int rows, int64_t slots, int num_sms);
+size_t attend_partial_bytes(const LayerArgs& L, int rows, int splits);
+cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s);
+
+}  // namespace csa
