@@ -131,7 +131,7 @@ def encode_rows(x: np.ndarray, fmt: str, d_rope: int = 64) -> np.ndarray:
         sigma = pow2_scale(np.max(np.abs(nope), axis=-1))
         out[..., :dn] = e4m3_encode(nope / sigma[..., None])
         out[..., dn:dn + 2 * d_rope] = bf16_encode(x[..., dn:]).view(np.uint8).reshape(lead + (2 * d_rope,))
-        out[..., D + 64:D + 68] = sigma.astype(np.float32).view(np.uint8).reshape(lead + (4,))
+        out[..., D + 64:D + 68] = sigma.astype(np.float32).reshape(lead + (1,)).view(np.uint8)
         return out
     raise ValueError(fmt)
 
