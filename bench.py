@@ -1,0 +1,499 @@
+#!/usr/bin/env python
+"""Decode benchmark of the CSA/HCA attention operator on B200.
+
+A step is one decode token through one CSA layer (m=4, top-k 1024) and one HCA
+layer (m'=128) at 1,048,576 tokens of context, batch 1, 128 query heads, KV
+dim 512 stored as BF16 rotary dims + FP8 remainder, indexer 32 x 128 FP8: the
+whole hot path (append + compress, indexer scores, top-k, sparse attention;
+append + compress, dense attention) through the C ABI's fused decode calls.
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
+and a device synchronisation, timed with CUDA events on the launching stream,
+max over ranks.  Each step runs on the next of R independent layer instances
+(caches at distinct addresses), so a step never finds its keys in L2 (R=8:
+>= 280 MB streamed between two uses of one instance vs 126 MB of L2).
+Steps are CUDA-graph replays of the public API calls.
+
+`value` = tokens x attention layers processed by all ranks / time (tok/s per
+attention layer).  `e2e` repeats the measurement with each step's inputs
+copied host->device from pinned memory and its outputs copied back.
+`--impl reference` times the CPU oracle on the same workload instead.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode tok/s per attention layer at 1M ctx (CSA top-k 1024 + HCA m'=128, interleaved)"
+UNIT = "tok/s"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="csa_hca_decode_1m",
+                   choices=["csa_hca_decode_1m", "csa_decode_128k", "hca_decode_128k"])
+    p.add_argument("--replicas", type=int, default=8)
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def workload_config(wl, replicas):
+    layers = []
+    for L in wl.layers:
+        if L.kind == "csa":
+            layers.append(f"csa m={L.m} overlap={L.ov} top-k={L.top_k} indexer {L.H_I}x{L.d_I} {L.idx_format}")
+        else:
+            layers.append(f"hca m'={L.m}")
+    return {"workload": wl.name, "batch": wl.B, "context": wl.n, "layers": layers, "heads": wl.layers[0].H,
+            "kv_dim": wl.layers[0].D, "kv_format": wl.layers[0].kv_format, "window": wl.layers[0].window,
+            "l2": f"rotating {replicas} layer instances (inputs larger than L2)"}
+
+
+# ----------------------------------------------------------------------------- algorithmic bytes
+
+def index_kernel_bytes(layer, n_vis, B):
+    """Algorithmic bytes of one indexer-score launch: keys + key scales read, scores written, queries."""
+    per_entry = layer.d_I + 4 + 4
+    per_query = layer.H_I * layer.d_I + 2 * 4 * layer.H_I
+    return B * (n_vis * per_entry + per_query)
+
+
+def step_bytes(layer, n, B):
+    """Algorithmic HBM bytes of one decode step of a layer (per sequence x B)."""
+    rb = {"f32": 4 * layer.D, "bf16": 2 * layer.D, "mixed": layer.D + 68}[layer.kv_format]
+    ab = 4 if layer.act_format == "f32" else 2
+    nv = n // layer.m
+    w = min(layer.window, n)
+    qo = 2 * layer.H * layer.D * ab
+    if layer.kind == "csa":
+        idx = nv * (layer.d_I + 4 + 4) + layer.H_I * layer.d_I
+        att = (min(layer.top_k, nv) + w) * rb
+        return B * (idx + att + qo)
+    return B * ((nv + w) * rb + qo)
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Polls NVML SM clock and clock-event reasons on a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def sample(self):
+        if not self.ok:
+            return
+        nv = self.nv
+        try:
+            mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+            try:
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:  # noqa: BLE001
+                r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+            self.samples.append((time.perf_counter(), mhz, r))
+        except Exception:  # noqa: BLE001
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self.sample()
+            time.sleep(0.005)
+
+    def start(self):
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+
+    def stop(self):
+        self._stop.set()
+        if hasattr(self, "t"):
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": getattr(self, "err", "no samples")}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:   # timed region shorter than one poll: nearest samples around it
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:4]
+        mhz = [s[1] for s in inside]
+        bits = 0
+        for s in inside:
+            bits |= s[2]
+        reasons = [name for b, name in self.REASONS.items() if bits & b and name != "gpu_idle"]
+        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": float(self.max_mhz), "reasons": reasons,
+                "samples": len(inside)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_step(oracle_layers, datas):
+    from oracle import csa as O
+    outs = []
+    for L, d in zip(oracle_layers, datas):
+        for b in range(len(d["t"])):
+            outs.append(O.decode_step(L, d, b)["o"])
+    return outs
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return int(max(n)) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def run_cpu_oracle(wl, datas, budget_s, min_steps=1, max_steps=None):
+    from oracle import csa as O
+    Ls = [O.LayerSpec.of(L) for L in wl.layers]
+    times = []
+    t_all = time.perf_counter()
+    while True:
+        t0 = time.perf_counter()
+        oracle_step(Ls, datas)
+        times.append(time.perf_counter() - t0)
+        if max_steps is not None and len(times) >= max_steps:
+            break
+        if len(times) >= min_steps and time.perf_counter() - t_all >= budget_s:
+            break
+    return times
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from csa_synth import decode_inputs, get_workload
+    wl = get_workload(args.workload)
+    datas = [decode_inputs(wl, li) for li in range(len(wl.layers))]
+    from oracle import csa as O
+    Ls = [O.LayerSpec.of(L) for L in wl.layers]
+    for _ in range(args.warmup):
+        oracle_step(Ls, datas)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(Ls, datas)
+    T = time.perf_counter() - t0
+    units = wl.B * len(wl.layers) * args.steps
+    value = units / T
+    cores = cpu_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * T / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} full decode steps (every layer, every sequence) of the workload"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def sha_of(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+INDEX_KERNEL_SOURCES = ["long_context_sparse_csa_b200/csrc/index_score.cu", "long_context_sparse_csa_b200/csrc/sm100.cuh",
+                        "long_context_sparse_csa_b200/csrc/common.cuh"]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch of the indexer kernel from the committed ncu summary, if it is current."""
+    p = os.path.join(ROOT, "profiles", "index_score_tc_traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)
+    except OSError:
+        return None
+    if rec.get("kernel_sha") != sha_of(INDEX_KERNEL_SOURCES):
+        return None
+    return rec.get("per_launch_bytes", {}).get(workload)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from csa_synth import decode_inputs, get_workload
+    from long_context_sparse_csa_b200 import binding as C
+    from long_context_sparse_csa_b200.state import LayerState, to_device
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    C.lib()
+    wl = get_workload(args.workload)
+    R = max(1, args.replicas)
+    dev = torch.device("cuda", local)
+
+    datas, layers = [], []
+    for li, spec in enumerate(wl.layers):
+        d = decode_inputs(wl, li)
+        datas.append(d)
+        base = LayerState.from_arrays(spec, wl.B, d, device=dev)
+        insts = [base]
+        for _ in range(R - 1):
+            insts.append(LayerState(spec, wl.B, 0, entries=base.entries.clone(), window=base.window.clone(),
+                                    raw=base.raw.clone(), gate=base.gate.clone(),
+                                    idx_keys=None if base.idx_keys is None else base.idx_keys.clone(),
+                                    idx_key_scale=None if base.idx_key_scale is None else base.idx_key_scale.clone(),
+                                    pos_bias=base.pos_bias, gamma_kv=base.gamma_kv, gamma_q=base.gamma_q,
+                                    sinks=base.sinks))
+        cap = d["entries"].shape[1]
+        io = {k: to_device(d[k], dev) for k in ["q", "x_new", "g_new", "t"]}
+        if spec.kind == "csa":
+            for k in ["idx_q", "idx_q_scale", "head_w"]:
+                io[k] = to_device(d[k], dev)
+            io["topk"] = torch.zeros((wl.B, spec.top_k), dtype=torch.int32, device=dev)
+        io["out"] = torch.zeros((wl.B, spec.H, spec.D), dtype=torch.int16 if spec.act_format == "bf16" else torch.float32,
+                                device=dev)
+        ws = base.workspace("decode_step", 1, cap)
+        layers.append({"spec": spec, "insts": insts, "io": io, "ws": ws,
+                       "caches": [s.cache() for s in insts], "params": base.params(), "L": base.L})
+
+    def run_step(r):
+        for li, lay in enumerate(layers):
+            io, spec = lay["io"], lay["spec"]
+            if spec.kind == "csa":
+                C.csa_decode_step(lay["L"], lay["caches"][r], lay["params"], io["q"], io["idx_q"], io["idx_q_scale"],
+                                  io["head_w"], io["x_new"], io["g_new"], io["t"], io["out"], io["topk"], lay["ws"])
+            else:
+                C.hca_decode_step(lay["L"], lay["caches"][r], lay["params"], io["q"], io["x_new"], io["g_new"],
+                                  io["t"], io["out"], lay["ws"])
+
+    # eager warm-up of every instance (module load, attributes), then one graph per instance
+    for r in range(R):
+        run_step(r)
+    torch.cuda.synchronize()
+    for lay in layers:
+        assert C.csa_device_error(lay["ws"]) == 0
+    has_csa = any(l["spec"].kind == "csa" for l in layers)
+    ev = lambda: torch.cuda.Event(enable_timing=True, external=True)  # noqa: E731
+    stream = torch.cuda.Stream(device=dev)
+
+    def capture(rs, with_events):
+        """One CUDA graph running the steps of instances rs in order; optional per-step events."""
+        evs = []
+        if with_events:
+            for _ in rs:
+                e = {"idx": (ev(), ev()), "lay": [(ev(), ev()) for _ in layers]}
+                for x in list(e["idx"]) + [y for p in e["lay"] for y in p]:
+                    x.record()
+                evs.append(e)
+            torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        n0 = C.csa_launch_count()
+        with torch.cuda.graph(g, stream=stream):
+            for j, r in enumerate(rs):
+                for li, lay in enumerate(layers):
+                    if with_events:
+                        evs[j]["lay"][li][0].record()
+                    io, spec = lay["io"], lay["spec"]
+                    if spec.kind == "csa":
+                        if with_events:
+                            C.csa_profile_events(*evs[j]["idx"])
+                        C.csa_decode_step(lay["L"], lay["caches"][r], lay["params"], io["q"], io["idx_q"],
+                                          io["idx_q_scale"], io["head_w"], io["x_new"], io["g_new"], io["t"],
+                                          io["out"], io["topk"], lay["ws"])
+                        C.csa_profile_events(None, None)
+                    else:
+                        C.hca_decode_step(lay["L"], lay["caches"][r], lay["params"], io["q"], io["x_new"],
+                                          io["g_new"], io["t"], io["out"], lay["ws"])
+                    if with_events:
+                        evs[j]["lay"][li][1].record()
+        return g, evs, C.csa_launch_count() - n0
+
+    cycle, cycle_ev, n_launch = capture(list(range(R)), True)
+    launches_per_step = n_launch // R
+    singles = [capture([r], False)[0] for r in range(R)]
+    torch.cuda.synchronize()
+
+    def run_steps(k):
+        """Exactly k decode steps: whole cycles of the R instances, then single steps."""
+        for _ in range(k // R):
+            cycle.replay()
+        for r in range(k % R):
+            singles[r].replay()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    cur = torch.cuda.current_stream()
+    clocks = ClockSampler(local)
+    clocks.start()
+    # warm-up: W steps, plus a short burn so clocks settle at load before the timed region
+    run_steps(args.warmup)
+    t_burn = time.perf_counter()
+    while time.perf_counter() - t_burn < 0.5:
+        cycle.replay()
+        torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.sample()
+    w0 = time.perf_counter()
+    e0.record(cur)
+    run_steps(args.steps)
+    e1.record(cur)
+    torch.cuda.synchronize()
+    w1 = time.perf_counter()
+    clocks.sample()
+    barrier()
+    T_ms = max_over_ranks(e0.elapsed_time(e1))
+    clk = clocks.summary(w0, w1)
+    # per-kernel / per-layer device times: the last replay of the cycle graph (one step per instance);
+    # the burn above replayed it after the warm-up, so these are steady-state launches
+    idx_ms = [e["idx"][0].elapsed_time(e["idx"][1]) for e in cycle_ev] if has_csa else []
+    lay_ms = [[e["lay"][li][0].elapsed_time(e["lay"][li][1]) for e in cycle_ev] for li in range(len(layers))]
+
+    # ------------------------------------------------------------------ end to end through host memory
+    h2d, d2h = [], []
+    for lay in layers:
+        for k in ["q", "idx_q", "idx_q_scale", "head_w", "x_new", "g_new", "t"]:
+            if k in lay["io"]:
+                t = lay["io"][k]
+                h2d.append((torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t), t))
+        o = lay["io"]["out"]
+        d2h.append((o, torch.empty(o.shape, dtype=o.dtype, pin_memory=True)))
+    h2d_bytes = sum(h.numel() * h.element_size() for h, _ in h2d)
+    d2h_bytes = sum(h.numel() * h.element_size() for _, h in d2h)
+    for s in range(args.warmup):
+        for h, dv in h2d:
+            dv.copy_(h, non_blocking=True)
+        singles[s % R].replay()
+        for dv, h in d2h:
+            h.copy_(dv, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(cur)
+    for s in range(args.steps):
+        for h, dv in h2d:
+            dv.copy_(h, non_blocking=True)
+        singles[s % R].replay()
+        for dv, h in d2h:
+            h.copy_(dv, non_blocking=True)
+    f1.record(cur)
+    torch.cuda.synchronize()
+    barrier()
+    E_ms = max_over_ranks(f0.elapsed_time(f1))
+    clocks.stop()
+
+    for lay in layers:
+        assert C.csa_device_error(lay["ws"]) == 0
+
+    units = wl.B * len(layers) * args.steps * world
+    value = units / (T_ms / 1e3)
+    e2e_value = units / (E_ms / 1e3)
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": T_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3+bf16 (fp32 accumulate)", "data": "synthetic",
+            "config": workload_config(wl, R)}
+    line["per_layer_us"] = {f"{l['spec'].kind}{li}": 1e3 * float(np.mean(lay_ms[li])) for li, l in enumerate(layers)}
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+        peak, peak_note = float(peaks["hbm_gbs"]), "of measured"
+    except (OSError, KeyError, ValueError):
+        peak, peak_note = 6650.0, "of fallback"
+    if has_csa:
+        csa_li = [i for i, l in enumerate(layers) if l["spec"].kind == "csa"][0]
+        spec = layers[csa_li]["spec"]
+        nv = wl.n // spec.m
+        bytes_idx = index_kernel_bytes(spec, nv, wl.B)
+        t_idx = float(np.mean(idx_ms)) / 1e3
+        achieved = bytes_idx / t_idx / 1e9
+        line["roofline"] = {"bound": "hbm", "kernel": "index_score_tc_kernel", "achieved": achieved, "peak": peak,
+                            "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_note,
+                            "traffic": recorded_traffic(wl.name), "algorithmic_bytes": bytes_idx,
+                            "launch_us": 1e6 * t_idx}
+    else:
+        spec = layers[0]["spec"]
+        b = step_bytes(spec, wl.n, wl.B)
+        t = float(np.mean(lay_ms[0])) / 1e3
+        line["roofline"] = {"bound": "hbm", "kernel": "hca layer step", "achieved": b / t / 1e9, "peak": peak,
+                            "unit": "GB/s", "frac": b / t / 1e9 / peak, "peak_source": peak_note, "traffic": None,
+                            "algorithmic_bytes": b}
+    step_alg = sum(step_bytes(l["spec"], wl.n, wl.B) for l in layers)
+    line["step_hbm"] = {"algorithmic_bytes": step_alg, "achieved_gbs": step_alg / (T_ms / args.steps / 1e3) / 1e9,
+                        "frac": step_alg / (T_ms / args.steps / 1e3) / 1e9 / peak}
+    line["e2e"] = {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
+                   "ms_per_step": E_ms / args.steps}
+    line["gpu_launches"] = int(launches_per_step) * args.steps
+    line["clocks"] = clk
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        times = run_cpu_oracle(wl, datas, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": wl.B * len(layers) / float(np.mean(times)), "unit": UNIT,
+                                "cores": cpu_threads(), "kind": "oracle",
+                                "sample": f"{len(times)} full decode steps of the workload ({args.cpu_seconds:.0f} s budget)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del cycle, singles
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

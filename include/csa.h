@@ -162,6 +162,17 @@ CSA_API const char* csa_version(void);
  * (0 = none); returns CSA_ERR_DEVICE_TIMEOUT if any bit was set. */
 CSA_API csa_status_t csa_device_error(void* workspace, size_t ws_bytes, void* stream, int32_t* code);
 
+/* Profiling aid (no counterpart on the pages).  When ev_start and ev_stop (cudaEvent_t handles
+ * created with timing enabled) are both non-NULL, every later call made from this host thread
+ * records ev_start immediately before and ev_stop immediately after the launch of the indexer
+ * score kernel (the dominant kernel of a CSA decode step), with the external-record flag so the
+ * records become event nodes when the stream is being captured into a CUDA graph.  NULL, NULL
+ * turns it off.  Host only; never fails. */
+CSA_API void csa_profile_events(void* ev_start, void* ev_stop);
+
+/* Number of kernels this process has launched through the library so far (host counter). */
+CSA_API uint64_t csa_launch_count(void);
+
 /* Append Tq new tokens per sequence: raw rows x_new[b][j] (and gate rows
  * g_new) are written into the raw / gate rings at slot (r - raw_base) mod
  * raw_cap (skipped when x_new is NULL: the rows are then already in the raw

@@ -60,6 +60,8 @@ _SIGS = {
     "csa_workspace_size": (_SZ, [_LAYER, _I32, _I32, _I64]),
     "csa_last_error": (ctypes.c_char_p, []),
     "csa_version": (ctypes.c_char_p, []),
+    "csa_profile_events": (None, [_P, _P]),
+    "csa_launch_count": (ctypes.c_uint64, []),
     "csa_device_error": (ctypes.c_int, [_P, _SZ, _P, ctypes.POINTER(_I32)]),
     "csa_append": (ctypes.c_int, [_LAYER, _CACHE, _P, _P, _P, _I32, _P]),
     "csa_compress": (ctypes.c_int, [_LAYER, _CACHE, _PARAMS, _P, _I32, _P]),
@@ -146,6 +148,19 @@ def csa_workspace_size(L: CsaLayer, op: str, Tq: int, entry_cap: int) -> int:
 
 def csa_version() -> str:
     return lib().csa_version().decode()
+
+
+def csa_profile_events(ev_start, ev_stop):
+    """Record these torch.cuda.Events around each later indexer-score launch (None, None: off)."""
+    h = lib()
+    if ev_start is None or ev_stop is None:
+        h.csa_profile_events(None, None)
+    else:
+        h.csa_profile_events(ctypes.c_void_p(ev_start.cuda_event), ctypes.c_void_p(ev_stop.cuda_event))
+
+
+def csa_launch_count() -> int:
+    return lib().csa_launch_count()
 
 
 def csa_device_error(workspace, stream=None) -> int:

@@ -1,4 +1,5 @@
 // C ABI of the CSA/HCA operator: argument checks, workspace layout, launches.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -12,6 +13,8 @@ using namespace csa;
 namespace {
 
 thread_local std::string g_err;
+thread_local cudaEvent_t g_prof_start = nullptr, g_prof_stop = nullptr;
+std::atomic<uint64_t> g_launches{0};
 
 csa_status_t fail(csa_status_t st, const char* fmt, ...) {
   char buf[512];
@@ -210,7 +213,10 @@ csa_status_t run_index_topk(const csa_layer_t* L, const csa_cache_t* cache, cons
   a.head_w = head_w;
   a.scores = scores;
   a.err = err;
+  const bool prof = g_prof_start && g_prof_stop;
+  if (prof) cudaEventRecordWithFlags(g_prof_start, s, cudaEventRecordExternal);
   cudaError_t e = launch_index_scores(a, num_sms(), s);
+  if (prof) cudaEventRecordWithFlags(g_prof_stop, s, cudaEventRecordExternal);
   if (e != cudaSuccess) return cuda_fail(e, "index-score launch");
   TopkArgs t;
   t.scores = scores; t.n_max = n_max; t.rows = L->B * Tq; t.Tq = Tq; t.m = L->m; t.k = L->top_k;
@@ -255,6 +261,10 @@ csa_status_t check_params(const csa_layer_t* L, const csa_params_t* P, bool need
 
 }  // namespace
 
+namespace csa {
+void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace csa
+
 // ============================================================================= exported
 extern "C" {
 
@@ -268,6 +278,13 @@ size_t csa_workspace_size(const csa_layer_t* L, int32_t op, int32_t Tq, int64_t 
 const char* csa_last_error(void) { return g_err.c_str(); }
 
 const char* csa_version(void) { return "csa-b200 0.1 (sm_100a)"; }
+
+void csa_profile_events(void* ev_start, void* ev_stop) {
+  g_prof_start = static_cast<cudaEvent_t>(ev_start);
+  g_prof_stop = static_cast<cudaEvent_t>(ev_stop);
+}
+
+uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 csa_status_t csa_device_error(void* workspace, size_t ws_bytes, void* stream, int32_t* code) {
   if (!workspace || ws_bytes < 4) return fail(CSA_ERR_WORKSPACE, "workspace is NULL");

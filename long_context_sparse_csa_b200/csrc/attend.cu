@@ -540,9 +540,11 @@ cudaError_t launch_mma(const AttendArgs& a, cudaStream_t s) {
   }
   dim3 grid(a.splits, a.L.H / HG, a.rows);
   attend_mma_kernel<HG, FMT><<<grid, HG * 8, smem, s>>>(a);
+  note_launches(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || a.splits == 1) return e;
   attend_combine_kernel<HG><<<dim3(a.L.H, a.rows), kD / 4, 0, s>>>(a);
+  note_launches(1);
   return cudaGetLastError();
 }
 
@@ -578,6 +580,7 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
   const int HG = attend_head_group(a.L);
   if (HG == 0) {
     attend_generic_kernel<<<a.rows, a.L.H * 32, 0, s>>>(a);
+    note_launches(1);
     return cudaGetLastError();
   }
   const bool mixed = a.L.kv_fmt == CSA_FMT_MIXED;

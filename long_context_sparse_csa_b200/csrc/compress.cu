@@ -148,6 +148,7 @@ __global__ void append_compress_kernel(const __grid_constant__ AppendCompressArg
 cudaError_t launch_append_compress(const AppendCompressArgs& a, int B, int Tq, cudaStream_t s) {
   dim3 grid(Tq, B);
   append_compress_kernel<<<grid, a.L.D / 4, 0, s>>>(a);
+  note_launches(1);
   return cudaGetLastError();
 }
 

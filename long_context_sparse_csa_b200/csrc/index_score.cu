@@ -306,6 +306,7 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
       if (e != cudaSuccess) return e;
     }
     index_score_generic_kernel<<<grid, 128, sm, s>>>(a);
+    note_launches(1);
     return cudaGetLastError();
   }
   a.QN = a.Tq == 1 ? 1 : min(256 / a.H_I, a.Tq);
@@ -328,6 +329,7 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
   }
   const int64_t grid = a.total_items < num_sms ? a.total_items : num_sms;
   index_score_tc_kernel<<<(unsigned)grid, kThreads, smem, s>>>(kmap, qmap, a, N, cols);
+  note_launches(1);
   return cudaGetLastError();
 }
 

@@ -9,6 +9,9 @@
 
 namespace csa {
 
+// Host-side count of kernel launches issued by the library (for launch accounting).
+void note_launches(int n);
+
 // ----------------------------------------------------------------------------- append + compress
 struct AppendCompressArgs {
   LayerArgs L;

@@ -146,6 +146,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
     configured = smem;
   }
   topk_rows_kernel<<<a.rows, kThreads, smem, s>>>(a, use_smem);
+  note_launches(1);
   return cudaGetLastError();
 }
 

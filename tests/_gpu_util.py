@@ -58,10 +58,13 @@ def assert_rows_match(gpu_rows, ref_vals, fmt, D, d_rope=64, slack_rel=2e-5, max
     """GPU-written stored rows vs the oracle's exact float64 values (before encoding)."""
     g = F.decode_rows(gpu_rows, fmt, D, d_rope)
     x = np.asarray(ref_vals, np.float64)
+    # float32 rounding in the kernel is relative to the row's scale (the summands), not to a value
+    # that happens to land near zero: allow 2e-6 of the row's rms on top of one quantum.
+    row_rms = np.sqrt(np.mean(x * x, axis=-1, keepdims=True))
     if fmt == "f32":
-        tol = 1e-5 * np.abs(x) + 1e-6
+        tol = 1e-5 * np.abs(x) + 2e-6 * row_rms
     elif fmt == "bf16":
-        tol = _quantum_bf16(x) + slack_rel * np.abs(x) + 1e-7
+        tol = _quantum_bf16(x) + slack_rel * np.abs(x) + 2e-6 * row_rms
     else:
         dn = D - d_rope
         sig_g = np.ascontiguousarray(gpu_rows[..., D + 64:D + 68]).view(np.float32)[..., 0].astype(np.float64)
@@ -70,7 +73,7 @@ def assert_rows_match(gpu_rows, ref_vals, fmt, D, d_rope=64, slack_rel=2e-5, max
         tol = np.empty_like(x)
         tol[..., :dn] = _quantum_e4m3(x[..., :dn] / sig) * sig
         tol[..., dn:] = _quantum_bf16(x[..., dn:])
-        tol += slack_rel * np.abs(x) + 1e-7
+        tol += slack_rel * np.abs(x) + 2e-6 * row_rms
         assert np.mean(sig_g == sig_o) > 0.99, "row scales disagree on more than 1% of rows"
     err = np.abs(g - x)
     bad = err > tol
@@ -101,11 +104,16 @@ def check_topk(gpu_idx, oracle_scores, k, rel=1e-4):
     return len(diff) // 2
 
 
-def assert_out_close(gpu, ref, max_abs=2e-2, mean_abs=2e-3, rel_l2=1e-2):
+STATS = []
+
+
+def assert_out_close(gpu, ref, max_abs=2e-2, mean_abs=2e-3, rel_l2=1e-2, tag=""):
     gpu = np.asarray(gpu, np.float64)
     ref = np.asarray(ref, np.float64)
     d = np.abs(gpu - ref)
     rl2 = np.linalg.norm(gpu - ref) / max(np.linalg.norm(ref), 1e-30)
+    STATS.append({"tag": tag, "max_abs": float(d.max()), "mean_abs": float(d.mean()), "rel_l2": float(rl2),
+                  "ref_rms": float(np.sqrt(np.mean(ref * ref)))})
     assert d.max() <= max_abs, f"max-abs {d.max()}"
     assert d.mean() <= mean_abs, f"mean-abs {d.mean()}"
     assert rl2 <= rel_l2, f"relative L2 {rl2}"

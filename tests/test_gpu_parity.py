@@ -5,6 +5,9 @@ from oracle/.  Sizes span several tiles with ragged tails; the full-size
 workloads are checked on their own launch configuration.
 """
 
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -16,6 +19,7 @@ from long_context_sparse_csa_b200.state import LayerState
 from oracle import csa as O
 from oracle import formats as F
 
+import _gpu_util
 from _gpu_util import assert_out_close, assert_rows_match, check_topk, dev, host, out_values
 
 pytestmark = pytest.mark.gpu
@@ -28,6 +32,10 @@ def _cuda():
     C.lib()
     yield
     torch.cuda.synchronize()
+    out = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "gpurun_out")
+    if os.path.isdir(out):
+        with open(os.path.join(out, "parity_stats.json"), "w") as f:
+            json.dump(_gpu_util.STATS, f, indent=1)
 
 
 def _layer(**kw):
@@ -193,7 +201,7 @@ def _run_decode(wl, li=0, n=None, d=None, sharp=1.0):
     return d, st, out, topk
 
 
-def _check_decode(wl, li=0, n=None, bs=None, sharp=1.0, rel_l2=1e-2):
+def _check_decode(wl, li=0, n=None, bs=None, sharp=1.0, rel_l2=1e-2, max_abs=2e-2, mean_abs=2e-3):
     layer = wl.layers[li]
     d, st, out, topk = _run_decode(wl, li, n, sharp=sharp)
     got = out_values(out, layer.act_format)
@@ -225,7 +233,8 @@ def _check_decode(wl, li=0, n=None, bs=None, sharp=1.0, rel_l2=1e-2):
                 # a tie-band swap: attend over the GPU's (valid) selection
                 d2 = dict(d)
                 ref = _oracle_with_selection(L, d, b, tk)
-        assert_out_close(got[b], ref["o"], rel_l2=rel_l2)
+        assert_out_close(got[b], ref["o"], max_abs=max_abs, mean_abs=mean_abs, rel_l2=rel_l2,
+                         tag=f"{wl.name}/L{li}/n={n}/b={b}/sharp={sharp}")
 
 
 def _oracle_with_selection(L, d, b, sel):
@@ -311,7 +320,10 @@ def test_decode_csa_128k():
 
 
 def test_decode_csa_128k_sharp_logits():
-    _check_decode(get_workload("csa_decode_128k", B=2), sharp=8.0, rel_l2=4e-2)
+    # Logits 8x sharper than 1/sqrt(D).  The kernel rounds q~ to bf16 (relative 2^-9 per element), so a
+    # logit moves by up to ~8 * 2^-9 * sum|q_d k_d| / sqrt(D) ~ 0.04 and the output, dominated by a few
+    # keys of size ~3, by up to ~0.1: the bound here is 4x the standard one.
+    _check_decode(get_workload("csa_decode_128k", B=2), sharp=8.0, rel_l2=4e-2, max_abs=8e-2, mean_abs=8e-3)
 
 
 @pytest.mark.parametrize("li", [0, 1])
