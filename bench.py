@@ -48,6 +48,7 @@ def parse():
     p.add_argument("--replicas", type=int, default=8)
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--burn-seconds", type=float, default=0.5, help="untimed replays before timing (clocks settle)")
     return p.parse_args()
 
 
@@ -373,7 +374,7 @@ def run_ours(args):
     # warm-up: W steps, plus a short burn so clocks settle at load before the timed region
     run_steps(args.warmup)
     t_burn = time.perf_counter()
-    while time.perf_counter() - t_burn < 0.5:
+    while time.perf_counter() - t_burn < args.burn_seconds:
         cycle.replay()
         torch.cuda.synchronize()
     torch.cuda.synchronize()

@@ -137,10 +137,18 @@ csa_status_t check_cache_raw(const csa_layer_t* L, const csa_cache_t* c, bool ne
 
 // ----------------------------------------------------------------------------- workspace layout
 constexpr size_t kAlign = 256;
+
+// Long decode rows take the multi-CTA top-k, fed by the tensor-core indexer's histogram.
+bool use_split_topk(const csa_layer_t* L, int32_t Tq, int64_t n_max) {
+  return Tq == 1 && n_max >= kTopkSplitMinN && n_max <= kTopkSplitMaxN &&
+         index_tc_supported(L->idx_format, L->H_I, L->d_I);
+}
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Workspace {
   size_t err = 0;          // int error word
+  size_t hist = 0, hist_bytes = 0;      // split top-k: histogram [rows][4096] + counters [rows][4]
+  size_t sure = 0, cand = 0;            // split top-k scratch
   size_t scores = 0, scores_bytes = 0;
   size_t topk = 0, topk_bytes = 0;
   size_t part = 0, part_bytes = 0;
@@ -155,6 +163,11 @@ Workspace layout(const csa_layer_t* L, int op, int32_t Tq, int64_t n_max) {
   const bool csa = L->kind == CSA_KIND_CSA;
   if (csa && (op == CSA_OP_INDEX_TOPK || op == CSA_OP_DECODE_STEP || op == CSA_OP_PREFILL)) {
     w.scores = off; w.scores_bytes = rows * (size_t)(n_max > 0 ? n_max : 1) * 4; off = up(off + w.scores_bytes);
+    if (use_split_topk(L, Tq, n_max)) {
+      w.hist = off; w.hist_bytes = rows * (4096 + 4) * 4; off = up(off + w.hist_bytes);
+      w.sure = off; off = up(off + rows * (size_t)L->top_k * 4);
+      w.cand = off; off = up(off + rows * (size_t)n_max * 8);
+    }
   }
   if (csa && (op == CSA_OP_DECODE_STEP || op == CSA_OP_PREFILL)) {
     w.topk = off; w.topk_bytes = rows * (size_t)L->top_k * 4; off = up(off + w.topk_bytes);
@@ -199,7 +212,16 @@ csa_status_t run_append_compress(const csa_layer_t* L, const csa_cache_t* cache,
 
 csa_status_t run_index_topk(const csa_layer_t* L, const csa_cache_t* cache, const void* idx_q,
                             const float* idx_q_scale, const float* head_w, const int64_t* q_pos, int32_t Tq,
-                            int64_t n_max, int32_t* topk, float* scores, int* err, cudaStream_t s) {
+                            int64_t n_max, int32_t* topk, float* scores, const Workspace& w, void* ws,
+                            cudaStream_t s) {
+  int* err = reinterpret_cast<int*>(at(ws, w.err));
+  const bool split = use_split_topk(L, Tq, n_max);
+  const int rows = L->B * Tq;
+  uint32_t* hist = split ? reinterpret_cast<uint32_t*>(at(ws, w.hist)) : nullptr;
+  if (split) {
+    cudaError_t e = cudaMemsetAsync(hist, 0, w.hist_bytes, s);
+    if (e != cudaSuccess) return cuda_fail(e, "histogram reset");
+  }
   IndexArgs a;
   memset(&a, 0, sizeof(a));
   a.B = L->B; a.Tq = Tq; a.H_I = L->H_I; a.d_I = L->d_I; a.m = L->m;
@@ -212,6 +234,7 @@ csa_status_t run_index_topk(const csa_layer_t* L, const csa_cache_t* cache, cons
   a.q_scale = idx_q_scale;
   a.head_w = head_w;
   a.scores = scores;
+  a.hist = hist;
   a.err = err;
   const bool prof = g_prof_start && g_prof_stop;
   if (prof) cudaEventRecordWithFlags(g_prof_start, s, cudaEventRecordExternal);
@@ -219,9 +242,20 @@ csa_status_t run_index_topk(const csa_layer_t* L, const csa_cache_t* cache, cons
   if (prof) cudaEventRecordWithFlags(g_prof_stop, s, cudaEventRecordExternal);
   if (e != cudaSuccess) return cuda_fail(e, "index-score launch");
   TopkArgs t;
-  t.scores = scores; t.n_max = n_max; t.rows = L->B * Tq; t.Tq = Tq; t.m = L->m; t.k = L->top_k;
+  t.scores = scores; t.n_max = n_max; t.rows = rows; t.Tq = Tq; t.m = L->m; t.k = L->top_k;
   t.pos0 = L->pos0; t.q_pos = q_pos; t.out = topk;
-  e = launch_topk(t, s);
+  if (split) {
+    TopkSplitArgs sa;
+    sa.base = t;
+    sa.hist = hist;
+    sa.cnt = hist + (size_t)rows * 4096;
+    sa.sure = reinterpret_cast<int32_t*>(at(ws, w.sure));
+    sa.cand = reinterpret_cast<uint2*>(at(ws, w.cand));
+    sa.G = topk_split_ctas(rows, n_max, num_sms());
+    e = launch_topk_split(sa, s);
+  } else {
+    e = launch_topk(t, s);
+  }
   return e == cudaSuccess ? CSA_OK : cuda_fail(e, "top-k launch");
 }
 
@@ -345,8 +379,8 @@ csa_status_t csa_index_topk(const csa_layer_t* L, const csa_cache_t* cache, cons
   CSA_TRY(check_ws(w, workspace, ws_bytes));
   if (scores) CSA_TRY(need_ptr(scores, "scores", 4));
   float* sc = scores ? scores : reinterpret_cast<float*>(at(workspace, w.scores));
-  return run_index_topk(L, cache, idx_q, idx_q_scale, head_w, q_pos, Tq, n_max, topk_idx, sc,
-                        reinterpret_cast<int*>(at(workspace, w.err)), static_cast<cudaStream_t>(stream));
+  return run_index_topk(L, cache, idx_q, idx_q_scale, head_w, q_pos, Tq, n_max, topk_idx, sc, w, workspace,
+                        static_cast<cudaStream_t>(stream));
 }
 
 csa_status_t csa_sparse_attend(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P,
@@ -413,7 +447,7 @@ csa_status_t csa_decode_step(const csa_layer_t* L, const csa_cache_t* cache, con
   CSA_TRY(run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, s));
   int32_t* tk = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(at(workspace, w.topk));
   CSA_TRY(run_index_topk(L, cache, idx_q, idx_q_scale, head_w, q_pos, 1, cache->entry_cap, tk,
-                         reinterpret_cast<float*>(at(workspace, w.scores)), reinterpret_cast<int*>(at(workspace, w.err)), s));
+                         reinterpret_cast<float*>(at(workspace, w.scores)), w, workspace, s));
   return run_attend(L, cache, P, q, q_pos, 1, tk, cache->entry_cap, out, w, workspace, s);
 }
 
@@ -471,7 +505,7 @@ csa_status_t csa_prefill(const csa_layer_t* L, const csa_cache_t* cache, const c
   if (csa) {
     tk = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(at(workspace, w.topk));
     CSA_TRY(run_index_topk(L, cache, idx_q, idx_q_scale, head_w, q_pos, Tq, n_max, tk,
-                           reinterpret_cast<float*>(at(workspace, w.scores)), reinterpret_cast<int*>(at(workspace, w.err)), s));
+                           reinterpret_cast<float*>(at(workspace, w.scores)), w, workspace, s));
   }
   return run_attend(L, cache, P, q, q_pos, Tq, tk, n_max, out, w, workspace, s);
 }

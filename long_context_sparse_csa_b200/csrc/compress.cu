@@ -32,23 +32,25 @@ __device__ __forceinline__ void rope4(float v[4], int c0, const LayerArgs& L, do
   v[2] = a * c - b * s; v[3] = a * s + b * c;
 }
 
-// Block-cooperative store of one row in the cache format (all threads call).
-__device__ __forceinline__ void pack_row(uint8_t* dst, const LayerArgs& L, int c0, const float v[4],
+// Block-cooperative store of one row in the cache format.  Every thread of the block calls it
+// (the FP8 scale needs a block-wide max); threads with active == false hold no channels.
+__device__ __forceinline__ void pack_row(uint8_t* dst, const LayerArgs& L, int c0, const float v[4], bool active,
                                          float* scratch) {
   if (L.kv_fmt == CSA_FMT_F32) {
-    *reinterpret_cast<float4*>(dst + 4 * (size_t)c0) = make_float4(v[0], v[1], v[2], v[3]);
+    if (active) *reinterpret_cast<float4*>(dst + 4 * (size_t)c0) = make_float4(v[0], v[1], v[2], v[3]);
     return;
   }
   if (L.kv_fmt == CSA_FMT_BF16) {
-    store_act4(dst, CSA_FMT_BF16, c0, v);
+    if (active) store_act4(dst, CSA_FMT_BF16, c0, v);
     return;
   }
   const int dn = L.D - L.d_rope;
   float am = 0.f;
-  if (c0 < dn) am = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+  if (active && c0 < dn) am = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
   am = block_max(am, scratch);
   float inv;
   const float sig = pow2_scale(am, &inv);
+  if (!active) return;
   if (c0 < dn) {
     uint32_t w = (uint32_t)f_to_e4m3_sat(v[0] * inv) | ((uint32_t)f_to_e4m3_sat(v[1] * inv) << 8) |
                  ((uint32_t)f_to_e4m3_sat(v[2] * inv) << 16) | ((uint32_t)f_to_e4m3_sat(v[3] * inv) << 24);
@@ -63,28 +65,38 @@ __device__ __forceinline__ void pack_row(uint8_t* dst, const LayerArgs& L, int c
   }
 }
 
-__global__ void append_compress_kernel(const __grid_constant__ AppendCompressArgs a) {
+constexpr int kRowBatch = 8;   // rows whose loads are issued together per thread
+
+// Block = (D/4) channel threads x RG row groups.  Row group 0 appends the new token; every row
+// group pools a strided subset of the entry's source rows with an online softmax; the groups'
+// partial (max, sum, weighted sum) are merged through shared memory.
+__global__ void __launch_bounds__(512) append_compress_kernel(const __grid_constant__ AppendCompressArgs a) {
   __shared__ float scratch[32];
+  extern __shared__ float part[];                  // [RG][3][D]
   const LayerArgs& L = a.L;
   const CacheArgs& C = a.C;
   const int j = blockIdx.x, b = blockIdx.y;
-  const int c0 = threadIdx.x * 4;
+  const int CT = L.D / 4;                          // channel threads per row group
+  const int RG = blockDim.x / CT;
+  const int ct = threadIdx.x % CT, rg = threadIdx.x / CT;
+  const int c0 = ct * 4;
+  const bool lead = rg == 0;
   const int64_t t = a.q_pos[(int64_t)b * a.Tq + j];
   const int64_t r = t - L.pos0;
   if (r < 0) return;  // uniform over the block
   const size_t arow = (size_t)L.D * act_bytes(L.act_fmt);
   const bool have_new = a.x_new != nullptr;
-  float x[4], g[4] = {0.f, 0.f, 0.f, 0.f};
+  float x[4] = {0.f, 0.f, 0.f, 0.f}, g[4] = {0.f, 0.f, 0.f, 0.f};
   if (have_new) {
     load_act4(a.x_new + ((size_t)b * a.Tq + j) * arow, L.act_fmt, c0, x);
     load_act4(a.g_new + ((size_t)b * a.Tq + j) * arow, L.act_fmt, c0, g);
-  } else {
+  } else if (a.do_append) {
     const int64_t s = ring_slot(r, C.raw_base, C.raw_cap);
     load_act4(C.raw + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, x);
   }
 
   if (a.do_append) {
-    if (have_new) {
+    if (have_new && lead) {
       const int64_t s = ring_slot(r, C.raw_base, C.raw_cap);
       store_act4(C.raw + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, x);
       store_act4(C.gate + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, g);
@@ -92,62 +104,115 @@ __global__ void append_compress_kernel(const __grid_constant__ AppendCompressArg
     float w[4] = {x[0], x[1], x[2], x[3]};
     rope4(w, c0, L, (double)t);
     uint8_t* dst = C.window + ((size_t)b * C.window_cap + (size_t)(r % C.window_cap)) * L.row_bytes;
-    pack_row(dst, L, c0, w, scratch);
+    pack_row(dst, L, c0, w, lead, scratch);
   }
 
-  if (a.do_compress && ((r + 1) % L.m) == 0) {
-    const int64_t i = (r + 1) / L.m - 1;
-    const int64_t lo = (i - L.ov) * (int64_t)L.m;
-    const int64_t r_begin = lo < 0 ? 0 : lo;
-    float mx[4], sum[4], acc[4];
+  if (!(a.do_compress && ((r + 1) % L.m) == 0)) return;
+  const int64_t i = (r + 1) / L.m - 1;
+  const int64_t lo = (i - L.ov) * (int64_t)L.m;
+  const int64_t r_begin = lo < 0 ? 0 : lo;
+  float mx[4], sum[4], acc[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) { mx[k] = -INFINITY; sum[k] = 0.f; acc[k] = 0.f; }
-    for (int64_t rr = r_begin; rr <= r; ++rr) {
-      float xv[4], gv[4];
+  for (int k = 0; k < 4; ++k) { mx[k] = -INFINITY; sum[k] = 0.f; acc[k] = 0.f; }
+  // rows r_begin + rg, + RG, ... in batches whose loads are all in flight together
+  for (int64_t rb = r_begin + rg; rb <= r; rb += (int64_t)RG * kRowBatch) {
+    float xv[kRowBatch][4], gv[kRowBatch][4];
+#pragma unroll
+    for (int u = 0; u < kRowBatch; ++u) {
+      const int64_t rr = rb + (int64_t)u * RG;
+      if (rr > r) break;
       if (rr == r && have_new) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) { xv[k] = x[k]; gv[k] = g[k]; }
+        for (int k = 0; k < 4; ++k) { xv[u][k] = x[k]; gv[u][k] = g[k]; }
       } else {
         const int64_t s = ring_slot(rr, C.raw_base, C.raw_cap);
-        load_act4(C.raw + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, xv);
-        load_act4(C.gate + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, gv);
+        load_act4(C.raw + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, xv[u]);
+        load_act4(C.gate + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, gv[u]);
       }
+    }
+#pragma unroll
+    for (int u = 0; u < kRowBatch; ++u) {
+      const int64_t rr = rb + (int64_t)u * RG;
+      if (rr > r) break;
       const float4 bias = *reinterpret_cast<const float4*>(a.pos_bias + (size_t)(rr - lo) * L.D + c0);
       const float bz[4] = {bias.x, bias.y, bias.z, bias.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float z = gv[k] + bz[k];
+        const float z = gv[u][k] + bz[k];
         if (z > mx[k]) {
           const float sc = expf(mx[k] - z);
           sum[k] = sum[k] * sc + 1.f;
-          acc[k] = acc[k] * sc + xv[k];
+          acc[k] = acc[k] * sc + xv[u][k];
           mx[k] = z;
         } else {
           const float e = expf(z - mx[k]);
           sum[k] += e;
-          acc[k] += e * xv[k];
+          acc[k] += e * xv[u][k];
         }
       }
     }
-    float e[4];
-    float ss = 0.f;
+  }
+  // merge the row groups
+  if (RG > 1) {
+    float* pm = part + (size_t)rg * 3 * L.D;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      pm[c0 + k] = mx[k];
+      pm[L.D + c0 + k] = sum[k];
+      pm[2 * L.D + c0 + k] = acc[k];
+    }
+    __syncthreads();
+    if (lead) {
+      for (int q = 1; q < RG; ++q) {
+        const float* po = part + (size_t)q * 3 * L.D;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float m2 = po[c0 + k];
+          if (m2 == -INFINITY) continue;
+          const float M = fmaxf(mx[k], m2);
+          const float f1 = expf(mx[k] - M), f2 = expf(m2 - M);
+          sum[k] = sum[k] * f1 + po[L.D + c0 + k] * f2;
+          acc[k] = acc[k] * f1 + po[2 * L.D + c0 + k] * f2;
+          mx[k] = M;
+        }
+      }
+    }
+  }
+  float e[4] = {0.f, 0.f, 0.f, 0.f};
+  float ss = 0.f;
+  if (lead) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) { e[k] = acc[k] / sum[k]; ss += e[k] * e[k]; }
-    ss = block_sum(ss, scratch);
-    const float rs = 1.0f / sqrtf(ss / (float)L.D + L.eps);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) e[k] *= rs * (a.gamma_kv ? a.gamma_kv[c0 + k] : 1.f);
-    rope4(e, c0, L, (double)(L.pos0 + i * (int64_t)L.m));
-    uint8_t* dst = C.entries + ((size_t)b * C.entry_cap + (size_t)i) * L.row_bytes;
-    pack_row(dst, L, c0, e, scratch);
   }
+  ss = block_sum(ss, scratch);
+  const float rs = 1.0f / sqrtf(ss / (float)L.D + L.eps);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) e[k] *= rs * (a.gamma_kv ? a.gamma_kv[c0 + k] : 1.f);
+  rope4(e, c0, L, (double)(L.pos0 + i * (int64_t)L.m));
+  uint8_t* dst = C.entries + ((size_t)b * C.entry_cap + (size_t)i) * L.row_bytes;
+  pack_row(dst, L, c0, e, lead, scratch);
 }
 
 }  // namespace
 
 cudaError_t launch_append_compress(const AppendCompressArgs& a, int B, int Tq, cudaStream_t s) {
   dim3 grid(Tq, B);
-  append_compress_kernel<<<grid, a.L.D / 4, 0, s>>>(a);
+  const int ct = a.L.D / 4;
+  // decode: spread the entry's source rows over row groups; a chunk has parallelism across tokens
+  int rg = 1;
+  if (a.do_compress && Tq <= 64) {
+    const int rows = (1 + a.L.ov) * a.L.m;
+    rg = 512 / ct;
+    while (rg > 1 && (rg / 2) * kRowBatch >= rows) rg /= 2;
+  }
+  const size_t smem = rg > 1 ? (size_t)rg * 3 * a.L.D * sizeof(float) : 0;
+  static size_t configured = 0;
+  if (smem > 48 * 1024 && smem > configured) {
+    cudaError_t e = cudaFuncSetAttribute(append_compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  append_compress_kernel<<<grid, ct * rg, smem, s>>>(a);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -36,12 +36,6 @@ constexpr int kDI = 128;                    // index-key bytes per entry
 constexpr int kTileBytes = kTileE * kDI;    // 16 KB
 constexpr int kThreads = 192;               // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 
-struct Item {
-  int b, j0, et;
-  int64_t g;
-  bool valid;
-};
-
 __device__ __forceinline__ int64_t n_visible(const IndexArgs& a, int b, int j) {
   const int64_t t = a.q_pos[(int64_t)b * a.Tq + j];
   const int64_t r1 = t - a.pos0 + 1;
@@ -49,18 +43,28 @@ __device__ __forceinline__ int64_t n_visible(const IndexArgs& a, int b, int j) {
   return nv < a.n_max ? nv : a.n_max;
 }
 
-__device__ __forceinline__ Item item_at(const IndexArgs& a, int64_t w) {
-  Item it;
-  it.g = w / a.tiles_per_group;
-  it.et = (int)(w % a.tiles_per_group);
-  it.b = (int)(it.g / a.groups_per_seq);
-  it.j0 = (int)(it.g % a.groups_per_seq) * a.QN;
-  const int j1 = min(it.j0 + a.QN, a.Tq);
+// A work item is (group g of QN queries of one sequence, entry tile et).  Tiles of a group past
+// its last visible entry are skipped; validity is monotone in et within a group.
+struct Group {
+  int64_t g;
+  int b, j0, j1;
+  int last_et;                // last tile holding a visible entry (-1: none)
+};
+
+__device__ __forceinline__ Group group_info(const IndexArgs& a, int64_t g) {
+  Group G;
+  G.g = g;
+  G.b = (int)(g / a.groups_per_seq);
+  G.j0 = (int)(g % a.groups_per_seq) * a.QN;
+  G.j1 = min(G.j0 + a.QN, a.Tq);
   int64_t nv = 0;
-  for (int j = it.j0; j < j1; ++j) nv = max(nv, n_visible(a, it.b, j));
-  it.valid = (int64_t)it.et * kTileE < nv;
-  return it;
+  for (int j = G.j0; j < G.j1; ++j) nv = max(nv, n_visible(a, G.b, j));
+  G.last_et = (int)((nv + kTileE - 1) / kTileE) - 1;
+  return G;
 }
+
+constexpr int kHistBins = 4096;               // top 12 bits of the order-preserving score key
+constexpr int kMaxQH = 256;                   // QN * H_I
 
 struct __align__(8) Barriers {
   uint64_t full[kStages], empty[kStages];
@@ -68,6 +72,15 @@ struct __align__(8) Barriers {
   uint64_t tfull[2], tempty[2];
   uint32_t tmem_base;
 };
+
+struct EpiSmem {
+  float w[kMaxQH];            // head weights of the group's queries
+  float qs[kMaxQH];           // index-query scales
+  int64_t nv[kMaxQH / 16];    // visible entries per query (QN <= 16)
+  uint32_t hist[kHistBins];   // score histogram of the current group (decode)
+};
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kThreads, 1)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
@@ -77,10 +90,12 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
   uint8_t* A = smem;                                  // [kStages][kTileBytes]
   uint8_t* Bq = A + kStages * kTileBytes;             // [2][N * 128]
   Barriers* bars = reinterpret_cast<Barriers*>(Bq + 2 * N * kDI);
+  EpiSmem* es = reinterpret_cast<EpiSmem*>(reinterpret_cast<uint8_t*>(bars) + ((sizeof(Barriers) + 15) & ~size_t(15)));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t w0 = a.total_items * blockIdx.x / gridDim.x;
   const int64_t w1 = a.total_items * (blockIdx.x + 1) / gridDim.x;
+  const int64_t tpg = a.tiles_per_group;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&bars->full[s], 1); mbar_init(&bars->empty[s], 1); }
@@ -106,30 +121,34 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       // ---------------------------------------------------------------- TMA producer
       int stage = 0;
       uint32_t phase = 0;
-      int64_t prev_g = -1;
+      Group G;
+      G.g = -1;
       int gi = -1;
       int issued_par[kStages];
       for (int s = 0; s < kStages; ++s) issued_par[s] = -1;
       int b_issued_par[2] = {-1, -1};
       bool ok = true;
       for (int64_t w = w0; w < w1 && ok; ++w) {
-        const Item it = item_at(a, w);
-        if (!it.valid) continue;
-        if (it.g != prev_g) {
-          prev_g = it.g;
+        const int64_t g = w / tpg;
+        const int et = (int)(w - g * tpg);
+        if (g != G.g) G = group_info(a, g);
+        if (et > G.last_et) continue;
+        // validity is monotone in et, so the first item of a group in this CTA is its first valid one
+        const bool first_of_group = (w == w0) || (w - 1) / tpg != g;
+        if (first_of_group) {
           ++gi;
           const int slot = gi & 1;
           const uint32_t use = (uint32_t)(gi >> 1);
           if (!mbar_wait(&bars->bempty[slot], (use & 1u) ^ 1u)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars->bfull[slot], (uint32_t)(N * kDI));
           tma_load_2d(Bq + slot * N * kDI, &qmap, &bars->bfull[slot], 0,
-                      (int)(((int64_t)it.b * a.Tq + it.j0) * a.H_I));
+                      (int)(((int64_t)G.b * a.Tq + G.j0) * a.H_I));
           b_issued_par[slot] = (int)(use & 1u);
         }
         if (!mbar_wait(&bars->empty[stage], phase ^ 1u)) { ok = false; break; }
         mbar_arrive_expect_tx(&bars->full[stage], (uint32_t)kTileBytes);
         tma_load_2d(A + stage * kTileBytes, &kmap, &bars->full[stage], 0,
-                    (int)((int64_t)it.b * a.entry_cap + (int64_t)it.et * kTileE));
+                    (int)((int64_t)G.b * a.entry_cap + (int64_t)et * kTileE));
         issued_par[stage] = (int)phase;
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
@@ -146,15 +165,18 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       const uint32_t idesc = instr_desc(128, N, 0u);
       int stage = 0, acc = 0, gi = -1;
       uint32_t phase = 0, acc_phase = 0;
-      int64_t prev_g = -1;
+      Group G;
+      G.g = -1;
       int last_acc = -1;
       uint32_t last_acc_par = 0;
       bool ok = true;
       for (int64_t w = w0; w < w1; ++w) {
-        const Item it = item_at(a, w);
-        if (!it.valid) continue;
-        if (it.g != prev_g) {
-          prev_g = it.g;
+        const int64_t g = w / tpg;
+        const int et = (int)(w - g * tpg);
+        if (g != G.g) G = group_info(a, g);
+        if (et > G.last_et) continue;
+        const bool first_of_group = (w == w0) || (w - 1) / tpg != g;
+        if (first_of_group) {
           ++gi;
           if (!mbar_wait(&bars->bfull[gi & 1], (uint32_t)((gi >> 1) & 1))) { ok = false; break; }
         }
@@ -172,11 +194,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         last_acc = acc;
         last_acc_par = acc_phase;
         // release the query tile after the group's last valid item in this CTA
-        bool last_of_group = (w + 1 >= w1);
-        if (!last_of_group) {
-          const Item nx = item_at(a, w + 1);
-          last_of_group = (nx.g != it.g) || !nx.valid;
-        }
+        const bool last_of_group = (w + 1 >= w1) || (et == G.last_et) || ((w + 1) / tpg != g);
         if (last_of_group) umma_commit(&bars->bempty[slot]);
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
@@ -187,39 +205,75 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     }
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..5)
+    // Every epilogue warp runs the same sequence of named barriers whatever happens (a wait that
+    // times out only stops the warp's work), so the 128-thread barrier can never be left short.
+    const int te = threadIdx.x - 64;           // 0..127
     const int quarter = warp & 3;              // TMEM lanes [32*quarter, 32*quarter + 32)
     const int e_loc = quarter * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const bool use_hist = a.hist != nullptr && a.QN == 1;
+    const int QH = a.QN * a.H_I;
+    if (use_hist)
+      for (int i = te; i < kHistBins; i += 128) es->hist[i] = 0u;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int64_t w = w0; w < w1; ++w) {
-      const Item it = item_at(a, w);
-      if (!it.valid) continue;
-      if (!mbar_wait(&bars->tfull[acc], acc_phase)) { ok = false; break; }
-      tc_fence_after();
-      const int64_t e = (int64_t)it.et * kTileE + e_loc;
-      const bool in_range = e < a.n_max;
-      const float ks = in_range ? __ldg(a.k_scale + (int64_t)it.b * a.entry_cap + e) : 0.f;
-      const int j1 = min(it.j0 + a.QN, a.Tq);
-      for (int j = it.j0; j < j1; ++j) {
-        const int64_t row = (int64_t)it.b * a.Tq + j;
-        const float* qs = a.q_scale + row * a.H_I;
-        const float* hw = a.head_w + row * a.H_I;
-        float s = 0.f;
-        for (int hc = 0; hc < a.H_I; hc += 16) {
-          float v[16];
-          tmem_ld_32x32b_x16(lane_addr + (uint32_t)(acc * N + (j - it.j0) * a.H_I + hc), v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < 16; ++h) s += __ldg(hw + hc + h) * fmaxf(v[h] * (__ldg(qs + hc + h) * ks), 0.f);
-        }
-        if (in_range) a.scores[row * a.n_max + e] = (e < n_visible(a, it.b, j)) ? s : -INFINITY;
+    Group G;
+    G.g = -1;
+    auto flush_hist = [&](const Group& H) {
+      const int64_t row = (int64_t)H.b * a.Tq + H.j0;
+      for (int i = te; i < kHistBins; i += 128) {
+        const uint32_t v = es->hist[i];
+        if (v) { atomicAdd(a.hist + row * kHistBins + i, v); es->hist[i] = 0u; }
       }
-      tc_fence_before();
-      mbar_arrive(&bars->tempty[acc]);
+    };
+    for (int64_t w = w0; w < w1; ++w) {
+      const int64_t g = w / tpg;
+      const int et = (int)(w - g * tpg);
+      if (g != G.g) {
+        epi_bar();
+        if (use_hist && G.g >= 0 && G.last_et >= 0) flush_hist(G);
+        G = group_info(a, g);
+        for (int i = te; i < QH; i += 128) {
+          const int j = G.j0 + i / a.H_I;
+          const int64_t row = (int64_t)G.b * a.Tq + (j < a.Tq ? j : a.Tq - 1);
+          es->w[i] = a.head_w[row * a.H_I + i % a.H_I];
+          es->qs[i] = a.q_scale[row * a.H_I + i % a.H_I];
+        }
+        if (te < a.QN) es->nv[te] = (G.j0 + te < a.Tq) ? n_visible(a, G.b, G.j0 + te) : 0;
+        epi_bar();
+      }
+      if (et > G.last_et) continue;
+      if (ok) ok = mbar_wait(&bars->tfull[acc], acc_phase);
+      if (ok) {
+        tc_fence_after();
+        const int64_t e = (int64_t)et * kTileE + e_loc;
+        const bool in_range = e < a.n_max;
+        const float ks = in_range ? __ldg(a.k_scale + (int64_t)G.b * a.entry_cap + e) : 0.f;
+        for (int j = G.j0; j < G.j1; ++j) {
+          const int q = j - G.j0;
+          const int64_t row = (int64_t)G.b * a.Tq + j;
+          const float* wq = es->w + q * a.H_I;
+          const float* sq = es->qs + q * a.H_I;
+          float s = 0.f;
+          for (int hc = 0; hc < a.H_I; hc += 16) {
+            float v[16];
+            tmem_ld_32x32b_x16(lane_addr + (uint32_t)(acc * N + q * a.H_I + hc), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < 16; ++h) s += wq[hc + h] * fmaxf(v[h] * (sq[hc + h] * ks), 0.f);
+          }
+          const bool vis = e < es->nv[q];
+          if (in_range) a.scores[row * a.n_max + e] = vis ? s : -INFINITY;
+          if (use_hist && vis) atomicAdd(&es->hist[float_key(s) >> 20], 1u);
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->tempty[acc]);
+      }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    epi_bar();
+    if (use_hist && G.g >= 0 && G.last_et >= 0) flush_hist(G);
     if (!ok) set_device_error(a.err, kErrWaitTimeout);
   }
 
@@ -319,7 +373,8 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
   if (!make_map(&qmap, a.idx_q, (uint64_t)a.B * a.Tq * a.H_I, (uint32_t)N)) return cudaErrorInvalidValue;
   uint32_t cols = 32;
   while (cols < (uint32_t)(2 * N)) cols <<= 1;
-  const size_t smem = 1024 + (size_t)kStages * kTileBytes + 2 * (size_t)N * kDI + sizeof(Barriers) + 64;
+  const size_t smem = 1024 + (size_t)kStages * kTileBytes + 2 * (size_t)N * kDI + ((sizeof(Barriers) + 15) & ~size_t(15)) +
+                     sizeof(EpiSmem) + 64;
   static size_t configured = 0;
   if (smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(index_score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -39,6 +39,7 @@ struct IndexArgs {
   const float* q_scale;     // [B][Tq][H_I]
   const float* head_w;      // [B][Tq][H_I]
   float* scores;            // [B][Tq][n_max]
+  uint32_t* hist;           // decode (Tq == 1): [B][4096] histogram of the scores' top 12 key bits, or null
   int* err;
   // tensor-core path tiling
   int QN;                   // queries per MMA N-tile (N = QN * H_I)
@@ -60,6 +61,20 @@ struct TopkArgs {
   int32_t* out;             // [rows][k]
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
+
+// Decode rows too long for one CTA: many CTAs per row, fed by the indexer's score histogram.
+struct TopkSplitArgs {
+  TopkArgs base;
+  const uint32_t* hist;     // [rows][4096] (zeroed before the indexer runs)
+  int32_t* sure;            // [rows][k] scratch
+  uint2* cand;              // [rows][n_max] scratch
+  uint32_t* cnt;            // [rows][4] counters (zeroed before the indexer runs)
+  int G;                    // CTAs per row
+};
+constexpr int64_t kTopkSplitMinN = 16384;     // rows at least this long use the split kernel
+constexpr int64_t kTopkSplitMaxN = 786432;    // the resolving CTA's bitmaps must fit shared memory
+int topk_split_ctas(int rows, int64_t n_max, int num_sms);
+cudaError_t launch_topk_split(const TopkSplitArgs& a, cudaStream_t s);
 
 // ----------------------------------------------------------------------------- attention
 struct AttendArgs {

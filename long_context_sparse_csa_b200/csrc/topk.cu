@@ -30,22 +30,44 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x, int lane) {
   return x;
 }
 
-// Exclusive block scan (blockDim.x == kThreads); *total = sum over the block.
+// Exclusive block scan (blockDim.x a multiple of 32); *total = sum over the block.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, uint32_t* total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const uint32_t inc = warp_incl_scan(v, lane);
   if (lane == 31) wsum[wid] = inc;
   __syncthreads();
   if (wid == 0) {
-    uint32_t x = wsum[lane];
+    uint32_t x = lane < nwarps ? wsum[lane] : 0u;
     x = warp_incl_scan(x, lane);
     wsum[lane] = x;
   }
   __syncthreads();
   const uint32_t before = wid > 0 ? wsum[wid - 1] : 0u;
-  *total = wsum[31];
+  *total = wsum[nwarps - 1];
   __syncthreads();
   return before + inc - v;
+}
+
+// Among the bins nb-1 .. 0 (descending), the bin b with above(b) < need <= above(b) + hist[b],
+// where above(b) counts the bins above b.  Every thread gets (bin, above).
+__device__ __forceinline__ void find_bin(const uint32_t* hist, int nb, uint32_t need, uint32_t* wsum,
+                                         uint32_t* s_bin, uint32_t* s_above) {
+  const int per = (nb + blockDim.x - 1) / blockDim.x;
+  uint32_t c_local = 0;
+  for (int q = 0; q < per; ++q) {
+    const int bin = nb - 1 - per * (int)threadIdx.x - q;
+    if (bin >= 0) c_local += hist[bin];
+  }
+  uint32_t tot;
+  uint32_t above = block_excl_scan(c_local, wsum, &tot);
+  for (int q = 0; q < per; ++q) {
+    const int bin = nb - 1 - per * (int)threadIdx.x - q;
+    if (bin < 0) break;
+    const uint32_t h = hist[bin];
+    if (above < need && need <= above + h) { *s_bin = (uint32_t)bin; *s_above = above; }
+    above += h;
+  }
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kThreads, 1) topk_rows_kernel(const __grid_constant__ TopkArgs a, int use_smem) {
@@ -90,19 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_rows_kernel(const __grid_con
       if (fixed == 0 || (k >> (32 - fixed)) == prefix) atomicAdd(&hist[(k >> shift) & (nb - 1)], 1u);
     }
     __syncthreads();
-    // suffix counts: thread t owns the bins (nb-1 - per*t - q), q < per, in descending order
-    const int per = nb / kThreads;             // 2 or 1
-    uint32_t c_local = 0;
-    for (int q = 0; q < per; ++q) c_local += hist[nb - 1 - per * tid - q];
-    uint32_t tot;
-    uint32_t above = block_excl_scan(c_local, wsum, &tot);
-    for (int q = 0; q < per; ++q) {
-      const int bin = nb - 1 - per * tid - q;
-      const uint32_t h = hist[bin];
-      if (above < remaining && remaining <= above + h) { sel_bin = (uint32_t)bin; sel_above = above; }
-      above += h;
-    }
-    __syncthreads();
+    find_bin(hist, nb, remaining, wsum, &sel_bin, &sel_above);
     remaining -= sel_above;
     prefix = (prefix << wbits) | sel_bin;
     fixed += wbits;
@@ -133,7 +143,168 @@ __global__ void __launch_bounds__(kThreads, 1) topk_rows_kernel(const __grid_con
   }
 }
 
+
+// ----------------------------------------------------------------------------- split mode (long decode rows)
+// Many CTAs per row.  The indexer epilogue has already histogrammed the top 12 key bits of the
+// row's visible scores; every CTA finds the bin b* that holds the k-th largest key, then streams
+// its slice of the row: keys above b* are certainly selected (appended to `sure`), keys in b* are
+// candidates (appended to `cand`).  The last CTA of the row to finish (a ticket counter, no
+// waiting) resolves the candidates with two 10-bit radix passes, marks the selection in a
+// shared-memory bitmap over the row's indices, and emits it in ascending index order.
+constexpr int kSplitThreads = 512;
+constexpr int kHistBins = 4096;
+
+__global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __grid_constant__ TopkSplitArgs a) {
+  extern __shared__ uint32_t bm[];              // last CTA: sel[nw] | eq[nw]
+  __shared__ uint32_t h2[1024];
+  __shared__ uint32_t wsum[32];
+  __shared__ uint32_t s_bin, s_above, s_last;
+  const TopkArgs& A = a.base;
+  const int row = blockIdx.y, g = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+  const int64_t t = A.q_pos[row];
+  const int64_t r1 = t - A.pos0 + 1;
+  int64_t nv64 = r1 > 0 ? r1 / A.m : 0;
+  if (nv64 > A.n_max) nv64 = A.n_max;
+  const int nv = (int)nv64;
+  const int k = A.k;
+  int32_t* out = A.out + (size_t)row * k;
+  if (nv <= k) {
+    if (g == 0)
+      for (int i = tid; i < k; i += kSplitThreads) out[i] = i < nv ? i : -1;
+    return;
+  }
+  uint32_t* cnt = a.cnt + (size_t)row * 4;
+  int32_t* sure = a.sure + (size_t)row * k;
+  uint2* cand = a.cand + (size_t)row * A.n_max;
+
+  // ---------------------------------------------------------------- 1. bin of the k-th largest key
+  find_bin(a.hist + (size_t)row * kHistBins, kHistBins, (uint32_t)k, wsum, &s_bin, &s_above);
+  const uint32_t bstar = s_bin;
+
+  // ---------------------------------------------------------------- 2. filter this CTA's slice
+  const int lo = (int)((int64_t)nv * g / gridDim.x), hi = (int)((int64_t)nv * (g + 1) / gridDim.x);
+  const float* sc = A.scores + (size_t)row * A.n_max;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int base = lo; base < hi; base += kSplitThreads) {
+    const int i = base + tid;
+    uint32_t key = 0, bin = 0;
+    const bool in = i < hi;
+    if (in) { key = float_key(__ldg(sc + i)); bin = key >> 20; }
+    const bool is_sure = in && bin > bstar, is_cand = in && bin == bstar;
+    const uint32_t ms = __ballot_sync(0xffffffffu, is_sure), mc = __ballot_sync(0xffffffffu, is_cand);
+    uint32_t ps = 0, pc = 0;
+    if (lane == 0) {
+      if (ms) ps = atomicAdd(cnt + 0, (uint32_t)__popc(ms));
+      if (mc) pc = atomicAdd(cnt + 1, (uint32_t)__popc(mc));
+    }
+    ps = __shfl_sync(0xffffffffu, ps, 0);
+    pc = __shfl_sync(0xffffffffu, pc, 0);
+    if (is_sure) sure[ps + __popc(ms & lt_mask)] = i;
+    if (is_cand) cand[pc + __popc(mc & lt_mask)] = make_uint2(key, (uint32_t)i);
+  }
+
+  // ---------------------------------------------------------------- 3. last CTA of the row resolves
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    s_last = atomicAdd(cnt + 2, 1u) == gridDim.x - 1 ? 1u : 0u;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const uint32_t n_sure = atomicAdd(cnt + 0, 0u), nc = atomicAdd(cnt + 1, 0u);
+  uint32_t rem = (uint32_t)k - n_sure;        // >= 1: fewer than k keys lie above b*
+
+  // two 10-bit radix passes over the candidates' low 20 bits pin the exact key T
+  uint32_t prefix = bstar;
+  int fixed = 12;
+  for (int pass = 0; pass < 2; ++pass) {
+    const int shift = 32 - fixed - 10;
+    for (int i = tid; i < 1024; i += kSplitThreads) h2[i] = 0u;
+    __syncthreads();
+    for (uint32_t j = tid; j < nc; j += kSplitThreads) {
+      const uint32_t key = cand[j].x;
+      if ((key >> (32 - fixed)) == prefix) atomicAdd(&h2[(key >> shift) & 1023u], 1u);
+    }
+    __syncthreads();
+    find_bin(h2, 1024, rem, wsum, &s_bin, &s_above);
+    rem -= s_above;
+    prefix = (prefix << 10) | s_bin;
+    fixed += 10;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;                   // keys > T are taken; `rem` keys == T, smallest indices
+
+  const int nw = (nv + 31) >> 5;
+  uint32_t* sel = bm;
+  uint32_t* eqm = bm + nw;
+  for (int i = tid; i < 2 * nw; i += kSplitThreads) bm[i] = 0u;
+  __syncthreads();
+  for (uint32_t j = tid; j < n_sure; j += kSplitThreads) {
+    const uint32_t i = (uint32_t)sure[j];
+    atomicOr(&sel[i >> 5], 1u << (i & 31));
+  }
+  for (uint32_t j = tid; j < nc; j += kSplitThreads) {
+    const uint2 c = cand[j];
+    if (c.x > T) atomicOr(&sel[c.y >> 5], 1u << (c.y & 31));
+    else if (c.x == T) atomicOr(&eqm[c.y >> 5], 1u << (c.y & 31));
+  }
+  __syncthreads();
+
+  // ordered emission: thread t owns words [t*wpt, (t+1)*wpt)
+  const int wpt = (nw + kSplitThreads - 1) / kSplitThreads;
+  const int w_lo = min(tid * wpt, nw), w_hi = min(w_lo + wpt, nw);
+  uint32_t eq_local = 0;
+  for (int wd = w_lo; wd < w_hi; ++wd) eq_local += __popc(eqm[wd]);
+  uint32_t tot;
+  uint32_t eq_before = block_excl_scan(eq_local, wsum, &tot);
+  uint32_t n_local = 0;
+  for (int wd = w_lo; wd < w_hi; ++wd) {
+    uint32_t e = eqm[wd], keep = 0;
+    while (e && eq_before < rem) {
+      const uint32_t low = e & (0u - e);
+      keep |= low;
+      e ^= low;
+      ++eq_before;
+    }
+    eq_before += __popc(e);
+    sel[wd] |= keep;
+    n_local += __popc(sel[wd]);
+  }
+  uint32_t pos = block_excl_scan(n_local, wsum, &tot);
+  for (int wd = w_lo; wd < w_hi; ++wd) {
+    uint32_t b = sel[wd];
+    while (b) {
+      const int bit = __ffs(b) - 1;
+      b &= b - 1;
+      out[pos++] = wd * 32 + bit;
+    }
+  }
+}
+
 }  // namespace
+
+int topk_split_ctas(int rows, int64_t n_max, int num_sms) {
+  int64_t g = (2 * (int64_t)num_sms + rows - 1) / rows;
+  const int64_t by_size = (n_max + 4095) / 4096;
+  if (g > by_size) g = by_size;
+  if (g < 1) g = 1;
+  return (int)g;
+}
+
+cudaError_t launch_topk_split(const TopkSplitArgs& a, cudaStream_t s) {
+  if (a.base.rows <= 0 || a.base.k <= 0) return cudaSuccess;
+  const size_t smem = 2 * (size_t)((a.base.n_max + 31) / 32) * 4;
+  static size_t configured = 0;
+  if (smem > 48 * 1024 && smem > configured) {
+    cudaError_t e = cudaFuncSetAttribute(topk_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  topk_split_kernel<<<dim3(a.G, a.base.rows), kSplitThreads, smem, s>>>(a);
+  note_launches(1);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   if (a.rows <= 0 || a.k <= 0) return cudaSuccess;

@@ -138,9 +138,11 @@ def test_index_topk_parity(name, n):
         check_topk(got_k[b], ref, layer.top_k)
 
 
-def test_topk_ties_go_to_smaller_index():
+@pytest.mark.parametrize("n", [9000, 160000])
+def test_topk_ties_go_to_smaller_index(n):
     # identical index keys: every visible entry scores the same -> the k smallest indices
-    wl = get_workload("csa_decode_128k", B=2, n=9000)
+    # (n = 160000: 40,000 entries, the multi-CTA path with every candidate tied at the k-th key)
+    wl = get_workload("csa_decode_128k", B=2, n=n)
     d, layer, st = _index_case(wl)
     d["idx_k"][:] = d["idx_k"][:, :1]
     d["idx_k_scale"][:] = d["idx_k_scale"][:, :1]
@@ -152,6 +154,26 @@ def test_topk_ties_go_to_smaller_index():
                      cap, topk, None, ws)
     got = host(topk)
     assert np.array_equal(got, np.tile(np.arange(layer.top_k), (2, 1)))
+
+
+def test_topk_long_row_with_duplicated_keys():
+    # blocks of 7 identical keys: many exact ties around the k-th score in a multi-CTA row
+    wl = get_workload("csa_decode_128k", B=2, n=4 * 70001)
+    d, layer, st = _index_case(wl)
+    d["idx_k"][:] = np.repeat(d["idx_k"][:, ::7], 7, axis=1)[:, :d["idx_k"].shape[1]]
+    d["idx_k_scale"][:] = np.repeat(d["idx_k_scale"][:, ::7], 7, axis=1)[:, :d["idx_k"].shape[1]]
+    st = LayerState.from_arrays(layer, wl.B, d)
+    cap = d["entries"].shape[1]
+    topk = torch.zeros((2, layer.top_k), dtype=torch.int32, device="cuda")
+    ws = st.workspace("index_topk", 1, cap)
+    C.csa_index_topk(st.L, st.cache(), dev(d["idx_q"]), dev(d["idx_q_scale"]), dev(d["head_w"]), dev(d["t"]), 1,
+                     cap, topk, None, ws)
+    got = host(topk)
+    for b in range(2):
+        iq = F.decode_idx(d["idx_q"][b], layer.idx_format)
+        ref = O.index_scores(iq, d["idx_q_scale"][b], d["head_w"][b], F.decode_idx(d["idx_k"][b], "e4m3"),
+                             d["idx_k_scale"][b])
+        check_topk(got[b], ref, layer.top_k)
 
 
 def test_topk_fewer_visible_than_k_pads():
