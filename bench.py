@@ -397,6 +397,47 @@ def run_ours(args):
     idx_ms = [e["idx"][0].elapsed_time(e["idx"][1]) for e in cycle_ev] if has_csa else []
     lay_ms = [[e["lay"][li][0].elapsed_time(e["lay"][li][1]) for e in cycle_ev] for li in range(len(layers))]
 
+    # ------------------------------------------------------------------ per-kernel timeline (diagnostic, untimed)
+    labels = {"csa": ["append+compress", "histogram reset", "indexer scores", "top-k", "attention", "combine"],
+              "hca": ["append+compress", "attention", "combine"]}
+    tl_events = []
+    g_tl = torch.cuda.CUDAGraph()
+    for lay in layers:
+        evs = [ev() for _ in range(17)]
+        for x in evs:
+            x.record()
+        tl_events.append(evs)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g_tl, stream=stream):
+        for li, lay in enumerate(layers):
+            io, spec = lay["io"], lay["spec"]
+            evs = tl_events[li]
+            C.csa_profile_timeline(evs[:16])
+            if spec.kind == "csa":
+                C.csa_decode_step(lay["L"], lay["caches"][0], lay["params"], io["q"], io["idx_q"], io["idx_q_scale"],
+                                  io["head_w"], io["x_new"], io["g_new"], io["t"], io["out"], io["topk"], lay["ws"])
+            else:
+                C.hca_decode_step(lay["L"], lay["caches"][0], lay["params"], io["q"], io["x_new"], io["g_new"],
+                                  io["t"], io["out"], lay["ws"])
+            lay["tl_n"] = C.csa_profile_timeline_count()
+            C.csa_profile_timeline(None)
+            evs[lay["tl_n"]].record()
+    timeline = {}
+    reps = []
+    for rep in range(5):
+        for r in range(1, R):          # touch the other instances so instance 0 is cold in L2
+            singles[r].replay()
+        g_tl.replay()
+        torch.cuda.synchronize()
+        reps.append([[tl_events[li][i].elapsed_time(tl_events[li][i + 1]) * 1e3 for i in range(lay["tl_n"])]
+                     for li, lay in enumerate(layers)])
+    for li, lay in enumerate(layers):
+        med = np.median(np.array([r[li] for r in reps]), axis=0)
+        names = labels[lay["spec"].kind] if len(labels[lay["spec"].kind]) == lay["tl_n"] else \
+            [f"launch{i}" for i in range(lay["tl_n"])]
+        timeline[f"{lay['spec'].kind}{li}"] = {n: round(float(v), 2) for n, v in zip(names, med)}
+    del g_tl
+
     # ------------------------------------------------------------------ end to end through host memory
     h2d, d2h = [], []
     for lay in layers:
@@ -474,6 +515,7 @@ def run_ours(args):
     line["e2e"] = {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                    "ms_per_step": E_ms / args.steps}
     line["gpu_launches"] = int(launches_per_step) * args.steps
+    line["timeline_us"] = timeline
     line["clocks"] = clk
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

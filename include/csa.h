@@ -170,6 +170,16 @@ CSA_API csa_status_t csa_device_error(void* workspace, size_t ws_bytes, void* st
  * turns it off.  Host only; never fails. */
 CSA_API void csa_profile_events(void* ev_start, void* ev_stop);
 
+/* Profiling aid (no counterpart on the pages).  Arms a timeline on this host thread: later
+ * calls record events[0], events[1], ... (cudaEvent_t handles with timing enabled), one just
+ * before each kernel launch or memset they issue, until `capacity` events are used; the records
+ * use the external flag, so they become event nodes under stream capture.  The caller records
+ * one more event after the last call to close the last interval.  NULL disarms it. */
+CSA_API void csa_profile_timeline(void** events, int32_t capacity);
+
+/* Events of the armed timeline used so far. */
+CSA_API int32_t csa_profile_timeline_count(void);
+
 /* Number of kernels this process has launched through the library so far (host counter). */
 CSA_API uint64_t csa_launch_count(void);
 

@@ -62,6 +62,8 @@ _SIGS = {
     "csa_version": (ctypes.c_char_p, []),
     "csa_profile_events": (None, [_P, _P]),
     "csa_launch_count": (ctypes.c_uint64, []),
+    "csa_profile_timeline": (None, [_P, _I32]),
+    "csa_profile_timeline_count": (_I32, []),
     "csa_device_error": (ctypes.c_int, [_P, _SZ, _P, ctypes.POINTER(_I32)]),
     "csa_append": (ctypes.c_int, [_LAYER, _CACHE, _P, _P, _P, _I32, _P]),
     "csa_compress": (ctypes.c_int, [_LAYER, _CACHE, _PARAMS, _P, _I32, _P]),
@@ -157,6 +159,26 @@ def csa_profile_events(ev_start, ev_stop):
         h.csa_profile_events(None, None)
     else:
         h.csa_profile_events(ctypes.c_void_p(ev_start.cuda_event), ctypes.c_void_p(ev_stop.cuda_event))
+
+
+_timeline_keep = None
+
+
+def csa_profile_timeline(events):
+    """Arm a timeline of torch.cuda.Events (recorded before each later launch); None disarms."""
+    global _timeline_keep
+    h = lib()
+    if not events:
+        h.csa_profile_timeline(None, 0)
+        _timeline_keep = None
+        return
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    _timeline_keep = arr
+    h.csa_profile_timeline(ctypes.cast(arr, ctypes.c_void_p), len(events))
+
+
+def csa_profile_timeline_count() -> int:
+    return lib().csa_profile_timeline_count()
 
 
 def csa_launch_count() -> int:

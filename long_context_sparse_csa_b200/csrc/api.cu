@@ -1,5 +1,6 @@
 // C ABI of the CSA/HCA operator: argument checks, workspace layout, launches.
 #include <atomic>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -14,6 +15,8 @@ namespace {
 
 thread_local std::string g_err;
 thread_local cudaEvent_t g_prof_start = nullptr, g_prof_stop = nullptr;
+thread_local cudaEvent_t* g_tl = nullptr;
+thread_local int g_tl_cap = 0, g_tl_n = 0;
 std::atomic<uint64_t> g_launches{0};
 
 csa_status_t fail(csa_status_t st, const char* fmt, ...) {
@@ -88,6 +91,8 @@ LayerArgs layer_args(const csa_layer_t* L) {
   a.eps = L->eps;
   a.scale = L->softmax_scale > 0 ? L->softmax_scale : 1.0f / sqrtf((float)L->D);
   a.pos0 = L->pos0;
+  for (int u = 0; u < 32; ++u)
+    a.theta_pi[u] = u < L->d_rope / 2 ? std::pow(L->rope_base, -2.0 * u / (double)L->d_rope) / M_PI : 0.0;
   return a;
 }
 
@@ -219,6 +224,7 @@ csa_status_t run_index_topk(const csa_layer_t* L, const csa_cache_t* cache, cons
   const int rows = L->B * Tq;
   uint32_t* hist = split ? reinterpret_cast<uint32_t*>(at(ws, w.hist)) : nullptr;
   if (split) {
+    profile_mark(s);
     cudaError_t e = cudaMemsetAsync(hist, 0, w.hist_bytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "histogram reset");
   }
@@ -297,6 +303,9 @@ csa_status_t check_params(const csa_layer_t* L, const csa_params_t* P, bool need
 
 namespace csa {
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+void profile_mark(cudaStream_t s) {
+  if (g_tl && g_tl_n < g_tl_cap) cudaEventRecordWithFlags(g_tl[g_tl_n++], s, cudaEventRecordExternal);
+}
 }  // namespace csa
 
 // ============================================================================= exported
@@ -319,6 +328,14 @@ void csa_profile_events(void* ev_start, void* ev_stop) {
 }
 
 uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void csa_profile_timeline(void** events, int32_t capacity) {
+  g_tl = reinterpret_cast<cudaEvent_t*>(events);
+  g_tl_cap = events ? capacity : 0;
+  g_tl_n = 0;
+}
+
+int32_t csa_profile_timeline_count(void) { return g_tl_n; }
 
 csa_status_t csa_device_error(void* workspace, size_t ws_bytes, void* stream, int32_t* code) {
   if (!workspace || ws_bytes < 4) return fail(CSA_ERR_WORKSPACE, "workspace is NULL");

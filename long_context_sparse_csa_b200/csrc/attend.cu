@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
 
   if (tid < 32) {
     float c, s;
-    rope_cos_sin((double)t, tid, 64, L.rope_base, &c, &s);
+    rope_cos_sin((double)t, tid, L, &c, &s);
     cs[tid] = c;
     sn[tid] = s;
   }
@@ -399,29 +399,46 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
     }
 }
 
-// Merge the splits of one (query, head): sink, normalisation, inverse rotation.
+// Merge the splits of one (query, head): sink, normalisation, inverse rotation.  The split
+// maxima and sums are staged in shared memory first, so every partial-output load of the
+// weighted sum is independent and can be in flight together.
 template <int HG>
 __global__ void attend_combine_kernel(const __grid_constant__ AttendArgs a) {
+  __shared__ float fac[1024];
+  __shared__ float s_inv;
   const LayerArgs& L = a.L;
   const int h = blockIdx.x, row = blockIdx.y;
   const int hg = h / HG, hl = h % HG;
-  const float* base = a.part + ((size_t)row * (L.H / HG) + hg) * a.splits * (size_t)(HG * (kD + 2));
   const size_t pstride = (size_t)HG * (kD + 2);
+  const float* base = a.part + ((size_t)row * (L.H / HG) + hg) * a.splits * pstride;
   const float sk = a.sinks[h] * kLog2e;
-  float M = sk;
-  for (int s = 0; s < a.splits; ++s) M = fmaxf(M, base[s * pstride + HG * kD + hl]);
-  float den = exp2f(sk - M);
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const int S = a.splits;
+  for (int s = threadIdx.x; s < S; s += blockDim.x) fac[s] = base[s * pstride + HG * kD + hl];
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float M = sk;
+    for (int s = threadIdx.x; s < S; s += 32) M = fmaxf(M, fac[s]);
+    M = warp_max(M);
+    float den = 0.f;
+    for (int s = threadIdx.x; s < S; s += 32) {
+      const float f = exp2f(fac[s] - M);
+      den += base[s * pstride + HG * kD + HG + hl] * f;
+      fac[s] = f;
+    }
+    den = warp_sum(den) + exp2f(sk - M);
+    if (threadIdx.x == 0) s_inv = 1.f / den;
+  }
+  __syncthreads();
   const int d0 = threadIdx.x * 4;
-  for (int s = 0; s < a.splits; ++s) {
-    const float* p = base + s * pstride;
-    const float ms = p[HG * kD + hl];
-    const float f = exp2f(ms - M);
-    den += p[HG * kD + HG + hl] * f;
-    const float4 v = *reinterpret_cast<const float4*>(p + (size_t)hl * kD + d0);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const float* p = base + (size_t)hl * kD + d0;
+#pragma unroll 8
+  for (int s = 0; s < S; ++s) {
+    const float4 v = *reinterpret_cast<const float4*>(p + s * pstride);
+    const float f = fac[s];
     acc[0] += v.x * f; acc[1] += v.y * f; acc[2] += v.z * f; acc[3] += v.w * f;
   }
-  const float inv = 1.f / den;
+  const float inv = s_inv;
 #pragma unroll
   for (int k = 0; k < 4; ++k) acc[k] *= inv;
   if (d0 >= kD - 64) {
@@ -429,7 +446,7 @@ __global__ void attend_combine_kernel(const __grid_constant__ AttendArgs a) {
 #pragma unroll
     for (int k = 0; k < 4; k += 2) {
       float c, s;
-      rope_cos_sin(-(double)t, (d0 + k - (kD - 64)) >> 1, 64, L.rope_base, &c, &s);
+      rope_cos_sin(-(double)t, (d0 + k - (kD - 64)) >> 1, L, &c, &s);
       const float x0 = acc[k], x1 = acc[k + 1];
       acc[k] = x0 * c - x1 * s;
       acc[k + 1] = x0 * s + x1 * c;
@@ -465,7 +482,7 @@ __global__ void attend_generic_kernel(const __grid_constant__ AttendArgs a) {
     const int d = lane * dpl + k;
     if (d >= dn) {
       float c, s;
-      rope_cos_sin((double)t, (d - dn) >> 1, L.d_rope, L.rope_base, &c, &s);
+      rope_cos_sin((double)t, (d - dn) >> 1, L, &c, &s);
       const float x0 = q[k], x1 = q[k + 1];
       q[k] = x0 * c - x1 * s;
       q[k + 1] = x0 * s + x1 * c;
@@ -508,7 +525,7 @@ __global__ void attend_generic_kernel(const __grid_constant__ AttendArgs a) {
     const int d = lane * dpl + k;
     if (d >= dn) {
       float c, s;
-      rope_cos_sin(-(double)t, (d - dn) >> 1, L.d_rope, L.rope_base, &c, &s);
+      rope_cos_sin(-(double)t, (d - dn) >> 1, L, &c, &s);
       const float x0 = o[k], x1 = o[k + 1];
       o[k] = x0 * c - x1 * s;
       o[k + 1] = x0 * s + x1 * c;
@@ -539,10 +556,12 @@ cudaError_t launch_mma(const AttendArgs& a, cudaStream_t s) {
     configured = true;
   }
   dim3 grid(a.splits, a.L.H / HG, a.rows);
+  profile_mark(s);
   attend_mma_kernel<HG, FMT><<<grid, HG * 8, smem, s>>>(a);
   note_launches(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || a.splits == 1) return e;
+  profile_mark(s);
   attend_combine_kernel<HG><<<dim3(a.L.H, a.rows), kD / 4, 0, s>>>(a);
   note_launches(1);
   return cudaGetLastError();
@@ -579,6 +598,7 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
   if (a.rows <= 0) return cudaSuccess;
   const int HG = attend_head_group(a.L);
   if (HG == 0) {
+    profile_mark(s);
     attend_generic_kernel<<<a.rows, a.L.H * 32, 0, s>>>(a);
     note_launches(1);
     return cudaGetLastError();

@@ -21,6 +21,7 @@ struct LayerArgs {
   double rope_base;
   float eps, scale;
   int64_t pos0;
+  double theta_pi[32];   // base^(-2u/d_rope) / pi, u < d_rope/2, formed on the host in float64
 };
 
 struct CacheArgs {
@@ -65,12 +66,11 @@ __device__ __forceinline__ float pow2_scale(float amax, float* inv) {
   return ldexpf(1.f, k);
 }
 
-// Rotary angle of pair u at position pos, reduced in float64, returned as float cos/sin.
-__device__ __forceinline__ void rope_cos_sin(double pos, int u, int d_rope, double base,
-                                             float* c, float* s) {
-  double theta = pow(base, -2.0 * (double)u / (double)d_rope);
+// Rotary angle of pair u at position pos, formed in float64 as pos * theta_u; taken as
+// sincospi(pos * theta_u / pi), whose argument reduction (modulo 2) is exact.  Returns float cos/sin.
+__device__ __forceinline__ void rope_cos_sin(double pos, int u, const LayerArgs& L, float* c, float* s) {
   double sd, cd;
-  sincos(pos * theta, &sd, &cd);
+  sincospi(pos * L.theta_pi[u], &sd, &cd);
   *c = (float)cd;
   *s = (float)sd;
 }

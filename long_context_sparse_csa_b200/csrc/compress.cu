@@ -24,10 +24,10 @@ __device__ __forceinline__ void rope4(float v[4], int c0, const LayerArgs& L, do
   if (c0 < dn) return;
   const int u = (c0 - dn) >> 1;
   float c, s, a, b;
-  rope_cos_sin(pos, u, L.d_rope, L.rope_base, &c, &s);
+  rope_cos_sin(pos, u, L, &c, &s);
   a = v[0]; b = v[1];
   v[0] = a * c - b * s; v[1] = a * s + b * c;
-  rope_cos_sin(pos, u + 1, L.d_rope, L.rope_base, &c, &s);
+  rope_cos_sin(pos, u + 1, L, &c, &s);
   a = v[2]; b = v[3];
   v[2] = a * c - b * s; v[3] = a * s + b * c;
 }
@@ -212,6 +212,7 @@ cudaError_t launch_append_compress(const AppendCompressArgs& a, int B, int Tq, c
     if (e != cudaSuccess) return e;
     configured = smem;
   }
+  profile_mark(s);
   append_compress_kernel<<<grid, ct * rg, smem, s>>>(a);
   note_launches(1);
   return cudaGetLastError();

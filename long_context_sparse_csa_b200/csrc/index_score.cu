@@ -66,10 +66,12 @@ __device__ __forceinline__ Group group_info(const IndexArgs& a, int64_t g) {
 constexpr int kHistBins = 4096;               // top 12 bits of the order-preserving score key
 constexpr int kMaxQH = 256;                   // QN * H_I
 
+constexpr int kMaxAcc = 4;                    // TMEM accumulators (decode: 4 x N columns; N = 256: 2)
+
 struct __align__(8) Barriers {
   uint64_t full[kStages], empty[kStages];
   uint64_t bfull[2], bempty[2];
-  uint64_t tfull[2], tempty[2];
+  uint64_t tfull[kMaxAcc], tempty[kMaxAcc];
   uint32_t tmem_base;
 };
 
@@ -84,7 +86,7 @@ __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: 
 
 __global__ void __launch_bounds__(kThreads, 1)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
-                      const __grid_constant__ IndexArgs a, int N, uint32_t tmem_cols) {
+                      const __grid_constant__ IndexArgs a, int N, int nacc, uint32_t tmem_cols) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* A = smem;                                  // [kStages][kTileBytes]
@@ -99,10 +101,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&bars->full[s], 1); mbar_init(&bars->empty[s], 1); }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars->bfull[s], 1); mbar_init(&bars->bempty[s], 1);
-      mbar_init(&bars->tfull[s], 1); mbar_init(&bars->tempty[s], 128);
-    }
+    for (int s = 0; s < 2; ++s) { mbar_init(&bars->bfull[s], 1); mbar_init(&bars->bempty[s], 1); }
+    for (int s = 0; s < kMaxAcc; ++s) { mbar_init(&bars->tfull[s], 1); mbar_init(&bars->tempty[s], 128); }
     fence_barrier_init();
     prefetch_tensormap(&kmap);
     prefetch_tensormap(&qmap);
@@ -197,7 +197,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         const bool last_of_group = (w + 1 >= w1) || (et == G.last_et) || ((w + 1) / tpg != g);
         if (last_of_group) umma_commit(&bars->bempty[slot]);
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (++acc == nacc) { acc = 0; acc_phase ^= 1u; }
       }
       if (!ok) set_device_error(a.err, kErrWaitTimeout);
       // the accumulator must be idle before TMEM is released
@@ -220,6 +220,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     bool ok = true;
     Group G;
     G.g = -1;
+    float ks_next = 0.f;
+    int64_t ks_w = -1;
     auto flush_hist = [&](const Group& H) {
       const int64_t row = (int64_t)H.b * a.Tq + H.j0;
       for (int i = te; i < kHistBins; i += 128) {
@@ -244,33 +246,47 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         epi_bar();
       }
       if (et > G.last_et) continue;
+      const int64_t e = (int64_t)et * kTileE + e_loc;
+      const bool in_range = e < a.n_max;
+      // this tile's key scale was prefetched by the previous iteration when it was the same group's
+      float ks;
+      if (ks_w == w) ks = ks_next;
+      else ks = in_range ? __ldg(a.k_scale + (int64_t)G.b * a.entry_cap + e) : 0.f;
+      if (et + 1 <= G.last_et && w + 1 < w1) {
+        const int64_t e2 = e + kTileE;
+        ks_next = e2 < a.n_max ? __ldg(a.k_scale + (int64_t)G.b * a.entry_cap + e2) : 0.f;
+        ks_w = w + 1;
+      }
       if (ok) ok = mbar_wait(&bars->tfull[acc], acc_phase);
       if (ok) {
         tc_fence_after();
-        const int64_t e = (int64_t)et * kTileE + e_loc;
-        const bool in_range = e < a.n_max;
-        const float ks = in_range ? __ldg(a.k_scale + (int64_t)G.b * a.entry_cap + e) : 0.f;
         for (int j = G.j0; j < G.j1; ++j) {
           const int q = j - G.j0;
           const int64_t row = (int64_t)G.b * a.Tq + j;
           const float* wq = es->w + q * a.H_I;
           const float* sq = es->qs + q * a.H_I;
           float s = 0.f;
-          for (int hc = 0; hc < a.H_I; hc += 16) {
-            float v[16];
+          for (int hc = 0; hc < a.H_I; hc += 32) {
+            float v[32];
             tmem_ld_32x32b_x16(lane_addr + (uint32_t)(acc * N + q * a.H_I + hc), v);
+            if (hc + 16 < a.H_I) tmem_ld_32x32b_x16(lane_addr + (uint32_t)(acc * N + q * a.H_I + hc + 16), v + 16);
             tmem_wait_ld();
+            if (j + 1 == G.j1 && hc + 32 >= a.H_I) {
+              // every column of this accumulator is in registers: hand it back to the MMA warp
+              tc_fence_before();
+              mbar_arrive(&bars->tempty[acc]);
+            }
+            const int nh = min(32, a.H_I - hc);
 #pragma unroll
-            for (int h = 0; h < 16; ++h) s += wq[hc + h] * fmaxf(v[h] * (sq[hc + h] * ks), 0.f);
+            for (int h = 0; h < 32; ++h)
+              if (h < nh) s += wq[hc + h] * fmaxf(v[h] * (sq[hc + h] * ks), 0.f);
           }
           const bool vis = e < es->nv[q];
           if (in_range) a.scores[row * a.n_max + e] = vis ? s : -INFINITY;
           if (use_hist && vis) atomicAdd(&es->hist[float_key(s) >> 20], 1u);
         }
-        tc_fence_before();
-        mbar_arrive(&bars->tempty[acc]);
       }
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (++acc == nacc) { acc = 0; acc_phase ^= 1u; }
     }
     epi_bar();
     if (use_hist && G.g >= 0 && G.last_et >= 0) flush_hist(G);
@@ -359,6 +375,7 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
                                            (int)sm);
       if (e != cudaSuccess) return e;
     }
+    profile_mark(s);
     index_score_generic_kernel<<<grid, 128, sm, s>>>(a);
     note_launches(1);
     return cudaGetLastError();
@@ -371,8 +388,9 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
   CUtensorMap kmap, qmap;
   if (!make_map(&kmap, a.idx_k, (uint64_t)a.B * a.entry_cap, kTileE)) return cudaErrorInvalidValue;
   if (!make_map(&qmap, a.idx_q, (uint64_t)a.B * a.Tq * a.H_I, (uint32_t)N)) return cudaErrorInvalidValue;
+  const int nacc = N <= 128 ? 4 : 2;
   uint32_t cols = 32;
-  while (cols < (uint32_t)(2 * N)) cols <<= 1;
+  while (cols < (uint32_t)(nacc * N)) cols <<= 1;
   const size_t smem = 1024 + (size_t)kStages * kTileBytes + 2 * (size_t)N * kDI + ((sizeof(Barriers) + 15) & ~size_t(15)) +
                      sizeof(EpiSmem) + 64;
   static size_t configured = 0;
@@ -383,7 +401,8 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
     configured = smem;
   }
   const int64_t grid = a.total_items < num_sms ? a.total_items : num_sms;
-  index_score_tc_kernel<<<(unsigned)grid, kThreads, smem, s>>>(kmap, qmap, a, N, cols);
+  profile_mark(s);
+  index_score_tc_kernel<<<(unsigned)grid, kThreads, smem, s>>>(kmap, qmap, a, N, nacc, cols);
   note_launches(1);
   return cudaGetLastError();
 }

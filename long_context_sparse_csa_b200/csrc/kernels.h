@@ -11,6 +11,8 @@ namespace csa {
 
 // Host-side count of kernel launches issued by the library (for launch accounting).
 void note_launches(int n);
+// Records the next timeline event (if a timeline is armed on this thread) just before a launch.
+void profile_mark(cudaStream_t s);
 
 // ----------------------------------------------------------------------------- append + compress
 struct AppendCompressArgs {

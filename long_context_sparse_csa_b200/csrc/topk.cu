@@ -153,12 +153,13 @@ __global__ void __launch_bounds__(kThreads, 1) topk_rows_kernel(const __grid_con
 // shared-memory bitmap over the row's indices, and emits it in ascending index order.
 constexpr int kSplitThreads = 512;
 constexpr int kHistBins = 4096;
+constexpr int kChunk = 4096;                  // scores per filtering chunk
 
 __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __grid_constant__ TopkSplitArgs a) {
-  extern __shared__ uint32_t bm[];              // last CTA: sel[nw] | eq[nw]
+  extern __shared__ uint32_t bm[];              // filtering: chunk buffers; last CTA: sel[nw] | eq[nw]
   __shared__ uint32_t h2[1024];
   __shared__ uint32_t wsum[32];
-  __shared__ uint32_t s_bin, s_above, s_last;
+  __shared__ uint32_t s_bin, s_above, s_last, s_ns, s_nc, s_gs, s_gc;
   const TopkArgs& A = a.base;
   const int row = blockIdx.y, g = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
   const int64_t t = A.q_pos[row];
@@ -182,25 +183,43 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
   const uint32_t bstar = s_bin;
 
   // ---------------------------------------------------------------- 2. filter this CTA's slice
+  // Chunks of kChunk scores: appends go to shared-memory buffers, then one global atomic per
+  // counter reserves the chunk's space in `sure` / `cand`.
   const int lo = (int)((int64_t)nv * g / gridDim.x), hi = (int)((int64_t)nv * (g + 1) / gridDim.x);
   const float* sc = A.scores + (size_t)row * A.n_max;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int base = lo; base < hi; base += kSplitThreads) {
-    const int i = base + tid;
-    uint32_t key = 0, bin = 0;
-    const bool in = i < hi;
-    if (in) { key = float_key(__ldg(sc + i)); bin = key >> 20; }
-    const bool is_sure = in && bin > bstar, is_cand = in && bin == bstar;
-    const uint32_t ms = __ballot_sync(0xffffffffu, is_sure), mc = __ballot_sync(0xffffffffu, is_cand);
-    uint32_t ps = 0, pc = 0;
-    if (lane == 0) {
-      if (ms) ps = atomicAdd(cnt + 0, (uint32_t)__popc(ms));
-      if (mc) pc = atomicAdd(cnt + 1, (uint32_t)__popc(mc));
+  int32_t* b_sure = reinterpret_cast<int32_t*>(bm);             // [kChunk]
+  uint2* b_cand = reinterpret_cast<uint2*>(bm + kChunk);         // [kChunk]
+  for (int cb = lo; cb < hi; cb += kChunk) {
+    if (tid == 0) { s_ns = 0u; s_nc = 0u; }
+    __syncthreads();
+    const int ce = min(cb + kChunk, hi);
+    for (int base = cb; base < ce; base += kSplitThreads) {
+      const int i = base + tid;
+      uint32_t key = 0, bin = 0;
+      const bool in = i < ce;
+      if (in) { key = float_key(__ldg(sc + i)); bin = key >> 20; }
+      const bool is_sure = in && bin > bstar, is_cand = in && bin == bstar;
+      const uint32_t ms = __ballot_sync(0xffffffffu, is_sure), mc = __ballot_sync(0xffffffffu, is_cand);
+      uint32_t ps = 0, pc = 0;
+      if (lane == 0) {
+        if (ms) ps = atomicAdd(&s_ns, (uint32_t)__popc(ms));
+        if (mc) pc = atomicAdd(&s_nc, (uint32_t)__popc(mc));
+      }
+      ps = __shfl_sync(0xffffffffu, ps, 0);
+      pc = __shfl_sync(0xffffffffu, pc, 0);
+      if (is_sure) b_sure[ps + __popc(ms & lt_mask)] = i;
+      if (is_cand) b_cand[pc + __popc(mc & lt_mask)] = make_uint2(key, (uint32_t)i);
     }
-    ps = __shfl_sync(0xffffffffu, ps, 0);
-    pc = __shfl_sync(0xffffffffu, pc, 0);
-    if (is_sure) sure[ps + __popc(ms & lt_mask)] = i;
-    if (is_cand) cand[pc + __popc(mc & lt_mask)] = make_uint2(key, (uint32_t)i);
+    __syncthreads();
+    if (tid == 0) {
+      s_gs = s_ns ? atomicAdd(cnt + 0, s_ns) : 0u;
+      s_gc = s_nc ? atomicAdd(cnt + 1, s_nc) : 0u;
+    }
+    __syncthreads();
+    for (uint32_t j = tid; j < s_ns; j += kSplitThreads) sure[s_gs + j] = b_sure[j];
+    for (uint32_t j = tid; j < s_nc; j += kSplitThreads) cand[s_gc + j] = b_cand[j];
+    __syncthreads();
   }
 
   // ---------------------------------------------------------------- 3. last CTA of the row resolves
@@ -294,13 +313,15 @@ int topk_split_ctas(int rows, int64_t n_max, int num_sms) {
 
 cudaError_t launch_topk_split(const TopkSplitArgs& a, cudaStream_t s) {
   if (a.base.rows <= 0 || a.base.k <= 0) return cudaSuccess;
-  const size_t smem = 2 * (size_t)((a.base.n_max + 31) / 32) * 4;
+  size_t smem = 2 * (size_t)((a.base.n_max + 31) / 32) * 4;
+  if (smem < (size_t)kChunk * 12) smem = (size_t)kChunk * 12;
   static size_t configured = 0;
   if (smem > 48 * 1024 && smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(topk_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = smem;
   }
+  profile_mark(s);
   topk_split_kernel<<<dim3(a.G, a.base.rows), kSplitThreads, smem, s>>>(a);
   note_launches(1);
   return cudaGetLastError();
@@ -316,6 +337,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     configured = smem;
   }
+  profile_mark(s);
   topk_rows_kernel<<<a.rows, kThreads, smem, s>>>(a, use_smem);
   note_launches(1);
   return cudaGetLastError();
