@@ -207,7 +207,7 @@ cudaError_t launch_append_compress(const AppendCompressArgs& a, int B, int Tq, c
   }
   const size_t smem = rg > 1 ? (size_t)rg * 3 * a.L.D * sizeof(float) : 0;
   static size_t configured = 0;
-  if (smem > 48 * 1024 && smem > configured) {
+  if (smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(append_compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = smem;

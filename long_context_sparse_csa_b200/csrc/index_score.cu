@@ -63,6 +63,50 @@ __device__ __forceinline__ Group group_info(const IndexArgs& a, int64_t g) {
   return G;
 }
 
+// The work items of one CTA, in order: item k -> (group g, entry tile et).  When there are no
+// more groups than CTAs (decode), the CTAs are split evenly over the groups and each takes every
+// Gc-th tile of its group, so at any moment the grid streams neighbouring tiles of the key cache
+// rather than CTA-sized slabs far apart.  Otherwise (prefill) each CTA takes a contiguous range
+// of items, which keeps its query tile resident across consecutive items.
+struct Sched {
+  bool strided;
+  int64_t g0, w0, count, tpg;
+  int et0, step;
+  __device__ __forceinline__ void at(int64_t k, int64_t* g, int* et) const {
+    if (strided) { *g = g0; *et = et0 + (int)k * step; }
+    else { const int64_t w = w0 + k; *g = w / tpg; *et = (int)(w - *g * tpg); }
+  }
+};
+
+__device__ __forceinline__ Sched make_sched(const IndexArgs& a) {
+  Sched s;
+  s.tpg = a.tiles_per_group;
+  const int64_t groups = a.total_items / s.tpg;
+  if (groups <= (int64_t)gridDim.x) {
+    const int gc = (int)(gridDim.x / groups);
+    s.strided = true;
+    s.g0 = blockIdx.x / gc;
+    s.et0 = blockIdx.x % gc;
+    s.step = gc;
+    s.w0 = 0;
+    s.count = s.g0 < groups ? (s.tpg - s.et0 + gc - 1) / gc : 0;
+  } else {
+    s.strided = false;
+    s.w0 = a.total_items * blockIdx.x / gridDim.x;
+    s.count = a.total_items * (blockIdx.x + 1) / gridDim.x - s.w0;
+    s.g0 = 0; s.et0 = 0; s.step = 1;
+  }
+  return s;
+}
+
+#ifdef CSA_TRACE
+// Diagnostic build only: per-CTA timestamps (ns) of the indexer pipeline.
+__device__ uint64_t g_trace[160][40];
+#define TRACE(slot) (g_trace[blockIdx.x][(slot)] = global_timer_ns())
+#else
+#define TRACE(slot) ((void)0)
+#endif
+
 constexpr int kHistBins = 4096;               // top 12 bits of the order-preserving score key
 constexpr int kMaxQH = 256;                   // QN * H_I
 
@@ -95,9 +139,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
   EpiSmem* es = reinterpret_cast<EpiSmem*>(reinterpret_cast<uint8_t*>(bars) + ((sizeof(Barriers) + 15) & ~size_t(15)));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t w0 = a.total_items * blockIdx.x / gridDim.x;
-  const int64_t w1 = a.total_items * (blockIdx.x + 1) / gridDim.x;
-  const int64_t tpg = a.tiles_per_group;
+  const Sched sc = make_sched(a);
+  if (threadIdx.x == 0) TRACE(0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&bars->full[s], 1); mbar_init(&bars->empty[s], 1); }
@@ -115,6 +158,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  if (threadIdx.x == 0) TRACE(1);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -128,13 +172,17 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       for (int s = 0; s < kStages; ++s) issued_par[s] = -1;
       int b_issued_par[2] = {-1, -1};
       bool ok = true;
-      for (int64_t w = w0; w < w1 && ok; ++w) {
-        const int64_t g = w / tpg;
-        const int et = (int)(w - g * tpg);
+      for (int64_t k = 0; k < sc.count && ok; ++k) {
+        int64_t g;
+        int et;
+        sc.at(k, &g, &et);
         if (g != G.g) G = group_info(a, g);
         if (et > G.last_et) continue;
         // validity is monotone in et, so the first item of a group in this CTA is its first valid one
-        const bool first_of_group = (w == w0) || (w - 1) / tpg != g;
+        int64_t gp = -1;
+        int etp;
+        if (k > 0) sc.at(k - 1, &gp, &etp);
+        const bool first_of_group = (k == 0) || gp != g;
         if (first_of_group) {
           ++gi;
           const int slot = gi & 1;
@@ -149,6 +197,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         mbar_arrive_expect_tx(&bars->full[stage], (uint32_t)kTileBytes);
         tma_load_2d(A + stage * kTileBytes, &kmap, &bars->full[stage], 0,
                     (int)((int64_t)G.b * a.entry_cap + (int64_t)et * kTileE));
+        if (k == 0) TRACE(34);
         issued_par[stage] = (int)phase;
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
@@ -170,18 +219,23 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       int last_acc = -1;
       uint32_t last_acc_par = 0;
       bool ok = true;
-      for (int64_t w = w0; w < w1; ++w) {
-        const int64_t g = w / tpg;
-        const int et = (int)(w - g * tpg);
+      for (int64_t k = 0; k < sc.count; ++k) {
+        int64_t g;
+        int et;
+        sc.at(k, &g, &et);
         if (g != G.g) G = group_info(a, g);
         if (et > G.last_et) continue;
-        const bool first_of_group = (w == w0) || (w - 1) / tpg != g;
+        int64_t gp = -1;
+        int etp;
+        if (k > 0) sc.at(k - 1, &gp, &etp);
+        const bool first_of_group = (k == 0) || gp != g;
         if (first_of_group) {
           ++gi;
           if (!mbar_wait(&bars->bfull[gi & 1], (uint32_t)((gi >> 1) & 1))) { ok = false; break; }
         }
         const int slot = gi & 1;
         if (!mbar_wait(&bars->full[stage], phase)) { ok = false; break; }
+        if (k == 0) TRACE(35);
         if (!mbar_wait(&bars->tempty[acc], acc_phase ^ 1u)) { ok = false; break; }
         tc_fence_after();
         const uint64_t ad = desc_kmajor_sw128(smem_u32(A + stage * kTileBytes));
@@ -194,7 +248,13 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         last_acc = acc;
         last_acc_par = acc_phase;
         // release the query tile after the group's last valid item in this CTA
-        const bool last_of_group = (w + 1 >= w1) || (et == G.last_et) || ((w + 1) / tpg != g);
+        bool last_of_group = k + 1 >= sc.count;
+        if (!last_of_group) {
+          int64_t gn;
+          int etn;
+          sc.at(k + 1, &gn, &etn);
+          last_of_group = gn != g || etn > G.last_et;
+        }
         if (last_of_group) umma_commit(&bars->bempty[slot]);
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
         if (++acc == nacc) { acc = 0; acc_phase ^= 1u; }
@@ -221,7 +281,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     Group G;
     G.g = -1;
     float ks_next = 0.f;
-    int64_t ks_w = -1;
+    int64_t ks_w = -1;  // item whose key scale is in ks_next
     auto flush_hist = [&](const Group& H) {
       const int64_t row = (int64_t)H.b * a.Tq + H.j0;
       for (int i = te; i < kHistBins; i += 128) {
@@ -229,9 +289,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         if (v) { atomicAdd(a.hist + row * kHistBins + i, v); es->hist[i] = 0u; }
       }
     };
-    for (int64_t w = w0; w < w1; ++w) {
-      const int64_t g = w / tpg;
-      const int et = (int)(w - g * tpg);
+    int done = 0;
+    for (int64_t k = 0; k < sc.count; ++k) {
+      int64_t g;
+      int et;
+      sc.at(k, &g, &et);
       if (g != G.g) {
         epi_bar();
         if (use_hist && G.g >= 0 && G.last_et >= 0) flush_hist(G);
@@ -250,12 +312,17 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       const bool in_range = e < a.n_max;
       // this tile's key scale was prefetched by the previous iteration when it was the same group's
       float ks;
-      if (ks_w == w) ks = ks_next;
+      if (ks_w == k) ks = ks_next;
       else ks = in_range ? __ldg(a.k_scale + (int64_t)G.b * a.entry_cap + e) : 0.f;
-      if (et + 1 <= G.last_et && w + 1 < w1) {
-        const int64_t e2 = e + kTileE;
-        ks_next = e2 < a.n_max ? __ldg(a.k_scale + (int64_t)G.b * a.entry_cap + e2) : 0.f;
-        ks_w = w + 1;
+      if (k + 1 < sc.count) {
+        int64_t gn;
+        int etn;
+        sc.at(k + 1, &gn, &etn);
+        if (gn == g && etn <= G.last_et) {
+          const int64_t e2 = (int64_t)etn * kTileE + e_loc;
+          ks_next = e2 < a.n_max ? __ldg(a.k_scale + (int64_t)G.b * a.entry_cap + e2) : 0.f;
+          ks_w = k + 1;
+        }
       }
       if (ok) ok = mbar_wait(&bars->tfull[acc], acc_phase);
       if (ok) {
@@ -287,6 +354,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         }
       }
       if (++acc == nacc) { acc = 0; acc_phase ^= 1u; }
+      if (threadIdx.x == 64 && done < 32) TRACE(2 + done);
+      ++done;
     }
     epi_bar();
     if (use_hist && G.g >= 0 && G.last_et >= 0) flush_hist(G);
@@ -295,6 +364,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) TRACE(36);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, tmem_cols);
@@ -361,6 +431,12 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows
 
 }  // namespace
 
+#ifdef CSA_TRACE
+extern "C" __attribute__((visibility("default"))) int csa_trace_read(uint64_t* host, int n) {
+  return (int)cudaMemcpyFromSymbol(host, g_trace, sizeof(uint64_t) * (size_t)n);
+}
+#endif
+
 bool index_tc_supported(int idx_fmt, int H_I, int d_I) {
   return idx_fmt == CSA_FMT_E4M3 && d_I == kDI && (H_I == 16 || H_I == 32 || H_I == 64);
 }
@@ -370,7 +446,7 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
   if (!index_tc_supported(a.idx_fmt, a.H_I, a.d_I)) {
     dim3 grid((unsigned)((a.n_max + 127) / 128), (unsigned)(a.B * a.Tq));
     const size_t sm = (size_t)a.H_I * a.d_I * sizeof(float);
-    if (sm > 48 * 1024) {
+    if (sm > 0) {
       cudaError_t e = cudaFuncSetAttribute(index_score_generic_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)sm);
       if (e != cudaSuccess) return e;

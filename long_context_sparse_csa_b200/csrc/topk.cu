@@ -316,7 +316,7 @@ cudaError_t launch_topk_split(const TopkSplitArgs& a, cudaStream_t s) {
   size_t smem = 2 * (size_t)((a.base.n_max + 31) / 32) * 4;
   if (smem < (size_t)kChunk * 12) smem = (size_t)kChunk * 12;
   static size_t configured = 0;
-  if (smem > 48 * 1024 && smem > configured) {
+  if (smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(topk_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = smem;
@@ -332,7 +332,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   const int use_smem = a.n_max <= kSmemKeys ? 1 : 0;
   const size_t smem = use_smem ? (size_t)a.n_max * 4 : 0;
   static size_t configured = 0;
-  if (smem > 48 * 1024 && smem > configured) {
+  if (smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = smem;
