@@ -54,15 +54,18 @@ __device__ __forceinline__ void mma_bf16(float d[4], const uint32_t a[4], uint32
 }
 
 __device__ __forceinline__ uint4 ldg_nc_v4(const uint8_t* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
+  return __ldg(reinterpret_cast<const uint4*>(p));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  return (uint32_t)f_to_bf16_bits(lo) | ((uint32_t)f_to_bf16_bits(hi) << 16);
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Two e4m3 codes (low byte first) -> two floats, via the hardware e4m3x2 -> f16x2 conversion.
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t codes) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)codes, __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
 // Swizzled byte offset of 16-byte chunk `ch` of row `row` in a tile whose rows are `pitch` bytes.
@@ -191,42 +194,60 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
     __syncthreads();
 
     // ------------------------------------------------------------ gather the key/value tile (bf16, swizzled)
+    // Every load of the tile is issued before any is consumed, so the row fetches overlap.
     if (FMT == CSA_FMT_BF16) {
-      for (int idx = tid; idx < kTile * 64; idx += NT) {
-        const int rr = idx >> 6, ch = idx & 63;
+      constexpr int kPer = kTile * 64 / NT;        // 16-byte chunks per thread
+      uint4 v[kPer];
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int idx = tid + u * NT, rr = idx >> 6, ch = idx & 63;
         const uint8_t* p = rowptr[rr];
-        const uint4 v = p ? ldg_nc_v4(p + ch * 16) : make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(Ks + swz(rr, ch, 1024)) = v;
+        v[u] = p ? ldg_nc_v4(p + ch * 16) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int idx = tid + u * NT, rr = idx >> 6, ch = idx & 63;
+        *reinterpret_cast<uint4*>(Ks + swz(rr, ch, 1024)) = v[u];
       }
     } else {
-      for (int idx = tid; idx < kTile * 36; idx += NT) {
-        const int rr = idx / 36, ch = idx % 36;
-        const uint8_t* p = rowptr[rr];
-        if (ch < 28) {
-          uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-          if (p) {
-            const uint4 c = ldg_nc_v4(p + ch * 16);
-            const float sig = __ldg(reinterpret_cast<const float*>(p + kD + 64));
-            const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-            uint32_t outw[8];
+      constexpr int kChunks = kTile * 36;
+      constexpr int kPer = (kChunks + NT - 1) / NT;
+      uint4 c[kPer];
+      float sig[kPer];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float f0 = e4m3_to_f((uint8_t)(w[q] & 0xFF)) * sig;
-              const float f1 = e4m3_to_f((uint8_t)((w[q] >> 8) & 0xFF)) * sig;
-              const float f2 = e4m3_to_f((uint8_t)((w[q] >> 16) & 0xFF)) * sig;
-              const float f3 = e4m3_to_f((uint8_t)(w[q] >> 24)) * sig;
-              outw[2 * q] = pack_bf16x2(f0, f1);
-              outw[2 * q + 1] = pack_bf16x2(f2, f3);
-            }
-            lo = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-            hi = make_uint4(outw[4], outw[5], outw[6], outw[7]);
+      for (int u = 0; u < kPer; ++u) {
+        const int idx = tid + u * NT;
+        c[u] = make_uint4(0u, 0u, 0u, 0u);
+        sig[u] = 0.f;
+        if (idx < kChunks) {
+          const int rr = idx / 36, ch = idx % 36;
+          const uint8_t* p = rowptr[rr];
+          if (p) {
+            c[u] = ldg_nc_v4(p + (ch < 28 ? ch * 16 : (kD - 64) + (ch - 28) * 16));
+            if (ch < 28) sig[u] = __ldg(reinterpret_cast<const float*>(p + kD + 64));
           }
-          *reinterpret_cast<uint4*>(Ks + swz(rr, 2 * ch, 1024)) = lo;
-          *reinterpret_cast<uint4*>(Ks + swz(rr, 2 * ch + 1, 1024)) = hi;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int idx = tid + u * NT;
+        if (idx >= kChunks) break;
+        const int rr = idx / 36, ch = idx % 36;
+        if (ch < 28) {
+          const uint32_t w[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+          uint32_t outw[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            // e4m3 pairs -> f16 pairs (exact), scale by the row's power of two, round to bf16 (exact)
+            const float2 lo = e4m3x2_to_float2((uint16_t)(w[q] & 0xFFFFu));
+            const float2 hi = e4m3x2_to_float2((uint16_t)(w[q] >> 16));
+            outw[2 * q] = pack_bf16x2(lo.x * sig[u], lo.y * sig[u]);
+            outw[2 * q + 1] = pack_bf16x2(hi.x * sig[u], hi.y * sig[u]);
+          }
+          *reinterpret_cast<uint4*>(Ks + swz(rr, 2 * ch, 1024)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+          *reinterpret_cast<uint4*>(Ks + swz(rr, 2 * ch + 1, 1024)) = make_uint4(outw[4], outw[5], outw[6], outw[7]);
         } else {
-          const int c2 = ch - 28;
-          const uint4 v = p ? ldg_nc_v4(p + (kD - 64) + c2 * 16) : make_uint4(0u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(Ks + swz(rr, 56 + c2, 1024)) = v;
+          *reinterpret_cast<uint4*>(Ks + swz(rr, 56 + (ch - 28), 1024)) = c[u];
         }
       }
     }

@@ -111,44 +111,54 @@ __global__ void __launch_bounds__(512) append_compress_kernel(const __grid_const
   const int64_t i = (r + 1) / L.m - 1;
   const int64_t lo = (i - L.ov) * (int64_t)L.m;
   const int64_t r_begin = lo < 0 ? 0 : lo;
+  // Online softmax in base 2 (logits pre-scaled by log2 e): per batch of rows, one max, one
+  // rescale of the running sums, then one exp2 per element.  Ring slots advance incrementally.
   float mx[4], sum[4], acc[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) { mx[k] = -INFINITY; sum[k] = 0.f; acc[k] = 0.f; }
-  // rows r_begin + rg, + RG, ... in batches whose loads are all in flight together
-  for (int64_t rb = r_begin + rg; rb <= r; rb += (int64_t)RG * kRowBatch) {
-    float xv[kRowBatch][4], gv[kRowBatch][4];
+  const int64_t rstep = (int64_t)RG;
+  int64_t slot = ring_slot(r_begin + rg, C.raw_base, C.raw_cap);
+  const int64_t slot_step = rstep % C.raw_cap;
+  for (int64_t rb = r_begin + rg; rb <= r; rb += rstep * kRowBatch) {
+    float xv[kRowBatch][4], zv[kRowBatch][4];
 #pragma unroll
     for (int u = 0; u < kRowBatch; ++u) {
-      const int64_t rr = rb + (int64_t)u * RG;
-      if (rr > r) break;
-      if (rr == r && have_new) {
+      const int64_t rr = rb + (int64_t)u * rstep;
+      const bool in = rr <= r;
+      if (in && rr == r && have_new) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) { xv[u][k] = x[k]; gv[u][k] = g[k]; }
-      } else {
-        const int64_t s = ring_slot(rr, C.raw_base, C.raw_cap);
-        load_act4(C.raw + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, xv[u]);
-        load_act4(C.gate + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, gv[u]);
+        for (int k = 0; k < 4; ++k) { xv[u][k] = x[k]; zv[u][k] = g[k]; }
+      } else if (in) {
+        load_act4(C.raw + ((size_t)b * C.raw_cap + slot) * arow, L.act_fmt, c0, xv[u]);
+        load_act4(C.gate + ((size_t)b * C.raw_cap + slot) * arow, L.act_fmt, c0, zv[u]);
       }
+      if (in) {
+        const float4 bias = __ldg(reinterpret_cast<const float4*>(a.pos_bias + (size_t)(rr - lo) * L.D + c0));
+        zv[u][0] = (zv[u][0] + bias.x) * kLog2e; zv[u][1] = (zv[u][1] + bias.y) * kLog2e;
+        zv[u][2] = (zv[u][2] + bias.z) * kLog2e; zv[u][3] = (zv[u][3] + bias.w) * kLog2e;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) { xv[u][k] = 0.f; zv[u][k] = -INFINITY; }
+      }
+      slot += slot_step;
+      if (slot >= C.raw_cap) slot -= C.raw_cap;
     }
 #pragma unroll
-    for (int u = 0; u < kRowBatch; ++u) {
-      const int64_t rr = rb + (int64_t)u * RG;
-      if (rr > r) break;
-      const float4 bias = *reinterpret_cast<const float4*>(a.pos_bias + (size_t)(rr - lo) * L.D + c0);
-      const float bz[4] = {bias.x, bias.y, bias.z, bias.w};
+    for (int k = 0; k < 4; ++k) {
+      float bm = zv[0][k];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float z = gv[u][k] + bz[k];
-        if (z > mx[k]) {
-          const float sc = expf(mx[k] - z);
-          sum[k] = sum[k] * sc + 1.f;
-          acc[k] = acc[k] * sc + xv[u][k];
-          mx[k] = z;
-        } else {
-          const float e = expf(z - mx[k]);
-          sum[k] += e;
-          acc[k] += e * xv[u][k];
-        }
+      for (int u = 1; u < kRowBatch; ++u) bm = fmaxf(bm, zv[u][k]);
+      if (bm > mx[k]) {
+        const float sc = exp2f(mx[k] - bm);
+        sum[k] *= sc;
+        acc[k] *= sc;
+        mx[k] = bm;
+      }
+#pragma unroll
+      for (int u = 0; u < kRowBatch; ++u) {
+        const float e = exp2f(zv[u][k] - mx[k]);
+        sum[k] += e;
+        acc[k] = fmaf(e, xv[u][k], acc[k]);
       }
     }
   }
@@ -170,7 +180,7 @@ __global__ void __launch_bounds__(512) append_compress_kernel(const __grid_const
           const float m2 = po[c0 + k];
           if (m2 == -INFINITY) continue;
           const float M = fmaxf(mx[k], m2);
-          const float f1 = expf(mx[k] - M), f2 = expf(m2 - M);
+          const float f1 = exp2f(mx[k] - M), f2 = exp2f(m2 - M);
           sum[k] = sum[k] * f1 + po[L.D + c0 + k] * f2;
           acc[k] = acc[k] * f1 + po[2 * L.D + c0 + k] * f2;
           mx[k] = M;
@@ -186,8 +196,8 @@ __global__ void __launch_bounds__(512) append_compress_kernel(const __grid_const
   }
   ss = block_sum(ss, scratch);
   const float rs = 1.0f / sqrtf(ss / (float)L.D + L.eps);
-#pragma unroll
-  for (int k = 0; k < 4; ++k) e[k] *= rs * (a.gamma_kv ? a.gamma_kv[c0 + k] : 1.f);
+  const float4 gk = a.gamma_kv ? __ldg(reinterpret_cast<const float4*>(a.gamma_kv + c0)) : make_float4(1.f, 1.f, 1.f, 1.f);
+  e[0] *= rs * gk.x; e[1] *= rs * gk.y; e[2] *= rs * gk.z; e[3] *= rs * gk.w;
   rope4(e, c0, L, (double)(L.pos0 + i * (int64_t)L.m));
   uint8_t* dst = C.entries + ((size_t)b * C.entry_cap + (size_t)i) * L.row_bytes;
   pack_row(dst, L, c0, e, lead, scratch);

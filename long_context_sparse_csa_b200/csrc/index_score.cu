@@ -30,7 +30,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kStages = 6;
+constexpr int kMaxStages = 6;                 // prefill ring depth; decode runs 4 stages, 2 CTAs per SM
 constexpr int kTileE = 128;                 // entries per tile (MMA M)
 constexpr int kDI = 128;                    // index-key bytes per entry
 constexpr int kTileBytes = kTileE * kDI;    // 16 KB
@@ -101,7 +101,7 @@ __device__ __forceinline__ Sched make_sched(const IndexArgs& a) {
 
 #ifdef CSA_TRACE
 // Diagnostic build only: per-CTA timestamps (ns) of the indexer pipeline.
-__device__ uint64_t g_trace[160][40];
+__device__ uint64_t g_trace[320][80];
 #define TRACE(slot) (g_trace[blockIdx.x][(slot)] = global_timer_ns())
 #else
 #define TRACE(slot) ((void)0)
@@ -113,7 +113,7 @@ constexpr int kMaxQH = 256;                   // QN * H_I
 constexpr int kMaxAcc = 4;                    // TMEM accumulators (decode: 4 x N columns; N = 256: 2)
 
 struct __align__(8) Barriers {
-  uint64_t full[kStages], empty[kStages];
+  uint64_t full[kMaxStages], empty[kMaxStages];
   uint64_t bfull[2], bempty[2];
   uint64_t tfull[kMaxAcc], tempty[kMaxAcc];
   uint32_t tmem_base;
@@ -122,12 +122,15 @@ struct __align__(8) Barriers {
 struct EpiSmem {
   float w[kMaxQH];            // head weights of the group's queries
   float qs[kMaxQH];           // index-query scales
+  float wq[kMaxQH];           // w * qs (used when every scale is positive)
+  int pos[kMaxQH / 16];       // 1 when all of the query's index-query scales are > 0
   int64_t nv[kMaxQH / 16];    // visible entries per query (QN <= 16)
   uint32_t hist[kHistBins];   // score histogram of the current group (decode)
 };
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void epi_bar() { asm volatile("barrier.sync.aligned 5, 128;" ::: "memory"); }
 
+template <int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                       const __grid_constant__ IndexArgs a, int N, int nacc, uint32_t tmem_cols) {
@@ -141,6 +144,15 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Sched sc = make_sched(a);
   if (threadIdx.x == 0) TRACE(0);
+  // the first group's visibility (a q_pos load) is fetched while the barriers and TMEM are set up
+  Group G0;
+  G0.g = -1;
+  if (sc.count > 0) {
+    int64_t g;
+    int et;
+    sc.at(0, &g, &et);
+    G0 = group_info(a, g);
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&bars->full[s], 1); mbar_init(&bars->empty[s], 1); }
@@ -160,83 +172,101 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
   const uint32_t tmem = bars->tmem_base;
   if (threadIdx.x == 0) TRACE(1);
 
+  // The producer and MMA warps run their loops with all 32 lanes (every wait is warp-uniform) and
+  // let lane 0 alone issue the bulk copies, MMAs and commits, so no warp reaches a block barrier
+  // while one of its lanes is still working.
+  auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity)) != 0;
+  };
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- TMA producer
-      int stage = 0;
-      uint32_t phase = 0;
-      Group G;
-      G.g = -1;
-      int gi = -1;
-      int issued_par[kStages];
-      for (int s = 0; s < kStages; ++s) issued_par[s] = -1;
-      int b_issued_par[2] = {-1, -1};
-      bool ok = true;
-      for (int64_t k = 0; k < sc.count && ok; ++k) {
-        int64_t g;
-        int et;
-        sc.at(k, &g, &et);
-        if (g != G.g) G = group_info(a, g);
-        if (et > G.last_et) continue;
-        // validity is monotone in et, so the first item of a group in this CTA is its first valid one
-        int64_t gp = -1;
-        int etp;
-        if (k > 0) sc.at(k - 1, &gp, &etp);
-        const bool first_of_group = (k == 0) || gp != g;
-        if (first_of_group) {
-          ++gi;
-          const int slot = gi & 1;
-          const uint32_t use = (uint32_t)(gi >> 1);
-          if (!mbar_wait(&bars->bempty[slot], (use & 1u) ^ 1u)) { ok = false; break; }
+    // ------------------------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    Group G;
+    G.g = -1;
+    int gi = -1;
+    G = G0;
+    int issued_par[kStages];
+    for (int s = 0; s < kStages; ++s) issued_par[s] = -1;
+    int b_issued_par[2] = {-1, -1};
+    bool ok = true;
+    for (int64_t k = 0; k < sc.count && ok; ++k) {
+      int64_t g;
+      int et;
+      sc.at(k, &g, &et);
+      if (g != G.g) G = group_info(a, g);
+      if (et > G.last_et) continue;
+      // validity is monotone in et, so the first item of a group in this CTA is its first valid one
+      int64_t gp = -1;
+      int etp;
+      if (k > 0) sc.at(k - 1, &gp, &etp);
+      const bool first_of_group = (k == 0) || gp != g;
+      if (first_of_group) {
+        ++gi;
+        const int slot = gi & 1;
+        const uint32_t use = (uint32_t)(gi >> 1);
+        if (!wait_all(&bars->bempty[slot], (use & 1u) ^ 1u)) { ok = false; break; }
+        if (lane == 0) {
           mbar_arrive_expect_tx(&bars->bfull[slot], (uint32_t)(N * kDI));
           tma_load_2d(Bq + slot * N * kDI, &qmap, &bars->bfull[slot], 0,
                       (int)(((int64_t)G.b * a.Tq + G.j0) * a.H_I));
-          b_issued_par[slot] = (int)(use & 1u);
         }
-        if (!mbar_wait(&bars->empty[stage], phase ^ 1u)) { ok = false; break; }
+        __syncwarp();
+        b_issued_par[slot] = (int)(use & 1u);
+      }
+      if (!wait_all(&bars->empty[stage], phase ^ 1u)) { ok = false; break; }
+      if (lane == 0) {
         mbar_arrive_expect_tx(&bars->full[stage], (uint32_t)kTileBytes);
         tma_load_2d(A + stage * kTileBytes, &kmap, &bars->full[stage], 0,
                     (int)((int64_t)G.b * a.entry_cap + (int64_t)et * kTileE));
-        if (k == 0) TRACE(34);
-        issued_par[stage] = (int)phase;
-        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        if (k < 16) TRACE(2 + k);
       }
-      if (!ok) set_device_error(a.err, kErrWaitTimeout);
-      // never leave a bulk copy in flight when the CTA exits
-      for (int s = 0; s < kStages; ++s)
-        if (issued_par[s] >= 0) mbar_wait(&bars->full[s], (uint32_t)issued_par[s]);
-      for (int s = 0; s < 2; ++s)
-        if (b_issued_par[s] >= 0) mbar_wait(&bars->bfull[s], (uint32_t)b_issued_par[s]);
+      __syncwarp();
+      issued_par[stage] = (int)phase;
+      if (++stage == kStages) { stage = 0; phase ^= 1u; }
     }
+    if (!ok && lane == 0) set_device_error(a.err, kErrWaitTimeout);
+    // never leave a bulk copy in flight when the CTA exits
+    for (int s = 0; s < kStages; ++s)
+      if (issued_par[s] >= 0) wait_all(&bars->full[s], (uint32_t)issued_par[s]);
+    for (int s = 0; s < 2; ++s)
+      if (b_issued_par[s] >= 0) wait_all(&bars->bfull[s], (uint32_t)b_issued_par[s]);
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer
-      const uint32_t idesc = instr_desc(128, N, 0u);
-      int stage = 0, acc = 0, gi = -1;
-      uint32_t phase = 0, acc_phase = 0;
-      Group G;
-      G.g = -1;
-      int last_acc = -1;
-      uint32_t last_acc_par = 0;
-      bool ok = true;
-      for (int64_t k = 0; k < sc.count; ++k) {
-        int64_t g;
-        int et;
-        sc.at(k, &g, &et);
-        if (g != G.g) G = group_info(a, g);
-        if (et > G.last_et) continue;
-        int64_t gp = -1;
-        int etp;
-        if (k > 0) sc.at(k - 1, &gp, &etp);
-        const bool first_of_group = (k == 0) || gp != g;
-        if (first_of_group) {
-          ++gi;
-          if (!mbar_wait(&bars->bfull[gi & 1], (uint32_t)((gi >> 1) & 1))) { ok = false; break; }
-        }
-        const int slot = gi & 1;
-        if (!mbar_wait(&bars->full[stage], phase)) { ok = false; break; }
-        if (k == 0) TRACE(35);
-        if (!mbar_wait(&bars->tempty[acc], acc_phase ^ 1u)) { ok = false; break; }
+    // ------------------------------------------------------------------ MMA issuer
+    const uint32_t idesc = instr_desc(128, N, 0u);
+    int stage = 0, acc = 0, gi = -1;
+    uint32_t phase = 0, acc_phase = 0;
+    Group G = G0;
+    int last_acc = -1;
+    uint32_t last_acc_par = 0;
+    bool ok = true;
+    for (int64_t k = 0; k < sc.count; ++k) {
+      int64_t g;
+      int et;
+      sc.at(k, &g, &et);
+      if (g != G.g) G = group_info(a, g);
+      if (et > G.last_et) continue;
+      int64_t gp = -1;
+      int etp;
+      if (k > 0) sc.at(k - 1, &gp, &etp);
+      const bool first_of_group = (k == 0) || gp != g;
+      if (first_of_group) {
+        ++gi;
+        if (!wait_all(&bars->bfull[gi & 1], (uint32_t)((gi >> 1) & 1))) { ok = false; break; }
+      }
+      const int slot = gi & 1;
+      if (!wait_all(&bars->full[stage], phase)) { ok = false; break; }
+      if (lane == 0 && k < 16) TRACE(18 + k);
+      if (!wait_all(&bars->tempty[acc], acc_phase ^ 1u)) { ok = false; break; }
+      // release the query tile after the group's last valid item in this CTA
+      bool last_of_group = k + 1 >= sc.count;
+      if (!last_of_group) {
+        int64_t gn;
+        int etn;
+        sc.at(k + 1, &gn, &etn);
+        last_of_group = gn != g || etn > G.last_et;
+      }
+      if (lane == 0) {
         tc_fence_after();
         const uint64_t ad = desc_kmajor_sw128(smem_u32(A + stage * kTileBytes));
         const uint64_t bd = desc_kmajor_sw128(smem_u32(Bq + slot * N * kDI));
@@ -245,24 +275,17 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
           umma_f8f6f4(tmem + (uint32_t)(acc * N), ad + 2u * kk, bd + 2u * kk, idesc, kk > 0 ? 1u : 0u);
         umma_commit(&bars->empty[stage]);
         umma_commit(&bars->tfull[acc]);
-        last_acc = acc;
-        last_acc_par = acc_phase;
-        // release the query tile after the group's last valid item in this CTA
-        bool last_of_group = k + 1 >= sc.count;
-        if (!last_of_group) {
-          int64_t gn;
-          int etn;
-          sc.at(k + 1, &gn, &etn);
-          last_of_group = gn != g || etn > G.last_et;
-        }
         if (last_of_group) umma_commit(&bars->bempty[slot]);
-        if (++stage == kStages) { stage = 0; phase ^= 1u; }
-        if (++acc == nacc) { acc = 0; acc_phase ^= 1u; }
       }
-      if (!ok) set_device_error(a.err, kErrWaitTimeout);
-      // the accumulator must be idle before TMEM is released
-      if (last_acc >= 0) mbar_wait(&bars->tfull[last_acc], last_acc_par);
+      __syncwarp();
+      last_acc = acc;
+      last_acc_par = acc_phase;
+      if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      if (++acc == nacc) { acc = 0; acc_phase ^= 1u; }
     }
+    if (!ok && lane == 0) set_device_error(a.err, kErrWaitTimeout);
+    // the accumulator must be idle before TMEM is released
+    if (last_acc >= 0) wait_all(&bars->tfull[last_acc], last_acc_par);
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..5)
     // Every epilogue warp runs the same sequence of named barriers whatever happens (a wait that
@@ -301,10 +324,18 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         for (int i = te; i < QH; i += 128) {
           const int j = G.j0 + i / a.H_I;
           const int64_t row = (int64_t)G.b * a.Tq + (j < a.Tq ? j : a.Tq - 1);
-          es->w[i] = a.head_w[row * a.H_I + i % a.H_I];
-          es->qs[i] = a.q_scale[row * a.H_I + i % a.H_I];
+          const float wv = a.head_w[row * a.H_I + i % a.H_I], qv = a.q_scale[row * a.H_I + i % a.H_I];
+          es->w[i] = wv;
+          es->qs[i] = qv;
+          es->wq[i] = wv * qv;
         }
         if (te < a.QN) es->nv[te] = (G.j0 + te < a.Tq) ? n_visible(a, G.b, G.j0 + te) : 0;
+        epi_bar();
+        if (te < a.QN) {
+          int p = 1;
+          for (int h = 0; h < a.H_I; ++h) p &= es->qs[te * a.H_I + h] > 0.f;
+          es->pos[te] = p;
+        }
         epi_bar();
       }
       if (et > G.last_et) continue;
@@ -325,6 +356,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         }
       }
       if (ok) ok = mbar_wait(&bars->tfull[acc], acc_phase);
+      if (threadIdx.x == 64 && done < 16) TRACE(34 + done);
       if (ok) {
         tc_fence_after();
         for (int j = G.j0; j < G.j1; ++j) {
@@ -332,6 +364,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
           const int64_t row = (int64_t)G.b * a.Tq + j;
           const float* wq = es->w + q * a.H_I;
           const float* sq = es->qs + q * a.H_I;
+          const float* wqq = es->wq + q * a.H_I;
+          // positive scales: ReLU(qs * ks * v) = qs * ks * ReLU(v), so s = ks * sum_h (w*qs)_h ReLU(v_h)
+          const bool fast = es->pos[q] && ks > 0.f;
           float s = 0.f;
           for (int hc = 0; hc < a.H_I; hc += 32) {
             float v[32];
@@ -344,17 +379,29 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
               mbar_arrive(&bars->tempty[acc]);
             }
             const int nh = min(32, a.H_I - hc);
+            if (fast) {
 #pragma unroll
-            for (int h = 0; h < 32; ++h)
-              if (h < nh) s += wq[hc + h] * fmaxf(v[h] * (sq[hc + h] * ks), 0.f);
+              for (int h = 0; h < 32; ++h)
+                if (h < nh) s = fmaf(wqq[hc + h], fmaxf(v[h], 0.f), s);
+            } else {
+#pragma unroll
+              for (int h = 0; h < 32; ++h)
+                if (h < nh) s += wq[hc + h] * fmaxf(v[h] * (sq[hc + h] * ks), 0.f);
+            }
           }
+          if (fast) s *= ks;
           const bool vis = e < es->nv[q];
           if (in_range) a.scores[row * a.n_max + e] = vis ? s : -INFINITY;
-          if (use_hist && vis) atomicAdd(&es->hist[float_key(s) >> 20], 1u);
+          if (use_hist) {
+            // one shared-memory atomic per distinct bin in the warp
+            const uint32_t bin = vis ? (float_key(s) >> 20) : 0xFFFFFFFFu;
+            const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+            if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&es->hist[bin], (uint32_t)__popc(peers));
+          }
         }
       }
       if (++acc == nacc) { acc = 0; acc_phase ^= 1u; }
-      if (threadIdx.x == 64 && done < 32) TRACE(2 + done);
+      if (threadIdx.x == 64 && done < 16) TRACE(50 + done);
       ++done;
     }
     epi_bar();
@@ -362,9 +409,12 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     if (!ok) set_device_error(a.err, kErrWaitTimeout);
   }
 
+  if (threadIdx.x == 0) TRACE(68);
+  if (threadIdx.x == 64) TRACE(70);
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0) TRACE(36);
+  if (threadIdx.x == 0) TRACE(66);
+  if (threadIdx.x == 64) TRACE(67);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, tmem_cols);
@@ -467,18 +517,22 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
   const int nacc = N <= 128 ? 4 : 2;
   uint32_t cols = 32;
   while (cols < (uint32_t)(nacc * N)) cols <<= 1;
-  const size_t smem = 1024 + (size_t)kStages * kTileBytes + 2 * (size_t)N * kDI + ((sizeof(Barriers) + 15) & ~size_t(15)) +
+  const bool decode = a.Tq == 1;
+  const int stages = decode ? 4 : 6;
+  const size_t smem = 1024 + (size_t)stages * kTileBytes + 2 * (size_t)N * kDI + ((sizeof(Barriers) + 15) & ~size_t(15)) +
                      sizeof(EpiSmem) + 64;
-  static size_t configured = 0;
-  if (smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(index_score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+  static size_t configured[2] = {0, 0};
+  auto kern = decode ? index_score_tc_kernel<4> : index_score_tc_kernel<6>;
+  if (smem > configured[decode]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    configured = smem;
+    configured[decode] = smem;
   }
-  const int64_t grid = a.total_items < num_sms ? a.total_items : num_sms;
+  // decode: two CTAs per SM (two independent pipelines); each CTA's smem and TMEM allow it
+  const int64_t ctas = decode ? 2 * (int64_t)num_sms : num_sms;
+  const int64_t grid = a.total_items < ctas ? a.total_items : ctas;
   profile_mark(s);
-  index_score_tc_kernel<<<(unsigned)grid, kThreads, smem, s>>>(kmap, qmap, a, N, nacc, cols);
+  kern<<<(unsigned)grid, kThreads, smem, s>>>(kmap, qmap, a, N, nacc, cols);
   note_launches(1);
   return cudaGetLastError();
 }

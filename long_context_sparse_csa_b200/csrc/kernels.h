@@ -74,7 +74,7 @@ struct TopkSplitArgs {
   int G;                    // CTAs per row
 };
 constexpr int64_t kTopkSplitMinN = 16384;     // rows at least this long use the split kernel
-constexpr int64_t kTopkSplitMaxN = 786432;    // the resolving CTA's bitmaps must fit shared memory
+constexpr int64_t kTopkSplitMaxN = 655360;    // the resolving CTA's bitmaps + staged candidates fit shared memory
 int topk_split_ctas(int rows, int64_t n_max, int num_sms);
 cudaError_t launch_topk_split(const TopkSplitArgs& a, cudaStream_t s);
 

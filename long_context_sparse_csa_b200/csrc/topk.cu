@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_rows_kernel(const __grid_con
 constexpr int kSplitThreads = 512;
 constexpr int kHistBins = 4096;
 constexpr int kChunk = 4096;                  // scores per filtering chunk
+constexpr int kCandCap = 4096;                // candidates staged in shared memory by the resolving CTA
 
 __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __grid_constant__ TopkSplitArgs a) {
   extern __shared__ uint32_t bm[];              // filtering: chunk buffers; last CTA: sel[nw] | eq[nw]
@@ -194,11 +195,19 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
     if (tid == 0) { s_ns = 0u; s_nc = 0u; }
     __syncthreads();
     const int ce = min(cb + kChunk, hi);
-    for (int base = cb; base < ce; base += kSplitThreads) {
-      const int i = base + tid;
+    constexpr int kPer = kChunk / kSplitThreads;
+    float vals[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = cb + u * kSplitThreads + tid;
+      vals[u] = i < ce ? __ldg(sc + i) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = cb + u * kSplitThreads + tid;
       uint32_t key = 0, bin = 0;
       const bool in = i < ce;
-      if (in) { key = float_key(__ldg(sc + i)); bin = key >> 20; }
+      if (in) { key = float_key(vals[u]); bin = key >> 20; }
       const bool is_sure = in && bin > bstar, is_cand = in && bin == bstar;
       const uint32_t ms = __ballot_sync(0xffffffffu, is_sure), mc = __ballot_sync(0xffffffffu, is_cand);
       uint32_t ps = 0, pc = 0;
@@ -233,6 +242,17 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
   __threadfence();
   const uint32_t n_sure = atomicAdd(cnt + 0, 0u), nc = atomicAdd(cnt + 1, 0u);
   uint32_t rem = (uint32_t)k - n_sure;        // >= 1: fewer than k keys lie above b*
+  const int nw = (nv + 31) >> 5;
+  uint32_t* sel = bm;
+  uint32_t* eqm = bm + nw;
+  // candidates are read three times below: stage them in shared memory when they fit
+  uint2* cs = reinterpret_cast<uint2*>(bm + 2 * (((A.n_max + 31) >> 5)));
+  const bool staged = nc <= (uint32_t)kCandCap;
+  if (staged)
+    for (uint32_t j = tid; j < nc; j += kSplitThreads) cs[j] = cand[j];
+  const uint2* cv = staged ? cs : cand;
+  for (int i = tid; i < 2 * nw; i += kSplitThreads) bm[i] = 0u;
+  __syncthreads();
 
   // two 10-bit radix passes over the candidates' low 20 bits pin the exact key T
   uint32_t prefix = bstar;
@@ -242,7 +262,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
     for (int i = tid; i < 1024; i += kSplitThreads) h2[i] = 0u;
     __syncthreads();
     for (uint32_t j = tid; j < nc; j += kSplitThreads) {
-      const uint32_t key = cand[j].x;
+      const uint32_t key = cv[j].x;
       if ((key >> (32 - fixed)) == prefix) atomicAdd(&h2[(key >> shift) & 1023u], 1u);
     }
     __syncthreads();
@@ -254,17 +274,12 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
   }
   const uint32_t T = prefix;                   // keys > T are taken; `rem` keys == T, smallest indices
 
-  const int nw = (nv + 31) >> 5;
-  uint32_t* sel = bm;
-  uint32_t* eqm = bm + nw;
-  for (int i = tid; i < 2 * nw; i += kSplitThreads) bm[i] = 0u;
-  __syncthreads();
   for (uint32_t j = tid; j < n_sure; j += kSplitThreads) {
     const uint32_t i = (uint32_t)sure[j];
     atomicOr(&sel[i >> 5], 1u << (i & 31));
   }
   for (uint32_t j = tid; j < nc; j += kSplitThreads) {
-    const uint2 c = cand[j];
+    const uint2 c = cv[j];
     if (c.x > T) atomicOr(&sel[c.y >> 5], 1u << (c.y & 31));
     else if (c.x == T) atomicOr(&eqm[c.y >> 5], 1u << (c.y & 31));
   }
@@ -313,7 +328,7 @@ int topk_split_ctas(int rows, int64_t n_max, int num_sms) {
 
 cudaError_t launch_topk_split(const TopkSplitArgs& a, cudaStream_t s) {
   if (a.base.rows <= 0 || a.base.k <= 0) return cudaSuccess;
-  size_t smem = 2 * (size_t)((a.base.n_max + 31) / 32) * 4;
+  size_t smem = 2 * (size_t)((a.base.n_max + 31) / 32) * 4 + (size_t)kCandCap * 8;
   if (smem < (size_t)kChunk * 12) smem = (size_t)kChunk * 12;
   static size_t configured = 0;
   if (smem > configured) {
