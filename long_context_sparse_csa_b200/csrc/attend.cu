@@ -424,9 +424,11 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
 // maxima and sums are staged in shared memory first, so every partial-output load of the
 // weighted sum is independent and can be in flight together.
 template <int HG>
-__global__ void attend_combine_kernel(const __grid_constant__ AttendArgs a) {
+__global__ void __launch_bounds__(512) attend_combine_kernel(const __grid_constant__ AttendArgs a) {
+  constexpr int kGroups = 4;                       // split groups; 128 dim-threads each
   __shared__ float fac[1024];
   __shared__ float s_inv;
+  __shared__ float4 red[kGroups - 1][kD / 4];
   const LayerArgs& L = a.L;
   const int h = blockIdx.x, row = blockIdx.y;
   const int hg = h / HG, hl = h % HG;
@@ -434,30 +436,51 @@ __global__ void attend_combine_kernel(const __grid_constant__ AttendArgs a) {
   const float* base = a.part + ((size_t)row * (L.H / HG) + hg) * a.splits * pstride;
   const float sk = a.sinks[h] * kLog2e;
   const int S = a.splits;
-  for (int s = threadIdx.x; s < S; s += blockDim.x) fac[s] = base[s * pstride + HG * kD + hl];
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float M = sk;
-    for (int s = threadIdx.x; s < S; s += 32) M = fmaxf(M, fac[s]);
-    M = warp_max(M);
-    float den = 0.f;
-    for (int s = threadIdx.x; s < S; s += 32) {
-      const float f = exp2f(fac[s] - M);
-      den += base[s * pstride + HG * kD + HG + hl] * f;
-      fac[s] = f;
-    }
-    den = warp_sum(den) + exp2f(sk - M);
-    if (threadIdx.x == 0) s_inv = 1.f / den;
+  const int tid = threadIdx.x, grp = tid >> 7, dt = tid & 127;
+  float lsum = 0.f;
+  for (int s = tid; s < S; s += blockDim.x) {
+    fac[s] = base[s * pstride + HG * kD + hl];
+    fac[512 + s] = base[s * pstride + HG * kD + HG + hl];
   }
   __syncthreads();
-  const int d0 = threadIdx.x * 4;
+  if (tid < 32) {
+    float M = sk;
+    for (int s = tid; s < S; s += 32) M = fmaxf(M, fac[s]);
+    M = warp_max(M);
+    for (int s = tid; s < S; s += 32) {
+      const float f = exp2f(fac[s] - M);
+      lsum += fac[512 + s] * f;
+      fac[s] = f;
+    }
+    lsum = warp_sum(lsum) + exp2f(sk - M);
+    if (tid == 0) s_inv = 1.f / lsum;
+  }
+  __syncthreads();
+  // each split group sums every kGroups-th split, 8 loads in flight per thread
+  const int d0 = dt * 4;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   const float* p = base + (size_t)hl * kD + d0;
-#pragma unroll 8
-  for (int s = 0; s < S; ++s) {
-    const float4 v = *reinterpret_cast<const float4*>(p + s * pstride);
-    const float f = fac[s];
-    acc[0] += v.x * f; acc[1] += v.y * f; acc[2] += v.z * f; acc[3] += v.w * f;
+  for (int s0 = grp; s0 < S; s0 += kGroups * 8) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int s = s0 + u * kGroups;
+      v[u] = s < S ? *reinterpret_cast<const float4*>(p + s * pstride) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int s = s0 + u * kGroups;
+      const float f = s < S ? fac[s] : 0.f;
+      acc[0] += v[u].x * f; acc[1] += v[u].y * f; acc[2] += v[u].z * f; acc[3] += v[u].w * f;
+    }
+  }
+  if (grp > 0) red[grp - 1][dt] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  __syncthreads();
+  if (grp != 0) return;
+#pragma unroll
+  for (int q = 0; q < kGroups - 1; ++q) {
+    const float4 o = red[q][dt];
+    acc[0] += o.x; acc[1] += o.y; acc[2] += o.z; acc[3] += o.w;
   }
   const float inv = s_inv;
 #pragma unroll
@@ -583,7 +606,7 @@ cudaError_t launch_mma(const AttendArgs& a, cudaStream_t s) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || a.splits == 1) return e;
   profile_mark(s);
-  attend_combine_kernel<HG><<<dim3(a.L.H, a.rows), kD / 4, 0, s>>>(a);
+  attend_combine_kernel<HG><<<dim3(a.L.H, a.rows), 512, 0, s>>>(a);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -12,12 +12,25 @@
 // One CTA per (token, sequence), D/4 threads, 4 consecutive channels per
 // thread; raw rows are read once with 8/16-byte vector loads and the
 // per-channel softmax runs online in registers.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
+
+namespace cg = cooperative_groups;
 
 namespace csa {
 
 namespace {
+
+#ifdef CSA_TRACE
+__device__ uint64_t g_trace_c[4][16];
+#define CTRACE(slot) do { if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) { \
+    uint64_t _t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(_t) :: "memory"); \
+    g_trace_c[(L.m == 4) ? 0 : 1][(slot)] = _t; } } while (0)
+#else
+#define CTRACE(slot) ((void)0)
+#endif
 
 __device__ __forceinline__ void rope4(float v[4], int c0, const LayerArgs& L, double pos) {
   const int dn = L.D - L.d_rope;
@@ -32,10 +45,28 @@ __device__ __forceinline__ void rope4(float v[4], int c0, const LayerArgs& L, do
   v[2] = a * c - b * s; v[3] = a * s + b * c;
 }
 
-// Block-cooperative store of one row in the cache format.  Every thread of the block calls it
-// (the FP8 scale needs a block-wide max); threads with active == false hold no channels.
-__device__ __forceinline__ void pack_row(uint8_t* dst, const LayerArgs& L, int c0, const float v[4], bool active,
-                                         float* scratch) {
+constexpr int kRowBatch = 8;   // rows whose loads are issued together per thread
+
+// Sum / max of one value per CTA over the CTA's cluster, through distributed shared memory.
+// `slot` is a shared-memory float used by this reduction only; every thread gets the result.
+__device__ __forceinline__ float cluster_reduce(float v, float* slot, float* bcast, bool is_max) {
+  cg::cluster_group cl = cg::this_cluster();
+  if (threadIdx.x == 0) *slot = v;
+  cl.sync();
+  if (threadIdx.x < 32) {
+    float r = is_max ? -INFINITY : 0.f;
+    if ((unsigned)threadIdx.x < cl.num_blocks()) r = *cl.map_shared_rank(slot, threadIdx.x);
+    r = is_max ? warp_max(r) : warp_sum(r);
+    if (threadIdx.x == 0) *bcast = r;
+  }
+  __syncthreads();
+  return *bcast;
+}
+
+// Stores this CTA's channels of one row in the cache format.  `am` is the cluster-wide max |x|
+// over the FP8 dims (mixed format only); threads with active == false hold no channels.
+__device__ __forceinline__ void pack_slice(uint8_t* dst, const LayerArgs& L, int c0, const float v[4], bool active,
+                                           float am, bool writes_scale) {
   if (L.kv_fmt == CSA_FMT_F32) {
     if (active) *reinterpret_cast<float4*>(dst + 4 * (size_t)c0) = make_float4(v[0], v[1], v[2], v[3]);
     return;
@@ -45,57 +76,69 @@ __device__ __forceinline__ void pack_row(uint8_t* dst, const LayerArgs& L, int c
     return;
   }
   const int dn = L.D - L.d_rope;
-  float am = 0.f;
-  if (active && c0 < dn) am = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-  am = block_max(am, scratch);
   float inv;
   const float sig = pow2_scale(am, &inv);
-  if (!active) return;
-  if (c0 < dn) {
-    uint32_t w = (uint32_t)f_to_e4m3_sat(v[0] * inv) | ((uint32_t)f_to_e4m3_sat(v[1] * inv) << 8) |
-                 ((uint32_t)f_to_e4m3_sat(v[2] * inv) << 16) | ((uint32_t)f_to_e4m3_sat(v[3] * inv) << 24);
-    *reinterpret_cast<uint32_t*>(dst + c0) = w;
-  } else {
-    store_act4(dst + dn, CSA_FMT_BF16, c0 - dn, v);
+  if (active) {
+    if (c0 < dn) {
+      uint32_t w = (uint32_t)f_to_e4m3_sat(v[0] * inv) | ((uint32_t)f_to_e4m3_sat(v[1] * inv) << 8) |
+                   ((uint32_t)f_to_e4m3_sat(v[2] * inv) << 16) | ((uint32_t)f_to_e4m3_sat(v[3] * inv) << 24);
+      *reinterpret_cast<uint32_t*>(dst + c0) = w;
+    } else {
+      store_act4(dst + dn, CSA_FMT_BF16, c0 - dn, v);
+    }
   }
-  if (threadIdx.x == 0) {
+  if (writes_scale && threadIdx.x == 0) {
     *reinterpret_cast<float*>(dst + L.D + 64) = sig;
     *reinterpret_cast<uint32_t*>(dst + L.D + 68) = 0u;
     *reinterpret_cast<uint2*>(dst + L.D + 72) = make_uint2(0u, 0u);
   }
 }
 
-constexpr int kRowBatch = 8;   // rows whose loads are issued together per thread
+__device__ __forceinline__ float local_amax(const float v[4], int c0, int dn, bool active) {
+  return (active && c0 < dn) ? fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))) : 0.f;
+}
 
-// Block = (D/4) channel threads x RG row groups.  Row group 0 appends the new token; every row
-// group pools a strided subset of the entry's source rows with an online softmax; the groups'
-// partial (max, sum, weighted sum) are merged through shared memory.
-__global__ void __launch_bounds__(512) append_compress_kernel(const __grid_constant__ AppendCompressArgs a) {
+// One token per cluster of CL CTAs; CTA rank q owns channels [q*D/CL, (q+1)*D/CL).  Inside a CTA:
+// (D/CL/4) channel threads x RG row groups.  Row group 0 appends the token (its window row); every
+// row group pools a strided subset of the completed entry's source rows with an online softmax;
+// groups merge through shared memory and the row-wide RMSNorm sum and FP8 amax are reduced over
+// the cluster.  With CL = 1 (chunked prefill) the cluster reductions are plain block reductions.
+__global__ void __launch_bounds__(512) append_compress_kernel(const __grid_constant__ AppendCompressArgs a, int CL) {
   __shared__ float scratch[32];
-  extern __shared__ float part[];                  // [RG][3][D]
+  __shared__ float red[4], bcast;
+  extern __shared__ float part[];                  // [RG][3][DC]
+  cg::cluster_group cluster = cg::this_cluster();
   const LayerArgs& L = a.L;
   const CacheArgs& C = a.C;
-  const int j = blockIdx.x, b = blockIdx.y;
-  const int CT = L.D / 4;                          // channel threads per row group
+  const int q = (int)cluster.block_rank();
+  const int j = blockIdx.x / CL, b = blockIdx.y;
+  const int DC = L.D / CL;                         // channels of this CTA
+  const int CT = DC / 4;                           // channel threads per row group
   const int RG = blockDim.x / CT;
   const int ct = threadIdx.x % CT, rg = threadIdx.x / CT;
-  const int c0 = ct * 4;
+  const int c0 = q * DC + ct * 4;                  // first channel of this thread (row-wide index)
   const bool lead = rg == 0;
+  const int dn = L.D - L.d_rope;
+  CTRACE(0);
   const int64_t t = a.q_pos[(int64_t)b * a.Tq + j];
   const int64_t r = t - L.pos0;
-  if (r < 0) return;  // uniform over the block
+  const bool valid = r >= 0;                       // uniform over the cluster
   const size_t arow = (size_t)L.D * act_bytes(L.act_fmt);
   const bool have_new = a.x_new != nullptr;
   float x[4] = {0.f, 0.f, 0.f, 0.f}, g[4] = {0.f, 0.f, 0.f, 0.f};
-  if (have_new) {
-    load_act4(a.x_new + ((size_t)b * a.Tq + j) * arow, L.act_fmt, c0, x);
-    load_act4(a.g_new + ((size_t)b * a.Tq + j) * arow, L.act_fmt, c0, g);
-  } else if (a.do_append) {
-    const int64_t s = ring_slot(r, C.raw_base, C.raw_cap);
-    load_act4(C.raw + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, x);
+  if (valid) {
+    if (have_new) {
+      load_act4(a.x_new + ((size_t)b * a.Tq + j) * arow, L.act_fmt, c0, x);
+      load_act4(a.g_new + ((size_t)b * a.Tq + j) * arow, L.act_fmt, c0, g);
+    } else if (a.do_append) {
+      const int64_t s = ring_slot(r, C.raw_base, C.raw_cap);
+      load_act4(C.raw + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, x);
+    }
   }
+  CTRACE(1);
+  const bool compress = valid && a.do_compress && ((r + 1) % L.m) == 0;
 
-  if (a.do_append) {
+  if (valid && a.do_append) {
     if (have_new && lead) {
       const int64_t s = ring_slot(r, C.raw_base, C.raw_cap);
       store_act4(C.raw + ((size_t)b * C.raw_cap + s) * arow, L.act_fmt, c0, x);
@@ -103,129 +146,186 @@ __global__ void __launch_bounds__(512) append_compress_kernel(const __grid_const
     }
     float w[4] = {x[0], x[1], x[2], x[3]};
     rope4(w, c0, L, (double)t);
+    float am = 0.f;
+    if (L.kv_fmt == CSA_FMT_MIXED) am = cluster_reduce(block_max(local_amax(w, c0, dn, lead), scratch), &red[0], &bcast, true);
     uint8_t* dst = C.window + ((size_t)b * C.window_cap + (size_t)(r % C.window_cap)) * L.row_bytes;
-    pack_row(dst, L, c0, w, lead, scratch);
+    pack_slice(dst, L, c0, w, lead, am, q == 0);
   }
+  CTRACE(2);
+  CTRACE(3);
 
-  if (!(a.do_compress && ((r + 1) % L.m) == 0)) return;
-  const int64_t i = (r + 1) / L.m - 1;
-  const int64_t lo = (i - L.ov) * (int64_t)L.m;
-  const int64_t r_begin = lo < 0 ? 0 : lo;
-  // Online softmax in base 2 (logits pre-scaled by log2 e): per batch of rows, one max, one
-  // rescale of the running sums, then one exp2 per element.  Ring slots advance incrementally.
-  float mx[4], sum[4], acc[4];
+  if (compress) {
+    const int64_t i = (r + 1) / L.m - 1;
+    const int64_t lo = (i - L.ov) * (int64_t)L.m;
+    const int64_t r_begin = lo < 0 ? 0 : lo;
+    // Online softmax in base 2 (logits pre-scaled by log2 e): per batch of rows, one max, one
+    // rescale of the running sums, then one exp2 per element.  Ring slots advance incrementally.
+    float mx[4], sum[4], acc[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) { mx[k] = -INFINITY; sum[k] = 0.f; acc[k] = 0.f; }
-  const int64_t rstep = (int64_t)RG;
-  int64_t slot = ring_slot(r_begin + rg, C.raw_base, C.raw_cap);
-  const int64_t slot_step = rstep % C.raw_cap;
-  for (int64_t rb = r_begin + rg; rb <= r; rb += rstep * kRowBatch) {
-    float xv[kRowBatch][4], zv[kRowBatch][4];
+    for (int k = 0; k < 4; ++k) { mx[k] = -INFINITY; sum[k] = 0.f; acc[k] = 0.f; }
+    const int64_t rstep = (int64_t)RG;
+    int64_t slot = ring_slot(r_begin + rg, C.raw_base, C.raw_cap);
+    const int64_t slot_step = rstep % C.raw_cap;
+    for (int64_t rb = r_begin + rg; rb <= r; rb += rstep * kRowBatch) {
+      // 1) issue every load of the batch (rows past r re-read a valid row and are masked below)
+      float xv[kRowBatch][4], zv[kRowBatch][4];
+      float4 bias[kRowBatch];
+      int64_t slots[kRowBatch];
 #pragma unroll
-    for (int u = 0; u < kRowBatch; ++u) {
-      const int64_t rr = rb + (int64_t)u * rstep;
-      const bool in = rr <= r;
-      if (in && rr == r && have_new) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) { xv[u][k] = x[k]; zv[u][k] = g[k]; }
-      } else if (in) {
-        load_act4(C.raw + ((size_t)b * C.raw_cap + slot) * arow, L.act_fmt, c0, xv[u]);
-        load_act4(C.gate + ((size_t)b * C.raw_cap + slot) * arow, L.act_fmt, c0, zv[u]);
-      }
-      if (in) {
-        const float4 bias = __ldg(reinterpret_cast<const float4*>(a.pos_bias + (size_t)(rr - lo) * L.D + c0));
-        zv[u][0] = (zv[u][0] + bias.x) * kLog2e; zv[u][1] = (zv[u][1] + bias.y) * kLog2e;
-        zv[u][2] = (zv[u][2] + bias.z) * kLog2e; zv[u][3] = (zv[u][3] + bias.w) * kLog2e;
-      } else {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) { xv[u][k] = 0.f; zv[u][k] = -INFINITY; }
-      }
-      slot += slot_step;
-      if (slot >= C.raw_cap) slot -= C.raw_cap;
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float bm = zv[0][k];
-#pragma unroll
-      for (int u = 1; u < kRowBatch; ++u) bm = fmaxf(bm, zv[u][k]);
-      if (bm > mx[k]) {
-        const float sc = exp2f(mx[k] - bm);
-        sum[k] *= sc;
-        acc[k] *= sc;
-        mx[k] = bm;
+      for (int u = 0; u < kRowBatch; ++u) {
+        slots[u] = slot;
+        slot += slot_step;
+        if (slot >= C.raw_cap) slot -= C.raw_cap;
       }
 #pragma unroll
       for (int u = 0; u < kRowBatch; ++u) {
-        const float e = exp2f(zv[u][k] - mx[k]);
-        sum[k] += e;
-        acc[k] = fmaf(e, xv[u][k], acc[k]);
+        const int64_t rr = rb + (int64_t)u * rstep;
+        const int64_t sl = rr <= r ? slots[u] : slots[0];
+        load_act4(C.raw + ((size_t)b * C.raw_cap + sl) * arow, L.act_fmt, c0, xv[u]);
+        load_act4(C.gate + ((size_t)b * C.raw_cap + sl) * arow, L.act_fmt, c0, zv[u]);
+        const int64_t br = (rr <= r ? rr : rb) - lo;
+        bias[u] = __ldg(reinterpret_cast<const float4*>(a.pos_bias + (size_t)br * L.D + c0));
+      }
+      // 2) logits in base 2, masked rows, the just-appended row from registers
+#pragma unroll
+      for (int u = 0; u < kRowBatch; ++u) {
+        const int64_t rr = rb + (int64_t)u * rstep;
+        if (rr == r && have_new) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) { xv[u][k] = x[k]; zv[u][k] = g[k]; }
+        }
+        if (rr <= r) {
+          zv[u][0] = (zv[u][0] + bias[u].x) * kLog2e; zv[u][1] = (zv[u][1] + bias[u].y) * kLog2e;
+          zv[u][2] = (zv[u][2] + bias[u].z) * kLog2e; zv[u][3] = (zv[u][3] + bias[u].w) * kLog2e;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) { xv[u][k] = 0.f; zv[u][k] = -INFINITY; }
+        }
+      }
+      // 3) batch max, one rescale, exp2 per element
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float bm = zv[0][k];
+#pragma unroll
+        for (int u = 1; u < kRowBatch; ++u) bm = fmaxf(bm, zv[u][k]);
+        if (bm > mx[k]) {
+          const float sc = exp2f(mx[k] - bm);
+          sum[k] *= sc;
+          acc[k] *= sc;
+          mx[k] = bm;
+        }
+#pragma unroll
+        for (int u = 0; u < kRowBatch; ++u) {
+          const float e = exp2f(zv[u][k] - mx[k]);
+          sum[k] += e;
+          acc[k] = fmaf(e, xv[u][k], acc[k]);
+        }
       }
     }
-  }
-  // merge the row groups
-  if (RG > 1) {
-    float* pm = part + (size_t)rg * 3 * L.D;
+    CTRACE(4);
+    // merge the row groups
+    if (RG > 1) {
+      float* pm = part + (size_t)rg * 3 * DC;
+      const int cl0 = ct * 4;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      pm[c0 + k] = mx[k];
-      pm[L.D + c0 + k] = sum[k];
-      pm[2 * L.D + c0 + k] = acc[k];
-    }
-    __syncthreads();
-    if (lead) {
-      for (int q = 1; q < RG; ++q) {
-        const float* po = part + (size_t)q * 3 * L.D;
+      for (int k = 0; k < 4; ++k) {
+        pm[cl0 + k] = mx[k];
+        pm[DC + cl0 + k] = sum[k];
+        pm[2 * DC + cl0 + k] = acc[k];
+      }
+      __syncthreads();
+      if (lead) {
+        // max over the groups first, then independent exp2 terms (no serial rescale chain)
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const float m2 = po[c0 + k];
-          if (m2 == -INFINITY) continue;
-          const float M = fmaxf(mx[k], m2);
-          const float f1 = exp2f(mx[k] - M), f2 = exp2f(m2 - M);
-          sum[k] = sum[k] * f1 + po[L.D + c0 + k] * f2;
-          acc[k] = acc[k] * f1 + po[2 * L.D + c0 + k] * f2;
+          float M = mx[k];
+          for (int qq = 1; qq < RG; ++qq) M = fmaxf(M, part[(size_t)qq * 3 * DC + cl0 + k]);
+          float sm = sum[k] * exp2f(mx[k] - M), ac = acc[k] * exp2f(mx[k] - M);
+          for (int qq = 1; qq < RG; ++qq) {
+            const float* po = part + (size_t)qq * 3 * DC;
+            const float m2 = po[cl0 + k];
+            const float f = m2 == -INFINITY ? 0.f : exp2f(m2 - M);
+            sm += po[DC + cl0 + k] * f;
+            ac += po[2 * DC + cl0 + k] * f;
+          }
+          sum[k] = sm;
+          acc[k] = ac;
           mx[k] = M;
         }
       }
     }
-  }
-  float e[4] = {0.f, 0.f, 0.f, 0.f};
-  float ss = 0.f;
-  if (lead) {
+    CTRACE(5);
+    float e[4] = {0.f, 0.f, 0.f, 0.f};
+    float ss = 0.f;
+    if (lead) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) { e[k] = acc[k] / sum[k]; ss += e[k] * e[k]; }
+      for (int k = 0; k < 4; ++k) { e[k] = acc[k] / sum[k]; ss += e[k] * e[k]; }
+    }
+    ss = cluster_reduce(block_sum(ss, scratch), &red[1], &bcast, false);
+    const float rs = 1.0f / sqrtf(ss / (float)L.D + L.eps);
+    const float4 gk = a.gamma_kv ? __ldg(reinterpret_cast<const float4*>(a.gamma_kv + c0)) : make_float4(1.f, 1.f, 1.f, 1.f);
+    e[0] *= rs * gk.x; e[1] *= rs * gk.y; e[2] *= rs * gk.z; e[3] *= rs * gk.w;
+    CTRACE(6);
+    rope4(e, c0, L, (double)(L.pos0 + i * (int64_t)L.m));
+    CTRACE(7);
+    float am = 0.f;
+    if (L.kv_fmt == CSA_FMT_MIXED) am = cluster_reduce(block_max(local_amax(e, c0, dn, lead), scratch), &red[2], &bcast, true);
+    uint8_t* dst = C.entries + ((size_t)b * C.entry_cap + (size_t)i) * L.row_bytes;
+    pack_slice(dst, L, c0, e, lead, am, q == 0);
+    CTRACE(8);
   }
-  ss = block_sum(ss, scratch);
-  const float rs = 1.0f / sqrtf(ss / (float)L.D + L.eps);
-  const float4 gk = a.gamma_kv ? __ldg(reinterpret_cast<const float4*>(a.gamma_kv + c0)) : make_float4(1.f, 1.f, 1.f, 1.f);
-  e[0] *= rs * gk.x; e[1] *= rs * gk.y; e[2] *= rs * gk.z; e[3] *= rs * gk.w;
-  rope4(e, c0, L, (double)(L.pos0 + i * (int64_t)L.m));
-  uint8_t* dst = C.entries + ((size_t)b * C.entry_cap + (size_t)i) * L.row_bytes;
-  pack_row(dst, L, c0, e, lead, scratch);
+  // no CTA may leave while a peer can still read its shared memory
+  cluster.sync();
 }
 
 }  // namespace
 
+#ifdef CSA_TRACE
+extern "C" __attribute__((visibility("default"))) int csa_trace_read_c(uint64_t* host) {
+  return (int)cudaMemcpyFromSymbol(host, g_trace_c, sizeof(g_trace_c));
+}
+#endif
+
 cudaError_t launch_append_compress(const AppendCompressArgs& a, int B, int Tq, cudaStream_t s) {
-  dim3 grid(Tq, B);
-  const int ct = a.L.D / 4;
-  // decode: spread the entry's source rows over row groups; a chunk has parallelism across tokens
-  int rg = 1;
-  if (a.do_compress && Tq <= 64) {
-    const int rows = (1 + a.L.ov) * a.L.m;
-    rg = 512 / ct;
-    while (rg > 1 && (rg / 2) * kRowBatch >= rows) rg /= 2;
+  // decode (few tokens): a cluster of CL CTAs per token splits the channels, and row groups split
+  // the entry's source rows; a chunk has parallelism across tokens and runs one CTA per token.
+  const bool spread = Tq <= 64;
+  int CL = 1;
+  if (spread) {
+    CL = a.L.D / 64;
+    if (CL > 8) CL = 8;
+    if (CL < 1) CL = 1;
   }
-  const size_t smem = rg > 1 ? (size_t)rg * 3 * a.L.D * sizeof(float) : 0;
+  const int ct = a.L.D / CL / 4;
+  int rg = 1;
+  if (spread && a.do_compress) {
+    const int rows = (1 + a.L.ov) * a.L.m;
+    rg = rows < 16 ? rows : 16;
+    while (rg > 1 && ct * rg > 512) rg >>= 1;
+  }
+  const size_t smem = rg > 1 ? (size_t)rg * 3 * (a.L.D / CL) * sizeof(float) : 0;
   static size_t configured = 0;
   if (smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(append_compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = smem;
   }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(Tq * CL), (unsigned)B, 1);
+  cfg.blockDim = dim3((unsigned)(ct * rg), 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   profile_mark(s);
-  append_compress_kernel<<<grid, ct * rg, smem, s>>>(a);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, append_compress_kernel, a, CL);
   note_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace csa

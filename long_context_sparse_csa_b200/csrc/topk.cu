@@ -52,20 +52,26 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, 
 // where above(b) counts the bins above b.  Every thread gets (bin, above).
 __device__ __forceinline__ void find_bin(const uint32_t* hist, int nb, uint32_t need, uint32_t* wsum,
                                          uint32_t* s_bin, uint32_t* s_above) {
+  constexpr int kMaxPer = 8;                 // nb <= 8 * blockDim.x
   const int per = (nb + blockDim.x - 1) / blockDim.x;
-  uint32_t c_local = 0;
-  for (int q = 0; q < per; ++q) {
+  uint32_t c[kMaxPer];
+#pragma unroll
+  for (int q = 0; q < kMaxPer; ++q) {        // all loads first (hist may live in global memory)
     const int bin = nb - 1 - per * (int)threadIdx.x - q;
-    if (bin >= 0) c_local += hist[bin];
+    c[q] = (q < per && bin >= 0) ? hist[bin] : 0u;
   }
+  uint32_t c_local = 0;
+#pragma unroll
+  for (int q = 0; q < kMaxPer; ++q) c_local += c[q];
   uint32_t tot;
   uint32_t above = block_excl_scan(c_local, wsum, &tot);
-  for (int q = 0; q < per; ++q) {
+#pragma unroll
+  for (int q = 0; q < kMaxPer; ++q) {
     const int bin = nb - 1 - per * (int)threadIdx.x - q;
-    if (bin < 0) break;
-    const uint32_t h = hist[bin];
-    if (above < need && need <= above + h) { *s_bin = (uint32_t)bin; *s_above = above; }
-    above += h;
+    if (q < per && bin >= 0) {
+      if (above < need && need <= above + c[q]) { *s_bin = (uint32_t)bin; *s_above = above; }
+      above += c[q];
+    }
   }
   __syncthreads();
 }
@@ -151,6 +157,14 @@ __global__ void __launch_bounds__(kThreads, 1) topk_rows_kernel(const __grid_con
 // candidates (appended to `cand`).  The last CTA of the row to finish (a ticket counter, no
 // waiting) resolves the candidates with two 10-bit radix passes, marks the selection in a
 // shared-memory bitmap over the row's indices, and emits it in ascending index order.
+#ifdef CSA_TRACE
+__device__ uint64_t g_trace_t[80][24];
+#define TTRACE(slot) do { if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.x < 80) { \
+    uint64_t _t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(_t) :: "memory"); g_trace_t[blockIdx.x][(slot)] = _t; } } while (0)
+#else
+#define TTRACE(slot) ((void)0)
+#endif
+
 constexpr int kSplitThreads = 512;
 constexpr int kHistBins = 4096;
 constexpr int kChunk = 4096;                  // scores per filtering chunk
@@ -179,9 +193,11 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
   int32_t* sure = a.sure + (size_t)row * k;
   uint2* cand = a.cand + (size_t)row * A.n_max;
 
+  TTRACE(0);
   // ---------------------------------------------------------------- 1. bin of the k-th largest key
   find_bin(a.hist + (size_t)row * kHistBins, kHistBins, (uint32_t)k, wsum, &s_bin, &s_above);
   const uint32_t bstar = s_bin;
+  TTRACE(1);
 
   // ---------------------------------------------------------------- 2. filter this CTA's slice
   // Chunks of kChunk scores: appends go to shared-memory buffers, then one global atomic per
@@ -199,27 +215,29 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
     float vals[kPer];
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
-      const int i = cb + u * kSplitThreads + tid;
+      const int i = cb + tid * kPer + u;           // a thread's kPer consecutive scores
       vals[u] = i < ce ? __ldg(sc + i) : 0.f;
     }
+    uint32_t keys[kPer], ns = 0, nc2 = 0;
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
-      const int i = cb + u * kSplitThreads + tid;
-      uint32_t key = 0, bin = 0;
-      const bool in = i < ce;
-      if (in) { key = float_key(vals[u]); bin = key >> 20; }
-      const bool is_sure = in && bin > bstar, is_cand = in && bin == bstar;
-      const uint32_t ms = __ballot_sync(0xffffffffu, is_sure), mc = __ballot_sync(0xffffffffu, is_cand);
-      uint32_t ps = 0, pc = 0;
-      if (lane == 0) {
-        if (ms) ps = atomicAdd(&s_ns, (uint32_t)__popc(ms));
-        if (mc) pc = atomicAdd(&s_nc, (uint32_t)__popc(mc));
-      }
-      ps = __shfl_sync(0xffffffffu, ps, 0);
-      pc = __shfl_sync(0xffffffffu, pc, 0);
-      if (is_sure) b_sure[ps + __popc(ms & lt_mask)] = i;
-      if (is_cand) b_cand[pc + __popc(mc & lt_mask)] = make_uint2(key, (uint32_t)i);
+      const int i = cb + tid * kPer + u;
+      keys[u] = float_key(vals[u]);
+      const uint32_t bin = keys[u] >> 20;
+      ns += (i < ce && bin > bstar);
+      nc2 += (i < ce && bin == bstar);
     }
+    uint32_t tot2;
+    const uint32_t ex = block_excl_scan(ns | (nc2 << 16), wsum, &tot2);
+    uint32_t ps = ex & 0xFFFFu, pc = ex >> 16;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = cb + tid * kPer + u;
+      const uint32_t bin = keys[u] >> 20;
+      if (i < ce && bin > bstar) b_sure[ps++] = i;
+      if (i < ce && bin == bstar) b_cand[pc++] = make_uint2(keys[u], (uint32_t)i);
+    }
+    if (tid == 0) { s_ns = tot2 & 0xFFFFu; s_nc = tot2 >> 16; }
     __syncthreads();
     if (tid == 0) {
       s_gs = s_ns ? atomicAdd(cnt + 0, s_ns) : 0u;
@@ -231,6 +249,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
     __syncthreads();
   }
 
+  TTRACE(2);
   // ---------------------------------------------------------------- 3. last CTA of the row resolves
   __syncthreads();
   if (tid == 0) {
@@ -238,10 +257,15 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
     s_last = atomicAdd(cnt + 2, 1u) == gridDim.x - 1 ? 1u : 0u;
   }
   __syncthreads();
+  TTRACE(3);
   if (!s_last) return;
   __threadfence();
-  const uint32_t n_sure = atomicAdd(cnt + 0, 0u), nc = atomicAdd(cnt + 1, 0u);
+  const uint32_t n_sure = __ldcg(cnt + 0), nc = __ldcg(cnt + 1);   // after the fence: every CTA's appends
   uint32_t rem = (uint32_t)k - n_sure;        // >= 1: fewer than k keys lie above b*
+#ifdef CSA_TRACE
+  if (tid == 0 && blockIdx.x < 80) { g_trace_t[blockIdx.x][8] = n_sure; g_trace_t[blockIdx.x][9] = nc; }
+#endif
+  TTRACE(10);
   const int nw = (nv + 31) >> 5;
   uint32_t* sel = bm;
   uint32_t* eqm = bm + nw;
@@ -253,6 +277,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
   const uint2* cv = staged ? cs : cand;
   for (int i = tid; i < 2 * nw; i += kSplitThreads) bm[i] = 0u;
   __syncthreads();
+  TTRACE(4);
 
   // two 10-bit radix passes over the candidates' low 20 bits pin the exact key T
   uint32_t prefix = bstar;
@@ -273,6 +298,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
     __syncthreads();
   }
   const uint32_t T = prefix;                   // keys > T are taken; `rem` keys == T, smallest indices
+  TTRACE(5);
 
   for (uint32_t j = tid; j < n_sure; j += kSplitThreads) {
     const uint32_t i = (uint32_t)sure[j];
@@ -285,38 +311,95 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
   }
   __syncthreads();
 
-  // ordered emission: thread t owns words [t*wpt, (t+1)*wpt)
-  const int wpt = (nw + kSplitThreads - 1) / kSplitThreads;
-  const int w_lo = min(tid * wpt, nw), w_hi = min(w_lo + wpt, nw);
-  uint32_t eq_local = 0;
-  for (int wd = w_lo; wd < w_hi; ++wd) eq_local += __popc(eqm[wd]);
+  TTRACE(6);
+  // ordered emission.  Warp w owns words [w*CW, (w+1)*CW), CW a multiple of 256; in round i lane l
+  // holds the 8 consecutive words w*CW + 256i + 8l .. +7 (two 128-bit loads, no bank conflicts),
+  // and one warp scan per round orders the lanes.
+  const int nwarps = kSplitThreads / 32, wid = tid >> 5;
+  const int CW = ((nw + nwarps - 1) / nwarps + 255) & ~255;
+  const int wbeg = wid * CW, wend = min(wbeg + CW, nw);
+  auto load8 = [&](const uint32_t* bmp, int w0, uint32_t v[8]) {
+    if (w0 + 8 <= nw) {
+      const uint4 x = *reinterpret_cast<const uint4*>(bmp + w0), y = *reinterpret_cast<const uint4*>(bmp + w0 + 4);
+      v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w; v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = (w0 + q < nw) ? bmp[w0 + q] : 0u;
+    }
+  };
+  uint32_t eq_w = 0;
+  for (int base = wbeg; base < wend; base += 256) {
+    uint32_t v[8];
+    load8(eqm, base + 8 * lane, v);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) eq_w += __popc(v[q]);
+  }
+  eq_w = __reduce_add_sync(0xffffffffu, eq_w);
   uint32_t tot;
-  uint32_t eq_before = block_excl_scan(eq_local, wsum, &tot);
-  uint32_t n_local = 0;
-  for (int wd = w_lo; wd < w_hi; ++wd) {
-    uint32_t e = eqm[wd], keep = 0;
-    while (e && eq_before < rem) {
-      const uint32_t low = e & (0u - e);
-      keep |= low;
-      e ^= low;
-      ++eq_before;
+  uint32_t eq_before = block_excl_scan(lane == 0 ? eq_w : 0u, wsum, &tot);
+  eq_before = __shfl_sync(0xffffffffu, eq_before, 0);
+  TTRACE(11);
+  uint32_t sel_w = 0;
+  for (int base = wbeg; base < wend; base += 256) {
+    const int w0 = base + 8 * lane;
+    uint32_t e[8], sv[8];
+    load8(eqm, w0, e);
+    load8(sel, w0, sv);
+    uint32_t pe = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) pe += __popc(e[q]);
+    const uint32_t inc = warp_incl_scan(pe, lane);
+    uint32_t before = eq_before + inc - pe;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint32_t keep = 0, ew = e[q];
+      while (ew && before < rem) {
+        const uint32_t low = ew & (0u - ew);
+        keep |= low;
+        ew ^= low;
+        ++before;
+      }
+      before += __popc(ew);
+      if (keep && w0 + q < nw) sel[w0 + q] = sv[q] | keep;
+      sel_w += __popc(sv[q] | keep);
     }
-    eq_before += __popc(e);
-    sel[wd] |= keep;
-    n_local += __popc(sel[wd]);
+    eq_before += __shfl_sync(0xffffffffu, inc, 31);
   }
-  uint32_t pos = block_excl_scan(n_local, wsum, &tot);
-  for (int wd = w_lo; wd < w_hi; ++wd) {
-    uint32_t b = sel[wd];
-    while (b) {
-      const int bit = __ffs(b) - 1;
-      b &= b - 1;
-      out[pos++] = wd * 32 + bit;
+  TTRACE(12);
+  sel_w = __reduce_add_sync(0xffffffffu, sel_w);
+  uint32_t pos0 = block_excl_scan(lane == 0 ? sel_w : 0u, wsum, &tot);
+  pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+  TTRACE(13);
+  for (int base = wbeg; base < wend; base += 256) {
+    const int w0 = base + 8 * lane;
+    uint32_t v[8];
+    load8(sel, w0, v);
+    uint32_t pb = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) pb += __popc(v[q]);
+    const uint32_t inc = warp_incl_scan(pb, lane);
+    uint32_t pos = pos0 + inc - pb;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint32_t bits = v[q];
+      while (bits) {
+        const int bit = __ffs(bits) - 1;
+        bits &= bits - 1;
+        out[pos++] = (w0 + q) * 32 + bit;
+      }
     }
+    pos0 += __shfl_sync(0xffffffffu, inc, 31);
   }
+  TTRACE(7);
 }
 
 }  // namespace
+
+#ifdef CSA_TRACE
+extern "C" __attribute__((visibility("default"))) int csa_trace_read_t(uint64_t* host) {
+  return (int)cudaMemcpyFromSymbol(host, g_trace_t, sizeof(g_trace_t));
+}
+#endif
 
 int topk_split_ctas(int rows, int64_t n_max, int num_sms) {
   int64_t g = (2 * (int64_t)num_sms + rows - 1) / rows;
