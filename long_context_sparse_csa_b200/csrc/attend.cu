@@ -31,6 +31,14 @@ namespace {
 constexpr int kD = 512;
 constexpr int kTile = 64;
 
+#ifdef CSA_TRACE
+__device__ uint64_t g_trace_a[320][16];
+#define ATRACE(slot) do { if (threadIdx.x == 0 && blockIdx.z == 0 && blockIdx.y == 0 && blockIdx.x < 320) { \
+    uint64_t _t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(_t) :: "memory"); g_trace_a[blockIdx.x][(slot)] = _t; } } while (0)
+#else
+#define ATRACE(slot) ((void)0)
+#endif
+
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -135,6 +143,7 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
   const int64_t T = (si.R + kTile - 1) / kTile;
   const int64_t t0 = T * sp / a.splits, t1 = T * (sp + 1) / a.splits;
   const float cl2 = L.scale * kLog2e;
+  ATRACE(0);
 
   if (tid < 32) {
     float c, s;
@@ -188,7 +197,9 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
   __syncthreads();
 
   const int mt = warp >> 2, np = warp & 3;   // S-phase tile of this warp: heads mt*16.., slots np*16..
-  for (int64_t tile = t0; tile < t1; ++tile) {
+  ATRACE(1);
+  int ti = 0;
+  for (int64_t tile = t0; tile < t1; ++tile, ++ti) {
     const int64_t s0 = tile * kTile;
     if (tid < kTile) rowptr[tid] = slot_row(a, si, row, b, s0 + tid);
     __syncthreads();
@@ -252,6 +263,7 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
       }
     }
     __syncthreads();
+    if (ti < 2) ATRACE(2 + 4 * ti);
 
     // ------------------------------------------------------------ S = Q K^T for (heads mt*16.., slots np*16..)
     float sacc[2][4];
@@ -282,6 +294,7 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
         sacc[nt][i] = v;
         if (i < 2) pm0 = fmaxf(pm0, v); else pm1 = fmaxf(pm1, v);
       }
+    if (ti < 2) ATRACE(3 + 4 * ti);
     pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, 1));
     pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, 2));
     pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, 1));
@@ -331,6 +344,7 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
     if (tid < HG)
       l_run[tid] = l_run[tid] * corr[tid] + (psum[tid] + psum[HG + tid]) + (psum[2 * HG + tid] + psum[3 * HG + tid]);
 
+    if (ti < 2) ATRACE(4 + 4 * ti);
     // ------------------------------------------------------------ O = O * corr + P V (warp owns dims warp*DW..)
 #pragma unroll
     for (int m2 = 0; m2 < MT; ++m2) {
@@ -368,6 +382,7 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
     __syncthreads();
   }
 
+  ATRACE(10);
   // ---------------------------------------------------------------- epilogue
   if (a.splits > 1) {
     float* part = a.part + (((size_t)row * (L.H / HG) + hg) * a.splits + sp) * (size_t)(HG * (kD + 2));
@@ -384,6 +399,7 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
       part[HG * kD + tid] = m_run[tid];
       part[HG * kD + HG + tid] = l_run[tid];
     }
+    ATRACE(11);
     return;
   }
   // single split: merge the sink, normalise, rotate back by -t, store
@@ -582,6 +598,12 @@ __global__ void attend_generic_kernel(const __grid_constant__ AttendArgs a) {
     else reinterpret_cast<uint16_t*>(dst)[d] = f_to_bf16_bits(o[k]);
   }
 }
+
+#ifdef CSA_TRACE
+extern "C" __attribute__((visibility("default"))) int csa_trace_read_a(uint64_t* host) {
+  return (int)cudaMemcpyFromSymbol(host, g_trace_a, sizeof(g_trace_a));
+}
+#endif
 
 template <int HG>
 size_t mma_smem_bytes() {

@@ -267,15 +267,16 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
 #endif
   TTRACE(10);
   const int nw = (nv + 31) >> 5;
+  const int nw4 = (nw + 3) & ~3;               // keeps the second bitmap 16-byte aligned
   uint32_t* sel = bm;
-  uint32_t* eqm = bm + nw;
+  uint32_t* eqm = bm + nw4;
   // candidates are read three times below: stage them in shared memory when they fit
-  uint2* cs = reinterpret_cast<uint2*>(bm + 2 * (((A.n_max + 31) >> 5)));
+  uint2* cs = reinterpret_cast<uint2*>(bm + 2 * ((((A.n_max + 31) >> 5) + 3) & ~(int64_t)3));
   const bool staged = nc <= (uint32_t)kCandCap;
   if (staged)
     for (uint32_t j = tid; j < nc; j += kSplitThreads) cs[j] = cand[j];
   const uint2* cv = staged ? cs : cand;
-  for (int i = tid; i < 2 * nw; i += kSplitThreads) bm[i] = 0u;
+  for (int i = tid; i < 2 * nw4; i += kSplitThreads) bm[i] = 0u;
   __syncthreads();
   TTRACE(4);
 
@@ -411,7 +412,7 @@ int topk_split_ctas(int rows, int64_t n_max, int num_sms) {
 
 cudaError_t launch_topk_split(const TopkSplitArgs& a, cudaStream_t s) {
   if (a.base.rows <= 0 || a.base.k <= 0) return cudaSuccess;
-  size_t smem = 2 * (size_t)((a.base.n_max + 31) / 32) * 4 + (size_t)kCandCap * 8;
+  size_t smem = 2 * (size_t)((((a.base.n_max + 31) / 32) + 3) & ~(int64_t)3) * 4 + (size_t)kCandCap * 8;
   if (smem < (size_t)kChunk * 12) smem = (size_t)kChunk * 12;
   static size_t configured = 0;
   if (smem > configured) {
