@@ -12,7 +12,8 @@ and a device synchronisation, timed with CUDA events on the launching stream,
 max over ranks.  Each step runs on the next of R independent layer instances
 (caches at distinct addresses), so a step never finds its keys in L2 (R=8:
 >= 280 MB streamed between two uses of one instance vs 126 MB of L2).
-Steps are CUDA-graph replays of the public API calls.
+Steps are CUDA-graph replays of the public API calls; the only event nodes in
+the timed graphs bracket one indexer launch per cycle (the roofline sample).
 
 `value` = tokens x attention layers processed by all ranks / time (tok/s per
 attention layer).  `e2e` repeats the measurement with each step's inputs
@@ -313,27 +314,25 @@ def run_ours(args):
     ev = lambda: torch.cuda.Event(enable_timing=True, external=True)  # noqa: E731
     stream = torch.cuda.Stream(device=dev)
 
-    def capture(rs, with_events):
-        """One CUDA graph running the steps of instances rs in order; optional per-step events."""
-        evs = []
-        if with_events:
-            for _ in rs:
-                e = {"idx": (ev(), ev()), "lay": [(ev(), ev()) for _ in layers]}
-                for x in list(e["idx"]) + [y for p in e["lay"] for y in p]:
-                    x.record()
-                evs.append(e)
+    def capture(rs, idx_events):
+        """One CUDA graph running the steps of instances rs in order.  With idx_events, a pair of
+        events brackets the indexer-score launch of the first step (the only event nodes: each one
+        breaks the chain of kernel nodes and costs a few microseconds)."""
+        pair = None
+        if idx_events:
+            pair = (ev(), ev())
+            for x in pair:
+                x.record()
             torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         n0 = C.csa_launch_count()
         with torch.cuda.graph(g, stream=stream):
             for j, r in enumerate(rs):
                 for li, lay in enumerate(layers):
-                    if with_events:
-                        evs[j]["lay"][li][0].record()
                     io, spec = lay["io"], lay["spec"]
                     if spec.kind == "csa":
-                        if with_events:
-                            C.csa_profile_events(*evs[j]["idx"])
+                        if idx_events and j == 0:
+                            C.csa_profile_events(*pair)
                         C.csa_decode_step(lay["L"], lay["caches"][r], lay["params"], io["q"], io["idx_q"],
                                           io["idx_q_scale"], io["head_w"], io["x_new"], io["g_new"], io["t"],
                                           io["out"], io["topk"], lay["ws"])
@@ -341,19 +340,20 @@ def run_ours(args):
                     else:
                         C.hca_decode_step(lay["L"], lay["caches"][r], lay["params"], io["q"], io["x_new"],
                                           io["g_new"], io["t"], io["out"], lay["ws"])
-                    if with_events:
-                        evs[j]["lay"][li][1].record()
-        return g, evs, C.csa_launch_count() - n0
+        return g, pair, C.csa_launch_count() - n0
 
-    cycle, cycle_ev, n_launch = capture(list(range(R)), True)
-    launches_per_step = n_launch // R
+    # n_cyc copies of the cycle graph, replayed round-robin: the last replay of each copy lies in the
+    # timed region, so its event pair samples one indexer launch of the timed steps
+    n_cyc = max(1, min(8, args.steps // R))
+    cycles = [capture(list(range(R)), has_csa) for _ in range(n_cyc)]
+    launches_per_step = cycles[0][2] // R
     singles = [capture([r], False)[0] for r in range(R)]
     torch.cuda.synchronize()
 
     def run_steps(k):
         """Exactly k decode steps: whole cycles of the R instances, then single steps."""
-        for _ in range(k // R):
-            cycle.replay()
+        for c in range(k // R):
+            cycles[c % n_cyc][0].replay()
         for r in range(k % R):
             singles[r].replay()
 
@@ -375,7 +375,7 @@ def run_ours(args):
     run_steps(args.warmup)
     t_burn = time.perf_counter()
     while time.perf_counter() - t_burn < args.burn_seconds:
-        cycle.replay()
+        cycles[0][0].replay()
         torch.cuda.synchronize()
     torch.cuda.synchronize()
     barrier()
@@ -392,13 +392,11 @@ def run_ours(args):
     barrier()
     T_ms = max_over_ranks(e0.elapsed_time(e1))
     clk = clocks.summary(w0, w1)
-    # per-kernel / per-layer device times: the last replay of the cycle graph (one step per instance);
-    # the burn above replayed it after the warm-up, so these are steady-state launches
-    idx_ms = [e["idx"][0].elapsed_time(e["idx"][1]) for e in cycle_ev] if has_csa else []
-    lay_ms = [[e["lay"][li][0].elapsed_time(e["lay"][li][1]) for e in cycle_ev] for li in range(len(layers))]
+    # indexer launch durations sampled inside the timed region (one per cycle-graph copy)
+    idx_ms = [c[1][0].elapsed_time(c[1][1]) for c in cycles] if has_csa else []
 
     # ------------------------------------------------------------------ per-kernel timeline (diagnostic, untimed)
-    labels = {"csa": ["append+compress", "histogram reset", "indexer scores", "top-k", "attention", "combine"],
+    labels = {"csa": ["append+compress", "indexer scores", "top-k", "attention", "combine"],
               "hca": ["append+compress", "attention", "combine"]}
     tl_events = []
     g_tl = torch.cuda.CUDAGraph()
@@ -483,7 +481,6 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": T_ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e4m3+bf16 (fp32 accumulate)", "data": "synthetic",
             "config": workload_config(wl, R)}
-    line["per_layer_us"] = {f"{l['spec'].kind}{li}": 1e3 * float(np.mean(lay_ms[li])) for li, l in enumerate(layers)}
     peaks = {}
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -501,11 +498,11 @@ def run_ours(args):
         line["roofline"] = {"bound": "hbm", "kernel": "index_score_tc_kernel", "achieved": achieved, "peak": peak,
                             "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_note,
                             "traffic": recorded_traffic(wl.name), "algorithmic_bytes": bytes_idx,
-                            "launch_us": 1e6 * t_idx}
+                            "launch_us": 1e6 * t_idx, "launches_sampled": len(idx_ms)}
     else:
         spec = layers[0]["spec"]
         b = step_bytes(spec, wl.n, wl.B)
-        t = float(np.mean(lay_ms[0])) / 1e3
+        t = T_ms / args.steps / 1e3
         line["roofline"] = {"bound": "hbm", "kernel": "hca layer step", "achieved": b / t / 1e9, "peak": peak,
                             "unit": "GB/s", "frac": b / t / 1e9 / peak, "peak_source": peak_note, "traffic": None,
                             "algorithmic_bytes": b}
@@ -525,7 +522,7 @@ def run_ours(args):
                                 "sample": f"{len(times)} full decode steps of the workload ({args.cpu_seconds:.0f} s budget)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del cycle, singles
+    del cycles, singles
     if world > 1:
         dist.destroy_process_group()
 

@@ -38,8 +38,9 @@
  *     a wait that gives up sets a bit in the workspace's device error word,
  *     read back by csa_device_error().
  *   - Workspace: csa_workspace_size() bytes of device memory, zero-filled by
- *     the caller before its FIRST use (the library leaves its counters at zero
- *     after every call).  Concurrent calls must not share a workspace.
+ *     the caller before its FIRST use (the library leaves its counters and
+ *     histograms at zero after every call; zero it again after a device
+ *     error).  Concurrent calls must not share a workspace.
  *   - Positions: q_pos[b * Tq + j] (device int64) is the absolute position t
  *     of query token j of sequence b; raw row index r = t - pos0.
  *

@@ -222,12 +222,8 @@ csa_status_t run_index_topk(const csa_layer_t* L, const csa_cache_t* cache, cons
   int* err = reinterpret_cast<int*>(at(ws, w.err));
   const bool split = use_split_topk(L, Tq, n_max);
   const int rows = L->B * Tq;
+  // the split top-k leaves its histogram and counters zeroed; the caller zero-fills the workspace once
   uint32_t* hist = split ? reinterpret_cast<uint32_t*>(at(ws, w.hist)) : nullptr;
-  if (split) {
-    profile_mark(s);
-    cudaError_t e = cudaMemsetAsync(hist, 0, w.hist_bytes, s);
-    if (e != cudaSuccess) return cuda_fail(e, "histogram reset");
-  }
   IndexArgs a;
   memset(&a, 0, sizeof(a));
   a.B = L->B; a.Tq = Tq; a.H_I = L->H_I; a.d_I = L->d_I; a.m = L->m;
@@ -258,6 +254,7 @@ csa_status_t run_index_topk(const csa_layer_t* L, const csa_cache_t* cache, cons
     sa.sure = reinterpret_cast<int32_t*>(at(ws, w.sure));
     sa.cand = reinterpret_cast<uint2*>(at(ws, w.cand));
     sa.G = topk_split_ctas(rows, n_max, num_sms());
+    sa.err = err;
     e = launch_topk_split(sa, s);
   } else {
     e = launch_topk(t, s);

@@ -154,37 +154,125 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
   if (tid < HG) { m_run[tid] = -INFINITY; l_run[tid] = 0.f; }
   __syncthreads();
 
-  // ---------------------------------------------------------------- q~ = RoPE_t(RMSNorm(q) * gamma_q), bf16
-  const size_t ab = L.act_fmt == CSA_FMT_F32 ? 4 : 2;
-  for (int hh = warp; hh < HG; hh += NW) {
-    const int h = hg * HG + hh;
-    const uint8_t* qrow = a.q + ((size_t)row * L.H + h) * kD * ab;
-    float v[16];
+  // ---------------------------------------------------------------- key/value tile gather
+  // gather_load issues every 16-byte load of a 64-row tile into registers; gather_store converts
+  // (FP8 codes x the row's power-of-two scale -> bf16, exact) into the swizzled shared tile.  The
+  // first tile's loads are issued before the query prologue so their latency is hidden by it.
+  constexpr int kChunksRow = FMT == CSA_FMT_BF16 ? 64 : 36;
+  constexpr int kPer = (kTile * kChunksRow + NT - 1) / NT;
+  struct Gl { uint4 c[kPer]; float sig[kPer]; };
+  auto gather_load = [&](Gl& g) {
 #pragma unroll
-    for (int k = 0; k < 16; k += 4) load_act4(qrow, L.act_fmt, 16 * lane + k, v + k);
-    float ss = 0.f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) ss += v[k] * v[k];
-    ss = warp_sum(ss);
-    const float rs = 1.0f / sqrtf(ss / (float)kD + L.eps);
-#pragma unroll
-    for (int k = 0; k < 16; ++k) v[k] *= rs * (a.gamma_q ? a.gamma_q[16 * lane + k] : 1.f);
-    if (lane >= 28) {
-#pragma unroll
-      for (int k = 0; k < 16; k += 2) {
-        const int u = (16 * lane + k - (kD - 64)) >> 1;
-        const float x0 = v[k], x1 = v[k + 1];
-        v[k] = x0 * cs[u] - x1 * sn[u];
-        v[k + 1] = x0 * sn[u] + x1 * cs[u];
+    for (int u = 0; u < kPer; ++u) {
+      const int idx = tid + u * NT;
+      g.c[u] = make_uint4(0u, 0u, 0u, 0u);
+      g.sig[u] = 0.f;
+      if (idx < kTile * kChunksRow) {
+        const int rr = idx / kChunksRow, ch = idx % kChunksRow;
+        const uint8_t* p = rowptr[rr];
+        if (p) {
+          if (FMT == CSA_FMT_BF16) {
+            g.c[u] = ldg_nc_v4(p + ch * 16);
+          } else {
+            g.c[u] = ldg_nc_v4(p + (ch < 28 ? ch * 16 : (kD - 64) + (ch - 28) * 16));
+            if (ch < 28) g.sig[u] = __ldg(reinterpret_cast<const float*>(p + kD + 64));
+          }
+        }
       }
     }
-    uint4 p0, p1;
-    p0.x = pack_bf16x2(v[0], v[1]); p0.y = pack_bf16x2(v[2], v[3]);
-    p0.z = pack_bf16x2(v[4], v[5]); p0.w = pack_bf16x2(v[6], v[7]);
-    p1.x = pack_bf16x2(v[8], v[9]); p1.y = pack_bf16x2(v[10], v[11]);
-    p1.z = pack_bf16x2(v[12], v[13]); p1.w = pack_bf16x2(v[14], v[15]);
-    *reinterpret_cast<uint4*>(Qs + swz(hh, 2 * lane, 1024)) = p0;
-    *reinterpret_cast<uint4*>(Qs + swz(hh, 2 * lane + 1, 1024)) = p1;
+  };
+  auto gather_store = [&](const Gl& g) {
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int idx = tid + u * NT;
+      if (idx >= kTile * kChunksRow) break;
+      const int rr = idx / kChunksRow, ch = idx % kChunksRow;
+      if (FMT == CSA_FMT_BF16) {
+        *reinterpret_cast<uint4*>(Ks + swz(rr, ch, 1024)) = g.c[u];
+      } else if (ch < 28) {
+        const uint32_t w[4] = {g.c[u].x, g.c[u].y, g.c[u].z, g.c[u].w};
+        uint32_t outw[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 lo = e4m3x2_to_float2((uint16_t)(w[q] & 0xFFFFu));
+          const float2 hi = e4m3x2_to_float2((uint16_t)(w[q] >> 16));
+          outw[2 * q] = pack_bf16x2(lo.x * g.sig[u], lo.y * g.sig[u]);
+          outw[2 * q + 1] = pack_bf16x2(hi.x * g.sig[u], hi.y * g.sig[u]);
+        }
+        *reinterpret_cast<uint4*>(Ks + swz(rr, 2 * ch, 1024)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+        *reinterpret_cast<uint4*>(Ks + swz(rr, 2 * ch + 1, 1024)) = make_uint4(outw[4], outw[5], outw[6], outw[7]);
+      } else {
+        *reinterpret_cast<uint4*>(Ks + swz(rr, 56 + (ch - 28), 1024)) = g.c[u];
+      }
+    }
+  };
+  Gl gl;
+  if (t0 < t1) {
+    if (tid < kTile) rowptr[tid] = slot_row(a, si, row, b, t0 * kTile + tid);
+    __syncthreads();
+    gather_load(gl);
+  }
+
+  // ---------------------------------------------------------------- q~ = RoPE_t(RMSNorm(q) * gamma_q), bf16
+  // Each warp owns HG/NW heads; lane l holds dims [16l, 16l+16).  All of the warp's loads (its
+  // heads' q values and gamma) are issued before any head is normalised.
+  {
+    constexpr int HPW = HG / NW;
+    const size_t ab = L.act_fmt == CSA_FMT_F32 ? 4 : 2;
+    float gm[16];
+    if (a.gamma_q) {
+#pragma unroll
+      for (int k = 0; k < 16; k += 4) {
+        const float4 g4 = __ldg(reinterpret_cast<const float4*>(a.gamma_q + 16 * lane + k));
+        gm[k] = g4.x; gm[k + 1] = g4.y; gm[k + 2] = g4.z; gm[k + 3] = g4.w;
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) gm[k] = 1.f;
+    }
+    float v[HPW][16];
+#pragma unroll
+    for (int i = 0; i < HPW; ++i) {
+      const int h = hg * HG + warp + i * NW;
+      const uint8_t* qrow = a.q + ((size_t)row * L.H + h) * kD * ab;
+      if (L.act_fmt == CSA_FMT_F32) {
+#pragma unroll
+        for (int k = 0; k < 16; k += 4) load_act4(qrow, CSA_FMT_F32, 16 * lane + k, v[i] + k);
+      } else {
+        const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(qrow + 2 * 16 * lane));
+        const uint4 u1 = __ldg(reinterpret_cast<const uint4*>(qrow + 2 * 16 * lane + 16));
+        const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) { v[i][2 * k] = bf16_bits_to_f(w[k] & 0xFFFFu); v[i][2 * k + 1] = bf16_bits_to_f(w[k] >> 16); }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < HPW; ++i) {
+      const int hh = warp + i * NW;
+      float ss = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) ss += v[i][k] * v[i][k];
+      ss = warp_sum(ss);
+      const float rs = 1.0f / sqrtf(ss / (float)kD + L.eps);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) v[i][k] *= rs * gm[k];
+      if (lane >= 28) {
+#pragma unroll
+        for (int k = 0; k < 16; k += 2) {
+          const int u = (16 * lane + k - (kD - 64)) >> 1;
+          const float x0 = v[i][k], x1 = v[i][k + 1];
+          v[i][k] = x0 * cs[u] - x1 * sn[u];
+          v[i][k + 1] = x0 * sn[u] + x1 * cs[u];
+        }
+      }
+      uint4 p0, p1;
+      p0.x = pack_bf16x2(v[i][0], v[i][1]); p0.y = pack_bf16x2(v[i][2], v[i][3]);
+      p0.z = pack_bf16x2(v[i][4], v[i][5]); p0.w = pack_bf16x2(v[i][6], v[i][7]);
+      p1.x = pack_bf16x2(v[i][8], v[i][9]); p1.y = pack_bf16x2(v[i][10], v[i][11]);
+      p1.z = pack_bf16x2(v[i][12], v[i][13]); p1.w = pack_bf16x2(v[i][14], v[i][15]);
+      *reinterpret_cast<uint4*>(Qs + swz(hh, 2 * lane, 1024)) = p0;
+      *reinterpret_cast<uint4*>(Qs + swz(hh, 2 * lane + 1, 1024)) = p1;
+    }
   }
 
   float o[MT][NTW][4];
@@ -200,68 +288,12 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
   ATRACE(1);
   int ti = 0;
   for (int64_t tile = t0; tile < t1; ++tile, ++ti) {
-    const int64_t s0 = tile * kTile;
-    if (tid < kTile) rowptr[tid] = slot_row(a, si, row, b, s0 + tid);
-    __syncthreads();
-
-    // ------------------------------------------------------------ gather the key/value tile (bf16, swizzled)
-    // Every load of the tile is issued before any is consumed, so the row fetches overlap.
-    if (FMT == CSA_FMT_BF16) {
-      constexpr int kPer = kTile * 64 / NT;        // 16-byte chunks per thread
-      uint4 v[kPer];
-#pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const int idx = tid + u * NT, rr = idx >> 6, ch = idx & 63;
-        const uint8_t* p = rowptr[rr];
-        v[u] = p ? ldg_nc_v4(p + ch * 16) : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const int idx = tid + u * NT, rr = idx >> 6, ch = idx & 63;
-        *reinterpret_cast<uint4*>(Ks + swz(rr, ch, 1024)) = v[u];
-      }
-    } else {
-      constexpr int kChunks = kTile * 36;
-      constexpr int kPer = (kChunks + NT - 1) / NT;
-      uint4 c[kPer];
-      float sig[kPer];
-#pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const int idx = tid + u * NT;
-        c[u] = make_uint4(0u, 0u, 0u, 0u);
-        sig[u] = 0.f;
-        if (idx < kChunks) {
-          const int rr = idx / 36, ch = idx % 36;
-          const uint8_t* p = rowptr[rr];
-          if (p) {
-            c[u] = ldg_nc_v4(p + (ch < 28 ? ch * 16 : (kD - 64) + (ch - 28) * 16));
-            if (ch < 28) sig[u] = __ldg(reinterpret_cast<const float*>(p + kD + 64));
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const int idx = tid + u * NT;
-        if (idx >= kChunks) break;
-        const int rr = idx / 36, ch = idx % 36;
-        if (ch < 28) {
-          const uint32_t w[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
-          uint32_t outw[8];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            // e4m3 pairs -> f16 pairs (exact), scale by the row's power of two, round to bf16 (exact)
-            const float2 lo = e4m3x2_to_float2((uint16_t)(w[q] & 0xFFFFu));
-            const float2 hi = e4m3x2_to_float2((uint16_t)(w[q] >> 16));
-            outw[2 * q] = pack_bf16x2(lo.x * sig[u], lo.y * sig[u]);
-            outw[2 * q + 1] = pack_bf16x2(hi.x * sig[u], hi.y * sig[u]);
-          }
-          *reinterpret_cast<uint4*>(Ks + swz(rr, 2 * ch, 1024)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-          *reinterpret_cast<uint4*>(Ks + swz(rr, 2 * ch + 1, 1024)) = make_uint4(outw[4], outw[5], outw[6], outw[7]);
-        } else {
-          *reinterpret_cast<uint4*>(Ks + swz(rr, 56 + (ch - 28), 1024)) = c[u];
-        }
-      }
+    if (tile != t0) {
+      if (tid < kTile) rowptr[tid] = slot_row(a, si, row, b, tile * kTile + tid);
+      __syncthreads();
+      gather_load(gl);
     }
+    gather_store(gl);
     __syncthreads();
     if (ti < 2) ATRACE(2 + 4 * ti);
 
@@ -622,15 +654,9 @@ cudaError_t launch_mma(const AttendArgs& a, cudaStream_t s) {
     configured = true;
   }
   dim3 grid(a.splits, a.L.H / HG, a.rows);
-  profile_mark(s);
-  attend_mma_kernel<HG, FMT><<<grid, HG * 8, smem, s>>>(a);
-  note_launches(1);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(attend_mma_kernel<HG, FMT>, grid, dim3(HG * 8), smem, s, 0, a);
   if (e != cudaSuccess || a.splits == 1) return e;
-  profile_mark(s);
-  attend_combine_kernel<HG><<<dim3(a.L.H, a.rows), 512, 0, s>>>(a);
-  note_launches(1);
-  return cudaGetLastError();
+  return launch_kernel(attend_combine_kernel<HG>, dim3(a.L.H, a.rows), dim3(512), 0, s, 0, a);
 }
 
 }  // namespace
@@ -648,7 +674,8 @@ int attend_num_splits(const LayerArgs& L, int rows, int64_t slots, int num_sms) 
   if (HG == 0) return 1;
   const int64_t pairs = (int64_t)rows * (L.H / HG);
   const int64_t tiles = (slots + kTile - 1) / kTile;
-  int64_t want = (2 * (int64_t)num_sms + pairs - 1) / pairs;
+  // one CTA per SM (the kernel's registers allow no more): a single wave of CTAs
+  int64_t want = ((int64_t)num_sms + pairs - 1) / pairs;
   if (want > tiles) want = tiles;
   if (want < 1) want = 1;
   return (int)want;
@@ -664,10 +691,7 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
   if (a.rows <= 0) return cudaSuccess;
   const int HG = attend_head_group(a.L);
   if (HG == 0) {
-    profile_mark(s);
-    attend_generic_kernel<<<a.rows, a.L.H * 32, 0, s>>>(a);
-    note_launches(1);
-    return cudaGetLastError();
+    return launch_kernel(attend_generic_kernel, dim3(a.rows), dim3(a.L.H * 32), 0, s, 0, a);
   }
   const bool mixed = a.L.kv_fmt == CSA_FMT_MIXED;
   if (HG == 64) return mixed ? launch_mma<64, CSA_FMT_MIXED>(a, s) : launch_mma<64, CSA_FMT_BF16>(a, s);

@@ -150,6 +150,7 @@ __device__ __forceinline__ uint32_t float_key(float f) {
 // ----------------------------------------------------------------------------- error word
 enum : int {
   kErrWaitTimeout = 1,
+  kErrTopkOverflow = 2,     // split top-k: appends exceeded their reserved range (inconsistent histogram)
 };
 
 __device__ __forceinline__ void set_device_error(int* err, int bits) {

@@ -310,22 +310,8 @@ cudaError_t launch_append_compress(const AppendCompressArgs& a, int B, int Tq, c
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(Tq * CL), (unsigned)B, 1);
-  cfg.blockDim = dim3((unsigned)(ct * rg), 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  profile_mark(s);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, append_compress_kernel, a, CL);
-  note_launches(1);
-  return e;
+  return launch_kernel(append_compress_kernel, dim3((unsigned)(Tq * CL), (unsigned)B), dim3((unsigned)(ct * rg)), smem, s,
+                    CL, a, CL);
 }
 
 }  // namespace csa

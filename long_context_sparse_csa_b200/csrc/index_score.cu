@@ -501,10 +501,7 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
                                            (int)sm);
       if (e != cudaSuccess) return e;
     }
-    profile_mark(s);
-    index_score_generic_kernel<<<grid, 128, sm, s>>>(a);
-    note_launches(1);
-    return cudaGetLastError();
+    return launch_kernel(index_score_generic_kernel, grid, dim3(128), sm, s, 0, a);
   }
   a.QN = a.Tq == 1 ? 1 : min(256 / a.H_I, a.Tq);
   const int N = a.QN * a.H_I;
@@ -531,10 +528,7 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
   // decode: two CTAs per SM (two independent pipelines); each CTA's smem and TMEM allow it
   const int64_t ctas = decode ? 2 * (int64_t)num_sms : num_sms;
   const int64_t grid = a.total_items < ctas ? a.total_items : ctas;
-  profile_mark(s);
-  kern<<<(unsigned)grid, kThreads, smem, s>>>(kmap, qmap, a, N, nacc, cols);
-  note_launches(1);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3((unsigned)grid), dim3(kThreads), smem, s, 0, kmap, qmap, a, N, nacc, cols);
 }
 
 }  // namespace csa

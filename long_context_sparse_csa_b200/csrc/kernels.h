@@ -14,6 +14,34 @@ void note_launches(int n);
 // Records the next timeline event (if a timeline is armed on this thread) just before a launch.
 void profile_mark(cudaStream_t s);
 
+// Launches a kernel in stream order, with an optional thread-block cluster size (cluster > 0).
+// (Programmatic dependent launch was measured slower on the decode chain: CTAs parked at the
+// dependency wait take SM slots from the kernel still running.)
+template <typename Kernel, typename... Args>
+cudaError_t launch_kernel(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster,
+                          Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  int n = 0;
+  if (cluster > 0) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = (unsigned)cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  profile_mark(s);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  note_launches(1);
+  return e;
+}
+
 // ----------------------------------------------------------------------------- append + compress
 struct AppendCompressArgs {
   LayerArgs L;
@@ -67,11 +95,12 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 // Decode rows too long for one CTA: many CTAs per row, fed by the indexer's score histogram.
 struct TopkSplitArgs {
   TopkArgs base;
-  const uint32_t* hist;     // [rows][4096] (zeroed before the indexer runs)
+  const uint32_t* hist;     // [rows][4096] (zero on entry; the kernel leaves it zeroed)
   int32_t* sure;            // [rows][k] scratch
   uint2* cand;              // [rows][n_max] scratch
-  uint32_t* cnt;            // [rows][4] counters (zeroed before the indexer runs)
+  uint32_t* cnt;            // [rows][4] counters (zero on entry; left zeroed)
   int G;                    // CTAs per row
+  int* err;                 // device error word
 };
 constexpr int64_t kTopkSplitMinN = 16384;     // rows at least this long use the split kernel
 constexpr int64_t kTopkSplitMaxN = 655360;    // the resolving CTA's bitmaps + staged candidates fit shared memory

@@ -184,9 +184,12 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
   const int nv = (int)nv64;
   const int k = A.k;
   int32_t* out = A.out + (size_t)row * k;
+  uint32_t* hist_row = const_cast<uint32_t*>(a.hist) + (size_t)row * kHistBins;
   if (nv <= k) {
-    if (g == 0)
+    if (g == 0) {
       for (int i = tid; i < k; i += kSplitThreads) out[i] = i < nv ? i : -1;
+      for (int i = tid; i < kHistBins; i += kSplitThreads) hist_row[i] = 0u;   // leave it zeroed for the next call
+    }
     return;
   }
   uint32_t* cnt = a.cnt + (size_t)row * 4;
@@ -242,6 +245,12 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
     if (tid == 0) {
       s_gs = s_ns ? atomicAdd(cnt + 0, s_ns) : 0u;
       s_gc = s_nc ? atomicAdd(cnt + 1, s_nc) : 0u;
+      // a consistent histogram keeps every append in range; anything else is reported, not written
+      if (s_gs + s_ns > (uint32_t)k || s_gc + s_nc > (uint32_t)A.n_max) {
+        set_device_error(a.err, kErrTopkOverflow);
+        s_ns = 0u;
+        s_nc = 0u;
+      }
     }
     __syncthreads();
     for (uint32_t j = tid; j < s_ns; j += kSplitThreads) sure[s_gs + j] = b_sure[j];
@@ -261,6 +270,14 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
   if (!s_last) return;
   __threadfence();
   const uint32_t n_sure = __ldcg(cnt + 0), nc = __ldcg(cnt + 1);   // after the fence: every CTA's appends
+  if (n_sure >= (uint32_t)k || nc > (uint32_t)A.n_max) {   // inconsistent histogram: report, emit nothing
+    if (tid == 0) {
+      set_device_error(a.err, kErrTopkOverflow);
+      cnt[0] = 0u; cnt[1] = 0u; cnt[2] = 0u;
+    }
+    for (int i = tid; i < kHistBins; i += kSplitThreads) hist_row[i] = 0u;
+    return;
+  }
   uint32_t rem = (uint32_t)k - n_sure;        // >= 1: fewer than k keys lie above b*
 #ifdef CSA_TRACE
   if (tid == 0 && blockIdx.x < 80) { g_trace_t[blockIdx.x][8] = n_sure; g_trace_t[blockIdx.x][9] = nc; }
@@ -391,6 +408,10 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
     }
     pos0 += __shfl_sync(0xffffffffu, inc, 31);
   }
+  // leave the row's histogram and counters zeroed for the next call (every CTA of the row has
+  // read the histogram: each took its ticket after filtering)
+  for (int i = tid; i < kHistBins; i += kSplitThreads) hist_row[i] = 0u;
+  if (tid < 3) cnt[tid] = 0u;
   TTRACE(7);
 }
 
@@ -420,10 +441,7 @@ cudaError_t launch_topk_split(const TopkSplitArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  profile_mark(s);
-  topk_split_kernel<<<dim3(a.G, a.base.rows), kSplitThreads, smem, s>>>(a);
-  note_launches(1);
-  return cudaGetLastError();
+  return launch_kernel(topk_split_kernel, dim3(a.G, a.base.rows), dim3(kSplitThreads), smem, s, 0, a);
 }
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
@@ -436,10 +454,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  profile_mark(s);
-  topk_rows_kernel<<<a.rows, kThreads, smem, s>>>(a, use_smem);
-  note_launches(1);
-  return cudaGetLastError();
+  return launch_kernel(topk_rows_kernel, dim3(a.rows), dim3(kThreads), smem, s, 0, a, use_smem);
 }
 
 }  // namespace csa
