@@ -80,7 +80,7 @@ typedef enum csa_status {
   CSA_ERR_UNSUPPORTED = 2,     /* valid, but no kernel for this shape / format */
   CSA_ERR_WORKSPACE = 3,       /* workspace missing or smaller than csa_workspace_size() */
   CSA_ERR_CUDA = 4,            /* a CUDA runtime call failed (message in csa_last_error) */
-  CSA_ERR_DEVICE_TIMEOUT = 5   /* a bounded device wait gave up (csa_device_error) */
+  CSA_ERR_DEVICE_TIMEOUT = 5   /* a kernel set a bit of the device error word (csa_device_error) */
 } csa_status_t;
 
 enum {
@@ -159,8 +159,12 @@ CSA_API const char* csa_last_error(void);
 CSA_API const char* csa_version(void);
 
 /* Reads and clears the workspace's device error word (synchronises the
- * stream).  *code gets the bits set by kernels whose bounded waits gave up
- * (0 = none); returns CSA_ERR_DEVICE_TIMEOUT if any bit was set. */
+ * stream).  *code gets the bits kernels set (0 = none):
+ *   1  a bounded wait (mbarrier / tensor-memory pipeline) gave up;
+ *   2  the multi-CTA top-k found its score histogram inconsistent with the
+ *      scores (appends past their reserved range); that row's top-k output
+ *      was left unwritten instead.
+ * Returns CSA_ERR_DEVICE_TIMEOUT if any bit was set. */
 CSA_API csa_status_t csa_device_error(void* workspace, size_t ws_bytes, void* stream, int32_t* code);
 
 /* Profiling aid (no counterpart on the pages).  When ev_start and ev_stop (cudaEvent_t handles
@@ -266,6 +270,35 @@ CSA_API csa_status_t csa_decode_step(const csa_layer_t* L, const csa_cache_t* ca
                              const void* x_new, const void* g_new, const int64_t* q_pos,
                              void* out, int32_t* topk_idx,
                              void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of the static device scratch used by csa_decode_step_scratch. */
+#define CSA_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* csa_decode_step without a caller workspace (no counterpart on the pages:
+ * a convenience of this library).  The workspace is a fixed array of
+ * CSA_SCRATCH_BYTES in the library's static device memory, one per device,
+ * so the call allocates nothing.
+ *   - Limit: csa_workspace_size(L, CSA_OP_DECODE_STEP, 1, cache->entry_cap)
+ *     must be <= CSA_SCRATCH_BYTES (B = 1 covers entry_cap up to 2^18, i.e.
+ *     a 1M-token context at m = 4); a larger call returns CSA_ERR_WORKSPACE
+ *     and touches no device state.
+ *   - The array's address is looked up (cudaGetSymbolAddress, which may load
+ *     the module) on the first call on each device: make that first call
+ *     outside any CUDA stream capture.
+ *   - Every call on a device shares its one array: two calls whose executions
+ *     overlap (different streams or threads, concurrent graph replays) race
+ *     on it and give undefined results.  Serialise them.
+ *   - device_error: NULL, or a host int32 that receives the device error word
+ *     (see csa_device_error); non-NULL synchronises the stream (not allowed
+ *     during stream capture) and, when the word is non-zero, zero-fills the
+ *     scratch again and returns CSA_ERR_DEVICE_TIMEOUT.
+ * Other arguments, layouts and errors as csa_decode_step. */
+CSA_API csa_status_t csa_decode_step_scratch(const csa_layer_t* L, const csa_cache_t* cache,
+                             const csa_params_t* P, const void* q,
+                             const void* idx_q, const float* idx_q_scale, const float* head_w,
+                             const void* x_new, const void* g_new, const int64_t* q_pos,
+                             void* out, int32_t* topk_idx, int32_t* device_error,
+                             void* stream);
 
 /* One fused HCA decode step: csa_append -> csa_compress -> hca_attend. */
 CSA_API csa_status_t hca_decode_step(const csa_layer_t* L, const csa_cache_t* cache,

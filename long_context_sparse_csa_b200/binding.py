@@ -72,6 +72,8 @@ _SIGS = {
     "hca_attend": (ctypes.c_int, [_LAYER, _CACHE, _PARAMS, _P, _P, _I32, _I64, _P, _P, _SZ, _P]),
     "csa_decode_step": (ctypes.c_int, [_LAYER, _CACHE, _PARAMS, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "hca_decode_step": (ctypes.c_int, [_LAYER, _CACHE, _PARAMS, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "csa_decode_step_scratch": (ctypes.c_int, [_LAYER, _CACHE, _PARAMS, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                               ctypes.POINTER(_I32), _P]),
     "csa_prefill": (ctypes.c_int, [_LAYER, _CACHE, _PARAMS, _P, _P, _P, _P, _P, _I32, _I64, _P, _P, _P, _SZ, _P]),
 }
 
@@ -229,6 +231,18 @@ def csa_decode_step(L, cache, params, q, idx_q, idx_q_scale, head_w, x_new, g_ne
                                  ptr(idx_q_scale), ptr(head_w), ptr(x_new), ptr(g_new), ptr(q_pos), ptr(out),
                                  ptr(topk_idx), ptr(workspace), workspace.numel() * workspace.element_size(),
                                  _stream(stream)))
+
+
+def csa_decode_step_scratch(L, cache, params, q, idx_q, idx_q_scale, head_w, x_new, g_new, q_pos, out, topk_idx,
+                            read_device_error=False, stream=None):
+    """csa_decode_step on the library's static device scratch (no workspace argument).  With
+    read_device_error the call synchronises and returns the device error word (else None)."""
+    code = _I32(0)
+    _check(lib().csa_decode_step_scratch(ctypes.byref(L), ctypes.byref(cache), ctypes.byref(params), ptr(q),
+                                         ptr(idx_q), ptr(idx_q_scale), ptr(head_w), ptr(x_new), ptr(g_new),
+                                         ptr(q_pos), ptr(out), ptr(topk_idx),
+                                         ctypes.byref(code) if read_device_error else None, _stream(stream)))
+    return code.value if read_device_error else None
 
 
 def hca_decode_step(L, cache, params, q, x_new, g_new, q_pos, out, workspace, stream=None):

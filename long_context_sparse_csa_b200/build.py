@@ -14,7 +14,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libcsa.so")
 
-SOURCES = ["compress.cu", "index_score.cu", "topk.cu", "attend.cu", "api.cu"]
+SOURCES = ["compress.cu", "index_score.cu", "topk.cu", "attend.cu", "api.cu", "static_scratch.cu"]
 HEADERS = ["common.cuh", "sm100.cuh", "kernels.h"]
 
 NVCC_FLAGS = [

@@ -299,6 +299,8 @@ csa_status_t check_params(const csa_layer_t* L, const csa_params_t* P, bool need
 }  // namespace
 
 namespace csa {
+csa_status_t report_error(csa_status_t st, const char* msg) { return fail(st, "%s", msg); }
+
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 void profile_mark(cudaStream_t s) {
   if (g_tl && g_tl_n < g_tl_cap) cudaEventRecordWithFlags(g_tl[g_tl_n++], s, cudaEventRecordExternal);

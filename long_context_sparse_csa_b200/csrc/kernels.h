@@ -13,6 +13,8 @@ namespace csa {
 void note_launches(int n);
 // Records the next timeline event (if a timeline is armed on this thread) just before a launch.
 void profile_mark(cudaStream_t s);
+// Sets this thread's csa_last_error() text and returns st (for entry points outside api.cu).
+csa_status_t report_error(csa_status_t st, const char* msg);
 
 // Launches a kernel in stream order, with an optional thread-block cluster size (cluster > 0).
 // (Programmatic dependent launch was measured slower on the decode chain: CTAs parked at the
