@@ -220,6 +220,24 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- multi-rank plumbing
+
+def max_over_ranks(x, world, dist=None, device=None):
+    """Maximum of a per-rank float over all ranks (the slowest rank's time); identity at world 1."""
+    if world == 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(units_per_rank, world, T_ms):
+    """Whole-job throughput under weak scaling: every rank processes units_per_rank units (its own
+    replicas, no data-path exchange), so the job's units over the slowest rank's time."""
+    return units_per_rank * world / (T_ms / 1e3)
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def sha_of(paths):
@@ -361,13 +379,6 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     cur = torch.cuda.current_stream()
     clocks = ClockSampler(local)
     clocks.start()
@@ -390,7 +401,7 @@ def run_ours(args):
     w1 = time.perf_counter()
     clocks.sample()
     barrier()
-    T_ms = max_over_ranks(e0.elapsed_time(e1))
+    T_ms = max_over_ranks(e0.elapsed_time(e1), world, dist, dev)
     clk = clocks.summary(w0, w1)
     # indexer launch durations sampled inside the timed region (one per cycle-graph copy)
     idx_ms = [c[1][0].elapsed_time(c[1][1]) for c in cycles] if has_csa else []
@@ -467,15 +478,15 @@ def run_ours(args):
     f1.record(cur)
     torch.cuda.synchronize()
     barrier()
-    E_ms = max_over_ranks(f0.elapsed_time(f1))
+    E_ms = max_over_ranks(f0.elapsed_time(f1), world, dist, dev)
     clocks.stop()
 
     for lay in layers:
         assert C.csa_device_error(lay["ws"]) == 0
 
-    units = wl.B * len(layers) * args.steps * world
-    value = units / (T_ms / 1e3)
-    e2e_value = units / (E_ms / 1e3)
+    units = wl.B * len(layers) * args.steps
+    value = job_value(units, world, T_ms)
+    e2e_value = job_value(units, world, E_ms)
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": T_ms / args.steps, "higher_is_better": True, "scaling": "weak",
