@@ -162,8 +162,7 @@ CSA_API const char* csa_version(void);
  * stream).  *code gets the bits kernels set (0 = none):
  *   1  a bounded wait (mbarrier / tensor-memory pipeline) gave up;
  *   2  the multi-CTA top-k found its score histogram inconsistent with the
- *      scores (appends past their reserved range); that row's top-k output
- *      was left unwritten instead.
+ *      scores; that row's top-k output is incomplete (padded with -1).
  * Returns CSA_ERR_DEVICE_TIMEOUT if any bit was set. */
 CSA_API csa_status_t csa_device_error(void* workspace, size_t ws_bytes, void* stream, int32_t* code);
 
@@ -263,7 +262,12 @@ CSA_API csa_status_t hca_attend(const csa_layer_t* L, const csa_cache_t* cache,
 /* One fused CSA decode step for token t = q_pos[b] of every sequence:
  * csa_append (x_new, g_new) -> csa_compress (when t completes a group) ->
  * csa_index_topk over entry_cap entries -> csa_sparse_attend.  Tq = 1.
- * topk_idx: [B][top_k] int32 output, or NULL (kept in the workspace). */
+ * topk_idx: [B][top_k] int32 output, or NULL (kept in the workspace).
+ * The index keys are inputs, so append+compress does not feed the indexer:
+ * the library runs it on an internal second stream (one per thread and
+ * device, created by the first call made outside stream capture), forked
+ * from and joined back into `stream` before attention.  Ordering with
+ * respect to `stream` is unchanged, and the pattern is graph-capturable. */
 CSA_API csa_status_t csa_decode_step(const csa_layer_t* L, const csa_cache_t* cache,
                              const csa_params_t* P, const void* q,
                              const void* idx_q, const float* idx_q_scale, const float* head_w,

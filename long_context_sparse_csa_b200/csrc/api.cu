@@ -46,6 +46,43 @@ int num_sms() {
   return n;
 }
 
+// A second stream per (thread, device) for the CSA decode step's fork/join: compression does not
+// feed the indexer (index keys are inputs), so append+compress runs beside indexer + top-k and
+// joins before attention.  Created on first use outside stream capture; nullptr means "run in
+// sequence on the caller's stream" (creation failed, the caller is capturing before the first
+// eager call, or a launch timeline is armed: its intervals then stay one kernel each).
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool failed = false;
+};
+thread_local SideStream g_side[64];
+
+SideStream* side_stream(cudaStream_t main) {
+  if (g_tl) return nullptr;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  SideStream& ss = g_side[dev];
+  if (ss.s) return &ss;
+  if (ss.failed) return nullptr;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(main, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+    cudaGetLastError();
+    if (ss.s) cudaStreamDestroy(ss.s);
+    if (ss.fork) cudaEventDestroy(ss.fork);
+    ss = SideStream();
+    ss.failed = true;
+    return nullptr;
+  }
+  return &ss;
+}
+
 size_t row_bytes_of(const csa_layer_t* L) {
   switch (L->kv_format) {
     case CSA_FMT_F32: return 4 * (size_t)L->D;
@@ -152,8 +189,8 @@ size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Workspace {
   size_t err = 0;          // int error word
-  size_t hist = 0, hist_bytes = 0;      // split top-k: histogram [rows][4096] + counters [rows][4]
-  size_t sure = 0, cand = 0;            // split top-k scratch
+  size_t hist = 0, hist_bytes = 0;      // split top-k: histogram [rows][4096], counters [rows][4], histogram 2 [rows][4096]
+  size_t counts = 0, list = 0;          // split top-k scratch
   size_t scores = 0, scores_bytes = 0;
   size_t topk = 0, topk_bytes = 0;
   size_t part = 0, part_bytes = 0;
@@ -169,9 +206,9 @@ Workspace layout(const csa_layer_t* L, int op, int32_t Tq, int64_t n_max) {
   if (csa && (op == CSA_OP_INDEX_TOPK || op == CSA_OP_DECODE_STEP || op == CSA_OP_PREFILL)) {
     w.scores = off; w.scores_bytes = rows * (size_t)(n_max > 0 ? n_max : 1) * 4; off = up(off + w.scores_bytes);
     if (use_split_topk(L, Tq, n_max)) {
-      w.hist = off; w.hist_bytes = rows * (4096 + 4) * 4; off = up(off + w.hist_bytes);
-      w.sure = off; off = up(off + rows * (size_t)L->top_k * 4);
-      w.cand = off; off = up(off + rows * (size_t)n_max * 8);
+      w.hist = off; w.hist_bytes = rows * (4096 + 4 + 4096) * 4; off = up(off + w.hist_bytes);
+      w.counts = off; off = up(off + rows * (size_t)kTopkSplitMaxCtas * 4);
+      w.list = off; off = up(off + rows * (size_t)n_max * 8);
     }
   }
   if (csa && (op == CSA_OP_DECODE_STEP || op == CSA_OP_PREFILL)) {
@@ -251,8 +288,9 @@ csa_status_t run_index_topk(const csa_layer_t* L, const csa_cache_t* cache, cons
     sa.base = t;
     sa.hist = hist;
     sa.cnt = hist + (size_t)rows * 4096;
-    sa.sure = reinterpret_cast<int32_t*>(at(ws, w.sure));
-    sa.cand = reinterpret_cast<uint2*>(at(ws, w.cand));
+    sa.hist2 = sa.cnt + (size_t)rows * 4;
+    sa.counts = reinterpret_cast<uint32_t*>(at(ws, w.counts));
+    sa.list = reinterpret_cast<uint2*>(at(ws, w.list));
     sa.G = topk_split_ctas(rows, n_max, num_sms());
     sa.err = err;
     e = launch_topk_split(sa, s);
@@ -262,10 +300,9 @@ csa_status_t run_index_topk(const csa_layer_t* L, const csa_cache_t* cache, cons
   return e == cudaSuccess ? CSA_OK : cuda_fail(e, "top-k launch");
 }
 
-csa_status_t run_attend(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P, const void* q,
-                        const int64_t* q_pos, int32_t Tq, const int32_t* topk, int64_t n_max, void* out,
-                        const Workspace& w, void* ws, cudaStream_t s) {
-  AttendArgs a;
+csa_status_t make_attend_args(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P, const void* q,
+                              const int64_t* q_pos, int32_t Tq, const int32_t* topk, int64_t n_max, void* out,
+                              const Workspace& w, void* ws, AttendArgs& a) {
   a.L = layer_args(L);
   if (attend_head_group(a.L) == 0 && L->H > 32)
     return fail(CSA_ERR_UNSUPPORTED, "attention: H=%d needs D=512 with bf16/mixed rows and H%%32==0, or H<=32", L->H);
@@ -284,7 +321,15 @@ csa_status_t run_attend(const csa_layer_t* L, const csa_cache_t* cache, const cs
     return fail(CSA_ERR_WORKSPACE, "workspace too small for the attention partials");
   a.part = reinterpret_cast<float*>(at(ws, w.part));
   a.out = static_cast<uint8_t*>(out);
-  cudaError_t e = launch_attend(a, s);
+  return CSA_OK;
+}
+
+csa_status_t run_attend(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P, const void* q,
+                        const int64_t* q_pos, int32_t Tq, const int32_t* topk, int64_t n_max, void* out,
+                        const Workspace& w, void* ws, cudaStream_t s) {
+  AttendArgs a;
+  CSA_TRY(make_attend_args(L, cache, P, q, q_pos, Tq, topk, n_max, out, w, ws, a));
+  const cudaError_t e = launch_attend(a, s);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e, "attention launch");
 }
 
@@ -460,8 +505,27 @@ csa_status_t csa_decode_step(const csa_layer_t* L, const csa_cache_t* cache, con
   const Workspace w = layout(L, CSA_OP_DECODE_STEP, 1, cache->entry_cap);
   CSA_TRY(check_ws(w, workspace, ws_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  CSA_TRY(run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, s));
   int32_t* tk = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(at(workspace, w.topk));
+  SideStream* ss = side_stream(s);
+  if (ss) {
+    // fork: append+compress on the side stream, indexer + top-k here; join before attention
+    cudaError_t e = cudaEventRecord(ss->fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->s, ss->fork, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "csa_decode_step fork");
+    const csa_status_t sc = run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, ss->s);
+    const csa_status_t si = sc == CSA_OK ? run_index_topk(L, cache, idx_q, idx_q_scale, head_w, q_pos, 1,
+                                                          cache->entry_cap, tk,
+                                                          reinterpret_cast<float*>(at(workspace, w.scores)), w,
+                                                          workspace, s)
+                                         : sc;
+    // the join is recorded whatever happened, so a capture never ends with the side stream unjoined
+    e = cudaEventRecord(ss->join, ss->s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
+    if (si != CSA_OK) return si;
+    if (e != cudaSuccess) return cuda_fail(e, "csa_decode_step join");
+    return run_attend(L, cache, P, q, q_pos, 1, tk, cache->entry_cap, out, w, workspace, s);
+  }
+  CSA_TRY(run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, s));
   CSA_TRY(run_index_topk(L, cache, idx_q, idx_q_scale, head_w, q_pos, 1, cache->entry_cap, tk,
                          reinterpret_cast<float*>(at(workspace, w.scores)), w, workspace, s));
   return run_attend(L, cache, P, q, q_pos, 1, tk, cache->entry_cap, out, w, workspace, s);

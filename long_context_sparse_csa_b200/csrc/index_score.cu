@@ -103,8 +103,12 @@ __device__ __forceinline__ Sched make_sched(const IndexArgs& a) {
 // Diagnostic build only: per-CTA timestamps (ns) of the indexer pipeline.
 __device__ uint64_t g_trace[320][80];
 #define TRACE(slot) (g_trace[blockIdx.x][(slot)] = global_timer_ns())
+#define TRACE_VAL(slot, v) (g_trace[blockIdx.x][(slot)] = (uint64_t)(v))
+#define CYC() clock64()
 #else
 #define TRACE(slot) ((void)0)
+#define TRACE_VAL(slot, v) ((void)0)
+#define CYC() 0ll
 #endif
 
 constexpr int kHistBins = 4096;               // top 12 bits of the order-preserving score key
@@ -119,19 +123,85 @@ struct __align__(8) Barriers {
   uint32_t tmem_base;
 };
 
+constexpr int kKsChunk = 8;                   // key-scale prefetch distance, in work items
+
 struct EpiSmem {
   float w[kMaxQH];            // head weights of the group's queries
   float qs[kMaxQH];           // index-query scales
   float wq[kMaxQH];           // w * qs (used when every scale is positive)
   int pos[kMaxQH / 16];       // 1 when all of the query's index-query scales are > 0
   int64_t nv[kMaxQH / 16];    // visible entries per query (QN <= 16)
-  uint32_t hist[kHistBins];   // score histogram of the current group (decode)
+  uint32_t hist[kHistBins];   // score histogram of the current group (decode); 16-byte aligned
+  float ks[kKsChunk][kTileE]; // key scales of the current chunk of items (each thread its own entry)
 };
 
 __device__ __forceinline__ void epi_bar() { asm volatile("barrier.sync.aligned 5, 128;" ::: "memory"); }
+// Set-up barrier: the producer warp arrives without waiting, the other five warps wait.
+__device__ __forceinline__ void setup_arrive() { asm volatile("barrier.arrive.aligned 1, 192;" ::: "memory"); }
+__device__ __forceinline__ void setup_sync() { asm volatile("barrier.sync.aligned 1, 192;" ::: "memory"); }
 
-template <int kStages>
-__global__ void __launch_bounds__(kThreads, 1)
+// Schedule bounds of group g as the three roles walk it.  In the strided (decode) schedule every
+// tile below n_max is streamed, so that no query-position load gates the first key copy (entries
+// past a query's visibility are masked by the epilogue); otherwise tiles past the group's last
+// visible entry are skipped.
+__device__ __forceinline__ Group sched_group(const IndexArgs& a, int64_t g, bool strided) {
+  if (!strided) return group_info(a, g);
+  Group G;
+  G.g = g;
+  G.b = (int)(g / a.groups_per_seq);
+  G.j0 = (int)(g % a.groups_per_seq) * a.QN;
+  G.j1 = min(G.j0 + a.QN, a.Tq);
+  G.last_et = a.tiles_per_group - 1;
+  return G;
+}
+
+// A group's per-query constants, as loaded by epilogue thread te (of 128): head weight and
+// index-query scale of columns te and te + 128, the visibility of query te (te < QN).
+struct GroupConsts {
+  float w[2], qs[2];
+  int64_t nv;
+};
+
+__device__ __forceinline__ GroupConsts load_group_consts(const IndexArgs& a, int64_t g, int te) {
+  GroupConsts c;
+  const int b = (int)(g / a.groups_per_seq), j0 = (int)(g % a.groups_per_seq) * a.QN;
+  const int QH = a.QN * a.H_I;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int i = te + 128 * r;
+    c.w[r] = 0.f;
+    c.qs[r] = 0.f;
+    if (i < QH) {
+      const int j = j0 + i / a.H_I;
+      const int64_t row = (int64_t)b * a.Tq + (j < a.Tq ? j : a.Tq - 1);
+      c.w[r] = __ldg(a.head_w + row * a.H_I + i % a.H_I);
+      c.qs[r] = __ldg(a.q_scale + row * a.H_I + i % a.H_I);
+    }
+  }
+  c.nv = (te < a.QN && j0 + te < a.Tq) ? n_visible(a, b, j0 + te) : 0;
+  return c;
+}
+
+// Issues the key-scale loads of items [k0, k0 + kKsChunk) for entry lane e_loc (0 past the end).
+__device__ __forceinline__ void load_key_scales(const IndexArgs& a, const Sched& sc, int64_t k0, int e_loc,
+                                                float ks[kKsChunk]) {
+#pragma unroll
+  for (int u = 0; u < kKsChunk; ++u) {
+    ks[u] = 0.f;
+    if (k0 + u < sc.count) {
+      int64_t g;
+      int et;
+      sc.at(k0 + u, &g, &et);
+      const int64_t e = (int64_t)et * kTileE + e_loc;
+      if (e < a.n_max) ks[u] = __ldg(a.k_scale + (g / a.groups_per_seq) * a.entry_cap + e);
+    }
+  }
+}
+
+// kHI > 0: decode specialisation (one query per group, kHI index heads, head weights in registers);
+// kHI == 0: any QN x H_I (prefill).
+template <int kStages, int kHI>
+__global__ void __launch_bounds__(kThreads, kHI > 0 ? 2 : 1)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                       const __grid_constant__ IndexArgs a, int N, int nacc, uint32_t tmem_cols) {
   extern __shared__ uint8_t smem_raw[];
@@ -144,14 +214,18 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Sched sc = make_sched(a);
   if (threadIdx.x == 0) TRACE(0);
-  // the first group's visibility (a q_pos load) is fetched while the barriers and TMEM are set up
-  Group G0;
-  G0.g = -1;
-  if (sc.count > 0) {
+  // Epilogue warps issue the first group's constants and the first chunk of key scales now: their
+  // latency then overlaps the set-up below and the first key tile's copy.
+  const int te = threadIdx.x - 64;            // epilogue thread 0..127
+  const int e_loc = (warp & 3) * 32 + lane;   // epilogue: entry row = TMEM lane of this warp's quarter
+  GroupConsts gc0;
+  float ks_cur[kKsChunk];
+  if (warp >= 2 && sc.count > 0) {
     int64_t g;
     int et;
     sc.at(0, &g, &et);
-    G0 = group_info(a, g);
+    gc0 = load_group_consts(a, g, te);
+    load_key_scales(a, sc, 0, e_loc, ks_cur);
   }
 
   if (threadIdx.x == 0) {
@@ -166,10 +240,20 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     tmem_alloc(&bars->tmem_base, tmem_cols);
     tmem_relinquish();
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = bars->tmem_base;
+  // The producer needs neither TMEM nor the other warps: it arrives at the set-up barrier (its
+  // barrier initialisation is then visible to the waiting warps) and starts copying at once.
+  uint32_t tmem = 0;
+  if (warp == 0) {
+    __syncwarp();
+    setup_arrive();
+  } else {
+    tc_fence_before();
+    setup_sync();
+    tc_fence_after();
+    tmem = bars->tmem_base;
+    if (threadIdx.x == 32) TRACE(71);
+    if (threadIdx.x == 64) TRACE(72);
+  }
   if (threadIdx.x == 0) TRACE(1);
 
   // The producer and MMA warps run their loops with all 32 lanes (every wait is warp-uniform) and
@@ -185,7 +269,6 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     Group G;
     G.g = -1;
     int gi = -1;
-    G = G0;
     int issued_par[kStages];
     for (int s = 0; s < kStages; ++s) issued_par[s] = -1;
     int b_issued_par[2] = {-1, -1};
@@ -194,7 +277,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       int64_t g;
       int et;
       sc.at(k, &g, &et);
-      if (g != G.g) G = group_info(a, g);
+      if (g != G.g) G = sched_group(a, g, sc.strided);
       if (et > G.last_et) continue;
       // validity is monotone in et, so the first item of a group in this CTA is its first valid one
       int64_t gp = -1;
@@ -236,7 +319,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     const uint32_t idesc = instr_desc(128, N, 0u);
     int stage = 0, acc = 0, gi = -1;
     uint32_t phase = 0, acc_phase = 0;
-    Group G = G0;
+    Group G;
+    G.g = -1;
     int last_acc = -1;
     uint32_t last_acc_par = 0;
     bool ok = true;
@@ -244,7 +328,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       int64_t g;
       int et;
       sc.at(k, &g, &et);
-      if (g != G.g) G = group_info(a, g);
+      if (g != G.g) G = sched_group(a, g, sc.strided);
       if (et > G.last_et) continue;
       int64_t gp = -1;
       int etp;
@@ -290,10 +374,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     // ------------------------------------------------------------------ epilogue (warps 2..5)
     // Every epilogue warp runs the same sequence of named barriers whatever happens (a wait that
     // times out only stops the warp's work), so the 128-thread barrier can never be left short.
-    const int te = threadIdx.x - 64;           // 0..127
-    const int quarter = warp & 3;              // TMEM lanes [32*quarter, 32*quarter + 32)
-    const int e_loc = quarter * 32 + lane;
-    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const bool use_hist = a.hist != nullptr && a.QN == 1;
     const int QH = a.QN * a.H_I;
     if (use_hist)
@@ -303,109 +384,177 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     bool ok = true;
     Group G;
     G.g = -1;
-    float ks_next = 0.f;
-    int64_t ks_w = -1;  // item whose key scale is in ks_next
-    auto flush_hist = [&](const Group& H) {
-      const int64_t row = (int64_t)H.b * a.Tq + H.j0;
-      for (int i = te; i < kHistBins; i += 128) {
-        const uint32_t v = es->hist[i];
-        if (v) { atomicAdd(a.hist + row * kHistBins + i, v); es->hist[i] = 0u; }
+    // decode: the group's w * qs per head, its scale positivity and visibility, in registers
+    float wr[kHI > 0 ? kHI : 1];
+    int pos_reg = 0;
+    int64_t nv_reg = 0;
+    // adds the shared histogram into the row's global one (one reduction per non-empty bin)
+    auto flush_hist = [&](const Group& H, bool clear) {
+      uint32_t* dst = a.hist + ((int64_t)H.b * a.Tq + H.j0) * kHistBins;
+      uint4* src = reinterpret_cast<uint4*>(es->hist);
+      uint4 v[kHistBins / 4 / 128];
+#pragma unroll
+      for (int r = 0; r < kHistBins / 4 / 128; ++r) v[r] = src[te + 128 * r];
+#pragma unroll
+      for (int r = 0; r < kHistBins / 4 / 128; ++r) {
+        uint32_t* d = dst + 4 * (te + 128 * r);
+        if (v[r].x) atomicAdd(d + 0, v[r].x);
+        if (v[r].y) atomicAdd(d + 1, v[r].y);
+        if (v[r].z) atomicAdd(d + 2, v[r].z);
+        if (v[r].w) atomicAdd(d + 3, v[r].w);
+        if (clear) src[te + 128 * r] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    auto enter_group = [&](int64_t g, const GroupConsts& c) {
+      epi_bar();
+      if (use_hist && G.g >= 0) flush_hist(G, true);
+      G = sched_group(a, g, sc.strided);
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int i = te + 128 * r;
+        if (i < QH) {
+          es->w[i] = c.w[r];
+          es->qs[i] = c.qs[r];
+          es->wq[i] = c.w[r] * c.qs[r];
+        }
+      }
+      if (te < a.QN) es->nv[te] = c.nv;
+      epi_bar();
+      if (te < a.QN) {
+        int p = 1;
+        for (int h = 0; h < a.H_I; ++h) p &= es->qs[te * a.H_I + h] > 0.f;
+        es->pos[te] = p;
+      }
+      epi_bar();
+      if constexpr (kHI > 0) {
+#pragma unroll
+        for (int h = 0; h < kHI; ++h) wr[h] = es->wq[h];
+        pos_reg = es->pos[0];
+        nv_reg = es->nv[0];
       }
     };
     int done = 0;
-    for (int64_t k = 0; k < sc.count; ++k) {
-      int64_t g;
-      int et;
-      sc.at(k, &g, &et);
-      if (g != G.g) {
-        epi_bar();
-        if (use_hist && G.g >= 0 && G.last_et >= 0) flush_hist(G);
-        G = group_info(a, g);
-        for (int i = te; i < QH; i += 128) {
-          const int j = G.j0 + i / a.H_I;
-          const int64_t row = (int64_t)G.b * a.Tq + (j < a.Tq ? j : a.Tq - 1);
-          const float wv = a.head_w[row * a.H_I + i % a.H_I], qv = a.q_scale[row * a.H_I + i % a.H_I];
-          es->w[i] = wv;
-          es->qs[i] = qv;
-          es->wq[i] = wv * qv;
+    long long cyc_wait = 0, cyc_ld = 0, cyc_st = 0, cyc_all = 0;
+    float ks_nxt[kKsChunk];
+    for (int64_t k0 = 0; k0 < sc.count; k0 += kKsChunk) {
+      // this chunk's key scales (loaded one chunk ago) go to shared memory, the next chunk's are
+      // issued now and land while this chunk is processed
+#pragma unroll
+      for (int u = 0; u < kKsChunk; ++u) es->ks[u][e_loc] = ks_cur[u];
+      const bool more = k0 + kKsChunk < sc.count;
+      if (more) load_key_scales(a, sc, k0 + kKsChunk, e_loc, ks_nxt);
+      const int kn = (int)min((int64_t)kKsChunk, sc.count - k0);
+      for (int u = 0; u < kn; ++u) {
+        const int64_t k = k0 + u;
+        int64_t g;
+        int et;
+        sc.at(k, &g, &et);
+        if (g != G.g) {
+          enter_group(g, G.g < 0 ? gc0 : load_group_consts(a, g, te));
+          if (threadIdx.x == 64 && done == 0) TRACE(73);
         }
-        if (te < a.QN) es->nv[te] = (G.j0 + te < a.Tq) ? n_visible(a, G.b, G.j0 + te) : 0;
-        epi_bar();
-        if (te < a.QN) {
-          int p = 1;
-          for (int h = 0; h < a.H_I; ++h) p &= es->qs[te * a.H_I + h] > 0.f;
-          es->pos[te] = p;
-        }
-        epi_bar();
-      }
-      if (et > G.last_et) continue;
-      const int64_t e = (int64_t)et * kTileE + e_loc;
-      const bool in_range = e < a.n_max;
-      // this tile's key scale was prefetched by the previous iteration when it was the same group's
-      float ks;
-      if (ks_w == k) ks = ks_next;
-      else ks = in_range ? __ldg(a.k_scale + (int64_t)G.b * a.entry_cap + e) : 0.f;
-      if (k + 1 < sc.count) {
-        int64_t gn;
-        int etn;
-        sc.at(k + 1, &gn, &etn);
-        if (gn == g && etn <= G.last_et) {
-          const int64_t e2 = (int64_t)etn * kTileE + e_loc;
-          ks_next = e2 < a.n_max ? __ldg(a.k_scale + (int64_t)G.b * a.entry_cap + e2) : 0.f;
-          ks_w = k + 1;
-        }
-      }
-      if (ok) ok = mbar_wait(&bars->tfull[acc], acc_phase);
-      if (threadIdx.x == 64 && done < 16) TRACE(34 + done);
-      if (ok) {
-        tc_fence_after();
-        for (int j = G.j0; j < G.j1; ++j) {
-          const int q = j - G.j0;
-          const int64_t row = (int64_t)G.b * a.Tq + j;
-          const float* wq = es->w + q * a.H_I;
-          const float* sq = es->qs + q * a.H_I;
-          const float* wqq = es->wq + q * a.H_I;
-          // positive scales: ReLU(qs * ks * v) = qs * ks * ReLU(v), so s = ks * sum_h (w*qs)_h ReLU(v_h)
-          const bool fast = es->pos[q] && ks > 0.f;
+        if (et > G.last_et) continue;
+        const int64_t e = (int64_t)et * kTileE + e_loc;
+        const bool in_range = e < a.n_max;
+        const float ks = es->ks[u][e_loc];
+        long long c0 = CYC();
+        if (ok) ok = mbar_wait(&bars->tfull[acc], acc_phase);
+        long long c1 = CYC();
+        if (threadIdx.x == 64 && done < 16) TRACE(34 + done);
+        if (ok && kHI > 0) {
+          // decode: one query, kHI columns of the accumulator
+          tc_fence_after();
+          float v[kHI > 0 ? kHI : 1];
+          if constexpr (kHI == 16) {
+            tmem_ld_32x32b_x16(lane_addr + (uint32_t)(acc * N), v);
+          } else if constexpr (kHI > 0) {
+#pragma unroll
+            for (int hc = 0; hc < kHI; hc += 32) tmem_ld_32x32b_x32(lane_addr + (uint32_t)(acc * N + hc), v + hc);
+          }
+          tmem_wait_ld();
+          cyc_ld += CYC() - c1;
+          tc_fence_before();
+          mbar_arrive(&bars->tempty[acc]);
           float s = 0.f;
-          for (int hc = 0; hc < a.H_I; hc += 32) {
-            float v[32];
-            tmem_ld_32x32b_x16(lane_addr + (uint32_t)(acc * N + q * a.H_I + hc), v);
-            if (hc + 16 < a.H_I) tmem_ld_32x32b_x16(lane_addr + (uint32_t)(acc * N + q * a.H_I + hc + 16), v + 16);
-            tmem_wait_ld();
-            if (j + 1 == G.j1 && hc + 32 >= a.H_I) {
-              // every column of this accumulator is in registers: hand it back to the MMA warp
-              tc_fence_before();
-              mbar_arrive(&bars->tempty[acc]);
-            }
-            const int nh = min(32, a.H_I - hc);
-            if (fast) {
+          if (pos_reg && ks > 0.f) {
+            // positive scales: ReLU(qs * ks * v) = qs * ks * ReLU(v)
 #pragma unroll
-              for (int h = 0; h < 32; ++h)
-                if (h < nh) s = fmaf(wqq[hc + h], fmaxf(v[h], 0.f), s);
-            } else {
+            for (int h = 0; h < kHI; ++h) s = fmaf(wr[h], fmaxf(v[h], 0.f), s);
+            s *= ks;
+          } else {
 #pragma unroll
-              for (int h = 0; h < 32; ++h)
-                if (h < nh) s += wq[hc + h] * fmaxf(v[h] * (sq[hc + h] * ks), 0.f);
-            }
+            for (int h = 0; h < kHI; ++h) s += es->w[h] * fmaxf(v[h] * (es->qs[h] * ks), 0.f);
           }
-          if (fast) s *= ks;
-          const bool vis = e < es->nv[q];
-          if (in_range) a.scores[row * a.n_max + e] = vis ? s : -INFINITY;
-          if (use_hist) {
-            // one shared-memory atomic per distinct bin in the warp
-            const uint32_t bin = vis ? (float_key(s) >> 20) : 0xFFFFFFFFu;
-            const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-            if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&es->hist[bin], (uint32_t)__popc(peers));
+          long long c2 = CYC();
+          const bool vis = e < nv_reg;
+          if (in_range) a.scores[((int64_t)G.b * a.Tq + G.j0) * a.n_max + e] = vis ? s : -INFINITY;
+          if (use_hist && vis) atomicAdd(&es->hist[float_key(s) >> 20], 1u);
+          cyc_st += CYC() - c2;
+        } else if (ok) {
+          tc_fence_after();
+          for (int j = G.j0; j < G.j1; ++j) {
+            const int q = j - G.j0;
+            const int64_t row = (int64_t)G.b * a.Tq + j;
+            const float* wq = es->w + q * a.H_I;
+            const float* sq = es->qs + q * a.H_I;
+            const float* wqq = es->wq + q * a.H_I;
+            // positive scales: ReLU(qs * ks * v) = qs * ks * ReLU(v), so s = ks * sum_h (w*qs)_h ReLU(v_h)
+            const bool fast = es->pos[q] && ks > 0.f;
+            float s = 0.f;
+            for (int hc = 0; hc < a.H_I; hc += 32) {
+              float v[32];
+              tmem_ld_32x32b_x16(lane_addr + (uint32_t)(acc * N + q * a.H_I + hc), v);
+              if (hc + 16 < a.H_I) tmem_ld_32x32b_x16(lane_addr + (uint32_t)(acc * N + q * a.H_I + hc + 16), v + 16);
+              tmem_wait_ld();
+              cyc_ld += CYC() - c1;
+              if (j + 1 == G.j1 && hc + 32 >= a.H_I) {
+                // every column of this accumulator is in registers: hand it back to the MMA warp
+                tc_fence_before();
+                mbar_arrive(&bars->tempty[acc]);
+              }
+              const int nh = min(32, a.H_I - hc);
+              if (fast) {
+#pragma unroll
+                for (int h = 0; h < 32; ++h)
+                  if (h < nh) s = fmaf(wqq[hc + h], fmaxf(v[h], 0.f), s);
+              } else {
+#pragma unroll
+                for (int h = 0; h < 32; ++h)
+                  if (h < nh) s += wq[hc + h] * fmaxf(v[h] * (sq[hc + h] * ks), 0.f);
+              }
+            }
+            if (fast) s *= ks;
+            long long c2 = CYC();
+            const bool vis = e < es->nv[q];
+            if (in_range) a.scores[row * a.n_max + e] = vis ? s : -INFINITY;
+            if (use_hist) {
+              // one shared-memory atomic per distinct bin in the warp
+              const uint32_t bin = vis ? (float_key(s) >> 20) : 0xFFFFFFFFu;
+              const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+              if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&es->hist[bin], (uint32_t)__popc(peers));
+            }
+            cyc_st += CYC() - c2;
           }
         }
+        cyc_wait += c1 - c0;
+        cyc_all += CYC() - c0;
+        if (++acc == nacc) { acc = 0; acc_phase ^= 1u; }
+        if (threadIdx.x == 64 && done < 16) TRACE(50 + done);
+        ++done;
       }
-      if (++acc == nacc) { acc = 0; acc_phase ^= 1u; }
-      if (threadIdx.x == 64 && done < 16) TRACE(50 + done);
-      ++done;
+      if (more) {
+#pragma unroll
+        for (int u = 0; u < kKsChunk; ++u) ks_cur[u] = ks_nxt[u];
+      }
+    }
+    if (threadIdx.x == 64) {
+      TRACE_VAL(74, cyc_wait);
+      TRACE_VAL(75, cyc_ld);
+      TRACE_VAL(76, cyc_st);
+      TRACE_VAL(77, cyc_all);
     }
     epi_bar();
-    if (use_hist && G.g >= 0 && G.last_et >= 0) flush_hist(G);
+    if (use_hist && G.g >= 0) flush_hist(G, false);
     if (!ok) set_device_error(a.err, kErrWaitTimeout);
   }
 
@@ -518,12 +667,16 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
   const int stages = decode ? 4 : 6;
   const size_t smem = 1024 + (size_t)stages * kTileBytes + 2 * (size_t)N * kDI + ((sizeof(Barriers) + 15) & ~size_t(15)) +
                      sizeof(EpiSmem) + 64;
-  static size_t configured[2] = {0, 0};
-  auto kern = decode ? index_score_tc_kernel<4> : index_score_tc_kernel<6>;
-  if (smem > configured[decode]) {
+  static size_t configured[4] = {0, 0, 0, 0};
+  const int ki = !decode ? 0 : a.H_I == 16 ? 1 : a.H_I == 32 ? 2 : 3;
+  auto kern = ki == 0 ? index_score_tc_kernel<6, 0>
+            : ki == 1 ? index_score_tc_kernel<4, 16>
+            : ki == 2 ? index_score_tc_kernel<4, 32>
+                      : index_score_tc_kernel<4, 64>;
+  if (smem > configured[ki]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    configured[decode] = smem;
+    configured[ki] = smem;
   }
   // decode: two CTAs per SM (two independent pipelines); each CTA's smem and TMEM allow it
   const int64_t ctas = decode ? 2 * (int64_t)num_sms : num_sms;

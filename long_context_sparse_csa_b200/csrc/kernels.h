@@ -98,14 +98,16 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 struct TopkSplitArgs {
   TopkArgs base;
   const uint32_t* hist;     // [rows][4096] (zero on entry; the kernel leaves it zeroed)
-  int32_t* sure;            // [rows][k] scratch
-  uint2* cand;              // [rows][n_max] scratch
+  uint32_t* counts;         // [rows][kTopkSplitMaxCtas] list length of each CTA's slice (scratch)
+  uint2* list;              // [rows][n_max] (key, index) of the slice's scores at or above the threshold bin
   uint32_t* cnt;            // [rows][4] counters (zero on entry; left zeroed)
-  int G;                    // CTAs per row
+  uint32_t* hist2;          // [rows][4096] histogram of key bits 19..8 in the threshold bin (zero on entry; left zeroed)
+  int G;                    // CTAs per row (<= kTopkSplitMaxCtas)
   int* err;                 // device error word
 };
+constexpr int kTopkSplitMaxCtas = 512;
 constexpr int64_t kTopkSplitMinN = 16384;     // rows at least this long use the split kernel
-constexpr int64_t kTopkSplitMaxN = 655360;    // the resolving CTA's bitmaps + staged candidates fit shared memory
+constexpr int64_t kTopkSplitMaxN = 655360;    // longer rows take the one-CTA-per-row kernel
 int topk_split_ctas(int rows, int64_t n_max, int num_sms);
 cudaError_t launch_topk_split(const TopkSplitArgs& a, cudaStream_t s);
 

@@ -151,32 +151,69 @@ __global__ void __launch_bounds__(kThreads, 1) topk_rows_kernel(const __grid_con
 
 
 // ----------------------------------------------------------------------------- split mode (long decode rows)
-// Many CTAs per row.  The indexer epilogue has already histogrammed the top 12 key bits of the
-// row's visible scores; every CTA finds the bin b* that holds the k-th largest key, then streams
-// its slice of the row: keys above b* are certainly selected (appended to `sure`), keys in b* are
-// candidates (appended to `cand`).  The last CTA of the row to finish (a ticket counter, no
-// waiting) resolves the candidates with two 10-bit radix passes, marks the selection in a
-// shared-memory bitmap over the row's indices, and emits it in ascending index order.
+// Many CTAs per row; the indexer epilogue has already histogrammed the top 12 key bits of the
+// row's visible scores (the steps are described above the kernel).
 #ifdef CSA_TRACE
 __device__ uint64_t g_trace_t[80][24];
 #define TTRACE(slot) do { if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.x < 80) { \
     uint64_t _t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(_t) :: "memory"); g_trace_t[blockIdx.x][(slot)] = _t; } } while (0)
+#define TTRACE_CYC(slot) do { if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.x < 80) \
+    g_trace_t[blockIdx.x][(slot)] = (uint64_t)clock64(); } while (0)
 #else
 #define TTRACE(slot) ((void)0)
+#define TTRACE_CYC(slot) ((void)0)
 #endif
 
 constexpr int kSplitThreads = 512;
 constexpr int kHistBins = 4096;
-constexpr int kChunk = 4096;                  // scores per filtering chunk
-constexpr int kCandCap = 4096;                // candidates staged in shared memory by the resolving CTA
+constexpr int kPer = 8;                               // scores / list entries per thread per pass
+constexpr int kChunk = kSplitThreads * kPer;          // 4096 per block pass
+static_assert(kHistBins == kChunk, "one histogram bin group of 8 per thread");
+static_assert(kTopkSplitMaxCtas <= kSplitThreads, "one slice count per thread");
 
+// find_bin over the row's global 4096-bin histogram: thread t holds bins 4095-8t .. 4088-8t (two
+// 128-bit loads), descending.
+__device__ __forceinline__ void find_bin_hist(const uint32_t* hist, uint32_t need, uint32_t* wsum, uint32_t* s_bin,
+                                              uint32_t* s_above) {
+  const int top = kHistBins - kPer * (int)threadIdx.x;   // exclusive upper bin of this thread
+  const uint4* p = reinterpret_cast<const uint4*>(hist + top - kPer);
+  const uint4 lo4 = __ldcg(p), hi4 = __ldcg(p + 1);
+  const uint32_t c[kPer] = {hi4.w, hi4.z, hi4.y, hi4.x, lo4.w, lo4.z, lo4.y, lo4.x};   // bins top-1 .. top-8
+  uint32_t c_local = 0;
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) c_local += c[q];
+  uint32_t tot;
+  uint32_t above = block_excl_scan(c_local, wsum, &tot);
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    if (above < need && need <= above + c[q]) { *s_bin = (uint32_t)(top - 1 - q); *s_above = above; }
+    above += c[q];
+  }
+  __syncthreads();
+}
+
+// Multi-CTA top-k of one long row (decode).  The key of a score is its order-preserving 32-bit
+// image; the k-th largest key T is pinned 12 + 12 + 8 bits at a time:
+//  1. every CTA finds the bin b1 of the key's top 12 bits that holds the k-th largest key, from the
+//     histogram the indexer filled while writing the scores;
+//  2. CTA g filters its slice [lo_g, hi_g) of the row: it writes (key, index) of every score whose
+//     top bits are >= b1 into the slice's own region of `list`, in ascending index order (a block
+//     scan per 4096 scores), adds each key of bin b1 to a second histogram of key bits 19..8, and
+//     stores its count;
+//  3. the last CTA to finish (a ticket counter; no CTA waits for another) finds the bin b2 of the
+//     second histogram, then the exact key with an 8-bit histogram of the few keys left;
+//  4. it concatenates the regions in CTA order (= ascending index order) and emits the entries with
+//     key > T and the first (k - #{key > T}) entries with key == T, each at its rank (one block scan
+//     of packed counts): ascending index order, ties to the smaller index.
 __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __grid_constant__ TopkSplitArgs a) {
-  extern __shared__ uint32_t bm[];              // filtering: chunk buffers; last CTA: sel[nw] | eq[nw]
-  __shared__ uint32_t h2[1024];
+  __shared__ uint32_t h3[256];
   __shared__ uint32_t wsum[32];
-  __shared__ uint32_t s_bin, s_above, s_last, s_ns, s_nc, s_gs, s_gc;
+  __shared__ uint32_t s_off[kTopkSplitMaxCtas + 1];
+  __shared__ uint32_t s_lo[kTopkSplitMaxCtas];          // first index of each CTA's slice
+  __shared__ uint32_t s_bin, s_above, s_last;
   const TopkArgs& A = a.base;
-  const int row = blockIdx.y, g = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+  const int row = blockIdx.y, g = blockIdx.x, tid = threadIdx.x;
+  const int G = gridDim.x;
   const int64_t t = A.q_pos[row];
   const int64_t r1 = t - A.pos0 + 1;
   int64_t nv64 = r1 > 0 ? r1 / A.m : 0;
@@ -185,6 +222,7 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
   const int k = A.k;
   int32_t* out = A.out + (size_t)row * k;
   uint32_t* hist_row = const_cast<uint32_t*>(a.hist) + (size_t)row * kHistBins;
+  uint32_t* hist2_row = a.hist2 + (size_t)row * kHistBins;
   if (nv <= k) {
     if (g == 0) {
       for (int i = tid; i < k; i += kSplitThreads) out[i] = i < nv ? i : -1;
@@ -193,225 +231,167 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
     return;
   }
   uint32_t* cnt = a.cnt + (size_t)row * 4;
-  int32_t* sure = a.sure + (size_t)row * k;
-  uint2* cand = a.cand + (size_t)row * A.n_max;
+  uint32_t* counts = a.counts + (size_t)row * kTopkSplitMaxCtas;
+  uint2* lst = a.list + (size_t)row * A.n_max;
+  auto slice_lo = [&](int gg) { return (int)((int64_t)nv * gg / G); };
 
   TTRACE(0);
-  // ---------------------------------------------------------------- 1. bin of the k-th largest key
-  find_bin(a.hist + (size_t)row * kHistBins, kHistBins, (uint32_t)k, wsum, &s_bin, &s_above);
-  const uint32_t bstar = s_bin;
+  // ---------------------------------------------------------------- 1. bin b1 of the k-th largest key
+  if (tid == 0) { s_bin = 0xFFFFFFFFu; s_above = 0u; }   // stays so if the histogram holds fewer than k
+  find_bin_hist(hist_row, (uint32_t)k, wsum, &s_bin, &s_above);
+  const uint32_t b1 = s_bin, n_above1 = s_above;
   TTRACE(1);
 
   // ---------------------------------------------------------------- 2. filter this CTA's slice
-  // Chunks of kChunk scores: appends go to shared-memory buffers, then one global atomic per
-  // counter reserves the chunk's space in `sure` / `cand`.
-  const int lo = (int)((int64_t)nv * g / gridDim.x), hi = (int)((int64_t)nv * (g + 1) / gridDim.x);
+  const int lo = slice_lo(g), hi = slice_lo(g + 1);
   const float* sc = A.scores + (size_t)row * A.n_max;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  int32_t* b_sure = reinterpret_cast<int32_t*>(bm);             // [kChunk]
-  uint2* b_cand = reinterpret_cast<uint2*>(bm + kChunk);         // [kChunk]
+  uint32_t n_mine = 0;
   for (int cb = lo; cb < hi; cb += kChunk) {
-    if (tid == 0) { s_ns = 0u; s_nc = 0u; }
-    __syncthreads();
     const int ce = min(cb + kChunk, hi);
-    constexpr int kPer = kChunk / kSplitThreads;
     float vals[kPer];
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
       const int i = cb + tid * kPer + u;           // a thread's kPer consecutive scores
-      vals[u] = i < ce ? __ldg(sc + i) : 0.f;
+      vals[u] = i < ce ? __ldcg(sc + i) : 0.f;
     }
-    uint32_t keys[kPer], ns = 0, nc2 = 0;
+    uint32_t keys[kPer], n = 0;
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
-      const int i = cb + tid * kPer + u;
       keys[u] = float_key(vals[u]);
-      const uint32_t bin = keys[u] >> 20;
-      ns += (i < ce && bin > bstar);
-      nc2 += (i < ce && bin == bstar);
+      n += (cb + tid * kPer + u < ce && (keys[u] >> 20) >= b1);
     }
-    uint32_t tot2;
-    const uint32_t ex = block_excl_scan(ns | (nc2 << 16), wsum, &tot2);
-    uint32_t ps = ex & 0xFFFFu, pc = ex >> 16;
+    uint32_t tot;
+    uint32_t pos = (uint32_t)lo + n_mine + block_excl_scan(n, wsum, &tot);
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
       const int i = cb + tid * kPer + u;
-      const uint32_t bin = keys[u] >> 20;
-      if (i < ce && bin > bstar) b_sure[ps++] = i;
-      if (i < ce && bin == bstar) b_cand[pc++] = make_uint2(keys[u], (uint32_t)i);
-    }
-    if (tid == 0) { s_ns = tot2 & 0xFFFFu; s_nc = tot2 >> 16; }
-    __syncthreads();
-    if (tid == 0) {
-      s_gs = s_ns ? atomicAdd(cnt + 0, s_ns) : 0u;
-      s_gc = s_nc ? atomicAdd(cnt + 1, s_nc) : 0u;
-      // a consistent histogram keeps every append in range; anything else is reported, not written
-      if (s_gs + s_ns > (uint32_t)k || s_gc + s_nc > (uint32_t)A.n_max) {
-        set_device_error(a.err, kErrTopkOverflow);
-        s_ns = 0u;
-        s_nc = 0u;
+      if (i < ce && (keys[u] >> 20) >= b1) {
+        lst[pos++] = make_uint2(keys[u], (uint32_t)i);
+        if ((keys[u] >> 20) == b1) atomicAdd(hist2_row + ((keys[u] >> 8) & 4095u), 1u);
       }
     }
-    __syncthreads();
-    for (uint32_t j = tid; j < s_ns; j += kSplitThreads) sure[s_gs + j] = b_sure[j];
-    for (uint32_t j = tid; j < s_nc; j += kSplitThreads) cand[s_gc + j] = b_cand[j];
-    __syncthreads();
+    n_mine += tot;
   }
-
+  if (tid == 0) counts[g] = n_mine;
   TTRACE(2);
   // ---------------------------------------------------------------- 3. last CTA of the row resolves
-  __syncthreads();
+  __syncthreads();                   // every list entry and histogram add of this CTA is issued ...
   if (tid == 0) {
-    __threadfence();
-    s_last = atomicAdd(cnt + 2, 1u) == gridDim.x - 1 ? 1u : 0u;
+    __threadfence();                 // ... and released (cumulatively) before the ticket
+    s_last = atomicAdd(cnt + 2, 1u) == (uint32_t)G - 1 ? 1u : 0u;
   }
   __syncthreads();
   TTRACE(3);
   if (!s_last) return;
   __threadfence();
-  const uint32_t n_sure = __ldcg(cnt + 0), nc = __ldcg(cnt + 1);   // after the fence: every CTA's appends
-  if (n_sure >= (uint32_t)k || nc > (uint32_t)A.n_max) {   // inconsistent histogram: report, emit nothing
-    if (tid == 0) {
-      set_device_error(a.err, kErrTopkOverflow);
-      cnt[0] = 0u; cnt[1] = 0u; cnt[2] = 0u;
+  // second level: bits 19..8 of the bin-b1 keys (its loads overlap the slice counts' below)
+  uint32_t rem = (uint32_t)k - n_above1;       // >= 1 when the histogram is consistent
+  if (tid == 0) { s_bin = 0xFFFFFFFFu; s_above = 0u; }
+  const uint32_t c_mine = tid < G ? __ldcg(counts + tid) : 0u;
+  find_bin_hist(hist2_row, rem, wsum, &s_bin, &s_above);
+  const uint32_t b2 = s_bin;
+  rem -= s_above;
+  const uint32_t p24 = (b1 << 12) | b2;        // top 24 bits of T
+  {
+    uint32_t tot;
+    const uint32_t ex = block_excl_scan(c_mine, wsum, &tot);
+    if (tid < G) {
+      s_off[tid] = ex;
+      s_lo[tid] = (uint32_t)slice_lo(tid);
     }
-    for (int i = tid; i < kHistBins; i += kSplitThreads) hist_row[i] = 0u;
-    return;
+    if (tid == 0) s_off[G] = tot;
+    if (tid < 256) h3[tid] = 0u;
   }
-  uint32_t rem = (uint32_t)k - n_sure;        // >= 1: fewer than k keys lie above b*
-#ifdef CSA_TRACE
-  if (tid == 0 && blockIdx.x < 80) { g_trace_t[blockIdx.x][8] = n_sure; g_trace_t[blockIdx.x][9] = nc; }
-#endif
-  TTRACE(10);
-  const int nw = (nv + 31) >> 5;
-  const int nw4 = (nw + 3) & ~3;               // keeps the second bitmap 16-byte aligned
-  uint32_t* sel = bm;
-  uint32_t* eqm = bm + nw4;
-  // candidates are read three times below: stage them in shared memory when they fit
-  uint2* cs = reinterpret_cast<uint2*>(bm + 2 * ((((A.n_max + 31) >> 5) + 3) & ~(int64_t)3));
-  const bool staged = nc <= (uint32_t)kCandCap;
-  if (staged)
-    for (uint32_t j = tid; j < nc; j += kSplitThreads) cs[j] = cand[j];
-  const uint2* cv = staged ? cs : cand;
-  for (int i = tid; i < 2 * nw4; i += kSplitThreads) bm[i] = 0u;
   __syncthreads();
+  const uint32_t L = s_off[G];
+  // every CTA of the row read both histograms' bins before its ticket: leave them zeroed now
+  for (int i = tid; i < kHistBins; i += kSplitThreads) { hist_row[i] = 0u; hist2_row[i] = 0u; }
+  if (tid < 3) cnt[tid] = 0u;
   TTRACE(4);
-
-  // two 10-bit radix passes over the candidates' low 20 bits pin the exact key T
-  uint32_t prefix = bstar;
-  int fixed = 12;
-  for (int pass = 0; pass < 2; ++pass) {
-    const int shift = 32 - fixed - 10;
-    for (int i = tid; i < 1024; i += kSplitThreads) h2[i] = 0u;
-    __syncthreads();
-    for (uint32_t j = tid; j < nc; j += kSplitThreads) {
-      const uint32_t key = cv[j].x;
-      if ((key >> (32 - fixed)) == prefix) atomicAdd(&h2[(key >> shift) & 1023u], 1u);
+  // entries p = base + kPer*tid + u of the concatenation (index ~0u past the end)
+  auto load_chunk = [&](uint32_t base, uint32_t kk[kPer], uint32_t ii[kPer]) {
+    const uint32_t p0 = base + kPer * (uint32_t)tid;
+    int gg = 0;
+    if (p0 < L) {                    // the slice holding p0: largest gg with s_off[gg] <= p0
+      int lo2 = 0, hi2 = G - 1;
+      while (lo2 < hi2) {
+        const int mid = (lo2 + hi2 + 1) >> 1;
+        if (s_off[mid] <= p0) lo2 = mid; else hi2 = mid - 1;
+      }
+      gg = lo2;
     }
-    __syncthreads();
-    find_bin(h2, 1024, rem, wsum, &s_bin, &s_above);
-    rem -= s_above;
-    prefix = (prefix << 10) | s_bin;
-    fixed += 10;
-    __syncthreads();
-  }
-  const uint32_t T = prefix;                   // keys > T are taken; `rem` keys == T, smallest indices
-  TTRACE(5);
-
-  for (uint32_t j = tid; j < n_sure; j += kSplitThreads) {
-    const uint32_t i = (uint32_t)sure[j];
-    atomicOr(&sel[i >> 5], 1u << (i & 31));
-  }
-  for (uint32_t j = tid; j < nc; j += kSplitThreads) {
-    const uint2 c = cv[j];
-    if (c.x > T) atomicOr(&sel[c.y >> 5], 1u << (c.y & 31));
-    else if (c.x == T) atomicOr(&eqm[c.y >> 5], 1u << (c.y & 31));
-  }
-  __syncthreads();
-
-  TTRACE(6);
-  // ordered emission.  Warp w owns words [w*CW, (w+1)*CW), CW a multiple of 256; in round i lane l
-  // holds the 8 consecutive words w*CW + 256i + 8l .. +7 (two 128-bit loads, no bank conflicts),
-  // and one warp scan per round orders the lanes.
-  const int nwarps = kSplitThreads / 32, wid = tid >> 5;
-  const int CW = ((nw + nwarps - 1) / nwarps + 255) & ~255;
-  const int wbeg = wid * CW, wend = min(wbeg + CW, nw);
-  auto load8 = [&](const uint32_t* bmp, int w0, uint32_t v[8]) {
-    if (w0 + 8 <= nw) {
-      const uint4 x = *reinterpret_cast<const uint4*>(bmp + w0), y = *reinterpret_cast<const uint4*>(bmp + w0 + 4);
-      v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w; v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
-    } else {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = (w0 + q < nw) ? bmp[w0 + q] : 0u;
+    for (int u = 0; u < kPer; ++u) {
+      const uint32_t p = p0 + u;
+      kk[u] = 0u;
+      ii[u] = ~0u;
+      if (p < L) {
+        while (p >= s_off[gg + 1]) ++gg;
+        const uint2 e = __ldcg(lst + s_lo[gg] + (p - s_off[gg]));
+        kk[u] = e.x;
+        ii[u] = e.y;
+      }
     }
   };
-  uint32_t eq_w = 0;
-  for (int base = wbeg; base < wend; base += 256) {
-    uint32_t v[8];
-    load8(eqm, base + 8 * lane, v);
+  const bool one = L <= (uint32_t)kChunk;      // the usual case: the list stays in registers
+  uint32_t kk[kPer], ii[kPer];
+  if (one) load_chunk(0, kk, ii);
+
+  // third level: the low 8 bits of the keys whose top 24 bits are p24
+  const bool lvl2 = b2 != 0xFFFFFFFFu && b1 != 0xFFFFFFFFu;
+  if (lvl2) {
+    for (uint32_t base = 0; base < L; base += kChunk) {
+      if (!one) load_chunk(base, kk, ii);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) eq_w += __popc(v[q]);
-  }
-  eq_w = __reduce_add_sync(0xffffffffu, eq_w);
-  uint32_t tot;
-  uint32_t eq_before = block_excl_scan(lane == 0 ? eq_w : 0u, wsum, &tot);
-  eq_before = __shfl_sync(0xffffffffu, eq_before, 0);
-  TTRACE(11);
-  uint32_t sel_w = 0;
-  for (int base = wbeg; base < wend; base += 256) {
-    const int w0 = base + 8 * lane;
-    uint32_t e[8], sv[8];
-    load8(eqm, w0, e);
-    load8(sel, w0, sv);
-    uint32_t pe = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) pe += __popc(e[q]);
-    const uint32_t inc = warp_incl_scan(pe, lane);
-    uint32_t before = eq_before + inc - pe;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      uint32_t keep = 0, ew = e[q];
-      while (ew && before < rem) {
-        const uint32_t low = ew & (0u - ew);
-        keep |= low;
-        ew ^= low;
-        ++before;
-      }
-      before += __popc(ew);
-      if (keep && w0 + q < nw) sel[w0 + q] = sv[q] | keep;
-      sel_w += __popc(sv[q] | keep);
+      for (int u = 0; u < kPer; ++u)
+        if (ii[u] != ~0u && (kk[u] >> 8) == p24) atomicAdd(&h3[kk[u] & 255u], 1u);
     }
-    eq_before += __shfl_sync(0xffffffffu, inc, 31);
   }
-  TTRACE(12);
-  sel_w = __reduce_add_sync(0xffffffffu, sel_w);
-  uint32_t pos0 = block_excl_scan(lane == 0 ? sel_w : 0u, wsum, &tot);
-  pos0 = __shfl_sync(0xffffffffu, pos0, 0);
-  TTRACE(13);
-  for (int base = wbeg; base < wend; base += 256) {
-    const int w0 = base + 8 * lane;
-    uint32_t v[8];
-    load8(sel, w0, v);
-    uint32_t pb = 0;
+  __syncthreads();
+  if (tid == 0) { s_bin = 0xFFFFFFFFu; s_above = 0u; }
+  if (lvl2) find_bin(h3, 256, rem, wsum, &s_bin, &s_above);
+  else __syncthreads();
+  const bool resolved = lvl2 && s_bin != 0xFFFFFFFFu;
+  const uint32_t T = (p24 << 8) | (s_bin & 255u);   // every key > T is taken, and `rem` keys == T
+  rem -= resolved ? s_above : 0u;
+  TTRACE(5);
+
+  // ---------------------------------------------------------------- 4. ordered emission
+  uint32_t gt_run = 0, tie_run = 0;
+  if (resolved) {
+    for (uint32_t base = 0; base < L; base += kChunk) {
+      if (!one) load_chunk(base, kk, ii);
+      uint32_t ngt = 0, ntie = 0;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) pb += __popc(v[q]);
-    const uint32_t inc = warp_incl_scan(pb, lane);
-    uint32_t pos = pos0 + inc - pb;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      uint32_t bits = v[q];
-      while (bits) {
-        const int bit = __ffs(bits) - 1;
-        bits &= bits - 1;
-        out[pos++] = (w0 + q) * 32 + bit;
+      for (int u = 0; u < kPer; ++u) {
+        ngt += (ii[u] != ~0u && kk[u] > T);
+        ntie += (ii[u] != ~0u && kk[u] == T);
       }
+      uint32_t tot;
+      const uint32_t ex = block_excl_scan(ngt | (ntie << 16), wsum, &tot);
+      uint32_t gtb = gt_run + (ex & 0xFFFFu), tieb = tie_run + (ex >> 16);
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        if (ii[u] == ~0u) continue;
+        if (kk[u] > T) {
+          const uint32_t pos = gtb + min(tieb, rem);
+          if (pos < (uint32_t)k) out[pos] = (int32_t)ii[u];
+          ++gtb;
+        } else if (kk[u] == T) {
+          if (tieb < rem && gtb + tieb < (uint32_t)k) out[gtb + tieb] = (int32_t)ii[u];
+          ++tieb;
+        }
+      }
+      gt_run += tot & 0xFFFFu;
+      tie_run += tot >> 16;
     }
-    pos0 += __shfl_sync(0xffffffffu, inc, 31);
   }
-  // leave the row's histogram and counters zeroed for the next call (every CTA of the row has
-  // read the histogram: each took its ticket after filtering)
-  for (int i = tid; i < kHistBins; i += kSplitThreads) hist_row[i] = 0u;
-  if (tid < 3) cnt[tid] = 0u;
+  // a consistent histogram yields exactly k; otherwise report and pad what was not written
+  const uint32_t n_out = resolved ? gt_run + min(tie_run, rem) : 0u;
+  if (n_out != (uint32_t)k) {
+    if (tid == 0) set_device_error(a.err, kErrTopkOverflow);
+    for (uint32_t i = n_out + tid; i < (uint32_t)k; i += kSplitThreads) out[i] = -1;
+  }
   TTRACE(7);
 }
 
@@ -433,15 +413,8 @@ int topk_split_ctas(int rows, int64_t n_max, int num_sms) {
 
 cudaError_t launch_topk_split(const TopkSplitArgs& a, cudaStream_t s) {
   if (a.base.rows <= 0 || a.base.k <= 0) return cudaSuccess;
-  size_t smem = 2 * (size_t)((((a.base.n_max + 31) / 32) + 3) & ~(int64_t)3) * 4 + (size_t)kCandCap * 8;
-  if (smem < (size_t)kChunk * 12) smem = (size_t)kChunk * 12;
-  static size_t configured = 0;
-  if (smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(topk_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = smem;
-  }
-  return launch_kernel(topk_split_kernel, dim3(a.G, a.base.rows), dim3(kSplitThreads), smem, s, 0, a);
+  if (a.G < 1 || a.G > kTopkSplitMaxCtas) return cudaErrorInvalidValue;
+  return launch_kernel(topk_split_kernel, dim3(a.G, a.base.rows), dim3(kSplitThreads), 0, s, 0, a);
 }
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
