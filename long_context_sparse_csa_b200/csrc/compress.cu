@@ -63,6 +63,40 @@ __device__ __forceinline__ float cluster_reduce(float v, float* slot, float* bca
   return *bcast;
 }
 
+// Cluster-wide (sum of s, max of m) over one pair per thread, in one pass: a block reduction of
+// both, one cluster barrier, then every CTA reads the CTAs' pairs through distributed shared
+// memory.  scratch: 64 floats; slot2 / bcast2: 2 floats each.  Every thread gets the result.
+__device__ __forceinline__ float2 cluster_reduce_sum_max(float s, float m, float* scratch, float* slot2,
+                                                         float* bcast2) {
+  cg::cluster_group cl = cg::this_cluster();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  s = warp_sum(s);
+  m = warp_max(m);
+  __syncthreads();
+  if (lane == 0) { scratch[wid] = s; scratch[32 + wid] = m; }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float x = lane < nw ? scratch[lane] : 0.f, y = lane < nw ? scratch[32 + lane] : -INFINITY;
+    x = warp_sum(x);
+    y = warp_max(y);
+    if (lane == 0) { slot2[0] = x; slot2[1] = y; }
+  }
+  cl.sync();
+  if (threadIdx.x < 32) {
+    float x = 0.f, y = -INFINITY;
+    if ((unsigned)lane < cl.num_blocks()) {
+      const float* r = cl.map_shared_rank(slot2, lane);
+      x = r[0];
+      y = r[1];
+    }
+    x = warp_sum(x);
+    y = warp_max(y);
+    if (lane == 0) { bcast2[0] = x; bcast2[1] = y; }
+  }
+  __syncthreads();
+  return make_float2(bcast2[0], bcast2[1]);
+}
+
 // Stores this CTA's channels of one row in the cache format.  `am` is the cluster-wide max |x|
 // over the FP8 dims (mixed format only); threads with active == false hold no channels.
 __device__ __forceinline__ void pack_slice(uint8_t* dst, const LayerArgs& L, int c0, const float v[4], bool active,
@@ -103,9 +137,9 @@ __device__ __forceinline__ float local_amax(const float v[4], int c0, int dn, bo
 // row group pools a strided subset of the completed entry's source rows with an online softmax;
 // groups merge through shared memory and the row-wide RMSNorm sum and FP8 amax are reduced over
 // the cluster.  With CL = 1 (chunked prefill) the cluster reductions are plain block reductions.
-__global__ void __launch_bounds__(512) append_compress_kernel(const __grid_constant__ AppendCompressArgs a, int CL) {
-  __shared__ float scratch[32];
-  __shared__ float red[4], bcast;
+__global__ void __launch_bounds__(256) append_compress_kernel(const __grid_constant__ AppendCompressArgs a, int CL) {
+  __shared__ float scratch[64];
+  __shared__ float red[4], bcast, bcast2[2];
   extern __shared__ float part[];                  // [RG][3][DC]
   cg::cluster_group cluster = cg::this_cluster();
   const LayerArgs& L = a.L;
@@ -137,6 +171,9 @@ __global__ void __launch_bounds__(512) append_compress_kernel(const __grid_const
   }
   CTRACE(1);
   const bool compress = valid && a.do_compress && ((r + 1) % L.m) == 0;
+  // issued now, used after the pooling
+  const float4 gk = (compress && a.gamma_kv) ? __ldg(reinterpret_cast<const float4*>(a.gamma_kv + c0))
+                                             : make_float4(1.f, 1.f, 1.f, 1.f);
 
   if (valid && a.do_append) {
     if (have_new && lead) {
@@ -224,7 +261,56 @@ __global__ void __launch_bounds__(512) append_compress_kernel(const __grid_const
     }
     CTRACE(4);
     // merge the row groups
-    if (RG > 1) {
+    if (RG >= 4) {
+      // two levels over all threads: thread (channel c, slice j) merges groups j, j+J, ..., then
+      // the lead threads merge the J slices of their channels (max first, then independent exp2)
+      float* pm = part + (size_t)rg * 3 * DC;
+      const int cl0 = ct * 4;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        pm[cl0 + k] = mx[k];
+        pm[DC + cl0 + k] = sum[k];
+        pm[2 * DC + cl0 + k] = acc[k];
+      }
+      __syncthreads();
+      const int J = (int)blockDim.x / DC;            // = RG / 4 slices per channel
+      const int c = threadIdx.x % DC, jj = threadIdx.x / DC;
+      float M = -INFINITY;
+      for (int qq = jj; qq < RG; qq += J) M = fmaxf(M, part[(size_t)qq * 3 * DC + c]);
+      float sm = 0.f, ac = 0.f;
+      for (int qq = jj; qq < RG; qq += J) {
+        const float* po = part + (size_t)qq * 3 * DC;
+        const float m2 = po[c];
+        const float f = m2 == -INFINITY ? 0.f : exp2f(m2 - M);
+        sm += po[DC + c] * f;
+        ac += po[2 * DC + c] * f;
+      }
+      __syncthreads();
+      float* p1 = part + (size_t)jj * 3 * DC;
+      p1[c] = M;
+      p1[DC + c] = sm;
+      p1[2 * DC + c] = ac;
+      __syncthreads();
+      if (lead) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int cc = cl0 + k;
+          float M2 = -INFINITY;
+          for (int q2 = 0; q2 < J; ++q2) M2 = fmaxf(M2, part[(size_t)q2 * 3 * DC + cc]);
+          float s2 = 0.f, a2 = 0.f;
+          for (int q2 = 0; q2 < J; ++q2) {
+            const float* po = part + (size_t)q2 * 3 * DC;
+            const float m2 = po[cc];
+            const float f = m2 == -INFINITY ? 0.f : exp2f(m2 - M2);
+            s2 += po[DC + cc] * f;
+            a2 += po[2 * DC + cc] * f;
+          }
+          sum[k] = s2;
+          acc[k] = a2;
+          mx[k] = M2;
+        }
+      }
+    } else if (RG > 1) {
       float* pm = part + (size_t)rg * 3 * DC;
       const int cl0 = ct * 4;
 #pragma unroll
@@ -256,20 +342,22 @@ __global__ void __launch_bounds__(512) append_compress_kernel(const __grid_const
     }
     CTRACE(5);
     float e[4] = {0.f, 0.f, 0.f, 0.f};
-    float ss = 0.f;
+    float ss = 0.f, eg = 0.f;
     if (lead) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) { e[k] = acc[k] / sum[k]; ss += e[k] * e[k]; }
+      // FP8 dims are not rotated and rs > 0: max |e * rs * gamma| = rs * max |e * gamma|, so the
+      // scale's amax rides on the same cluster reduction as the RMSNorm sum
+      if (c0 < dn)
+        eg = fmaxf(fmaxf(fabsf(e[0] * gk.x), fabsf(e[1] * gk.y)), fmaxf(fabsf(e[2] * gk.z), fabsf(e[3] * gk.w)));
     }
-    ss = cluster_reduce(block_sum(ss, scratch), &red[1], &bcast, false);
-    const float rs = 1.0f / sqrtf(ss / (float)L.D + L.eps);
-    const float4 gk = a.gamma_kv ? __ldg(reinterpret_cast<const float4*>(a.gamma_kv + c0)) : make_float4(1.f, 1.f, 1.f, 1.f);
+    const float2 red2 = cluster_reduce_sum_max(ss, eg, scratch, &red[1], bcast2);
+    const float rs = 1.0f / sqrtf(red2.x / (float)L.D + L.eps);
     e[0] *= rs * gk.x; e[1] *= rs * gk.y; e[2] *= rs * gk.z; e[3] *= rs * gk.w;
     CTRACE(6);
     rope4(e, c0, L, (double)(L.pos0 + i * (int64_t)L.m));
     CTRACE(7);
-    float am = 0.f;
-    if (L.kv_fmt == CSA_FMT_MIXED) am = cluster_reduce(block_max(local_amax(e, c0, dn, lead), scratch), &red[2], &bcast, true);
+    const float am = L.kv_fmt == CSA_FMT_MIXED ? red2.y * rs : 0.f;
     uint8_t* dst = C.entries + ((size_t)b * C.entry_cap + (size_t)i) * L.row_bytes;
     pack_slice(dst, L, c0, e, lead, am, q == 0);
     CTRACE(8);
@@ -301,7 +389,7 @@ cudaError_t launch_append_compress(const AppendCompressArgs& a, int B, int Tq, c
   if (spread && a.do_compress) {
     const int rows = (1 + a.L.ov) * a.L.m;
     rg = rows < 16 ? rows : 16;
-    while (rg > 1 && ct * rg > 512) rg >>= 1;
+    while (rg > 1 && ct * rg > 256) rg >>= 1;
   }
   const size_t smem = rg > 1 ? (size_t)rg * 3 * (a.L.D / CL) * sizeof(float) : 0;
   static size_t configured = 0;
