@@ -194,6 +194,7 @@ struct Workspace {
   size_t scores = 0, scores_bytes = 0;
   size_t topk = 0, topk_bytes = 0;
   size_t part = 0, part_bytes = 0;
+  size_t qt = 0;                        // bf16 q~ of the tcgen05 attention [rows][H][D]
   size_t total = 0;
 };
 
@@ -217,8 +218,9 @@ Workspace layout(const csa_layer_t* L, int op, int32_t Tq, int64_t n_max) {
   if (op == CSA_OP_SPARSE_ATTEND || op == CSA_OP_HCA_ATTEND || op == CSA_OP_DECODE_STEP || op == CSA_OP_PREFILL) {
     const bool dense = (op == CSA_OP_HCA_ATTEND) || !csa;
     const int64_t slots = (dense ? (n_max > 0 ? n_max : 1) : (int64_t)L->top_k) + L->window;
-    const int splits = attend_num_splits(la, (int)rows, slots, num_sms());
-    w.part = off; w.part_bytes = attend_partial_bytes(la, (int)rows, splits); off = up(off + w.part_bytes);
+    const int splits = attend_num_splits(la, dense, (int)rows, slots, num_sms());
+    w.part = off; w.part_bytes = attend_partial_bytes(la, dense, (int)rows, splits); off = up(off + w.part_bytes);
+    if (attend_path(la, dense) == 2) { w.qt = off; off = up(off + rows * (size_t)L->H * L->D * 2); }
   }
   w.total = off;
   return w;
@@ -304,7 +306,7 @@ csa_status_t make_attend_args(const csa_layer_t* L, const csa_cache_t* cache, co
                               const int64_t* q_pos, int32_t Tq, const int32_t* topk, int64_t n_max, void* out,
                               const Workspace& w, void* ws, AttendArgs& a) {
   a.L = layer_args(L);
-  if (attend_head_group(a.L) == 0 && L->H > 32)
+  if (attend_path(a.L, topk == nullptr) == 0 && L->H > 32)
     return fail(CSA_ERR_UNSUPPORTED, "attention: H=%d needs D=512 with bf16/mixed rows and H%%32==0, or H<=32", L->H);
   a.C = cache_args(cache);
   a.q = static_cast<const uint8_t*>(q);
@@ -316,21 +318,34 @@ csa_status_t make_attend_args(const csa_layer_t* L, const csa_cache_t* cache, co
   a.gamma_q = P->gamma_q;
   a.sinks = P->sinks;
   const int64_t slots = (topk ? (int64_t)L->top_k : n_max) + L->window;
-  a.splits = attend_num_splits(a.L, a.rows, slots, num_sms());
-  if (attend_partial_bytes(a.L, a.rows, a.splits) > w.part_bytes)
+  a.splits = attend_num_splits(a.L, topk == nullptr, a.rows, slots, num_sms());
+  if (attend_partial_bytes(a.L, topk == nullptr, a.rows, a.splits) > w.part_bytes)
     return fail(CSA_ERR_WORKSPACE, "workspace too small for the attention partials");
   a.part = reinterpret_cast<float*>(at(ws, w.part));
+  a.qt = w.qt ? at(ws, w.qt) : nullptr;
+  a.err = reinterpret_cast<int*>(at(ws, w.err));
   a.out = static_cast<uint8_t*>(out);
   return CSA_OK;
 }
 
+// Attention, preceded by the q~ preparation unless the caller has launched it already (run_qprep).
 csa_status_t run_attend(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P, const void* q,
                         const int64_t* q_pos, int32_t Tq, const int32_t* topk, int64_t n_max, void* out,
-                        const Workspace& w, void* ws, cudaStream_t s) {
+                        const Workspace& w, void* ws, cudaStream_t s, bool with_qprep = true) {
   AttendArgs a;
   CSA_TRY(make_attend_args(L, cache, P, q, q_pos, Tq, topk, n_max, out, w, ws, a));
-  const cudaError_t e = launch_attend(a, s);
+  cudaError_t e = with_qprep ? launch_attend_qprep(a, s) : cudaSuccess;
+  if (e == cudaSuccess) e = launch_attend(a, s);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e, "attention launch");
+}
+
+csa_status_t run_qprep(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P, const void* q,
+                       const int64_t* q_pos, int32_t Tq, const int32_t* topk, int64_t n_max, const Workspace& w,
+                       void* ws, cudaStream_t s) {
+  AttendArgs a;
+  CSA_TRY(make_attend_args(L, cache, P, q, q_pos, Tq, topk, n_max, nullptr, w, ws, a));
+  const cudaError_t e = launch_attend_qprep(a, s);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e, "q preparation launch");
 }
 
 csa_status_t check_params(const csa_layer_t* L, const csa_params_t* P, bool need_bias) {
@@ -512,7 +527,8 @@ csa_status_t csa_decode_step(const csa_layer_t* L, const csa_cache_t* cache, con
     cudaError_t e = cudaEventRecord(ss->fork, s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->s, ss->fork, 0);
     if (e != cudaSuccess) return cuda_fail(e, "csa_decode_step fork");
-    const csa_status_t sc = run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, ss->s);
+    csa_status_t sc = run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, ss->s);
+    if (sc == CSA_OK) sc = run_qprep(L, cache, P, q, q_pos, 1, tk, cache->entry_cap, w, workspace, ss->s);
     const csa_status_t si = sc == CSA_OK ? run_index_topk(L, cache, idx_q, idx_q_scale, head_w, q_pos, 1,
                                                           cache->entry_cap, tk,
                                                           reinterpret_cast<float*>(at(workspace, w.scores)), w,
@@ -523,7 +539,7 @@ csa_status_t csa_decode_step(const csa_layer_t* L, const csa_cache_t* cache, con
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
     if (si != CSA_OK) return si;
     if (e != cudaSuccess) return cuda_fail(e, "csa_decode_step join");
-    return run_attend(L, cache, P, q, q_pos, 1, tk, cache->entry_cap, out, w, workspace, s);
+    return run_attend(L, cache, P, q, q_pos, 1, tk, cache->entry_cap, out, w, workspace, s, false);
   }
   CSA_TRY(run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, s));
   CSA_TRY(run_index_topk(L, cache, idx_q, idx_q_scale, head_w, q_pos, 1, cache->entry_cap, tk,
@@ -548,6 +564,21 @@ csa_status_t hca_decode_step(const csa_layer_t* L, const csa_cache_t* cache, con
   const Workspace w = layout(L, CSA_OP_HCA_ATTEND, 1, cache->entry_cap);
   CSA_TRY(check_ws(w, workspace, ws_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  SideStream* ss = side_stream(s);
+  if (ss) {
+    // fork: the attention's query preparation on the side stream beside append+compress
+    cudaError_t e = cudaEventRecord(ss->fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->s, ss->fork, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "hca_decode_step fork");
+    const csa_status_t sq = run_qprep(L, cache, P, q, q_pos, 1, nullptr, cache->entry_cap, w, workspace, ss->s);
+    const csa_status_t sc = run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, s);
+    e = cudaEventRecord(ss->join, ss->s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
+    if (sq != CSA_OK) return sq;
+    if (sc != CSA_OK) return sc;
+    if (e != cudaSuccess) return cuda_fail(e, "hca_decode_step join");
+    return run_attend(L, cache, P, q, q_pos, 1, nullptr, cache->entry_cap, out, w, workspace, s, false);
+  }
   CSA_TRY(run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, s));
   return run_attend(L, cache, P, q, q_pos, 1, nullptr, cache->entry_cap, out, w, workspace, s);
 }

@@ -23,6 +23,7 @@
 // slots, each writes (O, m, l) and a combine kernel merges the splits with
 // the sink and applies the inverse rotation.
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace csa {
 
@@ -30,13 +31,20 @@ namespace {
 
 constexpr int kD = 512;
 constexpr int kTile = 64;
+constexpr int kH128 = 128;
 
 #ifdef CSA_TRACE
 __device__ uint64_t g_trace_a[320][16];
 #define ATRACE(slot) do { if (threadIdx.x == 0 && blockIdx.z == 0 && blockIdx.y == 0 && blockIdx.x < 320) { \
     uint64_t _t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(_t) :: "memory"); g_trace_a[blockIdx.x][(slot)] = _t; } } while (0)
+#define ATRACE_C(thr, slot) do { if (threadIdx.x == (thr) && blockIdx.z == 0 && blockIdx.y == 0 && blockIdx.x < 320) \
+    g_trace_a[blockIdx.x][(slot)] = (uint64_t)clock64(); } while (0)
+#define ATRACE_T(thr, slot) do { if (threadIdx.x == (thr) && blockIdx.z == 0 && blockIdx.y == 0 && blockIdx.x < 320) { \
+    uint64_t _t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(_t) :: "memory"); g_trace_a[blockIdx.x][(slot)] = _t; } } while (0)
 #else
 #define ATRACE(slot) ((void)0)
+#define ATRACE_T(thr, slot) ((void)0)
+#define ATRACE_C(thr, slot) ((void)0)
 #endif
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -631,6 +639,479 @@ __global__ void attend_generic_kernel(const __grid_constant__ AttendArgs a) {
   }
 }
 
+// ----------------------------------------------------------------------------- tensor-core kernel (tcgen05)
+// One CTA per (query, 128-slot split, half of the output dims), all 128 heads as the MMA's M:
+//   S[h, s]  = q~[h, :] . k_s           tcgen05 kind::f16, A = q~ (smem, two 256-dim halves in turn),
+//                                       B = the split's rows as bf16 (K-major), D = TMEM cols [0, 128)
+//   P = exp2(S*scale*log2e - m), bf16   one thread per head reads its TMEM lane
+//   O[h, half] = P . V[:, half]         A = P (smem, K-major), B = the same bf16 rows read MN-major,
+//                                       D = TMEM cols [256, 512)
+// The split's rows are gathered once into the swizzled bf16 tile that serves both products.  The
+// CTA writes (O, m, l) for the combine kernel, or, when one split covers the query, finishes the
+// output itself (sink, normalisation, inverse rotation).
+constexpr int kTcN = 128;                  // key slots per CTA (S columns, PV K)
+constexpr int kTcHalf = 256;               // output dims per CTA
+constexpr int kTcThreads = 256;
+constexpr int kTcRegion = kTcN * 128;      // one 64-dim column block of the row tile: 16 KB
+constexpr int kTcRawRow = kD + 80;         // stored row of the mixed format: 592 B
+constexpr size_t kTcPartBytes = (size_t)kD * kH128 * 2 + 2 * kH128 * 4;   // one split's partial: bf16 O/l, m, l
+constexpr int kTcX = kTcN * kTcRawRow;     // raw rows / one q~ half / P: 75,776 B
+constexpr size_t kTcSmem = 1024 + 8 * (size_t)kTcRegion + kTcX + 64 + kTcN * 8 + 4 * 128 * 4 + kTcN * 8;
+static_assert(kTcSmem <= 227 * 1024, "tcgen05 attention shared memory");
+
+// q~ = RoPE_t(RMSNorm(q) * gamma_q) in bf16, once per (query, head): one warp per head, lane l
+// holds dims [16l, 16l+16) (the rotary pairs sit in lanes 28..31).
+__global__ void __launch_bounds__(128) qprep_kernel(const __grid_constant__ AttendArgs a) {
+  const LayerArgs& L = a.L;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.y, h = blockIdx.x * 4 + warp;
+  if (h >= L.H) return;
+  const int64_t t = a.q_pos[row];
+  const size_t ab = L.act_fmt == CSA_FMT_F32 ? 4 : 2;
+  const uint8_t* qrow = a.q + ((size_t)row * L.H + h) * kD * ab;
+  float gm[16], v[16];
+  if (a.gamma_q) {
+#pragma unroll
+    for (int k = 0; k < 16; k += 4) {
+      const float4 g4 = __ldg(reinterpret_cast<const float4*>(a.gamma_q + 16 * lane + k));
+      gm[k] = g4.x; gm[k + 1] = g4.y; gm[k + 2] = g4.z; gm[k + 3] = g4.w;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) gm[k] = 1.f;
+  }
+  if (L.act_fmt == CSA_FMT_F32) {
+#pragma unroll
+    for (int k = 0; k < 16; k += 4) load_act4(qrow, CSA_FMT_F32, 16 * lane + k, v + k);
+  } else {
+    const uint4 u0 = __ldg(reinterpret_cast<const uint4*>(qrow + 2 * 16 * lane));
+    const uint4 u1 = __ldg(reinterpret_cast<const uint4*>(qrow + 2 * 16 * lane + 16));
+    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) { v[2 * k] = bf16_bits_to_f(w[k] & 0xFFFFu); v[2 * k + 1] = bf16_bits_to_f(w[k] >> 16); }
+  }
+  float cs[8], sn[8];
+  if (lane >= 28) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) rope_cos_sin((double)t, (16 * lane + 2 * k - (kD - 64)) >> 1, L, &cs[k], &sn[k]);
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) ss += v[k] * v[k];
+  ss = warp_sum(ss);
+  const float rs = 1.0f / sqrtf(ss / (float)kD + L.eps);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] *= rs * gm[k];
+  if (lane >= 28) {
+#pragma unroll
+    for (int k = 0; k < 16; k += 2) {
+      const float x0 = v[k], x1 = v[k + 1];
+      v[k] = x0 * cs[k >> 1] - x1 * sn[k >> 1];
+      v[k + 1] = x0 * sn[k >> 1] + x1 * cs[k >> 1];
+    }
+  }
+  uint4 p0, p1;
+  p0.x = pack_bf16x2(v[0], v[1]); p0.y = pack_bf16x2(v[2], v[3]);
+  p0.z = pack_bf16x2(v[4], v[5]); p0.w = pack_bf16x2(v[6], v[7]);
+  p1.x = pack_bf16x2(v[8], v[9]); p1.y = pack_bf16x2(v[10], v[11]);
+  p1.z = pack_bf16x2(v[12], v[13]); p1.w = pack_bf16x2(v[14], v[15]);
+  uint4* dst = reinterpret_cast<uint4*>(a.qt + (((size_t)row * L.H + h) * kD + 16 * lane) * 2);
+  dst[0] = p0;
+  dst[1] = p1;
+}
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_wait() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
+}
+
+// Byte offset of 16-byte piece j (dims 8j..8j+7 of a 64-dim block) of row r in a 128-byte-swizzled
+// K-major tile of rows.
+__device__ __forceinline__ uint32_t sw128(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
+
+template <int FMT>
+__global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_constant__ AttendArgs a) {
+  using namespace sm100;
+  extern __shared__ uint8_t tc_smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* KV = sm;                                        // [8 blocks][128 slots][128 B] bf16 rows
+  uint8_t* X = KV + 8 * kTcRegion;                         // raw rows, then a q~ half [4][128][128 B], then P [2][128][128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(X + kTcX);  // S half 0, S half 1, O
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  uint32_t* vbits = tmem_slot + 1;                         // [4] slot validity bitmasks
+  int* valid = reinterpret_cast<int*>(tmem_slot + 8);      // [kTcN]
+  int32_t* sidx = valid + kTcN;                            // [kTcN] entries of the selected slots (CSA)
+  float* mls = reinterpret_cast<float*>(sidx + kTcN);      // [4][128]: max, sum of each column half, per head
+  const uint8_t** rptr = reinterpret_cast<const uint8_t**>(mls + 4 * 128);   // [kTcN] stored row of each slot
+
+  const LayerArgs& L = a.L;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = blockIdx.z, dh = blockIdx.y, sp = blockIdx.x;
+  const int b = row / a.Tq;
+  ATRACE_T(0, 0);
+  const int64_t t = a.q_pos[row];
+  const SlotInfo si = slot_info(a, t);
+  const int64_t s0 = (int64_t)sp * kTcN;
+  if (a.topk)
+    for (int i = tid; i < kTcN; i += kTcThreads) {
+      const int64_t s = s0 + i;
+      sidx[i] = s < si.n_sel ? a.topk[(size_t)row * L.top_k + s] : -1;
+    }
+  if (tid == 0) {
+    for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  ATRACE_T(0, 1);
+
+  // ---------------------------------------------------------------- the split's rows -> bf16 tile
+  // Compact loops throughout: this code runs once per CTA, so its instruction fetch counts.
+  {
+    const CacheArgs& C = a.C;
+    auto row_ptr = [&](int r) -> const uint8_t* {
+      const int64_t s = s0 + r;
+      if (s < si.n_sel) {
+        const int64_t e = a.topk ? (int64_t)sidx[r] : s;
+        if (e < 0 || e >= C.entry_cap) return nullptr;
+        return C.entries + ((size_t)b * C.entry_cap + (size_t)e) * L.row_bytes;
+      }
+      if (s < si.R) {
+        const int64_t wr = si.rt - si.n_win + 1 + (s - si.n_sel);
+        return C.window + ((size_t)b * C.window_cap + (size_t)(wr % C.window_cap)) * L.row_bytes;
+      }
+      return nullptr;
+    };
+    if (tid < kTcN) {
+      const uint8_t* p = row_ptr(tid);
+      rptr[tid] = p;
+      valid[tid] = p != nullptr;
+    }
+    __syncthreads();
+    if (FMT == CSA_FMT_BF16) {
+      // bf16 rows need no conversion: 16-byte asynchronous copies straight into the swizzled tile
+      for (int idx = tid; idx < kTcN * 64; idx += kTcThreads) {
+        const int r = idx >> 6, ch = idx & 63;
+        uint8_t* dst = KV + (ch >> 3) * kTcRegion + sw128(r, ch & 7);
+        if (valid[r]) cp_async16(dst, rptr[r] + ch * 16);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      cp_async_commit_wait();
+    } else {
+      // raw rows -> X by asynchronous copies, then codes x the row's power-of-two scale -> bf16
+      // (exact) into the swizzled tile; empty slots become zero rows
+      constexpr int kCh = kTcRawRow / 16;                 // 37 chunks: 28 code, 8 rotary, 1 scale
+      for (int idx = tid; idx < kTcN * kCh; idx += kTcThreads) {
+        const int r = idx / kCh, ch = idx - r * kCh;
+        if (valid[r]) cp_async16(X + r * kTcRawRow + ch * 16, rptr[r] + ch * 16);
+      }
+      cp_async_commit_wait();
+      __syncthreads();
+#pragma unroll 1
+      for (int idx = tid; idx < kTcN * 36; idx += kTcThreads) {
+        const int r = idx / 36, ch = idx - r * 36;
+        const bool ok = valid[r] != 0;
+        const uint8_t* src = X + r * kTcRawRow;
+        if (ch < 28) {
+          uint4 lo4 = make_uint4(0u, 0u, 0u, 0u), hi4 = lo4;
+          if (ok) {
+            const uint4 c = *reinterpret_cast<const uint4*>(src + ch * 16);
+            const float sg = *reinterpret_cast<const float*>(src + kD + 64);
+            const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+            uint32_t o[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float2 lo = e4m3x2_to_float2((uint16_t)(w[q] & 0xFFFFu));
+              const float2 hi = e4m3x2_to_float2((uint16_t)(w[q] >> 16));
+              o[2 * q] = pack_bf16x2(lo.x * sg, lo.y * sg);
+              o[2 * q + 1] = pack_bf16x2(hi.x * sg, hi.y * sg);
+            }
+            lo4 = make_uint4(o[0], o[1], o[2], o[3]);
+            hi4 = make_uint4(o[4], o[5], o[6], o[7]);
+          }
+          uint8_t* blk = KV + (ch >> 2) * kTcRegion;
+          const int j0 = (2 * ch) & 7;
+          *reinterpret_cast<uint4*>(blk + sw128(r, j0)) = lo4;
+          *reinterpret_cast<uint4*>(blk + sw128(r, j0 + 1)) = hi4;
+        } else {
+          *reinterpret_cast<uint4*>(KV + 7 * kTcRegion + sw128(r, ch - 28)) =
+              ok ? *reinterpret_cast<const uint4*>(src + ch * 16) : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+    }
+  }
+  if (warp == 0) {                   // slot validity as bit masks for the softmax
+#pragma unroll
+    for (int q = 0; q < kTcN / 32; ++q) {
+      const uint32_t m = __ballot_sync(0xffffffffu, valid[32 * q + lane] != 0);
+      if (lane == 0) vbits[q] = m;
+    }
+  }
+  __syncthreads();                   // X is free again; every raw row is converted
+  ATRACE_T(0, 2);
+
+  // ---------------------------------------------------------------- S = q~ K^T (two halves of q~)
+  const uint8_t* qsrc = a.qt + (size_t)row * kH128 * kD * 2;
+  const uint32_t idesc_s = instr_desc(128, kTcN, 1u);
+  bool ok = true;
+  for (int hf = 0; hf < 2; ++hf) {
+    // q~ dims [256 hf, 256 hf + 256): 128 heads x 4 blocks x 8 pieces of 16 bytes, into X
+    for (int idx = tid; idx < 128 * 32; idx += kTcThreads) {
+      const int h = idx >> 5, c = (idx >> 3) & 3, j = idx & 7;
+      cp_async16(X + c * (128 * 128) + sw128(h, j), qsrc + ((size_t)h * kD + hf * kTcHalf + c * 64 + j * 8) * 2);
+    }
+    cp_async_commit_wait();
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        const uint64_t ad = desc_kmajor_sw128(smem_u32(X + c * (128 * 128)));
+        const uint64_t bd = desc_kmajor_sw128(smem_u32(KV + (4 * hf + c) * kTcRegion));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) umma_f16(tmem, ad + 2u * k, bd + 2u * k, idesc_s, (hf | c | k) ? 1u : 0u);
+      }
+      umma_commit(&bars[hf]);
+    }
+    // X is overwritten (next q~ half, or P) only once these MMAs have read it
+    if (ok) ok = mbar_wait(&bars[hf], 0u);
+    ATRACE_T(0, 3 + hf);
+  }
+  tc_fence_after();
+
+  // ---------------------------------------------------------------- softmax over all 8 warps
+  // Warps w and w+4 read the same TMEM lanes (heads 32(w%4)..); warps 4..7 take slots 0..63,
+  // warps 0..3 slots 64..127.  The two halves exchange their maxima and sums through shared memory.
+  const float cl2 = L.scale * kLog2e;
+  const int h = (warp & 3) * 32 + lane;
+  const int hs = warp >= 4 ? 0 : 1;                       // slot half of this warp
+  const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+  ATRACE_C(128, 12);
+  {
+    float mm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+    for (int c0 = 64 * hs; c0 < 64 * hs + 64; c0 += 32) {
+      float v[32];
+      tmem_ld_32x32b_x32(lane_addr + c0, v);
+      const uint32_t bits = vbits[c0 >> 5];
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float z = ((bits >> j) & 1u) ? v[j] * cl2 : -INFINITY;
+        mm[j & 3] = fmaxf(mm[j & 3], z);
+      }
+    }
+    mls[hs * 128 + h] = fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3]));
+  }
+  __syncthreads();
+  const float m = fmaxf(mls[h], mls[128 + h]);
+  const float ms = m == -INFINITY ? 0.f : m;
+  ATRACE_C(128, 13);
+  {
+    float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int c0 = 64 * hs; c0 < 64 * hs + 64; c0 += 32) {
+      float v[32];
+      tmem_ld_32x32b_x32(lane_addr + c0, v);
+      const uint32_t cbits = vbits[c0 >> 5];
+      tmem_wait_ld();
+      uint32_t w[16];
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        const uint32_t bits = cbits >> j;
+        const float p0 = exp2f(((bits & 1u) ? v[j] * cl2 : -INFINITY) - ms);
+        const float p1 = exp2f(((bits & 2u) ? v[j + 1] * cl2 : -INFINITY) - ms);
+        w[j >> 1] = pack_bf16x2(p0, p1);
+        ls[(j >> 1) & 3] += bf16_bits_to_f(w[j >> 1] & 0xFFFFu) + bf16_bits_to_f(w[j >> 1] >> 16);
+      }
+      uint8_t* blk = X + (c0 >> 6) * (128 * 128);
+      const int j0 = (c0 & 63) >> 3;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(blk + sw128(h, j0 + q)) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+    }
+    mls[256 + hs * 128 + h] = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+  }
+  ATRACE_C(128, 14);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  ATRACE_T(128, 9);
+  ATRACE_C(128, 15);
+  const float l = mls[256 + h] + mls[384 + h];
+
+  // ---------------------------------------------------------------- O[:, half] = P V[:, half]
+  if (tid == 0) {
+    tc_fence_after();
+    const uint32_t idesc_o = instr_desc(128, kTcHalf, 1u) | (1u << 16);   // B (the rows) MN-major
+#pragma unroll 1
+    for (int kk = 0; kk < kTcN / 16; ++kk) {
+      const uint64_t ad = desc_kmajor_sw128(smem_u32(X + (kk >> 2) * (128 * 128))) + 2u * (kk & 3);
+      const uint64_t bd = desc_mnmajor_sw128(smem_u32(KV + 4 * dh * kTcRegion + kk * 16 * 128), kTcRegion, 1024u);
+      umma_f16(tmem + 256u, ad, bd, idesc_o, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&bars[2]);
+  }
+  ATRACE_T(0, 5);
+
+  // ---------------------------------------------------------------- epilogue over all 8 warps
+  // warps 4..7 take output columns 0..127 of this half, warps 0..3 columns 128..255
+  if (ok) ok = mbar_wait(&bars[2], 0u);
+  ATRACE_T(128, 10);
+  tc_fence_after();
+  const int e0 = hs * (kTcHalf / 2);
+  if (a.splits > 1) {
+    // partial of this split: O / l in bf16 as [dim / 4][head][4] (a warp's stores are contiguous,
+    // the combine reads a head's 4 dims in one 8-byte load), then (m, l) per head in fp32.  O / l
+    // is a convex combination of value rows, so its bf16 rounding is no coarser than the output's.
+    uint8_t* part = reinterpret_cast<uint8_t*>(a.part) + ((size_t)row * a.splits + sp) * kTcPartBytes;
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    uint2* od = reinterpret_cast<uint2*>(part);
+#pragma unroll 1
+    for (int c0 = e0; c0 < e0 + kTcHalf / 2; c0 += 32) {
+      float v[32];
+      tmem_ld_32x32b_x32(lane_addr + 256u + c0, v);
+      tmem_wait_ld();
+      uint2* dst = od + (size_t)((dh * kTcHalf + c0) >> 2) * kH128 + h;
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        dst[(size_t)(j >> 2) * kH128] = make_uint2(pack_bf16x2(v[j] * inv_l, v[j + 1] * inv_l),
+                                                   pack_bf16x2(v[j + 2] * inv_l, v[j + 3] * inv_l));
+    }
+    if (dh == 0 && hs == 0)
+      reinterpret_cast<float2*>(part + (size_t)kD * kH128 * 2)[h] = make_float2(m, l);
+  } else {
+    // one split covers the query: sink, normalisation, rotation back by -t, store
+    const float sk = a.sinks[h] * kLog2e;
+    const float M = fmaxf(m, sk);
+    const float f = exp2f(m - M) / (l * exp2f(m - M) + exp2f(sk - M));
+    const size_t ab = L.act_fmt == CSA_FMT_F32 ? 4 : 2;
+    uint8_t* dst = a.out + ((size_t)row * L.H + h) * kD * ab;
+#pragma unroll 1
+    for (int c0 = e0; c0 < e0 + kTcHalf / 2; c0 += 32) {
+      float v[32];
+      tmem_ld_32x32b_x32(lane_addr + 256u + c0, v);
+      tmem_wait_ld();
+      const int d0 = dh * kTcHalf + c0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= f;
+      if (d0 >= kD - 64) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          float c, s;
+          rope_cos_sin((double)t, (d0 + j - (kD - 64)) >> 1, L, &c, &s);
+          const float x0 = v[j], x1 = v[j + 1];
+          v[j] = x0 * c + x1 * s;
+          v[j + 1] = -x0 * s + x1 * c;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) store_act4(dst, L.act_fmt, d0 + j, v + j);
+    }
+  }
+  tc_fence_before();
+  ATRACE_T(128, 11);
+  if (!ok && tid == 0) set_device_error(a.err, kErrWaitTimeout);
+  __syncthreads();
+  ATRACE_T(0, 6);
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Merge of the tcgen05 kernel's splits for 4 output dims of one query and all 128 heads: four
+// groups of 128 threads (one per head) each take every 4th split and merge them online, 8 splits
+// per step with every load of the step in flight (one 8-byte load of a head's 4 dims and one of
+// its (m, l) per split, contiguous across a warp); the groups then merge through shared memory
+// with the sink.  Normalisation and inverse rotation as in the single-split epilogue.
+__global__ void __launch_bounds__(512) attend_tc_combine_kernel(const __grid_constant__ AttendArgs a) {
+  constexpr int kU = 8;
+  __shared__ float red[4][6][kH128];
+  const LayerArgs& L = a.L;
+  const int h = threadIdx.x & 127, g = threadIdx.x >> 7;
+  const int d0 = blockIdx.x * 4, row = blockIdx.y;
+  const int S = a.splits;
+  const uint8_t* base = reinterpret_cast<const uint8_t*>(a.part) + (size_t)row * S * kTcPartBytes;
+  float Mg = -INFINITY, lg = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s0 = g; s0 < S; s0 += 4 * kU) {
+    float2 ml[kU];
+    uint2 o[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int s = s0 + 4 * u;
+      ml[u] = make_float2(-INFINITY, 0.f);
+      o[u] = make_uint2(0u, 0u);
+      if (s < S) {
+        const uint8_t* ps = base + (size_t)s * kTcPartBytes;
+        ml[u] = reinterpret_cast<const float2*>(ps + (size_t)kD * kH128 * 2)[h];
+        o[u] = reinterpret_cast<const uint2*>(ps)[(size_t)(d0 >> 2) * kH128 + h];
+      }
+    }
+    float mx = Mg;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) mx = fmaxf(mx, ml[u].x);
+    if (mx == -INFINITY) continue;
+    const float sc = exp2f(Mg - mx);                   // 0 while nothing is merged yet
+    lg *= sc;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k] *= sc;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const float f = ml[u].y * exp2f(ml[u].x - mx);  // split weight: l_s * 2^(m_s - M)
+      lg += f;
+      acc[0] += f * bf16_bits_to_f(o[u].x & 0xFFFFu);
+      acc[1] += f * bf16_bits_to_f(o[u].x >> 16);
+      acc[2] += f * bf16_bits_to_f(o[u].y & 0xFFFFu);
+      acc[3] += f * bf16_bits_to_f(o[u].y >> 16);
+    }
+    Mg = mx;
+  }
+  red[g][0][h] = Mg;
+  red[g][1][h] = lg;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) red[g][2 + k][h] = acc[k];
+  __syncthreads();
+  if (g != 0) return;
+  const float sk = a.sinks[h] * kLog2e;
+  float M = sk;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) M = fmaxf(M, red[q][0][h]);
+  float lsum = exp2f(sk - M), out[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float f = red[q][0][h] == -INFINITY ? 0.f : exp2f(red[q][0][h] - M);
+    lsum += red[q][1][h] * f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) out[k] += red[q][2 + k][h] * f;
+  }
+  const float inv = 1.f / lsum;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) out[k] *= inv;
+  if (d0 >= kD - 64) {
+    const int64_t t = a.q_pos[row];
+#pragma unroll
+    for (int k = 0; k < 4; k += 2) {
+      float c, s;
+      rope_cos_sin(-(double)t, (d0 + k - (kD - 64)) >> 1, L, &c, &s);
+      const float x0 = out[k], x1 = out[k + 1];
+      out[k] = x0 * c - x1 * s;
+      out[k + 1] = x0 * s + x1 * c;
+    }
+  }
+  uint8_t* dst = a.out + ((size_t)row * L.H + h) * kD * (L.act_fmt == CSA_FMT_F32 ? 4 : 2);
+  store_act4(dst, L.act_fmt, d0, out);
+}
+
 #ifdef CSA_TRACE
 extern "C" __attribute__((visibility("default"))) int csa_trace_read_a(uint64_t* host) {
   return (int)cudaMemcpyFromSymbol(host, g_trace_a, sizeof(g_trace_a));
@@ -661,6 +1142,15 @@ cudaError_t launch_mma(const AttendArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+int attend_path(const LayerArgs& L, bool dense) {
+  // the tcgen05 kernel pays a fixed per-CTA latency that long dense slot lists amortise; sparse
+  // top-k lists (about 1,150 slots) stay on the mma.sync kernel, which spreads them over every SM
+  if (dense && L.H == kH128 && L.D == kD && L.d_rope == 64 &&
+      (L.kv_fmt == CSA_FMT_BF16 || L.kv_fmt == CSA_FMT_MIXED))
+    return 2;
+  return attend_head_group(L) > 0 ? 1 : 0;
+}
+
 int attend_head_group(const LayerArgs& L) {
   if (L.D != kD || L.d_rope != 64) return 0;
   if (L.kv_fmt != CSA_FMT_BF16 && L.kv_fmt != CSA_FMT_MIXED) return 0;
@@ -669,7 +1159,11 @@ int attend_head_group(const LayerArgs& L) {
   return 0;
 }
 
-int attend_num_splits(const LayerArgs& L, int rows, int64_t slots, int num_sms) {
+int attend_num_splits(const LayerArgs& L, bool dense, int rows, int64_t slots, int num_sms) {
+  if (attend_path(L, dense) == 2) {
+    const int64_t s = (slots + kTcN - 1) / kTcN;
+    return (int)(s < 1 ? 1 : s);
+  }
   const int HG = attend_head_group(L);
   if (HG == 0) return 1;
   const int64_t pairs = (int64_t)rows * (L.H / HG);
@@ -681,14 +1175,37 @@ int attend_num_splits(const LayerArgs& L, int rows, int64_t slots, int num_sms) 
   return (int)want;
 }
 
-size_t attend_partial_bytes(const LayerArgs& L, int rows, int splits) {
+size_t attend_partial_bytes(const LayerArgs& L, bool dense, int rows, int splits) {
+  if (attend_path(L, dense) == 2) return splits <= 1 ? 0 : (size_t)rows * splits * kTcPartBytes;
   const int HG = attend_head_group(L);
   if (HG == 0 || splits <= 1) return 0;
   return (size_t)rows * (L.H / HG) * splits * HG * (kD + 2) * sizeof(float);
 }
 
+cudaError_t launch_attend_qprep(const AttendArgs& a, cudaStream_t s) {
+  if (a.rows <= 0 || attend_path(a.L, a.topk == nullptr) != 2) return cudaSuccess;
+  return launch_kernel(qprep_kernel, dim3((unsigned)((a.L.H + 3) / 4), (unsigned)a.rows), dim3(128), 0, s, 0, a);
+}
+
+template <int FMT>
+cudaError_t launch_tc(const AttendArgs& a, cudaStream_t s) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kTcSmem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  cudaError_t e = launch_kernel(attend_tc_kernel<FMT>, dim3((unsigned)a.splits, 2, (unsigned)a.rows), dim3(kTcThreads),
+                                kTcSmem, s, 0, a);
+  if (e != cudaSuccess || a.splits == 1) return e;
+  return launch_kernel(attend_tc_combine_kernel, dim3(kD / 4, a.rows), dim3(4 * kH128), 0, s, 0, a);
+}
+
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
   if (a.rows <= 0) return cudaSuccess;
+  if (attend_path(a.L, a.topk == nullptr) == 2)
+    return a.L.kv_fmt == CSA_FMT_MIXED ? launch_tc<CSA_FMT_MIXED>(a, s) : launch_tc<CSA_FMT_BF16>(a, s);
   const int HG = attend_head_group(a.L);
   if (HG == 0) {
     return launch_kernel(attend_generic_kernel, dim3(a.rows), dim3(a.L.H * 32), 0, s, 0, a);

@@ -116,6 +116,8 @@ struct AttendArgs {
   LayerArgs L;
   CacheArgs C;
   const uint8_t* q;         // [rows][H][D] act
+  uint8_t* qt;              // [rows][H][D] bf16 q~ = RoPE_t(RMSNorm(q) * gamma_q) (tensor-core kernel)
+  int* err;                 // device error word
   const int64_t* q_pos;     // [rows]
   int Tq, rows;
   const int32_t* topk;      // CSA: [rows][k]; null for dense (HCA)
@@ -126,10 +128,17 @@ struct AttendArgs {
   float* part;              // [rows][H/HG][splits][HG*(D+2)] partial (O, m, l)
   uint8_t* out;             // [rows][H][D] act
 };
-// Head-group size of the tensor-core attention kernel for this layer (0: generic kernel).
+// Attention kernel family: 2 = tcgen05 (dense slots, H = 128, D = 512, bf16 or mixed rows),
+// 1 = mma.sync head groups, 0 = CUDA-core generic kernel.  `dense`: every visible entry (HCA) rather
+// than a top-k list.
+int attend_path(const LayerArgs& L, bool dense);
+// Head-group size of the mma.sync kernel (0: not applicable).
 int attend_head_group(const LayerArgs& L);
-int attend_num_splits(const LayerArgs& L, int rows, int64_t slots, int num_sms);
-size_t attend_partial_bytes(const LayerArgs& L, int rows, int splits);
+int attend_num_splits(const LayerArgs& L, bool dense, int rows, int64_t slots, int num_sms);
+size_t attend_partial_bytes(const LayerArgs& L, bool dense, int rows, int splits);
+// q~ for the tcgen05 kernel (a no-op for the other kernels, which prepare q themselves); it reads
+// only q, gamma_q and q_pos, so it may run beside compression.
+cudaError_t launch_attend_qprep(const AttendArgs& a, cudaStream_t s);
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s);
 
 }  // namespace csa

@@ -165,6 +165,24 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor: MN-major operand in the 128-byte swizzle layout.  An atom is 8
+// K-rows of 128 bytes (64 consecutive MN elements of 16 bits); `lbo` is the byte distance between
+// consecutive 64-element MN groups, `sbo` between consecutive 8-row K groups.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
+// Makes this thread's generic-proxy writes to shared memory visible to the tensor core (async proxy).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Instruction descriptor: M x N tile, fp32 accumulator, both operands K-major.
 // ab_format: kind::f8f6f4 -> 0 = e4m3; kind::f16 -> 1 = bf16.
 __host__ __device__ constexpr uint32_t instr_desc(int M, int N, uint32_t ab_format) {

@@ -60,7 +60,7 @@ def test_two_calls_in_a_row_match_oracle():
 
     if not torch.cuda.is_available():
         pytest.fail("CUDA device required for -m gpu tests")
-    wl = get_workload("csa_decode_128k")
+    wl = get_workload("csa_decode_128k", B=4)     # 11.7 MB of workspace: inside the 16 MiB scratch
     layer = wl.layers[0]
     d = decode_inputs(wl, 0)
     st = LayerState.from_arrays(layer, wl.B, d)
