@@ -658,6 +658,7 @@ constexpr size_t kTcPartBytes = (size_t)kD * kH128 * 2 + 2 * kH128 * 4;   // one
 constexpr int kTcX = kTcN * kTcRawRow;     // raw rows / one q~ half / P: 75,776 B
 constexpr size_t kTcSmem = 1024 + 8 * (size_t)kTcRegion + kTcX + 64 + kTcN * 8 + 4 * 128 * 4 + kTcN * 8;
 static_assert(kTcSmem <= 227 * 1024, "tcgen05 attention shared memory");
+static_assert(kTcN == 128, "row index masks assume 128 slots per CTA");
 
 // q~ = RoPE_t(RMSNorm(q) * gamma_q) in bf16, once per (query, head): one warp per head, lane l
 // holds dims [16l, 16l+16) (the rotary pairs sit in lanes 28..31).
@@ -798,8 +799,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
     __syncthreads();
     if (FMT == CSA_FMT_BF16) {
       // bf16 rows need no conversion: 16-byte asynchronous copies straight into the swizzled tile
-      for (int idx = tid; idx < kTcN * 64; idx += kTcThreads) {
-        const int r = idx >> 6, ch = idx & 63;
+      for (int idx = tid; idx < kTcN * 64; idx += kTcThreads) {     // rows fastest: distinct banks
+        const int r = idx & (kTcN - 1), ch = idx >> 7;
         uint8_t* dst = KV + (ch >> 3) * kTcRegion + sw128(r, ch & 7);
         if (valid[r]) cp_async16(dst, rptr[r] + ch * 16);
         else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
@@ -815,9 +816,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
       }
       cp_async_commit_wait();
       __syncthreads();
-#pragma unroll 1
+      ATRACE_T(0, 7);
+      // consecutive threads take consecutive rows of one chunk: with the 128-byte swizzle their
+      // 16-byte stores fall on distinct banks (consecutive chunks of one row would land in eight
+      // different 16 KB column blocks at the same bank offset)
+#pragma unroll 3
       for (int idx = tid; idx < kTcN * 36; idx += kTcThreads) {
-        const int r = idx / 36, ch = idx - r * 36;
+        const int r = idx & (kTcN - 1), ch = idx >> 7;
         const bool ok = valid[r] != 0;
         const uint8_t* src = X + r * kTcRawRow;
         if (ch < 28) {
