@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from csa_synth import compress_inputs, decode_inputs, get_workload, prefill_inputs
-from csa_synth.configs import Layer, Workload, raw_ring_rows
+from csa_synth.configs import CSA_PRO, HCA_128K, HCA_PRO, Layer, Workload, raw_ring_rows, scaled_layer
 from long_context_sparse_csa_b200 import binding as C
 from long_context_sparse_csa_b200.state import LayerState
 from oracle import csa as O
@@ -362,6 +362,18 @@ def test_decode_short_contexts(n):
     _check_decode(wl, li=1, n=n)
 
 
+def test_decode_hca_bf16_rows_128_heads():
+    # dense attention on bf16 rows with 128 heads: the tcgen05 kernel's bf16 row path
+    wl = get_workload("hca_decode_128k", B=2, layers=(scaled_layer(HCA_128K, H=128),))
+    _check_decode(wl)
+
+
+def test_decode_csa_bf16_rows():
+    # top-k attention on bf16 rows: the mma.sync kernel's bf16 tile path
+    wl = get_workload("csa_decode_128k", B=2, layers=(scaled_layer(CSA_PRO, kv_format="bf16"),))
+    _check_decode(wl)
+
+
 def test_decode_per_sequence_positions():
     wl = get_workload("csa_decode_128k", B=3, n=6000)
     layer = wl.layers[0]
@@ -387,8 +399,9 @@ def _prefill_case(wl, Tq=None, prefix=None):
     out = torch.zeros((wl.B, pf["Tq"], layer.H, layer.D), dtype=torch.int16, device="cuda")
     topk = torch.zeros((wl.B, pf["Tq"], layer.top_k), dtype=torch.int32, device="cuda")
     ws = st.workspace("prefill", pf["Tq"], n_max)
-    C.csa_prefill(st.L, st.cache(), st.params(), dev(pf["q"]), dev(pf["idx_q"]), dev(pf["idx_q_scale"]),
-                  dev(pf["head_w"]), dev(pf["t"]), pf["Tq"], n_max, out, topk, ws)
+    opt = lambda k: dev(pf[k]) if pf.get(k) is not None else None  # noqa: E731  (HCA layers have no indexer)
+    C.csa_prefill(st.L, st.cache(), st.params(), dev(pf["q"]), opt("idx_q"), opt("idx_q_scale"),
+                  opt("head_w"), dev(pf["t"]), pf["Tq"], n_max, out, topk if layer.kind == "csa" else None, ws)
     torch.cuda.synchronize()
     _no_device_error(ws)
     return pf, st, out, topk
@@ -428,6 +441,13 @@ def test_prefill_small_ragged():
 def test_prefill_from_empty_cache():
     wl = get_workload("csa_prefill_8k")
     _check_prefill(wl, Tq=200, prefix=0, queries=[0, 1, 2, 3, 4, 5, 50, 127, 128, 129, 199])
+
+
+def test_prefill_hca_dense():
+    # HCA chunked prefill: every query of the chunk attends densely (tcgen05 kernel, one row per query,
+    # one or two 128-slot splits per query)
+    wl = get_workload("csa_prefill_8k", layers=(HCA_PRO,))
+    _check_prefill(wl, Tq=200, prefix=4096 + 2, queries=[0, 1, 62, 63, 64, 127, 128, 199])
 
 
 def test_prefill_full_size_sampled():
