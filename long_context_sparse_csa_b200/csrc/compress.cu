@@ -28,8 +28,11 @@ __device__ uint64_t g_trace_c[4][16];
 #define CTRACE(slot) do { if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) { \
     uint64_t _t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(_t) :: "memory"); \
     g_trace_c[(L.m == 4) ? 0 : 1][(slot)] = _t; } } while (0)
+#define CTRACE_C(slot) do { if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) \
+    g_trace_c[(L.m == 4) ? 0 : 1][(slot)] = (uint64_t)clock64(); } while (0)
 #else
 #define CTRACE(slot) ((void)0)
+#define CTRACE_C(slot) ((void)0)
 #endif
 
 __device__ __forceinline__ void rope4(float v[4], int c0, const LayerArgs& L, double pos) {
@@ -190,6 +193,7 @@ __global__ void __launch_bounds__(256) append_compress_kernel(const __grid_const
   }
   CTRACE(2);
   CTRACE(3);
+  CTRACE_C(10);
 
   if (compress) {
     const int64_t i = (r + 1) / L.m - 1;
@@ -260,6 +264,7 @@ __global__ void __launch_bounds__(256) append_compress_kernel(const __grid_const
       }
     }
     CTRACE(4);
+    CTRACE_C(11);
     // merge the row groups
     if (RG >= 4) {
       // two levels over all threads: thread (channel c, slice j) merges groups j, j+J, ..., then
@@ -273,17 +278,26 @@ __global__ void __launch_bounds__(256) append_compress_kernel(const __grid_const
         pm[2 * DC + cl0 + k] = acc[k];
       }
       __syncthreads();
+      CTRACE_C(14);
+      // (every slice holds exactly 4 row groups, RG = 4 J; each level issues all of its shared-
+      // memory loads before any arithmetic, so their latencies overlap)
       const int J = (int)blockDim.x / DC;            // = RG / 4 slices per channel
       const int c = threadIdx.x % DC, jj = threadIdx.x / DC;
-      float M = -INFINITY;
-      for (int qq = jj; qq < RG; qq += J) M = fmaxf(M, part[(size_t)qq * 3 * DC + c]);
+      float m4[4], s4[4], a4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float* po = part + (size_t)(jj + u * J) * 3 * DC;
+        m4[u] = po[c];
+        s4[u] = po[DC + c];
+        a4[u] = po[2 * DC + c];
+      }
+      const float M = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       float sm = 0.f, ac = 0.f;
-      for (int qq = jj; qq < RG; qq += J) {
-        const float* po = part + (size_t)qq * 3 * DC;
-        const float m2 = po[c];
-        const float f = m2 == -INFINITY ? 0.f : exp2f(m2 - M);
-        sm += po[DC + c] * f;
-        ac += po[2 * DC + c] * f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float f = m4[u] == -INFINITY ? 0.f : exp2f(m4[u] - M);
+        sm += s4[u] * f;
+        ac += a4[u] * f;
       }
       __syncthreads();
       float* p1 = part + (size_t)jj * 3 * DC;
@@ -291,23 +305,44 @@ __global__ void __launch_bounds__(256) append_compress_kernel(const __grid_const
       p1[DC + c] = sm;
       p1[2 * DC + c] = ac;
       __syncthreads();
+      // level 2: one thread per channel merges the J slices; the result goes to the slot after the
+      // slices (RG = 4 J > J), where the lead threads pick up their 4 channels
+      float* pf = part + (size_t)J * 3 * DC;
+      if ((int)threadIdx.x < DC) {
+        constexpr int kMaxJ = 8;                     // RG <= 32
+        const int cc = threadIdx.x;
+        float mj[kMaxJ], sj[kMaxJ], aj[kMaxJ];
+#pragma unroll
+        for (int q2 = 0; q2 < kMaxJ; ++q2) {
+          mj[q2] = -INFINITY; sj[q2] = 0.f; aj[q2] = 0.f;
+          if (q2 < J) {
+            const float* po = part + (size_t)q2 * 3 * DC;
+            mj[q2] = po[cc];
+            sj[q2] = po[DC + cc];
+            aj[q2] = po[2 * DC + cc];
+          }
+        }
+        float M2 = mj[0];
+#pragma unroll
+        for (int q2 = 1; q2 < kMaxJ; ++q2) M2 = fmaxf(M2, mj[q2]);
+        float s2 = 0.f, a2 = 0.f;
+#pragma unroll
+        for (int q2 = 0; q2 < kMaxJ; ++q2) {
+          const float f = mj[q2] == -INFINITY ? 0.f : exp2f(mj[q2] - M2);
+          s2 += sj[q2] * f;
+          a2 += aj[q2] * f;
+        }
+        pf[cc] = M2;
+        pf[DC + cc] = s2;
+        pf[2 * DC + cc] = a2;
+      }
+      __syncthreads();
       if (lead) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int cc = cl0 + k;
-          float M2 = -INFINITY;
-          for (int q2 = 0; q2 < J; ++q2) M2 = fmaxf(M2, part[(size_t)q2 * 3 * DC + cc]);
-          float s2 = 0.f, a2 = 0.f;
-          for (int q2 = 0; q2 < J; ++q2) {
-            const float* po = part + (size_t)q2 * 3 * DC;
-            const float m2 = po[cc];
-            const float f = m2 == -INFINITY ? 0.f : exp2f(m2 - M2);
-            s2 += po[DC + cc] * f;
-            a2 += po[2 * DC + cc] * f;
-          }
-          sum[k] = s2;
-          acc[k] = a2;
-          mx[k] = M2;
+          mx[k] = pf[cl0 + k];
+          sum[k] = pf[DC + cl0 + k];
+          acc[k] = pf[2 * DC + cl0 + k];
         }
       }
     } else if (RG > 1) {
@@ -341,6 +376,7 @@ __global__ void __launch_bounds__(256) append_compress_kernel(const __grid_const
       }
     }
     CTRACE(5);
+    CTRACE_C(12);
     float e[4] = {0.f, 0.f, 0.f, 0.f};
     float ss = 0.f, eg = 0.f;
     if (lead) {
@@ -355,12 +391,14 @@ __global__ void __launch_bounds__(256) append_compress_kernel(const __grid_const
     const float rs = 1.0f / sqrtf(red2.x / (float)L.D + L.eps);
     e[0] *= rs * gk.x; e[1] *= rs * gk.y; e[2] *= rs * gk.z; e[3] *= rs * gk.w;
     CTRACE(6);
+    CTRACE_C(13);
     rope4(e, c0, L, (double)(L.pos0 + i * (int64_t)L.m));
     CTRACE(7);
     const float am = L.kv_fmt == CSA_FMT_MIXED ? red2.y * rs : 0.f;
     uint8_t* dst = C.entries + ((size_t)b * C.entry_cap + (size_t)i) * L.row_bytes;
     pack_slice(dst, L, c0, e, lead, am, q == 0);
     CTRACE(8);
+    CTRACE_C(15);
   }
   // no CTA may leave while a peer can still read its shared memory
   cluster.sync();
@@ -377,19 +415,32 @@ extern "C" __attribute__((visibility("default"))) int csa_trace_read_c(uint64_t*
 cudaError_t launch_append_compress(const AppendCompressArgs& a, int B, int Tq, cudaStream_t s) {
   // decode (few tokens): a cluster of CL CTAs per token splits the channels, and row groups split
   // the entry's source rows; a chunk has parallelism across tokens and runs one CTA per token.
+  // A long pooling window (HCA's m' = 128 rows) takes a 16-CTA cluster (32 channels per CTA, up to
+  // 32 row groups): twice the SMs issue its row loads; short windows keep 8 CTAs of 64 channels.
   const bool spread = Tq <= 64;
+  const int rows = (1 + a.L.ov) * a.L.m;
+  const bool wide = spread && a.do_compress && rows >= 64 && a.L.D >= 512;
   int CL = 1;
   if (spread) {
-    CL = a.L.D / 64;
-    if (CL > 8) CL = 8;
+    CL = wide ? a.L.D / 32 : a.L.D / 64;
+    const int cmax = wide ? 16 : 8;
+    if (CL > cmax) CL = cmax;
     if (CL < 1) CL = 1;
   }
   const int ct = a.L.D / CL / 4;
   int rg = 1;
   if (spread && a.do_compress) {
-    const int rows = (1 + a.L.ov) * a.L.m;
-    rg = rows < 16 ? rows : 16;
+    const int rg_max = wide ? 32 : 16;
+    rg = rows < rg_max ? rows : rg_max;
     while (rg > 1 && ct * rg > 256) rg >>= 1;
+  }
+  if (CL > 8) {
+    static bool nonportable = false;
+    if (!nonportable) {
+      cudaError_t e = cudaFuncSetAttribute(append_compress_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+      nonportable = true;
+    }
   }
   const size_t smem = rg > 1 ? (size_t)rg * 3 * (a.L.D / CL) * sizeof(float) : 0;
   static size_t configured = 0;
