@@ -22,8 +22,15 @@
 // accumulation and an online softmax.  When several CTAs split one query's
 // slots, each writes (O, m, l) and a combine kernel merges the splits with
 // the sink and applies the inverse rotation.
+#include <cooperative_groups.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "kernels.h"
 #include "sm100.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace csa {
 
@@ -41,10 +48,14 @@ __device__ uint64_t g_trace_a[320][16];
     g_trace_a[blockIdx.x][(slot)] = (uint64_t)clock64(); } while (0)
 #define ATRACE_T(thr, slot) do { if (threadIdx.x == (thr) && blockIdx.z == 0 && blockIdx.y == 0 && blockIdx.x < 320) { \
     uint64_t _t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(_t) :: "memory"); g_trace_a[blockIdx.x][(slot)] = _t; } } while (0)
+__device__ uint64_t g_trace_cb[256][4];
+#define CBTRACE(slot) do { if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.x < 256) { \
+    uint64_t _t; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(_t) :: "memory"); g_trace_cb[blockIdx.x][(slot)] = _t; } } while (0)
 #else
 #define ATRACE(slot) ((void)0)
 #define ATRACE_T(thr, slot) ((void)0)
 #define ATRACE_C(thr, slot) ((void)0)
+#define CBTRACE(slot) ((void)0)
 #endif
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -76,6 +87,15 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const uint8_t* p) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t w) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&w));
 }
 
 // Two e4m3 codes (low byte first) -> two floats, via the hardware e4m3x2 -> f16x2 conversion.
@@ -640,23 +660,29 @@ __global__ void attend_generic_kernel(const __grid_constant__ AttendArgs a) {
 }
 
 // ----------------------------------------------------------------------------- tensor-core kernel (tcgen05)
-// One CTA per (query, 128-slot split, half of the output dims), all 128 heads as the MMA's M:
-//   S[h, s]  = q~[h, :] . k_s           tcgen05 kind::f16, A = q~ (smem, two 256-dim halves in turn),
-//                                       B = the split's rows as bf16 (K-major), D = TMEM cols [0, 128)
-//   P = exp2(S*scale*log2e - m), bf16   one thread per head reads its TMEM lane
-//   O[h, half] = P . V[:, half]         A = P (smem, K-major), B = the same bf16 rows read MN-major,
-//                                       D = TMEM cols [256, 512)
-// The split's rows are gathered once into the swizzled bf16 tile that serves both products.  The
-// CTA writes (O, m, l) for the combine kernel, or, when one split covers the query, finishes the
-// output itself (sink, normalisation, inverse rotation).
+// A cluster of two CTAs per (query, 128-slot split); CTA dh owns dims [256 dh, 256 dh + 256) of
+// q~ and of the split's rows (keys and values are the same rows), all 128 heads as the MMA's M:
+//   S_dh[h, s] = q~[h, half] . k_s[half]   tcgen05 kind::f16, A = q~ half (smem, by the tensor
+//                                          memory accelerator), B = the half rows as bf16 (K-major),
+//                                          D = TMEM cols [0, 128)
+//   S = S_0 + S_1                          each thread sends its 64 partial scores to its twin in
+//                                          the peer CTA through distributed shared memory
+//   P = exp2(S*scale*log2e - m), bf16      one thread per (head, slot half), from registers
+//   O[h, half] = P . V[:, half]            A = P (smem, K-major), B = the same bf16 half rows read
+//                                          MN-major, D = TMEM cols [256, 512)
+// Each CTA thus reads half of q~ and half of each row, and the q~ copy overlaps the rows' copy and
+// conversion.  The CTA writes (O, m, l) of its half for the combine kernel, or, when one split
+// covers the query, finishes its half of the output (sink, normalisation, inverse rotation).
 constexpr int kTcN = 128;                  // key slots per CTA (S columns, PV K)
 constexpr int kTcHalf = 256;               // output dims per CTA
 constexpr int kTcThreads = 256;
 constexpr int kTcRegion = kTcN * 128;      // one 64-dim column block of the row tile: 16 KB
-constexpr int kTcRawRow = kD + 80;         // stored row of the mixed format: 592 B
+constexpr int kTcHalfRow = 336;           // a half of a stored mixed-format row in X (<= 21 pieces)
 constexpr size_t kTcPartBytes = (size_t)kD * kH128 * 2 + 2 * kH128 * 4;   // one split's partial: bf16 O/l, m, l
-constexpr int kTcX = kTcN * kTcRawRow;     // raw rows / one q~ half / P: 75,776 B
+constexpr int kTcX = kTcN * kTcHalfRow;    // raw half rows / P: 43,008 B
 constexpr size_t kTcSmem = 1024 + 8 * (size_t)kTcRegion + kTcX + 64 + kTcN * 8 + 4 * 128 * 4 + kTcN * 8;
+static_assert(kTcX >= 2 * 128 * 128, "P fits where the raw half rows were");
+static_assert(kTcX % 1024 == 0, "X stays 1024-byte aligned");
 static_assert(kTcSmem <= 227 * 1024, "tcgen05 attention shared memory");
 static_assert(kTcN == 128, "row index masks assume 128 slots per CTA");
 
@@ -733,13 +759,15 @@ __device__ __forceinline__ void cp_async_commit_wait() {
 __device__ __forceinline__ uint32_t sw128(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
 
 template <int FMT>
-__global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_constant__ AttendArgs a) {
+__global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                                 const __grid_constant__ AttendArgs a) {
   using namespace sm100;
   extern __shared__ uint8_t tc_smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* KV = sm;                                        // [8 blocks][128 slots][128 B] bf16 rows
-  uint8_t* X = KV + 8 * kTcRegion;                         // raw rows, then a q~ half [4][128][128 B], then P [2][128][128 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(X + kTcX);  // S half 0, S half 1, O
+  uint8_t* KV = sm;                                        // [4 blocks][128 slots][128 B] bf16: this CTA's dims
+  uint8_t* Q = KV + 4 * kTcRegion;                         // q~ half [4][128][128 B], then the peer's S partial
+  uint8_t* X = Q + 4 * kTcRegion;                          // raw half rows, then P [2][128][128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(X + kTcX);  // S, (unused), O, q~
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
   uint32_t* vbits = tmem_slot + 1;                         // [4] slot validity bitmasks
   int* valid = reinterpret_cast<int*>(tmem_slot + 8);      // [kTcN]
@@ -747,11 +775,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   float* mls = reinterpret_cast<float*>(sidx + kTcN);      // [4][128]: max, sum of each column half, per head
   const uint8_t** rptr = reinterpret_cast<const uint8_t**>(mls + 4 * 128);   // [kTcN] stored row of each slot
 
+  cg::cluster_group cluster = cg::this_cluster();
   const LayerArgs& L = a.L;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int row = blockIdx.z, dh = blockIdx.y, sp = blockIdx.x;
+  const int row = blockIdx.z, dh = (int)cluster.block_rank(), sp = blockIdx.x >> 1;
   const int b = row / a.Tq;
   ATRACE_T(0, 0);
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+    fence_barrier_init();
+    // q~ dims [256 dh, 256 dh + 256) with the tensor memory accelerator: four 64-dim boxes of 128
+    // heads, 128-byte swizzled (the K-major operand layout); in flight while the rows come in
+    mbar_arrive_expect_tx(&bars[3], 4u * 128u * 128u);
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) tma_load_2d(Q + c * (128 * 128), &qmap, &bars[3], dh * kTcHalf + c * 64, row * kH128);
+  }
   const int64_t t = a.q_pos[row];
   const SlotInfo si = slot_info(a, t);
   const int64_t s0 = (int64_t)sp * kTcN;
@@ -760,10 +798,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
       const int64_t s = s0 + i;
       sidx[i] = s < si.n_sel ? a.topk[(size_t)row * L.top_k + s] : -1;
     }
-  if (tid == 0) {
-    for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
-    fence_barrier_init();
-  }
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -774,7 +808,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   const uint32_t tmem = *tmem_slot;
   ATRACE_T(0, 1);
 
-  // ---------------------------------------------------------------- the split's rows -> bf16 tile
+  // ---------------------------------------------------------------- this CTA's half of the rows -> bf16 tile
   // Compact loops throughout: this code runs once per CTA, so its instruction fetch counts.
   {
     const CacheArgs& C = a.C;
@@ -798,38 +832,41 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
     }
     __syncthreads();
     if (FMT == CSA_FMT_BF16) {
-      // bf16 rows need no conversion: 16-byte asynchronous copies straight into the swizzled tile
-      for (int idx = tid; idx < kTcN * 64; idx += kTcThreads) {     // rows fastest: distinct banks
+      // bf16 rows need no conversion: this half's 32 pieces of 16 bytes straight into the swizzled tile
+      for (int idx = tid; idx < kTcN * 32; idx += kTcThreads) {     // rows fastest: distinct banks
         const int r = idx & (kTcN - 1), ch = idx >> 7;
         uint8_t* dst = KV + (ch >> 3) * kTcRegion + sw128(r, ch & 7);
-        if (valid[r]) cp_async16(dst, rptr[r] + ch * 16);
+        if (valid[r]) cp_async16(dst, rptr[r] + (dh * 32 + ch) * 16);
         else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
       }
       cp_async_commit_wait();
     } else {
-      // raw rows -> X by asynchronous copies, then codes x the row's power-of-two scale -> bf16
-      // (exact) into the swizzled tile; empty slots become zero rows
-      constexpr int kCh = kTcRawRow / 16;                 // 37 chunks: 28 code, 8 rotary, 1 scale
-      for (int idx = tid; idx < kTcN * kCh; idx += kTcThreads) {
-        const int r = idx / kCh, ch = idx - r * kCh;
-        if (valid[r]) cp_async16(X + r * kTcRawRow + ch * 16, rptr[r] + ch * 16);
+      // The stored row: 448 e4m3 codes, 64 bf16 rotary dims, the fp32 power-of-two scale (+ pad).
+      // Half 0 takes codes 0..255 and the scale (17 pieces); half 1 codes 256..447, the rotary
+      // dims and the scale (21 pieces), each at kTcHalfRow bytes per row of X.
+      const int npc = dh ? 21 : 17;
+      for (int idx = tid; idx < kTcN * npc; idx += kTcThreads) {
+        const int r = idx / npc, pc = idx - r * npc;
+        const int src = dh ? kTcHalf + 16 * pc : (pc < 16 ? 16 * pc : kD + 64);
+        if (valid[r]) cp_async16(X + r * kTcHalfRow + pc * 16, rptr[r] + src);
       }
       cp_async_commit_wait();
       __syncthreads();
       ATRACE_T(0, 7);
-      // consecutive threads take consecutive rows of one chunk: with the 128-byte swizzle their
-      // 16-byte stores fall on distinct banks (consecutive chunks of one row would land in eight
-      // different 16 KB column blocks at the same bank offset)
-#pragma unroll 3
-      for (int idx = tid; idx < kTcN * 36; idx += kTcThreads) {
-        const int r = idx & (kTcN - 1), ch = idx >> 7;
+      // codes x the row's scale -> bf16 (exact), rotary dims copied; consecutive threads take
+      // consecutive rows of one piece, so their swizzled 16-byte stores fall on distinct banks
+      const int ncode = dh ? 12 : 16, nit = dh ? 20 : 16;
+      const int sc_off = dh ? 320 : 256;
+#pragma unroll 2
+      for (int idx = tid; idx < kTcN * nit; idx += kTcThreads) {
+        const int r = idx & (kTcN - 1), it = idx >> 7;
         const bool ok = valid[r] != 0;
-        const uint8_t* src = X + r * kTcRawRow;
-        if (ch < 28) {
+        const uint8_t* src = X + r * kTcHalfRow;
+        if (it < ncode) {
           uint4 lo4 = make_uint4(0u, 0u, 0u, 0u), hi4 = lo4;
           if (ok) {
-            const uint4 c = *reinterpret_cast<const uint4*>(src + ch * 16);
-            const float sg = *reinterpret_cast<const float*>(src + kD + 64);
+            const uint4 c = *reinterpret_cast<const uint4*>(src + it * 16);
+            const float sg = *reinterpret_cast<const float*>(src + sc_off);
             const uint32_t w[4] = {c.x, c.y, c.z, c.w};
             uint32_t o[8];
 #pragma unroll
@@ -842,13 +879,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
             lo4 = make_uint4(o[0], o[1], o[2], o[3]);
             hi4 = make_uint4(o[4], o[5], o[6], o[7]);
           }
-          uint8_t* blk = KV + (ch >> 2) * kTcRegion;
-          const int j0 = (2 * ch) & 7;
+          uint8_t* blk = KV + (it >> 2) * kTcRegion;
+          const int j0 = (2 * it) & 7;
           *reinterpret_cast<uint4*>(blk + sw128(r, j0)) = lo4;
           *reinterpret_cast<uint4*>(blk + sw128(r, j0 + 1)) = hi4;
         } else {
-          *reinterpret_cast<uint4*>(KV + 7 * kTcRegion + sw128(r, ch - 28)) =
-              ok ? *reinterpret_cast<const uint4*>(src + ch * 16) : make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(KV + 3 * kTcRegion + sw128(r, it - 12)) =
+              ok ? *reinterpret_cast<const uint4*>(src + 192 + (it - 12) * 16) : make_uint4(0u, 0u, 0u, 0u);
         }
       }
     }
@@ -860,58 +897,83 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
       if (lane == 0) vbits[q] = m;
     }
   }
+  fence_proxy_async_smem();
   __syncthreads();                   // X is free again; every raw row is converted
   ATRACE_T(0, 2);
 
-  // ---------------------------------------------------------------- S = q~ K^T (two halves of q~)
-  const uint8_t* qsrc = a.qt + (size_t)row * kH128 * kD * 2;
+  // ---------------------------------------------------------------- S partial = q~[:, half] K[:, half]^T
   const uint32_t idesc_s = instr_desc(128, kTcN, 1u);
   bool ok = true;
-  for (int hf = 0; hf < 2; ++hf) {
-    // q~ dims [256 hf, 256 hf + 256): 128 heads x 4 blocks x 8 pieces of 16 bytes, into X
-    for (int idx = tid; idx < 128 * 32; idx += kTcThreads) {
-      const int h = idx >> 5, c = (idx >> 3) & 3, j = idx & 7;
-      cp_async16(X + c * (128 * 128) + sw128(h, j), qsrc + ((size_t)h * kD + hf * kTcHalf + c * 64 + j * 8) * 2);
-    }
-    cp_async_commit_wait();
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
+  if (tid == 0) {
+    ok = mbar_wait(&bars[3], 0u);
+    if (ok) {
       tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
-        const uint64_t ad = desc_kmajor_sw128(smem_u32(X + c * (128 * 128)));
-        const uint64_t bd = desc_kmajor_sw128(smem_u32(KV + (4 * hf + c) * kTcRegion));
+        const uint64_t ad = desc_kmajor_sw128(smem_u32(Q + c * (128 * 128)));
+        const uint64_t bd = desc_kmajor_sw128(smem_u32(KV + c * kTcRegion));
 #pragma unroll
-        for (int k = 0; k < 4; ++k) umma_f16(tmem, ad + 2u * k, bd + 2u * k, idesc_s, (hf | c | k) ? 1u : 0u);
+        for (int k = 0; k < 4; ++k) umma_f16(tmem, ad + 2u * k, bd + 2u * k, idesc_s, (c | k) ? 1u : 0u);
       }
-      umma_commit(&bars[hf]);
+      umma_commit(&bars[0]);
     }
-    // X is overwritten (next q~ half, or P) only once these MMAs have read it
-    if (ok) ok = mbar_wait(&bars[hf], 0u);
-    ATRACE_T(0, 3 + hf);
   }
+  if (ok) ok = mbar_wait(&bars[0], 0u);
   tc_fence_after();
+  ATRACE_T(0, 3);
 
-  // ---------------------------------------------------------------- softmax over all 8 warps
+  // ---------------------------------------------------------------- S = the two partials (cluster pair)
   // Warps w and w+4 read the same TMEM lanes (heads 32(w%4)..); warps 4..7 take slots 0..63,
-  // warps 0..3 slots 64..127.  The two halves exchange their maxima and sums through shared memory.
+  // warps 0..3 slots 64..127.  Each thread sends its 64 partial scores, rounded to fp16, to the
+  // thread with the same (head, slot half) in the peer CTA, into the peer's q~ region (free once
+  // the peer's MMAs have read it: the first cluster barrier), as [slot half][8 groups of 8][head]
+  // 16-byte pieces.  The fp16 rounding (2^-11 relative) is finer than P's own bf16 rounding.
   const float cl2 = L.scale * kLog2e;
   const int h = (warp & 3) * 32 + lane;
   const int hs = warp >= 4 ? 0 : 1;                       // slot half of this warp
   const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+  float s[64];
+  tmem_ld_32x32b_x32(lane_addr + 64 * hs, s);
+  tmem_ld_32x32b_x32(lane_addr + 64 * hs + 32, s + 32);
+  tmem_wait_ld();
+  cluster.sync();
+  ATRACE_T(0, 4);
+  {
+    uint4* peer = reinterpret_cast<uint4*>(cluster.map_shared_rank(Q, dh ^ 1)) + (size_t)hs * 8 * kH128 + h;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float* v = s + 8 * j;
+      peer[(size_t)j * kH128] = make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]),
+                                           pack_f16x2(v[6], v[7]));
+    }
+  }
+  cluster.sync();
+  ATRACE_T(0, 8);
+  {
+    const uint4* mine = reinterpret_cast<const uint4*>(Q) + (size_t)hs * 8 * kH128 + h;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint4 v = mine[(size_t)j * kH128];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = unpack_f16x2(w[q]);
+        s[8 * j + 2 * q] += f.x;
+        s[8 * j + 2 * q + 1] += f.y;
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- softmax from registers
   ATRACE_C(128, 12);
   {
     float mm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-    for (int c0 = 64 * hs; c0 < 64 * hs + 64; c0 += 32) {
-      float v[32];
-      tmem_ld_32x32b_x32(lane_addr + c0, v);
-      const uint32_t bits = vbits[c0 >> 5];
-      tmem_wait_ld();
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint32_t bits = vbits[2 * hs + q];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const float z = ((bits >> j) & 1u) ? v[j] * cl2 : -INFINITY;
+        const float z = ((bits >> j) & 1u) ? s[32 * q + j] * cl2 : -INFINITY;
         mm[j & 3] = fmaxf(mm[j & 3], z);
       }
     }
@@ -923,26 +985,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   ATRACE_C(128, 13);
   {
     float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-    for (int c0 = 64 * hs; c0 < 64 * hs + 64; c0 += 32) {
-      float v[32];
-      tmem_ld_32x32b_x32(lane_addr + c0, v);
-      const uint32_t cbits = vbits[c0 >> 5];
-      tmem_wait_ld();
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint32_t cbits = vbits[2 * hs + q];
       uint32_t w[16];
 #pragma unroll
       for (int j = 0; j < 32; j += 2) {
         const uint32_t bits = cbits >> j;
-        const float p0 = exp2f(((bits & 1u) ? v[j] * cl2 : -INFINITY) - ms);
-        const float p1 = exp2f(((bits & 2u) ? v[j + 1] * cl2 : -INFINITY) - ms);
+        const float p0 = exp2f(((bits & 1u) ? s[32 * q + j] * cl2 : -INFINITY) - ms);
+        const float p1 = exp2f(((bits & 2u) ? s[32 * q + j + 1] * cl2 : -INFINITY) - ms);
         w[j >> 1] = pack_bf16x2(p0, p1);
         ls[(j >> 1) & 3] += bf16_bits_to_f(w[j >> 1] & 0xFFFFu) + bf16_bits_to_f(w[j >> 1] >> 16);
       }
-      uint8_t* blk = X + (c0 >> 6) * (128 * 128);
-      const int j0 = (c0 & 63) >> 3;
+      uint8_t* blk = X + hs * (128 * 128);
+      const int j0 = 4 * q;
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(blk + sw128(h, j0 + q)) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<uint4*>(blk + sw128(h, j0 + u)) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
     }
     mls[256 + hs * 128 + h] = (ls[0] + ls[1]) + (ls[2] + ls[3]);
   }
@@ -961,7 +1020,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
 #pragma unroll 1
     for (int kk = 0; kk < kTcN / 16; ++kk) {
       const uint64_t ad = desc_kmajor_sw128(smem_u32(X + (kk >> 2) * (128 * 128))) + 2u * (kk & 3);
-      const uint64_t bd = desc_mnmajor_sw128(smem_u32(KV + 4 * dh * kTcRegion + kk * 16 * 128), kTcRegion, 1024u);
+      const uint64_t bd = desc_mnmajor_sw128(smem_u32(KV + kk * 16 * 128), kTcRegion, 1024u);
       umma_f16(tmem + 256u, ad, bd, idesc_o, kk > 0 ? 1u : 0u);
     }
     umma_commit(&bars[2]);
@@ -1046,6 +1105,7 @@ __global__ void __launch_bounds__(512) attend_tc_combine_kernel(const __grid_con
   const int h = threadIdx.x & 127, g = threadIdx.x >> 7;
   const int d0 = blockIdx.x * 4, row = blockIdx.y;
   const int S = a.splits;
+  CBTRACE(0);
   const uint8_t* base = reinterpret_cast<const uint8_t*>(a.part) + (size_t)row * S * kTcPartBytes;
   float Mg = -INFINITY, lg = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
   for (int s0 = g; s0 < S; s0 += 4 * kU) {
@@ -1081,6 +1141,7 @@ __global__ void __launch_bounds__(512) attend_tc_combine_kernel(const __grid_con
     }
     Mg = mx;
   }
+  CBTRACE(1);
   red[g][0][h] = Mg;
   red[g][1][h] = lg;
 #pragma unroll
@@ -1115,9 +1176,13 @@ __global__ void __launch_bounds__(512) attend_tc_combine_kernel(const __grid_con
   }
   uint8_t* dst = a.out + ((size_t)row * L.H + h) * kD * (L.act_fmt == CSA_FMT_F32 ? 4 : 2);
   store_act4(dst, L.act_fmt, d0, out);
+  CBTRACE(2);
 }
 
 #ifdef CSA_TRACE
+extern "C" __attribute__((visibility("default"))) int csa_trace_read_cb(uint64_t* host) {
+  return (int)cudaMemcpyFromSymbol(host, g_trace_cb, sizeof(g_trace_cb));
+}
 extern "C" __attribute__((visibility("default"))) int csa_trace_read_a(uint64_t* host) {
   return (int)cudaMemcpyFromSymbol(host, g_trace_a, sizeof(g_trace_a));
 }
@@ -1192,6 +1257,32 @@ cudaError_t launch_attend_qprep(const AttendArgs& a, cudaStream_t s) {
   return launch_kernel(qprep_kernel, dim3((unsigned)((a.L.H + 3) / 4), (unsigned)a.rows), dim3(128), 0, s, 0, a);
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 tma_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// q~ [rows * 128 heads][512] bf16 as boxes of 64 dims x 128 heads, 128-byte swizzled.
+bool make_qt_map(CUtensorMap* m, const void* qt, int rows) {
+  auto fn = tma_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows * kH128};
+  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kH128};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(qt), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int FMT>
 cudaError_t launch_tc(const AttendArgs& a, cudaStream_t s) {
   static bool configured = false;
@@ -1201,8 +1292,10 @@ cudaError_t launch_tc(const AttendArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  cudaError_t e = launch_kernel(attend_tc_kernel<FMT>, dim3((unsigned)a.splits, 2, (unsigned)a.rows), dim3(kTcThreads),
-                                kTcSmem, s, 0, a);
+  CUtensorMap qmap;
+  if (!make_qt_map(&qmap, a.qt, a.rows)) return cudaErrorInvalidValue;
+  cudaError_t e = launch_kernel(attend_tc_kernel<FMT>, dim3((unsigned)(2 * a.splits), 1, (unsigned)a.rows),
+                                dim3(kTcThreads), kTcSmem, s, 2, qmap, a);
   if (e != cudaSuccess || a.splits == 1) return e;
   return launch_kernel(attend_tc_combine_kernel, dim3(kD / 4, a.rows), dim3(4 * kH128), 0, s, 0, a);
 }
