@@ -1213,9 +1213,11 @@ cudaError_t launch_mma(const AttendArgs& a, cudaStream_t s) {
 }  // namespace
 
 int attend_path(const LayerArgs& L, bool dense) {
-  // the tcgen05 kernel pays a fixed per-CTA latency that long dense slot lists amortise; sparse
-  // top-k lists (about 1,150 slots) stay on the mma.sync kernel, which spreads them over every SM
-  if (dense && L.H == kH128 && L.D == kD && L.d_rope == 64 &&
+  // 128 heads of 512 dims take the tcgen05 kernel, dense and top-k alike (a top-k list of about
+  // 1,150 slots is 9 cluster pairs, measured faster than the mma.sync kernel over every SM);
+  // other head counts take the mma.sync kernel
+  (void)dense;
+  if (L.H == kH128 && L.D == kD && L.d_rope == 64 &&
       (L.kv_fmt == CSA_FMT_BF16 || L.kv_fmt == CSA_FMT_MIXED))
     return 2;
   return attend_head_group(L) > 0 ? 1 : 0;
