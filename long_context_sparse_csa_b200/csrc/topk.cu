@@ -277,18 +277,21 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
   // ---------------------------------------------------------------- 3. last CTA of the row resolves
   __syncthreads();                   // every list entry and histogram add of this CTA is issued ...
   if (tid == 0) {
-    __threadfence();                 // ... and released (cumulatively) before the ticket
-    s_last = atomicAdd(cnt + 2, 1u) == (uint32_t)G - 1 ? 1u : 0u;
+    __threadfence();                 // ... and released (cumulatively) before the ticket; the ticket
+    uint32_t old;                    // acquires, and the barrier below passes that on to the CTA
+    asm volatile("atom.add.acquire.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(cnt + 2) : "memory");
+    s_last = old == (uint32_t)G - 1 ? 1u : 0u;
   }
   __syncthreads();
   TTRACE(3);
   if (!s_last) return;
-  __threadfence();
+  TTRACE(8);
   // second level: bits 19..8 of the bin-b1 keys (its loads overlap the slice counts' below)
   uint32_t rem = (uint32_t)k - n_above1;       // >= 1 when the histogram is consistent
   if (tid == 0) { s_bin = 0xFFFFFFFFu; s_above = 0u; }
   const uint32_t c_mine = tid < G ? __ldcg(counts + tid) : 0u;
   find_bin_hist(hist2_row, rem, wsum, &s_bin, &s_above);
+  TTRACE(9);
   const uint32_t b2 = s_bin;
   rem -= s_above;
   const uint32_t p24 = (b1 << 12) | b2;        // top 24 bits of T
@@ -303,11 +306,8 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
     if (tid < 256) h3[tid] = 0u;
   }
   __syncthreads();
+  TTRACE(10);
   const uint32_t L = s_off[G];
-  // every CTA of the row read both histograms' bins before its ticket: leave them zeroed now
-  for (int i = tid; i < kHistBins; i += kSplitThreads) { hist_row[i] = 0u; hist2_row[i] = 0u; }
-  if (tid < 3) cnt[tid] = 0u;
-  TTRACE(4);
   // entries p = base + kPer*tid + u of the concatenation (index ~0u past the end)
   auto load_chunk = [&](uint32_t base, uint32_t kk[kPer], uint32_t ii[kPer]) {
     const uint32_t p0 = base + kPer * (uint32_t)tid;
@@ -336,6 +336,22 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
   const bool one = L <= (uint32_t)kChunk;      // the usual case: the list stays in registers
   uint32_t kk[kPer], ii[kPer];
   if (one) load_chunk(0, kk, ii);
+  // every CTA of the row read both histograms' bins before its ticket: leave them zeroed now,
+  // while the list's loads are in flight
+  {
+    uint4* h1 = reinterpret_cast<uint4*>(hist_row);
+    uint4* h2 = reinterpret_cast<uint4*>(hist2_row);
+    for (int i = tid; i < kHistBins / 4; i += kSplitThreads) {
+      h1[i] = make_uint4(0u, 0u, 0u, 0u);
+      h2[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (tid < 3) cnt[tid] = 0u;
+  }
+  TTRACE(4);
+#ifdef CSA_TRACE
+  if (one) { uint32_t x = 0; for (int u = 0; u < kPer; ++u) x += kk[u]; if (x == 12345u) s_bin = x; }
+#endif
+  TTRACE(11);
 
   // third level: the low 8 bits of the keys whose top 24 bits are p24
   const bool lvl2 = b2 != 0xFFFFFFFFu && b1 != 0xFFFFFFFFu;
@@ -348,9 +364,24 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
     }
   }
   __syncthreads();
-  if (tid == 0) { s_bin = 0xFFFFFFFFu; s_above = 0u; }
-  if (lvl2) find_bin(h3, 256, rem, wsum, &s_bin, &s_above);
-  else __syncthreads();
+  TTRACE(12);
+  if (tid < 32) {
+    // one warp: lane l holds bins 255-8l .. 248-8l (descending)
+    uint32_t c[8], c_local = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) { c[q] = lvl2 ? h3[255 - 8 * tid - q] : 0u; c_local += c[q]; }
+    uint32_t above = warp_incl_scan(c_local, tid) - c_local;
+    uint32_t bin = 0xFFFFFFFFu, ab = 0u;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (above < rem && rem <= above + c[q]) { bin = (uint32_t)(255 - 8 * tid - q); ab = above; }
+      above += c[q];
+    }
+    const uint32_t hit = __ballot_sync(0xffffffffu, bin != 0xFFFFFFFFu);
+    if (tid == 0 && !hit) { s_bin = 0xFFFFFFFFu; s_above = 0u; }
+    if (bin != 0xFFFFFFFFu) { s_bin = bin; s_above = ab; }
+  }
+  __syncthreads();
   const bool resolved = lvl2 && s_bin != 0xFFFFFFFFu;
   const uint32_t T = (p24 << 8) | (s_bin & 255u);   // every key > T is taken, and `rem` keys == T
   rem -= resolved ? s_above : 0u;
