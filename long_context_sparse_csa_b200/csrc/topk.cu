@@ -236,6 +236,18 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
   auto slice_lo = [&](int gg) { return (int)((int64_t)nv * gg / G); };
 
   TTRACE(0);
+  // the slice's first scores do not depend on the histogram: their loads overlap its reads
+  const int lo = slice_lo(g), hi = slice_lo(g + 1);
+  const float* sc = A.scores + (size_t)row * A.n_max;
+  auto load_scores = [&](int cb, int ce, float vals[kPer]) {
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = cb + tid * kPer + u;           // a thread's kPer consecutive scores
+      vals[u] = i < ce ? __ldcg(sc + i) : 0.f;
+    }
+  };
+  float vals[kPer];
+  load_scores(lo, min(lo + kChunk, hi), vals);
   // ---------------------------------------------------------------- 1. bin b1 of the k-th largest key
   if (tid == 0) { s_bin = 0xFFFFFFFFu; s_above = 0u; }   // stays so if the histogram holds fewer than k
   find_bin_hist(hist_row, (uint32_t)k, wsum, &s_bin, &s_above);
@@ -243,17 +255,10 @@ __global__ void __launch_bounds__(kSplitThreads, 1) topk_split_kernel(const __gr
   TTRACE(1);
 
   // ---------------------------------------------------------------- 2. filter this CTA's slice
-  const int lo = slice_lo(g), hi = slice_lo(g + 1);
-  const float* sc = A.scores + (size_t)row * A.n_max;
   uint32_t n_mine = 0;
   for (int cb = lo; cb < hi; cb += kChunk) {
     const int ce = min(cb + kChunk, hi);
-    float vals[kPer];
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int i = cb + tid * kPer + u;           // a thread's kPer consecutive scores
-      vals[u] = i < ce ? __ldcg(sc + i) : 0.f;
-    }
+    if (cb != lo) load_scores(cb, ce, vals);
     uint32_t keys[kPer], n = 0;
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
