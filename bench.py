@@ -407,8 +407,9 @@ def run_ours(args):
     idx_ms = [c[1][0].elapsed_time(c[1][1]) for c in cycles] if has_csa else []
 
     # ------------------------------------------------------------------ per-kernel timeline (diagnostic, untimed)
-    labels = {"csa": ["append+compress", "indexer scores", "top-k", "attention", "combine"],
-              "hca": ["append+compress", "attention", "combine"]}
+    # launch order of the sequential (diagnostic) step: the second stream is off while it is timed
+    labels = {"csa": ["append+compress", "indexer scores", "top-k", "q preparation", "attention", "combine"],
+              "hca": ["append+compress", "q preparation", "attention", "combine"]}
     tl_events = []
     g_tl = torch.cuda.CUDAGraph()
     for lay in layers:
