@@ -45,7 +45,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="csa_hca_decode_1m",
-                   choices=["csa_hca_decode_1m", "csa_decode_128k", "hca_decode_128k"])
+                   choices=["csa_hca_decode_1m", "csa_decode_128k", "hca_decode_128k", "csa_prefill_8k"])
     p.add_argument("--replicas", type=int, default=8)
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -539,10 +539,93 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ----------------------------------------------------------------------------- chunked prefill (diagnostic mode)
+
+def run_prefill(args):
+    """Times csa_prefill on the 8,192-query chunk (one GPU): tokens/s, the launch list of one call
+    (CUDA events before each launch), and the indexer's FP8 and the attention's BF16 TFLOP/s against
+    the measured dense BF16 peak (FP8 = 2x, the nominal ratio).  Not the headline line: the
+    workload's inputs (512 MiB of queries alone) exceed L2, so calls run back to back."""
+    import torch
+    from csa_synth import get_workload, prefill_inputs
+    from long_context_sparse_csa_b200 import binding as C
+    from long_context_sparse_csa_b200.state import LayerState, to_device
+    wl = get_workload(args.workload)
+    layer = wl.layers[0]
+    pf = prefill_inputs(wl)
+    st = LayerState.from_arrays(layer, wl.B, pf, raw_key="raw", gate_key="gate", raw_base=pf["raw_first_row"])
+    Tq, n_max = pf["Tq"], pf["n"] // layer.m
+    out = torch.zeros((wl.B, Tq, layer.H, layer.D), dtype=torch.int16, device="cuda")
+    topk = torch.zeros((wl.B, Tq, layer.top_k), dtype=torch.int32, device="cuda")
+    ws = st.workspace("prefill", Tq, n_max)
+    io = {k: to_device(pf[k]) for k in ("q", "idx_q", "idx_q_scale", "head_w", "t")}
+
+    def call():
+        C.csa_prefill(st.L, st.cache(), st.params(), io["q"], io["idx_q"], io["idx_q_scale"], io["head_w"], io["t"],
+                      Tq, n_max, out, topk, ws)
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 10))
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.sample()
+    w0 = time.perf_counter()
+    e0.record()
+    for _ in range(steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    w1 = time.perf_counter()
+    clocks.sample()
+    clocks.stop()
+    ms = e0.elapsed_time(e1) / steps
+    # launch list of one call
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(17)]
+    for x in evs:                      # recorded once here, so torch accepts the library's records
+        x.record()
+    torch.cuda.synchronize()
+    C.csa_profile_timeline(evs[:16])
+    call()
+    n = C.csa_profile_timeline_count()
+    C.csa_profile_timeline(None)
+    evs[n].record()
+    torch.cuda.synchronize()
+    launches_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(n)]
+    # work of the chunk: every query's visible entries (indexer) and its top-k + window rows (attention)
+    t = pf["t"][0]
+    n_vis = np.minimum((t + 1) // layer.m, n_max).astype(np.float64)
+    idx_flops = 2.0 * layer.H_I * layer.d_I * float(n_vis.sum()) * wl.B
+    rows = np.minimum(n_vis, layer.top_k) + np.minimum(t + 1, layer.window)
+    att_flops = 4.0 * layer.H * layer.D * float(rows.sum()) * wl.B
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16_peak, note = float(json.load(f)["bf16_tflops"]), "of measured"
+    except (OSError, KeyError, ValueError):
+        bf16_peak, note = 1590.0, "of fallback"
+    longest = sorted(range(n), key=lambda i: -launches_ms[i])
+    line = {"metric": "prefill tok/s (8,192-query CSA chunk after a 65,536-token prefix)",
+            "value": wl.B * Tq / (ms / 1e3), "unit": "tok/s", "n_gpus": 1, "steps": steps, "warmup": max(3, args.warmup),
+            "ms_per_call": ms, "higher_is_better": True, "dtype": "e4m3+bf16 (fp32 accumulate)", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.B, "queries": Tq, "prefix": pf["prefix"], "heads": layer.H,
+                       "kv_dim": layer.D, "kv_format": layer.kv_format, "top_k": layer.top_k,
+                       "l2": "inputs larger than L2 (queries alone 512 MiB)"},
+            "launch_ms": [round(x, 3) for x in launches_ms],
+            "work": {"indexer_fp8_tflop": idx_flops / 1e12, "attention_bf16_tflop": att_flops / 1e12},
+            "tensor": {"bf16_peak_tflops": bf16_peak, "fp8_peak_tflops": 2 * bf16_peak, "peak_source": note},
+            "longest_launches": [{"launch": i, "ms": round(launches_ms[i], 3)} for i in longest[:3]],
+            "clocks": clocks.summary(w0, w1)}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "csa_prefill_8k":
+        run_prefill(args)
     else:
         run_ours(args)
 
