@@ -140,6 +140,16 @@ __device__ __forceinline__ const uint8_t* slot_row(const AttendArgs& a, const Sl
   return nullptr;
 }
 
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_wait() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 template <int HG, int FMT>
 __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_constant__ AttendArgs a) {
   constexpr int NW = HG / 4;          // warps
@@ -148,10 +158,15 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
   constexpr int DW = kD / NW;         // output dims per warp in P*V
   constexpr int NTW = DW / 8;         // n-tiles per warp in P*V
 
+  // bf16 rows need no conversion: they arrive by asynchronous copies into two tile buffers, the
+  // next tile's copies in flight while the current tile is computed
+  constexpr bool kAsync = FMT == CSA_FMT_BF16;
+  constexpr int kBufs = kAsync ? 2 : 1;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* Qs = smem;                                   // [HG][1024]  bf16 q~
-  uint8_t* Ks = Qs + HG * 1024;                         // [64][1024]  bf16 key/value tile
-  uint8_t* Ps = Ks + kTile * 1024;                      // [HG][128]   bf16 probabilities
+  uint8_t* Kbuf = Qs + HG * 1024;                       // [kBufs][64][1024]  bf16 key/value tiles
+  uint8_t* Ks = Kbuf;                                   // the current tile
+  uint8_t* Ps = Kbuf + kBufs * kTile * 1024;            // [HG][128]   bf16 probabilities
   float* pmax = reinterpret_cast<float*>(Ps + HG * 128);  // [4][HG]
   float* psum = pmax + 4 * HG;                          // [4][HG]
   float* m_run = psum + 4 * HG;                         // [HG]
@@ -159,7 +174,8 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
   float* corr = l_run + HG;                             // [HG]
   float* cs = corr + HG;                                // [32]
   float* sn = cs + 32;                                  // [32]
-  const uint8_t** rowptr = reinterpret_cast<const uint8_t**>(sn + 32);  // [64]
+  const uint8_t** rowbuf = reinterpret_cast<const uint8_t**>(sn + 32);  // [kBufs][64]
+  const uint8_t** rowptr = rowbuf;                      // rows of the current tile
 
   const LayerArgs& L = a.L;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -234,11 +250,26 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
       }
     }
   };
+  // kAsync: every 16-byte piece of a 64-row tile by an asynchronous copy (empty slots -> zero rows)
+  auto gather_async = [&](uint8_t* dst, const uint8_t* const* rp) {
+    for (int idx = tid; idx < kTile * 64; idx += NT) {
+      const int rr = idx >> 6, ch = idx & 63;
+      uint8_t* d = dst + swz(rr, ch, 1024);
+      const uint8_t* p = rp[rr];
+      if (p) cp_async16(d, p + ch * 16);
+      else *reinterpret_cast<uint4*>(d) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
   Gl gl;
   if (t0 < t1) {
     if (tid < kTile) rowptr[tid] = slot_row(a, si, row, b, t0 * kTile + tid);
     __syncthreads();
-    gather_load(gl);
+    if constexpr (kAsync) {
+      gather_async(Kbuf, rowbuf);
+      cp_async_commit();
+    } else {
+      gather_load(gl);
+    }
   }
 
   // ---------------------------------------------------------------- q~ = RoPE_t(RMSNorm(q) * gamma_q), bf16
@@ -316,13 +347,31 @@ __global__ void __launch_bounds__(HG * 8, 1) attend_mma_kernel(const __grid_cons
   ATRACE(1);
   int ti = 0;
   for (int64_t tile = t0; tile < t1; ++tile, ++ti) {
-    if (tile != t0) {
-      if (tid < kTile) rowptr[tid] = slot_row(a, si, row, b, tile * kTile + tid);
+    if constexpr (kAsync) {
+      const int cur = ti & 1;
+      Ks = Kbuf + cur * kTile * 1024;
+      rowptr = rowbuf + cur * kTile;
+      if (tile + 1 < t1) {
+        // the other buffer was last read by the previous tile, which ended with a block barrier
+        const uint8_t** rp = rowbuf + (cur ^ 1) * kTile;
+        if (tid < kTile) rp[tid] = slot_row(a, si, row, b, (tile + 1) * kTile + tid);
+        __syncthreads();
+        gather_async(Kbuf + (cur ^ 1) * kTile * 1024, rp);
+        cp_async_commit();
+        cp_async_wait_group<1>();        // this tile's copies: the older group
+      } else {
+        cp_async_wait_group<0>();
+      }
       __syncthreads();
-      gather_load(gl);
+    } else {
+      if (tile != t0) {
+        if (tid < kTile) rowptr[tid] = slot_row(a, si, row, b, tile * kTile + tid);
+        __syncthreads();
+        gather_load(gl);
+      }
+      gather_store(gl);
+      __syncthreads();
     }
-    gather_store(gl);
-    __syncthreads();
     if (ti < 2) ATRACE(2 + 4 * ti);
 
     // ------------------------------------------------------------ S = Q K^T for (heads mt*16.., slots np*16..)
@@ -747,12 +796,6 @@ __global__ void __launch_bounds__(128) qprep_kernel(const __grid_constant__ Atte
   dst[1] = p1;
 }
 
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)), "l"(gmem_src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit_wait() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
-}
 
 // Byte offset of 16-byte piece j (dims 8j..8j+7 of a 64-dim block) of row r in a 128-byte-swizzled
 // K-major tile of rows.
@@ -1188,15 +1231,16 @@ extern "C" __attribute__((visibility("default"))) int csa_trace_read_a(uint64_t*
 }
 #endif
 
-template <int HG>
+template <int HG, int FMT>
 size_t mma_smem_bytes() {
-  return (size_t)HG * 1024 + (size_t)kTile * 1024 + (size_t)HG * 128 + (11 * HG + 64) * sizeof(float) +
-         kTile * sizeof(void*);
+  const size_t bufs = FMT == CSA_FMT_BF16 ? 2 : 1;
+  return (size_t)HG * 1024 + bufs * kTile * 1024 + (size_t)HG * 128 + (11 * HG + 64) * sizeof(float) +
+         bufs * kTile * sizeof(void*);
 }
 
 template <int HG, int FMT>
 cudaError_t launch_mma(const AttendArgs& a, cudaStream_t s) {
-  const size_t smem = mma_smem_bytes<HG>();
+  const size_t smem = mma_smem_bytes<HG, FMT>();
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(attend_mma_kernel<HG, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
