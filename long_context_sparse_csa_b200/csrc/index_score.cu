@@ -30,7 +30,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kMaxStages = 6;                 // prefill ring depth; decode runs 4 stages, 2 CTAs per SM
+constexpr int kMaxStages = 6;                 // ring depth bound: decode runs 4 stages, prefill 2 (2 CTAs per SM)
 constexpr int kTileE = 128;                 // entries per tile (MMA M)
 constexpr int kDI = 128;                    // index-key bytes per entry
 constexpr int kTileBytes = kTileE * kDI;    // 16 KB
@@ -131,9 +131,11 @@ struct EpiSmem {
   float wq[kMaxQH];           // w * qs (used when every scale is positive)
   int pos[kMaxQH / 16];       // 1 when all of the query's index-query scales are > 0
   int64_t nv[kMaxQH / 16];    // visible entries per query (QN <= 16)
-  uint32_t hist[kHistBins];   // score histogram of the current group (decode); 16-byte aligned
   float ks[kKsChunk][kTileE]; // key scales of the current chunk of items (each thread its own entry)
+  uint32_t hist[kHistBins];   // score histogram of the current group (decode only: the prefill
+                              // instantiation allocates the struct without it); 16-byte aligned
 };
+constexpr size_t kEpiSmemNoHist = sizeof(EpiSmem) - sizeof(uint32_t) * kHistBins;
 
 __device__ __forceinline__ void epi_bar() { asm volatile("barrier.sync.aligned 5, 128;" ::: "memory"); }
 // Set-up barrier: the producer warp arrives without waiting, the other five warps wait.
@@ -201,7 +203,7 @@ __device__ __forceinline__ void load_key_scales(const IndexArgs& a, const Sched&
 // kHI > 0: decode specialisation (one query per group, kHI index heads, head weights in registers);
 // kHI == 0: any QN x H_I (prefill).
 template <int kStages, int kHI>
-__global__ void __launch_bounds__(kThreads, kHI > 0 ? 2 : 1)
+__global__ void __launch_bounds__(kThreads, 2)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                       const __grid_constant__ IndexArgs a, int N, int nacc, uint32_t tmem_cols) {
   extern __shared__ uint8_t smem_raw[];
@@ -375,7 +377,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     // Every epilogue warp runs the same sequence of named barriers whatever happens (a wait that
     // times out only stops the warp's work), so the 128-thread barrier can never be left short.
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const bool use_hist = a.hist != nullptr && a.QN == 1;
+    const bool use_hist = kHI > 0 && a.hist != nullptr && a.QN == 1;
     const int QH = a.QN * a.H_I;
     if (use_hist)
       for (int i = te; i < kHistBins; i += 128) es->hist[i] = 0u;
@@ -660,16 +662,18 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
   CUtensorMap kmap, qmap;
   if (!make_map(&kmap, a.idx_k, (uint64_t)a.B * a.entry_cap, kTileE)) return cudaErrorInvalidValue;
   if (!make_map(&qmap, a.idx_q, (uint64_t)a.B * a.Tq * a.H_I, (uint32_t)N)) return cudaErrorInvalidValue;
-  const int nacc = N <= 128 ? 4 : 2;
+  const bool decode = a.Tq == 1;
+  // two CTAs per SM in both modes (two independent pipelines, twice the epilogue warps); their TMEM
+  // shares the SM's 512 columns: decode 4 accumulators of N <= 64 columns, prefill one of N = 256
+  const int nacc = decode ? 4 : 1;
   uint32_t cols = 32;
   while (cols < (uint32_t)(nacc * N)) cols <<= 1;
-  const bool decode = a.Tq == 1;
-  const int stages = decode ? 4 : 6;
+  const int stages = decode ? 4 : 2;
   const size_t smem = 1024 + (size_t)stages * kTileBytes + 2 * (size_t)N * kDI + ((sizeof(Barriers) + 15) & ~size_t(15)) +
-                     sizeof(EpiSmem) + 64;
+                     (decode ? sizeof(EpiSmem) : kEpiSmemNoHist) + 64;
   static size_t configured[4] = {0, 0, 0, 0};
   const int ki = !decode ? 0 : a.H_I == 16 ? 1 : a.H_I == 32 ? 2 : 3;
-  auto kern = ki == 0 ? index_score_tc_kernel<6, 0>
+  auto kern = ki == 0 ? index_score_tc_kernel<2, 0>
             : ki == 1 ? index_score_tc_kernel<4, 16>
             : ki == 2 ? index_score_tc_kernel<4, 32>
                       : index_score_tc_kernel<4, 64>;
@@ -678,8 +682,7 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     configured[ki] = smem;
   }
-  // decode: two CTAs per SM (two independent pipelines); each CTA's smem and TMEM allow it
-  const int64_t ctas = decode ? 2 * (int64_t)num_sms : num_sms;
+  const int64_t ctas = 2 * (int64_t)num_sms;
   const int64_t grid = a.total_items < ctas ? a.total_items : ctas;
   return launch_kernel(kern, dim3((unsigned)grid), dim3(kThreads), smem, s, 0, kmap, qmap, a, N, nacc, cols);
 }
