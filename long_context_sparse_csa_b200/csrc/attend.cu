@@ -722,18 +722,23 @@ __global__ void attend_generic_kernel(const __grid_constant__ AttendArgs a) {
 // Each CTA thus reads half of q~ and half of each row, and the q~ copy overlaps the rows' copy and
 // conversion.  The CTA writes (O, m, l) of its half for the combine kernel, or, when one split
 // covers the query, finishes its half of the output (sink, normalisation, inverse rotation).
-constexpr int kTcN = 128;                  // key slots per CTA (S columns, PV K)
+constexpr int kTcN = 128;                  // key slots per CTA of a dense slot list (S columns, PV K)
+constexpr int kTcNSparse = 64;             // ... of a top-k list: 18 cluster pairs for 1,152 slots
 constexpr int kTcHalf = 256;               // output dims per CTA
 constexpr int kTcThreads = 256;
-constexpr int kTcRegion = kTcN * 128;      // one 64-dim column block of the row tile: 16 KB
+constexpr int kTcQBlock = 128 * 128;       // one 64-dim column block of q~ (128 heads): 16 KB
 constexpr int kTcHalfRow = 336;           // a half of a stored mixed-format row in X (<= 21 pieces)
 constexpr size_t kTcPartBytes = (size_t)kD * kH128 * 2 + 2 * kH128 * 4;   // one split's partial: bf16 O/l, m, l
-constexpr int kTcX = kTcN * kTcHalfRow;    // raw half rows / P: 43,008 B
-constexpr size_t kTcSmem = 1024 + 8 * (size_t)kTcRegion + kTcX + 64 + kTcN * 8 + 4 * 128 * 4 + kTcN * 8;
-static_assert(kTcX >= 2 * 128 * 128, "P fits where the raw half rows were");
-static_assert(kTcX % 1024 == 0, "X stays 1024-byte aligned");
-static_assert(kTcSmem <= 227 * 1024, "tcgen05 attention shared memory");
-static_assert(kTcN == 128, "row index masks assume 128 slots per CTA");
+// X holds the raw half rows, then P [N / 64 blocks][128 heads][128 B]; 1024-byte multiple
+__host__ __device__ constexpr int tc_x_bytes(int n) {
+  const int raw = n * kTcHalfRow, p = (n / 64) * kTcQBlock;
+  return ((raw > p ? raw : p) + 1023) / 1024 * 1024;
+}
+constexpr size_t tc_smem_bytes(int n) {
+  return 1024 + 4 * (size_t)n * 128 + 4 * (size_t)kTcQBlock + tc_x_bytes(n) + 64 + n * 8 + 4 * 128 * 4 + n * 8;
+}
+static_assert(tc_x_bytes(kTcN) == kTcN * kTcHalfRow, "X at 128 slots: the raw half rows");
+static_assert(tc_smem_bytes(kTcN) <= 227 * 1024, "tcgen05 attention shared memory");
 
 // q~ = RoPE_t(RMSNorm(q) * gamma_q) in bf16, once per (query, head): one warp per head, lane l
 // holds dims [16l, 16l+16) (the rotary pairs sit in lanes 28..31).
@@ -801,22 +806,27 @@ __global__ void __launch_bounds__(128) qprep_kernel(const __grid_constant__ Atte
 // K-major tile of rows.
 __device__ __forceinline__ uint32_t sw128(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
 
-template <int FMT>
+template <int FMT, int kN>
 __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                                                                  const __grid_constant__ AttendArgs a) {
   using namespace sm100;
+  static_assert(kN == 64 || kN == 128, "64 or 128 slots per CTA");
+  constexpr int kRegion = kN * 128;          // one 64-dim column block of the row tile
+  constexpr int kLogN = kN == 128 ? 7 : 6;
+  constexpr int kHalf = kN / 2;              // slots per softmax thread
+  constexpr int kX = tc_x_bytes(kN);
   extern __shared__ uint8_t tc_smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* KV = sm;                                        // [4 blocks][128 slots][128 B] bf16: this CTA's dims
-  uint8_t* Q = KV + 4 * kTcRegion;                         // q~ half [4][128][128 B], then the peer's S partial
-  uint8_t* X = Q + 4 * kTcRegion;                          // raw half rows, then P [2][128][128 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(X + kTcX);  // S, (unused), O, q~
+  uint8_t* Q = KV + 4 * kRegion;                           // q~ half [4][128][128 B], then the peer's S partial
+  uint8_t* X = Q + 4 * kTcQBlock;                          // raw half rows, then P [N / 64][128][128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(X + kX);    // S, (unused), O, q~
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
   uint32_t* vbits = tmem_slot + 1;                         // [4] slot validity bitmasks
-  int* valid = reinterpret_cast<int*>(tmem_slot + 8);      // [kTcN]
-  int32_t* sidx = valid + kTcN;                            // [kTcN] entries of the selected slots (CSA)
-  float* mls = reinterpret_cast<float*>(sidx + kTcN);      // [4][128]: max, sum of each column half, per head
-  const uint8_t** rptr = reinterpret_cast<const uint8_t**>(mls + 4 * 128);   // [kTcN] stored row of each slot
+  int* valid = reinterpret_cast<int*>(tmem_slot + 8);      // [kN]
+  int32_t* sidx = valid + kN;                            // [kN] entries of the selected slots (CSA)
+  float* mls = reinterpret_cast<float*>(sidx + kN);      // [4][128]: max, sum of each column half, per head
+  const uint8_t** rptr = reinterpret_cast<const uint8_t**>(mls + 4 * 128);   // [kN] stored row of each slot
 
   cg::cluster_group cluster = cg::this_cluster();
   const LayerArgs& L = a.L;
@@ -835,9 +845,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   }
   const int64_t t = a.q_pos[row];
   const SlotInfo si = slot_info(a, t);
-  const int64_t s0 = (int64_t)sp * kTcN;
+  const int64_t s0 = (int64_t)sp * kN;
   if (a.topk)
-    for (int i = tid; i < kTcN; i += kTcThreads) {
+    for (int i = tid; i < kN; i += kTcThreads) {
       const int64_t s = s0 + i;
       sidx[i] = s < si.n_sel ? a.topk[(size_t)row * L.top_k + s] : -1;
     }
@@ -868,7 +878,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
       }
       return nullptr;
     };
-    if (tid < kTcN) {
+    if (tid < kN) {
       const uint8_t* p = row_ptr(tid);
       rptr[tid] = p;
       valid[tid] = p != nullptr;
@@ -876,9 +886,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
     __syncthreads();
     if (FMT == CSA_FMT_BF16) {
       // bf16 rows need no conversion: this half's 32 pieces of 16 bytes straight into the swizzled tile
-      for (int idx = tid; idx < kTcN * 32; idx += kTcThreads) {     // rows fastest: distinct banks
-        const int r = idx & (kTcN - 1), ch = idx >> 7;
-        uint8_t* dst = KV + (ch >> 3) * kTcRegion + sw128(r, ch & 7);
+      for (int idx = tid; idx < kN * 32; idx += kTcThreads) {     // rows fastest: distinct banks
+        const int r = idx & (kN - 1), ch = idx >> kLogN;
+        uint8_t* dst = KV + (ch >> 3) * kRegion + sw128(r, ch & 7);
         if (valid[r]) cp_async16(dst, rptr[r] + (dh * 32 + ch) * 16);
         else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
       }
@@ -888,7 +898,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
       // Half 0 takes codes 0..255 and the scale (17 pieces); half 1 codes 256..447, the rotary
       // dims and the scale (21 pieces), each at kTcHalfRow bytes per row of X.
       const int npc = dh ? 21 : 17;
-      for (int idx = tid; idx < kTcN * npc; idx += kTcThreads) {
+      for (int idx = tid; idx < kN * npc; idx += kTcThreads) {
         const int r = idx / npc, pc = idx - r * npc;
         const int src = dh ? kTcHalf + 16 * pc : (pc < 16 ? 16 * pc : kD + 64);
         if (valid[r]) cp_async16(X + r * kTcHalfRow + pc * 16, rptr[r] + src);
@@ -901,8 +911,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
       const int ncode = dh ? 12 : 16, nit = dh ? 20 : 16;
       const int sc_off = dh ? 320 : 256;
 #pragma unroll 2
-      for (int idx = tid; idx < kTcN * nit; idx += kTcThreads) {
-        const int r = idx & (kTcN - 1), it = idx >> 7;
+      for (int idx = tid; idx < kN * nit; idx += kTcThreads) {
+        const int r = idx & (kN - 1), it = idx >> kLogN;
         const bool ok = valid[r] != 0;
         const uint8_t* src = X + r * kTcHalfRow;
         if (it < ncode) {
@@ -922,12 +932,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
             lo4 = make_uint4(o[0], o[1], o[2], o[3]);
             hi4 = make_uint4(o[4], o[5], o[6], o[7]);
           }
-          uint8_t* blk = KV + (it >> 2) * kTcRegion;
+          uint8_t* blk = KV + (it >> 2) * kRegion;
           const int j0 = (2 * it) & 7;
           *reinterpret_cast<uint4*>(blk + sw128(r, j0)) = lo4;
           *reinterpret_cast<uint4*>(blk + sw128(r, j0 + 1)) = hi4;
         } else {
-          *reinterpret_cast<uint4*>(KV + 3 * kTcRegion + sw128(r, it - 12)) =
+          *reinterpret_cast<uint4*>(KV + 3 * kRegion + sw128(r, it - 12)) =
               ok ? *reinterpret_cast<const uint4*>(src + 192 + (it - 12) * 16) : make_uint4(0u, 0u, 0u, 0u);
         }
       }
@@ -935,7 +945,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   }
   if (warp == 0) {                   // slot validity as bit masks for the softmax
 #pragma unroll
-    for (int q = 0; q < kTcN / 32; ++q) {
+    for (int q = 0; q < kN / 32; ++q) {
       const uint32_t m = __ballot_sync(0xffffffffu, valid[32 * q + lane] != 0);
       if (lane == 0) vbits[q] = m;
     }
@@ -945,7 +955,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   ATRACE_T(0, 2);
 
   // ---------------------------------------------------------------- S partial = q~[:, half] K[:, half]^T
-  const uint32_t idesc_s = instr_desc(128, kTcN, 1u);
+  const uint32_t idesc_s = instr_desc(128, kN, 1u);
   bool ok = true;
   if (tid == 0) {
     ok = mbar_wait(&bars[3], 0u);
@@ -954,7 +964,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         const uint64_t ad = desc_kmajor_sw128(smem_u32(Q + c * (128 * 128)));
-        const uint64_t bd = desc_kmajor_sw128(smem_u32(KV + c * kTcRegion));
+        const uint64_t bd = desc_kmajor_sw128(smem_u32(KV + c * kRegion));
 #pragma unroll
         for (int k = 0; k < 4; ++k) umma_f16(tmem, ad + 2u * k, bd + 2u * k, idesc_s, (c | k) ? 1u : 0u);
       }
@@ -975,16 +985,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   const int h = (warp & 3) * 32 + lane;
   const int hs = warp >= 4 ? 0 : 1;                       // slot half of this warp
   const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-  float s[64];
-  tmem_ld_32x32b_x32(lane_addr + 64 * hs, s);
-  tmem_ld_32x32b_x32(lane_addr + 64 * hs + 32, s + 32);
+  float s[kHalf];
+#pragma unroll
+  for (int c = 0; c < kHalf; c += 32) tmem_ld_32x32b_x32(lane_addr + kHalf * hs + c, s + c);
   tmem_wait_ld();
   cluster.sync();
   ATRACE_T(0, 4);
   {
-    uint4* peer = reinterpret_cast<uint4*>(cluster.map_shared_rank(Q, dh ^ 1)) + (size_t)hs * 8 * kH128 + h;
+    uint4* peer = reinterpret_cast<uint4*>(cluster.map_shared_rank(Q, dh ^ 1)) + (size_t)hs * (kHalf / 8) * kH128 + h;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < kHalf / 8; ++j) {
       const float* v = s + 8 * j;
       peer[(size_t)j * kH128] = make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]),
                                            pack_f16x2(v[6], v[7]));
@@ -993,9 +1003,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   cluster.sync();
   ATRACE_T(0, 8);
   {
-    const uint4* mine = reinterpret_cast<const uint4*>(Q) + (size_t)hs * 8 * kH128 + h;
+    const uint4* mine = reinterpret_cast<const uint4*>(Q) + (size_t)hs * (kHalf / 8) * kH128 + h;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < kHalf / 8; ++j) {
       const uint4 v = mine[(size_t)j * kH128];
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -1012,8 +1022,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   {
     float mm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const uint32_t bits = vbits[2 * hs + q];
+    for (int q = 0; q < kHalf / 32; ++q) {
+      const uint32_t bits = vbits[(kHalf / 32) * hs + q];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const float z = ((bits >> j) & 1u) ? s[32 * q + j] * cl2 : -INFINITY;
@@ -1029,8 +1039,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   {
     float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const uint32_t cbits = vbits[2 * hs + q];
+    for (int q = 0; q < kHalf / 32; ++q) {
+      const uint32_t cbits = vbits[(kHalf / 32) * hs + q];
       uint32_t w[16];
 #pragma unroll
       for (int j = 0; j < 32; j += 2) {
@@ -1040,8 +1050,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
         w[j >> 1] = pack_bf16x2(p0, p1);
         ls[(j >> 1) & 3] += bf16_bits_to_f(w[j >> 1] & 0xFFFFu) + bf16_bits_to_f(w[j >> 1] >> 16);
       }
-      uint8_t* blk = X + hs * (128 * 128);
-      const int j0 = 4 * q;
+      const int s0p = kHalf * hs + 32 * q;           // first slot of these 32
+      uint8_t* blk = X + (s0p >> 6) * kTcQBlock;
+      const int j0 = (s0p & 63) >> 3;
 #pragma unroll
       for (int u = 0; u < 4; ++u)
         *reinterpret_cast<uint4*>(blk + sw128(h, j0 + u)) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
@@ -1061,9 +1072,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
     tc_fence_after();
     const uint32_t idesc_o = instr_desc(128, kTcHalf, 1u) | (1u << 16);   // B (the rows) MN-major
 #pragma unroll 1
-    for (int kk = 0; kk < kTcN / 16; ++kk) {
+    for (int kk = 0; kk < kN / 16; ++kk) {
       const uint64_t ad = desc_kmajor_sw128(smem_u32(X + (kk >> 2) * (128 * 128))) + 2u * (kk & 3);
-      const uint64_t bd = desc_mnmajor_sw128(smem_u32(KV + kk * 16 * 128), kTcRegion, 1024u);
+      const uint64_t bd = desc_mnmajor_sw128(smem_u32(KV + kk * 16 * 128), kRegion, 1024u);
       umma_f16(tmem + 256u, ad, bd, idesc_o, kk > 0 ? 1u : 0u);
     }
     umma_commit(&bars[2]);
@@ -1258,8 +1269,8 @@ cudaError_t launch_mma(const AttendArgs& a, cudaStream_t s) {
 
 int attend_path(const LayerArgs& L, bool dense) {
   // 128 heads of 512 dims take the tcgen05 kernel, dense and top-k alike (a top-k list of about
-  // 1,150 slots is 9 cluster pairs, measured faster than the mma.sync kernel over every SM);
-  // other head counts take the mma.sync kernel
+  // 1,150 slots is 18 cluster pairs of 64 slots, measured faster than the mma.sync kernel over
+  // every SM and than 9 pairs of 128); other head counts take the mma.sync kernel
   (void)dense;
   if (L.H == kH128 && L.D == kD && L.d_rope == 64 &&
       (L.kv_fmt == CSA_FMT_BF16 || L.kv_fmt == CSA_FMT_MIXED))
@@ -1277,7 +1288,8 @@ int attend_head_group(const LayerArgs& L) {
 
 int attend_num_splits(const LayerArgs& L, bool dense, int rows, int64_t slots, int num_sms) {
   if (attend_path(L, dense) == 2) {
-    const int64_t s = (slots + kTcN - 1) / kTcN;
+    const int n = dense ? kTcN : kTcNSparse;
+    const int64_t s = (slots + n - 1) / n;
     return (int)(s < 1 ? 1 : s);
   }
   const int HG = attend_head_group(L);
@@ -1329,21 +1341,28 @@ bool make_qt_map(CUtensorMap* m, const void* qt, int rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int FMT>
-cudaError_t launch_tc(const AttendArgs& a, cudaStream_t s) {
+template <int FMT, int kN>
+cudaError_t launch_tc_n(const AttendArgs& a, cudaStream_t s) {
+  constexpr size_t smem = tc_smem_bytes(kN);
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kTcSmem);
+    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<FMT, kN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   CUtensorMap qmap;
   if (!make_qt_map(&qmap, a.qt, a.rows)) return cudaErrorInvalidValue;
-  cudaError_t e = launch_kernel(attend_tc_kernel<FMT>, dim3((unsigned)(2 * a.splits), 1, (unsigned)a.rows),
-                                dim3(kTcThreads), kTcSmem, s, 2, qmap, a);
+  cudaError_t e = launch_kernel(attend_tc_kernel<FMT, kN>, dim3((unsigned)(2 * a.splits), 1, (unsigned)a.rows),
+                                dim3(kTcThreads), smem, s, 2, qmap, a);
   if (e != cudaSuccess || a.splits == 1) return e;
   return launch_kernel(attend_tc_combine_kernel, dim3(kD / 4, a.rows), dim3(4 * kH128), 0, s, 0, a);
+}
+
+// dense slot lists take 128-slot splits; top-k lists 64-slot splits (as attend_num_splits counts them)
+template <int FMT>
+cudaError_t launch_tc(const AttendArgs& a, cudaStream_t s) {
+  return a.topk ? launch_tc_n<FMT, kTcNSparse>(a, s) : launch_tc_n<FMT, kTcN>(a, s);
 }
 
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
