@@ -16,6 +16,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -50,54 +51,63 @@ __device__ __forceinline__ void rope4(float v[4], int c0, const LayerArgs& L, do
 
 constexpr int kRowBatch = 8;   // rows whose loads are issued together per thread
 
-// Sum / max of one value per CTA over the CTA's cluster, through distributed shared memory.
-// `slot` is a shared-memory float used by this reduction only; every thread gets the result.
-__device__ __forceinline__ float cluster_reduce(float v, float* slot, float* bcast, bool is_max) {
-  cg::cluster_group cl = cg::this_cluster();
-  if (threadIdx.x == 0) *slot = v;
-  cl.sync();
-  if (threadIdx.x < 32) {
-    float r = is_max ? -INFINITY : 0.f;
-    if ((unsigned)threadIdx.x < cl.num_blocks()) r = *cl.map_shared_rank(slot, threadIdx.x);
-    r = is_max ? warp_max(r) : warp_sum(r);
-    if (threadIdx.x == 0) *bcast = r;
-  }
-  __syncthreads();
-  return *bcast;
+// Cluster-wide reductions by mail: each CTA sends its partial to every CTA of the cluster (itself
+// included) with st.async into that CTA's mailbox, the bytes counted on the receiver's mbarrier, and
+// every CTA reduces the CL partials it received.  No cluster barrier per reduction: a barrier's
+// release would first wait for this CTA's outstanding global stores (the window and raw rows).
+// Mailbox k serves one reduction per launch: 0 the window row's FP8 amax, 1 the entry's RMSNorm
+// sum and FP8 amax.
+constexpr int kMailMaxCl = 16;
+struct ClusterMail {
+  uint64_t bar[2];
+  float2 box[2][kMailMaxCl];   // box[k][sender rank]
+};
+
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
+// Threads 0..CL-1 each send v to one CTA of the cluster.
+__device__ __forceinline__ void mail_send(ClusterMail* m, int k, int q, int CL, float2 v) {
+  if ((int)threadIdx.x >= CL) return;
+  const uint32_t to = threadIdx.x;
+  uint32_t rd, rb;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rd) : "r"(sm100::smem_u32(&m->box[k][q])), "r"(to));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rb) : "r"(sm100::smem_u32(&m->bar[k])), "r"(to));
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];"
+               ::"r"(rd), "f"(v.x), "f"(v.y), "r"(rb)
+               : "memory");
 }
 
-// Cluster-wide (sum of s, max of m) over one pair per thread, in one pass: a block reduction of
-// both, one cluster barrier, then every CTA reads the CTAs' pairs through distributed shared
-// memory.  scratch: 64 floats; slot2 / bcast2: 2 floats each.  Every thread gets the result.
-__device__ __forceinline__ float2 cluster_reduce_sum_max(float s, float m, float* scratch, float* slot2,
-                                                         float* bcast2) {
-  cg::cluster_group cl = cg::this_cluster();
+// Waits (bounded) for the CL partials of mailbox k; every thread gets (sum of .x, max of .y).
+__device__ __forceinline__ float2 mail_reduce(ClusterMail* m, int k, int CL) {
+  sm100::mbar_wait(&m->bar[k], 0u);
+  float x = 0.f, y = -INFINITY;
+  for (int p = 0; p < CL; ++p) {
+    const float2 v = m->box[k][p];
+    x += v.x;
+    y = fmaxf(y, v.y);
+  }
+  return make_float2(x, y);
+}
+
+// Block sum of s and block max of m, in thread 0 (scratch: 64 floats).
+__device__ __forceinline__ float2 block_sum_max(float s, float m, float* scratch) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
   s = warp_sum(s);
   m = warp_max(m);
   __syncthreads();
   if (lane == 0) { scratch[wid] = s; scratch[32 + wid] = m; }
   __syncthreads();
+  float x = 0.f, y = -INFINITY;
   if (threadIdx.x < 32) {
-    float x = lane < nw ? scratch[lane] : 0.f, y = lane < nw ? scratch[32 + lane] : -INFINITY;
+    x = lane < nw ? scratch[lane] : 0.f;
+    y = lane < nw ? scratch[32 + lane] : -INFINITY;
     x = warp_sum(x);
     y = warp_max(y);
-    if (lane == 0) { slot2[0] = x; slot2[1] = y; }
   }
-  cl.sync();
-  if (threadIdx.x < 32) {
-    float x = 0.f, y = -INFINITY;
-    if ((unsigned)lane < cl.num_blocks()) {
-      const float* r = cl.map_shared_rank(slot2, lane);
-      x = r[0];
-      y = r[1];
-    }
-    x = warp_sum(x);
-    y = warp_max(y);
-    if (lane == 0) { bcast2[0] = x; bcast2[1] = y; }
-  }
-  __syncthreads();
-  return make_float2(bcast2[0], bcast2[1]);
+  return make_float2(x, y);
 }
 
 // Stores this CTA's channels of one row in the cache format.  `am` is the cluster-wide max |x|
@@ -142,7 +152,7 @@ __device__ __forceinline__ float local_amax(const float v[4], int c0, int dn, bo
 // the cluster.  With CL = 1 (chunked prefill) the cluster reductions are plain block reductions.
 __global__ void __launch_bounds__(256) append_compress_kernel(const __grid_constant__ AppendCompressArgs a, int CL) {
   __shared__ float scratch[64];
-  __shared__ float red[4], bcast, bcast2[2];
+  __shared__ ClusterMail mail;
   extern __shared__ float part[];                  // [RG][3][DC]
   cg::cluster_group cluster = cg::this_cluster();
   const LayerArgs& L = a.L;
@@ -157,6 +167,17 @@ __global__ void __launch_bounds__(256) append_compress_kernel(const __grid_const
   const bool lead = rg == 0;
   const int dn = L.D - L.d_rope;
   CTRACE(0);
+  // mailboxes: each expects CL partials of 8 bytes; the cluster barrier's first phase (arrived now,
+  // awaited before the first send) makes every CTA's initialisation visible to its peers
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&mail.bar[0], 1);
+    sm100::mbar_init(&mail.bar[1], 1);
+    sm100::mbar_arrive_expect_tx(&mail.bar[0], 8u * (uint32_t)CL);
+    sm100::mbar_arrive_expect_tx(&mail.bar[1], 8u * (uint32_t)CL);
+    sm100::fence_barrier_init();
+  }
+  cluster_arrive_relaxed();
+  bool mail_open = false, done_mail = false;       // uniform over the cluster
   const int64_t t = a.q_pos[(int64_t)b * a.Tq + j];
   const int64_t r = t - L.pos0;
   const bool valid = r >= 0;                       // uniform over the cluster
@@ -187,7 +208,13 @@ __global__ void __launch_bounds__(256) append_compress_kernel(const __grid_const
     float w[4] = {x[0], x[1], x[2], x[3]};
     rope4(w, c0, L, (double)t);
     float am = 0.f;
-    if (L.kv_fmt == CSA_FMT_MIXED) am = cluster_reduce(block_max(local_amax(w, c0, dn, lead), scratch), &red[0], &bcast, true);
+    if (L.kv_fmt == CSA_FMT_MIXED) {
+      const float bm = block_max(local_amax(w, c0, dn, lead), scratch);
+      if (!mail_open) { cluster_wait(); mail_open = true; }
+      mail_send(&mail, 0, q, CL, make_float2(0.f, bm));
+      am = mail_reduce(&mail, 0, CL).y;
+      if (!compress) { cluster_arrive_relaxed(); done_mail = true; }   // this CTA's mail is all in
+    }
     uint8_t* dst = C.window + ((size_t)b * C.window_cap + (size_t)(r % C.window_cap)) * L.row_bytes;
     pack_slice(dst, L, c0, w, lead, am, q == 0);
   }
@@ -387,7 +414,12 @@ __global__ void __launch_bounds__(256) append_compress_kernel(const __grid_const
       if (c0 < dn)
         eg = fmaxf(fmaxf(fabsf(e[0] * gk.x), fabsf(e[1] * gk.y)), fmaxf(fabsf(e[2] * gk.z), fabsf(e[3] * gk.w)));
     }
-    const float2 red2 = cluster_reduce_sum_max(ss, eg, scratch, &red[1], bcast2);
+    const float2 bl = block_sum_max(ss, eg, scratch);
+    if (!mail_open) { cluster_wait(); mail_open = true; }
+    mail_send(&mail, 1, q, CL, bl);
+    const float2 red2 = mail_reduce(&mail, 1, CL);
+    cluster_arrive_relaxed();                      // this CTA's mail is all in
+    done_mail = true;
     const float rs = 1.0f / sqrtf(red2.x / (float)L.D + L.eps);
     e[0] *= rs * gk.x; e[1] *= rs * gk.y; e[2] *= rs * gk.z; e[3] *= rs * gk.w;
     CTRACE(6);
@@ -400,8 +432,10 @@ __global__ void __launch_bounds__(256) append_compress_kernel(const __grid_const
     CTRACE(8);
     CTRACE_C(15);
   }
-  // no CTA may leave while a peer can still read its shared memory
-  cluster.sync();
+  // second phase of the cluster barrier: no CTA leaves before every CTA has received its mail
+  if (!mail_open) cluster_wait();
+  if (!done_mail) cluster_arrive_relaxed();
+  cluster_wait();
 }
 
 }  // namespace
