@@ -734,8 +734,11 @@ __host__ __device__ constexpr int tc_x_bytes(int n) {
   const int raw = n * kTcHalfRow, p = (n / 64) * kTcQBlock;
   return ((raw > p ? raw : p) + 1023) / 1024 * 1024;
 }
+// the peer's fp16 partial scores: [slot half][N / 16 groups of 8][128 heads] x 16 bytes
+__host__ __device__ constexpr int tc_xr_bytes(int n) { return n * 256; }
 constexpr size_t tc_smem_bytes(int n) {
-  return 1024 + 4 * (size_t)n * 128 + 4 * (size_t)kTcQBlock + tc_x_bytes(n) + 64 + n * 8 + 4 * 128 * 4 + n * 8;
+  return 1024 + 4 * (size_t)n * 128 + 4 * (size_t)kTcQBlock + tc_x_bytes(n) + tc_xr_bytes(n) + 64 + n * 8 +
+         4 * 128 * 4 + n * 8;
 }
 static_assert(tc_x_bytes(kTcN) == kTcN * kTcHalfRow, "X at 128 slots: the raw half rows");
 static_assert(tc_smem_bytes(kTcN) <= 227 * 1024, "tcgen05 attention shared memory");
@@ -820,7 +823,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   uint8_t* KV = sm;                                        // [4 blocks][128 slots][128 B] bf16: this CTA's dims
   uint8_t* Q = KV + 4 * kRegion;                           // q~ half [4][128][128 B], then the peer's S partial
   uint8_t* X = Q + 4 * kTcQBlock;                          // raw half rows, then P [N / 64][128][128 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(X + kX);    // S, (unused), O, q~
+  uint8_t* XR = X + kX;                                    // the peer's partial scores (received)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(XR + tc_xr_bytes(kN));   // S, received scores, O, q~
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
   uint32_t* vbits = tmem_slot + 1;                         // [4] slot validity bitmasks
   int* valid = reinterpret_cast<int*>(tmem_slot + 8);      // [kN]
@@ -836,6 +840,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   ATRACE_T(0, 0);
   if (tid == 0) {
     for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+    mbar_arrive_expect_tx(&bars[1], (uint32_t)tc_xr_bytes(kN));   // the peer's scores, counted in bytes
     fence_barrier_init();
     // q~ dims [256 dh, 256 dh + 256) with the tensor memory accelerator: four 64-dim boxes of 128
     // heads, 128-byte swizzled (the K-major operand layout); in flight while the rows come in
@@ -843,6 +848,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) tma_load_2d(Q + c * (128 * 128), &qmap, &bars[3], dh * kTcHalf + c * 64, row * kH128);
   }
+  // first phase of the pair's cluster barrier: arrived now (each CTA's receive barrier is set up),
+  // awaited just before the scores are sent
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   const int64_t t = a.q_pos[row];
   const SlotInfo si = slot_info(a, t);
   const int64_t s0 = (int64_t)sp * kN;
@@ -976,11 +984,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   ATRACE_T(0, 3);
 
   // ---------------------------------------------------------------- S = the two partials (cluster pair)
-  // Warps w and w+4 read the same TMEM lanes (heads 32(w%4)..); warps 4..7 take slots 0..63,
-  // warps 0..3 slots 64..127.  Each thread sends its 64 partial scores, rounded to fp16, to the
-  // thread with the same (head, slot half) in the peer CTA, into the peer's q~ region (free once
-  // the peer's MMAs have read it: the first cluster barrier), as [slot half][8 groups of 8][head]
-  // 16-byte pieces.  The fp16 rounding (2^-11 relative) is finer than P's own bf16 rounding.
+  // Warps w and w+4 read the same TMEM lanes (heads 32(w%4)..); warps 4..7 take the first half of
+  // the slots, warps 0..3 the second.  Each thread sends its partial scores, rounded to fp16, to the
+  // thread with the same (head, slot half) in the peer CTA: st.async into the peer's receive buffer
+  // as [slot half][groups of 8][head] 16-byte pieces, the bytes counted on the peer's receive
+  // barrier (no cluster barrier per exchange).  The fp16 rounding (2^-11 relative) is finer than P's
+  // own bf16 rounding.
   const float cl2 = L.scale * kLog2e;
   const int h = (warp & 3) * 32 + lane;
   const int hs = warp >= 4 ? 0 : 1;                       // slot half of this warp
@@ -989,21 +998,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
 #pragma unroll
   for (int c = 0; c < kHalf; c += 32) tmem_ld_32x32b_x32(lane_addr + kHalf * hs + c, s + c);
   tmem_wait_ld();
-  cluster.sync();
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   ATRACE_T(0, 4);
   {
-    uint4* peer = reinterpret_cast<uint4*>(cluster.map_shared_rank(Q, dh ^ 1)) + (size_t)hs * (kHalf / 8) * kH128 + h;
+    uint32_t rd, rb;
+    const uint32_t ld = smem_u32(XR) + (uint32_t)(((size_t)hs * (kHalf / 8) * kH128 + h) * 16);
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rd) : "r"(ld), "r"(dh ^ 1));
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rb) : "r"(smem_u32(&bars[1])), "r"(dh ^ 1));
 #pragma unroll
     for (int j = 0; j < kHalf / 8; ++j) {
       const float* v = s + 8 * j;
-      peer[(size_t)j * kH128] = make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]),
-                                           pack_f16x2(v[6], v[7]));
+      asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+                   ::"r"(rd + (uint32_t)(j * kH128 * 16)), "r"(pack_f16x2(v[0], v[1])), "r"(pack_f16x2(v[2], v[3])),
+                     "r"(pack_f16x2(v[4], v[5])), "r"(pack_f16x2(v[6], v[7])), "r"(rb)
+                   : "memory");
     }
   }
-  cluster.sync();
+  if (!mbar_wait(&bars[1], 0u)) ok = false;
+  // second phase: this CTA has all of its peer's scores (awaited before the CTA leaves, so neither
+  // CTA of the pair exits while the other still sends to it)
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   ATRACE_T(0, 8);
   {
-    const uint4* mine = reinterpret_cast<const uint4*>(Q) + (size_t)hs * (kHalf / 8) * kH128 + h;
+    const uint4* mine = reinterpret_cast<const uint4*>(XR) + (size_t)hs * (kHalf / 8) * kH128 + h;
 #pragma unroll
     for (int j = 0; j < kHalf / 8; ++j) {
       const uint4 v = mine[(size_t)j * kH128];
@@ -1145,6 +1162,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 }
 
 // Merge of the tcgen05 kernel's splits for 4 output dims of one query and all 128 heads: four
