@@ -21,7 +21,8 @@
  *       shared-KV multi-query layout, BF16 rotary dims + FP8 remainder).
  *   HCA ("heavily compressed attention"): the same path with m'=128, no
  *   overlap, no indexer and dense attention over every visible entry.
- *     - same page, same section ("m' = 128 ... dense over what remains").
+ *     - same page, same section (m' = 128, and attention dense over all the
+ *       remaining entries).
  *
  * The pages give no formula for the indexer or the gate and no storage
  * layout; the definitions this library implements are stated at each call.
@@ -193,9 +194,9 @@ CSA_API uint64_t csa_launch_count(void);
  * buffer), and each token's window row RoPE_t(x) -- rotated at its own
  * position, not normalised -- is stored at window slot r mod window_cap.
  *   x_new, g_new: [B][Tq][D] act_format, or both NULL.
- * The sliding window is the pages' "small sliding-window branch of
- * uncompressed recent tokens" ("DeepSeek-V4 Explained: ...", "The attention
- * stack, and why it is two mechanisms"). */
+ * The sliding window is the pages' short branch over the most recent tokens,
+ * kept uncompressed ("DeepSeek-V4 Explained: ...", "The attention stack, and
+ * why it is two mechanisms"). */
 CSA_API csa_status_t csa_append(const csa_layer_t* L, const csa_cache_t* cache,
                         const void* x_new, const void* g_new,
                         const int64_t* q_pos, int32_t Tq, void* stream);
@@ -205,11 +206,11 @@ CSA_API csa_status_t csa_append(const csa_layer_t* L, const csa_cache_t* cache,
  * gamma_kv) with e_c = sum_r softmax_r(gate[r][c] + pos_bias[r - (i-ov)m][c])
  * * raw[r][c] over raw rows r in [(i-ov)m, (i+1)m) clipped at 0, written to
  * entries[b][i] in kv_format.  The raw buffer must hold those rows.
- * Pages: "compresses the key-value cache of every group of m consecutive
- * tokens into one entry using learned compression weights and positional
- * biases" ("DeepSeek-V4 Explained: ..."); "each compressed entry draws from
- * 2m source entries while the sequence still shrinks by m" ("DeepSeek-V4:
- * Making a Million Tokens Affordable", "Two ways to shrink attention"). */
+ * Pages: each group of m consecutive tokens becomes one entry, pooled with
+ * learned weights and per-slot position biases ("DeepSeek-V4 Explained: ...");
+ * an entry reads 2m source rows, yet the sequence still shrinks m-fold
+ * ("DeepSeek-V4: Making a Million Tokens Affordable", "Two ways to shrink
+ * attention"). */
 CSA_API csa_status_t csa_compress(const csa_layer_t* L, const csa_cache_t* cache,
                           const csa_params_t* P, const int64_t* q_pos, int32_t Tq,
                           void* stream);
@@ -226,9 +227,9 @@ CSA_API csa_status_t csa_compress(const csa_layer_t* L, const csa_cache_t* cache
  *                query's visible count are excluded)
  *   topk_idx:    [B][Tq][top_k] int32 (output)
  *   scores:      [B][Tq][n_max] float32 (output, optional: NULL keeps them in the workspace)
- * Pages: "a Lightning Indexer scores them in a low-rank way and each query
- * attends only to the top-k compressed entries" ("DeepSeek-V4 Explained");
- * "a few small heads run in FP8" ("DeepSeek-V4, explained.", step 3). */
+ * Pages: a cheap low-rank indexer scores the compressed entries and each query
+ * attends only to its k best ("DeepSeek-V4 Explained"); the indexer uses a
+ * few small FP8 heads ("DeepSeek-V4, explained.", step 3). */
 CSA_API csa_status_t csa_index_topk(const csa_layer_t* L, const csa_cache_t* cache,
                             const void* idx_q, const float* idx_q_scale, const float* head_w,
                             const int64_t* q_pos, int32_t Tq, int64_t n_max,
@@ -241,9 +242,9 @@ CSA_API csa_status_t csa_index_topk(const csa_layer_t* L, const csa_cache_t* cac
  *   [max(0, r_t - w + 1), r_t];  l_j = <q~_h, k_j> * softmax_scale;
  *   o_h = sum_j e^{l_j} k_j / (e^{sink_h} + sum_j e^{l_j});  out = RoPE_{-t}(o_h).
  *   q:   [B][Tq][H][D] act_format;  out: [B][Tq][H][D] act_format.
- * Pages: "a compressed entry serves as both key and value ... RoPE at
- * position -i is applied back to the attention output"; "learnable attention
- * sinks" ("DeepSeek-V4: Making a Million Tokens Affordable"). */
+ * Pages: an entry is both key and value, the output is rotated back by the
+ * query's position, and each head has a learned sink ("DeepSeek-V4: Making a
+ * Million Tokens Affordable"). */
 CSA_API csa_status_t csa_sparse_attend(const csa_layer_t* L, const csa_cache_t* cache,
                                const csa_params_t* P, const void* q, const int64_t* q_pos,
                                int32_t Tq, const int32_t* topk_idx, void* out,
@@ -252,8 +253,8 @@ CSA_API csa_status_t csa_sparse_attend(const csa_layer_t* L, const csa_cache_t* 
 /* Dense attention over every visible entry i < n_visible(t) (HCA) plus the
  * window rows, otherwise as csa_sparse_attend.  n_max bounds the visible
  * entries (<= entry_cap).
- * Pages: "keep attention fully dense over what remains. No indexer, no
- * top-k" ("DeepSeek-V4: Making a Million Tokens Affordable"). */
+ * Pages: after the heavy compression, attention stays dense, without an
+ * indexer or a top-k ("DeepSeek-V4: Making a Million Tokens Affordable"). */
 CSA_API csa_status_t hca_attend(const csa_layer_t* L, const csa_cache_t* cache,
                         const csa_params_t* P, const void* q, const int64_t* q_pos,
                         int32_t Tq, int64_t n_max, void* out,

@@ -1,14 +1,14 @@
 // Shared-KV multi-query attention over gathered KV rows with a sink logit.
 //
-// "a compressed entry serves as both key and value ... RoPE at position -i is
-// applied back to the attention output so the result carries relative
-// positions ... learnable attention sinks let a head route its attention
-// mass to nothing at all" and "queries and compressed entries get an extra
-// RMSNorm" -- "DeepSeek-V4: Making a Million Tokens Affordable", section
-// "Two ways to shrink attention, interleaved".  "Fetching whole contiguous
-// blocks, shared by the heads that share keys" -- "DeepSeek-V4, explained.",
-// step 8: every gathered row is loaded once per CTA and used by all of the
-// CTA's heads.
+// What it computes ("DeepSeek-V4: Making a Million Tokens Affordable", section "Two ways to
+// shrink attention, interleaved"):
+// - each compressed entry is both the key and the value;
+// - queries and entries are RMS-normalised;
+// - the output is rotated back by the query's position (RoPE at -t), so it depends only on relative
+//   positions;
+// - a learned per-head sink logit lets a head put part of its attention weight on nothing.
+// Step 8 of "DeepSeek-V4, explained." has heads that share keys read the same contiguous rows: here
+// every gathered row is loaded once per CTA and serves all of the CTA's heads.
 //
 // Key slots of a query at raw row r_t: [0, n_sel) are compressed entries
 // (the top-k list for CSA, -1 skipped; every visible entry for HCA), then

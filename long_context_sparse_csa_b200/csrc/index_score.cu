@@ -1,11 +1,10 @@
 // Lightning-indexer scores:  s_i = sum_h w_h * ReLU(sigma_q,h * sigma_k,i * <q_h, k_i>).
 //
-// The pages give the indexer only in words: "a Lightning Indexer scores them
-// in a low-rank way" ("DeepSeek-V4 Explained: ...", section "The attention
-// stack, and why it is two mechanisms") and "a separate lightning indexer, a
-// few small heads run in FP8, scores individual past tokens" ("DeepSeek-V4,
-// explained.", step 3 of "For one query ... works like this").  This file
-// holds the multi-head ReLU-weighted dot product the operator defines.
+// The pages describe the indexer only in words. "DeepSeek-V4 Explained: ...", section "The
+// attention stack, and why it is two mechanisms", calls it a cheap low-rank scorer of the
+// compressed entries. Step 3 of the per-query list in "DeepSeek-V4, explained." gives it a few small
+// FP8 heads that score each past entry. This file holds the multi-head ReLU-weighted dot product the
+// operator defines from that.
 //
 // Tensor-core path (FP8 e4m3 keys, d_I = 128): the score tile of 128 entries
 // x (QN queries * H_I heads) is one tcgen05 kind::f8f6f4 MMA chain (M = 128

@@ -1,9 +1,8 @@
 // Top-k selection of indexer scores: the k largest scores among a query's
 // visible entries, ties to the smaller entry index, emitted in ascending
-// entry order and padded with -1.  "Keep the k highest-scoring blocks"
-// ("DeepSeek-V4, explained.", step 4); "a top-k selector keeps only the best
-// ones for core attention" ("DeepSeek-V4: Making a Million Tokens
-// Affordable", section "Two ways to shrink attention, interleaved").
+// entry order and padded with -1. Only the k best-scoring entries go on to the core attention
+// (step 4 of "DeepSeek-V4, explained."; "DeepSeek-V4: Making a Million Tokens Affordable", section
+// "Two ways to shrink attention, interleaved").
 //
 // One 1024-thread CTA per query row runs a radix select on the
 // order-preserving 32-bit image of the scores (11 + 11 + 10 bits, shared-

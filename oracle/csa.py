@@ -7,11 +7,11 @@ heads sharing one KV head of dimension D, rotary on the last d_r = 64 dims.
 Readings taken where the pages are silent (each repeated at its function):
 
 R1  Overlap is look-back: entry i pools raw rows [(i-ov)m, (i+1)m), clipped at
-    row 0 ("each compressed entry draws from 2m source entries while the
-    sequence still shrinks by m" -- "DeepSeek-V4: Making a Million Tokens
-    Affordable", "Two ways to shrink attention, interleaved").  HCA uses ov=0.
-R2  "learned per-token compression weights and positional biases" (same
-    section) = one gate logit per raw row and channel plus one bias per window
+    row 0.  The pages have each entry read 2m source rows while the sequence
+    still shrinks m-fold ("DeepSeek-V4: Making a Million Tokens Affordable",
+    "Two ways to shrink attention, interleaved").  HCA uses ov=0.
+R2  The learned per-token compression weights and positional biases of the same
+    section = one gate logit per raw row and channel plus one bias per window
     slot and channel, normalised by a softmax over the window's rows, per
     channel.
 R3  Entry i is rotated at position pos0 + i*m and is visible to a query at
@@ -20,8 +20,8 @@ R4  Window rows are the most recent w raw rows including the current one,
     rotated at their own positions, not normalised; entries and window rows
     are separate key sets and nothing is de-duplicated.
 R5  Index score s_i = sum_h w_h * ReLU(sigma_q,h * sigma_k,i * <q_h, k_i>)
-    over H_I indexer heads (the pages give no formula: "the page does not give
-    V4's exact scorer" -- "DeepSeek-V4, explained.", glossary).
+    over H_I indexer heads.  The pages give no formula; the glossary of
+    "DeepSeek-V4, explained." says outright that V4's exact scorer is not given.
 R6  Top-k: the k largest scores, ties to the smaller entry index; returned in
     ascending entry order; fewer than k visible entries -> all of them, then -1.
 R7  Logits l_j = <q~, k~_j> / sqrt(D); sink: p_j = e^{l_j} / (e^{s_h} + sum e^{l}).
@@ -40,8 +40,8 @@ from . import formats as F
 def rope_cos_sin(pos, d_rope: int, base: float):
     """cos, sin of pos * theta_u for u < d_rope/2 (R8), float64 [..., d_rope/2].
 
-    "RoPE is applied to only the last 64 dimensions" -- "DeepSeek-V4: Making a
-    Million Tokens Affordable", "Two ways to shrink attention, interleaved".
+    Only the last 64 dimensions are rotated ("DeepSeek-V4: Making a Million Tokens
+    Affordable", "Two ways to shrink attention, interleaved").
     """
     pos = np.asarray(pos, dtype=np.float64)
     u = np.arange(d_rope // 2, dtype=np.float64)
@@ -65,9 +65,9 @@ def rope(x, pos, d_rope: int, base: float):
 def rms_norm(x, gamma, eps: float):
     """x / sqrt(mean(x^2) + eps) * gamma (R9).
 
-    "queries and compressed entries get an extra RMSNorm before core attention"
-    -- "DeepSeek-V4: Making a Million Tokens Affordable", "Two ways to shrink
-    attention, interleaved".
+    Queries and compressed entries are RMS-normalised before the core attention
+    ("DeepSeek-V4: Making a Million Tokens Affordable", "Two ways to shrink
+    attention, interleaved").
     """
     x = np.asarray(x, dtype=np.float64)
     r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
@@ -87,9 +87,9 @@ def pool_entry(raw_rows, gate_rows, bias, slots):
     """Per-channel softmax-weighted sum of one entry's source rows (R2).
 
     raw_rows, gate_rows: [r, D]; bias: [(1+ov)m, D]; slots: window slot of each row.
-    "compresses the key-value cache of every group of m consecutive tokens into
-    one entry using learned compression weights and positional biases" --
-    "DeepSeek-V4 Explained: ...", "The attention stack, and why it is two mechanisms".
+    Each group of m consecutive tokens is pooled into one entry with learned
+    weights and position biases ("DeepSeek-V4 Explained: ...", "The attention
+    stack, and why it is two mechanisms").
     """
     z = np.asarray(gate_rows, np.float64) + np.asarray(bias, np.float64)[slots]
     z = z - z.max(axis=0, keepdims=True)
@@ -134,9 +134,9 @@ def index_scores(iq, iq_scale, head_w, ik, ik_scale):
     """s_i = sum_h w_h * ReLU(sigma_q,h * sigma_k,i * <q_h, k_i>) (R5).
 
     iq [H_I, d_I], iq_scale [H_I], head_w [H_I], ik [N, d_I], ik_scale [N].
-    "a Lightning Indexer scores them in a low-rank way" -- "DeepSeek-V4
-    Explained: ..."; "a separate lightning indexer, a few small heads run in
-    FP8, scores individual past tokens" -- "DeepSeek-V4, explained.", step 3.
+    The indexer is a cheap low-rank scorer ("DeepSeek-V4 Explained: ...") made of
+    a few small FP8 heads that score each past entry ("DeepSeek-V4, explained.",
+    step 3).
     """
     dots = np.asarray(ik, np.float64) @ np.asarray(iq, np.float64).T          # [N, H_I]
     z = dots * np.asarray(ik_scale, np.float64)[:, None] * np.asarray(iq_scale, np.float64)[None, :]
@@ -146,9 +146,8 @@ def index_scores(iq, iq_scale, head_w, ik, ik_scale):
 def top_k(scores, k: int):
     """Indices of the k largest scores, ties to the smaller index, ascending, -1 padded (R6).
 
-    "Keep the k highest-scoring blocks" -- "DeepSeek-V4, explained.", step 4;
-    "a top-k selector keeps only the best ones for core attention" --
-    "DeepSeek-V4: Making a Million Tokens Affordable".
+    Only the k best-scoring entries reach the core attention ("DeepSeek-V4,
+    explained.", step 4; "DeepSeek-V4: Making a Million Tokens Affordable").
     """
     s = np.asarray(scores, np.float64)
     order = sorted(range(len(s)), key=lambda i: (-s[i], i))   # stable, explicit tie rule
@@ -179,13 +178,12 @@ def attend(q, t, rows, sinks, gamma_q, d_rope, base, scale=None, eps=1e-6):
     """Shared-KV multi-query attention with sinks and inverse RoPE on the output.
 
     q [H, D] (raw), rows [R, D] (keys = values), sinks [H] -> o [H, D].
-    "a compressed entry serves as both key and value ... RoPE at position -i is
-    applied back to the attention output so the result carries relative
-    positions ... learnable attention sinks let a head route its attention
-    mass to nothing at all" -- "DeepSeek-V4: Making a Million Tokens
-    Affordable", "Two ways to shrink attention, interleaved"; "an
-    attention-sink term lets each head's scores sum to less than one" --
-    "DeepSeek-V4 Explained: ...".  Readings R7, R8, R9.
+    An entry is both key and value; the output is rotated back by the query's
+    position so only relative positions matter; a learned per-head sink can take
+    part of a head's attention weight ("DeepSeek-V4: Making a Million Tokens
+    Affordable", "Two ways to shrink attention, interleaved"), so the weights on
+    the keys can sum to less than one ("DeepSeek-V4 Explained: ...").  Readings
+    R7, R8, R9.
     """
     rows = np.asarray(rows, np.float64)
     D = rows.shape[-1]

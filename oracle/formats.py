@@ -1,11 +1,11 @@
 """Storage formats of the KV cache and the indexer, decoded and encoded exactly.
 
-"The KV entries themselves are stored with BF16 for the rotary dimensions and
-FP8 for the rest" -- "DeepSeek-V4 Explained: ...", section "The attention
-stack, and why it is two mechanisms"; the same split, "roughly halves" the
-cache, in "DeepSeek-V4: Making a Million Tokens Affordable", section "Two
-ways to shrink attention, interleaved".  The pages name the formats only; the
-codecs below are written from the formats' own definitions:
+The pages store an entry's rotary dimensions in BF16 and the rest in FP8
+("DeepSeek-V4 Explained: ...", section "The attention stack, and why it is two
+mechanisms"); "DeepSeek-V4: Making a Million Tokens Affordable", section "Two
+ways to shrink attention, interleaved", gives the same split as about halving
+the cache.  The pages name the formats only; the codecs below are written from
+the formats' own definitions:
 
 * FP8 e4m3 ("e4m3fn" of the OCP 8-bit floating-point spec): 1 sign bit,
   4 exponent bits with bias 7, 3 mantissa bits; exponent field 0 is
