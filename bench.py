@@ -541,6 +541,19 @@ def run_ours(args):
 
 # ----------------------------------------------------------------------------- chunked prefill (diagnostic mode)
 
+def prefill_work(layer, t, n_max, B=1):
+    """Work of one chunked-prefill call for queries at positions t (pos0 = 0): FP8 indexer FLOPs (every
+    visible entry of every query, all index heads), BF16 attention FLOPs (QK^T and PV over each
+    query's top-k entries and window rows, all heads) and the rows the attention gathers (bytes)."""
+    t = np.asarray(t, dtype=np.int64)
+    n_vis = np.minimum((t + 1) // layer.m, n_max).astype(np.float64)
+    idx_flops = 2.0 * layer.H_I * layer.d_I * float(n_vis.sum()) * B
+    rows = np.minimum(n_vis, layer.top_k) + np.minimum(t + 1, layer.window)
+    att_flops = 4.0 * layer.H * layer.D * float(rows.sum()) * B
+    row_bytes = layer.D * 2 if layer.kv_format == "bf16" else layer.D * 4
+    return idx_flops, att_flops, float(rows.sum()) * B * row_bytes
+
+
 def run_prefill(args):
     """Times csa_prefill on the 8,192-query chunk (one GPU): tokens/s, the launch list of one call
     (CUDA events before each launch), and the indexer's FP8 and the attention's BF16 TFLOP/s against
@@ -594,12 +607,7 @@ def run_prefill(args):
     evs[n].record()
     torch.cuda.synchronize()
     launches_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(n)]
-    # work of the chunk: every query's visible entries (indexer) and its top-k + window rows (attention)
-    t = pf["t"][0]
-    n_vis = np.minimum((t + 1) // layer.m, n_max).astype(np.float64)
-    idx_flops = 2.0 * layer.H_I * layer.d_I * float(n_vis.sum()) * wl.B
-    rows = np.minimum(n_vis, layer.top_k) + np.minimum(t + 1, layer.window)
-    att_flops = 4.0 * layer.H * layer.D * float(rows.sum()) * wl.B
+    idx_flops, att_flops, gather_bytes = prefill_work(layer, pf["t"][0], n_max, wl.B)
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             bf16_peak, note = float(json.load(f)["bf16_tflops"]), "of measured"
@@ -613,7 +621,8 @@ def run_prefill(args):
                        "kv_dim": layer.D, "kv_format": layer.kv_format, "top_k": layer.top_k,
                        "l2": "inputs larger than L2 (queries alone 512 MiB)"},
             "launch_ms": [round(x, 3) for x in launches_ms],
-            "work": {"indexer_fp8_tflop": idx_flops / 1e12, "attention_bf16_tflop": att_flops / 1e12},
+            "work": {"indexer_fp8_tflop": idx_flops / 1e12, "attention_bf16_tflop": att_flops / 1e12,
+                     "attention_gather_gb": gather_bytes / 1e9},
             "tensor": {"bf16_peak_tflops": bf16_peak, "fp8_peak_tflops": 2 * bf16_peak, "peak_source": note},
             "longest_launches": [{"launch": i, "ms": round(launches_ms[i], 3)} for i in longest[:3]],
             "clocks": clocks.summary(w0, w1)}

@@ -11,6 +11,7 @@ import socket
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 import torch.multiprocessing as mp
 
@@ -82,3 +83,20 @@ def test_reference_arm_nonzero_rank_exits_without_work():
                         "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_prefill_work_matches_the_workload_arithmetic():
+    # the 8,192-query chunk after 65,536 tokens: 142.6 M (query, entry) pairs for the indexer
+    # (1.168 TFLOP in FP8 at 32 heads x 128 dims), 1,152 rows per query for the attention
+    # (1.237 TFLOP in BF16 at 64 heads x 512 dims) and 9.66 GB of gathered bf16 rows
+    from csa_synth import get_workload
+    wl = get_workload("csa_prefill_8k")
+    layer = wl.layers[0]
+    prefix = wl.n - wl.Tq
+    t = prefix + np.arange(wl.Tq)
+    idx, att, gather = bench.prefill_work(layer, t, wl.n // layer.m, wl.B)
+    pairs = sum(min((int(x) + 1) // layer.m, wl.n // layer.m) for x in t)
+    assert abs(pairs - 142.6e6) < 0.05e6
+    assert abs(idx - 1.168e12) < 0.001e12
+    assert abs(att - 1.237e12) < 0.001e12
+    assert abs(gather - 9.66e9) < 0.01e9
