@@ -1166,12 +1166,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
 }
 
 // Merge of the tcgen05 kernel's splits for 4 output dims of one query and all 128 heads: four
-// groups of 128 threads (one per head) each take every 4th split and merge them online, 8 splits
+// groups of 128 threads (one per head) each take every 4th split and merge them online, 17 splits
 // per step with every load of the step in flight (one 8-byte load of a head's 4 dims and one of
 // its (m, l) per split, contiguous across a warp); the groups then merge through shared memory
 // with the sink.  Normalisation and inverse rotation as in the single-split epilogue.
 __global__ void __launch_bounds__(512) attend_tc_combine_kernel(const __grid_constant__ AttendArgs a) {
-  constexpr int kU = 8;
+  constexpr int kU = 17;                              // splits per group and step: 68 per step in all
   __shared__ float red[4][6][kH128];
   const LayerArgs& L = a.L;
   const int h = threadIdx.x & 127, g = threadIdx.x >> 7;
