@@ -220,7 +220,7 @@ Workspace layout(const csa_layer_t* L, int op, int32_t Tq, int64_t n_max) {
     const int64_t slots = (dense ? (n_max > 0 ? n_max : 1) : (int64_t)L->top_k) + L->window;
     const int splits = attend_num_splits(la, dense, (int)rows, slots, num_sms());
     w.part = off; w.part_bytes = attend_partial_bytes(la, dense, (int)rows, splits); off = up(off + w.part_bytes);
-    if (attend_path(la, dense) == 2) { w.qt = off; off = up(off + rows * (size_t)L->H * L->D * 2); }
+    if (attend_path(la, dense, (int)rows) == 2) { w.qt = off; off = up(off + rows * (size_t)L->H * L->D * 2); }
   }
   w.total = off;
   return w;
@@ -306,7 +306,7 @@ csa_status_t make_attend_args(const csa_layer_t* L, const csa_cache_t* cache, co
                               const int64_t* q_pos, int32_t Tq, const int32_t* topk, int64_t n_max, void* out,
                               const Workspace& w, void* ws, AttendArgs& a) {
   a.L = layer_args(L);
-  if (attend_path(a.L, topk == nullptr) == 0 && L->H > 32)
+  if (attend_path(a.L, topk == nullptr, L->B * Tq) == 0 && L->H > 32)
     return fail(CSA_ERR_UNSUPPORTED, "attention: H=%d needs D=512 with bf16/mixed rows and H%%32==0, or H<=32", L->H);
   a.C = cache_args(cache);
   a.q = static_cast<const uint8_t*>(q);

@@ -1285,12 +1285,14 @@ cudaError_t launch_mma(const AttendArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-int attend_path(const LayerArgs& L, bool dense) {
-  // 128 heads of 512 dims take the tcgen05 kernel, dense and top-k alike (a top-k list of about
-  // 1,150 slots is 18 cluster pairs of 64 slots, measured faster than the mma.sync kernel over
-  // every SM and than 9 pairs of 128); other head counts take the mma.sync kernel
+int attend_path(const LayerArgs& L, bool dense, int rows) {
+  // Decode-like calls (few query rows) with 128 heads of 512 dims take the tcgen05 kernel, dense and
+  // top-k alike: a top-k list of about 1,150 slots is 18 cluster pairs of 64 slots, measured faster
+  // than the mma.sync kernel over every SM and than 9 pairs of 128.  That kernel gives every query
+  // one CTA pair per slot tile and a partial per tile, so calls with many query rows (chunked
+  // prefill) take the mma.sync kernel, which needs no split there; so do other head counts.
   (void)dense;
-  if (L.H == kH128 && L.D == kD && L.d_rope == 64 &&
+  if (rows <= kTcMaxRows && L.H == kH128 && L.D == kD && L.d_rope == 64 &&
       (L.kv_fmt == CSA_FMT_BF16 || L.kv_fmt == CSA_FMT_MIXED))
     return 2;
   return attend_head_group(L) > 0 ? 1 : 0;
@@ -1305,7 +1307,7 @@ int attend_head_group(const LayerArgs& L) {
 }
 
 int attend_num_splits(const LayerArgs& L, bool dense, int rows, int64_t slots, int num_sms) {
-  if (attend_path(L, dense) == 2) {
+  if (attend_path(L, dense, rows) == 2) {
     const int n = dense ? kTcN : kTcNSparse;
     const int64_t s = (slots + n - 1) / n;
     return (int)(s < 1 ? 1 : s);
@@ -1322,14 +1324,14 @@ int attend_num_splits(const LayerArgs& L, bool dense, int rows, int64_t slots, i
 }
 
 size_t attend_partial_bytes(const LayerArgs& L, bool dense, int rows, int splits) {
-  if (attend_path(L, dense) == 2) return splits <= 1 ? 0 : (size_t)rows * splits * kTcPartBytes;
+  if (attend_path(L, dense, rows) == 2) return splits <= 1 ? 0 : (size_t)rows * splits * kTcPartBytes;
   const int HG = attend_head_group(L);
   if (HG == 0 || splits <= 1) return 0;
   return (size_t)rows * (L.H / HG) * splits * HG * (kD + 2) * sizeof(float);
 }
 
 cudaError_t launch_attend_qprep(const AttendArgs& a, cudaStream_t s) {
-  if (a.rows <= 0 || attend_path(a.L, a.topk == nullptr) != 2) return cudaSuccess;
+  if (a.rows <= 0 || attend_path(a.L, a.topk == nullptr, a.rows) != 2) return cudaSuccess;
   return launch_kernel(qprep_kernel, dim3((unsigned)((a.L.H + 3) / 4), (unsigned)a.rows), dim3(128), 0, s, 0, a);
 }
 
@@ -1385,7 +1387,7 @@ cudaError_t launch_tc(const AttendArgs& a, cudaStream_t s) {
 
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
   if (a.rows <= 0) return cudaSuccess;
-  if (attend_path(a.L, a.topk == nullptr) == 2)
+  if (attend_path(a.L, a.topk == nullptr, a.rows) == 2)
     return a.L.kv_fmt == CSA_FMT_MIXED ? launch_tc<CSA_FMT_MIXED>(a, s) : launch_tc<CSA_FMT_BF16>(a, s);
   const int HG = attend_head_group(a.L);
   if (HG == 0) {

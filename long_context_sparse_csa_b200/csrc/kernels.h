@@ -128,10 +128,11 @@ struct AttendArgs {
   float* part;              // [rows][H/HG][splits][HG*(D+2)] partial (O, m, l)
   uint8_t* out;             // [rows][H][D] act
 };
-// Attention kernel family: 2 = tcgen05 (dense slots, H = 128, D = 512, bf16 or mixed rows),
-// 1 = mma.sync head groups, 0 = CUDA-core generic kernel.  `dense`: every visible entry (HCA) rather
-// than a top-k list.
-int attend_path(const LayerArgs& L, bool dense);
+// Attention kernel family for a call of `rows` query rows: 2 = tcgen05 (H = 128, D = 512, bf16 or
+// mixed rows, at most kTcMaxRows rows), 1 = mma.sync head groups, 0 = CUDA-core generic kernel.
+// `dense`: every visible entry (HCA) rather than a top-k list.
+constexpr int kTcMaxRows = 8;
+int attend_path(const LayerArgs& L, bool dense, int rows);
 // Head-group size of the mma.sync kernel (0: not applicable).
 int attend_head_group(const LayerArgs& L);
 int attend_num_splits(const LayerArgs& L, bool dense, int rows, int64_t slots, int num_sms);

@@ -108,3 +108,18 @@ def test_unsupported_attention_shape_is_reported():
     need = C.csa_workspace_size(L, "hca_attend", 1, 16)
     st = h.hca_attend(ctypes.byref(L), ctypes.byref(cache), ctypes.byref(params), p, p, 1, 16, p, p, need, None)
     assert st == 2, h.csa_last_error()
+
+
+def test_workspace_of_many_query_rows_has_no_per_tile_partials():
+    # 128 heads of 512 dims: decode-like calls (a few query rows) take the tcgen05 kernel, whose
+    # per-query slot tiles each leave a partial (about 132 KB) plus a bf16 q~ row block; a chunk of
+    # 8,192 queries takes the mma.sync kernel instead, so its workspace stays far from the
+    # 8,192 x 18 x 132 KB = 19 GB the tile partials would need
+    from csa_synth.configs import CSA_PRO
+    dec = C.layer_from_spec(CSA_PRO, 1)
+    need_dec = C.csa_workspace_size(dec, "decode_step", 1, 1 << 18)
+    one = C.layer_from_spec(CSA_PRO, 1)
+    need_pf = C.csa_workspace_size(one, "prefill", 8192, 18432)
+    scores = 8192 * 18432 * 4
+    assert need_dec > 18 * 128 * 512 * 2                # the decode step's 18 bf16 partials are there
+    assert need_pf < scores + (1 << 30)                 # scores + top-k + modest scratch, no 19 GB

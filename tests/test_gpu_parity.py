@@ -445,8 +445,8 @@ def test_prefill_from_empty_cache():
 
 
 def test_prefill_hca_dense():
-    # HCA chunked prefill: every query of the chunk attends densely (tcgen05 kernel, one row per query,
-    # one or two 128-slot splits per query)
+    # HCA chunked prefill: every query of the chunk attends densely (200 query rows: the mma.sync
+    # kernel; calls of at most 8 rows take the tcgen05 kernel, which the decode tests cover)
     wl = get_workload("csa_prefill_8k", layers=(HCA_PRO,))
     _check_prefill(wl, Tq=200, prefix=4096 + 2, queries=[0, 1, 62, 63, 64, 127, 128, 199])
 
