@@ -240,11 +240,20 @@ def job_value(units_per_rank, world, T_ms):
 
 # ----------------------------------------------------------------------------- our arm
 
+def _code_only(text):
+    """Source text without comments or blank lines, so a comment edit does not change the hash."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+    return "\n".join(ln for ln in lines if ln)
+
+
 def sha_of(paths):
+    """Hash of the kernel sources' code (comments excluded)."""
     h = hashlib.sha256()
     for p in paths:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, p), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -10,10 +10,12 @@
 // x (QN queries * H_I heads) is one tcgen05 kind::f8f6f4 MMA chain (M = 128
 // entries, N = QN*H_I, K = 128 in four K=32 steps) with A = index keys staged
 // by TMA in the 128-byte swizzle layout and B = index queries, accumulating
-// in TMEM.  A persistent CTA per SM runs a 3-role pipeline: warp 0 issues TMA
-// loads into a 6-stage ring, warp 1 issues the MMAs into two TMEM
-// accumulators, warps 2-5 read the accumulator back with tcgen05.ld, apply
-// the ReLU / head-weight epilogue and store the fp32 scores (coalesced).
+// in TMEM.  Two persistent CTAs per SM each run a 3-role pipeline: warp 0
+// issues TMA loads into a ring (decode 4 stages, prefill 2), warp 1 issues the
+// MMAs into TMEM accumulators (decode 4 of N = 32 columns, prefill 1 of
+// N = 256: the two CTAs share the SM's 512 columns), warps 2-5 read an
+// accumulator back with tcgen05.ld, apply the ReLU / head-weight epilogue and
+// store the fp32 scores (coalesced).
 // Decode streams the keys once from HBM; it is a bandwidth-bound kernel whose
 // MMA keeps the 64 FLOP/byte of 32 heads off the CUDA cores.
 #include <cudaTypedefs.h>
