@@ -9,9 +9,13 @@
 // the raw rows; the pooled vector gets an RMSNorm and rotary embedding on its
 // last 64 dims at position pos0 + i*m, and is stored in the cache format.
 //
-// One CTA per (token, sequence), D/4 threads, 4 consecutive channels per
-// thread; raw rows are read once with 8/16-byte vector loads and the
-// per-channel softmax runs online in registers.
+// Decode: a thread-block cluster per (token, sequence) splits the channels
+// (8 CTAs, or 16 for long pooling windows); inside a CTA, threads of 4
+// consecutive channels times row groups that pool strided subsets of the
+// window with an online softmax in registers, merged in shared memory; the
+// row-wide RMSNorm sum and FP8 amax are reduced over the cluster by mail.
+// Chunked prefill: one CTA per token.  Raw rows are read once with 8/16-byte
+// vector loads.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
