@@ -124,8 +124,9 @@ struct AttendArgs {
   int64_t n_max;            // dense: entries bound
   const float* gamma_q;     // [D] or null
   const float* sinks;       // [H]
-  int splits;               // CTAs per (row, head group) along the key slots
-  float* part;              // [rows][H/HG][splits][HG*(D+2)] partial (O, m, l)
+  int splits;               // slot splits per row (tcgen05: cluster pairs; mma.sync: CTAs per head group)
+  float* part;              // partials (O, m, l): mma.sync [rows][H/HG][splits][HG*(D+2)] fp32;
+                            // tcgen05 [rows][splits] x (bf16 O/l as [D/4][H][4], then (m, l) fp32 per head)
   uint8_t* out;             // [rows][H][D] act
 };
 // Attention kernel family for a call of `rows` query rows: 2 = tcgen05 (H = 128, D = 512, bf16 or
