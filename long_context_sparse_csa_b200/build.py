@@ -1,6 +1,10 @@
 """Build libcsa.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-Usage: python -m long_context_sparse_csa_b200.build [--force]
+Usage: python -m long_context_sparse_csa_b200.build [--force] [--trace]
+
+--trace builds libcsa_trace.so instead: the same kernels with CSA_TRACE defined, so they record
+per-CTA timestamps that `python -m long_context_sparse_csa_b200.diag_trace` reads (diagnostics only;
+the product library never has them).
 """
 
 import os
@@ -13,6 +17,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libcsa.so")
+TRACE_LIB = os.path.join(HERE, "libcsa_trace.so")
 
 SOURCES = ["compress.cu", "index_score.cu", "topk.cu", "attend.cu", "api.cu", "static_scratch.cu"]
 HEADERS = ["common.cuh", "sm100.cuh", "kernels.h"]
@@ -38,29 +43,31 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, trace: bool = False) -> str:
+    build_dir = os.path.join(BUILD, "trace") if trace else BUILD
+    lib = TRACE_LIB if trace else LIB
+    flags = NVCC_FLAGS + (["-DCSA_TRACE"] if trace else [])
+    os.makedirs(build_dir, exist_ok=True)
     nvcc = _nvcc()
     headers = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, "csa.h")]
     objs = []
     for src in SOURCES:
         s = os.path.join(CSRC, src)
-        o = os.path.join(BUILD, src.replace(".cu", ".o"))
+        o = os.path.join(build_dir, src.replace(".cu", ".o"))
         objs.append(o)
         if force or _stale(o, [s] + headers):
-            cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-c", s, "-o", o]
+            cmd = [nvcc, *flags, "-I", INCLUDE, "-c", s, "-o", o]
             if verbose:
                 print(" ".join(cmd), flush=True)
             subprocess.run(cmd, check=True)
-    if force or _stale(LIB, objs):
-        cmd = [nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", LIB,
+    if force or _stale(lib, objs):
+        cmd = [nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", lib,
                "-lcudart_static", "-ldl", "-lpthread", "-lrt"]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True, trace="--trace" in sys.argv))
