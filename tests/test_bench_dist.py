@@ -100,3 +100,17 @@ def test_prefill_work_matches_the_workload_arithmetic():
     assert abs(idx - 1.168e12) < 0.001e12
     assert abs(att - 1.237e12) < 0.001e12
     assert abs(gather - 9.66e9) < 0.01e9
+
+
+def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    # the recorded DRAM traffic stays valid across comment edits of the indexer sources, and is
+    # dropped (traffic null) once their code changes
+    src = "__global__ void k(int* p) {  // writes one\n  /* block\n comment */ p[0] = 1;\n}\n"
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    f = tmp_path / "k.cu"
+    f.write_text(src)
+    h0 = bench.sha_of(["k.cu"])
+    f.write_text(src.replace("writes one", "stores a 1").replace("block\n comment", "other words"))
+    assert bench.sha_of(["k.cu"]) == h0
+    f.write_text(src.replace("p[0] = 1", "p[0] = 2"))
+    assert bench.sha_of(["k.cu"]) != h0
