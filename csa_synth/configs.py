@@ -29,9 +29,10 @@ class Layer:
     H_I: int = 0              # indexer heads (CSA)
     d_I: int = 0              # indexer head dim (CSA)
     kv_format: str = "bf16"   # "f32" | "bf16" | "mixed" (e4m3 non-rotary + bf16 rotary + fp32 scale)
-    idx_format: str = "e4m3"  # "f32" | "e4m3"
+    idx_format: str = "e4m3"  # "f32" | "e4m3" | "e2m1" (FP4 keys with block scales, e4m3 queries)
     act_format: str = "bf16"  # query / raw-row / gate / output dtype: "f32" | "bf16"
     eps: float = 1e-6
+    idx_rank: int = 512       # CSA: width r of the query latent the index query is projected from
 
 
 @dataclass(frozen=True)

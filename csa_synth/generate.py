@@ -94,10 +94,34 @@ def kv_rows(seed: int, tag: str, layer_idx: int, lead_shape, layer: Layer) -> np
     raise ValueError(layer.kv_format)
 
 
+# magnitudes of the 8 non-negative e2m1 codes are 0, .5, 1, 1.5, 2, 3, 4, 6: a draw is binned at the
+# midpoints between them (random bytes in the FP4 key layout; nothing here scores or selects)
+_E2M1_MIDPOINTS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+
+
+def _fp4_keys(seed, layer_idx, lead_shape, d):
+    """Random FP4 index keys in storage form: packed e2m1 codes [..., d/2] (even dim in the low
+    nibble) of draws N(0, 2^2), and scale words [...] holding a per-key exponent from {-6, -5, -4}
+    (+127, bits 0..7) and per-32-dim block offsets from {0, 1, 2} (bits 8+4b..11+4b)."""
+    z = _normal(stream(seed, "idx_k", layer_idx), tuple(lead_shape) + (d,), 2.0)
+    mag = np.digitize(np.abs(z), _E2M1_MIDPOINTS).astype(np.uint8)
+    codes = np.where((z < 0) & (mag > 0), mag | 0x8, mag).astype(np.uint8)
+    packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+    e = stream(seed, "idx_k.exp", layer_idx).choice(np.array([-6, -5, -4]), size=tuple(lead_shape))
+    off = stream(seed, "idx_k.blk", layer_idx).integers(0, 3, size=tuple(lead_shape) + (d // 32,))
+    word = (e + 127).astype(np.uint64)
+    for b in range(d // 32):
+        word = word | (off[..., b].astype(np.uint64) << np.uint64(8 + 4 * b))
+    return packed, word.astype(np.uint32)
+
+
 def index_keys(seed, layer_idx, lead_shape, layer: Layer):
-    """Index keys N(0, 1/d_I): (keys, scales).  f32: keys float32, scales all 1."""
+    """Index keys N(0, 1/d_I): (keys, scales).  f32: keys float32, scales all 1.  e2m1: packed FP4
+    codes and scale words (_fp4_keys)."""
     std = 1.0 / np.sqrt(layer.d_I)
     shape = tuple(lead_shape) + (layer.d_I,)
+    if layer.idx_format == "e2m1":
+        return _fp4_keys(seed, layer_idx, lead_shape, layer.d_I)
     if layer.idx_format == "f32":
         return _normal(stream(seed, "idx_k", layer_idx), shape, std), np.ones(lead_shape, np.float32)
     return _fp8_with_row_scale(stream(seed, "idx_k", layer_idx), stream(seed, "idx_k.exp", layer_idx),
@@ -105,7 +129,8 @@ def index_keys(seed, layer_idx, lead_shape, layer: Layer):
 
 
 def index_queries(seed, layer_idx, lead_shape, layer: Layer):
-    """Index queries N(0,1) per head: (queries, scales) with scales [*lead_shape, H_I]."""
+    """Index queries N(0,1) per head: (queries, scales) with scales [*lead_shape, H_I] (e4m3 codes
+    for both the e4m3 and the e2m1 key formats)."""
     shape = tuple(lead_shape) + (layer.H_I, layer.d_I)
     if layer.idx_format == "f32":
         return _normal(stream(seed, "idx_q", layer_idx), shape), np.ones(shape[:-1], np.float32)
@@ -128,8 +153,27 @@ def _common(wl: Workload, li: int, layer: Layer, lead):
     return d
 
 
-def decode_inputs(wl: Workload, li: int = 0, n=None, entry_cap=None):
-    """State and step inputs of one decode step of layer ``li``.
+def index_stream_inputs(wl: Workload, li: int, lead_shape, layer: Layer):
+    """Inputs of the index side produced in a step: index-key stream rings and new rows, its slot
+    biases, the query latent c [*lead, r] N(0,1) and the up-projection W [H_I*d_I, r] N(0, 1/r)."""
+    B = lead_shape[0]
+    rr = raw_ring_rows(layer)
+    r = layer.idx_rank
+    return {
+        "idx_raw_ring": act_array(stream(wl.seed, "idx_raw_ring", li), (B, rr, layer.d_I), layer.act_format),
+        "idx_gate_ring": act_array(stream(wl.seed, "idx_gate_ring", li), (B, rr, layer.d_I), layer.act_format),
+        "idx_x_new": act_array(stream(wl.seed, "idx_x_new", li), tuple(lead_shape) + (layer.d_I,), layer.act_format),
+        "idx_g_new": act_array(stream(wl.seed, "idx_g_new", li), tuple(lead_shape) + (layer.d_I,), layer.act_format),
+        "idx_pos_bias": _normal(stream(wl.seed, "idx_pos_bias", li), ((1 + layer.ov) * layer.m, layer.d_I)),
+        "c_q": act_array(stream(wl.seed, "c_q", li), tuple(lead_shape) + (r,), layer.act_format),
+        "W_iq": act_array(stream(wl.seed, "W_iq", li), (layer.H_I * layer.d_I, r), layer.act_format,
+                          std=1.0 / np.sqrt(r)),
+    }
+
+
+def decode_inputs(wl: Workload, li: int = 0, n=None, entry_cap=None, indexed=False):
+    """State and step inputs of one decode step of layer ``li`` (with ``indexed``, also the inputs of
+    the index side produced in the step: index_stream_inputs).
 
     The step is for token t = pos0 + n - 1 of every sequence.  Caches hold
     random stored rows: entries [B, entry_cap, row], window ring
@@ -156,6 +200,8 @@ def decode_inputs(wl: Workload, li: int = 0, n=None, entry_cap=None):
     })
     if layer.kind == "csa":
         d["idx_k"], d["idx_k_scale"] = index_keys(wl.seed, li, (B, cap), layer)
+        if indexed:
+            d.update(index_stream_inputs(wl, li, (B,), layer))
     return d
 
 

@@ -28,6 +28,17 @@ R7  Logits l_j = <q~, k~_j> / sqrt(D); sink: p_j = e^{l_j} / (e^{s_h} + sum e^{l
 R8  RoPE: interleaved pairs (D-64+2u, D-64+2u+1), theta_u = base^(-2u/64),
     angle pos*theta_u in float64.
 R9  RMSNorm eps = 1e-6 with a learnable per-channel weight gamma.
+R14 Index keys come from an index-key stream compressed like the KV stream: every token carries
+    an index row and a row of gate logits of d_I channels, and the key of entry i pools the same
+    window rows with the same per-channel softmax of gate + slot bias (its own bias table), with
+    no RMSNorm and no rotation; it is stored as e4m3 codes with one power-of-two scale per key
+    (the R10 rule), or as float32.  "DeepSeek-V4 Explained: ...", "The attention stack, and why it
+    is two mechanisms", has the indexer score the compressed entries; the keys it scores are read
+    here as compressed the same way.
+R15 The low-rank index query: the query token's low-rank latent c (r values, an input) is mapped
+    by a learned up-projection W [H_I * d_I, r] to the H_I index-query heads, q_h = W_h c, each head
+    stored as e4m3 codes with its own power-of-two scale (R10).  The same section calls the
+    indexer low-rank; this is its plainest form.  Head weights w_h stay inputs.
 """
 
 import numpy as np
@@ -115,6 +126,28 @@ def compress(raw, gate, bias, gamma, m, ov, d_rope, base, pos0, entries, raw_fir
     return np.stack(out) if out else np.zeros((0, raw.shape[1]))
 
 
+def compress_index_keys(raw_i, gate_i, bias_i, m, ov, entries, raw_first_row=0):
+    """Index-key values (float64 [len(entries), d_I]) of the given entries (R14): pool only.
+
+    raw_i, gate_i: float64 [n_rows, d_I] index rows and gate logits of raw rows raw_first_row..;
+    bias_i: [(1+ov)m, d_I].
+    """
+    out = []
+    for i in entries:
+        rows, slots = entry_rows(int(i), m, ov)
+        idx = rows - raw_first_row
+        assert idx.min() >= 0 and idx.max() < raw_i.shape[0], "source rows not provided"
+        out.append(pool_entry(raw_i[idx], gate_i[idx], bias_i, slots))
+    return np.stack(out) if out else np.zeros((0, raw_i.shape[1]))
+
+
+def index_query(c, W, H_I: int, d_I: int):
+    """Index-query heads [H_I, d_I] from the query's low-rank latent c [r] (R15): q = W c."""
+    W = np.asarray(W, np.float64)
+    c = np.asarray(c, np.float64)
+    return (W @ c).reshape(H_I, d_I)
+
+
 # --------------------------------------------------------------------------- visibility
 
 def n_visible(t, pos0: int, m: int):
@@ -141,6 +174,20 @@ def index_scores(iq, iq_scale, head_w, ik, ik_scale):
     dots = np.asarray(ik, np.float64) @ np.asarray(iq, np.float64).T          # [N, H_I]
     z = dots * np.asarray(ik_scale, np.float64)[:, None] * np.asarray(iq_scale, np.float64)[None, :]
     return np.maximum(z, 0.0) @ np.asarray(head_w, np.float64)
+
+
+def index_operands(L, q_codes, k_codes, k_scales):
+    """(query values before their scale, key values, key scales) of the indexer in float64.
+
+    e4m3 / f32 keys keep their per-key scale apart; FP4 keys (idx_format "e2m1", read as the pages'
+    FP4 indexer: "DeepSeek-V4: Making a Million Tokens Affordable", "Two ways to shrink attention,
+    interleaved") are decoded with their block scales applied and a key scale of 1.  With FP4 keys the
+    index queries are e4m3 (the pages put the indexer's attention in FP4; the keys are its stored side).
+    """
+    if L.idx_format == "e2m1":
+        return (F.decode_idx(q_codes, "e4m3"), F.decode_fp4_keys(k_codes, k_scales),
+                np.ones(len(k_scales), np.float64))
+    return F.decode_idx(q_codes, L.idx_format), F.decode_idx(k_codes, L.idx_format), k_scales
 
 
 def top_k(scores, k: int):
@@ -283,9 +330,8 @@ def decode_step(L, st, b: int):
         return F.decode_rows(raw_bytes, L.kv_format, D, L.d_rope)
 
     if L.kind == "csa":
-        iq = F.decode_idx(st["idx_q"][b], L.idx_format)
-        ik = F.decode_idx(st["idx_k"][b][:n_vis], L.idx_format)
-        s = index_scores(iq, st["idx_q_scale"][b], st["head_w"][b], ik, st["idx_k_scale"][b][:n_vis])
+        iq, ik, iks = index_operands(L, st["idx_q"][b], st["idx_k"][b][:n_vis], st["idx_k_scale"][b][:n_vis])
+        s = index_scores(iq, st["idx_q_scale"][b], st["head_w"][b], ik, iks)
         sel = top_k_fast(s, L.top_k)
         res["scores"], res["topk"] = s, sel
         ent = entry_values(sel[sel >= 0])
@@ -297,6 +343,47 @@ def decode_step(L, st, b: int):
     q = F.decode_act(st["q"][b], L.act_format)
     res["o"] = attend(q, t, rows, st["sinks"], st["gamma_q"], L.d_rope, L.rope_base, L.scale, L.eps)
     res["n_rows"] = rows.shape[0]
+    return res
+
+
+def decode_step_indexed(L, st, b: int):
+    """decode_step with the index side produced in the step (R14, R15): the new token's index row
+    and gate row go into the index rings, the index key of the entry the token completes is
+    compressed from them, and the index query comes from the latent c through W.  st holds
+    decode_step's keys plus idx_raw_ring / idx_gate_ring [B, (1+ov)m, d_I], idx_x_new / idx_g_new
+    [B, d_I] (act format), idx_pos_bias [(1+ov)m, d_I], c_q [B, r] and W_iq [H_I*d_I, r] (act format).
+    Returns decode_step's result plus "index_key" (i, codes, scale) when a group completed and
+    "idx_q" (codes, scales)."""
+    t = int(st["t"][b])
+    r = t - L.pos0
+    m, ov = L.m, L.ov
+    rr = (1 + ov) * m
+    st2 = dict(st)
+    extra = {}
+    raw_i = F.decode_act(st["idx_raw_ring"][b], L.act_format).copy()
+    gate_i = F.decode_act(st["idx_gate_ring"][b], L.act_format).copy()
+    raw_i[r % rr] = F.decode_act(st["idx_x_new"][b], L.act_format)
+    gate_i[r % rr] = F.decode_act(st["idx_g_new"][b], L.act_format)
+    if (r + 1) % m == 0:
+        i = (r + 1) // m - 1
+        rows, slots = entry_rows(i, m, ov)
+        key = pool_entry(raw_i[rows % rr], gate_i[rows % rr], st["idx_pos_bias"], slots)
+        codes, scale = F.encode_idx(key[None], L.idx_format, "key")
+        idx_k = np.array(st["idx_k"], copy=True)
+        idx_ks = np.array(st["idx_k_scale"], copy=True)
+        idx_k[b, i] = codes[0]
+        idx_ks[b, i] = scale[0]
+        st2["idx_k"], st2["idx_k_scale"] = idx_k, idx_ks
+        extra["index_key"] = (i, codes[0], scale[0])
+    q = index_query(F.decode_act(st["c_q"][b], L.act_format), F.decode_act(st["W_iq"], L.act_format), L.H_I, L.d_I)
+    qc, qs = F.encode_idx(q, L.idx_format, "query")
+    iq = np.array(st["idx_q"], copy=True)
+    iqs = np.array(st["idx_q_scale"], copy=True)
+    iq[b], iqs[b] = qc, qs
+    st2["idx_q"], st2["idx_q_scale"] = iq, iqs
+    extra["idx_q"] = (qc, qs)
+    res = decode_step(L, st2, b)
+    res.update(extra)
     return res
 
 
@@ -332,9 +419,8 @@ def prefill_query(L, pf, entries, window, b: int, j: int):
     n_vis = int(n_visible(t, L.pos0, L.m))
     res = {}
     if L.kind == "csa":
-        iq = F.decode_idx(pf["idx_q"][b, j], L.idx_format)
-        ik = F.decode_idx(pf["idx_k"][b][:n_vis], L.idx_format)
-        s = index_scores(iq, pf["idx_q_scale"][b, j], pf["head_w"][b, j], ik, pf["idx_k_scale"][b][:n_vis])
+        iq, ik, iks = index_operands(L, pf["idx_q"][b, j], pf["idx_k"][b][:n_vis], pf["idx_k_scale"][b][:n_vis])
+        s = index_scores(iq, pf["idx_q_scale"][b, j], pf["head_w"][b, j], ik, iks)
         sel = top_k_fast(s, L.top_k)
         res["scores"], res["topk"] = s, sel
         ids = sel[sel >= 0]

@@ -145,6 +145,139 @@ def decode_act(a: np.ndarray, fmt: str) -> np.ndarray:
     raise ValueError(fmt)
 
 
+# --------------------------------------------------------------------------- FP4 (e2m1) index keys
+#
+# "DeepSeek-V4: Making a Million Tokens Affordable", "Two ways to shrink attention, interleaved":
+# the indexer's attention runs in FP4.  The format is read as OCP e2m1 (1 sign bit, 2 exponent bits
+# with bias 1, 1 mantissa bit; exponent field 0 is subnormal m * 0.5; no infinities or NaN; largest
+# finite 6) with block scaling.  Reading of the scales (the pages give none): a key of d dims has one
+# power-of-two scale sigma (the smallest with max|k| / sigma <= 6) and, per block of 32 dims, an
+# offset delta_b in 0..7 that scales the block further down by 2^-delta_b (the largest delta_b with
+# max_block|k| * 2^delta_b / sigma <= 6, capped at 7): value = code * sigma * 2^-delta_b.  Codes are
+# round-to-nearest-even with saturation at 6, two per byte (the even dim in the low nibble).  The scale
+# word of a key packs the exponent of sigma (+127) in bits 0..7 and delta_b in bits 8 + 4b .. 11 + 4b.
+
+E2M1_MAX = 6.0
+FP4_BLOCK = 32
+
+
+def _e2m1_value(code: int) -> float:
+    s = -1.0 if code & 0x8 else 1.0
+    e = (code >> 1) & 0x3
+    m = code & 0x1
+    if e == 0:
+        return s * m * 0.5
+    return s * (1.0 + m / 2.0) * 2.0 ** (e - 1)
+
+
+E2M1_TABLE = np.array([_e2m1_value(c) for c in range(16)], dtype=np.float64)
+_E2M1_POS = E2M1_TABLE[:8].copy()          # 0, 0.5, 1, 1.5, 2, 3, 4, 6 (strictly increasing)
+
+
+def e2m1_encode(x: np.ndarray) -> np.ndarray:
+    """Round to the nearest e2m1 value, ties to the even code, saturating at +-6 (uint8 codes 0..15)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), E2M1_MAX)
+    hi = np.minimum(np.searchsorted(_E2M1_POS, a, side="left"), 7)
+    lo = np.maximum(hi - 1, 0)
+    d_lo = a - _E2M1_POS[lo]
+    d_hi = _E2M1_POS[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(_E2M1_POS[hi] == a, hi, code).astype(np.uint8)
+    return np.where(np.signbit(x) & (code != 0), code | 0x8, code).astype(np.uint8)
+
+
+def e2m1_decode(codes: np.ndarray) -> np.ndarray:
+    return E2M1_TABLE[np.asarray(codes, dtype=np.uint8) & 0xF]
+
+
+def fp4_pack(codes: np.ndarray) -> np.ndarray:
+    """[..., d] codes (d even) -> [..., d/2] bytes, the even dim in the low nibble."""
+    c = np.asarray(codes, dtype=np.uint8)
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+def fp4_unpack(packed: np.ndarray) -> np.ndarray:
+    p = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = p >> 4
+    return out
+
+
+def pow2_scale_fp4(amax: np.ndarray) -> np.ndarray:
+    """Smallest power of two sigma with amax / sigma <= 6; 1 where amax == 0.  6 = 0.75 * 2^3: with
+    amax = f * 2^e (0.5 <= f < 1) the bound holds first at k = e - 3 when f <= 0.75, else e - 2."""
+    amax = np.asarray(amax, dtype=np.float64)
+    f, e = np.frexp(amax)
+    k = np.where(f <= 0.75, e - 3, e - 2)
+    return np.where(amax == 0, 1.0, np.ldexp(1.0, k))
+
+
+def encode_fp4_keys(x: np.ndarray):
+    """Keys float64 [..., d] (d a multiple of 32) -> (packed codes uint8 [..., d/2], scale words uint32 [...])."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    nb = d // FP4_BLOCK
+    blocks = x.reshape(x.shape[:-1] + (nb, FP4_BLOCK))
+    bmax = np.max(np.abs(blocks), axis=-1)                              # [..., nb]
+    sigma = pow2_scale_fp4(np.max(bmax, axis=-1))                       # [...]
+    # delta_b: largest integer with bmax * 2^delta / sigma <= 6, in 0..7
+    ratio = bmax / sigma[..., None]                                     # <= 6
+    delta = np.zeros_like(bmax, dtype=np.int64)
+    for dd in range(1, 8):
+        delta = np.where(ratio * 2.0 ** dd <= E2M1_MAX, dd, delta)
+    bscale = sigma[..., None] * np.exp2(-delta.astype(np.float64))      # [..., nb]
+    codes = e2m1_encode(blocks / bscale[..., None]).reshape(x.shape)
+    e = np.round(np.log2(sigma)).astype(np.int64) + 127
+    word = e.astype(np.uint64)
+    for b in range(nb):
+        word = word | (delta[..., b].astype(np.uint64) << np.uint64(8 + 4 * b))
+    return fp4_pack(codes), word.astype(np.uint32)
+
+
+def decode_fp4_keys(packed: np.ndarray, words: np.ndarray) -> np.ndarray:
+    """(packed codes [..., d/2], scale words [...]) -> exact values float64 [..., d]."""
+    codes = fp4_unpack(packed)
+    d = codes.shape[-1]
+    nb = d // FP4_BLOCK
+    w = np.asarray(words, dtype=np.uint32).astype(np.int64)
+    sigma = np.exp2((w & 0xFF) - 127.0)
+    vals = e2m1_decode(codes).reshape(codes.shape[:-1] + (nb, FP4_BLOCK))
+    delta = np.stack([(w >> (8 + 4 * b)) & 0xF for b in range(nb)], axis=-1).astype(np.float64)
+    return (vals * (sigma[..., None] * np.exp2(-delta))[..., None]).reshape(codes.shape)
+
+
+def encode_scaled_e4m3(x: np.ndarray):
+    """Values float64 [..., d] -> (e4m3 codes uint8 [..., d], float32 scale [...]) with one power-of-two
+    scale per leading index (the row-scale rule of the mixed rows: max|x| / scale <= 448)."""
+    x = np.asarray(x, dtype=np.float64)
+    sigma = pow2_scale(np.max(np.abs(x), axis=-1))
+    return e4m3_encode(x / sigma[..., None]), sigma.astype(np.float32)
+
+
+def encode_idx(x: np.ndarray, fmt: str, role: str = "key"):
+    """Index keys / queries in storage form: (codes, scales).  e4m3: scaled codes as encode_scaled_e4m3;
+    f32: the float32 values with scale 1; e2m1: keys as encode_fp4_keys (packed codes, scale words),
+    queries (role "query") as e4m3."""
+    x = np.asarray(x, dtype=np.float64)
+    if fmt == "e2m1":
+        return encode_fp4_keys(x) if role == "key" else encode_scaled_e4m3(x)
+    if fmt == "e4m3":
+        return encode_scaled_e4m3(x)
+    if fmt == "f32":
+        return x.astype(np.float32), np.ones(x.shape[:-1], np.float32)
+    raise ValueError(fmt)
+
+
+def decode_idx_keys(codes: np.ndarray, scales: np.ndarray, fmt: str) -> np.ndarray:
+    """Stored index keys -> exact values, scales applied (e2m1: block scales included)."""
+    if fmt == "e2m1":
+        return decode_fp4_keys(codes, scales)
+    return decode_idx(codes, fmt) * np.asarray(scales, np.float64)[..., None]
+
+
 def decode_idx(codes: np.ndarray, fmt: str) -> np.ndarray:
     """Index keys / queries: float32 values or e4m3 codes -> float64 (before the scale)."""
     if fmt == "f32":

@@ -106,3 +106,82 @@ def test_mixed_row_layout():
     assert np.frombuffer(row[574:576].tobytes(), np.uint16)[0] == 0xC040   # -3.0 in bf16
     assert np.frombuffer(row[576:580].tobytes(), np.float32)[0] == 1.0
     assert not row[580:].any()
+
+
+# ----------------------------------------------------------------------------- FP4 (e2m1) index keys
+
+def test_e2m1_table_matches_format_definition():
+    # 1 sign bit, 2 exponent bits (bias 1), 1 mantissa bit; exponent 0 is subnormal m * 0.5
+    expect = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert np.array_equal(F.E2M1_TABLE[:8], expect)
+    assert np.array_equal(F.E2M1_TABLE[8:], [-v for v in expect])
+
+
+def test_e2m1_encode_roundtrips_and_rounds_to_nearest_even():
+    for c in range(16):
+        v = F.E2M1_TABLE[c]
+        got = F.e2m1_encode(np.array([v]))[0]
+        assert F.E2M1_TABLE[got] == v                       # -0 may come back as +0
+    ties = {0.25: 0.0, 0.75: 1.0, 1.25: 1.0, 1.75: 2.0, 2.5: 2.0, 3.5: 4.0, 5.0: 4.0}
+    for x, y in ties.items():
+        assert F.e2m1_decode(F.e2m1_encode(np.array([x, -x]))).tolist() == [y, -y]
+    assert F.e2m1_decode(F.e2m1_encode(np.array([7.0, 1e9, -6.5]))).tolist() == [6.0, 6.0, -6.0]
+    rng = np.random.default_rng(0)
+    x = rng.uniform(-6, 6, 20000)
+    d = np.abs(F.e2m1_decode(F.e2m1_encode(x))[:, None] - x[:, None])
+    best = np.min(np.abs(F.E2M1_TABLE[None, :] - x[:, None]), axis=1)
+    assert np.allclose(d[:, 0], best)                       # always a nearest value
+
+
+def test_fp4_pack_order_and_roundtrip():
+    c = np.arange(16, dtype=np.uint8)
+    p = F.fp4_pack(c)
+    assert p[0] == (0 | (1 << 4)) and p[7] == (14 | (15 << 4))
+    assert np.array_equal(F.fp4_unpack(p), c)
+
+
+def test_fp4_block_scales_follow_their_rule():
+    rng = np.random.default_rng(1)
+    x = rng.normal(size=(200, 128)) * np.exp2(rng.integers(-10, 10, size=(200, 1)))
+    x[:, 32:64] *= np.exp2(-rng.integers(0, 12, size=(200, 1)))      # blocks of very different size
+    packed, words = F.encode_fp4_keys(x)
+    w = words.astype(np.int64)
+    sigma = np.exp2((w & 0xFF) - 127.0)
+    amax = np.abs(x).max(1)
+    assert np.all(amax / sigma <= 6) and np.all(amax / sigma > 3)     # the smallest power of two
+    for b in range(4):
+        delta = (w >> (8 + 4 * b)) & 0xF
+        bmax = np.abs(x[:, 32 * b:32 * b + 32]).max(1)
+        assert np.all((delta >= 0) & (delta <= 7))
+        fits = bmax * np.exp2(delta) / sigma <= 6
+        assert np.all(fits)
+        more = bmax * np.exp2(delta + 1) / sigma <= 6
+        assert np.all(~more | (delta == 7))                         # the largest offset that fits
+    v = F.decode_fp4_keys(packed, words)
+    # within half a code step of each block's scale (the e2m1 spacing at the value's size)
+    bs = np.repeat(np.stack([sigma * np.exp2(-((w >> (8 + 4 * b)) & 0xF)) for b in range(4)], 1), 32, axis=1)
+    a = np.abs(x / bs)
+    step = np.where(a < 2, 0.5, np.where(a < 4, 1.0, 2.0))
+    assert np.all(np.abs(v - x) <= 0.5 * step * bs + 1e-300)
+
+
+def test_fp4_scores_equal_fp8_scores_on_exactly_representable_keys():
+    # keys built from e2m1 values times powers of two are exact in both formats: same scores
+    rng = np.random.default_rng(2)
+    from oracle import csa as O
+    from csa_synth.configs import CSA_PRO, scaled_layer
+    codes = rng.integers(0, 16, size=(50, 128)).astype(np.uint8)
+    k = F.e2m1_decode(codes) * np.exp2(rng.integers(-6, -2, size=(50, 1)))
+    q = rng.normal(size=(32, 128))
+    qc, qs = F.encode_scaled_e4m3(q)
+    w = rng.normal(size=32)
+    k8, s8 = F.encode_scaled_e4m3(k)
+    k4, w4 = F.encode_fp4_keys(k)
+    L8 = O.LayerSpec.of(scaled_layer(CSA_PRO))
+    L4 = O.LayerSpec.of(scaled_layer(CSA_PRO, idx_format="e2m1"))
+    a8 = O.index_operands(L8, qc, k8, s8)
+    a4 = O.index_operands(L4, qc, k4, w4)
+    assert np.allclose(a8[1] * a8[2][:, None], a4[1] * a4[2][:, None], rtol=0, atol=0)
+    s_8 = O.index_scores(a8[0], qs, w, a8[1], a8[2])
+    s_4 = O.index_scores(a4[0], qs, w, a4[1], a4[2])
+    assert np.allclose(s_8, s_4, rtol=1e-14, atol=0)
