@@ -49,6 +49,7 @@ def parse():
     p.add_argument("--replicas", type=int, default=8)
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extra-configs", action="store_true", help="skip the 128K configurations' lines")
     p.add_argument("--burn-seconds", type=float, default=0.5, help="untimed replays before timing (clocks settle)")
     return p.parse_args()
 
@@ -190,6 +191,23 @@ def run_cpu_oracle(wl, datas, budget_s, min_steps=1, max_steps=None):
     return times
 
 
+def cpu_baseline(wl, datas, budget_s):
+    """The oracle timed on the host cores on whole decode steps of the workload: with every BLAS
+    thread (`value`, `cores`) and single-threaded (`single_thread`), each for about half the budget."""
+    units = wl.B * len(wl.layers)
+    times = run_cpu_oracle(wl, datas, budget_s / 2)
+    line = {"value": units / float(np.mean(times)), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{len(times)} full decode steps of the workload ({budget_s / 2:.0f} s budget per mode)"}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            t1 = run_cpu_oracle(wl, datas, budget_s / 2)
+        line["single_thread"] = {"value": units / float(np.mean(t1)), "cores": 1, "steps": len(t1)}
+    except Exception as e:  # noqa: BLE001
+        line["single_thread"] = {"value": None, "note": f"thread limit unavailable: {e}"}
+    return line
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -258,7 +276,8 @@ def sha_of(paths):
 
 
 INDEX_KERNEL_SOURCES = ["long_context_sparse_csa_b200/csrc/index_score.cu", "long_context_sparse_csa_b200/csrc/sm100.cuh",
-                        "long_context_sparse_csa_b200/csrc/common.cuh"]
+                        "long_context_sparse_csa_b200/csrc/common.cuh", "long_context_sparse_csa_b200/csrc/kernels.h",
+                        "long_context_sparse_csa_b200/csrc/api.cu"]
 
 
 def recorded_traffic(workload):
@@ -274,13 +293,151 @@ def recorded_traffic(workload):
     return rec.get("per_launch_bytes", {}).get(workload)
 
 
+class DecodeRig:
+    """Device state of one decode workload: R independent instances of every layer's caches (at
+    distinct addresses, so consecutive steps stream different bytes), the step inputs, one
+    workspace per layer, and CUDA graphs of whole steps through the C ABI's fused decode calls."""
+
+    def __init__(self, wl, R, dev):
+        import torch
+        from csa_synth import decode_inputs
+        from long_context_sparse_csa_b200.state import LayerState, to_device
+        self.wl, self.R, self.dev = wl, R, dev
+        self.datas, self.layers = [], []
+        for li, spec in enumerate(wl.layers):
+            d = decode_inputs(wl, li)
+            self.datas.append(d)
+            base = LayerState.from_arrays(spec, wl.B, d, device=dev)
+            insts = [base]
+            for _ in range(R - 1):
+                insts.append(LayerState(spec, wl.B, 0, entries=base.entries.clone(), window=base.window.clone(),
+                                        raw=base.raw.clone(), gate=base.gate.clone(),
+                                        idx_keys=None if base.idx_keys is None else base.idx_keys.clone(),
+                                        idx_key_scale=None if base.idx_key_scale is None else base.idx_key_scale.clone(),
+                                        pos_bias=base.pos_bias, gamma_kv=base.gamma_kv, gamma_q=base.gamma_q,
+                                        sinks=base.sinks))
+            cap = d["entries"].shape[1]
+            io = {k: to_device(d[k], dev) for k in ["q", "x_new", "g_new", "t"]}
+            if spec.kind == "csa":
+                for k in ["idx_q", "idx_q_scale", "head_w"]:
+                    io[k] = to_device(d[k], dev)
+                io["topk"] = torch.zeros((wl.B, spec.top_k), dtype=torch.int32, device=dev)
+            io["out"] = torch.zeros((wl.B, spec.H, spec.D),
+                                    dtype=torch.int16 if spec.act_format == "bf16" else torch.float32, device=dev)
+            ws = base.workspace("decode_step", 1, cap)
+            self.layers.append({"spec": spec, "insts": insts, "io": io, "ws": ws,
+                                "caches": [s.cache() for s in insts], "params": base.params(), "L": base.L})
+        self.stream = torch.cuda.Stream(device=dev)
+
+    def call(self, li, r):
+        """The public decode call of layer li on instance r (eager or under capture)."""
+        from long_context_sparse_csa_b200 import binding as C
+        lay = self.layers[li]
+        io, spec = lay["io"], lay["spec"]
+        if spec.kind == "csa":
+            C.csa_decode_step(lay["L"], lay["caches"][r], lay["params"], io["q"], io["idx_q"], io["idx_q_scale"],
+                              io["head_w"], io["x_new"], io["g_new"], io["t"], io["out"], io["topk"], lay["ws"])
+        else:
+            C.hca_decode_step(lay["L"], lay["caches"][r], lay["params"], io["q"], io["x_new"], io["g_new"],
+                              io["t"], io["out"], lay["ws"])
+
+    def warm(self):
+        """Eager steps of every instance (module load, attributes, the second stream), then a check
+        of every layer's device error word."""
+        import torch
+        from long_context_sparse_csa_b200 import binding as C
+        for r in range(self.R):
+            for li in range(len(self.layers)):
+                self.call(li, r)
+        torch.cuda.synchronize()
+        for lay in self.layers:
+            assert C.csa_device_error(lay["ws"]) == 0
+
+    def capture(self, rs, lis, idx_events=False):
+        """One CUDA graph running steps of instances rs (layers lis of each, in order).  With
+        idx_events, a pair of events brackets the indexer-score launch of the first step (the only
+        event nodes: each one breaks the chain of kernel nodes and costs a few microseconds)."""
+        import torch
+        from long_context_sparse_csa_b200 import binding as C
+        pair = None
+        if idx_events:
+            pair = (_ext_event(), _ext_event())
+            for x in pair:
+                x.record()
+            torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        n0 = C.csa_launch_count()
+        with torch.cuda.graph(g, stream=self.stream):
+            for j, r in enumerate(rs):
+                for li in lis:
+                    csa = self.layers[li]["spec"].kind == "csa"
+                    if idx_events and j == 0 and csa:
+                        C.csa_profile_events(*pair)
+                    self.call(li, r)
+                    C.csa_profile_events(None, None)
+        return g, pair, C.csa_launch_count() - n0
+
+    def graphs(self, lis, steps, idx_events=False):
+        """(cycle graphs, single-step graphs, launches per step) for layers lis: n_cyc copies of the
+        cycle over the R instances, replayed round-robin (the last replay of each copy lies in the
+        timed region, so its event pair samples one indexer launch of the timed steps)."""
+        n_cyc = max(1, min(8, steps // self.R))
+        cycles = [self.capture(list(range(self.R)), lis, idx_events) for _ in range(n_cyc)]
+        singles = [self.capture([r], lis)[0] for r in range(self.R)]
+        return cycles, singles, cycles[0][2] // self.R
+
+
+def _ext_event():
+    import torch
+    return torch.cuda.Event(enable_timing=True, external=True)
+
+
+def run_steps(cycles, singles, R, k):
+    """Exactly k decode steps: whole cycles of the R instances, then single steps."""
+    for c in range(k // R):
+        cycles[c % len(cycles)][0].replay()
+    for r in range(k % R):
+        singles[r].replay()
+
+
+def timed(fn, world, dist, dev):
+    """Device time (ms) of fn() on the current stream, bracketed by a barrier and a device
+    synchronisation on both sides, max over ranks."""
+    import torch
+    cur = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    fn()
+    e1.record(cur)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    return max_over_ranks(e0.elapsed_time(e1), world, dist, dev)
+
+
+# Replicas of the 128K configurations: enough instances that one cycle streams more than the 126 MB
+# of L2 (config B: 4.7 MB of rows per instance; config C: 190 MB).
+EXTRA_CONFIGS = {"hca_decode_128k": 32, "csa_decode_128k": 2}
+
+
+def hbm_summary(wl, ms_per_step, peak):
+    """tok/s, algorithmic bytes and HBM fraction of one decode step of every layer of wl."""
+    b = sum(step_bytes(L, wl.n, wl.B) for L in wl.layers)
+    gbs = b / (ms_per_step / 1e3) / 1e9
+    return {"tok_s": wl.B * len(wl.layers) / (ms_per_step / 1e3), "us_per_step": 1e3 * ms_per_step,
+            "algorithmic_bytes": b, "achieved_gbs": gbs, "hbm_frac": gbs / peak}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    from csa_synth import decode_inputs, get_workload
+    from csa_synth import get_workload
     from long_context_sparse_csa_b200 import binding as C
-    from long_context_sparse_csa_b200.state import LayerState, to_device
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -295,125 +452,50 @@ def run_ours(args):
     wl = get_workload(args.workload)
     R = max(1, args.replicas)
     dev = torch.device("cuda", local)
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, peak_note = float(json.load(f)["hbm_gbs"]), "of measured"
+    except (OSError, KeyError, ValueError):
+        peak, peak_note = 6650.0, "of fallback"
 
-    datas, layers = [], []
-    for li, spec in enumerate(wl.layers):
-        d = decode_inputs(wl, li)
-        datas.append(d)
-        base = LayerState.from_arrays(spec, wl.B, d, device=dev)
-        insts = [base]
-        for _ in range(R - 1):
-            insts.append(LayerState(spec, wl.B, 0, entries=base.entries.clone(), window=base.window.clone(),
-                                    raw=base.raw.clone(), gate=base.gate.clone(),
-                                    idx_keys=None if base.idx_keys is None else base.idx_keys.clone(),
-                                    idx_key_scale=None if base.idx_key_scale is None else base.idx_key_scale.clone(),
-                                    pos_bias=base.pos_bias, gamma_kv=base.gamma_kv, gamma_q=base.gamma_q,
-                                    sinks=base.sinks))
-        cap = d["entries"].shape[1]
-        io = {k: to_device(d[k], dev) for k in ["q", "x_new", "g_new", "t"]}
-        if spec.kind == "csa":
-            for k in ["idx_q", "idx_q_scale", "head_w"]:
-                io[k] = to_device(d[k], dev)
-            io["topk"] = torch.zeros((wl.B, spec.top_k), dtype=torch.int32, device=dev)
-        io["out"] = torch.zeros((wl.B, spec.H, spec.D), dtype=torch.int16 if spec.act_format == "bf16" else torch.float32,
-                                device=dev)
-        ws = base.workspace("decode_step", 1, cap)
-        layers.append({"spec": spec, "insts": insts, "io": io, "ws": ws,
-                       "caches": [s.cache() for s in insts], "params": base.params(), "L": base.L})
-
-    def run_step(r):
-        for li, lay in enumerate(layers):
-            io, spec = lay["io"], lay["spec"]
-            if spec.kind == "csa":
-                C.csa_decode_step(lay["L"], lay["caches"][r], lay["params"], io["q"], io["idx_q"], io["idx_q_scale"],
-                                  io["head_w"], io["x_new"], io["g_new"], io["t"], io["out"], io["topk"], lay["ws"])
-            else:
-                C.hca_decode_step(lay["L"], lay["caches"][r], lay["params"], io["q"], io["x_new"], io["g_new"],
-                                  io["t"], io["out"], lay["ws"])
-
-    # eager warm-up of every instance (module load, attributes), then one graph per instance
-    for r in range(R):
-        run_step(r)
-    torch.cuda.synchronize()
-    for lay in layers:
-        assert C.csa_device_error(lay["ws"]) == 0
+    rig = DecodeRig(wl, R, dev)
+    layers, datas = rig.layers, rig.datas
+    rig.warm()
+    all_li = list(range(len(layers)))
     has_csa = any(l["spec"].kind == "csa" for l in layers)
-    ev = lambda: torch.cuda.Event(enable_timing=True, external=True)  # noqa: E731
-    stream = torch.cuda.Stream(device=dev)
-
-    def capture(rs, idx_events):
-        """One CUDA graph running the steps of instances rs in order.  With idx_events, a pair of
-        events brackets the indexer-score launch of the first step (the only event nodes: each one
-        breaks the chain of kernel nodes and costs a few microseconds)."""
-        pair = None
-        if idx_events:
-            pair = (ev(), ev())
-            for x in pair:
-                x.record()
-            torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        n0 = C.csa_launch_count()
-        with torch.cuda.graph(g, stream=stream):
-            for j, r in enumerate(rs):
-                for li, lay in enumerate(layers):
-                    io, spec = lay["io"], lay["spec"]
-                    if spec.kind == "csa":
-                        if idx_events and j == 0:
-                            C.csa_profile_events(*pair)
-                        C.csa_decode_step(lay["L"], lay["caches"][r], lay["params"], io["q"], io["idx_q"],
-                                          io["idx_q_scale"], io["head_w"], io["x_new"], io["g_new"], io["t"],
-                                          io["out"], io["topk"], lay["ws"])
-                        C.csa_profile_events(None, None)
-                    else:
-                        C.hca_decode_step(lay["L"], lay["caches"][r], lay["params"], io["q"], io["x_new"],
-                                          io["g_new"], io["t"], io["out"], lay["ws"])
-        return g, pair, C.csa_launch_count() - n0
-
-    # n_cyc copies of the cycle graph, replayed round-robin: the last replay of each copy lies in the
-    # timed region, so its event pair samples one indexer launch of the timed steps
-    n_cyc = max(1, min(8, args.steps // R))
-    cycles = [capture(list(range(R)), has_csa) for _ in range(n_cyc)]
-    launches_per_step = cycles[0][2] // R
-    singles = [capture([r], False)[0] for r in range(R)]
+    cycles, singles, launches_per_step = rig.graphs(all_li, args.steps, idx_events=has_csa)
     torch.cuda.synchronize()
 
-    def run_steps(k):
-        """Exactly k decode steps: whole cycles of the R instances, then single steps."""
-        for c in range(k // R):
-            cycles[c % n_cyc][0].replay()
-        for r in range(k % R):
-            singles[r].replay()
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    cur = torch.cuda.current_stream()
     clocks = ClockSampler(local)
     clocks.start()
     # warm-up: W steps, plus a short burn so clocks settle at load before the timed region
-    run_steps(args.warmup)
+    run_steps(cycles, singles, R, args.warmup)
     t_burn = time.perf_counter()
     while time.perf_counter() - t_burn < args.burn_seconds:
         cycles[0][0].replay()
         torch.cuda.synchronize()
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks.sample()
     w0 = time.perf_counter()
-    e0.record(cur)
-    run_steps(args.steps)
-    e1.record(cur)
-    torch.cuda.synchronize()
+    T_ms = timed(lambda: run_steps(cycles, singles, R, args.steps), world, dist, dev)
     w1 = time.perf_counter()
     clocks.sample()
-    barrier()
-    T_ms = max_over_ranks(e0.elapsed_time(e1), world, dist, dev)
     clk = clocks.summary(w0, w1)
     # indexer launch durations sampled inside the timed region (one per cycle-graph copy)
     idx_ms = [c[1][0].elapsed_time(c[1][1]) for c in cycles] if has_csa else []
+
+    # ------------------------------------------------------------------ each layer on its own (timed the same way)
+    per_layer = {}
+    if len(layers) > 1:
+        for li, lay in enumerate(layers):
+            cy, si, _ = rig.graphs([li], args.steps)
+            run_steps(cy, si, R, args.warmup)
+            ms = timed(lambda: run_steps(cy, si, R, args.steps), world, dist, dev) / args.steps
+            spec = lay["spec"]
+            b = step_bytes(spec, wl.n, wl.B)
+            per_layer[f"{spec.kind}{li}"] = {"us_per_step": 1e3 * ms, "tok_s": wl.B / (ms / 1e3),
+                                             "algorithmic_bytes": b, "achieved_gbs": b / (ms / 1e3) / 1e9,
+                                             "hbm_frac": b / (ms / 1e3) / 1e9 / peak}
+            del cy, si
 
     # ------------------------------------------------------------------ per-kernel timeline (diagnostic, untimed)
     # launch order of the sequential (diagnostic) step: the second stream is off while it is timed
@@ -422,22 +504,16 @@ def run_ours(args):
     tl_events = []
     g_tl = torch.cuda.CUDAGraph()
     for lay in layers:
-        evs = [ev() for _ in range(17)]
+        evs = [_ext_event() for _ in range(17)]
         for x in evs:
             x.record()
         tl_events.append(evs)
     torch.cuda.synchronize()
-    with torch.cuda.graph(g_tl, stream=stream):
+    with torch.cuda.graph(g_tl, stream=rig.stream):
         for li, lay in enumerate(layers):
-            io, spec = lay["io"], lay["spec"]
             evs = tl_events[li]
             C.csa_profile_timeline(evs[:16])
-            if spec.kind == "csa":
-                C.csa_decode_step(lay["L"], lay["caches"][0], lay["params"], io["q"], io["idx_q"], io["idx_q_scale"],
-                                  io["head_w"], io["x_new"], io["g_new"], io["t"], io["out"], io["topk"], lay["ws"])
-            else:
-                C.hca_decode_step(lay["L"], lay["caches"][0], lay["params"], io["q"], io["x_new"], io["g_new"],
-                                  io["t"], io["out"], lay["ws"])
+            rig.call(li, 0)
             lay["tl_n"] = C.csa_profile_timeline_count()
             C.csa_profile_timeline(None)
             evs[lay["tl_n"]].record()
@@ -468,27 +544,17 @@ def run_ours(args):
         d2h.append((o, torch.empty(o.shape, dtype=o.dtype, pin_memory=True)))
     h2d_bytes = sum(h.numel() * h.element_size() for h, _ in h2d)
     d2h_bytes = sum(h.numel() * h.element_size() for _, h in d2h)
-    for s in range(args.warmup):
-        for h, dv in h2d:
-            dv.copy_(h, non_blocking=True)
-        singles[s % R].replay()
-        for dv, h in d2h:
-            h.copy_(dv, non_blocking=True)
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(cur)
-    for s in range(args.steps):
-        for h, dv in h2d:
-            dv.copy_(h, non_blocking=True)
-        singles[s % R].replay()
-        for dv, h in d2h:
-            h.copy_(dv, non_blocking=True)
-    f1.record(cur)
-    torch.cuda.synchronize()
-    barrier()
-    E_ms = max_over_ranks(f0.elapsed_time(f1), world, dist, dev)
+
+    def e2e_steps(k):
+        for s in range(k):
+            for h, dv in h2d:
+                dv.copy_(h, non_blocking=True)
+            singles[s % R].replay()
+            for dv, h in d2h:
+                h.copy_(dv, non_blocking=True)
+
+    e2e_steps(args.warmup)
+    E_ms = timed(lambda: e2e_steps(args.steps), world, dist, dev)
     clocks.stop()
 
     for lay in layers:
@@ -502,13 +568,6 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": T_ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e4m3+bf16 (fp32 accumulate)", "data": "synthetic",
             "config": workload_config(wl, R)}
-    peaks = {}
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peaks = json.load(f)
-        peak, peak_note = float(peaks["hbm_gbs"]), "of measured"
-    except (OSError, KeyError, ValueError):
-        peak, peak_note = 6650.0, "of fallback"
     if has_csa:
         csa_li = [i for i, l in enumerate(layers) if l["spec"].kind == "csa"][0]
         spec = layers[csa_li]["spec"]
@@ -530,20 +589,37 @@ def run_ours(args):
     step_alg = sum(step_bytes(l["spec"], wl.n, wl.B) for l in layers)
     line["step_hbm"] = {"algorithmic_bytes": step_alg, "achieved_gbs": step_alg / (T_ms / args.steps / 1e3) / 1e9,
                         "frac": step_alg / (T_ms / args.steps / 1e3) / 1e9 / peak}
+    if per_layer:
+        line["layers"] = per_layer
     line["e2e"] = {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                    "ms_per_step": E_ms / args.steps}
     line["gpu_launches"] = int(launches_per_step) * args.steps
     line["timeline_us"] = timeline
     line["clocks"] = clk
+    del cycles, singles
+
+    # ------------------------------------------------------------------ the 128K configurations
+    if args.workload == "csa_hca_decode_1m" and not args.no_extra_configs:
+        extra = {}
+        for name, r_extra in EXTRA_CONFIGS.items():
+            wl2 = get_workload(name)
+            rig2 = DecodeRig(wl2, r_extra, dev)
+            rig2.warm()
+            cy, si, _ = rig2.graphs(list(range(len(rig2.layers))), args.steps)
+            run_steps(cy, si, r_extra, args.warmup)
+            ms = timed(lambda: run_steps(cy, si, r_extra, args.steps), world, dist, dev) / args.steps
+            for lay in rig2.layers:
+                assert C.csa_device_error(lay["ws"]) == 0
+            extra[name] = dict(hbm_summary(wl2, ms, peak), batch=wl2.B, context=wl2.n,
+                               l2=f"rotating {r_extra} instances (inputs larger than L2)")
+            del cy, si, rig2
+            torch.cuda.empty_cache()
+        line["configs"] = extra
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        times = run_cpu_oracle(wl, datas, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": wl.B * len(layers) / float(np.mean(times)), "unit": UNIT,
-                                "cores": cpu_threads(), "kind": "oracle",
-                                "sample": f"{len(times)} full decode steps of the workload ({args.cpu_seconds:.0f} s budget)"}
+        line["cpu_baseline"] = cpu_baseline(wl, datas, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del cycles, singles
     if world > 1:
         dist.destroy_process_group()
 

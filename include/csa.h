@@ -56,6 +56,18 @@
  *                 max|x| / sigma <= 448 (1 for an all-zero part), codes are
  *                 round-to-nearest-even with saturation.
  *
+ * Index-key formats (idx_format), one key of d_I dims per entry:
+ *   CSA_FMT_F32   d_I float32, idx_key_scale all 1.
+ *   CSA_FMT_E4M3  d_I e4m3 codes; idx_key_scale[i] = the key's power-of-two scale.
+ *   CSA_FMT_E2M1  d_I / 2 bytes of FP4 e2m1 codes (1 sign, 2 exponent bits with bias 1, 1 mantissa
+ *                 bit; magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6), two per byte with the even dim in the
+ *                 low nibble; idx_key_scale[i] holds a uint32 scale word (stored in the float
+ *                 array's 4 bytes): bits 0..7 = e + 127 for the key scale sigma = 2^e, bits
+ *                 8+4b..11+4b = the offset delta_b (0..7) of dims [32b, 32b+32); the value of dim d
+ *                 is code * sigma * 2^-delta_b.  d_I a multiple of 32.  Index queries stay e4m3.
+ *                 ("DeepSeek-V4: Making a Million Tokens Affordable", "Two ways to shrink
+ *                 attention, interleaved": the indexer's attention runs in FP4.)
+ *
  * Rotary convention: interleaved pairs (D-64+2u, D-64+2u+1), u < 32, angle
  * pos * base^(-2u/64) formed and reduced in float64.
  */
@@ -88,7 +100,8 @@ enum {
   CSA_FMT_F32 = 0,
   CSA_FMT_BF16 = 1,
   CSA_FMT_MIXED = 2,           /* kv_format only */
-  CSA_FMT_E4M3 = 3             /* idx_format only */
+  CSA_FMT_E4M3 = 3,            /* idx_format only */
+  CSA_FMT_E2M1 = 4             /* idx_format only: FP4 index keys, e4m3 index queries (see below) */
 };
 
 enum { CSA_KIND_CSA = 0, CSA_KIND_HCA = 1 };
@@ -107,7 +120,7 @@ typedef struct csa_layer {
   int32_t H_I;           /* CSA: indexer heads */
   int32_t d_I;           /* CSA: indexer head dim */
   int32_t kv_format;     /* CSA_FMT_F32 | CSA_FMT_BF16 | CSA_FMT_MIXED */
-  int32_t idx_format;    /* CSA_FMT_F32 | CSA_FMT_E4M3 (index keys and index queries) */
+  int32_t idx_format;    /* CSA_FMT_F32 | CSA_FMT_E4M3 | CSA_FMT_E2M1 (index keys; queries e4m3 for E2M1) */
   int32_t act_format;    /* CSA_FMT_F32 | CSA_FMT_BF16: queries, raw rows, gate logits, output */
   double rope_base;      /* rotary base (10000) */
   float eps;             /* RMSNorm epsilon (1e-6) */
@@ -143,8 +156,18 @@ enum {
   CSA_OP_SPARSE_ATTEND = 1,
   CSA_OP_HCA_ATTEND = 2,
   CSA_OP_DECODE_STEP = 3,   /* csa_decode_step / hca_decode_step */
-  CSA_OP_PREFILL = 4        /* csa_prefill */
+  CSA_OP_PREFILL = 4,       /* csa_prefill */
+  CSA_OP_DECODE_STEP_INDEXED = 5  /* csa_decode_step_indexed */
 };
+
+/* Index-key stream of a CSA layer: per token one index row and one row of gate logits of d_I
+ * values (act_format), kept in rings with the same slots as cache->raw / cache->gate
+ * (row r at slot (r - raw_base) mod raw_cap), and the slot biases of their compression. */
+typedef struct csa_index_stream {
+  void* raw;              /* [B][raw_cap][d_I] index rows */
+  void* gate;             /* [B][raw_cap][d_I] gate logits */
+  const float* pos_bias;  /* [(1+overlap)*m][d_I] positional bias per window slot and channel */
+} csa_index_stream_t;
 
 /* Bytes of one stored row for the layer's kv_format (host). */
 CSA_API size_t csa_row_bytes(const csa_layer_t* L);
@@ -159,13 +182,46 @@ CSA_API const char* csa_last_error(void);
 /* Library version string (host). */
 CSA_API const char* csa_version(void);
 
-/* Reads and clears the workspace's device error word (synchronises the
- * stream).  *code gets the bits kernels set (0 = none):
- *   1  a bounded wait (mbarrier / tensor-memory pipeline) gave up;
+/* Reads and clears the device error words (synchronises the stream): the
+ * workspace's word (workspace may be NULL: then it is skipped) and the
+ * library's own word on the current device, where the kernels of the calls
+ * that take no workspace (csa_append, csa_compress) report.  *code gets the
+ * OR of the bits kernels set (0 = none):
+ *   1  a bounded wait (mbarrier / tensor-memory pipeline / cluster
+ *      reduction) gave up; the results of that launch are incomplete;
  *   2  the multi-CTA top-k found its score histogram inconsistent with the
  *      scores; that row's top-k output is incomplete (padded with -1).
  * Returns CSA_ERR_DEVICE_TIMEOUT if any bit was set. */
 CSA_API csa_status_t csa_device_error(void* workspace, size_t ws_bytes, void* stream, int32_t* code);
+
+/* Test and diagnostic aids (no counterpart on the pages). */
+
+/* Workspace segments, for csa_debug_workspace_segment. */
+enum {
+  CSA_SEG_ERROR_WORD = 0,      /* the int32 device error word */
+  CSA_SEG_SCORES = 1,          /* indexer scores [rows][entry_cap] float32 */
+  CSA_SEG_TOPK_HISTOGRAM = 2,  /* multi-CTA top-k: [rows][4096] uint32 score histogram, then
+                                  [rows][4] counters, then [rows][4096] second histogram */
+  CSA_SEG_TOPK = 3,            /* top-k indices of the fused calls [rows][top_k] int32 */
+  CSA_SEG_PARTIALS = 4,        /* attention partials */
+  CSA_SEG_INDEX_QUERY = 5,     /* csa_decode_step_indexed: the produced index query [B][H_I][d_I] */
+  CSA_SEG_INDEX_QUERY_SCALE = 6  /* ... and its per-head scales [B][H_I] float32 */
+};
+
+/* Byte offset and size of one segment of the workspace that
+ * csa_workspace_size(L, op, Tq, entry_cap) describes (host; *bytes = 0 when
+ * the operation has no such segment).  Lets a test inject state (e.g. an
+ * inconsistent score histogram) into a caller-owned workspace. */
+CSA_API csa_status_t csa_debug_workspace_segment(const csa_layer_t* L, int32_t op, int32_t Tq, int64_t entry_cap,
+                                                 int32_t segment, size_t* offset, size_t* bytes);
+
+/* Launches one CTA that waits, with the library's bounded wait and a limit
+ * of limit_ns nanoseconds (0 < limit_ns <= 1e9), on an mbarrier phase that
+ * nothing completes; when the limit passes it sets bit 1 of the workspace's
+ * error word and returns.  Nothing is in flight in the CTA when it gives up,
+ * so the context stays usable.  Lets a test drive the failure-reporting path
+ * (csa_device_error -> CSA_ERR_DEVICE_TIMEOUT) without a device fault. */
+CSA_API csa_status_t csa_debug_wait_probe(void* workspace, size_t ws_bytes, uint64_t limit_ns, void* stream);
 
 /* Profiling aid (no counterpart on the pages).  When ev_start and ev_stop (cudaEvent_t handles
  * created with timing enabled) are both non-NULL, every later call made from this host thread
@@ -276,6 +332,40 @@ CSA_API csa_status_t csa_decode_step(const csa_layer_t* L, const csa_cache_t* ca
                              void* out, int32_t* topk_idx,
                              void* workspace, size_t ws_bytes, void* stream);
 
+/* Index keys produced from the index-key stream.  Appends the Tq tokens' index rows x_new / g_new
+ * ([B][Tq][d_I] act_format; both NULL when the rows are already in S->raw / S->gate) to the stream's
+ * rings, then writes the key of every entry the tokens complete: the entry's window rows
+ * [(i-ov)m, (i+1)m) clipped at 0 pooled with a per-channel softmax of gate + S->pos_bias[slot], no
+ * RMSNorm, no rotation, into cache->idx_keys[b][i] (e4m3 codes of k / sigma with sigma the smallest
+ * power of two with max|k| / sigma <= 448, into cache->idx_key_scale[b][i]; float32 keys get scale 1).
+ * Reading of the pages: the lightning indexer scores the compressed entries "in a low-rank way"
+ * ("DeepSeek-V4 Explained: ...", "The attention stack, and why it is two mechanisms"); its keys are
+ * read as compressed like the entries themselves.  Needs d_I a multiple of 32, <= 128. */
+CSA_API csa_status_t csa_index_keys(const csa_layer_t* L, const csa_cache_t* cache, const csa_index_stream_t* S,
+                                    const void* x_new, const void* g_new, const int64_t* q_pos, int32_t Tq,
+                                    void* stream);
+
+/* Low-rank index queries: for each of `rows` query tokens, q_h = W_h c with c [rows][rank] (bf16,
+ * the query's low-rank latent) and W [H_I * d_I][rank] (bf16, row h*d_I + d of W is output dim d of
+ * head h), stored as idx_q [rows][H_I][d_I] e4m3 codes of q_h / sigma_h with idx_q_scale
+ * [rows][H_I] the per-head power-of-two scale (the same rule as the keys), or float32 values with
+ * scale 1.  rank a multiple of 16; d_I a multiple of 32, <= 128.  Same page and section (a low-rank
+ * indexer); the up-projection of a latent is this library's reading of it. */
+CSA_API csa_status_t csa_index_query(const csa_layer_t* L, const void* c, const void* W, int32_t rank,
+                                     int32_t rows, void* idx_q, float* idx_q_scale, void* stream);
+
+/* csa_decode_step with the index side produced in the step: csa_index_keys for the token (its
+ * index row idx_x_new / idx_g_new [B][d_I]) and csa_index_query from its latent c [B][rank] run
+ * first, on `stream`, and the indexer then scores the keys and queries they wrote (the index query
+ * lives in the workspace of CSA_OP_DECODE_STEP_INDEXED).  Other arguments as csa_decode_step. */
+CSA_API csa_status_t csa_decode_step_indexed(const csa_layer_t* L, const csa_cache_t* cache,
+                                             const csa_params_t* P, const csa_index_stream_t* S,
+                                             const void* q, const void* c, const void* W, int32_t rank,
+                                             const float* head_w, const void* x_new, const void* g_new,
+                                             const void* idx_x_new, const void* idx_g_new,
+                                             const int64_t* q_pos, void* out, int32_t* topk_idx,
+                                             void* workspace, size_t ws_bytes, void* stream);
+
 /* Bytes of the static device scratch used by csa_decode_step_scratch. */
 #define CSA_SCRATCH_BYTES ((size_t)16 << 20)
 
@@ -296,7 +386,15 @@ CSA_API csa_status_t csa_decode_step(const csa_layer_t* L, const csa_cache_t* ca
  *   - device_error: NULL, or a host int32 that receives the device error word
  *     (see csa_device_error); non-NULL synchronises the stream (not allowed
  *     during stream capture) and, when the word is non-zero, zero-fills the
- *     scratch again and returns CSA_ERR_DEVICE_TIMEOUT.
+ *     scratch again and returns CSA_ERR_DEVICE_TIMEOUT.  A call with NULL
+ *     leaves any bits its kernels set in the scratch's word: the next call
+ *     with a non-NULL device_error reports them (with its own), so after
+ *     NULL calls that report covers every call since the last non-NULL one.
+ *   - After a device error the scratch's histograms may be left non-zero.
+ *     Every call therefore starts with a small guard kernel that, when the
+ *     scratch's error word is set, zero-fills the scratch's top-k histograms
+ *     and counters (keeping the word), so later calls, NULL or not, select
+ *     from clean histograms.
  * Other arguments, layouts and errors as csa_decode_step. */
 CSA_API csa_status_t csa_decode_step_scratch(const csa_layer_t* L, const csa_cache_t* cache,
                              const csa_params_t* P, const void* q,

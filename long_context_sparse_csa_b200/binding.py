@@ -15,9 +15,11 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libcsa.so")
 
-FMT = {"f32": 0, "bf16": 1, "mixed": 2, "e4m3": 3}
+FMT = {"f32": 0, "bf16": 1, "mixed": 2, "e4m3": 3, "e2m1": 4}
+SEGMENT = {"error_word": 0, "scores": 1, "topk_histogram": 2, "topk": 3, "partials": 4, "index_query": 5,
+           "index_query_scale": 6}
 KIND = {"csa": 0, "hca": 1}
-OP = {"index_topk": 0, "sparse_attend": 1, "hca_attend": 2, "decode_step": 3, "prefill": 4}
+OP = {"index_topk": 0, "sparse_attend": 1, "hca_attend": 2, "decode_step": 3, "prefill": 4, "decode_step_indexed": 5}
 STATUS = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED", 3: "CSA_ERR_WORKSPACE",
           4: "CSA_ERR_CUDA", 5: "CSA_ERR_DEVICE_TIMEOUT"}
 
@@ -49,7 +51,12 @@ class CsaParams(ctypes.Structure):
                 ("sinks", ctypes.c_void_p)]
 
 
+class CsaIndexStream(ctypes.Structure):
+    _fields_ = [("raw", ctypes.c_void_p), ("gate", ctypes.c_void_p), ("pos_bias", ctypes.c_void_p)]
+
+
 _P = ctypes.c_void_p
+_STREAM_S = ctypes.POINTER(CsaIndexStream)
 _LAYER = ctypes.POINTER(CsaLayer)
 _CACHE = ctypes.POINTER(CsaCache)
 _PARAMS = ctypes.POINTER(CsaParams)
@@ -75,6 +82,13 @@ _SIGS = {
     "csa_decode_step_scratch": (ctypes.c_int, [_LAYER, _CACHE, _PARAMS, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                                ctypes.POINTER(_I32), _P]),
     "csa_prefill": (ctypes.c_int, [_LAYER, _CACHE, _PARAMS, _P, _P, _P, _P, _P, _I32, _I64, _P, _P, _P, _SZ, _P]),
+    "csa_debug_workspace_segment": (ctypes.c_int, [_LAYER, _I32, _I32, _I64, _I32, ctypes.POINTER(_SZ),
+                                                   ctypes.POINTER(_SZ)]),
+    "csa_debug_wait_probe": (ctypes.c_int, [_P, _SZ, ctypes.c_uint64, _P]),
+    "csa_index_keys": (ctypes.c_int, [_LAYER, _CACHE, _STREAM_S, _P, _P, _P, _I32, _P]),
+    "csa_index_query": (ctypes.c_int, [_LAYER, _P, _P, _I32, _I32, _P, _P, _P]),
+    "csa_decode_step_indexed": (ctypes.c_int, [_LAYER, _CACHE, _PARAMS, _STREAM_S, _P, _P, _P, _I32, _P, _P, _P, _P,
+                                               _P, _P, _P, _P, _P, _SZ, _P]),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -136,6 +150,11 @@ def make_cache(entries, window, raw=None, gate=None, idx_keys=None, idx_key_scal
                     gate.data_ptr() if gate is not None else None, raw.shape[1] if raw is not None else 0, raw_base)
 
 
+def make_index_stream(raw, gate, pos_bias) -> CsaIndexStream:
+    """Index-key stream struct over rings [B, raw_cap, d_I] and the slot biases [(1+ov)m, d_I]."""
+    return CsaIndexStream(raw.data_ptr(), gate.data_ptr(), pos_bias.data_ptr())
+
+
 def make_params(pos_bias=None, gamma_kv=None, gamma_q=None, sinks=None) -> CsaParams:
     g = lambda t: t.data_ptr() if t is not None else None  # noqa: E731
     return CsaParams(g(pos_bias), g(gamma_kv), g(gamma_q), g(sinks))
@@ -188,12 +207,27 @@ def csa_launch_count() -> int:
 
 
 def csa_device_error(workspace, stream=None) -> int:
+    """OR of the workspace's error word (None: skipped) and the library's own word; both cleared."""
     code = _I32(0)
-    st = lib().csa_device_error(ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream),
-                                ctypes.byref(code))
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().csa_device_error(ptr(workspace), nbytes, _stream(stream), ctypes.byref(code))
     if st not in (0, 5):
         _check(st)
     return code.value
+
+
+def csa_debug_workspace_segment(L, op, Tq, entry_cap, segment):
+    """(byte offset, bytes) of a workspace segment (test aid)."""
+    off, nb = _SZ(0), _SZ(0)
+    _check(lib().csa_debug_workspace_segment(ctypes.byref(L), OP[op], Tq, entry_cap, SEGMENT[segment],
+                                             ctypes.byref(off), ctypes.byref(nb)))
+    return off.value, nb.value
+
+
+def csa_debug_wait_probe(workspace, limit_ns, stream=None):
+    """Launch the bounded-wait probe: its wait runs out after limit_ns and sets the error word (test aid)."""
+    _check(lib().csa_debug_wait_probe(ptr(workspace), workspace.numel() * workspace.element_size(), int(limit_ns),
+                                      _stream(stream)))
 
 
 def csa_append(L, cache, x_new, g_new, q_pos, Tq, stream=None):
@@ -256,3 +290,22 @@ def csa_prefill(L, cache, params, q, idx_q, idx_q_scale, head_w, q_pos, Tq, n_ma
     _check(lib().csa_prefill(ctypes.byref(L), ctypes.byref(cache), ctypes.byref(params), ptr(q), ptr(idx_q),
                              ptr(idx_q_scale), ptr(head_w), ptr(q_pos), Tq, n_max, ptr(out), ptr(topk_idx),
                              ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def csa_index_keys(L, cache, index_stream, x_new, g_new, q_pos, Tq, stream=None):
+    _check(lib().csa_index_keys(ctypes.byref(L), ctypes.byref(cache), ctypes.byref(index_stream), ptr(x_new),
+                                ptr(g_new), ptr(q_pos), Tq, _stream(stream)))
+
+
+def csa_index_query(L, c, W, rank, rows, idx_q, idx_q_scale, stream=None):
+    _check(lib().csa_index_query(ctypes.byref(L), ptr(c), ptr(W), rank, rows, ptr(idx_q), ptr(idx_q_scale),
+                                 _stream(stream)))
+
+
+def csa_decode_step_indexed(L, cache, params, index_stream, q, c, W, rank, head_w, x_new, g_new, idx_x_new,
+                            idx_g_new, q_pos, out, topk_idx, workspace, stream=None):
+    _check(lib().csa_decode_step_indexed(ctypes.byref(L), ctypes.byref(cache), ctypes.byref(params),
+                                         ctypes.byref(index_stream), ptr(q), ptr(c), ptr(W), rank, ptr(head_w),
+                                         ptr(x_new), ptr(g_new), ptr(idx_x_new), ptr(idx_g_new), ptr(q_pos), ptr(out),
+                                         ptr(topk_idx), ptr(workspace), workspace.numel() * workspace.element_size(),
+                                         _stream(stream)))

@@ -3,8 +3,8 @@
 Usage: python -m long_context_sparse_csa_b200.build [--force] [--trace]
 
 --trace builds libcsa_trace.so instead: the same kernels with CSA_TRACE defined, so they record
-per-CTA timestamps that `python -m long_context_sparse_csa_b200.diag_trace` reads (diagnostics only;
-the product library never has them).
+per-CTA %globaltimer stamps into device arrays that the csa_trace_read* symbols of that library copy
+out (a diagnostic build; the product library never has them).
 """
 
 import os
@@ -19,7 +19,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libcsa.so")
 TRACE_LIB = os.path.join(HERE, "libcsa_trace.so")
 
-SOURCES = ["compress.cu", "index_score.cu", "topk.cu", "attend.cu", "api.cu", "static_scratch.cu"]
+SOURCES = ["compress.cu", "index_score.cu", "topk.cu", "attend.cu", "api.cu", "static_scratch.cu", "debug.cu", "index_decode.cu", "index_prep.cu"]
 HEADERS = ["common.cuh", "sm100.cuh", "kernels.h"]
 
 NVCC_FLAGS = [

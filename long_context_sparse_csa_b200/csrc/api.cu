@@ -4,7 +4,10 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
+#include <mutex>
 #include <string>
+#include <utility>
 
 #include "csa.h"
 #include "kernels.h"
@@ -110,9 +113,11 @@ csa_status_t check_layer(const csa_layer_t* L) {
   if (L->kind == CSA_KIND_CSA) {
     if (L->top_k < 1) return fail(CSA_ERR_INVALID_ARG, "top_k=%d", L->top_k);
     if (L->H_I < 1 || L->d_I < 1) return fail(CSA_ERR_INVALID_ARG, "H_I=%d d_I=%d", L->H_I, L->d_I);
-    if (L->idx_format != CSA_FMT_F32 && L->idx_format != CSA_FMT_E4M3)
+    if (L->idx_format != CSA_FMT_F32 && L->idx_format != CSA_FMT_E4M3 && L->idx_format != CSA_FMT_E2M1)
       return fail(CSA_ERR_INVALID_ARG, "idx_format=%d", L->idx_format);
     if (L->d_I % 16) return fail(CSA_ERR_UNSUPPORTED, "d_I=%d (needs a multiple of 16)", L->d_I);
+    if (L->idx_format == CSA_FMT_E2M1 && L->d_I % 32)
+      return fail(CSA_ERR_UNSUPPORTED, "d_I=%d (FP4 keys need a multiple of 32)", L->d_I);
     if ((size_t)L->H_I * L->d_I * 4 > 96 * 1024) return fail(CSA_ERR_UNSUPPORTED, "H_I*d_I too large");
   }
   return CSA_OK;
@@ -180,10 +185,10 @@ csa_status_t check_cache_raw(const csa_layer_t* L, const csa_cache_t* c, bool ne
 // ----------------------------------------------------------------------------- workspace layout
 constexpr size_t kAlign = 256;
 
-// Long decode rows take the multi-CTA top-k, fed by the tensor-core indexer's histogram.
+// Long decode rows take the multi-CTA top-k, fed by the decode indexer's score histogram.
 bool use_split_topk(const csa_layer_t* L, int32_t Tq, int64_t n_max) {
   return Tq == 1 && n_max >= kTopkSplitMinN && n_max <= kTopkSplitMaxN &&
-         index_tc_supported(L->idx_format, L->H_I, L->d_I);
+         index_decode_supported(L->idx_format, L->H_I, L->d_I);
 }
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -195,6 +200,7 @@ struct Workspace {
   size_t topk = 0, topk_bytes = 0;
   size_t part = 0, part_bytes = 0;
   size_t qt = 0;                        // bf16 q~ of the tcgen05 attention [rows][H][D]
+  size_t idxq = 0, idxqs = 0;           // indexed decode step: produced index query and its scales
   size_t total = 0;
 };
 
@@ -204,7 +210,8 @@ Workspace layout(const csa_layer_t* L, int op, int32_t Tq, int64_t n_max) {
   const size_t rows = (size_t)L->B * (size_t)(Tq > 0 ? Tq : 1);
   size_t off = up(64);
   const bool csa = L->kind == CSA_KIND_CSA;
-  if (csa && (op == CSA_OP_INDEX_TOPK || op == CSA_OP_DECODE_STEP || op == CSA_OP_PREFILL)) {
+  const bool step = op == CSA_OP_DECODE_STEP || op == CSA_OP_DECODE_STEP_INDEXED;
+  if (csa && (op == CSA_OP_INDEX_TOPK || step || op == CSA_OP_PREFILL)) {
     w.scores = off; w.scores_bytes = rows * (size_t)(n_max > 0 ? n_max : 1) * 4; off = up(off + w.scores_bytes);
     if (use_split_topk(L, Tq, n_max)) {
       w.hist = off; w.hist_bytes = rows * (4096 + 4 + 4096) * 4; off = up(off + w.hist_bytes);
@@ -212,10 +219,15 @@ Workspace layout(const csa_layer_t* L, int op, int32_t Tq, int64_t n_max) {
       w.list = off; off = up(off + rows * (size_t)n_max * 8);
     }
   }
-  if (csa && (op == CSA_OP_DECODE_STEP || op == CSA_OP_PREFILL)) {
+  if (csa && (step || op == CSA_OP_PREFILL)) {
     w.topk = off; w.topk_bytes = rows * (size_t)L->top_k * 4; off = up(off + w.topk_bytes);
   }
-  if (op == CSA_OP_SPARSE_ATTEND || op == CSA_OP_HCA_ATTEND || op == CSA_OP_DECODE_STEP || op == CSA_OP_PREFILL) {
+  if (csa && op == CSA_OP_DECODE_STEP_INDEXED) {
+    const size_t qb = L->idx_format == CSA_FMT_F32 ? 4 : 1;
+    w.idxq = off; off = up(off + rows * (size_t)L->H_I * L->d_I * qb);
+    w.idxqs = off; off = up(off + rows * (size_t)L->H_I * 4);
+  }
+  if (op == CSA_OP_SPARSE_ATTEND || op == CSA_OP_HCA_ATTEND || step || op == CSA_OP_PREFILL) {
     const bool dense = (op == CSA_OP_HCA_ATTEND) || !csa;
     const int64_t slots = (dense ? (n_max > 0 ? n_max : 1) : (int64_t)L->top_k) + L->window;
     const int splits = attend_num_splits(la, dense, (int)rows, slots, num_sms());
@@ -238,7 +250,7 @@ uint8_t* at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
 // ----------------------------------------------------------------------------- step bodies
 csa_status_t run_append_compress(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P,
                                  const void* x_new, const void* g_new, const int64_t* q_pos, int32_t Tq,
-                                 bool do_append, bool do_compress, cudaStream_t s) {
+                                 bool do_append, bool do_compress, int* err, cudaStream_t s) {
   AppendCompressArgs a;
   a.L = layer_args(L);
   a.C = cache_args(cache);
@@ -250,6 +262,7 @@ csa_status_t run_append_compress(const csa_layer_t* L, const csa_cache_t* cache,
   a.gamma_kv = P ? P->gamma_kv : nullptr;
   a.do_append = do_append;
   a.do_compress = do_compress;
+  a.err = err;
   cudaError_t e = launch_append_compress(a, L->B, Tq, s);
   return e == cudaSuccess ? CSA_OK : cuda_fail(e, "append/compress launch");
 }
@@ -362,8 +375,45 @@ namespace csa {
 csa_status_t report_error(csa_status_t st, const char* msg) { return fail(st, "%s", msg); }
 
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+namespace {
+std::mutex g_attr_mu;
+std::map<std::pair<int, const void*>, size_t> g_smem_attr;     // (device, kernel) -> bytes set
+std::map<std::pair<int, const void*>, bool> g_cluster_attr;    // (device, kernel) -> allowed
+}  // namespace
+
+cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  size_t& have = g_smem_attr[std::make_pair(dev, kernel)];
+  if (bytes <= have) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) have = bytes;
+  return e;
+}
+
+cudaError_t ensure_nonportable_cluster(const void* kernel) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  bool& ok = g_cluster_attr[std::make_pair(dev, kernel)];
+  if (ok) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess) ok = true;
+  return e;
+}
 void profile_mark(cudaStream_t s) {
-  if (g_tl && g_tl_n < g_tl_cap) cudaEventRecordWithFlags(g_tl[g_tl_n++], s, cudaEventRecordExternal);
+  if (!g_tl || g_tl_n >= g_tl_cap) return;
+  // under stream capture the record becomes an event node (external flag); on a stream that is
+  // not being captured it is a plain record, ordered after the launches issued before it
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) cudaGetLastError();
+  if (cap == cudaStreamCaptureStatusActive) cudaEventRecordWithFlags(g_tl[g_tl_n++], s, cudaEventRecordExternal);
+  else cudaEventRecord(g_tl[g_tl_n++], s);
 }
 }  // namespace csa
 
@@ -397,16 +447,52 @@ void csa_profile_timeline(void** events, int32_t capacity) {
 int32_t csa_profile_timeline_count(void) { return g_tl_n; }
 
 csa_status_t csa_device_error(void* workspace, size_t ws_bytes, void* stream, int32_t* code) {
-  if (!workspace || ws_bytes < 4) return fail(CSA_ERR_WORKSPACE, "workspace is NULL");
+  if (code) *code = 0;
+  if (workspace && ws_bytes < 4) return fail(CSA_ERR_WORKSPACE, "workspace smaller than its error word");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int32_t v = 0;
-  cudaError_t e = cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, s);
+  int* lib_word = nullptr;
+  cudaError_t e = library_error_word(&lib_word);
+  int32_t v[2] = {0, 0};
+  if (e == cudaSuccess && workspace) e = cudaMemcpyAsync(&v[0], workspace, 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&v[1], lib_word, 4, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e == cudaSuccess && v) e = cudaMemsetAsync(workspace, 0, 4, s);
+  if (e == cudaSuccess && v[0]) e = cudaMemsetAsync(workspace, 0, 4, s);
+  if (e == cudaSuccess && v[1]) e = cudaMemsetAsync(lib_word, 0, 4, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "csa_device_error");
-  if (code) *code = v;
-  return v ? fail(CSA_ERR_DEVICE_TIMEOUT, "device error word 0x%x", v) : CSA_OK;
+  const int32_t bits = v[0] | v[1];
+  if (code) *code = bits;
+  return bits ? fail(CSA_ERR_DEVICE_TIMEOUT, "device error word 0x%x", bits) : CSA_OK;
+}
+
+csa_status_t csa_debug_workspace_segment(const csa_layer_t* L, int32_t op, int32_t Tq, int64_t entry_cap,
+                                         int32_t segment, size_t* offset, size_t* bytes) {
+  CSA_TRY(check_layer(L));
+  if (!offset || !bytes) return fail(CSA_ERR_INVALID_ARG, "offset or bytes is NULL");
+  const Workspace w = layout(L, op, Tq, entry_cap);
+  *offset = 0;
+  *bytes = 0;
+  switch (segment) {
+    case CSA_SEG_ERROR_WORD: *offset = w.err; *bytes = 4; break;
+    case CSA_SEG_SCORES: *offset = w.scores; *bytes = w.scores_bytes; break;
+    case CSA_SEG_TOPK_HISTOGRAM: *offset = w.hist; *bytes = w.hist_bytes; break;
+    case CSA_SEG_TOPK: *offset = w.topk; *bytes = w.topk_bytes; break;
+    case CSA_SEG_PARTIALS: *offset = w.part; *bytes = w.part_bytes; break;
+    case CSA_SEG_INDEX_QUERY:
+      *offset = w.idxq;
+      *bytes = w.idxq ? (size_t)L->B * L->H_I * L->d_I * (L->idx_format == CSA_FMT_F32 ? 4 : 1) : 0;
+      break;
+    case CSA_SEG_INDEX_QUERY_SCALE: *offset = w.idxqs; *bytes = w.idxqs ? (size_t)L->B * L->H_I * 4 : 0; break;
+    default: return fail(CSA_ERR_INVALID_ARG, "segment %d", segment);
+  }
+  return CSA_OK;
+}
+
+csa_status_t csa_debug_wait_probe(void* workspace, size_t ws_bytes, uint64_t limit_ns, void* stream) {
+  if (!workspace || ws_bytes < 4) return fail(CSA_ERR_WORKSPACE, "workspace is NULL");
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return fail(CSA_ERR_INVALID_ARG, "limit_ns outside (0, 1e9]");
+  const cudaError_t e = launch_wait_probe(static_cast<int*>(workspace), limit_ns, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e, "wait probe launch");
 }
 
 csa_status_t csa_append(const csa_layer_t* L, const csa_cache_t* cache, const void* x_new, const void* g_new,
@@ -420,7 +506,11 @@ csa_status_t csa_append(const csa_layer_t* L, const csa_cache_t* cache, const vo
   if ((x_new == nullptr) != (g_new == nullptr)) return fail(CSA_ERR_INVALID_ARG, "x_new and g_new must both be given or both NULL");
   if (x_new) { CSA_TRY(need_ptr(x_new, "x_new")); CSA_TRY(need_ptr(g_new, "g_new")); }
   if (cache->window_cap < L->window) return fail(CSA_ERR_INVALID_ARG, "window_cap < window");
-  return run_append_compress(L, cache, nullptr, x_new, g_new, q_pos, Tq, true, false, static_cast<cudaStream_t>(stream));
+  int* err = nullptr;
+  const cudaError_t e = library_error_word(&err);
+  if (e != cudaSuccess) return cuda_fail(e, "library error word");
+  return run_append_compress(L, cache, nullptr, x_new, g_new, q_pos, Tq, true, false, err,
+                             static_cast<cudaStream_t>(stream));
 }
 
 csa_status_t csa_compress(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P,
@@ -432,7 +522,11 @@ csa_status_t csa_compress(const csa_layer_t* L, const csa_cache_t* cache, const 
   CSA_TRY(check_params(L, P, true));
   CSA_TRY(need_ptr(q_pos, "q_pos", 8));
   if (Tq < 1) return fail(CSA_ERR_INVALID_ARG, "Tq=%d", Tq);
-  return run_append_compress(L, cache, P, nullptr, nullptr, q_pos, Tq, false, true, static_cast<cudaStream_t>(stream));
+  int* err = nullptr;
+  const cudaError_t e = library_error_word(&err);
+  if (e != cudaSuccess) return cuda_fail(e, "library error word");
+  return run_append_compress(L, cache, P, nullptr, nullptr, q_pos, Tq, false, true, err,
+                             static_cast<cudaStream_t>(stream));
 }
 
 csa_status_t csa_index_topk(const csa_layer_t* L, const csa_cache_t* cache, const void* idx_q,
@@ -495,45 +589,38 @@ csa_status_t hca_attend(const csa_layer_t* L, const csa_cache_t* cache, const cs
   return run_attend(L, cache, P, q, q_pos, Tq, nullptr, n_max, out, w, workspace, static_cast<cudaStream_t>(stream));
 }
 
-csa_status_t csa_decode_step(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P, const void* q,
-                             const void* idx_q, const float* idx_q_scale, const float* head_w, const void* x_new,
-                             const void* g_new, const int64_t* q_pos, void* out, int32_t* topk_idx,
-                             void* workspace, size_t ws_bytes, void* stream) {
-  CSA_TRY(check_layer(L));
-  if (L->kind != CSA_KIND_CSA) return fail(CSA_ERR_INVALID_ARG, "csa_decode_step needs a CSA layer");
-  CSA_TRY(check_cache_attend(L, cache));
-  CSA_TRY(check_cache_raw(L, cache, true));
-  CSA_TRY(need_ptr(cache->idx_keys, "cache.idx_keys"));
-  CSA_TRY(need_ptr(cache->idx_key_scale, "cache.idx_key_scale", 4));
-  CSA_TRY(check_params(L, P, true));
-  CSA_TRY(need_ptr(P->sinks, "params.sinks", 4));
-  CSA_TRY(need_ptr(q, "q"));
-  CSA_TRY(need_ptr(idx_q, "idx_q"));
-  CSA_TRY(need_ptr(idx_q_scale, "idx_q_scale", 4));
-  CSA_TRY(need_ptr(head_w, "head_w", 4));
-  CSA_TRY(need_ptr(x_new, "x_new"));
-  CSA_TRY(need_ptr(g_new, "g_new"));
-  CSA_TRY(need_ptr(q_pos, "q_pos", 8));
-  CSA_TRY(need_ptr(out, "out"));
-  if (topk_idx) CSA_TRY(need_ptr(topk_idx, "topk_idx", 4));
-  if (cache->raw_cap < (1 + L->overlap) * (int64_t)L->m) return fail(CSA_ERR_INVALID_ARG, "raw_cap < (1+overlap)*m");
-  const Workspace w = layout(L, CSA_OP_DECODE_STEP, 1, cache->entry_cap);
-  CSA_TRY(check_ws(w, workspace, ws_bytes));
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+}  // extern "C"
+
+namespace {
+
+// The CSA decode step after argument checks: append+compress and q preparation on the side stream;
+// on the caller's stream the index-side production (when `prep` is given), the indexer and top-k;
+// the two join before the attention.
+csa_status_t csa_decode_step_run(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P,
+                                 const void* q, const void* idx_q, const float* idx_q_scale, const float* head_w,
+                                 const void* x_new, const void* g_new, const int64_t* q_pos, void* out,
+                                 int32_t* topk_idx, const Workspace& w, void* workspace, cudaStream_t s,
+                                 const IndexPrepArgs* prep) {
   int32_t* tk = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(at(workspace, w.topk));
+  int* ws_err = reinterpret_cast<int*>(at(workspace, w.err));
+  float* scores = reinterpret_cast<float*>(at(workspace, w.scores));
+  auto index_side = [&]() -> csa_status_t {
+    if (prep) {
+      const cudaError_t e = launch_index_prep(*prep, s);
+      if (e != cudaSuccess) return cuda_fail(e, "index preparation launch");
+    }
+    return run_index_topk(L, cache, idx_q, idx_q_scale, head_w, q_pos, 1, cache->entry_cap, tk, scores, w,
+                          workspace, s);
+  };
   SideStream* ss = side_stream(s);
   if (ss) {
     // fork: append+compress on the side stream, indexer + top-k here; join before attention
     cudaError_t e = cudaEventRecord(ss->fork, s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->s, ss->fork, 0);
     if (e != cudaSuccess) return cuda_fail(e, "csa_decode_step fork");
-    csa_status_t sc = run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, ss->s);
+    csa_status_t sc = run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, ws_err, ss->s);
     if (sc == CSA_OK) sc = run_qprep(L, cache, P, q, q_pos, 1, tk, cache->entry_cap, w, workspace, ss->s);
-    const csa_status_t si = sc == CSA_OK ? run_index_topk(L, cache, idx_q, idx_q_scale, head_w, q_pos, 1,
-                                                          cache->entry_cap, tk,
-                                                          reinterpret_cast<float*>(at(workspace, w.scores)), w,
-                                                          workspace, s)
-                                         : sc;
+    const csa_status_t si = sc == CSA_OK ? index_side() : sc;
     // the join is recorded whatever happened, so a capture never ends with the side stream unjoined
     e = cudaEventRecord(ss->join, ss->s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
@@ -541,10 +628,159 @@ csa_status_t csa_decode_step(const csa_layer_t* L, const csa_cache_t* cache, con
     if (e != cudaSuccess) return cuda_fail(e, "csa_decode_step join");
     return run_attend(L, cache, P, q, q_pos, 1, tk, cache->entry_cap, out, w, workspace, s, false);
   }
-  CSA_TRY(run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, s));
-  CSA_TRY(run_index_topk(L, cache, idx_q, idx_q_scale, head_w, q_pos, 1, cache->entry_cap, tk,
-                         reinterpret_cast<float*>(at(workspace, w.scores)), w, workspace, s));
+  CSA_TRY(run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, ws_err, s));
+  CSA_TRY(index_side());
   return run_attend(L, cache, P, q, q_pos, 1, tk, cache->entry_cap, out, w, workspace, s);
+}
+
+csa_status_t check_decode_common(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P,
+                                 const void* q, const float* head_w, const void* x_new, const void* g_new,
+                                 const int64_t* q_pos, void* out, int32_t* topk_idx, const char* who) {
+  CSA_TRY(check_layer(L));
+  if (L->kind != CSA_KIND_CSA) return fail(CSA_ERR_INVALID_ARG, "%s needs a CSA layer", who);
+  CSA_TRY(check_cache_attend(L, cache));
+  CSA_TRY(check_cache_raw(L, cache, true));
+  CSA_TRY(need_ptr(cache->idx_keys, "cache.idx_keys"));
+  CSA_TRY(need_ptr(cache->idx_key_scale, "cache.idx_key_scale", 4));
+  CSA_TRY(check_params(L, P, true));
+  CSA_TRY(need_ptr(P->sinks, "params.sinks", 4));
+  CSA_TRY(need_ptr(q, "q"));
+  CSA_TRY(need_ptr(head_w, "head_w", 4));
+  CSA_TRY(need_ptr(x_new, "x_new"));
+  CSA_TRY(need_ptr(g_new, "g_new"));
+  CSA_TRY(need_ptr(q_pos, "q_pos", 8));
+  CSA_TRY(need_ptr(out, "out"));
+  if (topk_idx) CSA_TRY(need_ptr(topk_idx, "topk_idx", 4));
+  if (cache->raw_cap < (1 + L->overlap) * (int64_t)L->m) return fail(CSA_ERR_INVALID_ARG, "raw_cap < (1+overlap)*m");
+  return CSA_OK;
+}
+
+// Index-side arguments shared by csa_index_keys, csa_index_query and the indexed decode step.
+csa_status_t check_index_side(const csa_layer_t* L, const void* c, const void* W, int32_t rank) {
+  if (L->kind != CSA_KIND_CSA) return fail(CSA_ERR_INVALID_ARG, "the index side needs a CSA layer");
+  if (L->d_I % 32 || L->d_I > 128) return fail(CSA_ERR_UNSUPPORTED, "d_I=%d (index production needs a multiple of 32, <= 128)", L->d_I);
+  if (c || W) {
+    CSA_TRY(need_ptr(c, "c", 4));
+    CSA_TRY(need_ptr(W, "W", 4));
+    if (rank < 16 || rank % 16) return fail(CSA_ERR_UNSUPPORTED, "rank=%d (needs a positive multiple of 16)", rank);
+    if (L->act_format != CSA_FMT_BF16) return fail(CSA_ERR_UNSUPPORTED, "the index query needs bf16 latents and weights");
+  }
+  return CSA_OK;
+}
+
+IndexPrepArgs index_prep_args(const csa_layer_t* L, const csa_cache_t* cache, const csa_index_stream_t* S,
+                              const int64_t* q_pos, int32_t Tq) {
+  IndexPrepArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = L->B; a.Tq = Tq; a.H_I = L->H_I; a.d_I = L->d_I; a.m = L->m; a.ov = L->overlap;
+  a.act_fmt = L->act_format; a.idx_fmt = L->idx_format;
+  a.pos0 = L->pos0;
+  a.entry_cap = cache ? cache->entry_cap : 0;
+  a.raw_cap = cache ? cache->raw_cap : 0;
+  a.raw_base = cache ? cache->raw_base : 0;
+  a.q_pos = q_pos;
+  if (S) {
+    a.raw = static_cast<uint8_t*>(S->raw);
+    a.gate = static_cast<uint8_t*>(S->gate);
+    a.pos_bias = S->pos_bias;
+  }
+  return a;
+}
+
+csa_status_t check_index_stream(const csa_layer_t* L, const csa_cache_t* cache, const csa_index_stream_t* S) {
+  if (!S) return fail(CSA_ERR_INVALID_ARG, "index stream is NULL");
+  CSA_TRY(need_ptr(S->raw, "index_stream.raw"));
+  CSA_TRY(need_ptr(S->gate, "index_stream.gate"));
+  CSA_TRY(need_ptr(S->pos_bias, "index_stream.pos_bias", 4));
+  CSA_TRY(need_ptr(cache->idx_keys, "cache.idx_keys"));
+  CSA_TRY(need_ptr(cache->idx_key_scale, "cache.idx_key_scale", 4));
+  if (cache->raw_cap < 1) return fail(CSA_ERR_INVALID_ARG, "raw_cap=%lld", (long long)cache->raw_cap);
+  (void)L;
+  return CSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+csa_status_t csa_decode_step(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P, const void* q,
+                             const void* idx_q, const float* idx_q_scale, const float* head_w, const void* x_new,
+                             const void* g_new, const int64_t* q_pos, void* out, int32_t* topk_idx,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  CSA_TRY(check_decode_common(L, cache, P, q, head_w, x_new, g_new, q_pos, out, topk_idx, "csa_decode_step"));
+  CSA_TRY(need_ptr(idx_q, "idx_q"));
+  CSA_TRY(need_ptr(idx_q_scale, "idx_q_scale", 4));
+  const Workspace w = layout(L, CSA_OP_DECODE_STEP, 1, cache->entry_cap);
+  CSA_TRY(check_ws(w, workspace, ws_bytes));
+  return csa_decode_step_run(L, cache, P, q, idx_q, idx_q_scale, head_w, x_new, g_new, q_pos, out, topk_idx, w,
+                             workspace, static_cast<cudaStream_t>(stream), nullptr);
+}
+
+csa_status_t csa_index_keys(const csa_layer_t* L, const csa_cache_t* cache, const csa_index_stream_t* S,
+                            const void* x_new, const void* g_new, const int64_t* q_pos, int32_t Tq, void* stream) {
+  CSA_TRY(check_layer(L));
+  if (!cache) return fail(CSA_ERR_INVALID_ARG, "cache is NULL");
+  CSA_TRY(check_index_side(L, nullptr, nullptr, 0));
+  CSA_TRY(check_index_stream(L, cache, S));
+  CSA_TRY(need_ptr(q_pos, "q_pos", 8));
+  if (Tq < 1) return fail(CSA_ERR_INVALID_ARG, "Tq=%d", Tq);
+  if ((x_new == nullptr) != (g_new == nullptr)) return fail(CSA_ERR_INVALID_ARG, "x_new and g_new must both be given or both NULL");
+  if (x_new) { CSA_TRY(need_ptr(x_new, "x_new", 4)); CSA_TRY(need_ptr(g_new, "g_new", 4)); }
+  IndexPrepArgs a = index_prep_args(L, cache, S, q_pos, Tq);
+  a.x_new = static_cast<const uint8_t*>(x_new);
+  a.g_new = static_cast<const uint8_t*>(g_new);
+  a.keys = static_cast<uint8_t*>(cache->idx_keys);
+  a.key_scale = const_cast<float*>(cache->idx_key_scale);
+  const cudaError_t e = launch_index_prep(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e, "index key launch");
+}
+
+csa_status_t csa_index_query(const csa_layer_t* L, const void* c, const void* W, int32_t rank, int32_t rows,
+                             void* idx_q, float* idx_q_scale, void* stream) {
+  CSA_TRY(check_layer(L));
+  if (!c || !W) return fail(CSA_ERR_INVALID_ARG, "c and W are required");
+  CSA_TRY(check_index_side(L, c, W, rank));
+  CSA_TRY(need_ptr(idx_q, "idx_q", 4));
+  CSA_TRY(need_ptr(idx_q_scale, "idx_q_scale", 4));
+  if (rows < 1) return fail(CSA_ERR_INVALID_ARG, "rows=%d", rows);
+  IndexPrepArgs a = index_prep_args(L, nullptr, nullptr, nullptr, 1);
+  a.c = static_cast<const uint8_t*>(c);
+  a.W = static_cast<const uint8_t*>(W);
+  a.rank = rank;
+  a.rows = rows;
+  a.q_out = static_cast<uint8_t*>(idx_q);
+  a.q_scale_out = idx_q_scale;
+  const cudaError_t e = launch_index_prep(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e, "index query launch");
+}
+
+csa_status_t csa_decode_step_indexed(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P,
+                                     const csa_index_stream_t* S, const void* q, const void* c, const void* W,
+                                     int32_t rank, const float* head_w, const void* x_new, const void* g_new,
+                                     const void* idx_x_new, const void* idx_g_new, const int64_t* q_pos, void* out,
+                                     int32_t* topk_idx, void* workspace, size_t ws_bytes, void* stream) {
+  CSA_TRY(check_decode_common(L, cache, P, q, head_w, x_new, g_new, q_pos, out, topk_idx,
+                              "csa_decode_step_indexed"));
+  if (!c || !W) return fail(CSA_ERR_INVALID_ARG, "c and W are required");
+  CSA_TRY(check_index_side(L, c, W, rank));
+  CSA_TRY(check_index_stream(L, cache, S));
+  CSA_TRY(need_ptr(idx_x_new, "idx_x_new", 4));
+  CSA_TRY(need_ptr(idx_g_new, "idx_g_new", 4));
+  const Workspace w = layout(L, CSA_OP_DECODE_STEP_INDEXED, 1, cache->entry_cap);
+  CSA_TRY(check_ws(w, workspace, ws_bytes));
+  IndexPrepArgs a = index_prep_args(L, cache, S, q_pos, 1);
+  a.x_new = static_cast<const uint8_t*>(idx_x_new);
+  a.g_new = static_cast<const uint8_t*>(idx_g_new);
+  a.keys = static_cast<uint8_t*>(cache->idx_keys);
+  a.key_scale = const_cast<float*>(cache->idx_key_scale);
+  a.c = static_cast<const uint8_t*>(c);
+  a.W = static_cast<const uint8_t*>(W);
+  a.rank = rank;
+  a.rows = L->B;
+  a.q_out = at(workspace, w.idxq);
+  a.q_scale_out = reinterpret_cast<float*>(at(workspace, w.idxqs));
+  return csa_decode_step_run(L, cache, P, q, a.q_out, a.q_scale_out, head_w, x_new, g_new, q_pos, out, topk_idx, w,
+                             workspace, static_cast<cudaStream_t>(stream), &a);
 }
 
 csa_status_t hca_decode_step(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P, const void* q,
@@ -564,6 +800,7 @@ csa_status_t hca_decode_step(const csa_layer_t* L, const csa_cache_t* cache, con
   const Workspace w = layout(L, CSA_OP_HCA_ATTEND, 1, cache->entry_cap);
   CSA_TRY(check_ws(w, workspace, ws_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* ws_err = reinterpret_cast<int*>(at(workspace, w.err));
   SideStream* ss = side_stream(s);
   if (ss) {
     // fork: the attention's query preparation on the side stream beside append+compress
@@ -571,7 +808,7 @@ csa_status_t hca_decode_step(const csa_layer_t* L, const csa_cache_t* cache, con
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->s, ss->fork, 0);
     if (e != cudaSuccess) return cuda_fail(e, "hca_decode_step fork");
     const csa_status_t sq = run_qprep(L, cache, P, q, q_pos, 1, nullptr, cache->entry_cap, w, workspace, ss->s);
-    const csa_status_t sc = run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, s);
+    const csa_status_t sc = run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, ws_err, s);
     e = cudaEventRecord(ss->join, ss->s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
     if (sq != CSA_OK) return sq;
@@ -579,7 +816,7 @@ csa_status_t hca_decode_step(const csa_layer_t* L, const csa_cache_t* cache, con
     if (e != cudaSuccess) return cuda_fail(e, "hca_decode_step join");
     return run_attend(L, cache, P, q, q_pos, 1, nullptr, cache->entry_cap, out, w, workspace, s, false);
   }
-  CSA_TRY(run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, s));
+  CSA_TRY(run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, ws_err, s));
   return run_attend(L, cache, P, q, q_pos, 1, nullptr, cache->entry_cap, out, w, workspace, s);
 }
 
@@ -611,7 +848,8 @@ csa_status_t csa_prefill(const csa_layer_t* L, const csa_cache_t* cache, const c
   const Workspace w = layout(L, CSA_OP_PREFILL, Tq, n_max);
   CSA_TRY(check_ws(w, workspace, ws_bytes));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  CSA_TRY(run_append_compress(L, cache, P, nullptr, nullptr, q_pos, Tq, true, true, s));
+  int* ws_err = reinterpret_cast<int*>(at(workspace, w.err));
+  CSA_TRY(run_append_compress(L, cache, P, nullptr, nullptr, q_pos, Tq, true, true, ws_err, s));
   int32_t* tk = nullptr;
   if (csa) {
     tk = topk_idx ? topk_idx : reinterpret_cast<int32_t*>(at(workspace, w.topk));

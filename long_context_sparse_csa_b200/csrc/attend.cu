@@ -98,6 +98,9 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t w) {
   return __half22float2(*reinterpret_cast<const __half2*>(&w));
 }
 
+// 2^e as a float, for integer e in [-126, 127] (built from the exponent field: exact).
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
+
 // Two e4m3 codes (low byte first) -> two floats, via the hardware e4m3x2 -> f16x2 conversion.
 __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t codes) {
   const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)codes, __NV_E4M3);
@@ -734,8 +737,9 @@ __host__ __device__ constexpr int tc_x_bytes(int n) {
   const int raw = n * kTcHalfRow, p = (n / 64) * kTcQBlock;
   return ((raw > p ? raw : p) + 1023) / 1024 * 1024;
 }
-// the peer's fp16 partial scores: [slot half][N / 16 groups of 8][128 heads] x 16 bytes
-__host__ __device__ constexpr int tc_xr_bytes(int n) { return n * 256; }
+// the peer's partial scores: [slot half][N / 16 groups of 8][128 heads] x 16 bytes of fp16, then the
+// power-of-two exponent each sending thread scaled them by: [slot half][128 heads] int32
+__host__ __device__ constexpr int tc_xr_bytes(int n) { return n * 256 + 2 * 128 * 4; }
 constexpr size_t tc_smem_bytes(int n) {
   return 1024 + 4 * (size_t)n * 128 + 4 * (size_t)kTcQBlock + tc_x_bytes(n) + tc_xr_bytes(n) + 64 + n * 8 +
          4 * 128 * 4 + n * 8;
@@ -985,11 +989,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
 
   // ---------------------------------------------------------------- S = the two partials (cluster pair)
   // Warps w and w+4 read the same TMEM lanes (heads 32(w%4)..); warps 4..7 take the first half of
-  // the slots, warps 0..3 the second.  Each thread sends its partial scores, rounded to fp16, to the
-  // thread with the same (head, slot half) in the peer CTA: st.async into the peer's receive buffer
-  // as [slot half][groups of 8][head] 16-byte pieces, the bytes counted on the peer's receive
-  // barrier (no cluster barrier per exchange).  The fp16 rounding (2^-11 relative) is finer than P's
-  // own bf16 rounding.
+  // the slots, warps 0..3 the second.  Each thread sends its partial scores to the thread with the
+  // same (head, slot half) in the peer CTA: st.async into the peer's receive buffer as [slot half]
+  // [groups of 8][head] 16-byte pieces of fp16, the bytes counted on the peer's receive barrier (no
+  // cluster barrier per exchange).  Before rounding, the thread scales its scores by 2^-e, with e
+  // chosen from their largest magnitude so that it lands in [2^14, 2^15): no partial score of any
+  // size overflows fp16's range, and each keeps fp16's 2^-11 relative rounding, finer than the bf16
+  // of q~ it is made of.  e itself crosses as one more 4-byte st.async.
   const float cl2 = L.scale * kLog2e;
   const int h = (warp & 3) * 32 + lane;
   const int hs = warp >= 4 ? 0 : 1;                       // slot half of this warp
@@ -998,21 +1004,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
 #pragma unroll
   for (int c = 0; c < kHalf; c += 32) tmem_ld_32x32b_x32(lane_addr + kHalf * hs + c, s + c);
   tmem_wait_ld();
+  int32_t* XE = reinterpret_cast<int32_t*>(XR + kN * 256);   // [slot half][head] exponents received
   asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   ATRACE_T(0, 4);
   {
-    uint32_t rd, rb;
+    float amx = 0.f;
+#pragma unroll
+    for (int c = 0; c < kHalf; ++c) amx = fmaxf(amx, fabsf(s[c]));
+    // floor(log2 amx) from the exponent field (amx >= 0; a subnormal or zero amx gives -127)
+    int e = (int)((__float_as_uint(amx) >> 23) & 0xFFu) - 127 - 14;
+    e = e < -110 ? -110 : (e > 110 ? 110 : e);
+    const float sc = pow2i(-e);
+    uint32_t rd, rb, re;
     const uint32_t ld = smem_u32(XR) + (uint32_t)(((size_t)hs * (kHalf / 8) * kH128 + h) * 16);
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rd) : "r"(ld), "r"(dh ^ 1));
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rb) : "r"(smem_u32(&bars[1])), "r"(dh ^ 1));
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(re) : "r"(smem_u32(XE + hs * kH128 + h)), "r"(dh ^ 1));
 #pragma unroll
     for (int j = 0; j < kHalf / 8; ++j) {
       const float* v = s + 8 * j;
       asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
-                   ::"r"(rd + (uint32_t)(j * kH128 * 16)), "r"(pack_f16x2(v[0], v[1])), "r"(pack_f16x2(v[2], v[3])),
-                     "r"(pack_f16x2(v[4], v[5])), "r"(pack_f16x2(v[6], v[7])), "r"(rb)
+                   ::"r"(rd + (uint32_t)(j * kH128 * 16)), "r"(pack_f16x2(v[0] * sc, v[1] * sc)),
+                     "r"(pack_f16x2(v[2] * sc, v[3] * sc)), "r"(pack_f16x2(v[4] * sc, v[5] * sc)),
+                     "r"(pack_f16x2(v[6] * sc, v[7] * sc)), "r"(rb)
                    : "memory");
     }
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+                 ::"r"(re), "r"(e), "r"(rb)
+                 : "memory");
   }
   if (!mbar_wait(&bars[1], 0u)) ok = false;
   // second phase: this CTA has all of its peer's scores (awaited before the CTA leaves, so neither
@@ -1021,6 +1040,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   ATRACE_T(0, 8);
   {
     const uint4* mine = reinterpret_cast<const uint4*>(XR) + (size_t)hs * (kHalf / 8) * kH128 + h;
+    const float up = pow2i(XE[hs * kH128 + h]);
 #pragma unroll
     for (int j = 0; j < kHalf / 8; ++j) {
       const uint4 v = mine[(size_t)j * kH128];
@@ -1028,8 +1048,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float2 f = unpack_f16x2(w[q]);
-        s[8 * j + 2 * q] += f.x;
-        s[8 * j + 2 * q + 1] += f.y;
+        s[8 * j + 2 * q] += f.x * up;
+        s[8 * j + 2 * q + 1] += f.y * up;
       }
     }
   }
@@ -1270,12 +1290,10 @@ size_t mma_smem_bytes() {
 template <int HG, int FMT>
 cudaError_t launch_mma(const AttendArgs& a, cudaStream_t s) {
   const size_t smem = mma_smem_bytes<HG, FMT>();
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attend_mma_kernel<HG, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+  {
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(attend_mma_kernel<HG, FMT>),
+                                         smem);
     if (e != cudaSuccess) return e;
-    configured = true;
   }
   dim3 grid(a.splits, a.L.H / HG, a.rows);
   cudaError_t e = launch_kernel(attend_mma_kernel<HG, FMT>, grid, dim3(HG * 8), smem, s, 0, a);
@@ -1364,12 +1382,10 @@ bool make_qt_map(CUtensorMap* m, const void* qt, int rows) {
 template <int FMT, int kN>
 cudaError_t launch_tc_n(const AttendArgs& a, cudaStream_t s) {
   constexpr size_t smem = tc_smem_bytes(kN);
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<FMT, kN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+  {
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(attend_tc_kernel<FMT, kN>),
+                                         smem);
     if (e != cudaSuccess) return e;
-    configured = true;
   }
   CUtensorMap qmap;
   if (!make_qt_map(&qmap, a.qt, a.rows)) return cudaErrorInvalidValue;

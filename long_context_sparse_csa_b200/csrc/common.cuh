@@ -50,6 +50,26 @@ __device__ __forceinline__ float e4m3_to_f(uint8_t c) {
   return float(v);
 }
 
+// FP4 e2m1 code (low 4 bits: sign, 2 exponent bits with bias 1, 1 mantissa bit) -> float.
+__device__ __forceinline__ float e2m1_to_f(uint32_t code) {
+  const uint32_t e = (code >> 1) & 3u, m = code & 1u;
+  const float mag = e == 0 ? 0.5f * (float)m : (1.f + 0.5f * (float)m) * (float)(1u << (e - 1));
+  return (code & 8u) ? -mag : mag;
+}
+
+// Round |x| (finite) to the nearest e2m1 magnitude code 0..7, ties to the even code, saturating at 6.
+// The magnitudes are 0, .5, 1, 1.5, 2, 3, 4, 6 and the midpoints between them .25, .75, 1.25, 1.75,
+// 2.5, 3.5, 5: the code is the number of midpoints below |x|, moved up to the even neighbour when
+// |x| sits exactly on an odd code's upper midpoint.
+__device__ __forceinline__ uint32_t e2m1_rne_magnitude(float ax) {
+  const float mid[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
+  uint32_t c = 0;
+#pragma unroll
+  for (int k = 0; k < 7; ++k) c += ax > mid[k] ? 1u : 0u;
+  if (c < 7 && ax == mid[c] && (c & 1u)) ++c;
+  return c;
+}
+
 __device__ __forceinline__ uint8_t f_to_e4m3_sat(float x) {
   return (uint8_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
 }
@@ -62,6 +82,18 @@ __device__ __forceinline__ float pow2_scale(float amax, float* inv) {
   int e;
   float f = frexpf(amax, &e);
   int k = (f <= 0.875f) ? e - 9 : e - 8;
+  *inv = ldexpf(1.f, -k);
+  return ldexpf(1.f, k);
+}
+
+// Smallest power of two sigma with amax / sigma <= 6, the FP4 maximum (1 for amax == 0); *inv = 1 /
+// sigma.  6 = 0.75 * 2^3: with amax = f * 2^e (0.5 <= f < 1) the bound first holds at k = e - 3 when
+// f <= 0.75, else at k = e - 2.
+__device__ __forceinline__ float pow2_scale_fp4(float amax, float* inv) {
+  if (!(amax > 0.f)) { *inv = 1.f; return 1.f; }
+  int e;
+  float f = frexpf(amax, &e);
+  int k = (f <= 0.75f) ? e - 3 : e - 2;
   *inv = ldexpf(1.f, -k);
   return ldexpf(1.f, k);
 }

@@ -18,6 +18,8 @@
 // vector loads.
 #include <cooperative_groups.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -27,6 +29,9 @@ namespace cg = cooperative_groups;
 namespace csa {
 
 namespace {
+
+// Error word of calls that take no workspace (csa_append, csa_compress), one per device.
+__device__ int g_library_error;
 
 #ifdef CSA_TRACE
 __device__ uint64_t g_trace_c[4][16];
@@ -84,9 +89,10 @@ __device__ __forceinline__ void mail_send(ClusterMail* m, int k, int q, int CL, 
                : "memory");
 }
 
-// Waits (bounded) for the CL partials of mailbox k; every thread gets (sum of .x, max of .y).
-__device__ __forceinline__ float2 mail_reduce(ClusterMail* m, int k, int CL) {
-  sm100::mbar_wait(&m->bar[k], 0u);
+// Waits (bounded) for the CL partials of mailbox k; every thread gets (sum of .x, max of .y).  A
+// wait that gives up sets the error word's timeout bit: the reduced values are then incomplete.
+__device__ __forceinline__ float2 mail_reduce(ClusterMail* m, int k, int CL, int* err) {
+  if (!sm100::mbar_wait(&m->bar[k], 0u)) set_device_error(err, kErrWaitTimeout);
   float x = 0.f, y = -INFINITY;
   for (int p = 0; p < CL; ++p) {
     const float2 v = m->box[k][p];
@@ -216,7 +222,7 @@ __global__ void __launch_bounds__(256) append_compress_kernel(const __grid_const
       const float bm = block_max(local_amax(w, c0, dn, lead), scratch);
       if (!mail_open) { cluster_wait(); mail_open = true; }
       mail_send(&mail, 0, q, CL, make_float2(0.f, bm));
-      am = mail_reduce(&mail, 0, CL).y;
+      am = mail_reduce(&mail, 0, CL, a.err).y;
       if (!compress) { cluster_arrive_relaxed(); done_mail = true; }   // this CTA's mail is all in
     }
     uint8_t* dst = C.window + ((size_t)b * C.window_cap + (size_t)(r % C.window_cap)) * L.row_bytes;
@@ -421,7 +427,7 @@ __global__ void __launch_bounds__(256) append_compress_kernel(const __grid_const
     const float2 bl = block_sum_max(ss, eg, scratch);
     if (!mail_open) { cluster_wait(); mail_open = true; }
     mail_send(&mail, 1, q, CL, bl);
-    const float2 red2 = mail_reduce(&mail, 1, CL);
+    const float2 red2 = mail_reduce(&mail, 1, CL, a.err);
     cluster_arrive_relaxed();                      // this CTA's mail is all in
     done_mail = true;
     const float rs = 1.0f / sqrtf(red2.x / (float)L.D + L.eps);
@@ -450,6 +456,24 @@ extern "C" __attribute__((visibility("default"))) int csa_trace_read_c(uint64_t*
 }
 #endif
 
+cudaError_t library_error_word(int** p) {
+  static std::mutex mu;
+  static int* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* q = nullptr;
+    e = cudaGetSymbolAddress(&q, g_library_error);
+    if (e != cudaSuccess) return e;
+    addr[dev] = static_cast<int*>(q);
+  }
+  *p = addr[dev];
+  return cudaSuccess;
+}
+
 cudaError_t launch_append_compress(const AppendCompressArgs& a, int B, int Tq, cudaStream_t s) {
   // decode (few tokens): a cluster of CL CTAs per token splits the channels, and row groups split
   // the entry's source rows; a chunk has parallelism across tokens and runs one CTA per token.
@@ -473,19 +497,13 @@ cudaError_t launch_append_compress(const AppendCompressArgs& a, int B, int Tq, c
     while (rg > 1 && ct * rg > 256) rg >>= 1;
   }
   if (CL > 8) {
-    static bool nonportable = false;
-    if (!nonportable) {
-      cudaError_t e = cudaFuncSetAttribute(append_compress_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (e != cudaSuccess) return e;
-      nonportable = true;
-    }
+    cudaError_t e = ensure_nonportable_cluster(reinterpret_cast<const void*>(append_compress_kernel));
+    if (e != cudaSuccess) return e;
   }
   const size_t smem = rg > 1 ? (size_t)rg * 3 * (a.L.D / CL) * sizeof(float) : 0;
-  static size_t configured = 0;
-  if (smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(append_compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  {
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(append_compress_kernel), smem);
     if (e != cudaSuccess) return e;
-    configured = smem;
   }
   return launch_kernel(append_compress_kernel, dim3((unsigned)(Tq * CL), (unsigned)B), dim3((unsigned)(ct * rg)), smem, s,
                     CL, a, CL);

@@ -103,8 +103,8 @@ __device__ __forceinline__ Sched make_sched(const IndexArgs& a) {
 #ifdef CSA_TRACE
 // Diagnostic build only: per-CTA timestamps (ns) of the indexer pipeline.
 __device__ uint64_t g_trace[320][80];
-#define TRACE(slot) (g_trace[blockIdx.x][(slot)] = global_timer_ns())
-#define TRACE_VAL(slot, v) (g_trace[blockIdx.x][(slot)] = (uint64_t)(v))
+#define TRACE(slot) do { if (blockIdx.x < 320) g_trace[blockIdx.x][(slot)] = global_timer_ns(); } while (0)
+#define TRACE_VAL(slot, v) do { if (blockIdx.x < 320) g_trace[blockIdx.x][(slot)] = (uint64_t)(v); } while (0)
 #define CYC() clock64()
 #else
 #define TRACE(slot) ((void)0)
@@ -588,13 +588,22 @@ __global__ void index_score_generic_kernel(const __grid_constant__ IndexArgs a) 
   if (e >= a.n_max) return;
   if (e >= n_visible(a, b, j)) { a.scores[row * a.n_max + e] = -INFINITY; return; }
   const int64_t krow = (int64_t)b * a.entry_cap + e;
-  const float ks = a.k_scale[krow];
+  // FP4 keys: the scale word holds the key scale's exponent and the 32-dim blocks' offsets
+  const uint32_t word = a.idx_fmt == CSA_FMT_E2M1 ? reinterpret_cast<const uint32_t*>(a.k_scale)[krow] : 0u;
+  const float ks = a.idx_fmt == CSA_FMT_E2M1 ? __uint_as_float((word & 0xFFu) << 23) : a.k_scale[krow];
   float s = 0.f;
   for (int h = 0; h < a.H_I; ++h) {
     float dot = 0.f;
     if (a.idx_fmt == CSA_FMT_F32) {
       const float* k = reinterpret_cast<const float*>(a.idx_k) + krow * a.d_I;
       for (int d = 0; d < a.d_I; ++d) dot += qv[h * a.d_I + d] * k[d];
+    } else if (a.idx_fmt == CSA_FMT_E2M1) {
+      const uint8_t* k = a.idx_k + krow * (a.d_I / 2);
+      for (int d = 0; d < a.d_I; ++d) {
+        const uint32_t code = (k[d >> 1] >> ((d & 1) * 4)) & 0xFu;
+        const int delta = (int)((word >> (8 + 4 * (d >> 5))) & 0xFu);
+        dot += qv[h * a.d_I + d] * (e2m1_to_f(code) * __uint_as_float((uint32_t)(127 - delta) << 23));
+      }
     } else {
       const uint8_t* k = a.idx_k + krow * a.d_I;
       for (int d = 0; d < a.d_I; ++d) dot += qv[h * a.d_I + d] * e4m3_to_f(k[d]);
@@ -645,12 +654,16 @@ bool index_tc_supported(int idx_fmt, int H_I, int d_I) {
 
 cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
   if (a.n_max <= 0 || a.Tq <= 0 || a.B <= 0) return cudaSuccess;
+  // decode with FP4 keys: the warp-level streaming kernel (it also fills the top-k's histogram); FP8
+  // decode keys take the tcgen05 kernel below, measured faster on the 1M-token step (20.5 against
+  // 28 us per launch)
+  if (a.Tq == 1 && a.idx_fmt == CSA_FMT_E2M1 && index_decode_supported(a.idx_fmt, a.H_I, a.d_I))
+    return launch_index_decode(a, num_sms, s);
   if (!index_tc_supported(a.idx_fmt, a.H_I, a.d_I)) {
     dim3 grid((unsigned)((a.n_max + 127) / 128), (unsigned)(a.B * a.Tq));
     const size_t sm = (size_t)a.H_I * a.d_I * sizeof(float);
     if (sm > 0) {
-      cudaError_t e = cudaFuncSetAttribute(index_score_generic_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)sm);
+      cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(index_score_generic_kernel), sm);
       if (e != cudaSuccess) return e;
     }
     return launch_kernel(index_score_generic_kernel, grid, dim3(128), sm, s, 0, a);
@@ -672,16 +685,14 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
   const int stages = decode ? 4 : 2;
   const size_t smem = 1024 + (size_t)stages * kTileBytes + 2 * (size_t)N * kDI + ((sizeof(Barriers) + 15) & ~size_t(15)) +
                      (decode ? sizeof(EpiSmem) : kEpiSmemNoHist) + 64;
-  static size_t configured[4] = {0, 0, 0, 0};
   const int ki = !decode ? 0 : a.H_I == 16 ? 1 : a.H_I == 32 ? 2 : 3;
   auto kern = ki == 0 ? index_score_tc_kernel<2, 0>
             : ki == 1 ? index_score_tc_kernel<4, 16>
             : ki == 2 ? index_score_tc_kernel<4, 32>
                       : index_score_tc_kernel<4, 64>;
-  if (smem > configured[ki]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  {
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
-    configured[ki] = smem;
   }
   const int64_t ctas = 2 * (int64_t)num_sms;
   const int64_t grid = a.total_items < ctas ? a.total_items : ctas;

@@ -15,6 +15,12 @@ void note_launches(int n);
 void profile_mark(cudaStream_t s);
 // Sets this thread's csa_last_error() text and returns st (for entry points outside api.cu).
 csa_status_t report_error(csa_status_t st, const char* msg);
+// Raises `kernel`'s dynamic shared-memory limit to at least `bytes` on the current device (function
+// attributes are per device: the setting is remembered per (device, kernel), under a lock).
+cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes);
+// Allows a non-portable cluster size (> 8 CTAs) for `kernel` on the current device (remembered
+// per (device, kernel)).
+cudaError_t ensure_nonportable_cluster(const void* kernel);
 
 // Launches a kernel in stream order, with an optional thread-block cluster size (cluster > 0).
 // (Programmatic dependent launch was measured slower on the decode chain: CTAs parked at the
@@ -44,6 +50,14 @@ cudaError_t launch_kernel(Kernel kernel, dim3 grid, dim3 block, size_t smem, cud
   return e;
 }
 
+// Test aid: one CTA waits (bounded by limit_ns) on an mbarrier phase nothing completes, then sets
+// the timeout bit of *err.
+cudaError_t launch_wait_probe(int* err, uint64_t limit_ns, cudaStream_t s);
+
+// Device address of the library's own error word on the current device: kernels of calls that take
+// no workspace (csa_append, csa_compress) report there; csa_device_error reads and clears it.
+cudaError_t library_error_word(int** p);
+
 // ----------------------------------------------------------------------------- append + compress
 struct AppendCompressArgs {
   LayerArgs L;
@@ -56,6 +70,7 @@ struct AppendCompressArgs {
   const float* gamma_kv;  // [D] or null
   int do_append;
   int do_compress;
+  int* err;               // device error word (bounded cluster waits); never null
 };
 cudaError_t launch_append_compress(const AppendCompressArgs& a, int B, int Tq, cudaStream_t s);
 
@@ -81,7 +96,34 @@ struct IndexArgs {
 };
 // True when the tcgen05 FP8 kernel handles this shape.
 bool index_tc_supported(int idx_fmt, int H_I, int d_I);
+// Decode (one query per sequence): the warp-level FP8 kernel (index_decode.cu) for these shapes.
+bool index_decode_supported(int idx_fmt, int H_I, int d_I);
+cudaError_t launch_index_decode(const IndexArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s);
+
+// ----------------------------------------------------------------------------- index side (keys, queries)
+struct IndexPrepArgs {
+  int B, Tq, H_I, d_I, m, ov, act_fmt, idx_fmt;
+  int64_t pos0, entry_cap, raw_cap, raw_base;
+  const int64_t* q_pos;     // [B][Tq]
+  // key role: append the tokens' index rows (x_new / g_new [B][Tq][d_I], or null) to the index rings
+  // and compress the index key of every entry they complete into keys / key_scale (null: no key role)
+  const uint8_t* x_new;
+  const uint8_t* g_new;
+  uint8_t* raw;             // [B][raw_cap][d_I] index-row ring (act_fmt), KV ring slots
+  uint8_t* gate;
+  const float* pos_bias;    // [(1+ov)m][d_I]
+  uint8_t* keys;            // [B][entry_cap][d_I] (e4m3, or float32)
+  float* key_scale;         // [B][entry_cap]
+  // query role: q_out [rows][H_I][d_I] = encode(W_h c_row) (c null: no query role)
+  const uint8_t* c;         // [rows][rank] bf16
+  const uint8_t* W;         // [H_I * d_I][rank] bf16
+  int rank, rows;
+  uint8_t* q_out;
+  float* q_scale_out;       // [rows][H_I]
+  int key_blocks;           // set by the launcher
+};
+cudaError_t launch_index_prep(IndexPrepArgs a, cudaStream_t s);
 
 // ----------------------------------------------------------------------------- top-k
 struct TopkArgs {

@@ -24,6 +24,15 @@ __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 std::mutex g_mu;
 void* g_addr[kMaxDevices] = {};
 
+// After a device error the split top-k may leave its histograms and counters non-zero.  Run
+// before every call: when the scratch's error word is set, zero those segments (the word itself is
+// kept for the next call that reads it); otherwise return at once.
+__global__ void __launch_bounds__(256) scratch_guard_kernel(const int* err, uint4* seg, size_t n16) {
+  if (*reinterpret_cast<const volatile int*>(err) == 0) return;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (size_t)gridDim.x * blockDim.x)
+    seg[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // Device address of g_scratch on the current device (looked up on the first call per device).
 csa_status_t scratch_address(void** out) {
   int dev = 0;
@@ -59,15 +68,32 @@ extern "C" CSA_API csa_status_t csa_decode_step_scratch(const csa_layer_t* L, co
              kScratchBytes);
     return csa::report_error(CSA_ERR_WORKSPACE, msg);
   }
+  if (device_error) *device_error = 0;
   void* ws = nullptr;
   csa_status_t st = scratch_address(&ws);
   if (st != CSA_OK) return st;
+  size_t err_off = 0, err_bytes = 0, seg_off = 0, seg_bytes = 0;
+  st = csa_debug_workspace_segment(L, CSA_OP_DECODE_STEP, 1, cache->entry_cap, CSA_SEG_ERROR_WORD, &err_off,
+                                   &err_bytes);
+  if (st == CSA_OK)
+    st = csa_debug_workspace_segment(L, CSA_OP_DECODE_STEP, 1, cache->entry_cap, CSA_SEG_TOPK_HISTOGRAM, &seg_off,
+                                     &seg_bytes);
+  if (st != CSA_OK) return st;
+  if (seg_bytes > 0) {
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    const int grid = (int)((seg_bytes / 16 + 255) / 256 < 64 ? (seg_bytes / 16 + 255) / 256 : 64);
+    const cudaError_t e = csa::launch_kernel(scratch_guard_kernel, dim3(grid), dim3(256), 0,
+                                             static_cast<cudaStream_t>(stream), 0,
+                                             reinterpret_cast<const int*>(base + err_off),
+                                             reinterpret_cast<uint4*>(base + seg_off), seg_bytes / 16);
+    if (e != cudaSuccess) return csa::report_error(CSA_ERR_CUDA, cudaGetErrorString(e));
+  }
   st = csa_decode_step(L, cache, P, q, idx_q, idx_q_scale, head_w, x_new, g_new, q_pos, out, topk_idx, ws,
                        kScratchBytes, stream);
   if (st != CSA_OK || !device_error) return st;
   // read back (and clear) the device error word; after an error, restore the all-zero scratch
   st = csa_device_error(ws, kScratchBytes, stream, device_error);
-  if (*device_error != 0) {
+  if (st == CSA_ERR_DEVICE_TIMEOUT) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(ws, 0, kScratchBytes, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);

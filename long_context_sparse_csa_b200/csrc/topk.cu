@@ -456,11 +456,9 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   if (a.rows <= 0 || a.k <= 0) return cudaSuccess;
   const int use_smem = a.n_max <= kSmemKeys ? 1 : 0;
   const size_t smem = use_smem ? (size_t)a.n_max * 4 : 0;
-  static size_t configured = 0;
-  if (smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  {
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(topk_rows_kernel), smem);
     if (e != cudaSuccess) return e;
-    configured = smem;
   }
   return launch_kernel(topk_rows_kernel, dim3(a.rows), dim3(kThreads), smem, s, 0, a, use_smem);
 }

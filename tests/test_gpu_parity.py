@@ -456,3 +456,119 @@ def test_prefill_full_size_sampled():
     Tq = wl.Tq
     queries = list(range(0, Tq, 512)) + [Tq - 1]
     _check_prefill(wl, Tq=Tq, prefix=None, queries=queries)
+
+
+# ----------------------------------------------------------------------------- the attention calls on their own
+
+def _scaled_rows(rows, fmt, D, factor):
+    """Stored rows whose values are exactly `factor` (a power of two) times the given ones."""
+    return F.encode_rows(F.decode_rows(rows, fmt, D) * factor, fmt)
+
+
+def _direct_attend(name, li, Tq=1, B=None, window_factor=1.0, logit_sharp=1.0):
+    """csa_sparse_attend (oracle top-k fed in) or hca_attend called directly on the stored caches.
+
+    Queries j < Tq of sequence b sit at positions t - Tq + 1 + j.  The window buffer holds
+    Tq + w - 1 rows, so every query finds its w rows.  With window_factor != 1 the window rows are
+    scaled by that power of two and the logit scale divided by it: logits keep their size while the
+    raw partial scores grow by the factor."""
+    over = {} if B is None else {"B": B}
+    wl = get_workload(name, **over)
+    layer = wl.layers[li]
+    d = decode_inputs(wl, li)
+    B, H, D, w = wl.B, layer.H, layer.D, layer.window
+    cap_w = w + Tq - 1 if Tq > 1 else w
+    if cap_w != w:
+        from csa_synth.generate import kv_rows
+        d["window"] = kv_rows(wl.seed, "window_chunk", li, (B, cap_w), layer)
+    if window_factor != 1.0:
+        d["window"] = _scaled_rows(d["window"], layer.kv_format, D, window_factor)
+    t_last = int(d["t"][0])
+    t = np.array([[t_last - Tq + 1 + j for j in range(Tq)] for _ in range(B)], dtype=np.int64)
+    from csa_synth.generate import act_array, stream
+    q = d["q"] if Tq == 1 else act_array(stream(wl.seed, "q_chunk", li), (B, Tq, H, D), layer.act_format)
+    st = LayerState.from_arrays(layer, B, d)
+    scale = logit_sharp / (window_factor * np.sqrt(D))
+    if scale != 1.0 / np.sqrt(D):
+        st.L.softmax_scale = scale
+    L = O.LayerSpec.of(layer)
+    L.scale = scale
+    out_dtype = torch.float32 if layer.act_format == "f32" else torch.int16
+    out = torch.zeros((B, Tq, H, D), dtype=out_dtype, device="cuda")
+    q_pos = dev(t.reshape(-1))
+    refs, sels = [], []
+    for b in range(B):
+        for j in range(Tq):
+            tj = int(t[b, j])
+            nv = int(O.n_visible(tj, 0, layer.m))
+            if layer.kind == "csa":
+                iq = F.decode_idx(d["idx_q"][b], layer.idx_format)
+                s = O.index_scores(iq, d["idx_q_scale"][b], d["head_w"][b],
+                                   F.decode_idx(d["idx_k"][b][:nv], layer.idx_format), d["idx_k_scale"][b][:nv])
+                sel = O.top_k_fast(s, layer.top_k)
+                ids = sel[sel >= 0]
+            else:
+                sel, ids = None, np.arange(nv)
+            sels.append(sel)
+            rows = np.concatenate([F.decode_rows(d["entries"][b][ids], layer.kv_format, D),
+                                   F.decode_rows(d["window"][b][O.window_row_ids(tj, 0, w) % cap_w],
+                                                 layer.kv_format, D)])
+            qv = F.decode_act(q.reshape(B, Tq, H, D)[b, j], layer.act_format)
+            refs.append(O.attend(qv, tj, rows, d["sinks"], d["gamma_q"], 64, layer.rope_base, scale, layer.eps))
+    cap = d["entries"].shape[1]
+    if layer.kind == "csa":
+        topk = dev(np.stack(sels).astype(np.int32))
+        ws = st.workspace("sparse_attend", Tq, cap)
+        C.csa_sparse_attend(st.L, st.cache(), st.params(), dev(q), q_pos, Tq, topk, out, ws)
+    else:
+        ws = st.workspace("hca_attend", Tq, cap)
+        C.hca_attend(st.L, st.cache(), st.params(), dev(q), q_pos, Tq, cap, out, ws)
+    torch.cuda.synchronize()
+    _no_device_error(ws)
+    got = out_values(out, layer.act_format).reshape(B * Tq, H, D)
+    return got, np.stack(refs)
+
+
+@pytest.mark.parametrize("name,li,Tq,B", [("csa_decode_tiny_2k", 0, 1, None), ("csa_decode_128k", 0, 1, None),
+                                          ("csa_hca_decode_1m", 0, 1, None), ("csa_decode_128k", 0, 3, 2),
+                                          ("csa_decode_128k", 0, 16, 1)])
+def test_sparse_attend_direct(name, li, Tq, B):
+    # oracle top-k fed in; Tq = 3 x B = 2 is 6 query rows (the tcgen05 kernel), Tq = 16 the mma.sync one
+    got, ref = _direct_attend(name, li, Tq, B)
+    tight = name == "csa_decode_tiny_2k"
+    for r in range(len(ref)):
+        if tight:
+            assert_out_close(got[r], ref[r], max_abs=1e-4, mean_abs=1e-5, rel_l2=1e-4)
+        else:
+            assert_out_close(got[r], ref[r], tag=f"sparse_attend/{name}/Tq={Tq}/row{r}")
+
+
+@pytest.mark.parametrize("name,li,Tq,B", [("hca_decode_128k", 0, 1, None), ("csa_hca_decode_1m", 1, 1, None),
+                                          ("csa_hca_decode_1m", 1, 4, 2)])
+def test_hca_attend_direct(name, li, Tq, B):
+    got, ref = _direct_attend(name, li, Tq, B)
+    for r in range(len(ref)):
+        assert_out_close(got[r], ref[r], tag=f"hca_attend/{name}/Tq={Tq}/row{r}")
+
+
+def _assert_relative(got, ref, rel_l2, rel_max):
+    d = np.abs(got - ref)
+    assert np.all(np.isfinite(got)), "non-finite outputs"
+    scale = np.abs(ref).max()
+    assert d.max() <= rel_max * scale, f"max-abs {d.max()} vs {rel_max} x {scale}"
+    rl2 = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rl2 <= rel_l2, f"relative L2 {rl2}"
+
+
+@pytest.mark.parametrize("name,li", [("csa_decode_128k", 0), ("csa_hca_decode_1m", 1), ("hca_decode_128k", 0)])
+@pytest.mark.parametrize("sharp", [1.0, 8.0])
+def test_large_window_rows(name, li, sharp):
+    """Window rows 1024x larger than the entries (raw activations are not normalised) with the logit
+    scale divided by 1024: the logits keep their size, but the raw partial scores reach ~7e4, beyond
+    fp16's range, so any half-precision exchange of unscaled partial scores would overflow.  With
+    the x8 sharper logits the bars are 4x wider (the bf16 rounding of q~ moves such logits more)."""
+    got, ref = _direct_attend(name, li, 1, 2 if name != "hca_decode_128k" else None, window_factor=1024.0,
+                              logit_sharp=sharp)
+    k = 1.0 if sharp == 1.0 else 4.0
+    for r in range(len(ref)):
+        _assert_relative(got[r], ref[r], rel_l2=1e-2 * k, rel_max=2e-2 * k)
