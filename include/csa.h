@@ -366,6 +366,52 @@ CSA_API csa_status_t csa_decode_step_indexed(const csa_layer_t* L, const csa_cac
                                              const int64_t* q_pos, void* out, int32_t* topk_idx,
                                              void* workspace, size_t ws_bytes, void* stream);
 
+/* Context-sharded CSA decode (one sequence's entries and index keys split into contiguous shards,
+ * one per rank).  A rank holding entries [entry_offset, entry_offset + n_local) at slots 0.. of its
+ * cache runs, for the B decode queries:
+ *   1. csa_index_topk over its shard, with a layer whose pos0 is pos0 + entry_offset * m (so each
+ *      shard entry's visibility is that of its global position) and n_max = n_local;
+ *   2. csa_shard_candidates: (score, global index) of its local top-k;
+ *   3. an all-gather of the candidates, [shards][B][top_k] each (the caller's collective);
+ *   4. csa_shard_select: the global top-k of the gathered candidates, identical on every rank;
+ *   5. csa_sparse_attend_partial over the selected entries it holds (one rank also the window rows);
+ *   6. an all-gather of the partials, [shards][B][H][D + 2] (the caller's collective);
+ *   7. csa_attend_merge: the output, with the sink counted once and the inverse rotation.
+ * The result equals csa_sparse_attend with the unsharded top-k: an entry of the global top-k is in
+ * its own shard's top-k, and attention over disjoint key sets merges by log-sum-exp weights.  The
+ * pages describe one layer, not its distribution; the sink and the inverse rotation are those of
+ * "DeepSeek-V4: Making a Million Tokens Affordable", "Two ways to shrink attention, interleaved". */
+
+/* Step 2.  scores: [B][n_local] float32 of the shard (csa_index_topk's optional output); topk_local:
+ * [B][top_k] its local top-k (-1 padded).  Writes cand_score [B][top_k] (-inf for padding) and
+ * cand_idx [B][top_k] = local index + entry_offset (-1 for padding). */
+CSA_API csa_status_t csa_shard_candidates(const csa_layer_t* L, const float* scores, int64_t n_local,
+                                          const int32_t* topk_local, int64_t entry_offset, float* cand_score,
+                                          int32_t* cand_idx, void* stream);
+
+/* Step 4.  cand_score / cand_idx: [shards][B][top_k], shard s's lists in ascending index order and
+ * the shards in ascending entry_offset order.  Writes topk_idx [B][top_k]: the top_k largest scores,
+ * ties to the smaller global index, in ascending index order, -1 padded when fewer exist.
+ * shards * top_k <= 262144. */
+CSA_API csa_status_t csa_shard_select(const csa_layer_t* L, int32_t shards, const float* cand_score,
+                                      const int32_t* cand_idx, int32_t* topk_idx, void* stream);
+
+/* Step 5.  topk_idx [B][top_k] holds global indices; the entries in [entry_offset, entry_offset +
+ * cache->entry_cap) are attended from cache slot (index - entry_offset), the others skipped; the
+ * window rows only when with_window != 0.  partial: [B][H][D + 2] float32, per (query, head) the
+ * weighted mean O/l of the attended rows (before the inverse rotation), then m and l in base 2
+ * (max logit * log2 e and the sum of 2^(logit * log2 e - m)); no sink.  Needs H = 128, D = 512,
+ * bf16 or mixed rows, B <= 8; workspace of CSA_OP_SPARSE_ATTEND. */
+CSA_API csa_status_t csa_sparse_attend_partial(const csa_layer_t* L, const csa_cache_t* cache,
+                                               const csa_params_t* P, const void* q, const int64_t* q_pos,
+                                               const int32_t* topk_idx, int64_t entry_offset, int32_t with_window,
+                                               float* partial, void* workspace, size_t ws_bytes, void* stream);
+
+/* Step 7.  partials: [parts][B][H][D + 2] as written by csa_sparse_attend_partial; out [B][H][D]
+ * act_format. */
+CSA_API csa_status_t csa_attend_merge(const csa_layer_t* L, const csa_params_t* P, const int64_t* q_pos,
+                                      int32_t parts, const float* partials, void* out, void* stream);
+
 /* Bytes of the static device scratch used by csa_decode_step_scratch. */
 #define CSA_SCRATCH_BYTES ((size_t)16 << 20)
 

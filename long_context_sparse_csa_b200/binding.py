@@ -89,6 +89,10 @@ _SIGS = {
     "csa_index_query": (ctypes.c_int, [_LAYER, _P, _P, _I32, _I32, _P, _P, _P]),
     "csa_decode_step_indexed": (ctypes.c_int, [_LAYER, _CACHE, _PARAMS, _STREAM_S, _P, _P, _P, _I32, _P, _P, _P, _P,
                                                _P, _P, _P, _P, _P, _SZ, _P]),
+    "csa_shard_candidates": (ctypes.c_int, [_LAYER, _P, _I64, _P, _I64, _P, _P, _P]),
+    "csa_shard_select": (ctypes.c_int, [_LAYER, _I32, _P, _P, _P, _P]),
+    "csa_sparse_attend_partial": (ctypes.c_int, [_LAYER, _CACHE, _PARAMS, _P, _P, _P, _I64, _I32, _P, _P, _SZ, _P]),
+    "csa_attend_merge": (ctypes.c_int, [_LAYER, _PARAMS, _P, _I32, _P, _P, _P]),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -309,3 +313,26 @@ def csa_decode_step_indexed(L, cache, params, index_stream, q, c, W, rank, head_
                                          ptr(x_new), ptr(g_new), ptr(idx_x_new), ptr(idx_g_new), ptr(q_pos), ptr(out),
                                          ptr(topk_idx), ptr(workspace), workspace.numel() * workspace.element_size(),
                                          _stream(stream)))
+
+
+def csa_shard_candidates(L, scores, n_local, topk_local, entry_offset, cand_score, cand_idx, stream=None):
+    _check(lib().csa_shard_candidates(ctypes.byref(L), ptr(scores), n_local, ptr(topk_local), entry_offset,
+                                      ptr(cand_score), ptr(cand_idx), _stream(stream)))
+
+
+def csa_shard_select(L, shards, cand_score, cand_idx, topk_idx, stream=None):
+    _check(lib().csa_shard_select(ctypes.byref(L), shards, ptr(cand_score), ptr(cand_idx), ptr(topk_idx),
+                                  _stream(stream)))
+
+
+def csa_sparse_attend_partial(L, cache, params, q, q_pos, topk_idx, entry_offset, with_window, partial, workspace,
+                              stream=None):
+    _check(lib().csa_sparse_attend_partial(ctypes.byref(L), ctypes.byref(cache), ctypes.byref(params), ptr(q),
+                                           ptr(q_pos), ptr(topk_idx), entry_offset, 1 if with_window else 0,
+                                           ptr(partial), ptr(workspace), workspace.numel() * workspace.element_size(),
+                                           _stream(stream)))
+
+
+def csa_attend_merge(L, params, q_pos, parts, partials, out, stream=None):
+    _check(lib().csa_attend_merge(ctypes.byref(L), ctypes.byref(params), ptr(q_pos), parts, ptr(partials), ptr(out),
+                                  _stream(stream)))

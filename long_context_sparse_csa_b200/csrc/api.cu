@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <climits>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -298,6 +299,7 @@ csa_status_t run_index_topk(const csa_layer_t* L, const csa_cache_t* cache, cons
   TopkArgs t;
   t.scores = scores; t.n_max = n_max; t.rows = rows; t.Tq = Tq; t.m = L->m; t.k = L->top_k;
   t.pos0 = L->pos0; t.q_pos = q_pos; t.out = topk;
+  t.map = nullptr; t.shards = 1;
   if (split) {
     TopkSplitArgs sa;
     sa.base = t;
@@ -338,6 +340,10 @@ csa_status_t make_attend_args(const csa_layer_t* L, const csa_cache_t* cache, co
   a.qt = w.qt ? at(ws, w.qt) : nullptr;
   a.err = reinterpret_cast<int*>(at(ws, w.err));
   a.out = static_cast<uint8_t*>(out);
+  a.entry_offset = 0;
+  a.entry_limit = cache->entry_cap;
+  a.no_window = 0;
+  a.partial_out = nullptr;
   return CSA_OK;
 }
 
@@ -818,6 +824,91 @@ csa_status_t hca_decode_step(const csa_layer_t* L, const csa_cache_t* cache, con
   }
   CSA_TRY(run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, ws_err, s));
   return run_attend(L, cache, P, q, q_pos, 1, nullptr, cache->entry_cap, out, w, workspace, s);
+}
+
+csa_status_t csa_shard_candidates(const csa_layer_t* L, const float* scores, int64_t n_local,
+                                  const int32_t* topk_local, int64_t entry_offset, float* cand_score,
+                                  int32_t* cand_idx, void* stream) {
+  CSA_TRY(check_layer(L));
+  if (L->kind != CSA_KIND_CSA) return fail(CSA_ERR_INVALID_ARG, "csa_shard_candidates needs a CSA layer");
+  CSA_TRY(need_ptr(scores, "scores", 4));
+  CSA_TRY(need_ptr(topk_local, "topk_local", 4));
+  CSA_TRY(need_ptr(cand_score, "cand_score", 4));
+  CSA_TRY(need_ptr(cand_idx, "cand_idx", 4));
+  if (n_local < 0 || entry_offset < 0 || entry_offset + n_local > INT32_MAX)
+    return fail(CSA_ERR_INVALID_ARG, "n_local=%lld entry_offset=%lld", (long long)n_local, (long long)entry_offset);
+  const cudaError_t e = launch_shard_candidates(scores, n_local, topk_local, L->B, L->top_k, entry_offset, cand_score,
+                                                cand_idx, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e, "shard candidates launch");
+}
+
+csa_status_t csa_shard_select(const csa_layer_t* L, int32_t shards, const float* cand_score, const int32_t* cand_idx,
+                              int32_t* topk_idx, void* stream) {
+  CSA_TRY(check_layer(L));
+  if (L->kind != CSA_KIND_CSA) return fail(CSA_ERR_INVALID_ARG, "csa_shard_select needs a CSA layer");
+  CSA_TRY(need_ptr(cand_score, "cand_score", 4));
+  CSA_TRY(need_ptr(cand_idx, "cand_idx", 4));
+  CSA_TRY(need_ptr(topk_idx, "topk_idx", 4));
+  if (shards < 1 || (int64_t)shards * L->top_k > 262144) return fail(CSA_ERR_INVALID_ARG, "shards=%d", shards);
+  TopkArgs t;
+  memset(&t, 0, sizeof(t));
+  t.scores = cand_score;
+  t.n_max = (int64_t)shards * L->top_k;
+  t.rows = L->B; t.Tq = 1; t.m = L->m; t.k = L->top_k; t.pos0 = L->pos0;
+  t.out = topk_idx;
+  t.map = cand_idx;
+  t.shards = shards;
+  const cudaError_t e = launch_topk(t, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e, "shard select launch");
+}
+
+csa_status_t csa_sparse_attend_partial(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P,
+                                       const void* q, const int64_t* q_pos, const int32_t* topk_idx,
+                                       int64_t entry_offset, int32_t with_window, float* partial, void* workspace,
+                                       size_t ws_bytes, void* stream) {
+  CSA_TRY(check_layer(L));
+  if (L->kind != CSA_KIND_CSA) return fail(CSA_ERR_INVALID_ARG, "csa_sparse_attend_partial needs a CSA layer");
+  CSA_TRY(check_cache_attend(L, cache));
+  CSA_TRY(check_params(L, P, false));
+  CSA_TRY(need_ptr(q, "q"));
+  CSA_TRY(need_ptr(q_pos, "q_pos", 8));
+  CSA_TRY(need_ptr(topk_idx, "topk_idx", 4));
+  CSA_TRY(need_ptr(partial, "partial", 8));
+  if (entry_offset < 0) return fail(CSA_ERR_INVALID_ARG, "entry_offset=%lld", (long long)entry_offset);
+  if (attend_path(layer_args(L), false, L->B) != 2)
+    return fail(CSA_ERR_UNSUPPORTED, "partial attention needs H=128, D=512, bf16 or mixed rows and B <= 8");
+  const Workspace w = layout(L, CSA_OP_SPARSE_ATTEND, 1, cache->entry_cap);
+  CSA_TRY(check_ws(w, workspace, ws_bytes));
+  AttendArgs a;
+  csa_params_t p = *P;
+  if (!p.sinks) {
+    static const float zero = 0.f;     // not read on this path (no sink in a partial)
+    p.sinks = &zero;
+  }
+  CSA_TRY(make_attend_args(L, cache, &p, q, q_pos, 1, topk_idx, cache->entry_cap, nullptr, w, workspace, a));
+  a.entry_offset = entry_offset;
+  a.entry_limit = cache->entry_cap;
+  a.no_window = with_window ? 0 : 1;
+  a.partial_out = partial;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_attend_qprep(a, s);
+  if (e == cudaSuccess) e = launch_attend(a, s);
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e, "partial attention launch");
+}
+
+csa_status_t csa_attend_merge(const csa_layer_t* L, const csa_params_t* P, const int64_t* q_pos, int32_t parts,
+                              const float* partials, void* out, void* stream) {
+  CSA_TRY(check_layer(L));
+  if (!P) return fail(CSA_ERR_INVALID_ARG, "params is NULL");
+  CSA_TRY(need_ptr(P->sinks, "params.sinks", 4));
+  CSA_TRY(need_ptr(q_pos, "q_pos", 8));
+  CSA_TRY(need_ptr(partials, "partials", 8));
+  CSA_TRY(need_ptr(out, "out"));
+  if (parts < 1) return fail(CSA_ERR_INVALID_ARG, "parts=%d", parts);
+  const LayerArgs la = layer_args(L);
+  const cudaError_t e = launch_attend_merge(la, P->sinks, q_pos, L->B, parts, partials, static_cast<uint8_t*>(out),
+                                            static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA_OK : cuda_fail(e, "attention merge launch");
 }
 
 csa_status_t csa_prefill(const csa_layer_t* L, const csa_cache_t* cache, const csa_params_t* P, const void* q,

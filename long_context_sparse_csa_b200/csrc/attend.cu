@@ -122,7 +122,7 @@ __device__ __forceinline__ SlotInfo slot_info(const AttendArgs& a, int64_t t) {
   const int64_t r1 = s.rt + 1 > 0 ? s.rt + 1 : 0;
   const int64_t nvis = r1 / a.L.m;
   s.n_sel = a.topk ? (int64_t)a.L.top_k : (nvis < a.n_max ? nvis : a.n_max);
-  s.n_win = r1 < a.L.window ? r1 : a.L.window;
+  s.n_win = a.no_window ? 0 : (r1 < a.L.window ? r1 : a.L.window);
   s.R = s.n_sel + s.n_win;
   return s;
 }
@@ -132,8 +132,8 @@ __device__ __forceinline__ const uint8_t* slot_row(const AttendArgs& a, const Sl
                                                    int64_t s) {
   const CacheArgs& C = a.C;
   if (s < si.n_sel) {
-    const int64_t e = a.topk ? (int64_t)a.topk[(size_t)row * a.L.top_k + s] : s;
-    if (e < 0 || e >= C.entry_cap) return nullptr;
+    const int64_t e = a.topk ? (int64_t)a.topk[(size_t)row * a.L.top_k + s] - a.entry_offset : s;
+    if (e < 0 || e >= a.entry_limit) return nullptr;
     return C.entries + ((size_t)b * C.entry_cap + (size_t)e) * a.L.row_bytes;
   }
   if (s < si.R) {
@@ -880,8 +880,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
     auto row_ptr = [&](int r) -> const uint8_t* {
       const int64_t s = s0 + r;
       if (s < si.n_sel) {
-        const int64_t e = a.topk ? (int64_t)sidx[r] : s;
-        if (e < 0 || e >= C.entry_cap) return nullptr;
+        const int64_t e = a.topk ? (int64_t)sidx[r] - a.entry_offset : s;
+        if (e < 0 || e >= a.entry_limit) return nullptr;
         return C.entries + ((size_t)b * C.entry_cap + (size_t)e) * L.row_bytes;
       }
       if (s < si.R) {
@@ -1124,7 +1124,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   ATRACE_T(128, 10);
   tc_fence_after();
   const int e0 = hs * (kTcHalf / 2);
-  if (a.splits > 1) {
+  if (a.splits > 1 || a.partial_out) {
     // partial of this split: O / l in bf16 as [dim / 4][head][4] (a warp's stores are contiguous,
     // the combine reads a head's 4 dims in one 8-byte load), then (m, l) per head in fp32.  O / l
     // is a convex combination of value rows, so its bf16 rounding is no coarser than the output's.
@@ -1240,6 +1240,30 @@ __global__ void __launch_bounds__(512) attend_tc_combine_kernel(const __grid_con
   for (int k = 0; k < 4; ++k) red[g][2 + k][h] = acc[k];
   __syncthreads();
   if (g != 0) return;
+  if (a.partial_out) {
+    // a shard's partial: the splits merged without the sink, O normalised by their total weight
+    float Mp = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) Mp = fmaxf(Mp, red[q][0][h]);
+    float lp = 0.f, op[4] = {0.f, 0.f, 0.f, 0.f};
+    if (Mp != -INFINITY) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float f = red[q][0][h] == -INFINITY ? 0.f : exp2f(red[q][0][h] - Mp);
+        lp += red[q][1][h] * f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) op[k] += red[q][2 + k][h] * f;
+      }
+    }
+    const float inv = lp > 0.f ? 1.f / lp : 0.f;
+    float* pd = a.partial_out + ((size_t)row * L.H + h) * (kD + 2);
+    for (int k = 0; k < 4; ++k) pd[d0 + k] = op[k] * inv;                 // rows of D + 2 floats: 8-byte aligned
+    if (d0 == 0) {
+      pd[kD] = Mp;
+      pd[kD + 1] = lp;
+    }
+    return;
+  }
   const float sk = a.sinks[h] * kLog2e;
   float M = sk;
 #pragma unroll
@@ -1391,7 +1415,7 @@ cudaError_t launch_tc_n(const AttendArgs& a, cudaStream_t s) {
   if (!make_qt_map(&qmap, a.qt, a.rows)) return cudaErrorInvalidValue;
   cudaError_t e = launch_kernel(attend_tc_kernel<FMT, kN>, dim3((unsigned)(2 * a.splits), 1, (unsigned)a.rows),
                                 dim3(kTcThreads), smem, s, 2, qmap, a);
-  if (e != cudaSuccess || a.splits == 1) return e;
+  if (e != cudaSuccess || (a.splits == 1 && !a.partial_out)) return e;
   return launch_kernel(attend_tc_combine_kernel, dim3(kD / 4, a.rows), dim3(4 * kH128), 0, s, 0, a);
 }
 

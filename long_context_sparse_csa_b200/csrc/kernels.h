@@ -133,6 +133,11 @@ struct TopkArgs {
   int64_t pos0;
   const int64_t* q_pos;     // [rows]
   int32_t* out;             // [rows][k]
+  // candidate mode (shard merge): `shards` lists of k candidates per row, laid out [shards][rows][k]
+  // (scores and their global indices `map`, -1 = none); the row's candidates in shard order are in
+  // ascending index order, and out[] gets their indices (ties to the smaller index, ascending)
+  const int32_t* map;
+  int shards;
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 
@@ -170,6 +175,13 @@ struct AttendArgs {
   float* part;              // partials (O, m, l): mma.sync [rows][H/HG][splits][HG*(D+2)] fp32;
                             // tcgen05 [rows][splits] x (bf16 O/l as [D/4][H][4], then (m, l) fp32 per head)
   uint8_t* out;             // [rows][H][D] act
+  // context-sharded decode: the selected indices are global and this cache holds entries
+  // [entry_offset, entry_offset + entry_limit) at slots 0.. (others are skipped); no_window leaves the
+  // window rows to another shard; partial_out (non-null) receives the merged (O/l, m, l) per (row,
+  // head) as [rows][H][D + 2] fp32 (m, l in base 2, no sink, no inverse rotation) instead of `out`
+  int64_t entry_offset, entry_limit;
+  int no_window;
+  float* partial_out;
 };
 // Attention kernel family for a call of `rows` query rows: 2 = tcgen05 (H = 128, D = 512, bf16 or
 // mixed rows, at most kTcMaxRows rows), 1 = mma.sync head groups, 0 = CUDA-core generic kernel.
@@ -184,5 +196,15 @@ size_t attend_partial_bytes(const LayerArgs& L, bool dense, int rows, int splits
 // only q, gamma_q and q_pos, so it may run beside compression.
 cudaError_t launch_attend_qprep(const AttendArgs& a, cudaStream_t s);
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s);
+
+// ----------------------------------------------------------------------------- context-sharded decode
+// Candidates of one shard: (score, global index) of its local top-k, [rows][k].
+cudaError_t launch_shard_candidates(const float* scores, int64_t n_local, const int32_t* topk_local, int rows,
+                                    int k, int64_t entry_offset, float* cand_score, int32_t* cand_idx,
+                                    cudaStream_t s);
+// out[rows][H][D] = merge of `parts` partials [parts][rows][H][D + 2] with the sink and the inverse
+// rotation.
+cudaError_t launch_attend_merge(const LayerArgs& L, const float* sinks, const int64_t* q_pos, int rows, int parts,
+                                const float* partials, uint8_t* out, cudaStream_t s);
 
 }  // namespace csa

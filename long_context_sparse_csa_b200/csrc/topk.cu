@@ -83,23 +83,38 @@ __global__ void __launch_bounds__(kThreads, 1) topk_rows_kernel(const __grid_con
 
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
-  const int64_t t = a.q_pos[row];
-  const int64_t r1 = t - a.pos0 + 1;
-  int64_t nv = r1 > 0 ? r1 / a.m : 0;
-  if (nv > a.n_max) nv = a.n_max;
+  const bool cand = a.map != nullptr;
+  int64_t nv;
+  if (cand) {
+    nv = (int64_t)a.shards * a.k;
+  } else {
+    const int64_t t = a.q_pos[row];
+    const int64_t r1 = t - a.pos0 + 1;
+    nv = r1 > 0 ? r1 / a.m : 0;
+    if (nv > a.n_max) nv = a.n_max;
+  }
   int32_t* out = a.out + (size_t)row * a.k;
   const float* sc = a.scores + (size_t)row * a.n_max;
+  // candidate mode: position i of the row is candidate i % k of shard i / k, stored [shard][row][k]
+  auto flat = [&](int i) -> size_t { return ((size_t)(i / a.k) * a.rows + row) * a.k + (size_t)(i % a.k); };
+  auto value_at = [&](int i) -> int32_t { return cand ? a.map[flat(i)] : i; };
+  // a candidate slot without an entry ranks below every score (key 0)
+  auto raw_key = [&](int i) -> uint32_t {
+    if (!cand) return float_key(__ldg(sc + i));
+    const size_t f = flat(i);
+    return a.map[f] >= 0 ? float_key(__ldg(a.scores + f)) : 0u;
+  };
 
   if (nv <= a.k) {
-    for (int i = tid; i < a.k; i += kThreads) out[i] = i < nv ? i : -1;
+    for (int i = tid; i < a.k; i += kThreads) out[i] = i < nv ? value_at(i) : -1;
     return;
   }
   const int n = (int)nv;
   if (use_smem) {
-    for (int i = tid; i < n; i += kThreads) keys_sm[i] = float_key(sc[i]);
+    for (int i = tid; i < n; i += kThreads) keys_sm[i] = raw_key(i);
     __syncthreads();
   }
-  auto key_at = [&](int i) -> uint32_t { return use_smem ? keys_sm[i] : float_key(__ldg(sc + i)); };
+  auto key_at = [&](int i) -> uint32_t { return use_smem ? keys_sm[i] : raw_key(i); };
 
   // ------------------------------------------------------------------ radix select of the k-th largest key
   uint32_t prefix = 0;        // fixed high bits of T
@@ -124,6 +139,9 @@ __global__ void __launch_bounds__(kThreads, 1) topk_rows_kernel(const __grid_con
     __syncthreads();
   }
   const uint32_t T = prefix;  // exact 32-bit key of the k-th largest score
+  // candidate mode with fewer than k real candidates: the k-th key is that of the empty slots, 0:
+  // take the real ones only and pad the tail with -1
+  if (cand && T == 0u) remaining = 0u;
 
   // ------------------------------------------------------------------ ordered emission
   uint32_t gt_run = 0, eq_run = 0;
@@ -141,11 +159,13 @@ __global__ void __launch_bounds__(kThreads, 1) topk_rows_kernel(const __grid_con
     const uint32_t eq_before = eq_run + (ex >> 16);
     if (gt || (eq && eq_before < remaining)) {
       const uint32_t pos = gt_before + min(eq_before, remaining);
-      out[pos] = i;
+      out[pos] = value_at(i);
     }
     gt_run += tot & 0xFFFFu;
     eq_run += tot >> 16;
   }
+  const uint32_t taken = gt_run + min(eq_run, remaining);
+  for (uint32_t p = taken + tid; p < (uint32_t)a.k; p += kThreads) out[p] = -1;
 }
 
 
@@ -454,8 +474,9 @@ cudaError_t launch_topk_split(const TopkSplitArgs& a, cudaStream_t s) {
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   if (a.rows <= 0 || a.k <= 0) return cudaSuccess;
-  const int use_smem = a.n_max <= kSmemKeys ? 1 : 0;
-  const size_t smem = use_smem ? (size_t)a.n_max * 4 : 0;
+  const int64_t n_row = a.map ? (int64_t)a.shards * a.k : a.n_max;   // keys of a row
+  const int use_smem = n_row <= kSmemKeys ? 1 : 0;
+  const size_t smem = use_smem ? (size_t)n_row * 4 : 0;
   {
     cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(topk_rows_kernel), smem);
     if (e != cudaSuccess) return e;
