@@ -69,8 +69,9 @@ def workload_config(wl, replicas):
 # ----------------------------------------------------------------------------- algorithmic bytes
 
 def index_kernel_bytes(layer, n_vis, B):
-    """Algorithmic bytes of one indexer-score launch: keys + key scales read, scores written, queries."""
-    per_entry = layer.d_I + 4 + 4
+    """Algorithmic bytes of one indexer-score launch: keys + key scales read, scores written, queries
+    (FP4 keys: d_I / 2 bytes of codes and a 4-byte scale word)."""
+    per_entry = (layer.d_I // 2 if layer.idx_format == "e2m1" else layer.d_I) + 4 + 4
     per_query = layer.H_I * layer.d_I + 2 * 4 * layer.H_I
     return B * (n_vis * per_entry + per_query)
 
@@ -83,7 +84,8 @@ def step_bytes(layer, n, B):
     w = min(layer.window, n)
     qo = 2 * layer.H * layer.D * ab
     if layer.kind == "csa":
-        idx = nv * (layer.d_I + 4 + 4) + layer.H_I * layer.d_I
+        kb = layer.d_I // 2 if layer.idx_format == "e2m1" else layer.d_I
+        idx = nv * (kb + 4 + 4) + layer.H_I * layer.d_I
         att = (min(layer.top_k, nv) + w) * rb
         return B * (idx + att + qo)
     return B * ((nv + w) * rb + qo)
@@ -298,14 +300,15 @@ class DecodeRig:
     distinct addresses, so consecutive steps stream different bytes), the step inputs, one
     workspace per layer, and CUDA graphs of whole steps through the C ABI's fused decode calls."""
 
-    def __init__(self, wl, R, dev):
+    def __init__(self, wl, R, dev, indexed=False):
         import torch
         from csa_synth import decode_inputs
+        from long_context_sparse_csa_b200 import binding as C
         from long_context_sparse_csa_b200.state import LayerState, to_device
-        self.wl, self.R, self.dev = wl, R, dev
+        self.wl, self.R, self.dev, self.indexed = wl, R, dev, indexed
         self.datas, self.layers = [], []
         for li, spec in enumerate(wl.layers):
-            d = decode_inputs(wl, li)
+            d = decode_inputs(wl, li, indexed=indexed and spec.kind == "csa")
             self.datas.append(d)
             base = LayerState.from_arrays(spec, wl.B, d, device=dev)
             insts = [base]
@@ -324,9 +327,19 @@ class DecodeRig:
                 io["topk"] = torch.zeros((wl.B, spec.top_k), dtype=torch.int32, device=dev)
             io["out"] = torch.zeros((wl.B, spec.H, spec.D),
                                     dtype=torch.int16 if spec.act_format == "bf16" else torch.float32, device=dev)
-            ws = base.workspace("decode_step", 1, cap)
-            self.layers.append({"spec": spec, "insts": insts, "io": io, "ws": ws,
-                                "caches": [s.cache() for s in insts], "params": base.params(), "L": base.L})
+            ix = indexed and spec.kind == "csa"
+            ws = base.workspace("decode_step_indexed" if ix else "decode_step", 1, cap)
+            lay = {"spec": spec, "insts": insts, "io": io, "ws": ws, "indexed": ix,
+                   "caches": [s.cache() for s in insts], "params": base.params(), "L": base.L}
+            if ix:
+                # the index side made in the step: index-key stream rings per instance, latent and weights
+                for k in ["c_q", "W_iq", "idx_x_new", "idx_g_new"]:
+                    io[k] = to_device(d[k], dev)
+                bias = to_device(np.asarray(d["idx_pos_bias"], np.float32), dev)
+                lay["rings"] = [(to_device(d["idx_raw_ring"], dev), to_device(d["idx_gate_ring"], dev), bias)
+                                for _ in range(R)]
+                lay["streams"] = [C.make_index_stream(*rg) for rg in lay["rings"]]
+            self.layers.append(lay)
         self.stream = torch.cuda.Stream(device=dev)
 
     def call(self, li, r):
@@ -334,7 +347,11 @@ class DecodeRig:
         from long_context_sparse_csa_b200 import binding as C
         lay = self.layers[li]
         io, spec = lay["io"], lay["spec"]
-        if spec.kind == "csa":
+        if spec.kind == "csa" and lay["indexed"]:
+            C.csa_decode_step_indexed(lay["L"], lay["caches"][r], lay["params"], lay["streams"][r], io["q"],
+                                      io["c_q"], io["W_iq"], spec.idx_rank, io["head_w"], io["x_new"], io["g_new"],
+                                      io["idx_x_new"], io["idx_g_new"], io["t"], io["out"], io["topk"], lay["ws"])
+        elif spec.kind == "csa":
             C.csa_decode_step(lay["L"], lay["caches"][r], lay["params"], io["q"], io["idx_q"], io["idx_q_scale"],
                               io["head_w"], io["x_new"], io["g_new"], io["t"], io["out"], io["topk"], lay["ws"])
         else:
@@ -615,6 +632,34 @@ def run_ours(args):
             del cy, si, rig2
             torch.cuda.empty_cache()
         line["configs"] = extra
+
+    # ------------------------------------------------------------------ variants of the 1M CSA layer
+    if args.workload == "csa_hca_decode_1m" and not args.no_extra_configs:
+        from csa_synth.configs import CSA_PRO, scaled_layer
+        variants = {}
+        for name, layer, indexed in [("csa_1m_fp4_keys", scaled_layer(CSA_PRO, idx_format="e2m1"), False),
+                                     ("csa_1m_index_side_in_step", CSA_PRO, True)]:
+            wl2 = get_workload("csa_hca_decode_1m", layers=(layer,))
+            rig2 = DecodeRig(wl2, R, dev, indexed=indexed)
+            rig2.warm()
+            cy, si, _ = rig2.graphs([0], args.steps, idx_events=True)
+            run_steps(cy, si, R, args.warmup)
+            ms = timed(lambda: run_steps(cy, si, R, args.steps), world, dist, dev) / args.steps
+            idx = [c[1][0].elapsed_time(c[1][1]) for c in cy]
+            for lay in rig2.layers:
+                assert C.csa_device_error(lay["ws"]) == 0
+            key_bytes = layer.d_I // 2 + 4 if layer.idx_format == "e2m1" else layer.d_I + 4
+            b = step_bytes(layer, wl2.n, wl2.B)
+            if indexed:
+                b += layer.H_I * layer.d_I * layer.idx_rank * 2 + (1 + layer.ov) * layer.m * layer.d_I * 2 * 2
+            variants[name] = {"us_per_step": 1e3 * ms, "tok_s": wl2.B / (ms / 1e3), "algorithmic_bytes": b,
+                              "hbm_frac": b / (ms / 1e3) / 1e9 / peak, "index_key_bytes_per_entry": key_bytes,
+                              "indexer_launch_us": 1e3 * float(np.mean(idx)),
+                              "indexer_gbs": index_kernel_bytes(layer, wl2.n // layer.m, wl2.B) /
+                              (float(np.mean(idx)) / 1e3) / 1e9}
+            del cy, si, rig2
+            torch.cuda.empty_cache()
+        line["variants"] = variants
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, datas, args.cpu_seconds)
