@@ -9,10 +9,12 @@
 // e4m3 codes with one power-of-two scale (the smallest with max|k| / scale <= 448), or as float32.
 //
 // Index queries: q_h = W_h c for the query's latent c of r values and the learned up-projection W
-// [H_I * d_I][r] (bf16), each head stored as e4m3 codes with its own power-of-two scale.  A CTA takes
-// 16 query rows and one head: four warps split the head's 128 output dims, each runs bf16 mma.sync
-// m16n8k16 over the r inputs (A = the latents, B = W's rows of the head read as a column-major
-// operand, fp32 accumulation), then the CTA reduces the head's max |q| per row for the scale.
+// [H_I * d_I][r] (bf16), each head stored as e4m3 codes with its own power-of-two scale.  A cluster of
+// four CTAs takes 16 query rows and one head, a quarter of the head's output dims each; the warps of
+// a CTA run bf16 mma.sync m16n8k16 over interleaved k-steps of the r inputs (A = the latents, B = W's
+// rows read as a column-major operand, fp32 accumulation), and the cluster reduces the head's max |q|
+// per row for the scale.  In decode (one row) the kernel is a stream over W: H_I * d_I * r * 2 bytes
+// (4 MiB for 32 x 128 x 512), read by 4 H_I SMs with every lane's weight loads in flight.
 #include "kernels.h"
 
 namespace csa {
@@ -20,6 +22,12 @@ namespace csa {
 namespace {
 
 constexpr int kPrepThreads = 128;
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
 
 __device__ __forceinline__ void mma_bf16_16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -127,102 +135,133 @@ __device__ void index_key_token(const IndexPrepArgs& a, int b, int j, float* red
   if (c == 0) a.key_scale[(size_t)b * a.entry_cap + (size_t)i] = sig;
 }
 
-// Rows [16 rt, 16 rt + 16) of head h: q = W_h c, then the head's scale per row and the codes.
-__device__ void index_query_tile(const IndexPrepArgs& a, int rt, int h, float* red) {
+// Rows [16 rt, 16 rt + 16) of head h, output dims [qd dq, qd dq + dq) with dq = d_I / 4.  The head's
+// four quarters are the four CTAs of one cluster, so the head's weights W_h are read by four SMs
+// at once; each CTA computes its quarter of q = W_h c, and the four exchange their per-row max |q|
+// through distributed shared memory so that every quarter is encoded with the head's one scale.
+// Inside the CTA the four warps split the rank's k-steps (warp w takes steps w, w + 4, ...), with
+// many independent weight loads in flight per lane, and add their partial sums in shared memory.
+__device__ void index_query_tile(const IndexPrepArgs& a, int rt, int h, float* part, float* qmax) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, j = lane & 3;
   const int d_I = a.d_I, r = a.rank;
+  const int qd = (int)cluster_rank();
+  const int dq = d_I / 4, nt = dq / 8;                      // 1..4 n-tiles of 8 dims
   const int row0 = 16 * rt + g, row1 = row0 + 8;
-  const int cols = d_I / 4;                                 // this warp's output dims: [warp * cols, +cols)
-  const int nt = cols / 8;                                  // n-tiles of 8
+  const bool ok0 = row0 < a.rows, ok1 = row1 < a.rows;
   const uint16_t* C = reinterpret_cast<const uint16_t*>(a.c);
-  const uint16_t* W = reinterpret_cast<const uint16_t*>(a.W) + (size_t)h * d_I * r;
-  float acc[4][4];                                          // up to 4 n-tiles (d_I <= 128)
+  const uint16_t* W = reinterpret_cast<const uint16_t*>(a.W) + ((size_t)h * d_I + (size_t)qd * dq) * r;
+  // the cluster's first phase: arrive now, wait before the first remote store (every CTA has started)
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  float acc[4][4];
 #pragma unroll
   for (int n = 0; n < 4; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-  for (int k0 = 0; k0 < r; k0 += 16) {
+  const int ksteps = r / 16;
+#pragma unroll 8
+  for (int st = warp; st < ksteps; st += 4) {
+    const int k0 = 16 * st;
     uint32_t af[4];
-    af[0] = row0 < a.rows ? *reinterpret_cast<const uint32_t*>(C + (size_t)row0 * r + k0 + 2 * j) : 0u;
-    af[1] = row1 < a.rows ? *reinterpret_cast<const uint32_t*>(C + (size_t)row1 * r + k0 + 2 * j) : 0u;
-    af[2] = row0 < a.rows ? *reinterpret_cast<const uint32_t*>(C + (size_t)row0 * r + k0 + 8 + 2 * j) : 0u;
-    af[3] = row1 < a.rows ? *reinterpret_cast<const uint32_t*>(C + (size_t)row1 * r + k0 + 8 + 2 * j) : 0u;
+    af[0] = ok0 ? __ldg(reinterpret_cast<const uint32_t*>(C + (size_t)row0 * r + k0 + 2 * j)) : 0u;
+    af[1] = ok1 ? __ldg(reinterpret_cast<const uint32_t*>(C + (size_t)row1 * r + k0 + 2 * j)) : 0u;
+    af[2] = ok0 ? __ldg(reinterpret_cast<const uint32_t*>(C + (size_t)row0 * r + k0 + 8 + 2 * j)) : 0u;
+    af[3] = ok1 ? __ldg(reinterpret_cast<const uint32_t*>(C + (size_t)row1 * r + k0 + 8 + 2 * j)) : 0u;
 #pragma unroll
     for (int n = 0; n < 4; ++n) {
       if (n < nt) {
-        const uint16_t* wr = W + (size_t)(warp * cols + 8 * n + g) * r + k0 + 2 * j;
+        const uint16_t* wr = W + (size_t)(8 * n + g) * r + k0 + 2 * j;
         mma_bf16_16816(acc[n], af, __ldg(reinterpret_cast<const uint32_t*>(wr)),
                        __ldg(reinterpret_cast<const uint32_t*>(wr + 8)));
       }
     }
   }
-  // acc[n][0..1]: row0, dims warp*cols + 8n + 2j (+1); acc[n][2..3]: row1
-  float m0 = 0.f, m1 = 0.f;
+  // acc[n][0..1]: row g, dims 8n + 2j (+1); acc[n][2..3]: row g + 8.  Partial sums -> [warp][row][32]
 #pragma unroll
-  for (int n = 0; n < 4; ++n)
+  for (int n = 0; n < 4; ++n) {
     if (n < nt) {
-      m0 = fmaxf(m0, fmaxf(fabsf(acc[n][0]), fabsf(acc[n][1])));
-      m1 = fmaxf(m1, fmaxf(fabsf(acc[n][2]), fabsf(acc[n][3])));
+      const int d = 8 * n + 2 * j;
+      part[(warp * 16 + g) * 32 + d] = acc[n][0];
+      part[(warp * 16 + g) * 32 + d + 1] = acc[n][1];
+      part[(warp * 16 + g + 8) * 32 + d] = acc[n][2];
+      part[(warp * 16 + g + 8) * 32 + d + 1] = acc[n][3];
     }
-#pragma unroll
-  for (int o = 1; o < 4; o <<= 1) {
-    m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
-    m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
-  }
-  if (j == 0) {
-    red[warp * 16 + g] = m0;
-    red[warp * 16 + g + 8] = m1;
   }
   __syncthreads();
-  const float am0 = fmaxf(fmaxf(red[g], red[16 + g]), fmaxf(red[32 + g], red[48 + g]));
-  const float am1 = fmaxf(fmaxf(red[g + 8], red[16 + g + 8]), fmaxf(red[32 + g + 8], red[48 + g + 8]));
-  float inv0 = 1.f, inv1 = 1.f, sg0 = 1.f, sg1 = 1.f;
-  const bool f32 = a.idx_fmt == CSA_FMT_F32;
-  if (!f32) {
-    sg0 = pow2_scale(am0, &inv0);
-    sg1 = pow2_scale(am1, &inv1);
-  }
+  // thread t: row t / 8 of the tile, dims 4 (t % 8) .. + 4 of the quarter
+  const int tr = threadIdx.x >> 3, td = 4 * (threadIdx.x & 7);
+  const bool mine = td < dq;                                // dq is a multiple of 8: all 4 dims or none
+  float v[4], mx = 0.f;
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int row = half ? row1 : row0;
-    if (row >= a.rows) continue;
-    const float inv = half ? inv1 : inv0;
-    uint8_t* q = a.q_out + ((size_t)row * a.H_I + h) * (size_t)d_I * (f32 ? 4 : 1);
+  for (int e = 0; e < 4; ++e) {
+    v[e] = 0.f;
+    if (mine) {
 #pragma unroll
-    for (int n = 0; n < 4; ++n) {
-      if (n >= nt) continue;
-      const int d = warp * cols + 8 * n + 2 * j;
-      const float v0 = acc[n][2 * half], v1 = acc[n][2 * half + 1];
-      if (f32) {
-        *reinterpret_cast<float2*>(q + 4 * (size_t)d) = make_float2(v0, v1);
-      } else {
-        *reinterpret_cast<uint16_t*>(q + d) =
-            (uint16_t)((uint32_t)f_to_e4m3_sat(v0 * inv) | ((uint32_t)f_to_e4m3_sat(v1 * inv) << 8));
-      }
+      for (int w = 0; w < 4; ++w) v[e] += part[(w * 16 + tr) * 32 + td + e];
     }
-    if (warp == 0 && j == 0) a.q_scale_out[(size_t)row * a.H_I + h] = half ? sg1 : sg0;
+    mx = fmaxf(mx, fabsf(v[e]));
   }
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+  if ((threadIdx.x & 7) == 0) {
+    const uint32_t local = (uint32_t)__cvta_generic_to_shared(qmax + qd * 16 + tr);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      uint32_t remote;
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(p));
+      asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(mx) : "memory");
+    }
+  }
+  // release our stores to the peers, acquire theirs; no remote access follows, so a CTA may exit
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+  const float am = fmaxf(fmaxf(qmax[tr], qmax[16 + tr]), fmaxf(qmax[32 + tr], qmax[48 + tr]));
+  const int row = 16 * rt + tr;
+  if (row >= a.rows) return;
+  const bool f32 = a.idx_fmt == CSA_FMT_F32;
+  float inv = 1.f, sg = 1.f;
+  if (!f32) sg = pow2_scale(am, &inv);
+  uint8_t* q = a.q_out + ((size_t)row * a.H_I + h) * (size_t)d_I * (f32 ? 4 : 1);
+  const int d = qd * dq + td;
+  if (mine) {
+    if (f32) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) reinterpret_cast<float*>(q)[d + e] = v[e];
+    } else {
+      uint32_t w = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) w |= (uint32_t)f_to_e4m3_sat(v[e] * inv) << (8 * e);
+      *reinterpret_cast<uint32_t*>(q + d) = w;
+    }
+  }
+  if (qd == 0 && td == 0) a.q_scale_out[(size_t)row * a.H_I + h] = sg;
 }
 
-// Blocks [0, key_blocks) compress index keys (one token each); the rest project index queries
-// (one (16-row tile, head) each).
+// Blocks [0, key_blocks) compress index keys (one token each; the count is rounded up to whole
+// clusters when queries follow); the rest project index queries, one cluster of four CTAs per
+// (16-row tile, head).
 __global__ void __launch_bounds__(kPrepThreads) index_prep_kernel(const __grid_constant__ IndexPrepArgs a) {
   __shared__ float red[64];
+  __shared__ float part[4 * 16 * 32];
+  __shared__ float qmax[4 * 16];
   const int blk = blockIdx.x;
   if (blk < a.key_blocks) {
-    index_key_token(a, blk / a.Tq, blk % a.Tq, red);
+    if (a.keys && blk < a.B * a.Tq) index_key_token(a, blk / a.Tq, blk % a.Tq, red);
     return;
   }
-  const int q = blk - a.key_blocks;
-  index_query_tile(a, q / a.H_I, q % a.H_I, red);
+  const int q = (blk - a.key_blocks) >> 2;
+  index_query_tile(a, q / a.H_I, q % a.H_I, part, qmax);
 }
 
 }  // namespace
 
 cudaError_t launch_index_prep(IndexPrepArgs a, cudaStream_t s) {
+  const int q_blocks = a.c ? ((a.rows + 15) / 16) * a.H_I * 4 : 0;
   a.key_blocks = a.keys ? a.B * a.Tq : 0;
-  const int q_blocks = a.c ? ((a.rows + 15) / 16) * a.H_I : 0;
+  if (q_blocks) a.key_blocks = (a.key_blocks + 3) & ~3;    // whole clusters of four
   if (a.key_blocks + q_blocks == 0) return cudaSuccess;
-  return launch_kernel(index_prep_kernel, dim3((unsigned)(a.key_blocks + q_blocks)), dim3(kPrepThreads), 0, s, 0, a);
+  return launch_kernel(index_prep_kernel, dim3((unsigned)(a.key_blocks + q_blocks)), dim3(kPrepThreads), 0, s,
+                       q_blocks ? 4 : 0, a);
 }
 
 }  // namespace csa

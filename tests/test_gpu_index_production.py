@@ -81,7 +81,7 @@ def test_index_keys_from_a_chunk(fmt, n):
         assert not got[b, N:].any(), "entries past the last complete group are not written"
 
 
-@pytest.mark.parametrize("rows,rank,H_I", [(37, 512, 32), (1, 1536, 16), (8, 128, 64)])
+@pytest.mark.parametrize("rows,rank,H_I", [(37, 512, 32), (1, 1536, 16), (8, 128, 64), (3, 48, 8)])
 def test_index_query_projection(rows, rank, H_I):
     layer = scaled_layer(CSA_PRO, H_I=H_I, idx_rank=rank)
     L = C.layer_from_spec(layer, 1)
