@@ -18,8 +18,22 @@
 // store the fp32 scores (coalesced).
 // Decode streams the keys once from HBM; it is a bandwidth-bound kernel whose
 // MMA keeps the 64 FLOP/byte of 32 heads off the CUDA cores.
+//
+// FP4 keys (e2m1 codes with a power-of-two key scale and per-32-dim block offsets, "DeepSeek-V4:
+// Making a Million Tokens Affordable", "Two ways to shrink attention, interleaved": the indexer's
+// attention runs in FP4) take the same pipeline at half the key bytes.  The tensor memory
+// accelerator reads a tile's packed codes (64 bytes per key) and writes them 16 codes to a 16-byte
+// chunk (8 bytes of codes, 8 of gap), so the shared-memory tile has the FP8 tile's 128-byte rows and
+// swizzle; a second copy brings the tile's 128 scale words.  The MMA is kind::mxf8f6f4.block_scale
+// with A = e2m1 keys and B = e4m3 queries: each 32-dim block of a key carries its own E8M0 scale,
+// sigma * 2^-delta_b, which is exactly the key format's block scale, so the accumulator holds
+// sigma_k * <q, k> and the epilogue is the FP8 one with a key scale of 1.  The MMA warp turns the
+// scale words into the block-scale matrices (one per K-block of 32 dims: key l's scale in TMEM lane
+// l % 32 of every 32-lane quarter, column l / 32) in shared memory and copies them into TMEM with
+// tcgen05.cp ahead of the tile's MMAs; the query side's scales are all 1 (E8M0 127).
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "kernels.h"
@@ -36,6 +50,10 @@ constexpr int kTileE = 128;                 // entries per tile (MMA M)
 constexpr int kDI = 128;                    // index-key bytes per entry
 constexpr int kTileBytes = kTileE * kDI;    // 16 KB
 constexpr int kThreads = 192;               // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kSfBytes = 512;               // FP4: 128 scale words of a tile; one 32 x 16 B scale matrix
+// FP4 shared memory past the key ring: [stages][128] scale words, [stages][4][512] block-scale
+// matrices, the query-scale matrix (1 KB slot, keeping the query tiles 1024-byte aligned)
+__host__ __device__ constexpr size_t fp4_extra_smem(int stages) { return (size_t)stages * 5 * kSfBytes + 1024; }
 
 __device__ __forceinline__ int64_t n_visible(const IndexArgs& a, int b, int j) {
   const int64_t t = a.q_pos[(int64_t)b * a.Tq + j];
@@ -186,11 +204,17 @@ __device__ __forceinline__ GroupConsts load_group_consts(const IndexArgs& a, int
 }
 
 // Issues the key-scale loads of items [k0, k0 + kKsChunk) for entry lane e_loc (0 past the end).
+// FP4 keys carry their scales into the MMA: the epilogue's key scale is 1.
+template <bool kFP4>
 __device__ __forceinline__ void load_key_scales(const IndexArgs& a, const Sched& sc, int64_t k0, int e_loc,
                                                 float ks[kKsChunk]) {
 #pragma unroll
   for (int u = 0; u < kKsChunk; ++u) {
     ks[u] = 0.f;
+    if (kFP4) {
+      ks[u] = 1.f;
+      continue;
+    }
     if (k0 + u < sc.count) {
       int64_t g;
       int et;
@@ -202,15 +226,19 @@ __device__ __forceinline__ void load_key_scales(const IndexArgs& a, const Sched&
 }
 
 // kHI > 0: decode specialisation (one query per group, kHI index heads, head weights in registers);
-// kHI == 0: any QN x H_I (prefill).
-template <int kStages, int kHI>
+// kHI == 0: any QN x H_I (prefill).  kFP4: e2m1 keys with block scales (smap: their scale words).
+template <int kStages, int kHI, bool kFP4>
 __global__ void __launch_bounds__(kThreads, 2)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
-                      const __grid_constant__ IndexArgs a, int N, int nacc, uint32_t tmem_cols) {
+                      const __grid_constant__ CUtensorMap smap, const __grid_constant__ IndexArgs a, int N,
+                      int nacc, uint32_t tmem_cols) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* A = smem;                                  // [kStages][kTileBytes]
-  uint8_t* Bq = A + kStages * kTileBytes;             // [2][N * 128]
+  uint8_t* SFw = A + kStages * kTileBytes;            // FP4: [kStages][128] key scale words
+  uint8_t* SFs = SFw + kStages * kSfBytes;            // FP4: [kStages][4 K-blocks][32 x 16 B] block scales
+  uint8_t* SFq = SFs + kStages * 4 * kSfBytes;        // FP4: the query side's block scales (all 1)
+  uint8_t* Bq = kFP4 ? A + kStages * kTileBytes + fp4_extra_smem(kStages) : A + kStages * kTileBytes;  // [2][N * 128]
   Barriers* bars = reinterpret_cast<Barriers*>(Bq + 2 * N * kDI);
   EpiSmem* es = reinterpret_cast<EpiSmem*>(reinterpret_cast<uint8_t*>(bars) + ((sizeof(Barriers) + 15) & ~size_t(15)));
 
@@ -228,7 +256,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     int et;
     sc.at(0, &g, &et);
     gc0 = load_group_consts(a, g, te);
-    load_key_scales(a, sc, 0, e_loc, ks_cur);
+    load_key_scales<kFP4>(a, sc, 0, e_loc, ks_cur);
   }
 
   if (threadIdx.x == 0) {
@@ -238,6 +266,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     fence_barrier_init();
     prefetch_tensormap(&kmap);
     prefetch_tensormap(&qmap);
+    if (kFP4) prefetch_tensormap(&smap);
   }
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, tmem_cols);
@@ -302,9 +331,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       }
       if (!wait_all(&bars->empty[stage], phase ^ 1u)) { ok = false; break; }
       if (lane == 0) {
-        mbar_arrive_expect_tx(&bars->full[stage], (uint32_t)kTileBytes);
+        // FP4: the box's packed codes are half its shared-memory footprint, plus the scale words
+        mbar_arrive_expect_tx(&bars->full[stage], kFP4 ? (uint32_t)(kTileBytes / 2 + kSfBytes) : (uint32_t)kTileBytes);
         tma_load_2d(A + stage * kTileBytes, &kmap, &bars->full[stage], 0,
                     (int)((int64_t)G.b * a.entry_cap + (int64_t)et * kTileE));
+        if (kFP4) tma_load_2d(SFw + stage * kSfBytes, &smap, &bars->full[stage], et * kTileE, G.b);
         if (k < 16) TRACE(2 + k);
       }
       __syncwarp();
@@ -319,7 +350,19 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       if (b_issued_par[s] >= 0) wait_all(&bars->bfull[s], (uint32_t)b_issued_par[s]);
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    const uint32_t idesc = instr_desc(128, N, 0u);
+    const uint32_t idesc = kFP4 ? instr_desc_block_scaled(128, N, 5u, 0u) : instr_desc(128, N, 0u);
+    // FP4: TMEM columns [sfa0 + 16 acc, + 16) hold accumulator acc's key block scales (4 columns per
+    // K-block), [sfq, sfq + 4) the query side's (all 1: E8M0 127)
+    const uint32_t sfa0 = ((uint32_t)(nacc * N) + 15u) & ~15u;
+    const uint32_t sfq = sfa0 + 16u * (uint32_t)nacc;
+    // (copied into TMEM just before the first MMA, so that every copy is followed by an MMA whose
+    // completion the end of the loop waits for)
+    bool sfq_copied = false;
+    if (kFP4) {
+      reinterpret_cast<uint4*>(SFq)[lane] = make_uint4(0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+      fence_proxy_async_smem();
+      __syncwarp();
+    }
     int stage = 0, acc = 0, gi = -1;
     uint32_t phase = 0, acc_phase = 0;
     Group G;
@@ -353,13 +396,49 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         sc.at(k + 1, &gn, &etn);
         last_of_group = gn != g || etn > G.last_et;
       }
+      uint8_t* sfs = SFs + stage * 4 * kSfBytes;
+      if (kFP4) {
+        // scale words of keys l, 32 + l, 64 + l, 96 + l -> row l of each K-block's block-scale matrix:
+        // E8M0 of sigma * 2^-delta_kk = (exponent byte) - delta_kk
+        const uint32_t* raw = reinterpret_cast<const uint32_t*>(SFw + stage * kSfBytes);
+        uint32_t wv[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) wv[c] = raw[32 * c + lane];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          uint32_t o[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int e8 = (int)(wv[c] & 0xFFu) - (int)((wv[c] >> (8 + 4 * kk)) & 0xFu);
+            o[c] = (uint32_t)(e8 > 0 ? e8 : 0) * 0x01010101u;
+          }
+          reinterpret_cast<uint4*>(sfs + kk * kSfBytes)[lane] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
       if (lane == 0) {
         tc_fence_after();
         const uint64_t ad = desc_kmajor_sw128(smem_u32(A + stage * kTileBytes));
         const uint64_t bd = desc_kmajor_sw128(smem_u32(Bq + slot * N * kDI));
+        if (kFP4) {
+          const uint32_t sfa = tmem + sfa0 + 16u * (uint32_t)acc;
+          if (!sfq_copied) {
+            tmem_cp_32x128b_x4(tmem + sfq, desc_noswizzle(smem_u32(SFq), 128u));
+            sfq_copied = true;
+          }
 #pragma unroll
-        for (int kk = 0; kk < kDI / 32; ++kk)
-          umma_f8f6f4(tmem + (uint32_t)(acc * N), ad + 2u * kk, bd + 2u * kk, idesc, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kDI / 32; ++kk)
+            tmem_cp_32x128b_x4(sfa + 4u * kk, desc_noswizzle(smem_u32(sfs + kk * kSfBytes), 128u));
+#pragma unroll
+          for (int kk = 0; kk < kDI / 32; ++kk)
+            umma_mxf8f6f4(tmem + (uint32_t)(acc * N), ad + 2u * kk, bd + 2u * kk, idesc, sfa + 4u * kk, tmem + sfq,
+                          kk > 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < kDI / 32; ++kk)
+            umma_f8f6f4(tmem + (uint32_t)(acc * N), ad + 2u * kk, bd + 2u * kk, idesc, kk > 0 ? 1u : 0u);
+        }
         umma_commit(&bars->empty[stage]);
         umma_commit(&bars->tfull[acc]);
         if (last_of_group) umma_commit(&bars->bempty[slot]);
@@ -445,7 +524,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
 #pragma unroll
       for (int u = 0; u < kKsChunk; ++u) es->ks[u][e_loc] = ks_cur[u];
       const bool more = k0 + kKsChunk < sc.count;
-      if (more) load_key_scales(a, sc, k0 + kKsChunk, e_loc, ks_nxt);
+      if (more) load_key_scales<kFP4>(a, sc, k0 + kKsChunk, e_loc, ks_nxt);
       const int kn = (int)min((int64_t)kKsChunk, sc.count - k0);
       for (int u = 0; u < kn; ++u) {
         const int64_t k = k0 + u;
@@ -640,6 +719,35 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// FP4 keys [rows][64 bytes] (128 e2m1 codes each) as 128 x 128 boxes: the codes land 16 to a 16-byte
+// chunk (8 bytes of codes, then 8 of gap), rows of 128 bytes in the 128-byte swizzle.  Needs a
+// 32-byte aligned base.
+bool make_map_fp4(CUtensorMap* m, const void* base, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kDI, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(kDI / 2)};
+  cuuint32_t box[2] = {(cuuint32_t)kDI, (cuuint32_t)kTileE};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// FP4 scale words [B][entry_cap] (uint32) as boxes of 128 words of one sequence, zero past entry_cap.
+// Needs entry_cap a multiple of 4 (16-byte row pitch) and a 16-byte aligned base.
+bool make_scale_map(CUtensorMap* m, const void* base, uint64_t entry_cap, uint64_t B) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)entry_cap, (cuuint64_t)B};
+  cuuint64_t strides[1] = {(cuuint64_t)(entry_cap * 4)};
+  cuuint32_t box[2] = {(cuuint32_t)kTileE, 1};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 #ifdef CSA_TRACE
@@ -652,14 +760,41 @@ bool index_tc_supported(int idx_fmt, int H_I, int d_I) {
   return idx_fmt == CSA_FMT_E4M3 && d_I == kDI && (H_I == 16 || H_I == 32 || H_I == 64);
 }
 
+namespace {
+
+// FP4 keys on the tensor-core kernel: d_I = 128, 16 or 32 heads (two CTAs per SM fit the extra
+// shared memory), a scale-word pitch the tensor memory accelerator can step (entry_cap a multiple of
+// 4), and the base alignments its boxes need.
+bool index_tc_fp4_ok(const IndexArgs& a) {
+  return a.idx_fmt == CSA_FMT_E2M1 && a.d_I == kDI && (a.H_I == 16 || a.H_I == 32) && a.entry_cap % 4 == 0 &&
+         (reinterpret_cast<uintptr_t>(a.idx_k) & 31u) == 0 && (reinterpret_cast<uintptr_t>(a.k_scale) & 15u) == 0;
+}
+
+template <bool kFP4>
+using TcKernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, IndexArgs, int, int, uint32_t);
+
+template <bool kFP4>
+TcKernel<kFP4> tc_kernel(bool decode, int H_I) {
+  if (!decode) return index_score_tc_kernel<2, 0, kFP4>;
+  if (H_I == 16) return index_score_tc_kernel<4, 16, kFP4>;
+  if constexpr (kFP4) {
+    return index_score_tc_kernel<4, 32, kFP4>;            // FP4 takes 16 or 32 heads
+  } else {
+    if (H_I == 32) return index_score_tc_kernel<4, 32, kFP4>;
+    return index_score_tc_kernel<4, 64, kFP4>;
+  }
+}
+
+}  // namespace
+
 cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
   if (a.n_max <= 0 || a.Tq <= 0 || a.B <= 0) return cudaSuccess;
-  // decode with FP4 keys: the warp-level streaming kernel (it also fills the top-k's histogram); FP8
-  // decode keys take the tcgen05 kernel below, measured faster on the 1M-token step (20.5 against
-  // 28 us per launch)
-  if (a.Tq == 1 && a.idx_fmt == CSA_FMT_E2M1 && index_decode_supported(a.idx_fmt, a.H_I, a.d_I))
+  const bool fp4 = index_tc_fp4_ok(a);
+  // FP4 keys the tensor-core kernel does not take: the warp-level streaming kernel in decode (it also
+  // fills the top-k's histogram), else the CUDA-core kernel below
+  if (a.idx_fmt == CSA_FMT_E2M1 && !fp4 && a.Tq == 1 && index_decode_supported(a.idx_fmt, a.H_I, a.d_I))
     return launch_index_decode(a, num_sms, s);
-  if (!index_tc_supported(a.idx_fmt, a.H_I, a.d_I)) {
+  if (!fp4 && !index_tc_supported(a.idx_fmt, a.H_I, a.d_I)) {
     dim3 grid((unsigned)((a.n_max + 127) / 128), (unsigned)(a.B * a.Tq));
     const size_t sm = (size_t)a.H_I * a.d_I * sizeof(float);
     if (sm > 0) {
@@ -668,35 +803,46 @@ cudaError_t launch_index_scores(IndexArgs a, int num_sms, cudaStream_t s) {
     }
     return launch_kernel(index_score_generic_kernel, grid, dim3(128), sm, s, 0, a);
   }
-  a.QN = a.Tq == 1 ? 1 : min(256 / a.H_I, a.Tq);
+  // FP4 prefill tiles hold at most 128 query columns, so the accumulator and the block-scale columns
+  // fit the CTA's 256 TMEM columns
+  a.QN = a.Tq == 1 ? 1 : min((fp4 ? 128 : 256) / a.H_I, a.Tq);
   const int N = a.QN * a.H_I;
   a.tiles_per_group = (int)((a.n_max + kTileE - 1) / kTileE);
   a.groups_per_seq = (a.Tq + a.QN - 1) / a.QN;
   a.total_items = (int64_t)a.B * a.groups_per_seq * a.tiles_per_group;
-  CUtensorMap kmap, qmap;
-  if (!make_map(&kmap, a.idx_k, (uint64_t)a.B * a.entry_cap, kTileE)) return cudaErrorInvalidValue;
+  CUtensorMap kmap, qmap, smap;
+  memset(&smap, 0, sizeof(smap));
+  if (fp4) {
+    if (!make_map_fp4(&kmap, a.idx_k, (uint64_t)a.B * a.entry_cap)) return cudaErrorInvalidValue;
+    if (!make_scale_map(&smap, a.k_scale, (uint64_t)a.entry_cap, (uint64_t)a.B)) return cudaErrorInvalidValue;
+  } else if (!make_map(&kmap, a.idx_k, (uint64_t)a.B * a.entry_cap, kTileE)) {
+    return cudaErrorInvalidValue;
+  }
   if (!make_map(&qmap, a.idx_q, (uint64_t)a.B * a.Tq * a.H_I, (uint32_t)N)) return cudaErrorInvalidValue;
   const bool decode = a.Tq == 1;
   // two CTAs per SM in both modes (two independent pipelines, twice the epilogue warps); their TMEM
   // shares the SM's 512 columns: decode 4 accumulators of N <= 64 columns, prefill one of N = 256
+  // (FP4: N <= 128, plus 16 block-scale columns per accumulator and 4 for the query side)
   const int nacc = decode ? 4 : 1;
+  const uint32_t need = fp4 ? (((uint32_t)(nacc * N) + 15u) & ~15u) + 16u * (uint32_t)nacc + 4u : (uint32_t)(nacc * N);
   uint32_t cols = 32;
-  while (cols < (uint32_t)(nacc * N)) cols <<= 1;
+  while (cols < need) cols <<= 1;
   const int stages = decode ? 4 : 2;
-  const size_t smem = 1024 + (size_t)stages * kTileBytes + 2 * (size_t)N * kDI + ((sizeof(Barriers) + 15) & ~size_t(15)) +
-                     (decode ? sizeof(EpiSmem) : kEpiSmemNoHist) + 64;
-  const int ki = !decode ? 0 : a.H_I == 16 ? 1 : a.H_I == 32 ? 2 : 3;
-  auto kern = ki == 0 ? index_score_tc_kernel<2, 0>
-            : ki == 1 ? index_score_tc_kernel<4, 16>
-            : ki == 2 ? index_score_tc_kernel<4, 32>
-                      : index_score_tc_kernel<4, 64>;
+  const size_t smem = 1024 + (size_t)stages * kTileBytes + (fp4 ? fp4_extra_smem(stages) : 0) + 2 * (size_t)N * kDI +
+                      ((sizeof(Barriers) + 15) & ~size_t(15)) + (decode ? sizeof(EpiSmem) : kEpiSmemNoHist) + 64;
+  const void* kern = fp4 ? reinterpret_cast<const void*>(tc_kernel<true>(decode, a.H_I))
+                         : reinterpret_cast<const void*>(tc_kernel<false>(decode, a.H_I));
   {
-    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
+    cudaError_t e = ensure_dynamic_smem(kern, smem);
     if (e != cudaSuccess) return e;
   }
   const int64_t ctas = 2 * (int64_t)num_sms;
   const int64_t grid = a.total_items < ctas ? a.total_items : ctas;
-  return launch_kernel(kern, dim3((unsigned)grid), dim3(kThreads), smem, s, 0, kmap, qmap, a, N, nacc, cols);
+  if (fp4)
+    return launch_kernel(tc_kernel<true>(decode, a.H_I), dim3((unsigned)grid), dim3(kThreads), smem, s, 0, kmap, qmap,
+                         smap, a, N, nacc, cols);
+  return launch_kernel(tc_kernel<false>(decode, a.H_I), dim3((unsigned)grid), dim3(kThreads), smem, s, 0, kmap, qmap,
+                       smap, a, N, nacc, cols);
 }
 
 }  // namespace csa

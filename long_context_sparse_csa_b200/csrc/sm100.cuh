@@ -102,6 +102,25 @@ __device__ __forceinline__ void umma_f8f6f4(uint32_t d_tmem, uint64_t adesc, uin
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T with one scale per 32 elements of K for every row of A and of B
+// (kind::mxf8f6f4.block_scale, E8M0 scales read from TMEM at sfa_tmem / sfb_tmem), fp32 accumulate.
+__device__ __forceinline__ void umma_mxf8f6f4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+
+// Copies a matrix of 32 rows x 16 bytes from shared memory into TMEM lanes 0..31, four 32-bit columns
+// from taddr, and the same into each of the other three 32-lane quarters (tcgen05.cp 32x128b.warpx4).
+// Ordered with the issuing thread's later tcgen05.mma.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, bf16/f16 inputs (kind::f16), fp32 accumulate.
 __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t accumulate) {
@@ -178,6 +197,18 @@ __device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t 
   return d;
 }
 
+// Shared-memory matrix descriptor without swizzle: rows of 16 bytes, each 8-row core matrix 128
+// contiguous bytes, consecutive core matrices along the rows `sbo` bytes apart (one core matrix
+// across, so the leading offset is unused).
+__device__ __forceinline__ uint64_t desc_noswizzle(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(128u >> 4) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;                      // descriptor version for sm_100; layout 0: no swizzle
+  return d;
+}
+
 // Makes this thread's generic-proxy writes to shared memory visible to the tensor core (async proxy).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -190,6 +221,16 @@ __host__ __device__ constexpr uint32_t instr_desc(int M, int N, uint32_t ab_form
          | (ab_format << 7)          // A format
          | (ab_format << 10)         // B format
          | ((uint32_t)(N >> 3) << 17)
+         | ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor of kind::mxf8f6f4.block_scale: M x N tile, fp32 accumulator, both operands
+// K-major, E8M0 scale factors, scale-factor ids 0.  Formats: 0 = e4m3, 5 = e2m1.
+__host__ __device__ constexpr uint32_t instr_desc_block_scaled(int M, int N, uint32_t a_format, uint32_t b_format) {
+  return (a_format << 7)               // A format
+         | (b_format << 10)            // B format
+         | ((uint32_t)(N >> 3) << 17)
+         | (1u << 23)                  // scale format E8M0
          | ((uint32_t)(M >> 4) << 24);
 }
 

@@ -42,7 +42,9 @@ def _scores_ref(layer, d, b):
     return O.index_scores(iq, d["idx_q_scale"][b], d["head_w"][b], ik, iks)
 
 
-@pytest.mark.parametrize("B,n", [(2, 4 * 20000 + 3), (3, 4 * 3000 + 1), (1, 1 << 20)])
+# entry counts that are multiples of 4 take the tensor-core kernel (block-scaled MMA); 20,001 entries
+# take the warp-level kernel
+@pytest.mark.parametrize("B,n", [(2, 4 * 20000 + 3), (3, 4 * 3000 + 1), (1, 1 << 20), (2, 4 * 20001 + 1)])
 def test_fp4_index_topk(B, n):
     wl = Workload(name="t", mode="decode", B=B, n=n, layers=(FP4_PRO,), seed=51)
     d = decode_inputs(wl)
@@ -159,13 +161,16 @@ def test_fp4_indexed_decode_step():
         assert_out_close(got[b], ref["o"], tag=f"fp4 indexed b{b}")
 
 
-def test_fp4_prefill_small():
-    # chunked prefill with FP4 keys: the CUDA-core indexer path, then top-k and attention
+@pytest.mark.parametrize("prefix", [4096 + 2, 4096 + 6])
+def test_fp4_prefill_small(prefix):
+    # chunked prefill with FP4 keys, then top-k and attention: 1,048 entries (a multiple of 4) take the
+    # tensor-core indexer, 1,049 the CUDA-core one
     layer = scaled_layer(CSA_PREFILL, idx_format="e2m1")
     wl = get_workload("csa_prefill_8k", layers=(layer,))
-    pf = prefill_inputs(wl, Tq=97, prefix=4096 + 2)
+    pf = prefill_inputs(wl, Tq=97, prefix=prefix)
     st = LayerState.from_arrays(layer, 1, pf, raw_key="raw", gate_key="gate", raw_base=pf["raw_first_row"])
     n_max = pf["n"] // layer.m
+    assert st.idx_keys.shape[1] % 4 == (0 if prefix == 4098 else 1)
     out = torch.zeros((1, 97, layer.H, layer.D), dtype=torch.int16, device="cuda")
     topk = torch.zeros((1, 97, layer.top_k), dtype=torch.int32, device="cuda")
     ws = st.workspace("prefill", 97, n_max)
