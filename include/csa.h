@@ -449,6 +449,15 @@ CSA_API csa_status_t csa_decode_step_scratch(const csa_layer_t* L, const csa_cac
                              void* out, int32_t* topk_idx, int32_t* device_error,
                              void* stream);
 
+/* Test aid for csa_decode_step_scratch (no counterpart on the pages): copies `bytes` bytes between
+ * `buf` (host or device memory) and the current device's static scratch at byte `offset`, in the
+ * direction `to_scratch` (1: buf -> scratch, 0: scratch -> buf), on `stream`, and synchronises it.
+ * Offsets of the scratch's segments are those csa_debug_workspace_segment gives for the decode step.
+ * Lets a test plant a device error and dirty histograms in the scratch.  A range outside the
+ * CSA_SCRATCH_BYTES array returns CSA_ERR_INVALID_ARG with no device work. */
+CSA_API csa_status_t csa_debug_scratch_copy(size_t offset, void* buf, size_t bytes, int32_t to_scratch,
+                                            void* stream);
+
 /* One fused HCA decode step: csa_append -> csa_compress -> hca_attend. */
 CSA_API csa_status_t hca_decode_step(const csa_layer_t* L, const csa_cache_t* cache,
                              const csa_params_t* P, const void* q,

@@ -85,6 +85,7 @@ _SIGS = {
     "csa_debug_workspace_segment": (ctypes.c_int, [_LAYER, _I32, _I32, _I64, _I32, ctypes.POINTER(_SZ),
                                                    ctypes.POINTER(_SZ)]),
     "csa_debug_wait_probe": (ctypes.c_int, [_P, _SZ, ctypes.c_uint64, _P]),
+    "csa_debug_scratch_copy": (ctypes.c_int, [_SZ, _P, _SZ, _I32, _P]),
     "csa_index_keys": (ctypes.c_int, [_LAYER, _CACHE, _STREAM_S, _P, _P, _P, _I32, _P]),
     "csa_index_query": (ctypes.c_int, [_LAYER, _P, _P, _I32, _I32, _P, _P, _P]),
     "csa_decode_step_indexed": (ctypes.c_int, [_LAYER, _CACHE, _PARAMS, _STREAM_S, _P, _P, _P, _I32, _P, _P, _P, _P,
@@ -234,6 +235,12 @@ def csa_debug_wait_probe(workspace, limit_ns, stream=None):
                                       _stream(stream)))
 
 
+def csa_debug_scratch_copy(offset, buf, to_scratch, stream=None):
+    """Copy between a tensor and the static scratch at byte `offset` (test aid; synchronises)."""
+    _check(lib().csa_debug_scratch_copy(int(offset), ptr(buf), buf.numel() * buf.element_size(),
+                                        1 if to_scratch else 0, _stream(stream)))
+
+
 def csa_append(L, cache, x_new, g_new, q_pos, Tq, stream=None):
     _check(lib().csa_append(ctypes.byref(L), ctypes.byref(cache), ptr(x_new), ptr(g_new), ptr(q_pos), Tq,
                             _stream(stream)))
@@ -276,10 +283,13 @@ def csa_decode_step_scratch(L, cache, params, q, idx_q, idx_q_scale, head_w, x_n
     """csa_decode_step on the library's static device scratch (no workspace argument).  With
     read_device_error the call synchronises and returns the device error word (else None)."""
     code = _I32(0)
-    _check(lib().csa_decode_step_scratch(ctypes.byref(L), ctypes.byref(cache), ctypes.byref(params), ptr(q),
-                                         ptr(idx_q), ptr(idx_q_scale), ptr(head_w), ptr(x_new), ptr(g_new),
-                                         ptr(q_pos), ptr(out), ptr(topk_idx),
-                                         ctypes.byref(code) if read_device_error else None, _stream(stream)))
+    st = lib().csa_decode_step_scratch(ctypes.byref(L), ctypes.byref(cache), ctypes.byref(params), ptr(q),
+                                       ptr(idx_q), ptr(idx_q_scale), ptr(head_w), ptr(x_new), ptr(g_new),
+                                       ptr(q_pos), ptr(out), ptr(topk_idx),
+                                       ctypes.byref(code) if read_device_error else None, _stream(stream))
+    if read_device_error and st == 5:      # CSA_ERR_DEVICE_TIMEOUT: the device error word is the result
+        return code.value
+    _check(st)
     return code.value if read_device_error else None
 
 

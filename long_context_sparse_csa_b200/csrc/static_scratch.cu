@@ -101,3 +101,21 @@ extern "C" CSA_API csa_status_t csa_decode_step_scratch(const csa_layer_t* L, co
   }
   return st;
 }
+
+extern "C" CSA_API csa_status_t csa_debug_scratch_copy(size_t offset, void* buf, size_t bytes, int32_t to_scratch,
+                                                       void* stream) {
+  if (bytes == 0) return CSA_OK;
+  if (!buf) return csa::report_error(CSA_ERR_INVALID_ARG, "buf is NULL");
+  if (offset > kScratchBytes || bytes > kScratchBytes - offset)
+    return csa::report_error(CSA_ERR_INVALID_ARG, "range outside the static scratch");
+  void* ws = nullptr;
+  csa_status_t st = scratch_address(&ws);
+  if (st != CSA_OK) return st;
+  unsigned char* p = static_cast<unsigned char*>(ws) + offset;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = to_scratch ? cudaMemcpyAsync(p, buf, bytes, cudaMemcpyDefault, s)
+                             : cudaMemcpyAsync(buf, p, bytes, cudaMemcpyDefault, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return csa::report_error(CSA_ERR_CUDA, cudaGetErrorString(e));
+  return CSA_OK;
+}
