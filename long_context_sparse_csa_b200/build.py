@@ -19,7 +19,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libcsa.so")
 TRACE_LIB = os.path.join(HERE, "libcsa_trace.so")
 
-SOURCES = ["compress.cu", "index_score.cu", "topk.cu", "attend.cu", "api.cu", "static_scratch.cu", "debug.cu", "index_decode.cu", "index_prep.cu", "shard.cu"]
+SOURCES = ["compress.cu", "index_score.cu", "topk.cu", "attend.cu", "api.cu", "static_scratch.cu", "debug.cu", "index_decode.cu", "index_prep.cu", "shard.cu", "attend_prefill.cu"]
 HEADERS = ["common.cuh", "sm100.cuh", "kernels.h"]
 
 NVCC_FLAGS = [

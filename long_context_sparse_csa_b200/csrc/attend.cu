@@ -1333,10 +1333,13 @@ int attend_path(const LayerArgs& L, bool dense, int rows) {
   // than the mma.sync kernel over every SM and than 9 pairs of 128.  That kernel gives every query
   // one CTA pair per slot tile and a partial per tile, so calls with many query rows (chunked
   // prefill) take the mma.sync kernel, which needs no split there; so do other head counts.
+  // Chunked prefill with 64 heads of bf16 rows takes the persistent tcgen05 kernel that computes the
+  // transposed products (keys, then dims, as the MMA's M; attend_prefill.cu).
   (void)dense;
   if (rows <= kTcMaxRows && L.H == kH128 && L.D == kD && L.d_rope == 64 &&
       (L.kv_fmt == CSA_FMT_BF16 || L.kv_fmt == CSA_FMT_MIXED))
     return 2;
+  if (attend_prefill_tc_supported(L, rows)) return 3;
   return attend_head_group(L) > 0 ? 1 : 0;
 }
 
@@ -1349,6 +1352,7 @@ int attend_head_group(const LayerArgs& L) {
 }
 
 int attend_num_splits(const LayerArgs& L, bool dense, int rows, int64_t slots, int num_sms) {
+  if (attend_path(L, dense, rows) == 3) return 1;
   if (attend_path(L, dense, rows) == 2) {
     const int n = dense ? kTcN : kTcNSparse;
     const int64_t s = (slots + n - 1) / n;
@@ -1427,8 +1431,10 @@ cudaError_t launch_tc(const AttendArgs& a, cudaStream_t s) {
 
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
   if (a.rows <= 0) return cudaSuccess;
-  if (attend_path(a.L, a.topk == nullptr, a.rows) == 2)
+  const int path = attend_path(a.L, a.topk == nullptr, a.rows);
+  if (path == 2)
     return a.L.kv_fmt == CSA_FMT_MIXED ? launch_tc<CSA_FMT_MIXED>(a, s) : launch_tc<CSA_FMT_BF16>(a, s);
+  if (path == 3) return launch_attend_prefill_tc(a, s);
   const int HG = attend_head_group(a.L);
   if (HG == 0) {
     return launch_kernel(attend_generic_kernel, dim3(a.rows), dim3(a.L.H * 32), 0, s, 0, a);

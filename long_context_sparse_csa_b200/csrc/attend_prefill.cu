@@ -1,0 +1,578 @@
+// Chunked-prefill attention on the tensor cores (tcgen05): many query rows, 64 query heads sharing one
+// KV head of 512 dims stored in bf16.  What it computes is the shared-KV multi-query attention with a
+// sink of "DeepSeek-V4: Making a Million Tokens Affordable", section "Two ways to shrink attention,
+// interleaved" (keys are also the values, q~ = RoPE_t(RMSNorm(q) * gamma_q), the output rotated back
+// by -t), over each query's own key slots: its top-k entries (CSA) or every visible entry (HCA), then
+// its window rows.
+//
+// Every query gathers its own keys, so the contraction is per query: S = q~ K^T (64 heads x R keys x
+// 512 dims), then O = P K.  Sixty-four heads fill only half of the 128-row MMA, so the kernel computes
+// the transposes, with the keys (then the dims) as the MMA's M:
+//   S^T[key, h]  = sum_d K[key, d] q~[h, d]    A = a 128-key tile of rows (K-major, 8 blocks of 64
+//                                              dims), B = q~ (K-major); M = 128, N = 64; TMEM [0, 64)
+//   O^T[d, h]   += sum_key K[key, d] P[key, h]  A = the same tile read dims-major (M-tile mt = dims
+//                                              128 mt ..), B = P (heads-major); TMEM [256 + 64 mt, +64)
+// and the online softmax over keys in between.  A softmax thread owns one key (its TMEM lane) and holds
+// that key's 64 head scores; the tile's per-head maxima come from a butterfly reduce-scatter across the
+// warp (each lane ends with heads 2l and 2l + 1) and shared memory across the four warps.  A head's
+// running maximum moves only when its tile maximum exceeds it by more than 8 (in log2 units); then
+// O^T's column and the partial sums are rescaled.  Exponentials are taken against the running maximum,
+// so they stay below 2^8.  Each softmax thread keeps its key's partial sums per head; they are reduced
+// once per query, in the epilogue.
+//
+// Roles, in one persistent CTA per SM (query rows strided by the grid):
+//   warp 0      the MMA issuer (one thread)
+//   warps 1-4   softmax; then per query the epilogue: 1 / (l + 2^(sink - m)), the rotation by -t,
+//               the bf16 store
+//   warps 5-6   loaders: q~ of each query (one head per thread: RMSNorm, gamma, the rotation by +t,
+//               bf16), then its key tiles, two key rows per thread, in 16-byte cp.async pieces into
+//               the 128-byte-swizzled tile, block by block.  A 64-dim block is refilled for the next tile as soon as the
+//               O^T MMAs that read it are done, while the other M-tiles still run.
+// Every mbarrier wait is bounded: a wait that gives up sets the device error word, and the role stops.
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace csa {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 512;
+constexpr int kHeads = 64;                    // query heads (MMA N)
+constexpr int kKeys = 128;                    // keys per tile (MMA M of S^T)
+constexpr int kBlocks = 8;                    // 64-dim column blocks of a row
+constexpr int kBlockBytes = kKeys * 128;      // one block of the key tile: 16 KB
+constexpr int kQBlockBytes = kHeads * 128;    // one block of q~: 8 KB
+constexpr int kThreads = 224;                 // warp 0 MMA, warps 1-4 softmax, warps 5-6 loaders
+constexpr int kLoaders = 64;
+constexpr float kRescale = 8.f;               // log2 margin before a running maximum moves
+
+struct __align__(8) PfBars {
+  uint64_t kvfull[kBlocks], kvfree[kBlocks];
+  uint64_t qfull, qfree, sfull, pfull, ofull, ofree, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// shared memory: key tile 128 KB, q~ 64 KB, P 16 KB, then the small arrays
+constexpr size_t kOffQ = (size_t)kBlocks * kBlockBytes;
+constexpr size_t kOffP = kOffQ + (size_t)kBlocks * kQBlockBytes;
+constexpr size_t kOffMx = kOffP + (size_t)kKeys * 128;
+constexpr size_t kOffBars = kOffMx + (4 * kHeads + 3 * kHeads + 4) * sizeof(float);
+constexpr size_t kSmemBytes = 1024 + kOffBars + sizeof(PfBars);
+static_assert(kSmemBytes <= 227 * 1024, "prefill attention shared memory");
+
+#ifdef CSA_TRACE
+// Diagnostic build only: per-CTA timestamps (ns) of the first tiles and queries.
+__device__ uint64_t g_trace_p[160][160];
+#define PTRACE(slot) do { if (blockIdx.x < 160 && (slot) < 160) g_trace_p[blockIdx.x][(slot)] = global_timer_ns(); } while (0)
+#else
+#define PTRACE(slot) ((void)0)
+#endif
+
+// An empty key slot is filled from this zero row, so that every piece of a tile is a cp.async whose
+// landing the block's barrier tracks.
+__device__ __align__(16) uint8_t g_zero_row[kD * 2];
+
+__device__ __forceinline__ uint32_t sw128(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+// Arrives on the mbarrier (without raising its expected count) once this thread's earlier cp.async
+// copies have landed.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void softmax_bar() { asm volatile("barrier.sync.aligned 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  return (uint32_t)f_to_bf16_bits(lo) | ((uint32_t)f_to_bf16_bits(hi) << 16);
+}
+
+// Key slots of the query at position t: [0, n_sel) entries, [n_sel, R) window rows.
+struct Slots {
+  int64_t rt, n_sel, n_win, R;
+  int tiles;
+};
+
+__device__ __forceinline__ Slots slots_of(const AttendArgs& a, int64_t t) {
+  Slots s;
+  s.rt = t - a.L.pos0;
+  const int64_t r1 = s.rt + 1 > 0 ? s.rt + 1 : 0;
+  const int64_t nvis = r1 / a.L.m;
+  s.n_sel = a.topk ? (int64_t)a.L.top_k : (nvis < a.n_max ? nvis : a.n_max);
+  s.n_win = r1 < a.L.window ? r1 : a.L.window;
+  s.R = s.n_sel + s.n_win;
+  const int64_t nt = (s.R + kKeys - 1) / kKeys;
+  s.tiles = nt < 1 ? 1 : (int)nt;               // at least one (all-masked) tile: every role walks it
+  return s;
+}
+
+// Stored row of slot s of query `row` (sequence b), or null for an empty slot (-1, out of range).
+__device__ __forceinline__ const uint8_t* slot_ptr(const AttendArgs& a, const Slots& si, int row, int b, int64_t s) {
+  const CacheArgs& C = a.C;
+  if (s < si.n_sel) {
+    const int64_t e = a.topk ? (int64_t)__ldg(a.topk + (size_t)row * a.L.top_k + s) : s;
+    if (e < 0 || e >= C.entry_cap) return nullptr;
+    return C.entries + ((size_t)b * C.entry_cap + (size_t)e) * a.L.row_bytes;
+  }
+  if (s < si.R) {
+    const int64_t wr = si.rt - si.n_win + 1 + (s - si.n_sel);
+    return C.window + ((size_t)b * C.window_cap + (size_t)(wr % C.window_cap)) * a.L.row_bytes;
+  }
+  return nullptr;
+}
+
+// Butterfly reduce-scatter of sums across the warp, 64 values per lane: lane l ends with the sums of
+// entries 2l and 2l + 1 in v[0], v[1].
+__device__ __forceinline__ void reduce_scatter_sum64(float v[64], int lane) {
+#pragma unroll
+  for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < n; ++j) {
+      const float send = upper ? v[j] : v[j + n];
+      const float keep = upper ? v[j + n] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t x, uint32_t y) {
+  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&x), b = *reinterpret_cast<__nv_bfloat162*>(&y);
+  __nv_bfloat162 r = __hmax2(a, b);
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// The same for maxima of 64 values held as 32 bf16 pairs (rounding to nearest is monotonic, so the
+// result is the rounded maximum): lane l ends with the maxima of entries 2l, 2l + 1 in w[0].  The
+// maximum is only the softmax's reference point, so its rounding is immaterial.
+__device__ __forceinline__ void reduce_scatter_max64(uint32_t w[32], int lane) {
+#pragma unroll
+  for (int o = 16, n = 16; o >= 1; o >>= 1, n >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < n; ++j) {
+      const uint32_t send = upper ? w[j] : w[j + n];
+      const uint32_t keep = upper ? w[j + n] : w[j];
+      w[j] = bf16x2_max(keep, __shfl_xor_sync(0xffffffffu, send, o));
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __grid_constant__ AttendArgs a) {
+  extern __shared__ uint8_t pf_smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* KV = sm;                                             // [8 blocks][128 keys][128 B]
+  uint8_t* Q = sm + kOffQ;                                      // [8 blocks][64 heads][128 B]
+  uint8_t* P = sm + kOffP;                                      // [128 keys][64 heads] bf16, swizzled
+  float* mx = reinterpret_cast<float*>(sm + kOffMx);            // [4 warps][64]: tile maxima / sums
+  float* mrun = mx + 4 * kHeads;                                // [64] running maxima (log2 units)
+  float* alph = mrun + kHeads;                                  // [64] rescale factors of this tile
+  float* fh = alph + kHeads;                                    // [64] output factors (epilogue)
+  int* flag = reinterpret_cast<int*>(fh + kHeads);              // [1] any head rescaled
+  PfBars* bars = reinterpret_cast<PfBars*>(sm + kOffBars);
+
+  const LayerArgs& L = a.L;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int c = 0; c < kBlocks; ++c) {
+      mbar_init(&bars->kvfull[c], kLoaders);
+      mbar_init(&bars->kvfree[c], 1);
+    }
+    mbar_init(&bars->qfull, kLoaders);
+    mbar_init(&bars->qfree, 1);
+    mbar_init(&bars->sfull, 1);
+    mbar_init(&bars->pfull, 128);
+    mbar_init(&bars->ofull, 1);
+    mbar_init(&bars->ofree, 128);
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const float cl2 = L.scale * kLog2e;
+  if (tid == 0) PTRACE(95);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = instr_desc(kKeys, kHeads, 1u);                          // both K-major
+      const uint32_t idesc_o = instr_desc(128, kHeads, 1u) | (1u << 15) | (1u << 16);  // both MN-major
+      bool ok = true;
+      uint32_t g = 0, j = 0;
+      bool issued = false;
+      for (int row = blockIdx.x; row < a.rows && ok; row += gridDim.x, ++j) {
+        const Slots si = slots_of(a, a.q_pos[row]);
+        if (!mbar_wait(&bars->qfull, j & 1u)) { ok = false; break; }
+        for (int i = 0; i < si.tiles; ++i, ++g) {
+          // S^T = K q~^T over the 8 blocks of this tile, as each block lands
+          for (int c = 0; c < kBlocks; ++c) {
+            if (!mbar_wait(&bars->kvfull[c], g & 1u)) { ok = false; break; }
+            fence_proxy_async_smem();                 // the loaders' copies, for the tensor core
+            tc_fence_after();
+            const uint64_t ad = desc_kmajor_sw128(smem_u32(KV + c * kBlockBytes));
+            const uint64_t bd = desc_kmajor_sw128(smem_u32(Q + c * kQBlockBytes));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) umma_f16(tmem, ad + 2u * kk, bd + 2u * kk, idesc_s, (c | kk) ? 1u : 0u);
+            issued = true;
+          }
+          if (!ok) break;
+          umma_commit(&bars->sfull);
+          if (g < 16) PTRACE(g);
+          if (i + 1 == si.tiles) umma_commit(&bars->qfree);
+          // O^T += K^T P once the softmax has written P (and rescaled O^T where needed); the first tile
+          // of a query overwrites O^T once the previous query's epilogue has read it
+          if (!mbar_wait(&bars->pfull, g & 1u)) { ok = false; break; }
+          if (g < 16) PTRACE(96 + g);
+          if (i == 0 && !mbar_wait(&bars->ofree, (j & 1u) ^ 1u)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+            for (int kk = 0; kk < kKeys / 16; ++kk) {
+              const uint64_t ad = desc_mnmajor_sw128(smem_u32(KV + 2 * mt * kBlockBytes + kk * 2048), kBlockBytes, 1024u);
+              const uint64_t bd = desc_mnmajor_sw128(smem_u32(P + kk * 2048), kBlockBytes, 1024u);
+              umma_f16(tmem + 256u + 64u * (uint32_t)mt, ad, bd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&bars->kvfree[2 * mt]);
+            umma_commit(&bars->kvfree[2 * mt + 1]);
+            if (mt == 0 && g < 16) PTRACE(112 + g);
+          }
+          if (g < 16) PTRACE(16 + g);
+        }
+        if (!ok) break;
+        umma_commit(&bars->ofull);
+      }
+      if (!ok) {
+        set_device_error(a.err, kErrWaitTimeout);
+        atomicExch(&bars->abort, 1);
+      }
+      // nothing of this thread is in flight when TMEM is released
+      if (issued) {
+        umma_commit(&bars->drain);
+        mbar_wait(&bars->drain, 0u);
+      }
+    }
+    __syncwarp();
+  } else if (warp <= 4) {
+    // ------------------------------------------------------------------ softmax and epilogue
+    const int w4 = warp & 3;                                  // TMEM lane quarter of this warp
+    const int key = w4 * 32 + lane;                           // key of S^T, dim of O^T's M-tile
+    const uint32_t lane_addr = tmem + ((uint32_t)(w4 * 32) << 16);
+    bool ok = true;
+    uint32_t g = 0, j = 0;
+    for (int row = blockIdx.x; row < a.rows && ok; row += gridDim.x, ++j) {
+      const int64_t t = a.q_pos[row];
+      const Slots si = slots_of(a, t);
+      const int b = row / a.Tq;
+      float lp[kHeads];                                       // this key's partial sums per head
+#pragma unroll
+      for (int h = 0; h < kHeads; ++h) lp[h] = 0.f;
+      if (key < kHeads) mrun[key] = -INFINITY;
+      softmax_bar();
+      for (int i = 0; i < si.tiles; ++i, ++g) {
+        const int64_t s = (int64_t)i * kKeys + key;
+        const bool valid = slot_ptr(a, si, row, b, s) != nullptr;
+        if (!mbar_wait(&bars->sfull, g & 1u)) { ok = false; break; }
+        if (tid == 32 && g < 16) PTRACE(32 + g);
+        tc_fence_after();
+        float z[kHeads];
+        tmem_ld_32x32b_x32(lane_addr, z);
+        tmem_ld_32x32b_x32(lane_addr + 32u, z + 32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < kHeads; ++h) z[h] = valid ? z[h] * cl2 : -INFINITY;
+        // the tile's maxima per head: lanes, then warps
+        {
+          uint32_t w[kHeads / 2];
+#pragma unroll
+          for (int q = 0; q < kHeads / 2; ++q) w[q] = pack_bf16x2(z[2 * q], z[2 * q + 1]);
+          reduce_scatter_max64(w, lane);
+          mx[w4 * kHeads + 2 * lane] = bf16_bits_to_f(w[0] & 0xFFFFu);
+          mx[w4 * kHeads + 2 * lane + 1] = bf16_bits_to_f(w[0] >> 16);
+        }
+        softmax_bar();
+        if (w4 == 0) {
+          int moved = 0;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int h = 2 * lane + u;
+            const float tm = fmaxf(fmaxf(mx[h], mx[kHeads + h]), fmaxf(mx[2 * kHeads + h], mx[3 * kHeads + h]));
+            const float mr = mrun[h];
+            float al = 1.f;
+            if (tm > mr + kRescale || (mr == -INFINITY && tm > -INFINITY)) {
+              al = mr == -INFINITY ? 0.f : exp2f(mr - tm);
+              mrun[h] = tm;
+              moved = 1;
+            }
+            alph[h] = al;
+          }
+          moved = __any_sync(0xffffffffu, moved);
+          if (lane == 0) flag[0] = moved;
+        }
+        softmax_bar();
+        // P = 2^(z - m) in bf16, this key's row of P; the partial sums (rescaled where the head's maximum
+        // moved) take the rounded values
+        const bool moved = flag[0] != 0;
+        uint8_t* prow = P;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          uint32_t w[4];
+          float mm[8], aa[8];
+          *reinterpret_cast<float4*>(mm) = reinterpret_cast<const float4*>(mrun)[2 * jj];
+          *reinterpret_cast<float4*>(mm + 4) = reinterpret_cast<const float4*>(mrun)[2 * jj + 1];
+          if (moved) {
+            *reinterpret_cast<float4*>(aa) = reinterpret_cast<const float4*>(alph)[2 * jj];
+            *reinterpret_cast<float4*>(aa + 4) = reinterpret_cast<const float4*>(alph)[2 * jj + 1];
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int h = 8 * jj + 2 * q;
+            const float m0 = mm[2 * q], m1 = mm[2 * q + 1];
+            const float p0 = m0 == -INFINITY ? 0.f : exp2f(z[h] - m0);
+            const float p1 = m1 == -INFINITY ? 0.f : exp2f(z[h + 1] - m1);
+            w[q] = pack_bf16x2(p0, p1);
+            if (moved) {
+              lp[h] *= aa[2 * q];
+              lp[h + 1] *= aa[2 * q + 1];
+            }
+            lp[h] += bf16_bits_to_f(w[q] & 0xFFFFu);
+            lp[h + 1] += bf16_bits_to_f(w[q] >> 16);
+          }
+          *reinterpret_cast<uint4*>(prow + sw128(key, jj)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        // rescale O^T, the previous tiles' sum (complete, as this tile's S^T is), where a maximum moved
+        if (moved && i > 0) {
+#pragma unroll 1
+          for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll 1
+            for (int hc = 0; hc < kHeads; hc += 32) {
+              float o[32];
+              tmem_ld_32x32b_x32(lane_addr + 256u + 64u * mt + hc, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int u = 0; u < 32; ++u) o[u] *= alph[hc + u];
+              tmem_st_32x32b_x32(lane_addr + 256u + 64u * mt + hc, o);
+            }
+          }
+          tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bars->pfull);
+        if (tid == 32 && g < 16) PTRACE(48 + g);
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------------- epilogue of this query
+      reduce_scatter_sum64(lp, lane);
+      mx[w4 * kHeads + 2 * lane] = lp[0];
+      mx[w4 * kHeads + 2 * lane + 1] = lp[1];
+      softmax_bar();
+      if (w4 == 0) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int h = 2 * lane + u;
+          const float l = (mx[h] + mx[kHeads + h]) + (mx[2 * kHeads + h] + mx[3 * kHeads + h]);
+          const float m = mrun[h];
+          const float sk = a.sinks[h] * kLog2e;
+          // o = O / (l + 2^(sink - m)), O and l relative to the running maximum m
+          fh[h] = m == -INFINITY ? 0.f : 1.f / (l + exp2f(sk - m));
+        }
+      }
+      softmax_bar();
+      if (!mbar_wait(&bars->ofull, j & 1u)) { ok = false; break; }
+      tc_fence_after();
+      // per M-tile: this thread's dim of all heads -> a [64 heads][128 dims] bf16 staging tile in P's
+      // buffer (free: the query's last P.V is done), then 16-byte coalesced stores of the heads' rows
+      uint8_t* out = a.out + (size_t)row * kHeads * kD * 2;
+      uint16_t* stage = reinterpret_cast<uint16_t*>(P);
+#pragma unroll 1
+      for (int mt = 0; mt < 4; ++mt) {
+        const int d = mt * 128 + key;
+        float c = 1.f, sn = 0.f;
+        const bool rot = d >= kD - 64;
+        if (rot) rope_cos_sin((double)t, (d - (kD - 64)) >> 1, L, &c, &sn);
+#pragma unroll
+        for (int hc = 0; hc < kHeads; hc += 32) {
+          float o[32];
+          tmem_ld_32x32b_x32(lane_addr + 256u + 64u * mt + hc, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            float v = o[u] * fh[hc + u];
+            // rotation by -t of the pair (d even, d + 1): partner in the neighbouring lane
+            const float pv = __shfl_xor_sync(0xffffffffu, v, 1);
+            if (rot) v = (d & 1) ? (-pv * sn + v * c) : (v * c + pv * sn);
+            stage[(hc + u) * 128 + key] = f_to_bf16_bits(v);
+          }
+        }
+        if (mt == 3) {                                        // every O^T column read: release it
+          tc_fence_before();
+          mbar_arrive(&bars->ofree);
+        }
+        softmax_bar();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int ch = k * 128 + key, hh = ch >> 4, part = ch & 15;
+          *reinterpret_cast<uint4*>(out + ((size_t)hh * kD + mt * 128) * 2 + part * 16) =
+              *reinterpret_cast<const uint4*>(P + hh * 256 + part * 16);
+        }
+        softmax_bar();
+      }
+      if (tid == 32 && j < 8) PTRACE(80 + j);
+    }
+    if (!ok) {
+      set_device_error(a.err, kErrWaitTimeout);
+      atomicExch(&bars->abort, 1);
+    }
+  } else {
+    // ------------------------------------------------------------------ loaders (q~, then key tiles)
+    const int lt = tid - 160;                                 // 0..63: q~ head lt; key rows lt, lt + 64
+    bool ok = true;
+    uint32_t g = 0, j = 0;
+    for (int row = blockIdx.x; row < a.rows && ok; row += gridDim.x, ++j) {
+      const int64_t t = a.q_pos[row];
+      const Slots si = slots_of(a, t);
+      const int b = row / a.Tq;
+      // q~ of this query once the previous query's S^T MMAs are done with q~: the raw head row lands in
+      // its q~ slots (all of its copies in flight at once), then is normalised and rotated in place
+      if (!mbar_wait(&bars->qfree, (j & 1u) ^ 1u)) { ok = false; break; }
+      {
+        const int h = lt;
+        const uint8_t* src = a.q + ((size_t)row * kHeads + h) * kD * 2;
+#pragma unroll 8
+        for (int p = 0; p < 64; ++p) cp_async16(Q + (p >> 3) * kQBlockBytes + sw128(h, p & 7), src + 16 * p);
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        float ss = 0.f;
+#pragma unroll 8
+        for (int p = 0; p < 64; ++p) {
+          const uint4 u = *reinterpret_cast<const uint4*>(Q + (p >> 3) * kQBlockBytes + sw128(h, p & 7));
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float x0 = bf16_bits_to_f(w[q] & 0xFFFFu), x1 = bf16_bits_to_f(w[q] >> 16);
+            ss = fmaf(x0, x0, fmaf(x1, x1, ss));
+          }
+        }
+        const float rs = 1.0f / sqrtf(ss / (float)kD + L.eps);
+#pragma unroll 2
+        for (int p = 0; p < 64; ++p) {
+          const int d0 = 8 * p;
+          uint4* slot = reinterpret_cast<uint4*>(Q + (p >> 3) * kQBlockBytes + sw128(h, p & 7));
+          const uint4 u = *slot;
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+          float v[8];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            v[2 * q] = bf16_bits_to_f(w[q] & 0xFFFFu);
+            v[2 * q + 1] = bf16_bits_to_f(w[q] >> 16);
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] *= rs * (a.gamma_q ? __ldg(a.gamma_q + d0 + e) : 1.f);
+          if (d0 >= kD - 64) {
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              float c, sn;
+              rope_cos_sin((double)t, (d0 + e - (kD - 64)) >> 1, L, &c, &sn);
+              const float x0 = v[e], x1 = v[e + 1];
+              v[e] = x0 * c - x1 * sn;
+              v[e + 1] = x0 * sn + x1 * c;
+            }
+          }
+          *slot = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                             pack_bf16x2(v[6], v[7]));
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->qfull);
+        if (tid == 160 && j < 8) PTRACE(88 + j);
+      }
+      // key tiles: rows lt and lt + 64 of each, block by block as the blocks come free; each block's
+      // copies arrive on its barrier when they land, so all free blocks are in flight at once
+      for (int i = 0; i < si.tiles && ok; ++i, ++g) {
+        const uint8_t* src[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) src[r] = slot_ptr(a, si, row, b, (int64_t)i * kKeys + lt + 64 * r);
+        for (int c = 0; c < kBlocks; ++c) {
+          if (!mbar_wait(&bars->kvfree[c], (g & 1u) ^ 1u)) { ok = false; break; }
+          if (tid == 160 && g < 16 && c == 0) PTRACE(128 + g);
+          if (tid == 160 && g < 16 && c == 7) PTRACE(144 + g);
+          uint8_t* dst = KV + c * kBlockBytes;
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int kr = lt + 64 * r;
+            const uint8_t* from = src[r] ? src[r] + c * 128 : g_zero_row + c * 128;
+#pragma unroll
+            for (int p = 0; p < 8; ++p) cp_async16(dst + sw128(kr, p), from + p * 16);
+          }
+          cp_async_arrive(&bars->kvfull[c]);
+        }
+        if (tid == 160 && g < 16) PTRACE(64 + g);
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (!ok) {
+      set_device_error(a.err, kErrWaitTimeout);
+      atomicExch(&bars->abort, 1);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+#ifdef CSA_TRACE
+}  // namespace
+extern "C" __attribute__((visibility("default"))) int csa_trace_read_p(uint64_t* host) {
+  return (int)cudaMemcpyFromSymbol(host, g_trace_p, sizeof(g_trace_p));
+}
+namespace {
+#endif
+
+int device_sms() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static int cached[64] = {0};
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+}  // namespace
+
+bool attend_prefill_tc_supported(const LayerArgs& L, int rows) {
+  return rows > kTcMaxRows && L.H == kHeads && L.D == kD && L.d_rope == 64 && L.kv_fmt == CSA_FMT_BF16 &&
+         L.act_fmt == CSA_FMT_BF16;
+}
+
+cudaError_t launch_attend_prefill_tc(const AttendArgs& a, cudaStream_t s) {
+  if (a.rows <= 0) return cudaSuccess;
+  {
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(attend_prefill_tc_kernel), kSmemBytes);
+    if (e != cudaSuccess) return e;
+  }
+  const int sms = device_sms();
+  const int grid = a.rows < sms ? a.rows : sms;
+  return launch_kernel(attend_prefill_tc_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, 0, a);
+}
+
+}  // namespace csa

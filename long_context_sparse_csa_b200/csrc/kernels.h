@@ -184,7 +184,8 @@ struct AttendArgs {
   float* partial_out;
 };
 // Attention kernel family for a call of `rows` query rows: 2 = tcgen05 (H = 128, D = 512, bf16 or
-// mixed rows, at most kTcMaxRows rows), 1 = mma.sync head groups, 0 = CUDA-core generic kernel.
+// mixed rows, at most kTcMaxRows rows), 3 = persistent tcgen05 prefill kernel (H = 64, D = 512, bf16
+// rows and activations, more than kTcMaxRows rows), 1 = mma.sync head groups, 0 = CUDA-core generic.
 // `dense`: every visible entry (HCA) rather than a top-k list.
 constexpr int kTcMaxRows = 8;
 int attend_path(const LayerArgs& L, bool dense, int rows);
@@ -196,6 +197,8 @@ size_t attend_partial_bytes(const LayerArgs& L, bool dense, int rows, int splits
 // only q, gamma_q and q_pos, so it may run beside compression.
 cudaError_t launch_attend_qprep(const AttendArgs& a, cudaStream_t s);
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s);
+bool attend_prefill_tc_supported(const LayerArgs& L, int rows);
+cudaError_t launch_attend_prefill_tc(const AttendArgs& a, cudaStream_t s);
 
 // ----------------------------------------------------------------------------- context-sharded decode
 // Candidates of one shard: (score, global index) of its local top-k, [rows][k].

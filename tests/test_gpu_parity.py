@@ -451,6 +451,48 @@ def test_prefill_hca_dense():
     _check_prefill(wl, Tq=200, prefix=4096 + 2, queries=[0, 1, 62, 63, 64, 127, 128, 199])
 
 
+def test_prefill_hca_dense_64_heads():
+    # HCA chunked prefill with 64 heads of bf16 rows: the persistent tcgen05 prefill kernel over dense
+    # slot lists (about 33 entries and up to 128 window rows: a full tile and a ragged one)
+    layer = scaled_layer(HCA_PRO, H=64, kv_format="bf16")
+    wl = get_workload("csa_prefill_8k", layers=(layer,))
+    _check_prefill(wl, Tq=200, prefix=4096 + 2, queries=[0, 1, 62, 63, 64, 127, 128, 199])
+
+
+def test_prefill_window_rows_dominate():
+    # window rows four times larger than usual (raw rows and stored window rows scaled by 4, exactly):
+    # the window's tile, the query's last, raises every head's running maximum by more than the
+    # kernel's margin, so the accumulated output and sums are rescaled mid-query
+    wl = get_workload("csa_prefill_8k")
+    layer = wl.layers[0]
+    Tq, prefix = 96, 4096 + 2
+    pf = prefill_inputs(wl, Tq=Tq, prefix=prefix)
+    pf["raw"] = F.bf16_encode(F.decode_act(pf["raw"], "bf16") * 4.0)
+    pf["window"] = _scaled_rows(pf["window"], layer.kv_format, layer.D, 4.0)
+    st = LayerState.from_arrays(layer, wl.B, pf, raw_key="raw", gate_key="gate", raw_base=pf["raw_first_row"])
+    n_max = pf["n"] // layer.m
+    out = torch.zeros((wl.B, Tq, layer.H, layer.D), dtype=torch.int16, device="cuda")
+    topk = torch.zeros((wl.B, Tq, layer.top_k), dtype=torch.int32, device="cuda")
+    ws = st.workspace("prefill", Tq, n_max)
+    C.csa_prefill(st.L, st.cache(), st.params(), dev(pf["q"]), dev(pf["idx_q"]), dev(pf["idx_q_scale"]),
+                  dev(pf["head_w"]), dev(pf["t"]), Tq, n_max, out, topk, ws)
+    torch.cuda.synchronize()
+    _no_device_error(ws)
+    L = O.LayerSpec.of(layer)
+    ents, win, _, _ = O.prefill_caches(L, pf, 0)
+    got = out_values(out, layer.act_format)[0]
+    tk = host(topk)[0]
+    # values and logits of the window keys are 4x the usual: the bf16 roundings of q~ and P move a
+    # logit of size |l| by about |l| 2^-8, so the absolute bars scale by 4 x 4 and the relative L2 bar
+    # by 4 (a missed or wrong rescale would put the error at the size of the output itself)
+    for j in range(0, Tq, 5):
+        ref = O.prefill_query(L, pf, ents, win, 0, j)
+        assert check_topk(tk[j], ref["scores"], layer.top_k) == 0
+        assert_out_close(got[j], ref["o"], max_abs=0.32, mean_abs=0.032, rel_l2=4e-2, tag=f"window x4 q{j}")
+    worst = max((x for x in _gpu_util.STATS if x["tag"].startswith("window x4")), key=lambda x: x["rel_l2"])
+    print("window x4 worst:", worst)
+
+
 def test_prefill_full_size_sampled():
     wl = get_workload("csa_prefill_8k")
     Tq = wl.Tq
