@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extra-configs", action="store_true", help="skip the 128K configurations' lines")
+    p.add_argument("--prefill-queries", type=int, default=None,
+                   help="chunk size of --workload csa_prefill_8k (default: the workload's 8,192)")
     p.add_argument("--burn-seconds", type=float, default=0.5, help="untimed replays before timing (clocks settle)")
     return p.parse_args()
 
@@ -661,6 +663,13 @@ def run_ours(args):
             torch.cuda.empty_cache()
         line["variants"] = variants
 
+    # ------------------------------------------------------------------ the chunked prefill (config E)
+    if args.workload == "csa_hca_decode_1m" and not args.no_extra_configs and world == 1:
+        res, _, _ = prefill_measure("csa_prefill_8k", args.steps, args.warmup)
+        res.pop("clocks", None)
+        line["prefill"] = res
+        torch.cuda.empty_cache()
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, datas, args.cpu_seconds)
     if rank == 0:
@@ -684,18 +693,20 @@ def prefill_work(layer, t, n_max, B=1):
     return idx_flops, att_flops, float(rows.sum()) * B * row_bytes
 
 
-def run_prefill(args):
-    """Times csa_prefill on the 8,192-query chunk (one GPU): tokens/s, the launch list of one call
-    (CUDA events before each launch), and the indexer's FP8 and the attention's BF16 TFLOP/s against
-    the measured dense BF16 peak (FP8 = 2x, the nominal ratio).  Not the headline line: the
-    workload's inputs (512 MiB of queries alone) exceed L2, so calls run back to back."""
+def prefill_measure(workload, steps, warmup, queries=None):
+    """Times csa_prefill on the 8,192-query chunk (one GPU): the whole call (CUDA events around
+    back-to-back calls), and the launch list of one call (an event before each launch, one after the
+    call: the last interval is the attention kernel's own).  The work of a call (FP8 indexer FLOPs,
+    BF16 attention FLOPs, gathered bytes) is set against the measured dense BF16 peak (FP8 = 2x, the
+    nominal ratio).  The workload's inputs (512 MiB of queries alone) exceed L2, so calls run back to
+    back."""
     import torch
     from csa_synth import get_workload, prefill_inputs
     from long_context_sparse_csa_b200 import binding as C
     from long_context_sparse_csa_b200.state import LayerState, to_device
-    wl = get_workload(args.workload)
+    wl = get_workload(workload)
     layer = wl.layers[0]
-    pf = prefill_inputs(wl)
+    pf = prefill_inputs(wl, Tq=queries)
     st = LayerState.from_arrays(layer, wl.B, pf, raw_key="raw", gate_key="gate", raw_base=pf["raw_first_row"])
     Tq, n_max = pf["Tq"], pf["n"] // layer.m
     out = torch.zeros((wl.B, Tq, layer.H, layer.D), dtype=torch.int16, device="cuda")
@@ -707,10 +718,10 @@ def run_prefill(args):
         C.csa_prefill(st.L, st.cache(), st.params(), io["q"], io["idx_q"], io["idx_q_scale"], io["head_w"], io["t"],
                       Tq, n_max, out, topk, ws)
 
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, warmup)):
         call()
     torch.cuda.synchronize()
-    steps = max(1, min(args.steps, 10))
+    steps = max(1, min(steps, 10))
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -725,7 +736,7 @@ def run_prefill(args):
     clocks.sample()
     clocks.stop()
     ms = e0.elapsed_time(e1) / steps
-    # launch list of one call
+    # launch list of one call (the library records an event before each of its launches)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(17)]
     for x in evs:                      # recorded once here, so torch accepts the library's records
         x.record()
@@ -736,6 +747,7 @@ def run_prefill(args):
     C.csa_profile_timeline(None)
     evs[n].record()
     torch.cuda.synchronize()
+    assert C.csa_device_error(ws) == 0
     launches_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(n)]
     idx_flops, att_flops, gather_bytes = prefill_work(layer, pf["t"][0], n_max, wl.B)
     try:
@@ -743,19 +755,35 @@ def run_prefill(args):
             bf16_peak, note = float(json.load(f)["bf16_tflops"]), "of measured"
     except (OSError, KeyError, ValueError):
         bf16_peak, note = 1590.0, "of fallback"
-    longest = sorted(range(n), key=lambda i: -launches_ms[i])
-    line = {"metric": "prefill tok/s (8,192-query CSA chunk after a 65,536-token prefix)",
-            "value": wl.B * Tq / (ms / 1e3), "unit": "tok/s", "n_gpus": 1, "steps": steps, "warmup": max(3, args.warmup),
-            "ms_per_call": ms, "higher_is_better": True, "dtype": "e4m3+bf16 (fp32 accumulate)", "data": "synthetic",
-            "config": {"workload": wl.name, "batch": wl.B, "queries": Tq, "prefix": pf["prefix"], "heads": layer.H,
-                       "kv_dim": layer.D, "kv_format": layer.kv_format, "top_k": layer.top_k,
+    res = {"workload": wl.name, "tok_s": wl.B * Tq / (ms / 1e3), "ms_per_call": ms, "queries": Tq,
+           "prefix": pf["prefix"], "heads": layer.H, "kv_format": layer.kv_format, "launch_ms": launches_ms,
+           "work": {"indexer_fp8_tflop": idx_flops / 1e12, "attention_bf16_tflop": att_flops / 1e12,
+                    "attention_gather_gb": gather_bytes / 1e9},
+           "bf16_peak_tflops": bf16_peak, "peak_source": note, "clocks": clocks.summary(w0, w1)}
+    if n == 4:          # append+compress, indexer scores, top-k, attention: the call's launches in order
+        names = ["append_compress", "indexer", "topk", "attention"]
+        res["kernels_ms"] = dict(zip(names, launches_ms))
+        att_ms, idx_ms = launches_ms[3], launches_ms[1]
+        res["attention"] = {"kernel": "attend_prefill_tc_kernel" if layer.H == 64 and layer.kv_format == "bf16"
+                            else "attend_mma_kernel", "ms": att_ms, "tflops": att_flops / (att_ms / 1e3) / 1e12,
+                            "frac_of_bf16_peak": att_flops / (att_ms / 1e3) / 1e12 / bf16_peak}
+        res["indexer"] = {"kernel": "index_score_tc_kernel", "ms": idx_ms, "tflops": idx_flops / (idx_ms / 1e3) / 1e12,
+                          "frac_of_fp8_peak": idx_flops / (idx_ms / 1e3) / 1e12 / (2 * bf16_peak)}
+    return res, steps, max(3, warmup)
+
+
+def run_prefill(args):
+    """The chunked-prefill line on its own (`--workload csa_prefill_8k`); the default decode line
+    carries the same measurement under its "prefill" key."""
+    res, steps, warmup = prefill_measure(args.workload, args.steps, args.warmup, args.prefill_queries)
+    line = {"metric": f"prefill tok/s ({res['queries']:,}-query CSA chunk after a {res['prefix']:,}-token prefix)",
+            "value": res["tok_s"], "unit": "tok/s", "n_gpus": 1, "steps": steps, "warmup": warmup,
+            "ms_per_call": res["ms_per_call"], "higher_is_better": True, "dtype": "e4m3+bf16 (fp32 accumulate)",
+            "data": "synthetic",
+            "config": {"workload": res["workload"], "queries": res["queries"], "prefix": res["prefix"],
+                       "heads": res["heads"], "kv_format": res["kv_format"],
                        "l2": "inputs larger than L2 (queries alone 512 MiB)"},
-            "launch_ms": [round(x, 3) for x in launches_ms],
-            "work": {"indexer_fp8_tflop": idx_flops / 1e12, "attention_bf16_tflop": att_flops / 1e12,
-                     "attention_gather_gb": gather_bytes / 1e9},
-            "tensor": {"bf16_peak_tflops": bf16_peak, "fp8_peak_tflops": 2 * bf16_peak, "peak_source": note},
-            "longest_launches": [{"launch": i, "ms": round(launches_ms[i], 3)} for i in longest[:3]],
-            "clocks": clocks.summary(w0, w1)}
+            "prefill": res, "clocks": res["clocks"]}
     print(json.dumps(line), flush=True)
 
 
