@@ -57,7 +57,7 @@ int num_sms() {
 // eager call, or a launch timeline is armed: its intervals then stay one kernel each).
 struct SideStream {
   cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr, mid = nullptr;
   bool failed = false;
 };
 thread_local SideStream g_side[64];
@@ -76,10 +76,12 @@ SideStream* side_stream(cudaStream_t main) {
   }
   if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
       cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ss.mid, cudaEventDisableTiming) != cudaSuccess) {
     cudaGetLastError();
     if (ss.s) cudaStreamDestroy(ss.s);
     if (ss.fork) cudaEventDestroy(ss.fork);
+    if (ss.join) cudaEventDestroy(ss.join);
     ss = SideStream();
     ss.failed = true;
     return nullptr;
@@ -201,6 +203,7 @@ struct Workspace {
   size_t topk = 0, topk_bytes = 0;
   size_t part = 0, part_bytes = 0;
   size_t qt = 0;                        // bf16 q~ of the tcgen05 attention [rows][H][D]
+  size_t extra = 0;                     // HCA decode: logits of the deferred rows [rows][2][H] fp32
   size_t idxq = 0, idxqs = 0;           // indexed decode step: produced index query and its scales
   size_t total = 0;
 };
@@ -234,6 +237,9 @@ Workspace layout(const csa_layer_t* L, int op, int32_t Tq, int64_t n_max) {
     const int splits = attend_num_splits(la, dense, (int)rows, slots, num_sms());
     w.part = off; w.part_bytes = attend_partial_bytes(la, dense, (int)rows, splits); off = up(off + w.part_bytes);
     if (attend_path(la, dense, (int)rows) == 2) { w.qt = off; off = up(off + rows * (size_t)L->H * L->D * 2); }
+    if (attend_path(la, dense, (int)rows) == 2 && dense) {
+      w.extra = off; off = up(off + rows * 2 * (size_t)L->H * 4);
+    }
   }
   w.total = off;
   return w;
@@ -344,6 +350,8 @@ csa_status_t make_attend_args(const csa_layer_t* L, const csa_cache_t* cache, co
   a.entry_limit = cache->entry_cap;
   a.no_window = 0;
   a.partial_out = nullptr;
+  a.defer_new = 0;
+  a.extra = w.extra ? reinterpret_cast<float*>(at(ws, w.extra)) : nullptr;
   return CSA_OK;
 }
 
@@ -808,6 +816,27 @@ csa_status_t hca_decode_step(const csa_layer_t* L, const csa_cache_t* cache, con
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* ws_err = reinterpret_cast<int*>(at(workspace, w.err));
   SideStream* ss = side_stream(s);
+  if (ss && w.extra) {
+    // append+compress on the side stream beside the attention over the earlier rows; the token's own
+    // window row and the entry it completes join in the combine as two extra keys
+    AttendArgs a;
+    CSA_TRY(make_attend_args(L, cache, P, q, q_pos, 1, nullptr, cache->entry_cap, out, w, workspace, a));
+    a.defer_new = 1;
+    cudaError_t e = cudaEventRecord(ss->fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->s, ss->fork, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "hca_decode_step fork");
+    const csa_status_t sc = run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, ws_err, ss->s);
+    e = launch_attend_qprep(a, s);
+    if (e == cudaSuccess) e = cudaEventRecord(ss->mid, s);
+    if (e == cudaSuccess) e = launch_attend_deferred(a, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->s, ss->mid, 0);
+    if (e == cudaSuccess) e = launch_attend_extra_logits(a, ss->s);
+    if (e == cudaSuccess) e = cudaEventRecord(ss->join, ss->s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
+    if (e == cudaSuccess) e = launch_attend_combine(a, s);
+    if (sc != CSA_OK) return sc;
+    return e == cudaSuccess ? CSA_OK : cuda_fail(e, "hca_decode_step launch");
+  }
   if (ss) {
     // fork: the attention's query preparation on the side stream beside append+compress
     cudaError_t e = cudaEventRecord(ss->fork, s);

@@ -114,6 +114,7 @@ __device__ __forceinline__ uint32_t swz(int row, int ch, int pitch) {
 
 struct SlotInfo {
   int64_t rt, n_sel, n_win, R;
+  int64_t wlast;             // last window row attended (r_t, or r_t - 1 when deferred)
 };
 
 __device__ __forceinline__ SlotInfo slot_info(const AttendArgs& a, int64_t t) {
@@ -123,6 +124,15 @@ __device__ __forceinline__ SlotInfo slot_info(const AttendArgs& a, int64_t t) {
   const int64_t nvis = r1 / a.L.m;
   s.n_sel = a.topk ? (int64_t)a.L.top_k : (nvis < a.n_max ? nvis : a.n_max);
   s.n_win = a.no_window ? 0 : (r1 < a.L.window ? r1 : a.L.window);
+  s.wlast = s.rt;
+  if (a.defer_new && !a.topk) {
+    // this step's own rows join in the combine: the entry the token completes, and its window row
+    if (r1 > 0 && r1 % a.L.m == 0 && nvis <= a.n_max && s.n_sel > 0) s.n_sel -= 1;
+    if (s.n_win > 0) {
+      s.n_win -= 1;
+      s.wlast = s.rt - 1;
+    }
+  }
   s.R = s.n_sel + s.n_win;
   return s;
 }
@@ -137,7 +147,7 @@ __device__ __forceinline__ const uint8_t* slot_row(const AttendArgs& a, const Sl
     return C.entries + ((size_t)b * C.entry_cap + (size_t)e) * a.L.row_bytes;
   }
   if (s < si.R) {
-    const int64_t wr = si.rt - si.n_win + 1 + (s - si.n_sel);
+    const int64_t wr = si.wlast - si.n_win + 1 + (s - si.n_sel);
     return C.window + ((size_t)b * C.window_cap + (size_t)(wr % C.window_cap)) * a.L.row_bytes;
   }
   return nullptr;
@@ -809,6 +819,72 @@ __global__ void __launch_bounds__(128) qprep_kernel(const __grid_constant__ Atte
 }
 
 
+// The rows a deferred attention leaves to the combine: [0] the token's window row, [1] the entry the
+// token completes (null when it completes none).
+struct DeferredRows {
+  const uint8_t* p[2];
+};
+
+__device__ __forceinline__ DeferredRows deferred_rows(const AttendArgs& a, int row) {
+  DeferredRows d;
+  d.p[0] = d.p[1] = nullptr;
+  const CacheArgs& C = a.C;
+  const int b = row / a.Tq;
+  const int64_t rt = a.q_pos[row] - a.L.pos0;
+  if (rt < 0 || a.no_window) return d;
+  d.p[0] = C.window + ((size_t)b * C.window_cap + (size_t)(rt % C.window_cap)) * a.L.row_bytes;
+  const int64_t r1 = rt + 1, nvis = r1 / a.L.m;
+  if (r1 % a.L.m == 0 && nvis <= a.n_max)
+    d.p[1] = C.entries + ((size_t)b * C.entry_cap + (size_t)(nvis - 1)) * a.L.row_bytes;
+  return d;
+}
+
+// Values of dims d0..d0+3 of a stored bf16 or mixed row (codes times the row's power-of-two scale).
+__device__ __forceinline__ void stored4(const uint8_t* row, const LayerArgs& L, int d0, float v[4]) {
+  if (L.kv_fmt == CSA_FMT_BF16 || d0 >= kD - 64) {
+    const uint8_t* p = L.kv_fmt == CSA_FMT_BF16 ? row + d0 * 2 : row + (kD - 64) + (d0 - (kD - 64)) * 2;
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    v[0] = bf16_bits_to_f(u.x & 0xFFFFu); v[1] = bf16_bits_to_f(u.x >> 16);
+    v[2] = bf16_bits_to_f(u.y & 0xFFFFu); v[3] = bf16_bits_to_f(u.y >> 16);
+    return;
+  }
+  const float sg = *reinterpret_cast<const float*>(row + kD + 64);
+  const uint32_t w = *reinterpret_cast<const uint32_t*>(row + d0);
+  const float2 lo = e4m3x2_to_float2((uint16_t)(w & 0xFFFFu)), hi = e4m3x2_to_float2((uint16_t)(w >> 16));
+  v[0] = lo.x * sg; v[1] = lo.y * sg; v[2] = hi.x * sg; v[3] = hi.y * sg;
+}
+
+// Logits (base 2) of the deferred rows for every head: one warp per (head, row), lane l taking dims
+// [16 l, 16 l + 16) of q~ (bf16) and of the stored row; -inf for a row that does not exist.
+__global__ void __launch_bounds__(128) attend_extra_logits_kernel(const __grid_constant__ AttendArgs a) {
+  const LayerArgs& L = a.L;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.y, hk = blockIdx.x * 4 + warp;
+  const int h = hk >> 1, k = hk & 1;
+  if (h >= L.H) return;
+  const DeferredRows dr = deferred_rows(a, row);
+  float* dst = a.extra + ((size_t)row * 2 + k) * L.H + h;
+  if (!dr.p[k]) {
+    if (lane == 0) *dst = -INFINITY;
+    return;
+  }
+  const uint4* qp = reinterpret_cast<const uint4*>(a.qt + (((size_t)row * L.H + h) * kD + 16 * lane) * 2);
+  const uint4 q0 = qp[0], q1 = qp[1];
+  const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+  float dot = 0.f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float v[4];
+    stored4(dr.p[k], L, 16 * lane + 4 * c, v);
+    dot = fmaf(bf16_bits_to_f(qw[2 * c] & 0xFFFFu), v[0], dot);
+    dot = fmaf(bf16_bits_to_f(qw[2 * c] >> 16), v[1], dot);
+    dot = fmaf(bf16_bits_to_f(qw[2 * c + 1] & 0xFFFFu), v[2], dot);
+    dot = fmaf(bf16_bits_to_f(qw[2 * c + 1] >> 16), v[3], dot);
+  }
+  dot = warp_sum(dot);
+  if (lane == 0) *dst = dot * (L.scale * kLog2e);
+}
+
 // Byte offset of 16-byte piece j (dims 8j..8j+7 of a 64-dim block) of row r in a 128-byte-swizzled
 // K-major tile of rows.
 __device__ __forceinline__ uint32_t sw128(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
@@ -885,7 +961,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
         return C.entries + ((size_t)b * C.entry_cap + (size_t)e) * L.row_bytes;
       }
       if (s < si.R) {
-        const int64_t wr = si.rt - si.n_win + 1 + (s - si.n_sel);
+        const int64_t wr = si.wlast - si.n_win + 1 + (s - si.n_sel);
         return C.window + ((size_t)b * C.window_cap + (size_t)(wr % C.window_cap)) * L.row_bytes;
       }
       return nullptr;
@@ -1124,7 +1200,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attend_tc_kernel(const __grid_c
   ATRACE_T(128, 10);
   tc_fence_after();
   const int e0 = hs * (kTcHalf / 2);
-  if (a.splits > 1 || a.partial_out) {
+  if (a.splits > 1 || a.partial_out || a.defer_new) {
     // partial of this split: O / l in bf16 as [dim / 4][head][4] (a warp's stores are contiguous,
     // the combine reads a head's 4 dims in one 8-byte load), then (m, l) per head in fp32.  O / l
     // is a convex combination of value rows, so its bf16 rounding is no coarser than the output's.
@@ -1268,6 +1344,19 @@ __global__ void __launch_bounds__(512) attend_tc_combine_kernel(const __grid_con
   float M = sk;
 #pragma unroll
   for (int q = 0; q < 4; ++q) M = fmaxf(M, red[q][0][h]);
+  // deferred rows of this step (the token's window row, the entry it completes): one key each, with
+  // its logit (base 2) from attend_extra_logits_kernel and its value read from the cache here
+  float ex[2] = {-INFINITY, -INFINITY}, xv[2][4];
+  if (a.defer_new) {
+    const DeferredRows dr = deferred_rows(a, row);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      if (!dr.p[k]) continue;
+      ex[k] = a.extra[((size_t)row * 2 + k) * L.H + h];
+      stored4(dr.p[k], L, d0, xv[k]);
+      M = fmaxf(M, ex[k]);
+    }
+  }
   float lsum = exp2f(sk - M), out[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -1275,6 +1364,14 @@ __global__ void __launch_bounds__(512) attend_tc_combine_kernel(const __grid_con
     lsum += red[q][1][h] * f;
 #pragma unroll
     for (int k = 0; k < 4; ++k) out[k] += red[q][2 + k][h] * f;
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    if (ex[k] == -INFINITY) continue;
+    const float f = exp2f(ex[k] - M);
+    lsum += f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) out[c] = fmaf(f, xv[k][c], out[c]);
   }
   const float inv = 1.f / lsum;
 #pragma unroll
@@ -1427,6 +1524,34 @@ cudaError_t launch_tc_n(const AttendArgs& a, cudaStream_t s) {
 template <int FMT>
 cudaError_t launch_tc(const AttendArgs& a, cudaStream_t s) {
   return a.topk ? launch_tc_n<FMT, kTcNSparse>(a, s) : launch_tc_n<FMT, kTcN>(a, s);
+}
+
+// The deferred-row form of the tcgen05 dense attention, in three launches that the caller orders
+// around the concurrent append+compress: the attention over the earlier rows (q~ prepared first),
+// the deferred rows' logits (after append+compress and q~), and the combine.
+cudaError_t launch_attend_deferred(const AttendArgs& a, cudaStream_t s) {
+  if (a.rows <= 0) return cudaSuccess;
+  constexpr size_t smem = tc_smem_bytes(kTcN);
+  auto kern = a.L.kv_fmt == CSA_FMT_MIXED ? attend_tc_kernel<CSA_FMT_MIXED, kTcN> : attend_tc_kernel<CSA_FMT_BF16, kTcN>;
+  {
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
+    if (e != cudaSuccess) return e;
+  }
+  CUtensorMap qmap;
+  if (!make_qt_map(&qmap, a.qt, a.rows)) return cudaErrorInvalidValue;
+  return launch_kernel(kern, dim3((unsigned)(2 * a.splits), 1, (unsigned)a.rows), dim3(kTcThreads), smem, s, 2,
+                       qmap, a);
+}
+
+cudaError_t launch_attend_extra_logits(const AttendArgs& a, cudaStream_t s) {
+  if (a.rows <= 0) return cudaSuccess;
+  return launch_kernel(attend_extra_logits_kernel, dim3((unsigned)((2 * a.L.H + 3) / 4), (unsigned)a.rows), dim3(128),
+                       0, s, 0, a);
+}
+
+cudaError_t launch_attend_combine(const AttendArgs& a, cudaStream_t s) {
+  if (a.rows <= 0) return cudaSuccess;
+  return launch_kernel(attend_tc_combine_kernel, dim3(kD / 4, a.rows), dim3(4 * kH128), 0, s, 0, a);
 }
 
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {

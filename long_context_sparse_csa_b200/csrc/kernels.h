@@ -182,6 +182,11 @@ struct AttendArgs {
   int64_t entry_offset, entry_limit;
   int no_window;
   float* partial_out;
+  // deferred rows (dense tcgen05 path): the attention kernel leaves out the token's own window row and
+  // the entry the token completes; the combine adds them as two keys, their logits (base 2) in
+  // extra [rows][2][H] (-inf for a row that does not exist)
+  int defer_new;
+  float* extra;
 };
 // Attention kernel family for a call of `rows` query rows: 2 = tcgen05 (H = 128, D = 512, bf16 or
 // mixed rows, at most kTcMaxRows rows), 3 = persistent tcgen05 prefill kernel (H = 64, D = 512, bf16
@@ -198,6 +203,9 @@ size_t attend_partial_bytes(const LayerArgs& L, bool dense, int rows, int splits
 cudaError_t launch_attend_qprep(const AttendArgs& a, cudaStream_t s);
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s);
 bool attend_prefill_tc_supported(const LayerArgs& L, int rows);
+cudaError_t launch_attend_deferred(const AttendArgs& a, cudaStream_t s);
+cudaError_t launch_attend_extra_logits(const AttendArgs& a, cudaStream_t s);
+cudaError_t launch_attend_combine(const AttendArgs& a, cudaStream_t s);
 cudaError_t launch_attend_prefill_tc(const AttendArgs& a, cudaStream_t s);
 
 // ----------------------------------------------------------------------------- context-sharded decode
