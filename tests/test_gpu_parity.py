@@ -390,6 +390,20 @@ def test_decode_per_sequence_positions():
         assert_out_close(got[b], ref["o"])
 
 
+def test_decode_hca_per_sequence_positions():
+    # HCA steps of one call where one sequence's token completes a group (its new entry joins in the
+    # combine) and the others' do not; every token's own window row joins there too
+    wl = get_workload("hca_decode_128k", B=3)
+    layer = wl.layers[0]
+    d = decode_inputs(wl)
+    d["t"] = np.array([131071, 130999, 1500], dtype=np.int64)
+    _, st, out, _ = _run_decode(wl, d=d)
+    got = out_values(out, layer.act_format)
+    for b in range(3):
+        ref = _oracle_step(layer, d, b)
+        assert_out_close(got[b], ref["o"], tag=f"hca positions b{b}")
+
+
 # ----------------------------------------------------------------------------- chunked prefill
 
 def _prefill_case(wl, Tq=None, prefix=None):
