@@ -57,7 +57,7 @@ int num_sms() {
 // eager call, or a launch timeline is armed: its intervals then stay one kernel each).
 struct SideStream {
   cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr, mid = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
   bool failed = false;
 };
 thread_local SideStream g_side[64];
@@ -76,8 +76,7 @@ SideStream* side_stream(cudaStream_t main) {
   }
   if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
       cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&ss.mid, cudaEventDisableTiming) != cudaSuccess) {
+      cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
     cudaGetLastError();
     if (ss.s) cudaStreamDestroy(ss.s);
     if (ss.fork) cudaEventDestroy(ss.fork);
@@ -818,7 +817,8 @@ csa_status_t hca_decode_step(const csa_layer_t* L, const csa_cache_t* cache, con
   SideStream* ss = side_stream(s);
   if (ss && w.extra) {
     // append+compress on the side stream beside the attention over the earlier rows; the token's own
-    // window row and the entry it completes join in the combine as two extra keys
+    // window row and the entry it completes join in the combine as two extra keys, their logits taken
+    // on the side stream after append+compress
     AttendArgs a;
     CSA_TRY(make_attend_args(L, cache, P, q, q_pos, 1, nullptr, cache->entry_cap, out, w, workspace, a));
     a.defer_new = 1;
@@ -827,9 +827,7 @@ csa_status_t hca_decode_step(const csa_layer_t* L, const csa_cache_t* cache, con
     if (e != cudaSuccess) return cuda_fail(e, "hca_decode_step fork");
     const csa_status_t sc = run_append_compress(L, cache, P, x_new, g_new, q_pos, 1, true, true, ws_err, ss->s);
     e = launch_attend_qprep(a, s);
-    if (e == cudaSuccess) e = cudaEventRecord(ss->mid, s);
     if (e == cudaSuccess) e = launch_attend_deferred(a, s);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->s, ss->mid, 0);
     if (e == cudaSuccess) e = launch_attend_extra_logits(a, ss->s);
     if (e == cudaSuccess) e = cudaEventRecord(ss->join, ss->s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);

@@ -855,7 +855,7 @@ __device__ __forceinline__ void stored4(const uint8_t* row, const LayerArgs& L, 
 }
 
 // Logits (base 2) of the deferred rows for every head: one warp per (head, row), lane l taking dims
-// [16 l, 16 l + 16) of q~ (bf16) and of the stored row; -inf for a row that does not exist.
+// [16 l, 16 l + 16) of q~ and of the stored row; -inf for a row that does not exist.
 __global__ void __launch_bounds__(128) attend_extra_logits_kernel(const __grid_constant__ AttendArgs a) {
   const LayerArgs& L = a.L;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -868,18 +868,51 @@ __global__ void __launch_bounds__(128) attend_extra_logits_kernel(const __grid_c
     if (lane == 0) *dst = -INFINITY;
     return;
   }
-  const uint4* qp = reinterpret_cast<const uint4*>(a.qt + (((size_t)row * L.H + h) * kD + 16 * lane) * 2);
-  const uint4 q0 = qp[0], q1 = qp[1];
-  const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+  // q~ of the head from q itself (so this kernel waits for nothing but append+compress): RMSNorm over
+  // the warp, gamma, the rotation by +t (dims 448..511 in lanes 28..31), rounded to bf16 as the
+  // attention's operand is
+  float qv[16], ss = 0.f;
+  if (L.act_fmt == CSA_FMT_F32) {
+#pragma unroll
+    for (int i = 0; i < 16; i += 4) load_act4(a.q + ((size_t)row * L.H + h) * kD * 4, CSA_FMT_F32, 16 * lane + i, qv + i);
+  } else {
+    const uint4* qp = reinterpret_cast<const uint4*>(a.q + (((size_t)row * L.H + h) * kD + 16 * lane) * 2);
+    const uint4 q0 = __ldg(qp), q1 = __ldg(qp + 1);
+    const uint32_t qw[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      qv[2 * i] = bf16_bits_to_f(qw[i] & 0xFFFFu);
+      qv[2 * i + 1] = bf16_bits_to_f(qw[i] >> 16);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) ss = fmaf(qv[i], qv[i], ss);
+  ss = warp_sum(ss);
+  const float rs = 1.0f / sqrtf(ss / (float)kD + L.eps);
+  const int64_t t = a.q_pos[row];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) qv[i] *= rs * (a.gamma_q ? __ldg(a.gamma_q + 16 * lane + i) : 1.f);
+  // rotary pair u's cos / sin computed by lane u (one float64 sincospi per lane), shuffled to the
+  // lanes holding dims 448..511
+  float cu, su;
+  rope_cos_sin((double)t, lane, L, &cu, &su);
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    const int u = (lane >= 28 ? 8 * (lane - 28) : 0) + (i >> 1);
+    const float c = __shfl_sync(0xffffffffu, cu, u), sn = __shfl_sync(0xffffffffu, su, u);
+    if (lane >= 28) {
+      const float x0 = qv[i], x1 = qv[i + 1];
+      qv[i] = x0 * c - x1 * sn;
+      qv[i + 1] = x0 * sn + x1 * c;
+    }
+  }
   float dot = 0.f;
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     float v[4];
     stored4(dr.p[k], L, 16 * lane + 4 * c, v);
-    dot = fmaf(bf16_bits_to_f(qw[2 * c] & 0xFFFFu), v[0], dot);
-    dot = fmaf(bf16_bits_to_f(qw[2 * c] >> 16), v[1], dot);
-    dot = fmaf(bf16_bits_to_f(qw[2 * c + 1] & 0xFFFFu), v[2], dot);
-    dot = fmaf(bf16_bits_to_f(qw[2 * c + 1] >> 16), v[3], dot);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dot = fmaf(bf16_bits_to_f(f_to_bf16_bits(qv[4 * c + e])), v[e], dot);
   }
   dot = warp_sum(dot);
   if (lane == 0) *dst = dot * (L.scale * kLog2e);

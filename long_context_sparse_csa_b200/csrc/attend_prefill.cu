@@ -62,7 +62,8 @@ struct __align__(8) PfBars {
 constexpr size_t kOffQ = (size_t)kBlocks * kBlockBytes;
 constexpr size_t kOffP = kOffQ + (size_t)kBlocks * kQBlockBytes;
 constexpr size_t kOffMx = kOffP + (size_t)kKeys * 128;
-constexpr size_t kOffBars = kOffMx + (4 * kHeads + 3 * kHeads + 4) * sizeof(float);
+constexpr size_t kOffRope = kOffMx + (4 * kHeads + 3 * kHeads + 4) * sizeof(float);
+constexpr size_t kOffBars = kOffRope + 64 * sizeof(float);
 constexpr size_t kSmemBytes = 1024 + kOffBars + sizeof(PfBars);
 static_assert(kSmemBytes <= 227 * 1024, "prefill attention shared memory");
 
@@ -177,6 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
   float* alph = mrun + kHeads;                                  // [64] rescale factors of this tile
   float* fh = alph + kHeads;                                    // [64] output factors (epilogue)
   int* flag = reinterpret_cast<int*>(fh + kHeads);              // [1] any head rescaled
+  float* rope_tab = reinterpret_cast<float*>(sm + kOffRope);    // [32][2] the query's rotary cos / sin (loaders)
   PfBars* bars = reinterpret_cast<PfBars*>(sm + kOffBars);
 
   const LayerArgs& L = a.L;
@@ -451,6 +453,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
       // q~ of this query once the previous query's S^T MMAs are done with q~: the raw head row lands in
       // its q~ slots (all of its copies in flight at once), then is normalised and rotated in place
       if (!mbar_wait(&bars->qfree, (j & 1u) ^ 1u)) { ok = false; break; }
+      // the query's 32 rotary angles, one float64 sincospi per thread, shared by the loaders
+      if (lt < 32) rope_cos_sin((double)t, lt, L, &rope_tab[2 * lt], &rope_tab[2 * lt + 1]);
+      asm volatile("barrier.sync.aligned 2, 64;" ::: "memory");
       {
         const int h = lt;
         const uint8_t* src = a.q + ((size_t)row * kHeads + h) * kD * 2;
@@ -486,8 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
           if (d0 >= kD - 64) {
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
-              float c, sn;
-              rope_cos_sin((double)t, (d0 + e - (kD - 64)) >> 1, L, &c, &sn);
+              const int u = (d0 + e - (kD - 64)) >> 1;
+              const float c = rope_tab[2 * u], sn = rope_tab[2 * u + 1];
               const float x0 = v[e], x1 = v[e + 1];
               v[e] = x0 * c - x1 * sn;
               v[e + 1] = x0 * sn + x1 * c;
