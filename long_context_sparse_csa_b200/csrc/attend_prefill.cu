@@ -12,9 +12,9 @@
 //                                              dims), B = q~ (K-major); M = 128, N = 64; TMEM [0, 64)
 //   O^T[d, h]   += sum_key K[key, d] P[key, h]  A = the same tile read dims-major (M-tile mt = dims
 //                                              128 mt ..), B = P (heads-major); TMEM [256 + 64 mt, +64)
-// and the online softmax over keys in between.  A softmax thread owns one key (its TMEM lane) and holds
-// that key's 64 head scores; the tile's per-head maxima come from a butterfly reduce-scatter across the
-// warp (each lane ends with heads 2l and 2l + 1) and shared memory across the four warps.  A head's
+// and the online softmax over keys in between.  A softmax thread owns one key (its TMEM lane) and half
+// of the heads, and holds that key's 32 head scores; the tile's per-head maxima come from a butterfly
+// reduce-scatter across the warp on bf16 pairs and shared memory across the four lane quarters.  A head's
 // running maximum moves only when its tile maximum exceeds it by more than 8 (in log2 units); then
 // O^T's column and the partial sums are rescaled.  Exponentials are taken against the running maximum,
 // so they stay below 2^8.  Each softmax thread keeps its key's partial sums per head; they are reduced
@@ -22,9 +22,9 @@
 //
 // Roles, in one persistent CTA per SM (query rows strided by the grid):
 //   warp 0      the MMA issuer (one thread)
-//   warps 1-4   softmax; then per query the epilogue: 1 / (l + 2^(sink - m)), the rotation by -t,
-//               the bf16 store
-//   warps 5-6   loaders: q~ of each query (one head per thread: RMSNorm, gamma, the rotation by +t,
+//   warps 1-8   softmax, two warps per TMEM lane quarter (32 heads each); then per query the
+//               epilogue: 1 / (l + 2^(sink - m)), the rotation by -t, the bf16 store
+//   warps 9-10  loaders: q~ of each query (one head per thread: RMSNorm, gamma, the rotation by +t,
 //               bf16), then its key tiles, two key rows per thread, in 16-byte cp.async pieces into
 //               the 128-byte-swizzled tile, block by block.  A 64-dim block is refilled for the next tile as soon as the
 //               O^T MMAs that read it are done, while the other M-tiles still run.
@@ -47,7 +47,7 @@ constexpr int kKeys = 128;                    // keys per tile (MMA M of S^T)
 constexpr int kBlocks = 8;                    // 64-dim column blocks of a row
 constexpr int kBlockBytes = kKeys * 128;      // one block of the key tile: 16 KB
 constexpr int kQBlockBytes = kHeads * 128;    // one block of q~: 8 KB
-constexpr int kThreads = 224;                 // warp 0 MMA, warps 1-4 softmax, warps 5-6 loaders
+constexpr int kThreads = 352;                 // warp 0 MMA, warps 1-8 softmax, warps 9-10 loaders
 constexpr int kLoaders = 64;
 constexpr float kRescale = 8.f;               // log2 margin before a running maximum moves
 
@@ -90,7 +90,7 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ void softmax_bar() { asm volatile("barrier.sync.aligned 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void softmax_bar() { asm volatile("barrier.sync.aligned 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return (uint32_t)f_to_bf16_bits(lo) | ((uint32_t)f_to_bf16_bits(hi) << 16);
@@ -130,41 +130,10 @@ __device__ __forceinline__ const uint8_t* slot_ptr(const AttendArgs& a, const Sl
   return nullptr;
 }
 
-// Butterfly reduce-scatter of sums across the warp, 64 values per lane: lane l ends with the sums of
-// entries 2l and 2l + 1 in v[0], v[1].
-__device__ __forceinline__ void reduce_scatter_sum64(float v[64], int lane) {
-#pragma unroll
-  for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
-    const bool upper = (lane & o) != 0;
-#pragma unroll
-    for (int j = 0; j < n; ++j) {
-      const float send = upper ? v[j] : v[j + n];
-      const float keep = upper ? v[j + n] : v[j];
-      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-    }
-  }
-}
-
 __device__ __forceinline__ uint32_t bf16x2_max(uint32_t x, uint32_t y) {
   __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&x), b = *reinterpret_cast<__nv_bfloat162*>(&y);
   __nv_bfloat162 r = __hmax2(a, b);
   return *reinterpret_cast<uint32_t*>(&r);
-}
-
-// The same for maxima of 64 values held as 32 bf16 pairs (rounding to nearest is monotonic, so the
-// result is the rounded maximum): lane l ends with the maxima of entries 2l, 2l + 1 in w[0].  The
-// maximum is only the softmax's reference point, so its rounding is immaterial.
-__device__ __forceinline__ void reduce_scatter_max64(uint32_t w[32], int lane) {
-#pragma unroll
-  for (int o = 16, n = 16; o >= 1; o >>= 1, n >>= 1) {
-    const bool upper = (lane & o) != 0;
-#pragma unroll
-    for (int j = 0; j < n; ++j) {
-      const uint32_t send = upper ? w[j] : w[j + n];
-      const uint32_t keep = upper ? w[j + n] : w[j];
-      w[j] = bf16x2_max(keep, __shfl_xor_sync(0xffffffffu, send, o));
-    }
-  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __grid_constant__ AttendArgs a) {
@@ -177,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
   float* mrun = mx + 4 * kHeads;                                // [64] running maxima (log2 units)
   float* alph = mrun + kHeads;                                  // [64] rescale factors of this tile
   float* fh = alph + kHeads;                                    // [64] output factors (epilogue)
-  int* flag = reinterpret_cast<int*>(fh + kHeads);              // [1] any head rescaled
+  int* flag = reinterpret_cast<int*>(fh + kHeads);              // [2] any head of a half rescaled
   float* rope_tab = reinterpret_cast<float*>(sm + kOffRope);    // [32][2] the query's rotary cos / sin (loaders)
   PfBars* bars = reinterpret_cast<PfBars*>(sm + kOffBars);
 
@@ -191,9 +160,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
     mbar_init(&bars->qfull, kLoaders);
     mbar_init(&bars->qfree, 1);
     mbar_init(&bars->sfull, 1);
-    mbar_init(&bars->pfull, 128);
+    mbar_init(&bars->pfull, 256);
     mbar_init(&bars->ofull, 1);
-    mbar_init(&bars->ofree, 128);
+    mbar_init(&bars->ofree, 256);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_barrier_init();
@@ -270,9 +239,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
       }
     }
     __syncwarp();
-  } else if (warp <= 4) {
+  } else if (warp <= 8) {
     // ------------------------------------------------------------------ softmax and epilogue
+    // Two warps per TMEM lane quarter: warp w takes key (or dim) 32 (w % 4) + lane and heads
+    // [32 hf, 32 hf + 32), hf = (w - 1) / 4.
     const int w4 = warp & 3;                                  // TMEM lane quarter of this warp
+    const int hf = (warp - 1) >> 2;                           // head half
+    const int h0 = 32 * hf;
     const int key = w4 * 32 + lane;                           // key of S^T, dim of O^T's M-tile
     const uint32_t lane_addr = tmem + ((uint32_t)(w4 * 32) << 16);
     bool ok = true;
@@ -281,10 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
       const int64_t t = a.q_pos[row];
       const Slots si = slots_of(a, t);
       const int b = row / a.Tq;
-      float lp[kHeads];                                       // this key's partial sums per head
+      float lp[32];                                           // this key's partial sums of its heads
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) lp[h] = 0.f;
-      if (key < kHeads) mrun[key] = -INFINITY;
+      for (int h = 0; h < 32; ++h) lp[h] = 0.f;
+      if (hf == 0 && key < kHeads) mrun[key] = -INFINITY;
       softmax_bar();
       for (int i = 0; i < si.tiles; ++i, ++g) {
         const int64_t s = (int64_t)i * kKeys + key;
@@ -292,54 +265,64 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         if (!mbar_wait(&bars->sfull, g & 1u)) { ok = false; break; }
         if (tid == 32 && g < 16) PTRACE(32 + g);
         tc_fence_after();
-        float z[kHeads];
-        tmem_ld_32x32b_x32(lane_addr, z);
-        tmem_ld_32x32b_x32(lane_addr + 32u, z + 32);
+        float z[32];
+        tmem_ld_32x32b_x32(lane_addr + (uint32_t)h0, z);
         tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h) z[h] = valid ? z[h] * cl2 : -INFINITY;
-        // the tile's maxima per head: lanes, then warps
+        for (int h = 0; h < 32; ++h) z[h] = valid ? z[h] * cl2 : -INFINITY;
+        // the tile's maxima per head: lanes (a butterfly over bf16 pairs, then the last pair's
+        // neighbours), then warps
         {
-          uint32_t w[kHeads / 2];
+          uint32_t w[16];
 #pragma unroll
-          for (int q = 0; q < kHeads / 2; ++q) w[q] = pack_bf16x2(z[2 * q], z[2 * q + 1]);
-          reduce_scatter_max64(w, lane);
-          mx[w4 * kHeads + 2 * lane] = bf16_bits_to_f(w[0] & 0xFFFFu);
-          mx[w4 * kHeads + 2 * lane + 1] = bf16_bits_to_f(w[0] >> 16);
+          for (int q = 0; q < 16; ++q) w[q] = pack_bf16x2(z[2 * q], z[2 * q + 1]);
+#pragma unroll
+          for (int o = 16, n = 8; o >= 2; o >>= 1, n >>= 1) {
+            const bool upper = (lane & o) != 0;
+#pragma unroll
+            for (int q = 0; q < n; ++q) {
+              const uint32_t send = upper ? w[q] : w[q + n];
+              const uint32_t keep = upper ? w[q + n] : w[q];
+              w[q] = bf16x2_max(keep, __shfl_xor_sync(0xffffffffu, send, o));
+            }
+          }
+          w[0] = bf16x2_max(w[0], __shfl_xor_sync(0xffffffffu, w[0], 1));
+          // lanes 2k and 2k + 1 now hold heads h0 + 2k, h0 + 2k + 1
+          if ((lane & 1) == 0) {
+            mx[w4 * kHeads + h0 + lane] = bf16_bits_to_f(w[0] & 0xFFFFu);
+            mx[w4 * kHeads + h0 + lane + 1] = bf16_bits_to_f(w[0] >> 16);
+          }
         }
         softmax_bar();
         if (w4 == 0) {
+          const int h = h0 + lane;
+          const float tm = fmaxf(fmaxf(mx[h], mx[kHeads + h]), fmaxf(mx[2 * kHeads + h], mx[3 * kHeads + h]));
+          const float mr = mrun[h];
+          float al = 1.f;
           int moved = 0;
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int h = 2 * lane + u;
-            const float tm = fmaxf(fmaxf(mx[h], mx[kHeads + h]), fmaxf(mx[2 * kHeads + h], mx[3 * kHeads + h]));
-            const float mr = mrun[h];
-            float al = 1.f;
-            if (tm > mr + kRescale || (mr == -INFINITY && tm > -INFINITY)) {
-              al = mr == -INFINITY ? 0.f : exp2f(mr - tm);
-              mrun[h] = tm;
-              moved = 1;
-            }
-            alph[h] = al;
+          if (tm > mr + kRescale || (mr == -INFINITY && tm > -INFINITY)) {
+            al = mr == -INFINITY ? 0.f : exp2f(mr - tm);
+            mrun[h] = tm;
+            moved = 1;
           }
+          alph[h] = al;
           moved = __any_sync(0xffffffffu, moved);
-          if (lane == 0) flag[0] = moved;
+          if (lane == 0) flag[hf] = moved;
         }
         softmax_bar();
-        // P = 2^(z - m) in bf16, this key's row of P; the partial sums (rescaled where the head's maximum
-        // moved) take the rounded values
-        const bool moved = flag[0] != 0;
+        // P = 2^(z - m) in bf16, this key's row of P (its heads' 64 bytes); the partial sums
+        // (rescaled where the head's maximum moved) take the rounded values
+        const bool moved = (flag[0] | flag[1]) != 0;
         uint8_t* prow = P;
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
+        for (int jj = 0; jj < 4; ++jj) {
           uint32_t w[4];
           float mm[8], aa[8];
-          *reinterpret_cast<float4*>(mm) = reinterpret_cast<const float4*>(mrun)[2 * jj];
-          *reinterpret_cast<float4*>(mm + 4) = reinterpret_cast<const float4*>(mrun)[2 * jj + 1];
+          *reinterpret_cast<float4*>(mm) = reinterpret_cast<const float4*>(mrun + h0)[2 * jj];
+          *reinterpret_cast<float4*>(mm + 4) = reinterpret_cast<const float4*>(mrun + h0)[2 * jj + 1];
           if (moved) {
-            *reinterpret_cast<float4*>(aa) = reinterpret_cast<const float4*>(alph)[2 * jj];
-            *reinterpret_cast<float4*>(aa + 4) = reinterpret_cast<const float4*>(alph)[2 * jj + 1];
+            *reinterpret_cast<float4*>(aa) = reinterpret_cast<const float4*>(alph + h0)[2 * jj];
+            *reinterpret_cast<float4*>(aa + 4) = reinterpret_cast<const float4*>(alph + h0)[2 * jj + 1];
           }
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -355,21 +338,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
             lp[h] += bf16_bits_to_f(w[q] & 0xFFFFu);
             lp[h + 1] += bf16_bits_to_f(w[q] >> 16);
           }
-          *reinterpret_cast<uint4*>(prow + sw128(key, jj)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(prow + sw128(key, 4 * hf + jj)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         // rescale O^T, the previous tiles' sum (complete, as this tile's S^T is), where a maximum moved
         if (moved && i > 0) {
 #pragma unroll 1
           for (int mt = 0; mt < 4; ++mt) {
-#pragma unroll 1
-            for (int hc = 0; hc < kHeads; hc += 32) {
-              float o[32];
-              tmem_ld_32x32b_x32(lane_addr + 256u + 64u * mt + hc, o);
-              tmem_wait_ld();
+            float o[32];
+            tmem_ld_32x32b_x32(lane_addr + 256u + 64u * mt + h0, o);
+            tmem_wait_ld();
 #pragma unroll
-              for (int u = 0; u < 32; ++u) o[u] *= alph[hc + u];
-              tmem_st_32x32b_x32(lane_addr + 256u + 64u * mt + hc, o);
-            }
+            for (int u = 0; u < 32; ++u) o[u] *= alph[h0 + u];
+            tmem_st_32x32b_x32(lane_addr + 256u + 64u * mt + h0, o);
           }
           tmem_wait_st();
         }
@@ -380,47 +360,51 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
       }
       if (!ok) break;
       // ---------------------------------------------------------------- epilogue of this query
-      reduce_scatter_sum64(lp, lane);
-      mx[w4 * kHeads + 2 * lane] = lp[0];
-      mx[w4 * kHeads + 2 * lane + 1] = lp[1];
+      // this warp's partial sums per head: lane l ends with head h0 + l
+#pragma unroll
+      for (int o = 16, n = 16; o >= 1; o >>= 1, n >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int q = 0; q < n; ++q) {
+          const float send = upper ? lp[q] : lp[q + n];
+          const float keep = upper ? lp[q + n] : lp[q];
+          lp[q] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      mx[w4 * kHeads + h0 + lane] = lp[0];
       softmax_bar();
       if (w4 == 0) {
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int h = 2 * lane + u;
-          const float l = (mx[h] + mx[kHeads + h]) + (mx[2 * kHeads + h] + mx[3 * kHeads + h]);
-          const float m = mrun[h];
-          const float sk = a.sinks[h] * kLog2e;
-          // o = O / (l + 2^(sink - m)), O and l relative to the running maximum m
-          fh[h] = m == -INFINITY ? 0.f : 1.f / (l + exp2f(sk - m));
-        }
+        const int h = h0 + lane;
+        const float l = (mx[h] + mx[kHeads + h]) + (mx[2 * kHeads + h] + mx[3 * kHeads + h]);
+        const float m = mrun[h];
+        const float sk = a.sinks[h] * kLog2e;
+        // o = O / (l + 2^(sink - m)), O and l relative to the running maximum m
+        fh[h] = m == -INFINITY ? 0.f : 1.f / (l + exp2f(sk - m));
       }
       softmax_bar();
       if (!mbar_wait(&bars->ofull, j & 1u)) { ok = false; break; }
       tc_fence_after();
-      // per M-tile: this thread's dim of all heads -> a [64 heads][128 dims] bf16 staging tile in P's
-      // buffer (free: the query's last P.V is done), then 16-byte coalesced stores of the heads' rows
+      // per M-tile: this thread's dim of its heads -> a [64 heads][128 dims] bf16 staging tile in
+      // P's buffer (free: the query's last P.V is done), then 16-byte coalesced stores of the rows
       uint8_t* out = a.out + (size_t)row * kHeads * kD * 2;
       uint16_t* stage = reinterpret_cast<uint16_t*>(P);
+      const int st = tid - 32;                                // 0..255
 #pragma unroll 1
       for (int mt = 0; mt < 4; ++mt) {
         const int d = mt * 128 + key;
         float c = 1.f, sn = 0.f;
         const bool rot = d >= kD - 64;
         if (rot) rope_cos_sin((double)t, (d - (kD - 64)) >> 1, L, &c, &sn);
+        float o[32];
+        tmem_ld_32x32b_x32(lane_addr + 256u + 64u * mt + h0, o);
+        tmem_wait_ld();
 #pragma unroll
-        for (int hc = 0; hc < kHeads; hc += 32) {
-          float o[32];
-          tmem_ld_32x32b_x32(lane_addr + 256u + 64u * mt + hc, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            float v = o[u] * fh[hc + u];
-            // rotation by -t of the pair (d even, d + 1): partner in the neighbouring lane
-            const float pv = __shfl_xor_sync(0xffffffffu, v, 1);
-            if (rot) v = (d & 1) ? (-pv * sn + v * c) : (v * c + pv * sn);
-            stage[(hc + u) * 128 + key] = f_to_bf16_bits(v);
-          }
+        for (int u = 0; u < 32; ++u) {
+          float v = o[u] * fh[h0 + u];
+          // rotation by -t of the pair (d even, d + 1): partner in the neighbouring lane
+          const float pv = __shfl_xor_sync(0xffffffffu, v, 1);
+          if (rot) v = (d & 1) ? (-pv * sn + v * c) : (v * c + pv * sn);
+          stage[(h0 + u) * 128 + key] = f_to_bf16_bits(v);
         }
         if (mt == 3) {                                        // every O^T column read: release it
           tc_fence_before();
@@ -428,8 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         }
         softmax_bar();
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int ch = k * 128 + key, hh = ch >> 4, part = ch & 15;
+        for (int k = 0; k < 4; ++k) {
+          const int ch = k * 256 + st, hh = ch >> 4, part = ch & 15;
           *reinterpret_cast<uint4*>(out + ((size_t)hh * kD + mt * 128) * 2 + part * 16) =
               *reinterpret_cast<const uint4*>(P + hh * 256 + part * 16);
         }
@@ -443,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
     }
   } else {
     // ------------------------------------------------------------------ loaders (q~, then key tiles)
-    const int lt = tid - 160;                                 // 0..63: q~ head lt; key rows lt, lt + 64
+    const int lt = tid - 288;                                 // 0..63: q~ head lt; key rows lt, lt + 64
     bool ok = true;
     uint32_t g = 0, j = 0;
     for (int row = blockIdx.x; row < a.rows && ok; row += gridDim.x, ++j) {
@@ -503,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         }
         fence_proxy_async_smem();
         mbar_arrive(&bars->qfull);
-        if (tid == 160 && j < 8) PTRACE(88 + j);
+        if (tid == 288 && j < 8) PTRACE(88 + j);
       }
       // key tiles: rows lt and lt + 64 of each, block by block as the blocks come free; each block's
       // copies arrive on its barrier when they land, so all free blocks are in flight at once
@@ -513,8 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         for (int r = 0; r < 2; ++r) src[r] = slot_ptr(a, si, row, b, (int64_t)i * kKeys + lt + 64 * r);
         for (int c = 0; c < kBlocks; ++c) {
           if (!mbar_wait(&bars->kvfree[c], (g & 1u) ^ 1u)) { ok = false; break; }
-          if (tid == 160 && g < 16 && c == 0) PTRACE(128 + g);
-          if (tid == 160 && g < 16 && c == 7) PTRACE(144 + g);
+          if (tid == 288 && g < 16 && c == 0) PTRACE(128 + g);
+          if (tid == 288 && g < 16 && c == 7) PTRACE(144 + g);
           uint8_t* dst = KV + c * kBlockBytes;
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
@@ -525,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
           }
           cp_async_arrive(&bars->kvfull[c]);
         }
-        if (tid == 160 && g < 16) PTRACE(64 + g);
+        if (tid == 288 && g < 16) PTRACE(64 + g);
       }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
