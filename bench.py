@@ -760,10 +760,10 @@ def prefill_measure(workload, steps, warmup, queries=None):
            "work": {"indexer_fp8_tflop": idx_flops / 1e12, "attention_bf16_tflop": att_flops / 1e12,
                     "attention_gather_gb": gather_bytes / 1e9},
            "bf16_peak_tflops": bf16_peak, "peak_source": note, "clocks": clocks.summary(w0, w1)}
-    if n == 4:          # append+compress, indexer scores, top-k, attention: the call's launches in order
-        names = ["append_compress", "indexer", "topk", "attention"]
+    if n in (4, 5):     # append+compress, indexer scores, top-k, (q preparation,) attention, in order
+        names = ["append_compress", "indexer", "topk"] + (["q_preparation"] if n == 5 else []) + ["attention"]
         res["kernels_ms"] = dict(zip(names, launches_ms))
-        att_ms, idx_ms = launches_ms[3], launches_ms[1]
+        att_ms, idx_ms = launches_ms[n - 1], launches_ms[1]
         res["attention"] = {"kernel": "attend_prefill_tc_kernel" if layer.H == 64 and layer.kv_format == "bf16"
                             else "attend_mma_kernel", "ms": att_ms, "tflops": att_flops / (att_ms / 1e3) / 1e12,
                             "frac_of_bf16_peak": att_flops / (att_ms / 1e3) / 1e12 / bf16_peak}

@@ -235,7 +235,8 @@ Workspace layout(const csa_layer_t* L, int op, int32_t Tq, int64_t n_max) {
     const int64_t slots = (dense ? (n_max > 0 ? n_max : 1) : (int64_t)L->top_k) + L->window;
     const int splits = attend_num_splits(la, dense, (int)rows, slots, num_sms());
     w.part = off; w.part_bytes = attend_partial_bytes(la, dense, (int)rows, splits); off = up(off + w.part_bytes);
-    if (attend_path(la, dense, (int)rows) == 2) { w.qt = off; off = up(off + rows * (size_t)L->H * L->D * 2); }
+    const int ap = attend_path(la, dense, (int)rows);
+    if (ap == 2 || ap == 3) { w.qt = off; off = up(off + rows * (size_t)L->H * L->D * 2); }
     if (attend_path(la, dense, (int)rows) == 2 && dense) {
       w.extra = off; off = up(off + rows * 2 * (size_t)L->H * 4);
     }

@@ -1507,7 +1507,8 @@ size_t attend_partial_bytes(const LayerArgs& L, bool dense, int rows, int splits
 }
 
 cudaError_t launch_attend_qprep(const AttendArgs& a, cudaStream_t s) {
-  if (a.rows <= 0 || attend_path(a.L, a.topk == nullptr, a.rows) != 2) return cudaSuccess;
+  const int path = a.rows > 0 ? attend_path(a.L, a.topk == nullptr, a.rows) : 0;
+  if (path != 2 && path != 3) return cudaSuccess;
   return launch_kernel(qprep_kernel, dim3((unsigned)((a.L.H + 3) / 4), (unsigned)a.rows), dim3(128), 0, s, 0, a);
 }
 

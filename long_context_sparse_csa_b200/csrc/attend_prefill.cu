@@ -24,9 +24,9 @@
 //   warp 0      the MMA issuer (one thread)
 //   warps 1-8   softmax, two warps per TMEM lane quarter (32 heads each); then per query the
 //               epilogue: 1 / (l + 2^(sink - m)), the rotation by -t, the bf16 store
-//   warps 9-10  loaders: q~ of each query (one head per thread: RMSNorm, gamma, the rotation by +t,
-//               bf16), then its key tiles, two key rows per thread, in 16-byte cp.async pieces into
-//               the 128-byte-swizzled tile, block by block.  A 64-dim block is refilled for the next tile as soon as the
+//   warps 9-10  loaders: q~ of each query (made beforehand by the q preparation kernel), then its
+//               key tiles, two key rows per thread, in 16-byte cp.async pieces into the
+//               128-byte-swizzled tile, block by block.  A 64-dim block is refilled for the next tile as soon as the
 //               O^T MMAs that read it are done, while the other M-tiles still run.
 // Every mbarrier wait is bounded: a wait that gives up sets the device error word, and the role stops.
 #include <cuda_bf16.h>
@@ -62,15 +62,14 @@ struct __align__(8) PfBars {
 constexpr size_t kOffQ = (size_t)kBlocks * kBlockBytes;
 constexpr size_t kOffP = kOffQ + (size_t)kBlocks * kQBlockBytes;
 constexpr size_t kOffMx = kOffP + (size_t)kKeys * 128;
-constexpr size_t kOffRope = kOffMx + (4 * kHeads + 3 * kHeads + 4) * sizeof(float);
-constexpr size_t kOffBars = kOffRope + 64 * sizeof(float);
+constexpr size_t kOffBars = kOffMx + (4 * kHeads + 3 * kHeads + 4) * sizeof(float);
 constexpr size_t kSmemBytes = 1024 + kOffBars + sizeof(PfBars);
 static_assert(kSmemBytes <= 227 * 1024, "prefill attention shared memory");
 
 #ifdef CSA_TRACE
 // Diagnostic build only: per-CTA timestamps (ns) of the first tiles and queries.
-__device__ uint64_t g_trace_p[160][160];
-#define PTRACE(slot) do { if (blockIdx.x < 160 && (slot) < 160) g_trace_p[blockIdx.x][(slot)] = global_timer_ns(); } while (0)
+__device__ uint64_t g_trace_p[160][176];
+#define PTRACE(slot) do { if (blockIdx.x < 160 && (slot) < 176) g_trace_p[blockIdx.x][(slot)] = global_timer_ns(); } while (0)
 #else
 #define PTRACE(slot) ((void)0)
 #endif
@@ -147,7 +146,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
   float* alph = mrun + kHeads;                                  // [64] rescale factors of this tile
   float* fh = alph + kHeads;                                    // [64] output factors (epilogue)
   int* flag = reinterpret_cast<int*>(fh + kHeads);              // [2] any head of a half rescaled
-  float* rope_tab = reinterpret_cast<float*>(sm + kOffRope);    // [32][2] the query's rotary cos / sin (loaders)
   PfBars* bars = reinterpret_cast<PfBars*>(sm + kOffBars);
 
   const LayerArgs& L = a.L;
@@ -382,7 +380,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         fh[h] = m == -INFINITY ? 0.f : 1.f / (l + exp2f(sk - m));
       }
       softmax_bar();
+      if (tid == 32 && j < 2) PTRACE(160 + 8 * j);
       if (!mbar_wait(&bars->ofull, j & 1u)) { ok = false; break; }
+      if (tid == 32 && j < 2) PTRACE(161 + 8 * j);
       tc_fence_after();
       // per M-tile: this thread's dim of its heads -> a [64 heads][128 dims] bf16 staging tile in
       // P's buffer (free: the query's last P.V is done), then 16-byte coalesced stores of the rows
@@ -418,6 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
               *reinterpret_cast<const uint4*>(P + hh * 256 + part * 16);
         }
         softmax_bar();
+        if (tid == 32 && j < 2) PTRACE(162 + 8 * j + mt);
       }
       if (tid == 32 && j < 8) PTRACE(80 + j);
     }
@@ -434,57 +435,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
       const int64_t t = a.q_pos[row];
       const Slots si = slots_of(a, t);
       const int b = row / a.Tq;
-      // q~ of this query once the previous query's S^T MMAs are done with q~: the raw head row lands in
-      // its q~ slots (all of its copies in flight at once), then is normalised and rotated in place
+      // q~ of this query (made by the q preparation kernel) once the previous query's S^T MMAs are
+      // done with the buffer: head lt's 1 KB row into its swizzled slots, all 64 pieces in flight
       if (!mbar_wait(&bars->qfree, (j & 1u) ^ 1u)) { ok = false; break; }
-      // the query's 32 rotary angles, one float64 sincospi per thread, shared by the loaders
-      if (lt < 32) rope_cos_sin((double)t, lt, L, &rope_tab[2 * lt], &rope_tab[2 * lt + 1]);
-      asm volatile("barrier.sync.aligned 2, 64;" ::: "memory");
       {
         const int h = lt;
-        const uint8_t* src = a.q + ((size_t)row * kHeads + h) * kD * 2;
+        const uint8_t* src = a.qt + ((size_t)row * kHeads + h) * kD * 2;
 #pragma unroll 8
         for (int p = 0; p < 64; ++p) cp_async16(Q + (p >> 3) * kQBlockBytes + sw128(h, p & 7), src + 16 * p);
         asm volatile("cp.async.wait_all;" ::: "memory");
-        float ss = 0.f;
-#pragma unroll 8
-        for (int p = 0; p < 64; ++p) {
-          const uint4 u = *reinterpret_cast<const uint4*>(Q + (p >> 3) * kQBlockBytes + sw128(h, p & 7));
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float x0 = bf16_bits_to_f(w[q] & 0xFFFFu), x1 = bf16_bits_to_f(w[q] >> 16);
-            ss = fmaf(x0, x0, fmaf(x1, x1, ss));
-          }
-        }
-        const float rs = 1.0f / sqrtf(ss / (float)kD + L.eps);
-#pragma unroll 2
-        for (int p = 0; p < 64; ++p) {
-          const int d0 = 8 * p;
-          uint4* slot = reinterpret_cast<uint4*>(Q + (p >> 3) * kQBlockBytes + sw128(h, p & 7));
-          const uint4 u = *slot;
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-          float v[8];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            v[2 * q] = bf16_bits_to_f(w[q] & 0xFFFFu);
-            v[2 * q + 1] = bf16_bits_to_f(w[q] >> 16);
-          }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) v[e] *= rs * (a.gamma_q ? __ldg(a.gamma_q + d0 + e) : 1.f);
-          if (d0 >= kD - 64) {
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              const int u = (d0 + e - (kD - 64)) >> 1;
-              const float c = rope_tab[2 * u], sn = rope_tab[2 * u + 1];
-              const float x0 = v[e], x1 = v[e + 1];
-              v[e] = x0 * c - x1 * sn;
-              v[e + 1] = x0 * sn + x1 * c;
-            }
-          }
-          *slot = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                             pack_bf16x2(v[6], v[7]));
-        }
         fence_proxy_async_smem();
         mbar_arrive(&bars->qfull);
         if (tid == 288 && j < 8) PTRACE(88 + j);

@@ -198,8 +198,8 @@ int attend_path(const LayerArgs& L, bool dense, int rows);
 int attend_head_group(const LayerArgs& L);
 int attend_num_splits(const LayerArgs& L, bool dense, int rows, int64_t slots, int num_sms);
 size_t attend_partial_bytes(const LayerArgs& L, bool dense, int rows, int splits);
-// q~ for the tcgen05 kernel (a no-op for the other kernels, which prepare q themselves); it reads
-// only q, gamma_q and q_pos, so it may run beside compression.
+// q~ for the tcgen05 kernels, decode and prefill (a no-op for the other kernels, which prepare q
+// themselves); it reads only q, gamma_q and q_pos, so it may run beside compression.
 cudaError_t launch_attend_qprep(const AttendArgs& a, cudaStream_t s);
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s);
 bool attend_prefill_tc_supported(const LayerArgs& L, int rows);
