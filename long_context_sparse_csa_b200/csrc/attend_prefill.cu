@@ -389,26 +389,28 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
       uint8_t* out = a.out + (size_t)row * kHeads * kD * 2;
       uint16_t* stage = reinterpret_cast<uint16_t*>(P);
       const int st = tid - 32;                                // 0..255
-#pragma unroll 1
+      // all of this thread's O^T values at once, then O^T is released (the next query's first P.V
+      // may overwrite it while this query's output is still being stored)
+      float o[4][32];
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) tmem_ld_32x32b_x32(lane_addr + 256u + 64u * mt + h0, o[mt]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars->ofree);
+      if (tid == 32 && j < 2) PTRACE(162 + 8 * j + 4);
+#pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
         const int d = mt * 128 + key;
         float c = 1.f, sn = 0.f;
         const bool rot = d >= kD - 64;
         if (rot) rope_cos_sin((double)t, (d - (kD - 64)) >> 1, L, &c, &sn);
-        float o[32];
-        tmem_ld_32x32b_x32(lane_addr + 256u + 64u * mt + h0, o);
-        tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
-          float v = o[u] * fh[h0 + u];
+          float v = o[mt][u] * fh[h0 + u];
           // rotation by -t of the pair (d even, d + 1): partner in the neighbouring lane
           const float pv = __shfl_xor_sync(0xffffffffu, v, 1);
           if (rot) v = (d & 1) ? (-pv * sn + v * c) : (v * c + pv * sn);
           stage[(h0 + u) * 128 + key] = f_to_bf16_bits(v);
-        }
-        if (mt == 3) {                                        // every O^T column read: release it
-          tc_fence_before();
-          mbar_arrive(&bars->ofree);
         }
         softmax_bar();
 #pragma unroll
@@ -418,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
               *reinterpret_cast<const uint4*>(P + hh * 256 + part * 16);
         }
         softmax_bar();
-        if (tid == 32 && j < 2) PTRACE(162 + 8 * j + mt);
+        if (tid == 32 && j < 2 && mt < 3) PTRACE(162 + 8 * j + mt);
       }
       if (tid == 32 && j < 8) PTRACE(80 + j);
     }
