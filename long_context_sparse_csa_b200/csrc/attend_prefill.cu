@@ -55,7 +55,6 @@ struct __align__(8) PfBars {
   uint64_t kvfull[kBlocks], kvfree[kBlocks];
   uint64_t qfull, qfree, sfull, pfull, ofull, ofree, drain;
   uint32_t tmem_base;
-  int abort;
 };
 
 // shared memory: key tile 128 KB, q~ 64 KB, P 16 KB, then the small arrays
@@ -162,7 +161,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
     mbar_init(&bars->ofull, 1);
     mbar_init(&bars->ofree, 256);
     mbar_init(&bars->drain, 1);
-    bars->abort = 0;
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -228,7 +226,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
       }
       if (!ok) {
         set_device_error(a.err, kErrWaitTimeout);
-        atomicExch(&bars->abort, 1);
       }
       // nothing of this thread is in flight when TMEM is released
       if (issued) {
@@ -426,7 +423,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
     }
     if (!ok) {
       set_device_error(a.err, kErrWaitTimeout);
-      atomicExch(&bars->abort, 1);
     }
   } else {
     // ------------------------------------------------------------------ loaders (q~, then key tiles)
@@ -476,7 +472,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
     asm volatile("cp.async.wait_all;" ::: "memory");
     if (!ok) {
       set_device_error(a.err, kErrWaitTimeout);
-      atomicExch(&bars->abort, 1);
     }
   }
 
