@@ -17,7 +17,8 @@
 // reduce-scatter across the warp on bf16 pairs and shared memory across the four lane quarters.  A head's
 // running maximum moves only when its tile maximum exceeds it by more than 8 (in log2 units); then
 // O^T's column and the partial sums are rescaled.  Exponentials are taken against the running maximum,
-// so they stay below 2^8.  Each softmax thread keeps its key's partial sums per head; they are reduced
+// so they stay below 2^8; a tile none of whose scores exceeds its head's running maximum by more than
+// the margin skips the maxima altogether.  Each softmax thread keeps its key's partial sums per head; they are reduced
 // once per query, in the epilogue.
 //
 // Roles, in one persistent CTA per SM (query rows strided by the grid):
@@ -25,9 +26,9 @@
 //   warps 1-8   softmax, two warps per TMEM lane quarter (32 heads each); then per query the
 //               epilogue: 1 / (l + 2^(sink - m)), the rotation by -t, the bf16 store
 //   warps 9-10  loaders: q~ of each query (made beforehand by the q preparation kernel), then its
-//               key tiles, two key rows per thread, in 16-byte cp.async pieces into the
-//               128-byte-swizzled tile, block by block.  A 64-dim block is refilled for the next tile as soon as the
-//               O^T MMAs that read it are done, while the other M-tiles still run.
+//               key tiles in 16-byte cp.async pieces into the 128-byte-swizzled tile, block by block,
+//               eight threads per 128-byte row segment.  A 64-dim block is refilled for the next tile
+//               as soon as the O^T MMAs that read it are done, while the other M-tiles still run.
 // Every mbarrier wait is bounded: a wait that gives up sets the device error word, and the role stops.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -67,8 +68,8 @@ static_assert(kSmemBytes <= 227 * 1024, "prefill attention shared memory");
 
 #ifdef CSA_TRACE
 // Diagnostic build only: per-CTA timestamps (ns) of the first tiles and queries.
-__device__ uint64_t g_trace_p[160][176];
-#define PTRACE(slot) do { if (blockIdx.x < 160 && (slot) < 176) g_trace_p[blockIdx.x][(slot)] = global_timer_ns(); } while (0)
+__device__ uint64_t g_trace_p[160][208];
+#define PTRACE(slot) do { if (blockIdx.x < 160 && (slot) < 208) g_trace_p[blockIdx.x][(slot)] = global_timer_ns(); } while (0)
 #else
 #define PTRACE(slot) ((void)0)
 #endif
@@ -89,6 +90,19 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 }
 
 __device__ __forceinline__ void softmax_bar() { asm volatile("barrier.sync.aligned 1, 256;" ::: "memory"); }
+// Barrier of the 256 softmax threads that also returns whether any of them passed true.
+__device__ __forceinline__ bool softmax_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "barrier.red.or.pred p, 3, 256, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return (uint32_t)f_to_bf16_bits(lo) | ((uint32_t)f_to_bf16_bits(hi) << 16);
@@ -179,6 +193,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
     if (lane == 0) {
       const uint32_t idesc_s = instr_desc(kKeys, kHeads, 1u);                          // both K-major
       const uint32_t idesc_o = instr_desc(128, kHeads, 1u) | (1u << 15) | (1u << 16);  // both MN-major
+      // operand descriptors of the buffers' starts; the MMAs below add constant offsets (16-byte
+      // units) to these, so the issue sequence holds no address arithmetic
+      const uint64_t kv_k = desc_kmajor_sw128(smem_u32(KV));
+      const uint64_t q_k = desc_kmajor_sw128(smem_u32(Q));
+      const uint64_t kv_mn = desc_mnmajor_sw128(smem_u32(KV), kBlockBytes, 1024u);
+      const uint64_t p_mn = desc_mnmajor_sw128(smem_u32(P), kBlockBytes, 1024u);
       bool ok = true;
       uint32_t g = 0, j = 0;
       bool issued = false;
@@ -187,14 +207,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         if (!mbar_wait(&bars->qfull, j & 1u)) { ok = false; break; }
         for (int i = 0; i < si.tiles; ++i, ++g) {
           // S^T = K q~^T over the 8 blocks of this tile, as each block lands
+#pragma unroll
           for (int c = 0; c < kBlocks; ++c) {
             if (!mbar_wait(&bars->kvfull[c], g & 1u)) { ok = false; break; }
             fence_proxy_async_smem();                 // the loaders' copies, for the tensor core
             tc_fence_after();
-            const uint64_t ad = desc_kmajor_sw128(smem_u32(KV + c * kBlockBytes));
-            const uint64_t bd = desc_kmajor_sw128(smem_u32(Q + c * kQBlockBytes));
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) umma_f16(tmem, ad + 2u * kk, bd + 2u * kk, idesc_s, (c | kk) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f16(tmem, kv_k + (uint64_t)(c * (kBlockBytes >> 4) + 2 * kk),
+                       q_k + (uint64_t)(c * (kQBlockBytes >> 4) + 2 * kk), idesc_s, (c | kk) ? 1u : 0u);
             issued = true;
           }
           if (!ok) break;
@@ -207,19 +228,26 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
           if (g < 16) PTRACE(96 + g);
           if (i == 0 && !mbar_wait(&bars->ofree, (j & 1u) ^ 1u)) { ok = false; break; }
           tc_fence_after();
-#pragma unroll 1
+#pragma unroll
           for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
-            for (int kk = 0; kk < kKeys / 16; ++kk) {
-              const uint64_t ad = desc_mnmajor_sw128(smem_u32(KV + 2 * mt * kBlockBytes + kk * 2048), kBlockBytes, 1024u);
-              const uint64_t bd = desc_mnmajor_sw128(smem_u32(P + kk * 2048), kBlockBytes, 1024u);
-              umma_f16(tmem + 256u + 64u * (uint32_t)mt, ad, bd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < kKeys / 16; ++kk)
+              umma_f16(tmem + 256u + 64u * (uint32_t)mt, kv_mn + (uint64_t)((2 * mt * kBlockBytes + kk * 2048) >> 4),
+                       p_mn + (uint64_t)((kk * 2048) >> 4), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
             umma_commit(&bars->kvfree[2 * mt]);
             umma_commit(&bars->kvfree[2 * mt + 1]);
             if (mt == 0 && g < 16) PTRACE(112 + g);
           }
           if (g < 16) PTRACE(16 + g);
+#ifdef CSA_TRACE
+          // diagnostic build: completion of the first and last M-tiles as the issuer sees them
+          if (g < 16) {
+            mbar_wait(&bars->kvfree[1], g & 1u);
+            PTRACE(176 + g);
+            mbar_wait(&bars->kvfree[7], g & 1u);
+            PTRACE(192 + g);
+          }
+#endif
         }
         if (!ok) break;
         umma_commit(&bars->ofull);
@@ -265,49 +293,61 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         tmem_wait_ld();
 #pragma unroll
         for (int h = 0; h < 32; ++h) z[h] = valid ? z[h] * cl2 : -INFINITY;
-        // the tile's maxima per head: lanes (a butterfly over bf16 pairs, then the last pair's
-        // neighbours), then warps
-        {
-          uint32_t w[16];
+        // The tile's maxima are needed only where a score exceeds its head's running maximum by more
+        // than the margin (always on a query's first tile); otherwise the maxima stay as they are.
+        bool over = false;
 #pragma unroll
-          for (int q = 0; q < 16; ++q) w[q] = pack_bf16x2(z[2 * q], z[2 * q + 1]);
+        for (int q = 0; q < 8; ++q) {
+          const float4 m4 = reinterpret_cast<const float4*>(mrun + h0)[q];
+          over |= (z[4 * q] > m4.x + kRescale) | (z[4 * q + 1] > m4.y + kRescale) |
+                  (z[4 * q + 2] > m4.z + kRescale) | (z[4 * q + 3] > m4.w + kRescale);
+        }
+        bool moved = false;
+        if (softmax_any(over)) {
+          // the tile's maxima per head: lanes (a butterfly over bf16 pairs, then the last pair's
+          // neighbours), then warps
+          {
+            uint32_t w[16];
 #pragma unroll
-          for (int o = 16, n = 8; o >= 2; o >>= 1, n >>= 1) {
-            const bool upper = (lane & o) != 0;
+            for (int q = 0; q < 16; ++q) w[q] = pack_bf16x2(z[2 * q], z[2 * q + 1]);
 #pragma unroll
-            for (int q = 0; q < n; ++q) {
-              const uint32_t send = upper ? w[q] : w[q + n];
-              const uint32_t keep = upper ? w[q + n] : w[q];
-              w[q] = bf16x2_max(keep, __shfl_xor_sync(0xffffffffu, send, o));
+            for (int o = 16, n = 8; o >= 2; o >>= 1, n >>= 1) {
+              const bool upper = (lane & o) != 0;
+#pragma unroll
+              for (int q = 0; q < n; ++q) {
+                const uint32_t send = upper ? w[q] : w[q + n];
+                const uint32_t keep = upper ? w[q + n] : w[q];
+                w[q] = bf16x2_max(keep, __shfl_xor_sync(0xffffffffu, send, o));
+              }
+            }
+            w[0] = bf16x2_max(w[0], __shfl_xor_sync(0xffffffffu, w[0], 1));
+            // lanes 2k and 2k + 1 now hold heads h0 + 2k, h0 + 2k + 1
+            if ((lane & 1) == 0) {
+              mx[w4 * kHeads + h0 + lane] = bf16_bits_to_f(w[0] & 0xFFFFu);
+              mx[w4 * kHeads + h0 + lane + 1] = bf16_bits_to_f(w[0] >> 16);
             }
           }
-          w[0] = bf16x2_max(w[0], __shfl_xor_sync(0xffffffffu, w[0], 1));
-          // lanes 2k and 2k + 1 now hold heads h0 + 2k, h0 + 2k + 1
-          if ((lane & 1) == 0) {
-            mx[w4 * kHeads + h0 + lane] = bf16_bits_to_f(w[0] & 0xFFFFu);
-            mx[w4 * kHeads + h0 + lane + 1] = bf16_bits_to_f(w[0] >> 16);
+          softmax_bar();
+          if (w4 == 0) {
+            const int h = h0 + lane;
+            const float tm = fmaxf(fmaxf(mx[h], mx[kHeads + h]), fmaxf(mx[2 * kHeads + h], mx[3 * kHeads + h]));
+            const float mr = mrun[h];
+            float al = 1.f;
+            int mv = 0;
+            if (tm > mr + kRescale || (mr == -INFINITY && tm > -INFINITY)) {
+              al = mr == -INFINITY ? 0.f : exp2f(mr - tm);
+              mrun[h] = tm;
+              mv = 1;
+            }
+            alph[h] = al;
+            mv = __any_sync(0xffffffffu, mv);
+            if (lane == 0) flag[hf] = mv;
           }
+          softmax_bar();
+          moved = (flag[0] | flag[1]) != 0;
         }
-        softmax_bar();
-        if (w4 == 0) {
-          const int h = h0 + lane;
-          const float tm = fmaxf(fmaxf(mx[h], mx[kHeads + h]), fmaxf(mx[2 * kHeads + h], mx[3 * kHeads + h]));
-          const float mr = mrun[h];
-          float al = 1.f;
-          int moved = 0;
-          if (tm > mr + kRescale || (mr == -INFINITY && tm > -INFINITY)) {
-            al = mr == -INFINITY ? 0.f : exp2f(mr - tm);
-            mrun[h] = tm;
-            moved = 1;
-          }
-          alph[h] = al;
-          moved = __any_sync(0xffffffffu, moved);
-          if (lane == 0) flag[hf] = moved;
-        }
-        softmax_bar();
         // P = 2^(z - m) in bf16, this key's row of P (its heads' 64 bytes); the partial sums
         // (rescaled where the head's maximum moved) take the rounded values
-        const bool moved = (flag[0] | flag[1]) != 0;
         uint8_t* prow = P;
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
@@ -426,44 +466,46 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
     }
   } else {
     // ------------------------------------------------------------------ loaders (q~, then key tiles)
-    const int lt = tid - 288;                                 // 0..63: q~ head lt; key rows lt, lt + 64
+    // Consecutive threads copy consecutive 16-byte pieces: eight threads cover one 128-byte row
+    // segment, so a warp's copy reads four whole segments and writes four whole swizzled rows.
+    const int lt = tid - 288;                                 // 0..63
+    const int lrow = lt >> 3, lp = lt & 7;                    // row within an 8-row group, piece
     bool ok = true;
     uint32_t g = 0, j = 0;
     for (int row = blockIdx.x; row < a.rows && ok; row += gridDim.x, ++j) {
       const int64_t t = a.q_pos[row];
       const Slots si = slots_of(a, t);
       const int b = row / a.Tq;
-      // q~ of this query (made by the q preparation kernel) once the previous query's S^T MMAs are
-      // done with the buffer: head lt's 1 KB row into its swizzled slots, all 64 pieces in flight
+      // q~ of this query (made by the q preparation kernel, 64 KB contiguous) once the previous
+      // query's S^T MMAs are done with the buffer
       if (!mbar_wait(&bars->qfree, (j & 1u) ^ 1u)) { ok = false; break; }
       {
-        const int h = lt;
-        const uint8_t* src = a.qt + ((size_t)row * kHeads + h) * kD * 2;
+        const uint8_t* src = a.qt + (size_t)row * kHeads * kD * 2;
 #pragma unroll 8
-        for (int p = 0; p < 64; ++p) cp_async16(Q + (p >> 3) * kQBlockBytes + sw128(h, p & 7), src + 16 * p);
+        for (int h = 0; h < kHeads; ++h)
+          cp_async16(Q + (lt >> 3) * kQBlockBytes + sw128(h, lt & 7), src + (size_t)h * kD * 2 + 16 * lt);
         asm volatile("cp.async.wait_all;" ::: "memory");
         fence_proxy_async_smem();
         mbar_arrive(&bars->qfull);
         if (tid == 288 && j < 8) PTRACE(88 + j);
       }
-      // key tiles: rows lt and lt + 64 of each, block by block as the blocks come free; each block's
-      // copies arrive on its barrier when they land, so all free blocks are in flight at once
+      // key tiles, block by block as the blocks come free; each block's copies arrive on its barrier
+      // when they land, so all free blocks are in flight at once
       for (int i = 0; i < si.tiles && ok; ++i, ++g) {
-        const uint8_t* src[2];
+        // this thread's piece of the tile's rows 8 it + lrow (an empty slot copies the zero row)
+        const uint8_t* src[16];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) src[r] = slot_ptr(a, si, row, b, (int64_t)i * kKeys + lt + 64 * r);
+        for (int it = 0; it < 16; ++it) {
+          const uint8_t* sp = slot_ptr(a, si, row, b, (int64_t)i * kKeys + 8 * it + lrow);
+          src[it] = (sp ? sp : g_zero_row) + 16 * lp;
+        }
         for (int c = 0; c < kBlocks; ++c) {
           if (!mbar_wait(&bars->kvfree[c], (g & 1u) ^ 1u)) { ok = false; break; }
           if (tid == 288 && g < 16 && c == 0) PTRACE(128 + g);
           if (tid == 288 && g < 16 && c == 7) PTRACE(144 + g);
           uint8_t* dst = KV + c * kBlockBytes;
 #pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const int kr = lt + 64 * r;
-            const uint8_t* from = src[r] ? src[r] + c * 128 : g_zero_row + c * 128;
-#pragma unroll
-            for (int p = 0; p < 8; ++p) cp_async16(dst + sw128(kr, p), from + p * 16);
-          }
+          for (int it = 0; it < 16; ++it) cp_async16(dst + sw128(8 * it + lrow, lp), src[it] + c * 128);
           cp_async_arrive(&bars->kvfull[c]);
         }
         if (tid == 288 && g < 16) PTRACE(64 + g);
