@@ -23,12 +23,12 @@
 //
 // Roles, in one persistent CTA per SM (query rows strided by the grid):
 //   warp 0      the MMA issuer (one thread)
-//   warps 1-8   softmax, two warps per TMEM lane quarter (32 heads each); then per query the
-//               epilogue: 1 / (l + 2^(sink - m)), the rotation by -t, the bf16 store
-//   warps 9-10  loaders: q~ of each query (made beforehand by the q preparation kernel), then its
-//               key tiles in 16-byte cp.async pieces into the 128-byte-swizzled tile, block by block,
-//               eight threads per 128-byte row segment.  A 64-dim block is refilled for the next tile
-//               as soon as the O^T MMAs that read it are done, while the other M-tiles still run.
+//   warps 1-8   softmax, two warps per TMEM lane quarter (32 heads each); after a tile's P they copy
+//               the next tile's key rows in 16-byte cp.async pieces into the 128-byte-swizzled tile,
+//               eight threads per 128-byte row segment, block by block: a 64-dim block is refilled as
+//               soon as the O^T MMAs that read it are done, while the other M-tiles still run.  Per
+//               query the epilogue: 1 / (l + 2^(sink - m)), the rotation by -t, the bf16 store
+//   warps 9-10  q~ loaders (q~ made beforehand by the q preparation kernel)
 // Every mbarrier wait is bounded: a wait that gives up sets the device error word, and the role stops.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -49,8 +49,12 @@ constexpr int kBlocks = 8;                    // 64-dim column blocks of a row
 constexpr int kBlockBytes = kKeys * 128;      // one block of the key tile: 16 KB
 constexpr int kQBlockBytes = kHeads * 128;    // one block of q~: 8 KB
 constexpr int kThreads = 352;                 // warp 0 MMA, warps 1-8 softmax, warps 9-10 loaders
-constexpr int kLoaders = 64;
+constexpr int kLoaders = 64;                  // q~ loaders
+constexpr int kCopiers = 256;                 // key tile copies (the softmax threads)
 constexpr float kRescale = 8.f;               // log2 margin before a running maximum moves
+// A head's running maximum before any key was seen: finite, so that 2^(z - m) needs no special
+// case (a masked score, -inf, still gives 0) and m + kRescale stays below every finite score.
+constexpr float kNoMax = -3.0e38f;
 
 struct __align__(8) PfBars {
   uint64_t kvfull[kBlocks], kvfree[kBlocks];
@@ -68,8 +72,8 @@ static_assert(kSmemBytes <= 227 * 1024, "prefill attention shared memory");
 
 #ifdef CSA_TRACE
 // Diagnostic build only: per-CTA timestamps (ns) of the first tiles and queries.
-__device__ uint64_t g_trace_p[160][208];
-#define PTRACE(slot) do { if (blockIdx.x < 160 && (slot) < 208) g_trace_p[blockIdx.x][(slot)] = global_timer_ns(); } while (0)
+__device__ uint64_t g_trace_p[160][272];
+#define PTRACE(slot) do { if (blockIdx.x < 160 && (slot) < 272) g_trace_p[blockIdx.x][(slot)] = global_timer_ns(); } while (0)
 #else
 #define PTRACE(slot) ((void)0)
 #endif
@@ -102,6 +106,15 @@ __device__ __forceinline__ bool softmax_any(bool v) {
       : "r"((uint32_t)v)
       : "memory");
   return r != 0;
+}
+
+// 2^x by the MUFU approximation (ex2.approx.ftz): relative error about 2^-22, results below 2^-126
+// flushed to 0.  The arguments here are at most the rescale margin, and the results are rounded to
+// bf16 or summed with them.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -142,6 +155,66 @@ __device__ __forceinline__ const uint8_t* slot_ptr(const AttendArgs& a, const Sl
   return nullptr;
 }
 
+// A copying thread's view of a key tile: the loads it needs (the query position and the top-k
+// entries of its four rows 32 it + crow), issued early, and the row addresses formed from them later.
+struct TileRaw {
+  int64_t t;
+  int32_t e[4];
+};
+
+__device__ __forceinline__ TileRaw tile_raw(const AttendArgs& a, int row, int i, int crow) {
+  TileRaw r;
+  r.t = a.q_pos[row];
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int s = i * kKeys + 32 * it + crow;
+    r.e[it] = (a.topk && s < a.L.top_k) ? __ldg(a.topk + (size_t)row * a.L.top_k + s) : s;
+  }
+  return r;
+}
+
+struct TileSrc {
+  const uint8_t* p[4];
+};
+
+// Piece `piece` of each of the four rows (an empty slot reads the zero row); the same slots as
+// slot_ptr, from the loaded entries.
+__device__ __forceinline__ TileSrc tile_src(const AttendArgs& a, const TileRaw& raw, int row, int i, int crow,
+                                            int piece) {
+  const Slots si = slots_of(a, raw.t);
+  const int b = row / a.Tq;
+  const CacheArgs& C = a.C;
+  TileSrc r;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int64_t s = (int64_t)i * kKeys + 32 * it + crow;
+    const uint8_t* sp = nullptr;
+    if (s < si.n_sel) {
+      const int64_t e = raw.e[it];
+      if (e >= 0 && e < C.entry_cap) sp = C.entries + ((size_t)b * C.entry_cap + (size_t)e) * a.L.row_bytes;
+    } else if (s < si.R) {
+      const int64_t wr = si.rt - si.n_win + 1 + (s - si.n_sel);
+      sp = C.window + ((size_t)b * C.window_cap + (size_t)(wr % C.window_cap)) * a.L.row_bytes;
+    }
+    r.p[it] = (sp ? sp : g_zero_row) + 16 * piece;
+  }
+  return r;
+}
+
+// Copies of tile g into the key buffer, block by block: block c once the O^T MMAs of tile g - 1 are
+// done with it; each block's copies arrive on its barrier when they land.  False if a wait gave up.
+__device__ __forceinline__ bool copy_tile(uint8_t* KV, PfBars* bars, const TileSrc& src, uint32_t g, int crow,
+                                          int piece) {
+  for (int c = 0; c < kBlocks; ++c) {
+    if (!mbar_wait(&bars->kvfree[c], (g & 1u) ^ 1u)) return false;
+    uint8_t* dst = KV + c * kBlockBytes;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) cp_async16(dst + sw128(32 * it + crow, piece), src.p[it] + c * 128);
+    cp_async_arrive(&bars->kvfull[c]);
+  }
+  return true;
+}
+
 __device__ __forceinline__ uint32_t bf16x2_max(uint32_t x, uint32_t y) {
   __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&x), b = *reinterpret_cast<__nv_bfloat162*>(&y);
   __nv_bfloat162 r = __hmax2(a, b);
@@ -165,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int c = 0; c < kBlocks; ++c) {
-      mbar_init(&bars->kvfull[c], kLoaders);
+      mbar_init(&bars->kvfull[c], kCopiers);
       mbar_init(&bars->kvfree[c], 1);
     }
     mbar_init(&bars->qfull, kLoaders);
@@ -210,6 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
 #pragma unroll
           for (int c = 0; c < kBlocks; ++c) {
             if (!mbar_wait(&bars->kvfull[c], g & 1u)) { ok = false; break; }
+            if (c == 0 && g < 16) PTRACE(256 + g);
             fence_proxy_async_smem();                 // the loaders' copies, for the tensor core
             tc_fence_after();
 #pragma unroll
@@ -271,8 +345,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
     const int h0 = 32 * hf;
     const int key = w4 * 32 + lane;                           // key of S^T, dim of O^T's M-tile
     const uint32_t lane_addr = tmem + ((uint32_t)(w4 * 32) << 16);
+    // Between a tile's P and the next tile's S^T these threads are idle, so they copy the next
+    // tile's key rows, block by block as the O^T MMAs release the blocks: thread st copies piece
+    // st % 8 of rows 32 it + st / 8 (it < 4), so eight threads cover a 128-byte row segment.  The
+    // loads those copies need are issued before the softmax and used after it.
+    const int st = tid - 32;                                  // 0..255
+    const int crow = st >> 3, cpiece = st & 7;
     bool ok = true;
     uint32_t g = 0, j = 0;
+    if (blockIdx.x < a.rows) {
+      const TileRaw raw = tile_raw(a, blockIdx.x, 0, crow);
+      ok = copy_tile(KV, bars, tile_src(a, raw, blockIdx.x, 0, crow, cpiece), 0u, crow, cpiece);
+    }
     for (int row = blockIdx.x; row < a.rows && ok; row += gridDim.x, ++j) {
       const int64_t t = a.q_pos[row];
       const Slots si = slots_of(a, t);
@@ -280,9 +364,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
       float lp[32];                                           // this key's partial sums of its heads
 #pragma unroll
       for (int h = 0; h < 32; ++h) lp[h] = 0.f;
-      if (hf == 0 && key < kHeads) mrun[key] = -INFINITY;
+      if (hf == 0 && key < kHeads) mrun[key] = kNoMax;
       softmax_bar();
       for (int i = 0; i < si.tiles; ++i, ++g) {
+        // the tile after this one: the next of this query, or the first of the CTA's next query
+        const bool more = i + 1 < si.tiles || row + (int)gridDim.x < a.rows;
+        const int row_n = i + 1 < si.tiles ? row : row + (int)gridDim.x;
+        const int i_n = i + 1 < si.tiles ? i + 1 : 0;
+        TileRaw raw_n;
+        if (more) raw_n = tile_raw(a, row_n, i_n, crow);
         const int64_t s = (int64_t)i * kKeys + key;
         const bool valid = slot_ptr(a, si, row, b, s) != nullptr;
         if (!mbar_wait(&bars->sfull, g & 1u)) { ok = false; break; }
@@ -291,6 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         float z[32];
         tmem_ld_32x32b_x32(lane_addr + (uint32_t)h0, z);
         tmem_wait_ld();
+        if (tid == 32 && g < 16) PTRACE(208 + g);
 #pragma unroll
         for (int h = 0; h < 32; ++h) z[h] = valid ? z[h] * cl2 : -INFINITY;
         // The tile's maxima are needed only where a score exceeds its head's running maximum by more
@@ -303,7 +394,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
                   (z[4 * q + 2] > m4.z + kRescale) | (z[4 * q + 3] > m4.w + kRescale);
         }
         bool moved = false;
-        if (softmax_any(over)) {
+        const bool any_over = softmax_any(over);
+        if (tid == 32 && g < 16) PTRACE(224 + g);
+        if (any_over) {
           // the tile's maxima per head: lanes (a butterfly over bf16 pairs, then the last pair's
           // neighbours), then warps
           {
@@ -334,8 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
             const float mr = mrun[h];
             float al = 1.f;
             int mv = 0;
-            if (tm > mr + kRescale || (mr == -INFINITY && tm > -INFINITY)) {
-              al = mr == -INFINITY ? 0.f : exp2f(mr - tm);
+            if (tm > mr + kRescale) {
+              al = fast_exp2(mr - tm);                // 0 on the first move
               mrun[h] = tm;
               mv = 1;
             }
@@ -363,8 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
           for (int q = 0; q < 4; ++q) {
             const int h = 8 * jj + 2 * q;
             const float m0 = mm[2 * q], m1 = mm[2 * q + 1];
-            const float p0 = m0 == -INFINITY ? 0.f : exp2f(z[h] - m0);
-            const float p1 = m1 == -INFINITY ? 0.f : exp2f(z[h + 1] - m1);
+            const float p0 = fast_exp2(z[h] - m0);
+            const float p1 = fast_exp2(z[h + 1] - m1);
             w[q] = pack_bf16x2(p0, p1);
             if (moved) {
               lp[h] *= aa[2 * q];
@@ -375,6 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
           }
           *reinterpret_cast<uint4*>(prow + sw128(key, 4 * hf + jj)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
+        if (tid == 32 && g < 16) PTRACE(240 + g);
         // rescale O^T, the previous tiles' sum (complete, as this tile's S^T is), where a maximum moved
         if (moved && i > 0) {
 #pragma unroll 1
@@ -392,6 +486,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         tc_fence_before();
         mbar_arrive(&bars->pfull);
         if (tid == 32 && g < 16) PTRACE(48 + g);
+        if (more && !copy_tile(KV, bars, tile_src(a, raw_n, row_n, i_n, crow, cpiece), g + 1, crow, cpiece)) {
+          ok = false;
+          break;
+        }
+        if (tid == 32 && g < 16) PTRACE(64 + g);
       }
       if (!ok) break;
       // ---------------------------------------------------------------- epilogue of this query
@@ -414,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         const float m = mrun[h];
         const float sk = a.sinks[h] * kLog2e;
         // o = O / (l + 2^(sink - m)), O and l relative to the running maximum m
-        fh[h] = m == -INFINITY ? 0.f : 1.f / (l + exp2f(sk - m));
+        fh[h] = m == kNoMax ? 0.f : 1.f / (l + exp2f(sk - m));
       }
       softmax_bar();
       if (tid == 32 && j < 2) PTRACE(160 + 8 * j);
@@ -425,7 +524,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
       // P's buffer (free: the query's last P.V is done), then 16-byte coalesced stores of the rows
       uint8_t* out = a.out + (size_t)row * kHeads * kD * 2;
       uint16_t* stage = reinterpret_cast<uint16_t*>(P);
-      const int st = tid - 32;                                // 0..255
       // all of this thread's O^T values at once, then O^T is released (the next query's first P.V
       // may overwrite it while this query's output is still being stored)
       float o[4][32];
@@ -461,21 +559,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
       }
       if (tid == 32 && j < 8) PTRACE(80 + j);
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     if (!ok) {
       set_device_error(a.err, kErrWaitTimeout);
     }
   } else {
-    // ------------------------------------------------------------------ loaders (q~, then key tiles)
-    // Consecutive threads copy consecutive 16-byte pieces: eight threads cover one 128-byte row
-    // segment, so a warp's copy reads four whole segments and writes four whole swizzled rows.
+    // ------------------------------------------------------------------ q~ loaders
+    // Consecutive threads copy consecutive 16-byte pieces of a head's row.
     const int lt = tid - 288;                                 // 0..63
-    const int lrow = lt >> 3, lp = lt & 7;                    // row within an 8-row group, piece
     bool ok = true;
-    uint32_t g = 0, j = 0;
+    uint32_t j = 0;
     for (int row = blockIdx.x; row < a.rows && ok; row += gridDim.x, ++j) {
-      const int64_t t = a.q_pos[row];
-      const Slots si = slots_of(a, t);
-      const int b = row / a.Tq;
       // q~ of this query (made by the q preparation kernel, 64 KB contiguous) once the previous
       // query's S^T MMAs are done with the buffer
       if (!mbar_wait(&bars->qfree, (j & 1u) ^ 1u)) { ok = false; break; }
@@ -488,27 +582,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
         fence_proxy_async_smem();
         mbar_arrive(&bars->qfull);
         if (tid == 288 && j < 8) PTRACE(88 + j);
-      }
-      // key tiles, block by block as the blocks come free; each block's copies arrive on its barrier
-      // when they land, so all free blocks are in flight at once
-      for (int i = 0; i < si.tiles && ok; ++i, ++g) {
-        // this thread's piece of the tile's rows 8 it + lrow (an empty slot copies the zero row)
-        const uint8_t* src[16];
-#pragma unroll
-        for (int it = 0; it < 16; ++it) {
-          const uint8_t* sp = slot_ptr(a, si, row, b, (int64_t)i * kKeys + 8 * it + lrow);
-          src[it] = (sp ? sp : g_zero_row) + 16 * lp;
-        }
-        for (int c = 0; c < kBlocks; ++c) {
-          if (!mbar_wait(&bars->kvfree[c], (g & 1u) ^ 1u)) { ok = false; break; }
-          if (tid == 288 && g < 16 && c == 0) PTRACE(128 + g);
-          if (tid == 288 && g < 16 && c == 7) PTRACE(144 + g);
-          uint8_t* dst = KV + c * kBlockBytes;
-#pragma unroll
-          for (int it = 0; it < 16; ++it) cp_async16(dst + sw128(8 * it + lrow, lp), src[it] + c * 128);
-          cp_async_arrive(&bars->kvfull[c]);
-        }
-        if (tid == 288 && g < 16) PTRACE(64 + g);
       }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
