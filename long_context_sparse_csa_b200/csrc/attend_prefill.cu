@@ -59,6 +59,7 @@ constexpr float kNoMax = -3.0e38f;
 struct __align__(8) PfBars {
   uint64_t kvfull[kBlocks], kvfree[kBlocks];
   uint64_t qfull, qfree, sfull, pfull, ofull, ofree, drain;
+  uint64_t ropefull[2];
   uint32_t tmem_base;
 };
 
@@ -66,7 +67,8 @@ struct __align__(8) PfBars {
 constexpr size_t kOffQ = (size_t)kBlocks * kBlockBytes;
 constexpr size_t kOffP = kOffQ + (size_t)kBlocks * kQBlockBytes;
 constexpr size_t kOffMx = kOffP + (size_t)kKeys * 128;
-constexpr size_t kOffBars = kOffMx + (4 * kHeads + 3 * kHeads + 4) * sizeof(float);
+constexpr size_t kOffRope = kOffMx + (4 * kHeads + 3 * kHeads + 4) * sizeof(float);
+constexpr size_t kOffBars = kOffRope + 2 * 32 * sizeof(float2);
 constexpr size_t kSmemBytes = 1024 + kOffBars + sizeof(PfBars);
 static_assert(kSmemBytes <= 227 * 1024, "prefill attention shared memory");
 
@@ -232,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
   float* alph = mrun + kHeads;                                  // [64] rescale factors of this tile
   float* fh = alph + kHeads;                                    // [64] output factors (epilogue)
   int* flag = reinterpret_cast<int*>(fh + kHeads);              // [2] any head of a half rescaled
+  float2* rope_cs = reinterpret_cast<float2*>(sm + kOffRope);  // [2 queries][32 pairs] (cos, sin)
   PfBars* bars = reinterpret_cast<PfBars*>(sm + kOffBars);
 
   const LayerArgs& L = a.L;
@@ -248,6 +251,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
     mbar_init(&bars->ofull, 1);
     mbar_init(&bars->ofree, 256);
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->ropefull[0], 32);
+    mbar_init(&bars->ropefull[1], 32);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -520,41 +525,64 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
       if (!mbar_wait(&bars->ofull, j & 1u)) { ok = false; break; }
       if (tid == 32 && j < 2) PTRACE(161 + 8 * j);
       tc_fence_after();
-      // per M-tile: this thread's dim of its heads -> a [64 heads][128 dims] bf16 staging tile in
-      // P's buffer (free: the query's last P.V is done), then 16-byte coalesced stores of the rows
+      // per M-tile: this thread's dim of its 32 heads -> the warp's own [32 heads][32 dims] bf16
+      // staging tile in P's buffer (free: the query's last P.V is done), then 16-byte stores of
+      // its heads' 64-byte row pieces
       uint8_t* out = a.out + (size_t)row * kHeads * kD * 2;
-      uint16_t* stage = reinterpret_cast<uint16_t*>(P);
-      // all of this thread's O^T values at once, then O^T is released (the next query's first P.V
-      // may overwrite it while this query's output is still being stored)
-      float o[4][32];
+      uint16_t* wst = reinterpret_cast<uint16_t*>(P) + (warp - 1) * 32 * 32;
+      // all of this thread's O^T values, then O^T is released (the next query's first P.V may
+      // overwrite it while this query's output is still being stored).  Scaled by the heads' output
+      // factors on the way; M-tiles 0-2 (no rotary dims) are rounded to bf16 at once, in pairs of
+      // heads, the last M-tile stays in fp32 for the rotation.
+      uint32_t ob[3][16];
+      float o3[32];
+      {
+        float o[3][32];
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt) tmem_ld_32x32b_x32(lane_addr + 256u + 64u * mt + h0, o[mt]);
+        for (int mt = 0; mt < 3; ++mt) tmem_ld_32x32b_x32(lane_addr + 256u + 64u * mt + h0, o[mt]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; u += 2) {
+          const float f0 = fh[h0 + u], f1 = fh[h0 + u + 1];
+#pragma unroll
+          for (int mt = 0; mt < 3; ++mt) ob[mt][u >> 1] = pack_bf16x2(o[mt][u] * f0, o[mt][u + 1] * f1);
+        }
+      }
+      tmem_ld_32x32b_x32(lane_addr + 256u + 64u * 3 + h0, o3);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&bars->ofree);
       if (tid == 32 && j < 2) PTRACE(162 + 8 * j + 4);
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
-        const int d = mt * 128 + key;
-        float c = 1.f, sn = 0.f;
-        const bool rot = d >= kD - 64;
-        if (rot) rope_cos_sin((double)t, (d - (kD - 64)) >> 1, L, &c, &sn);
+      for (int u = 0; u < 32; ++u) o3[u] *= fh[h0 + u];
+      if (!mbar_wait(&bars->ropefull[j & 1u], (j >> 1) & 1u)) { ok = false; break; }
+      // the rotary dims (the last 64) are the upper half of the last M-tile: whole warps
+      if (w4 >= 2) {
+        const int d = 3 * 128 + key;
+        const float2 cs = rope_cs[(j & 1u) * 32 + ((d - (kD - 64)) >> 1)];
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
-          float v = o[mt][u] * fh[h0 + u];
           // rotation by -t of the pair (d even, d + 1): partner in the neighbouring lane
-          const float pv = __shfl_xor_sync(0xffffffffu, v, 1);
-          if (rot) v = (d & 1) ? (-pv * sn + v * c) : (v * c + pv * sn);
-          stage[(h0 + u) * 128 + key] = f_to_bf16_bits(v);
+          const float v = o3[u], pv = __shfl_xor_sync(0xffffffffu, v, 1);
+          o3[u] = (d & 1) ? (-pv * cs.y + v * cs.x) : (v * cs.x + pv * cs.y);
         }
-        softmax_bar();
+      }
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+        for (int u = 0; u < 32; u += 2) {
+          uint32_t w2 = mt < 3 ? ob[mt < 3 ? mt : 0][u >> 1] : pack_bf16x2(o3[u], o3[u + 1]);
+          wst[u * 32 + lane] = (uint16_t)(w2 & 0xFFFFu);
+          wst[(u + 1) * 32 + lane] = (uint16_t)(w2 >> 16);
+        }
+        __syncwarp();
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int ch = k * 256 + st, hh = ch >> 4, part = ch & 15;
-          *reinterpret_cast<uint4*>(out + ((size_t)hh * kD + mt * 128) * 2 + part * 16) =
-              *reinterpret_cast<const uint4*>(P + hh * 256 + part * 16);
+          const int q = k * 32 + lane, u = q >> 2, part = q & 3;
+          *reinterpret_cast<uint4*>(out + ((size_t)(h0 + u) * kD + mt * 128 + w4 * 32) * 2 + part * 16) =
+              *reinterpret_cast<const uint4*>(wst + u * 32 + part * 8);
         }
-        softmax_bar();
+        __syncwarp();
         if (tid == 32 && j < 2 && mt < 3) PTRACE(162 + 8 * j + mt);
       }
       if (tid == 32 && j < 8) PTRACE(80 + j);
@@ -578,6 +606,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_tc_kernel(const __
 #pragma unroll 8
         for (int h = 0; h < kHeads; ++h)
           cp_async16(Q + (lt >> 3) * kQBlockBytes + sw128(h, lt & 7), src + (size_t)h * kD * 2 + 16 * lt);
+        // the rotation angles of this query's output (its 32 rotary pairs), while the copies land
+        if (lt < 32) {
+          float c, sn;
+          rope_cos_sin((double)a.q_pos[row], lt, L, &c, &sn);
+          rope_cs[(j & 1u) * 32 + lt] = make_float2(c, sn);
+          mbar_arrive(&bars->ropefull[j & 1u]);
+        }
         asm volatile("cp.async.wait_all;" ::: "memory");
         fence_proxy_async_smem();
         mbar_arrive(&bars->qfull);
