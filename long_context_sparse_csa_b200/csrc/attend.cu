@@ -759,12 +759,9 @@ static_assert(tc_smem_bytes(kTcN) <= 227 * 1024, "tcgen05 attention shared memor
 
 // q~ = RoPE_t(RMSNorm(q) * gamma_q) in bf16, once per (query, head): one warp per head, lane l
 // holds dims [16l, 16l+16) (the rotary pairs sit in lanes 28..31).
-__global__ void __launch_bounds__(128) qprep_kernel(const __grid_constant__ AttendArgs a) {
+// q~ of one (row, head): RMSNorm, gamma, the rotation of the last 64 dims by the row's angles rcs.
+__device__ __forceinline__ void qprep_head(const AttendArgs& a, int row, int h, int lane, const float2* rcs) {
   const LayerArgs& L = a.L;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.y, h = blockIdx.x * 4 + warp;
-  if (h >= L.H) return;
-  const int64_t t = a.q_pos[row];
   const size_t ab = L.act_fmt == CSA_FMT_F32 ? 4 : 2;
   const uint8_t* qrow = a.q + ((size_t)row * L.H + h) * kD * ab;
   float gm[16], v[16];
@@ -791,7 +788,11 @@ __global__ void __launch_bounds__(128) qprep_kernel(const __grid_constant__ Atte
   float cs[8], sn[8];
   if (lane >= 28) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) rope_cos_sin((double)t, (16 * lane + 2 * k - (kD - 64)) >> 1, L, &cs[k], &sn[k]);
+    for (int k = 0; k < 8; ++k) {
+      const float2 r = rcs[(16 * lane + 2 * k - (kD - 64)) >> 1];
+      cs[k] = r.x;
+      sn[k] = r.y;
+    }
   }
   float ss = 0.f;
 #pragma unroll
@@ -818,6 +819,27 @@ __global__ void __launch_bounds__(128) qprep_kernel(const __grid_constant__ Atte
   dst[1] = p1;
 }
 
+
+__global__ void __launch_bounds__(128) qprep_kernel(const __grid_constant__ AttendArgs a, int hpc) {
+  const LayerArgs& L = a.L;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.y;
+  const int64_t t = a.q_pos[row];
+  // the row's 32 rotation angles (the last 64 dims), once per CTA, one per thread
+  __shared__ float2 rcs[32];
+  if (threadIdx.x < 32) {
+    float c, sn;
+    rope_cos_sin((double)t, (int)threadIdx.x, L, &c, &sn);
+    rcs[threadIdx.x] = make_float2(c, sn);
+  }
+  __syncthreads();
+  // heads [hpc blockIdx.x, hpc blockIdx.x + hpc), one warp each in turn
+  for (int hh = warp; hh < hpc; hh += 4) {
+    const int h = blockIdx.x * hpc + hh;
+    if (h >= L.H) break;
+    qprep_head(a, row, h, lane, rcs);
+  }
+}
 
 // The rows a deferred attention leaves to the combine: [0] the token's window row, [1] the entry the
 // token completes (null when it completes none).
@@ -1509,7 +1531,11 @@ size_t attend_partial_bytes(const LayerArgs& L, bool dense, int rows, int splits
 cudaError_t launch_attend_qprep(const AttendArgs& a, cudaStream_t s) {
   const int path = a.rows > 0 ? attend_path(a.L, a.topk == nullptr, a.rows) : 0;
   if (path != 2 && path != 3) return cudaSuccess;
-  return launch_kernel(qprep_kernel, dim3((unsigned)((a.L.H + 3) / 4), (unsigned)a.rows), dim3(128), 0, s, 0, a);
+  // decode (few rows): 4 heads per CTA for parallelism; chunks: 16, so each row's angles are formed
+  // by fewer CTAs
+  const int hpc = a.rows > kTcMaxRows ? 16 : 4;
+  return launch_kernel(qprep_kernel, dim3((unsigned)((a.L.H + hpc - 1) / hpc), (unsigned)a.rows), dim3(128), 0, s, 0,
+                       a, hpc);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tma_encode_fn() {
