@@ -18,8 +18,12 @@
 // running maximum moves only when its tile maximum exceeds it by more than 8 (in log2 units); then
 // O^T's column and the partial sums are rescaled.  Exponentials are taken against the running maximum,
 // so they stay below 2^8; a tile none of whose scores exceeds its head's running maximum by more than
-// the margin skips the maxima altogether.  Each softmax thread keeps its key's partial sums per head; they are reduced
-// once per query, in the epilogue.
+// the margin skips the maxima altogether.  Each softmax thread keeps its key's partial sums per head;
+// they are reduced once per query, in the epilogue.
+//
+// With N = 64 each MMA reads 6 KB of shared memory per 131 K multiply-adds, so the MMAs run at the
+// shared memory's rate (about 60 % of the tensor pipe's), and a tile's MMAs share that bandwidth with
+// the copies of the next tile's rows.
 //
 // Roles, in one persistent CTA per SM (query rows strided by the grid):
 //   warp 0      the MMA issuer (one thread)
@@ -28,7 +32,8 @@
 //               eight threads per 128-byte row segment, block by block: a 64-dim block is refilled as
 //               soon as the O^T MMAs that read it are done, while the other M-tiles still run.  Per
 //               query the epilogue: 1 / (l + 2^(sink - m)), the rotation by -t, the bf16 store
-//   warps 9-10  q~ loaders (q~ made beforehand by the q preparation kernel)
+//   warps 9-10  q~ loaders (q~ made beforehand by the q preparation kernel), and the table of the
+//               query's rotation angles for the epilogue
 // Every mbarrier wait is bounded: a wait that gives up sets the device error word, and the role stops.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
