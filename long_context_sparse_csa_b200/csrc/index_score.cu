@@ -227,6 +227,49 @@ __device__ __forceinline__ void load_key_scales(const IndexArgs& a, const Sched&
 
 // kHI > 0: decode specialisation (one query per group, kHI index heads, head weights in registers);
 // kHI == 0: any QN x H_I (prefill).  kFP4: e2m1 keys with block scales (smap: their scale words).
+// Chunk mode: the scores of key e for the queries whose HI columns sit in v (64 accumulator columns
+// starting at column c0 of the group's ncol).  v is indexed with constants only, so it stays in
+// registers.
+template <int HI>
+__device__ __forceinline__ void chunk_scores(const IndexArgs& a, const EpiSmem* es, const Group& G, const float (&v)[64],
+                                             int c0, int ncol, int64_t e, float ks, bool in_range, bool use_hist,
+                                             uint32_t* hist, int lane) {
+#pragma unroll
+  for (int qq = 0; qq < 64 / HI; ++qq) {
+    if (c0 + qq * HI >= ncol) break;
+    const int q = c0 / HI + qq;
+    const int64_t row = (int64_t)G.b * a.Tq + G.j0 + q;
+    // positive scales: ReLU(qs * ks * v) = qs * ks * ReLU(v), so s = ks * sum_h (w*qs)_h ReLU(v_h)
+    const bool fast = es->pos[q] && ks > 0.f;
+    float sc = 0.f;
+    if (fast) {
+      const float4* wqq = reinterpret_cast<const float4*>(es->wq + q * HI);
+#pragma unroll
+      for (int h = 0; h < HI; h += 4) {
+        const float4 w4 = wqq[h / 4];
+        sc = fmaf(w4.x, fmaxf(v[qq * HI + h], 0.f), sc);
+        sc = fmaf(w4.y, fmaxf(v[qq * HI + h + 1], 0.f), sc);
+        sc = fmaf(w4.z, fmaxf(v[qq * HI + h + 2], 0.f), sc);
+        sc = fmaf(w4.w, fmaxf(v[qq * HI + h + 3], 0.f), sc);
+      }
+      sc *= ks;
+    } else {
+      const float* wq = es->w + q * HI;
+      const float* sq = es->qs + q * HI;
+#pragma unroll
+      for (int h = 0; h < HI; ++h) sc += wq[h] * fmaxf(v[qq * HI + h] * (sq[h] * ks), 0.f);
+    }
+    const bool vis = e < es->nv[q];
+    if (in_range) a.scores[row * a.n_max + e] = vis ? sc : -INFINITY;
+    if (use_hist) {
+      // one shared-memory atomic per distinct bin in the warp
+      const uint32_t bin = vis ? (float_key(sc) >> 20) : 0xFFFFFFFFu;
+      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+      if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+    }
+  }
+}
+
 template <int kStages, int kHI, bool kFP4>
 __global__ void __launch_bounds__(kThreads, 2)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
@@ -573,48 +616,26 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
           if (use_hist && vis) atomicAdd(&es->hist[float_key(s) >> 20], 1u);
           cyc_st += CYC() - c2;
         } else if (ok) {
+          // chunk mode: the group's queries j0 .. j1 - 1, H_I columns each, read 64 columns (two or four
+          // queries) per TMEM wait
           tc_fence_after();
-          for (int j = G.j0; j < G.j1; ++j) {
-            const int q = j - G.j0;
-            const int64_t row = (int64_t)G.b * a.Tq + j;
-            const float* wq = es->w + q * a.H_I;
-            const float* sq = es->qs + q * a.H_I;
-            const float* wqq = es->wq + q * a.H_I;
-            // positive scales: ReLU(qs * ks * v) = qs * ks * ReLU(v), so s = ks * sum_h (w*qs)_h ReLU(v_h)
-            const bool fast = es->pos[q] && ks > 0.f;
-            float s = 0.f;
-            for (int hc = 0; hc < a.H_I; hc += 32) {
-              float v[32];
-              tmem_ld_32x32b_x16(lane_addr + (uint32_t)(acc * N + q * a.H_I + hc), v);
-              if (hc + 16 < a.H_I) tmem_ld_32x32b_x16(lane_addr + (uint32_t)(acc * N + q * a.H_I + hc + 16), v + 16);
-              tmem_wait_ld();
-              cyc_ld += CYC() - c1;
-              if (j + 1 == G.j1 && hc + 32 >= a.H_I) {
-                // every column of this accumulator is in registers: hand it back to the MMA warp
-                tc_fence_before();
-                mbar_arrive(&bars->tempty[acc]);
-              }
-              const int nh = min(32, a.H_I - hc);
-              if (fast) {
-#pragma unroll
-                for (int h = 0; h < 32; ++h)
-                  if (h < nh) s = fmaf(wqq[hc + h], fmaxf(v[h], 0.f), s);
-              } else {
-#pragma unroll
-                for (int h = 0; h < 32; ++h)
-                  if (h < nh) s += wq[hc + h] * fmaxf(v[h] * (sq[hc + h] * ks), 0.f);
-              }
+          const int nq = G.j1 - G.j0, ncol = nq * a.H_I;
+          for (int c0 = 0; c0 < ncol; c0 += 64) {
+            float v[64];
+            tmem_ld_32x32b_x32(lane_addr + (uint32_t)(acc * N + c0), v);
+            if (c0 + 32 < ncol) tmem_ld_32x32b_x32(lane_addr + (uint32_t)(acc * N + c0 + 32), v + 32);
+            tmem_wait_ld();
+            cyc_ld += CYC() - c1;
+            if (c0 + 64 >= ncol) {
+              // every column of this accumulator is in registers: hand it back to the MMA warp
+              tc_fence_before();
+              mbar_arrive(&bars->tempty[acc]);
             }
-            if (fast) s *= ks;
             long long c2 = CYC();
-            const bool vis = e < es->nv[q];
-            if (in_range) a.scores[row * a.n_max + e] = vis ? s : -INFINITY;
-            if (use_hist) {
-              // one shared-memory atomic per distinct bin in the warp
-              const uint32_t bin = vis ? (float_key(s) >> 20) : 0xFFFFFFFFu;
-              const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-              if (bin != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&es->hist[bin], (uint32_t)__popc(peers));
-            }
+            if (a.H_I == 32)
+              chunk_scores<32>(a, es, G, v, c0, ncol, e, ks, in_range, use_hist, es->hist, lane);
+            else
+              chunk_scores<16>(a, es, G, v, c0, ncol, e, ks, in_range, use_hist, es->hist, lane);
             cyc_st += CYC() - c2;
           }
         }
