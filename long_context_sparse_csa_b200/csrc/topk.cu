@@ -8,9 +8,11 @@
 // order-preserving 32-bit image of the scores (11 + 11 + 10 bits, shared-
 // memory histograms), which pins the k-th largest key T and how many keys
 // equal to T are taken; a final pass over the row in index order writes the
-// selection with one block-wide scan per 1024 indices, so the output order
-// (ascending index) and the tie rule come out deterministic.  Rows up to
-// kSmemKeys scores are staged once in shared memory.
+// selection, so the output order (ascending index) and the tie rule come out
+// deterministic.  Rows up to kSmemKeys scores are staged once in shared memory;
+// their final pass gives each thread a contiguous run of indices and places
+// every selection with one block-wide scan of the runs' counts (rows read from
+// global memory take one scan per 1024 indices, coalesced).
 #include "kernels.h"
 
 namespace csa {
@@ -144,6 +146,34 @@ __global__ void __launch_bounds__(kThreads, 1) topk_rows_kernel(const __grid_con
   if (cand && T == 0u) remaining = 0u;
 
   // ------------------------------------------------------------------ ordered emission
+  if (use_smem) {
+    // each thread takes a contiguous run of `per` indices (odd, so the runs' shared-memory words
+    // fall in distinct banks across a warp); one scan of the runs' counts places every selection
+    const int per = ((n + kThreads - 1) / kThreads) | 1;
+    const int lo = tid * per, hi = min(lo + per, n);
+    uint32_t gt_n = 0, eq_n = 0;
+    for (int i = lo; i < hi; ++i) {
+      const uint32_t k = keys_sm[i];
+      gt_n += k > T;
+      eq_n += k == T;
+    }
+    uint32_t gt_tot, eq_tot;
+    uint32_t gt_run = block_excl_scan(gt_n, wsum, &gt_tot);
+    uint32_t eq_run = block_excl_scan(eq_n, wsum, &eq_tot);
+    for (int i = lo; i < hi; ++i) {
+      const uint32_t k = keys_sm[i];
+      if (k > T) {
+        out[gt_run + min(eq_run, remaining)] = value_at(i);
+        ++gt_run;
+      } else if (k == T) {
+        if (eq_run < remaining) out[gt_run + eq_run] = value_at(i);
+        ++eq_run;
+      }
+    }
+    const uint32_t taken = gt_tot + min(eq_tot, remaining);
+    for (uint32_t p = taken + tid; p < (uint32_t)a.k; p += kThreads) out[p] = -1;
+    return;
+  }
   uint32_t gt_run = 0, eq_run = 0;
   for (int base = 0; base < n; base += kThreads) {
     const int i = base + tid;
